@@ -1,0 +1,437 @@
+#!/usr/bin/env python
+"""Benchmark of the tile-binned differentiable Gaussian splatting rasterizer.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl native|reference]
+
+One step = one training frame through the whole hot path for one camera:
+project -> bin and sort -> forward blend -> L1 loss gradient -> backward blend
+-> projection backward.  Default workload: a seeded synthetic 400k-Gaussian
+scene (120 anisotropic clusters in a 10 m box, log-scales N(-4, 0.6), opacity
+logits N(1, 1.5)) seen from 16 ring cameras at 980 x 545, f = 1000, L1 loss
+against a seeded U(0, 1) target.  Inputs are resident in HBM; L2 (126 MB) is
+flushed between timed steps by writing a 256 MB buffer outside the timed
+events.  Each rank renders its own cameras (independent frames, no data-path
+collective); the reported value is all frames over the slowest rank's device
+time.  Prints one JSON line (rank 0).
+
+--impl reference times the CPU oracle (double precision, every host core) on
+a bounded sample of the same workload: full projection and brute-force
+binning, the blend and its backward on a seeded sample of tiles, the frame
+time extrapolated by tile count.
+"""
+from __future__ import annotations
+
+import argparse
+import datetime
+import hashlib
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+from scenes import SPECS, make_cameras, make_scene, make_target  # noqa: E402
+
+DEFAULT_WORKLOAD = "train400k_half"
+METRIC = "fwd and fwd+bwd frames/s at 400k Gaussians, 980x545; tile-pairs/s; % roofline"
+
+# Algorithmic FP32-pipe operations per (pixel, list entry) evaluation,
+# counted from the written formulas with a fused multiply-add as one
+# operation (per-entry work done once per tile, such as the conic scaling,
+# is not counted):
+#   visited entry (forward and backward): dx, dy (2); sigma from the half
+#     conic in FMA form (5); scale for exp (1); o G (1); min with 0.99 (1);
+#     sigma < 0 test (1); alpha < 1/255 test (1)                      = 12
+#   added entry, forward extra: T (1 - alpha) as one FMA (1); stop test (1);
+#     w = alpha T (1); colour accumulation (3)                         = 6
+#   added entry, backward extra: 1 - alpha (1); T_i = T r (1); w (1);
+#     colour gradients w g (3); c - R (3); <c - R, g> (3); dL/dalpha (1);
+#     R update (3); cap select (1); v = dL/dalpha alpha (1); the five
+#     geometric products v dx, v dy, v dx^2, v dx dy, v dy^2 (5); the nine
+#     per-Gaussian sums over pixels (9)                                = 32
+# plus one MUFU ex2 per visit (and one rcp per backward addition).
+OPS_VISIT = 12
+OPS_FWD_ADD = 6
+OPS_BWD_ADD = 32
+
+# Algorithmic HBM bytes of the streaming kernels (per Gaussian G, pair P):
+#   project      56 B/G raw parameters read + 68 B/G records written
+#   depth_keys   8 B/G read (depth, count) + 4 B/G written
+#   depth_sort   16 B/G per pass (key + value read and written)
+#   scan_emit    24 B/G read (sorted id, count, rectangle) + 8 B/P written
+#   tile_sort    16 B/P per pass
+#   ranges       4 B/P read
+#   project_bwd  56 B/G raw parameters + 48 B/G 2D gradients read,
+#                56 B/G raw gradients written
+BYTES = {
+    "project": lambda G, P: 124 * G,
+    "depth_keys": lambda G, P: 12 * G,
+    "depth_sort": lambda G, P: 16 * G,
+    "scan_emit": lambda G, P: 24 * G + 8 * P,
+    "tile_sort": lambda G, P: 16 * P,
+    "ranges": lambda G, P: 4 * P,
+    "project_bwd": lambda G, P: 160 * G,
+}
+ALU_KERNELS = ("render_fwd", "render_bwd")
+
+# DRAM traffic per launch of render_bwd measured by ncu
+# (dram__bytes_read.sum + dram__bytes_write.sum), valid only for the kernel
+# source it was taken on.
+TRAFFIC = {}  # {"render_bwd": {"src_sha": ..., "bytes_per_pair": ...}}
+
+
+def _peaks():
+    try:
+        with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
+            d = json.load(f)
+        return float(d["hbm_gbs"]), "measured", float(d.get("sm_max_mhz", 1965.0))
+    except Exception:
+        return 6650.0, "fallback", 1965.0
+
+
+def _src_sha(name):
+    p = os.path.join(ROOT, "gaussian_splatting_differentiable_tile_b200", "csrc", name)
+    return hashlib.sha256(open(p, "rb").read()).hexdigest()[:16]
+
+
+class ClockSampler:
+    """nvidia-smi samples every 200 ms while the timed region runs."""
+
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, device_id: str | None):
+        self.samples = []
+        self.proc = None
+        cmd = ["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits", "-lms", "200"]
+        if device_id:
+            cmd += ["-i", device_id]
+        try:
+            self.proc = subprocess.Popen(cmd, stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            self.thread = threading.Thread(target=self._read, daemon=True)
+            self.thread.start()
+        except Exception:
+            self.proc = None
+
+    def _read(self):
+        for line in self.proc.stdout:
+            parts = [p.strip() for p in line.split(",")]
+            if len(parts) >= 9:
+                self.samples.append(parts)
+
+    def stop(self) -> dict:
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        time.sleep(0.25)
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except Exception:
+            self.proc.kill()
+        sm = [float(s[1]) for s in self.samples if s[1].replace(".", "").isdigit()]
+        mx = [float(s[2]) for s in self.samples if s[2].replace(".", "").isdigit()]
+        names = ("hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap")
+        reasons = sorted({names[k] for s in self.samples for k in range(4) if s[5 + k].lower() == "active"})
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": max(mx) if mx else None,
+                "reasons": reasons, "samples": len(self.samples)}
+
+
+# ------------------------------------------------------------------ CPU side
+def cpu_frame_time(params_np, cam, sample_tiles: int, seed: int = 0) -> dict:
+    """The oracle, as it stands, on one frame: full projection and binning,
+    blend and backward on `sample_tiles` seeded tiles, projection backward;
+    returns the extrapolated seconds per frame."""
+    import oracle as O
+
+    tiles = cam.tiles
+    mask = np.zeros(tiles, np.uint8)
+    mask[np.random.default_rng(seed).choice(tiles, min(sample_tiles, tiles), replace=False)] = 1
+    t = {}
+    t0 = time.perf_counter()
+    p = O.project(params_np, cam)
+    t["project"] = time.perf_counter() - t0
+    t0 = time.perf_counter()
+    O.bin_pairs(p["rect"], p["valid"], p["depth32"], cam.width, cam.height)
+    t["bin"] = time.perf_counter() - t0
+    t0 = time.perf_counter()
+    O.render(p, cam, tile_mask=mask)
+    t["render_sample"] = time.perf_counter() - t0
+    dl = np.random.default_rng(seed + 1).normal(size=(cam.height, cam.width, 3)) / (3 * cam.pixels)
+    t0 = time.perf_counter()
+    g2, _ = O.render_bwd(p, cam, dl, tile_mask=mask)
+    t["render_bwd_sample"] = time.perf_counter() - t0
+    t0 = time.perf_counter()
+    O.project_bwd(params_np, cam, g2)
+    t["project_bwd"] = time.perf_counter() - t0
+    scale = tiles / float(mask.sum())
+    frame = t["project"] + t["bin"] + (t["render_sample"] + t["render_bwd_sample"]) * scale + t["project_bwd"]
+    fwd = t["project"] + t["bin"] + t["render_sample"] * scale
+    return {"frame_s": frame, "fwd_s": fwd, "parts": t, "sampled_tiles": int(mask.sum()), "tiles": tiles,
+            "threads": O.default_threads()}
+
+
+def run_reference(args, spec, rank, world):
+    if rank != 0:
+        return
+    params = make_scene(spec)
+    cams = make_cameras(spec)
+    for i in range(args.warmup):
+        cpu_frame_time(params, cams[i % len(cams)], args.ref_sample_tiles, seed=i)
+    times = []
+    info = None
+    for i in range(args.steps):
+        info = cpu_frame_time(params, cams[i % len(cams)], args.ref_sample_tiles, seed=100 + i)
+        times.append(info["frame_s"])
+    fps = 1.0 / statistics.mean(times)
+    sample = (f"per step one camera: full projection and brute-force binning of {spec.n} Gaussians, "
+              f"blend and backward on {info['sampled_tiles']} of {info['tiles']} seeded tiles, "
+              f"frame time extrapolated by tile count")
+    out = {"impl": "reference", "metric": METRIC, "value": fps, "unit": "frames/s", "n_gpus": world,
+           "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1000.0 * statistics.mean(times),
+           "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+           "data": "synthetic", "config": _config(spec, None),
+           "cpu_baseline": {"value": fps, "unit": "frames/s", "cores": info["threads"], "kind": "oracle",
+                            "sample": sample},
+           "e2e": {"value": fps, "unit": "frames/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(out), flush=True)
+
+
+def _config(spec, pairs):
+    return {"workload": spec.name, "n_gaussians": spec.n, "width": spec.width, "height": spec.height,
+            "focal": spec.focal, "cameras": f"{spec.n_cameras} {spec.cameras}", "pairs_per_frame": pairs,
+            "l2": "flushed between timed steps (256 MB write outside the timed events)",
+            "parallelism": "replicas (cameras split across ranks)"}
+
+
+# ------------------------------------------------------------------ GPU side
+def run_native(args, spec, rank, world, local):
+    import torch
+    import torch.distributed as dist
+
+    import gaussian_splatting_differentiable_tile_b200 as G
+
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    params_np = make_scene(spec)
+    cams = make_cameras(spec)
+    mine = [c for i, c in enumerate(cams) if i % world == rank] or cams[:1]
+    n = spec.n
+    P = {k: torch.from_numpy(v).to(dev) for k, v in params_np.items()}
+    targets = [torch.from_numpy(make_target(spec.width, spec.height, seed=i)).to(dev) for i in range(len(mine))]
+    ccams = [G.make_camera(c) for c in mine]
+
+    # size the pair list from the cameras this rank renders
+    r = G.Rasterizer(n, spec.width, spec.height, max_pairs=24 * n, device=dev)
+    pairs, stats = [], []
+    for c in mine:
+        r.forward(c, P, sync=True)
+        pairs.append(r.n_pairs)
+        stats.append(G.gs_render_stats(c, n, r.proj, r.bins, r.last))
+    bins = G.Bins(n, int(max(pairs) * 1.05) + 4096, spec.width, spec.height, device=dev)
+    proj = r.proj
+    H, W = spec.height, spec.width
+    image = torch.empty((H, W, 3), device=dev)
+    T = torch.empty((H, W), device=dev)
+    last = torch.empty((H, W), dtype=torch.int32, device=dev)
+    dl = torch.empty_like(image)
+    loss = torch.zeros(1, device=dev)
+    grad2d = torch.empty((n, 12), device=dev)
+    grads = {k: torch.empty_like(v) for k, v in P.items()}
+    flush = torch.empty(256 * 1024 * 1024, dtype=torch.uint8, device=dev)
+
+    def step_fwd(i):
+        c = ccams[i % len(ccams)]
+        G.gs_project(c, P, proj)
+        G.gs_bin_and_sort(c, n, proj, bins, sync=False)
+        G.gs_render_fwd(c, n, proj, bins, image, T, last)
+
+    def step_full(i, params=P, tgt=None):
+        c = ccams[i % len(ccams)]
+        G.gs_project(c, params, proj)
+        G.gs_bin_and_sort(c, n, proj, bins, sync=False)
+        G.gs_render_fwd(c, n, proj, bins, image, T, last)
+        G.gs_l1_loss_grad(image, targets[i % len(targets)] if tgt is None else tgt, dl, loss)
+        G.gs_render_bwd(c, n, params, proj, bins, T, last, dl, grad2d, grads)
+
+    def barrier():
+        if world > 1:
+            dist.barrier()
+
+    def timed(fn, steps, warmup, profile=False):
+        for i in range(warmup):
+            fn(i)
+        torch.cuda.synchronize()
+        ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(steps)]
+        barrier()
+        torch.cuda.synchronize()
+        if profile:
+            G.profile_begin(1 << 16)
+        for i in range(steps):
+            flush.zero_()
+            ev[i][0].record()
+            fn(i)
+            ev[i][1].record()
+        torch.cuda.synchronize()
+        prof = G.profile_end() if profile else None
+        barrier()
+        ms = sum(a.elapsed_time(b) for a, b in ev)
+        return ms, prof
+
+    device_id = None
+    try:
+        device_id = "GPU-" + str(torch.cuda.get_device_properties(local).uuid)
+    except Exception:
+        device_id = str(local)
+    sampler = ClockSampler(device_id)
+    full_ms, prof = timed(step_full, args.steps, args.warmup, profile=True)
+    clocks = sampler.stop()
+    fwd_ms, _ = timed(step_fwd, args.steps, args.warmup)
+
+    # end to end through the public API with host buffers: inputs copied from
+    # pinned host memory, loss and raw gradients copied back, every step
+    host_in = {k: torch.from_numpy(v).pin_memory() for k, v in params_np.items()}
+    host_tgt = [t.cpu().pin_memory() for t in targets]
+    host_out = {k: torch.empty(v.shape, dtype=v.dtype).pin_memory() for k, v in grads.items()}
+    host_loss = torch.empty(1).pin_memory()
+    dev_in = {k: torch.empty_like(v) for k, v in P.items()}
+    dev_tgt = torch.empty_like(targets[0])
+
+    def step_e2e(i):
+        for k in dev_in:
+            dev_in[k].copy_(host_in[k], non_blocking=True)
+        dev_tgt.copy_(host_tgt[i % len(host_tgt)], non_blocking=True)
+        step_full(i, params=dev_in, tgt=dev_tgt)
+        for k in grads:
+            host_out[k].copy_(grads[k], non_blocking=True)
+        host_loss.copy_(loss, non_blocking=True)
+
+    e2e_ms, _ = timed(step_e2e, args.steps, args.warmup)
+    h2d = sum(v.numel() * 4 for v in params_np.values()) + H * W * 3 * 4
+    d2h = sum(v.numel() * 4 for v in params_np.values()) + 4
+
+    t = torch.tensor([full_ms, fwd_ms, e2e_ms], dtype=torch.float64, device=dev)
+    if world > 1:
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    full_ms, fwd_ms, e2e_ms = t.tolist()
+    frames = args.steps * world
+    if rank != 0:
+        return
+
+    hbm_peak, peak_kind, sm_max = _peaks()
+    sms = torch.cuda.get_device_properties(local).multi_processor_count
+    clock_mhz = clocks["sm_max_mhz"] or sm_max
+    alu_peak = sms * 128 * clock_mhz * 1e6 / 1e12  # T FP32 lane-ops/s
+    # work per timed step (cameras cycle through `mine`)
+    sel = [i % len(mine) for i in range(args.steps)]
+    pairs_steps = [pairs[i] for i in sel]
+    fwd_ops = sum(OPS_VISIT * stats[i]["fwd_visits"] + OPS_FWD_ADD * stats[i]["contributions"] for i in sel)
+    bwd_ops = sum(OPS_VISIT * stats[i]["bwd_visits"] + OPS_BWD_ADD * stats[i]["contributions"] for i in sel)
+    stages = {}
+    gpu_launches = 0
+    for name, (launches, ms) in (prof or {}).items():
+        gpu_launches += launches
+        entry = {"launches": launches, "ms_total": ms, "ms_per_step": ms / args.steps}
+        if name in BYTES:
+            passes = launches / args.steps
+            per_step = [BYTES[name](n, pairs[i]) for i in sel]
+            total_bytes = sum(per_step) * (passes if name in ("depth_sort", "tile_sort") else 1)
+            ach = total_bytes / (ms * 1e-3) / 1e9
+            entry.update(bound="hbm", achieved=ach, peak=hbm_peak, unit="GB/s", frac=ach / hbm_peak)
+        elif name in ALU_KERNELS:
+            ops = fwd_ops if name == "render_fwd" else bwd_ops
+            ach = ops / (ms * 1e-3) / 1e12
+            entry.update(bound="alu", achieved=ach, peak=alu_peak, unit="Tops/s", frac=ach / alu_peak)
+        stages[name] = entry
+    dom = max(stages, key=lambda k: stages[k]["ms_total"]) if stages else None
+    roof = None
+    if dom and "bound" in stages[dom]:
+        s = stages[dom]
+        tr = TRAFFIC.get(dom)
+        traffic = None
+        if tr and tr.get("src_sha") == _src_sha("gs_render.cu"):
+            traffic = tr["bytes_per_pair"] * statistics.mean(pairs_steps)
+        roof = {"kernel": dom, "bound": s["bound"], "achieved": s["achieved"], "peak": s["peak"],
+                "unit": s["unit"], "frac": s["frac"], "traffic": traffic,
+                "peak_basis": (f"{sms} SMs x 128 FP32 lanes x {clock_mhz:.0f} MHz (FMA = 1 op)"
+                               if s["bound"] == "alu" else f"{peak_kind} HBM copy bandwidth")}
+    cpu = None
+    if world == 1 and not args.no_cpu_baseline:
+        info = cpu_frame_time(params_np, mine[0], args.cpu_sample_tiles)
+        cpu = {"value": 1.0 / info["frame_s"], "unit": "frames/s", "cores": info["threads"], "kind": "oracle",
+               "sample": (f"one camera: full projection and brute-force binning of {n} Gaussians, blend and "
+                          f"backward on {info['sampled_tiles']} of {info['tiles']} seeded tiles, frame time "
+                          f"extrapolated by tile count ({info['frame_s']:.1f} s/frame)"),
+               "fwd_frames_per_s": 1.0 / info["fwd_s"]}
+    mean_pairs = statistics.mean(pairs_steps)
+    out = {
+        "metric": METRIC,
+        "value": frames / (full_ms * 1e-3),
+        "unit": "frames/s",
+        "n_gpus": world,
+        "steps": args.steps,
+        "warmup": args.warmup,
+        "ms_per_step": full_ms / args.steps,
+        "higher_is_better": True,
+        "scaling": "weak",
+        "vs_baseline": None,
+        "dtype": "f32",
+        "data": "synthetic",
+        "config": _config(spec, int(mean_pairs)),
+        "fwd_frames_per_s": frames / (fwd_ms * 1e-3),
+        "fwd_ms_per_frame": fwd_ms / args.steps,
+        "tile_pairs_per_s": mean_pairs * frames / (fwd_ms * 1e-3),
+        "tiles_per_gaussian": mean_pairs / max(1, n),
+        "roofline": roof,
+        "stages": stages,
+        "cpu_baseline": cpu,
+        "e2e": {"value": frames / (e2e_ms * 1e-3), "unit": "frames/s", "h2d_bytes_per_step": h2d,
+                "d2h_bytes_per_step": d2h},
+        "gpu_launches": gpu_launches,
+        "clocks": clocks,
+    }
+    print(json.dumps(out), flush=True)
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=32)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=("native", "reference"), default="native")
+    ap.add_argument("--workload", default=DEFAULT_WORKLOAD, choices=sorted(SPECS))
+    ap.add_argument("--cpu-sample-tiles", type=int, default=48)
+    ap.add_argument("--ref-sample-tiles", type=int, default=8)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    rank = int(os.environ.get("RANK", 0))
+    world = int(os.environ.get("WORLD_SIZE", 1))
+    local = int(os.environ.get("LOCAL_RANK", 0))
+    spec = SPECS[args.workload]
+    if args.impl == "reference":
+        run_reference(args, spec, rank, world)
+        return
+    if world > 1:
+        import torch
+        import torch.distributed as dist
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", device_id=torch.device("cuda", local),
+                                timeout=datetime.timedelta(seconds=300))
+    try:
+        run_native(args, spec, rank, world, local)
+    finally:
+        if world > 1:
+            import torch.distributed as dist
+            dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,240 @@
+"""B200 tile-binned differentiable 3D Gaussian splatting rasterizer.
+
+A thin Python binding over libgs.so (include/gs.h).  The functions below carry
+the C entry points' names and only marshal arguments: every step of the path
+runs in the library's CUDA kernels.  PyTorch provides device memory and the
+current CUDA stream.
+
+    proj = Projected(n)
+    bins = Bins(n, max_pairs, width, height)
+    gs_project(cam, params, proj)
+    K = gs_bin_and_sort(cam, n, proj, bins)           # sync=True reads K back
+    gs_render_fwd(cam, n, proj, bins, image, T_final, last)
+    gs_render_bwd(cam, n, params, proj, bins, T_final, last, dL_dimage, grad2d, grads)
+
+``params`` and ``grads`` are dicts of contiguous float32 CUDA tensors with
+keys means (N,3), log_scales (N,3), quats (N,4), opacity_logits (N,),
+colors (N,3).  A camera is any object with viewmat (4x4 world-to-camera,
+OpenCV axes), fx, fy, cx, cy, width, height, near_z and bg.
+"""
+from __future__ import annotations
+
+import ctypes
+
+import torch
+
+from . import _abi
+from ._abi import (GS_ERR_ALIGNMENT, GS_ERR_CAPACITY, GS_ERR_CUDA, GS_ERR_DEVICE_TIMEOUT,  # noqa: F401
+                   GS_ERR_INVALID_ARG, GS_ERR_TOO_LARGE, GS_OK, GS_TILE)
+
+__all__ = [
+    "GSError", "Projected", "Bins", "make_camera", "gs_project", "gs_bin_and_sort", "gs_render_fwd",
+    "gs_render_bwd", "gs_render_stats", "gs_l1_loss_grad", "gs_read_status", "gs_error_string", "profile_begin",
+    "profile_end", "lib", "PARAM_KEYS",
+]
+
+PARAM_KEYS = ("means", "log_scales", "quats", "opacity_logits", "colors")
+
+
+def lib() -> ctypes.CDLL:
+    return _abi.load()
+
+
+class GSError(RuntimeError):
+    def __init__(self, code: int, what: str):
+        super().__init__(f"{what}: {gs_error_string(code)} (code {code})")
+        self.code = code
+
+
+def gs_error_string(code: int) -> str:
+    return lib().gs_error_string(int(code)).decode()
+
+
+def _check(rc: int, what: str) -> int:
+    if rc < 0:
+        raise GSError(rc, what)
+    return rc
+
+
+def _dev(t: torch.Tensor | None, name: str, dtype=None) -> ctypes.c_void_p:
+    if t is None:
+        return ctypes.c_void_p(0)
+    if not t.is_cuda:
+        raise ValueError(f"{name} must be a CUDA tensor")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+    if dtype is not None and t.dtype != dtype:
+        raise ValueError(f"{name} must be {dtype}, got {t.dtype}")
+    return ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(stream) -> ctypes.c_void_p:
+    s = torch.cuda.current_stream() if stream is None else stream
+    return ctypes.c_void_p(s.cuda_stream)
+
+
+def make_camera(cam) -> _abi.GsCamera:
+    """A gs_camera from a camera-like object (returned as is if it already is one)."""
+    if isinstance(cam, _abi.GsCamera):
+        return cam
+    c = _abi.GsCamera()
+    vm = [float(v) for v in torch.as_tensor(cam.viewmat, dtype=torch.float32).reshape(16).tolist()]
+    for k in range(16):
+        c.viewmat[k] = vm[k]
+    c.fx, c.fy, c.cx, c.cy = float(cam.fx), float(cam.fy), float(cam.cx), float(cam.cy)
+    c.width, c.height = int(cam.width), int(cam.height)
+    c.near_z = float(cam.near_z)
+    for k in range(3):
+        c.bg[k] = float(cam.bg[k])
+    return c
+
+
+def _params_struct(params: dict, cls=_abi.GsParams):
+    s = cls()
+    for k in PARAM_KEYS:
+        setattr(s, k, _dev(params[k], k, torch.float32).value)
+    return s
+
+
+class _Carved:
+    """A caller-owned device buffer carved into the library's arrays."""
+
+    def _view(self, ptr: int, count: int, dtype: torch.dtype, shape) -> torch.Tensor:
+        off = ptr - self.buffer.data_ptr()
+        nbytes = count * torch.tensor([], dtype=dtype).element_size()
+        return self.buffer[off:off + nbytes].view(dtype).view(*shape)
+
+
+class Projected(_Carved):
+    """gs_projected records for n Gaussians, in one device buffer."""
+
+    def __init__(self, n: int, device="cuda"):
+        self.n = int(n)
+        nbytes = max(int(lib().gs_projected_bytes(self.n)), 256)
+        self.buffer = torch.empty(nbytes, dtype=torch.uint8, device=device)
+        self.struct = _abi.GsProjected()
+        _check(lib().gs_projected_carve(ctypes.c_void_p(self.buffer.data_ptr()), self.n,
+                                        ctypes.byref(self.struct)), "gs_projected_carve")
+        n = self.n
+        self.xy_opacity_depth = self._view(self.struct.xy_opacity_depth, 4 * n, torch.float32, (n, 4))
+        self.conic_radius = self._view(self.struct.conic_radius, 4 * n, torch.float32, (n, 4))
+        self.rgb = self._view(self.struct.rgb, 4 * n, torch.float32, (n, 4))
+        self.rect = self._view(self.struct.rect, 4 * n, torch.int32, (n, 4))
+        self.count = self._view(self.struct.count, n, torch.int32, (n,))
+
+
+class Bins(_Carved):
+    """gs_bins for at most n Gaussians, max_pairs pairs, a width x height image."""
+
+    def __init__(self, n: int, max_pairs: int, width: int, height: int, device="cuda"):
+        self.n, self.max_pairs = int(n), int(max_pairs)
+        self.width, self.height = int(width), int(height)
+        nbytes = int(lib().gs_bins_bytes(self.n, self.max_pairs, self.width, self.height))
+        if nbytes == 0:
+            raise GSError(GS_ERR_INVALID_ARG, "gs_bins_bytes")
+        self.buffer = torch.empty(nbytes, dtype=torch.uint8, device=device)
+        self.struct = _abi.GsBins()
+        _check(lib().gs_bins_carve(ctypes.c_void_p(self.buffer.data_ptr()), self.n, self.max_pairs,
+                                   self.width, self.height, ctypes.byref(self.struct)), "gs_bins_carve")
+        tiles = int(self.struct.max_tiles)
+        self.tiles = tiles
+        self.pair_tile = self._view(self.struct.pair_tile, self.max_pairs, torch.int32, (self.max_pairs,))
+        self.pair_gid = self._view(self.struct.pair_gid, self.max_pairs, torch.int32, (self.max_pairs,))
+        self.ranges = self._view(self.struct.ranges, 2 * tiles, torch.int32, (tiles, 2))
+        self.n_pairs = self._view(self.struct.n_pairs, 1, torch.int64, (1,))
+        self.status = self._view(self.struct.status, 1, torch.int32, (1,))
+
+
+def gs_project(cam, params: dict, proj: Projected, stream=None) -> None:
+    n = int(params["means"].shape[0])
+    if n > proj.n:
+        raise ValueError("Projected buffer too small")
+    c = make_camera(cam)
+    p = _params_struct(params)
+    _check(lib().gs_project(ctypes.byref(c), n, ctypes.byref(p), ctypes.byref(proj.struct), _stream(stream)),
+           "gs_project")
+
+
+def gs_bin_and_sort(cam, n: int, proj: Projected, bins: Bins, sync: bool = True, stream=None):
+    """Returns K (sync=True; raises GSError with .code GS_ERR_CAPACITY when K
+    exceeds bins.max_pairs, the required K in .n_pairs) or None (sync=False)."""
+    c = make_camera(cam)
+    k = ctypes.c_int64(0)
+    rc = lib().gs_bin_and_sort(ctypes.byref(c), int(n), ctypes.byref(proj.struct), ctypes.byref(bins.struct),
+                               ctypes.byref(k) if sync else None, _stream(stream))
+    if rc < 0:
+        err = GSError(rc, "gs_bin_and_sort")
+        err.n_pairs = int(k.value)
+        raise err
+    return int(k.value) if sync else None
+
+
+def gs_render_fwd(cam, n: int, proj: Projected, bins: Bins, image: torch.Tensor, T_final: torch.Tensor,
+                  last: torch.Tensor, stream=None) -> None:
+    H, W = int(cam.height), int(cam.width)
+    if image.numel() != H * W * 3 or T_final.numel() != H * W or last.numel() != H * W:
+        raise ValueError("output tensors must be [H,W,3], [H,W], [H,W]")
+    c = make_camera(cam)
+    _check(lib().gs_render_fwd(ctypes.byref(c), int(n), ctypes.byref(proj.struct), ctypes.byref(bins.struct),
+                               _dev(image, "image", torch.float32), _dev(T_final, "T_final", torch.float32),
+                               _dev(last, "last", torch.int32), _stream(stream)), "gs_render_fwd")
+
+
+def gs_render_bwd(cam, n: int, params: dict, proj: Projected, bins: Bins, T_final: torch.Tensor,
+                  last: torch.Tensor, dL_dimage: torch.Tensor, grad2d: torch.Tensor, grads: dict,
+                  stream=None) -> None:
+    if grad2d.numel() < 12 * int(n):
+        raise ValueError("grad2d must hold [N,12] floats")
+    c = make_camera(cam)
+    p = _params_struct(params)
+    g = _params_struct(grads, _abi.GsGrads)
+    _check(lib().gs_render_bwd(ctypes.byref(c), int(n), ctypes.byref(p), ctypes.byref(proj.struct),
+                               ctypes.byref(bins.struct), _dev(T_final, "T_final", torch.float32),
+                               _dev(last, "last", torch.int32), _dev(dL_dimage, "dL_dimage", torch.float32),
+                               _dev(grad2d, "grad2d", torch.float32), ctypes.byref(g), _stream(stream)),
+           "gs_render_bwd")
+
+
+def gs_render_stats(cam, n: int, proj: Projected, bins: Bins, last: torch.Tensor, stream=None) -> dict:
+    """Exact work counts of the frame (synchronizes to read them back)."""
+    counts = torch.zeros(4, dtype=torch.int64, device=last.device)
+    c = make_camera(cam)
+    _check(lib().gs_render_stats(ctypes.byref(c), int(n), ctypes.byref(proj.struct), ctypes.byref(bins.struct),
+                                 _dev(last, "last", torch.int32), _dev(counts, "counts"), _stream(stream)),
+           "gs_render_stats")
+    v = counts.cpu().tolist()
+    return {"fwd_visits": v[0], "contributions": v[1], "bwd_visits": v[2], "pixels": v[3]}
+
+
+def gs_l1_loss_grad(image: torch.Tensor, target: torch.Tensor, dL_dimage: torch.Tensor,
+                    loss: torch.Tensor | None = None, stream=None) -> None:
+    if image.numel() != target.numel() or image.numel() != dL_dimage.numel():
+        raise ValueError("image, target and dL_dimage must have the same size")
+    _check(lib().gs_l1_loss_grad(_dev(image, "image", torch.float32), _dev(target, "target", torch.float32),
+                                 image.numel(), _dev(dL_dimage, "dL_dimage", torch.float32),
+                                 _dev(loss, "loss", torch.float32), _stream(stream)), "gs_l1_loss_grad")
+
+
+def gs_read_status(bins: Bins, stream=None):
+    """Synchronizes and returns (status code, K) of the last gs_bin_and_sort."""
+    k = ctypes.c_int64(0)
+    rc = lib().gs_read_status(ctypes.byref(bins.struct), ctypes.byref(k), _stream(stream))
+    if rc == GS_ERR_CUDA:
+        raise GSError(rc, "gs_read_status")
+    return rc, int(k.value)
+
+
+def profile_begin(max_launches: int = 1 << 16) -> None:
+    _check(lib().gs_profile_begin(int(max_launches)), "gs_profile_begin")
+
+
+def profile_end(max_stats: int = 64) -> dict:
+    """Returns {kernel name: (launches, total ms)} for launches since profile_begin."""
+    arr = (_abi.GsProfileStat * max_stats)()
+    m = _check(lib().gs_profile_end(arr, max_stats), "gs_profile_end")
+    return {arr[i].name.decode(): (int(arr[i].launches), float(arr[i].total_ms)) for i in range(m)}
+
+
+from .raster import Rasterizer, rasterize  # noqa: E402,F401
+
+__all__ += ["Rasterizer", "rasterize"]

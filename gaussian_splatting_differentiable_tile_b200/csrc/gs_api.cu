@@ -1,0 +1,351 @@
+// gs_api.cu -- the extern "C" entry points declared in include/gs.h:
+// argument checks, buffer carving, launches, status readback, profiling.
+#include <cmath>
+#include <cstdio>
+#include <cstring>
+#include <vector>
+
+#include "gs_internal.cuh"
+
+using namespace gs;
+
+namespace {
+
+constexpr int64_t kMaxCount = (int64_t(1) << 30) - 1;  // N and max_pairs limit
+
+inline bool aligned(const void *p, size_t a) {
+    return (reinterpret_cast<uintptr_t>(p) % a) == 0;
+}
+
+int make_cam(const gs_camera *cam, CamConst *out) {
+    if (!cam) return GS_ERR_INVALID_ARG;
+    if (cam->width < 1 || cam->height < 1 || cam->width > 65536 || cam->height > 65536)
+        return GS_ERR_INVALID_ARG;
+    if (!(cam->fx > 0.f) || !(cam->fy > 0.f) || !std::isfinite(cam->fx) || !std::isfinite(cam->fy) ||
+        !std::isfinite(cam->cx) || !std::isfinite(cam->cy) || !(cam->near_z > 0.f) ||
+        !std::isfinite(cam->near_z))
+        return GS_ERR_INVALID_ARG;
+    for (int k = 0; k < 16; k++)
+        if (!std::isfinite(cam->viewmat[k])) return GS_ERR_INVALID_ARG;
+    for (int k = 0; k < 3; k++)
+        if (!std::isfinite(cam->bg[k])) return GS_ERR_INVALID_ARG;
+    CamConst c{};
+    for (int i = 0; i < 3; i++) {
+        for (int j = 0; j < 3; j++) c.R[3 * i + j] = cam->viewmat[4 * i + j];
+        c.t[i] = cam->viewmat[4 * i + 3];
+    }
+    c.fx = cam->fx; c.fy = cam->fy; c.cx = cam->cx; c.cy = cam->cy;
+    // "Gaussian splatting in PyTorch" s3: frustum widened by 0.3 of the
+    // half-FoV tangent on each side (computed in double, rounded once).
+    const double tfx = 0.5 * cam->width / (double)cam->fx, tfy = 0.5 * cam->height / (double)cam->fy;
+    c.lim_x_lo = (float)(-((double)cam->cx / cam->fx + 0.3 * tfx));
+    c.lim_x_hi = (float)((cam->width - (double)cam->cx) / cam->fx + 0.3 * tfx);
+    c.lim_y_lo = (float)(-((double)cam->cy / cam->fy + 0.3 * tfy));
+    c.lim_y_hi = (float)((cam->height - (double)cam->cy) / cam->fy + 0.3 * tfy);
+    c.near_z = cam->near_z;
+    for (int k = 0; k < 3; k++) c.bg[k] = cam->bg[k];
+    c.width = cam->width;
+    c.height = cam->height;
+    c.tiles_x = (cam->width + kTile - 1) / kTile;
+    c.tiles_y = (cam->height + kTile - 1) / kTile;
+    *out = c;
+    return GS_OK;
+}
+
+int check_projected(const gs_projected *p, int64_t n) {
+    if (!p) return GS_ERR_INVALID_ARG;
+    if (n == 0) return GS_OK;
+    if (!p->xy_opacity_depth || !p->conic_radius || !p->rgb || !p->rect || !p->count)
+        return GS_ERR_INVALID_ARG;
+    if (!aligned(p->xy_opacity_depth, 16) || !aligned(p->conic_radius, 16) || !aligned(p->rgb, 16) ||
+        !aligned(p->rect, 16) || !aligned(p->count, 4))
+        return GS_ERR_ALIGNMENT;
+    return GS_OK;
+}
+
+int check_params(const gs_params *p, int64_t n) {
+    if (!p) return GS_ERR_INVALID_ARG;
+    if (n == 0) return GS_OK;
+    if (!p->means || !p->log_scales || !p->quats || !p->opacity_logits || !p->colors)
+        return GS_ERR_INVALID_ARG;
+    if (!aligned(p->means, 4) || !aligned(p->log_scales, 4) || !aligned(p->quats, 16) ||
+        !aligned(p->opacity_logits, 4) || !aligned(p->colors, 4))
+        return GS_ERR_ALIGNMENT;
+    return GS_OK;
+}
+
+int check_bins(const gs_bins *b, int64_t n, const CamConst &c, BinsLayout *L) {
+    if (!b || !b->scratch || !b->pair_tile || !b->pair_gid || !b->ranges || !b->n_pairs || !b->status)
+        return GS_ERR_INVALID_ARG;
+    if (n > b->max_n || (int64_t)c.tiles_x * c.tiles_y > b->max_tiles) return GS_ERR_INVALID_ARG;
+    if (b->max_n < 0 || b->max_pairs < 0 || b->max_n > kMaxCount || b->max_pairs > kMaxCount)
+        return GS_ERR_TOO_LARGE;
+    *L = bins_layout(b->max_n, b->max_pairs, b->max_tiles);
+    if (b->scratch_bytes < L->total || !aligned(b->scratch, 256)) return GS_ERR_INVALID_ARG;
+    return GS_OK;
+}
+
+inline cudaStream_t as_stream(void *s) { return reinterpret_cast<cudaStream_t>(s); }
+
+// ---------------------------------------------------------------- profiling
+struct ProfRec {
+    const char *name;
+    cudaEvent_t a, b;
+};
+std::vector<ProfRec> g_prof;
+std::vector<cudaEvent_t> g_pool;
+bool g_prof_on = false;
+bool g_prof_pending = false;
+int32_t g_prof_max = 0;
+
+cudaEvent_t pool_event() {
+    if (!g_pool.empty()) {
+        cudaEvent_t e = g_pool.back();
+        g_pool.pop_back();
+        return e;
+    }
+    cudaEvent_t e = nullptr;
+    cudaEventCreate(&e);
+    return e;
+}
+
+}  // namespace
+
+namespace gs {
+void prof_before(const char *name, cudaStream_t s) {
+    g_prof_pending = false;
+    if (!g_prof_on || (int32_t)g_prof.size() >= g_prof_max) return;
+    ProfRec r{name, pool_event(), pool_event()};
+    if (!r.a || !r.b) return;
+    cudaEventRecord(r.a, s);
+    g_prof.push_back(r);
+    g_prof_pending = true;
+}
+void prof_after(cudaStream_t s) {
+    if (!g_prof_pending) return;
+    cudaEventRecord(g_prof.back().b, s);
+    g_prof_pending = false;
+}
+}  // namespace gs
+
+extern "C" {
+
+int gs_version(void) { return 1; }
+
+const char *gs_error_string(int code) {
+    switch (code) {
+        case GS_OK: return "ok";
+        case GS_ERR_INVALID_ARG: return "invalid argument (size, pointer or camera value out of range)";
+        case GS_ERR_CAPACITY: return "pair list exceeds max_pairs: regrow the bins buffer and retry";
+        case GS_ERR_TOO_LARGE: return "N or max_pairs at or above 2^30";
+        case GS_ERR_ALIGNMENT: return "pointer not aligned as documented";
+        case GS_ERR_CUDA: return "CUDA runtime call or kernel launch failed";
+        case GS_ERR_DEVICE_TIMEOUT: return "a bounded device-side wait gave up";
+        default: return "unknown error code";
+    }
+}
+
+size_t gs_projected_bytes(int64_t n) {
+    if (n < 0) return 0;
+    const size_t v4 = align_up((size_t)n * 16, 256);
+    return 4 * v4 + align_up((size_t)n * 4, 256);
+}
+
+int gs_projected_carve(void *base, int64_t n, gs_projected *out) {
+    if (!out || n < 0 || (n > 0 && !base)) return GS_ERR_INVALID_ARG;
+    if (n > kMaxCount) return GS_ERR_TOO_LARGE;
+    if (!aligned(base, 256)) return GS_ERR_ALIGNMENT;
+    char *b = static_cast<char *>(base);
+    const size_t v4 = align_up((size_t)n * 16, 256);
+    out->xy_opacity_depth = reinterpret_cast<float *>(b);
+    out->conic_radius = reinterpret_cast<float *>(b + v4);
+    out->rgb = reinterpret_cast<float *>(b + 2 * v4);
+    out->rect = reinterpret_cast<int32_t *>(b + 3 * v4);
+    out->count = reinterpret_cast<uint32_t *>(b + 4 * v4);
+    return GS_OK;
+}
+
+size_t gs_bins_bytes(int64_t n, int64_t max_pairs, int32_t width, int32_t height) {
+    if (n < 0 || max_pairs < 0 || width < 1 || height < 1) return 0;
+    const int32_t tiles = ((width + kTile - 1) / kTile) * ((height + kTile - 1) / kTile);
+    return bins_layout(n, max_pairs, tiles).total;
+}
+
+int gs_bins_carve(void *base, int64_t n, int64_t max_pairs, int32_t width, int32_t height,
+                  gs_bins *out) {
+    if (!out || !base || n < 0 || max_pairs < 0 || width < 1 || height < 1 || width > 65536 ||
+        height > 65536)
+        return GS_ERR_INVALID_ARG;
+    if (n > kMaxCount || max_pairs > kMaxCount) return GS_ERR_TOO_LARGE;
+    if (!aligned(base, 256)) return GS_ERR_ALIGNMENT;
+    const int32_t tiles = ((width + kTile - 1) / kTile) * ((height + kTile - 1) / kTile);
+    const BinsLayout L = bins_layout(n, max_pairs, tiles);
+    char *b = static_cast<char *>(base);
+    std::memset(out, 0, sizeof(*out));
+    out->pair_tile = reinterpret_cast<uint32_t *>(b + L.pair_tile);
+    out->pair_gid = reinterpret_cast<uint32_t *>(b + L.pair_gid);
+    out->ranges = reinterpret_cast<uint32_t *>(b + L.ranges);
+    out->n_pairs = reinterpret_cast<uint64_t *>(b + L.n_pairs);
+    out->status = reinterpret_cast<int32_t *>(b + L.status);
+    out->max_pairs = max_pairs;
+    out->max_n = n;
+    out->max_tiles = tiles;
+    out->scratch = base;
+    out->scratch_bytes = L.total;
+    return GS_OK;
+}
+
+int gs_project(const gs_camera *cam, int64_t n, const gs_params *params, const gs_projected *out,
+               void *stream) {
+    CamConst c;
+    int rc = make_cam(cam, &c);
+    if (rc) return rc;
+    if (n < 0) return GS_ERR_INVALID_ARG;
+    if (n > kMaxCount) return GS_ERR_TOO_LARGE;
+    if ((rc = check_params(params, n)) || (rc = check_projected(out, n))) return rc;
+    return launch_project(c, n, *params, *out, as_stream(stream)) == cudaSuccess ? GS_OK : GS_ERR_CUDA;
+}
+
+int gs_read_status(const gs_bins *bins, int64_t *n_pairs_host, void *stream) {
+    if (!bins || !bins->status || !bins->n_pairs) return GS_ERR_INVALID_ARG;
+    int32_t st = 0;
+    uint64_t k = 0;
+    cudaStream_t s = as_stream(stream);
+    if (cudaMemcpyAsync(&st, bins->status, sizeof(st), cudaMemcpyDeviceToHost, s) != cudaSuccess ||
+        cudaMemcpyAsync(&k, bins->n_pairs, sizeof(k), cudaMemcpyDeviceToHost, s) != cudaSuccess ||
+        cudaStreamSynchronize(s) != cudaSuccess)
+        return GS_ERR_CUDA;
+    if (n_pairs_host) *n_pairs_host = (int64_t)k;
+    return st;
+}
+
+int gs_bin_and_sort(const gs_camera *cam, int64_t n, const gs_projected *proj, const gs_bins *bins,
+                    int64_t *n_pairs_host, void *stream) {
+    CamConst c;
+    int rc = make_cam(cam, &c);
+    if (rc) return rc;
+    if (n < 0) return GS_ERR_INVALID_ARG;
+    if (n > kMaxCount) return GS_ERR_TOO_LARGE;
+    BinsLayout L;
+    if ((rc = check_projected(proj, n)) || (rc = check_bins(bins, n, c, &L))) return rc;
+    if (launch_bin_and_sort(c, n, *proj, *bins, L, as_stream(stream)) != cudaSuccess) return GS_ERR_CUDA;
+    if (!n_pairs_host) return GS_OK;
+    rc = gs_read_status(bins, n_pairs_host, stream);
+    if (rc == GS_OK && *n_pairs_host > bins->max_pairs) rc = GS_ERR_CAPACITY;
+    return rc;
+}
+
+int gs_render_fwd(const gs_camera *cam, int64_t n, const gs_projected *proj, const gs_bins *bins,
+                  float *image, float *T_final, uint32_t *last, void *stream) {
+    CamConst c;
+    int rc = make_cam(cam, &c);
+    if (rc) return rc;
+    if (n < 0) return GS_ERR_INVALID_ARG;
+    BinsLayout L;
+    if ((rc = check_projected(proj, n)) || (rc = check_bins(bins, n, c, &L))) return rc;
+    if (!image || !T_final || !last) return GS_ERR_INVALID_ARG;
+    if (!aligned(image, 4) || !aligned(T_final, 4) || !aligned(last, 4)) return GS_ERR_ALIGNMENT;
+    return launch_render_fwd(c, *proj, *bins, image, T_final, last, as_stream(stream)) == cudaSuccess
+               ? GS_OK
+               : GS_ERR_CUDA;
+}
+
+int gs_render_bwd(const gs_camera *cam, int64_t n, const gs_params *params,
+                  const gs_projected *proj, const gs_bins *bins, const float *T_final,
+                  const uint32_t *last, const float *dL_dimage, float *grad2d,
+                  const gs_grads *grads, void *stream) {
+    CamConst c;
+    int rc = make_cam(cam, &c);
+    if (rc) return rc;
+    if (n < 0) return GS_ERR_INVALID_ARG;
+    BinsLayout L;
+    if ((rc = check_params(params, n)) || (rc = check_projected(proj, n)) ||
+        (rc = check_bins(bins, n, c, &L)))
+        return rc;
+    if (!T_final || !last || !dL_dimage || !grads) return GS_ERR_INVALID_ARG;
+    if (n > 0 && (!grad2d || !grads->means || !grads->log_scales || !grads->quats ||
+                  !grads->opacity_logits || !grads->colors))
+        return GS_ERR_INVALID_ARG;
+    if (!aligned(grad2d, 16) || !aligned(grads->quats, 16) || !aligned(T_final, 4) ||
+        !aligned(last, 4) || !aligned(dL_dimage, 4))
+        return GS_ERR_ALIGNMENT;
+    cudaStream_t s = as_stream(stream);
+    if (n > 0 && cudaMemsetAsync(grad2d, 0, (size_t)n * 12 * sizeof(float), s) != cudaSuccess)
+        return GS_ERR_CUDA;
+    if (launch_render_bwd(c, *proj, *bins, T_final, last, dL_dimage, grad2d, s) != cudaSuccess)
+        return GS_ERR_CUDA;
+    if (launch_project_bwd(c, n, *params, grad2d, *grads, s) != cudaSuccess) return GS_ERR_CUDA;
+    return GS_OK;
+}
+
+int gs_render_stats(const gs_camera *cam, int64_t n, const gs_projected *proj, const gs_bins *bins,
+                    const uint32_t *last, uint64_t *counts, void *stream) {
+    CamConst c;
+    int rc = make_cam(cam, &c);
+    if (rc) return rc;
+    if (n < 0) return GS_ERR_INVALID_ARG;
+    BinsLayout L;
+    if ((rc = check_projected(proj, n)) || (rc = check_bins(bins, n, c, &L))) return rc;
+    if (!last || !counts) return GS_ERR_INVALID_ARG;
+    if (!aligned(last, 4) || !aligned(counts, 8)) return GS_ERR_ALIGNMENT;
+    return launch_render_stats(c, *proj, *bins, last, counts, as_stream(stream)) == cudaSuccess
+               ? GS_OK
+               : GS_ERR_CUDA;
+}
+
+int gs_l1_loss_grad(const float *image, const float *target, int64_t count, float *dL_dimage,
+                    float *loss, void *stream) {
+    if (count < 0 || (count > 0 && (!image || !target || !dL_dimage))) return GS_ERR_INVALID_ARG;
+    return launch_l1(image, target, count, dL_dimage, loss, as_stream(stream)) == cudaSuccess
+               ? GS_OK
+               : GS_ERR_CUDA;
+}
+
+int gs_profile_begin(int32_t max_launches) {
+    if (max_launches < 0) return GS_ERR_INVALID_ARG;
+    for (auto &r : g_prof) {
+        g_pool.push_back(r.a);
+        g_pool.push_back(r.b);
+    }
+    g_prof.clear();
+    g_prof.reserve((size_t)max_launches);
+    g_prof_max = max_launches;
+    g_prof_on = true;
+    g_prof_pending = false;
+    return GS_OK;
+}
+
+int gs_profile_end(gs_profile_stat *out, int32_t max_stats) {
+    g_prof_on = false;
+    std::vector<gs_profile_stat> stats;
+    int rc = GS_OK;
+    for (auto &r : g_prof) {
+        float ms = 0.f;
+        if (cudaEventSynchronize(r.b) != cudaSuccess || cudaEventElapsedTime(&ms, r.a, r.b) != cudaSuccess) {
+            rc = GS_ERR_CUDA;
+            continue;
+        }
+        gs_profile_stat *hit = nullptr;
+        for (auto &s : stats)
+            if (std::strncmp(s.name, r.name, sizeof(s.name)) == 0) hit = &s;
+        if (!hit) {
+            gs_profile_stat s{};
+            std::snprintf(s.name, sizeof(s.name), "%s", r.name);
+            stats.push_back(s);
+            hit = &stats.back();
+        }
+        hit->launches += 1;
+        hit->total_ms += ms;
+    }
+    for (auto &r : g_prof) {
+        g_pool.push_back(r.a);
+        g_pool.push_back(r.b);
+    }
+    g_prof.clear();
+    if (rc != GS_OK) return rc;
+    const int32_t m = (int32_t)stats.size() < max_stats ? (int32_t)stats.size() : max_stats;
+    for (int32_t i = 0; i < m && out; i++) out[i] = stats[i];
+    return m;
+}
+
+}  // extern "C"

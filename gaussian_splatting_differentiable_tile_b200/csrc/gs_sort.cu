@@ -1,0 +1,471 @@
+// gs_sort.cu -- tile binning: depth sort, count scan, pair emit, pair sort,
+// per-tile ranges.
+//
+// Source: "SplatRs: The Week the Gap Closed", "Throughput: the tile
+// rasterizer" (project, count, emit, sort, range, blend) and "Gaussian
+// splatting in PyTorch" s5 (one global depth sort replaces per-tile sorts).
+//
+// The pages key each (tile, Gaussian) pair by (tile << 32 | depth bits) and
+// radix-sort the pairs on that key.  Here the depth half of the key is sorted
+// once per Gaussian instead of once per pair: Gaussians are first sorted by
+// depth (31 used bits of the positive float), their pairs are emitted in that
+// order, and a stable sort on the tile bits alone finishes the job.  The pair
+// order is identical (ties in depth by Gaussian id), while each pair passes
+// through ceil(tile_bits / 8) sort passes of 8 bytes instead of
+// ceil(43..45 / 8) passes of 12 bytes.
+//
+// Both sorts are LSD radix sorts built from one "onesweep" pass kernel:
+// a block ranks its 4096 keys with warp-level match/popc, publishes its digit
+// counts, and resolves its global offsets by a decoupled look-back over the
+// preceding partitions (bounded: a poll loop that runs out sets
+// GS_ERR_DEVICE_TIMEOUT and the kernel still finishes).  Partitions are taken
+// in ticket order so every block waits only on blocks already running.
+#include "gs_internal.cuh"
+
+namespace gs {
+namespace {
+
+__device__ __forceinline__ uint32_t lanemask_lt() {
+    uint32_t m;
+    asm("mov.u32 %0, %%lanemask_lt;" : "=r"(m));
+    return m;
+}
+
+// Exclusive block-wide scan of one value per thread (blockDim = 256).
+__device__ __forceinline__ uint32_t block_exclusive_scan_256(uint32_t v, uint32_t *s_warp,
+                                                             uint32_t *total) {
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    uint32_t x = v;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+        uint32_t y = __shfl_up_sync(0xffffffffu, x, o);
+        if (lane >= o) x += y;
+    }
+    if (lane == 31) s_warp[warp] = x;
+    __syncthreads();
+    uint32_t wpre = 0, tot = 0;
+#pragma unroll
+    for (int w = 0; w < 8; w++) {
+        uint32_t t = s_warp[w];
+        if (w < warp) wpre += t;
+        tot += t;
+    }
+    __syncthreads();
+    *total = tot;
+    return wpre + x - v;
+}
+
+// Depth keys of the drawable Gaussians and the four digit histograms of the
+// depth sort.
+__global__ void __launch_bounds__(256)
+k_depth_keys(int n, const float4 *__restrict__ xyod, const int4 *__restrict__ rect, int tiles_x,
+             int tiles_y, uint32_t *__restrict__ keys, uint32_t *__restrict__ hist) {
+    __shared__ uint32_t s_h[kMaxDepthPasses * kRadix];
+    for (int i = threadIdx.x; i < kMaxDepthPasses * kRadix; i += blockDim.x) s_h[i] = 0;
+    __syncthreads();
+    for (int g = blockIdx.x * blockDim.x + threadIdx.x; g < n; g += gridDim.x * blockDim.x) {
+        int x0, y0, w;
+        const uint32_t c = rect_tiles(rect[g], tiles_x, tiles_y, x0, y0, w);
+        const uint32_t key = c > 0 ? __float_as_uint(xyod[g].w) : kInvalidDepthKey;
+        keys[g] = key;
+#pragma unroll
+        for (int k = 0; k < kMaxDepthPasses; k++) atomicAdd(&s_h[k * kRadix + ((key >> (8 * k)) & 0xFF)], 1u);
+    }
+    __syncthreads();
+    for (int i = threadIdx.x; i < kMaxDepthPasses * kRadix; i += blockDim.x)
+        if (s_h[i]) atomicAdd(&hist[i], s_h[i]);
+}
+
+// One LSD radix pass over bits [shift, shift + bits) of 32-bit keys with
+// 32-bit values.  n = min(*n_dev, n_cap) when n_dev is given, else n_host.
+// With iota_vals the values are the input indices (first pass of a sort).
+// When check_status is set the pass does nothing if *status is non-zero.
+__global__ void __launch_bounds__(kSortThreads)
+k_onesweep(const uint32_t *__restrict__ keys_in, const uint32_t *__restrict__ vals_in,
+           uint32_t *__restrict__ keys_out, uint32_t *__restrict__ vals_out,
+           const uint64_t *__restrict__ n_dev, uint32_t n_host, uint32_t n_cap, int shift, int bits,
+           const uint32_t *__restrict__ hist, uint32_t *__restrict__ lookback,
+           uint32_t *__restrict__ ticket, int32_t *__restrict__ status, int iota_vals,
+           int check_status) {
+    __shared__ uint32_t s_warp_hist[kSortThreads / 32][kRadix];
+    __shared__ uint32_t s_digit_start[kRadix];
+    __shared__ uint32_t s_global_base[kRadix];
+    __shared__ uint32_t s_hist_excl[kRadix];
+    __shared__ uint32_t s_keys[kSortPart];
+    __shared__ uint32_t s_vals[kSortPart];
+    __shared__ uint32_t s_scan[8];
+    __shared__ uint32_t s_part;
+    __shared__ int s_skip;
+
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    if (tid == 0) s_skip = check_status ? (*(volatile int32_t *)status != 0) : 0;
+    __syncthreads();
+    if (s_skip) return;
+    uint32_t n = n_host;
+    if (n_dev) {
+        const uint64_t nd = *n_dev;
+        n = nd < (uint64_t)n_cap ? (uint32_t)nd : n_cap;
+    }
+    const uint32_t mask = (1u << bits) - 1u;
+    const int radix = 1 << bits;
+
+    // Exclusive scan of the global digit histogram: where each digit starts.
+    {
+        uint32_t tot;
+        const uint32_t h = tid < radix ? hist[tid] : 0u;
+        s_hist_excl[tid] = block_exclusive_scan_256(h, s_scan, &tot);
+    }
+
+    for (;;) {
+        if (tid == 0) s_part = atomicAdd(ticket, 1u);
+        __syncthreads();
+        const uint32_t p = s_part;
+        if ((uint64_t)p * kSortPart >= n) break;
+        for (int i = tid; i < (kSortThreads / 32) * kRadix; i += kSortThreads)
+            (&s_warp_hist[0][0])[i] = 0;
+        __syncthreads();
+
+        // Load: warp w owns keys [w*32*ITEMS, (w+1)*32*ITEMS) of the partition,
+        // item i of lane l at offset i*32 + l: coalesced, and index order is
+        // (warp, item, lane), which the ranking below preserves (stable).
+        const uint32_t base = p * kSortPart + warp * (32 * kSortItems);
+        uint32_t key[kSortItems], val[kSortItems], dig[kSortItems], rank[kSortItems];
+#pragma unroll
+        for (int i = 0; i < kSortItems; i++) {
+            const uint32_t idx = base + i * 32 + lane;
+            if (idx < n) {
+                key[i] = keys_in[idx];
+                val[i] = iota_vals ? idx : vals_in[idx];
+                dig[i] = (key[i] >> shift) & mask;
+            } else {
+                key[i] = 0; val[i] = 0;
+                dig[i] = kRadix;  // sentinel: not counted
+            }
+        }
+        // Warp-level ranking of each item among equal digits.
+#pragma unroll
+        for (int i = 0; i < kSortItems; i++) {
+            const uint32_t d = dig[i];
+            const uint32_t peers = __match_any_sync(0xffffffffu, d);
+            const int leader = __ffs(peers) - 1;
+            uint32_t b = 0;
+            if (d < kRadix) b = s_warp_hist[warp][d];
+            __syncwarp();
+            if (d < kRadix && lane == leader) s_warp_hist[warp][d] = b + __popc(peers);
+            __syncwarp();
+            rank[i] = b + __popc(peers & lanemask_lt());
+        }
+        __syncthreads();
+
+        // Per digit (thread = digit): warp offsets and the block's count.
+        uint32_t block_count = 0;
+        {
+            const int d = tid;
+#pragma unroll
+            for (int w = 0; w < kSortThreads / 32; w++) {
+                const uint32_t c = s_warp_hist[w][d];
+                s_warp_hist[w][d] = block_count;
+                block_count += c;
+            }
+        }
+        // Publish this partition's count for the digit, then look back.
+        {
+            const int d = tid;
+            uint32_t *lb = lookback + (size_t)p * kRadix + d;
+            uint32_t excl = 0;
+            if (d < radix) {
+                if (p == 0) {
+                    st_relaxed(lb, kFlagInclusive | block_count);
+                } else {
+                    st_relaxed(lb, kFlagAggregate | block_count);
+                    int64_t q = (int64_t)p - 1;
+                    uint32_t spins = 0;
+                    while (q >= 0) {
+                        const uint32_t w = ld_relaxed(lookback + (size_t)q * kRadix + d);
+                        const uint32_t flag = w & ~kValueMask;
+                        if (flag == 0u) {
+                            if (++spins > kSpinLimit) {
+                                set_status(status, GS_ERR_DEVICE_TIMEOUT);
+                                break;
+                            }
+                            continue;
+                        }
+                        excl += w & kValueMask;
+                        if (flag == kFlagInclusive) break;
+                        --q;
+                    }
+                    st_relaxed(lb, kFlagInclusive | ((excl + block_count) & kValueMask));
+                }
+            }
+            s_global_base[d] = s_hist_excl[d] + excl;
+            uint32_t tot;
+            s_digit_start[d] = block_exclusive_scan_256(d < radix ? block_count : 0u, s_scan, &tot);
+        }
+        __syncthreads();
+
+        // Local reorder through shared memory, then coalesced-run stores.
+        uint32_t valid_count = 0;
+#pragma unroll
+        for (int i = 0; i < kSortItems; i++) {
+            const uint32_t d = dig[i];
+            if (d < kRadix) {
+                const uint32_t loc = s_digit_start[d] + s_warp_hist[warp][d] + rank[i];
+                s_keys[loc] = key[i];
+                s_vals[loc] = val[i];
+            }
+        }
+        {
+            const uint64_t rem = (uint64_t)n - (uint64_t)p * kSortPart;
+            valid_count = rem < (uint64_t)kSortPart ? (uint32_t)rem : (uint32_t)kSortPart;
+        }
+        __syncthreads();
+        for (uint32_t j = tid; j < valid_count; j += kSortThreads) {
+            const uint32_t k = s_keys[j];
+            const uint32_t d = (k >> shift) & mask;
+            const uint32_t pos = s_global_base[d] + (j - s_digit_start[d]);
+            if (pos < n) {
+                keys_out[pos] = k;
+                vals_out[pos] = s_vals[j];
+            }
+        }
+        __syncthreads();
+    }
+}
+
+// Fused exclusive scan of the tile counts (in depth order) and pair emit.
+// One block per 2048 Gaussians of the depth order; the block's offset comes
+// from a decoupled look-back over 64-bit inclusive prefixes.  Each pair is
+// (tile, Gaussian id), written at its scanned offset; a Gaussian's tiles are
+// emitted row by row.  The digit histograms of the tile sort are gathered on
+// the way.  Pairs past max_pairs are not written: the block records
+// GS_ERR_CAPACITY, and n_pairs still receives the full count.
+__global__ void __launch_bounds__(kScanThreads)
+k_scan_emit(int n, const uint32_t *__restrict__ sorted_gid, const int4 *__restrict__ rect,
+            int tiles_x, int tiles_y, uint32_t *__restrict__ ptile,
+            uint32_t *__restrict__ pgid, uint64_t max_pairs, uint64_t *__restrict__ lookback,
+            uint32_t *__restrict__ ticket, uint64_t *__restrict__ n_pairs,
+            int32_t *__restrict__ status, uint32_t *__restrict__ tile_hist, int tile_passes,
+            int tile_bpp) {
+    __shared__ uint32_t s_incl[kScanPart];
+    __shared__ uint32_t s_gid[kScanPart];
+    __shared__ uint2 s_rect[kScanPart];
+    __shared__ uint32_t s_hist[kMaxTilePasses * kRadix];
+    __shared__ uint32_t s_scan[8];
+    __shared__ uint32_t s_part;
+    __shared__ unsigned long long s_prefix;
+
+    const int tid = threadIdx.x;
+    for (int i = tid; i < kMaxTilePasses * kRadix; i += kScanThreads) s_hist[i] = 0;
+    if (tid == 0) s_part = atomicAdd(ticket, 1u);
+    __syncthreads();
+    const uint32_t p = s_part;
+    const int64_t base = (int64_t)p * kScanPart;
+
+    uint32_t c[kScanItems], gid[kScanItems];
+    uint2 rc[kScanItems];
+    uint32_t tsum = 0;
+#pragma unroll
+    for (int i = 0; i < kScanItems; i++) {
+        const int64_t idx = base + tid * kScanItems + i;
+        gid[i] = 0;
+        c[i] = 0;
+        rc[i] = make_uint2(0u, 0u);
+        if (idx < n) {
+            gid[i] = sorted_gid[idx];
+            int x0, y0, w;
+            c[i] = rect_tiles(rect[gid[i]], tiles_x, tiles_y, x0, y0, w);
+            rc[i] = make_uint2((uint32_t)x0 | ((uint32_t)y0 << 16), (uint32_t)w);
+        }
+        tsum += c[i];
+    }
+    uint32_t block_total;
+    const uint32_t toff = block_exclusive_scan_256(tsum, s_scan, &block_total);
+    uint32_t run = toff;
+#pragma unroll
+    for (int i = 0; i < kScanItems; i++) {
+        const int k = tid * kScanItems + i;
+        run += c[i];
+        s_incl[k] = run;
+        s_gid[k] = gid[i];
+        s_rect[k] = rc[i];
+    }
+    if (tid == 0) {
+        uint64_t prefix = 0;
+        uint64_t *lb = lookback + p;
+        if (p == 0) {
+            st_relaxed64(lb, kFlag64Inclusive | (uint64_t)block_total);
+        } else {
+            st_relaxed64(lb, kFlag64Aggregate | (uint64_t)block_total);
+            int64_t q = (int64_t)p - 1;
+            uint32_t spins = 0;
+            while (q >= 0) {
+                const uint64_t w = ld_relaxed64(lookback + q);
+                const uint64_t flag = w & ~kValue64Mask;
+                if (flag == 0ull) {
+                    if (++spins > kSpinLimit) {
+                        set_status(status, GS_ERR_DEVICE_TIMEOUT);
+                        break;
+                    }
+                    continue;
+                }
+                prefix += w & kValue64Mask;
+                if (flag == kFlag64Inclusive) break;
+                --q;
+            }
+            st_relaxed64(lb, kFlag64Inclusive | ((prefix + block_total) & kValue64Mask));
+        }
+        s_prefix = prefix;
+        if (base + kScanPart >= n) *n_pairs = prefix + block_total;
+    }
+    __syncthreads();
+    const uint64_t prefix = s_prefix;
+    const uint32_t dmask = (1u << tile_bpp) - 1u;
+    bool overflow = false;
+    for (uint32_t j = tid; j < block_total; j += kScanThreads) {
+        // item k: the first whose inclusive prefix exceeds j
+        int lo = 0, hi = kScanPart - 1;
+        while (lo < hi) {
+            const int mid = (lo + hi) >> 1;
+            if (s_incl[mid] > j) hi = mid; else lo = mid + 1;
+        }
+        const uint32_t li = j - (lo == 0 ? 0u : s_incl[lo - 1]);
+        const uint2 r = s_rect[lo];
+        const uint32_t w = r.y;
+        const uint32_t row = li / w;
+        const uint32_t tile = ((r.x >> 16) + row) * (uint32_t)tiles_x + (r.x & 0xFFFFu) + (li - row * w);
+        const uint64_t pos = prefix + j;
+        if (pos < max_pairs) {
+            ptile[pos] = tile;
+            pgid[pos] = s_gid[lo];
+            for (int k = 0; k < tile_passes; k++)
+                atomicAdd(&s_hist[k * kRadix + ((tile >> (k * tile_bpp)) & dmask)], 1u);
+        } else {
+            overflow = true;
+        }
+    }
+    if (overflow) set_status(status, GS_ERR_CAPACITY);
+    __syncthreads();
+    for (int i = tid; i < tile_passes * kRadix; i += kScanThreads)
+        if (s_hist[i]) atomicAdd(&tile_hist[i], s_hist[i]);
+}
+
+// [start, end) of each tile in the sorted pair list.  Ranges were zeroed
+// beforehand, so empty tiles stay [0, 0); on a recorded error all stay empty.
+__global__ void __launch_bounds__(256)
+k_ranges(const uint32_t *__restrict__ ptile, const uint64_t *__restrict__ n_pairs,
+         uint32_t *__restrict__ ranges, const int32_t *__restrict__ status) {
+    if (*(volatile const int32_t *)status != 0) return;
+    const uint64_t K = *n_pairs;
+    for (uint64_t j = (uint64_t)blockIdx.x * blockDim.x + threadIdx.x; j < K;
+         j += (uint64_t)gridDim.x * blockDim.x) {
+        const uint32_t t = ptile[j];
+        if (j == 0 || ptile[j - 1] != t) ranges[2 * (size_t)t] = (uint32_t)j;
+        if (j == K - 1 || ptile[j + 1] != t) ranges[2 * (size_t)t + 1] = (uint32_t)(j + 1);
+    }
+}
+
+int num_sms() {
+    static int sms = 0;
+    if (sms == 0) {
+        int dev = 0;
+        cudaGetDevice(&dev);
+        cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+        if (sms <= 0) sms = 148;
+    }
+    return sms;
+}
+
+}  // namespace
+
+cudaError_t launch_bin_and_sort(const CamConst &c, int64_t n, const gs_projected &proj,
+                                const gs_bins &bins, const BinsLayout &L, cudaStream_t s) {
+    char *base = static_cast<char *>(bins.scratch);
+    auto U32 = [&](size_t off) { return reinterpret_cast<uint32_t *>(base + off); };
+    int32_t *status = reinterpret_cast<int32_t *>(base + L.status);
+    uint64_t *n_pairs = reinterpret_cast<uint64_t *>(base + L.n_pairs);
+    uint32_t *tickets = U32(L.tickets);
+    uint32_t *depth_hist = U32(L.depth_hist);
+    uint32_t *tile_hist = U32(L.tile_hist);
+    uint32_t *ranges = U32(L.ranges);
+    const int tiles = c.tiles_x * c.tiles_y;
+
+    cudaError_t e = cudaMemsetAsync(base, 0, L.zero_bytes, s);
+    if (e != cudaSuccess) return e;
+    if (n == 0) return cudaSuccess;  // K = 0, all ranges empty
+
+    const int sms = num_sms();
+    const uint32_t nn = (uint32_t)n;
+    // 1. depth keys + histograms
+    {
+        const int blocks = (int)std::min<int64_t>((n + 255) / 256, (int64_t)sms * 4);
+        prof_before("depth_keys", s);
+        k_depth_keys<<<blocks, 256, 0, s>>>((int)n, reinterpret_cast<const float4 *>(proj.xy_opacity_depth),
+                                             reinterpret_cast<const int4 *>(proj.rect), c.tiles_x, c.tiles_y,
+                                             U32(L.keys_a), depth_hist);
+        prof_after(s);
+    }
+    // 2. depth sort: 31 bits in four passes, A -> B -> A -> B -> A
+    {
+        const int shifts[4] = {0, 8, 16, 24}, bits[4] = {8, 8, 8, 7};
+        uint32_t *ka = U32(L.keys_a), *va = U32(L.vals_a), *kb = U32(L.keys_b), *vb = U32(L.vals_b);
+        const int64_t parts = (n + kSortPart - 1) / kSortPart;
+        const int blocks = (int)std::min<int64_t>(parts, (int64_t)sms * 4);
+        for (int pass = 0; pass < 4; pass++) {
+            const bool even = (pass % 2) == 0;
+            prof_before("depth_sort", s);
+            k_onesweep<<<blocks, kSortThreads, 0, s>>>(
+                even ? ka : kb, even ? va : vb, even ? kb : ka, even ? vb : va, nullptr, nn, nn,
+                shifts[pass], bits[pass], depth_hist + pass * kRadix,
+                U32(L.depth_lb) + (size_t)pass * L.depth_parts * kRadix, tickets + pass, status,
+                pass == 0 ? 1 : 0, 0);
+            prof_after(s);
+        }
+    }
+    // 3. scan + emit, in depth order
+    int tile_bits = 0;
+    while ((1 << tile_bits) < tiles) tile_bits++;
+    const int tile_passes = (tile_bits + kRadixBits - 1) / kRadixBits;
+    const int tile_bpp = tile_passes ? (tile_bits + tile_passes - 1) / tile_passes : 1;
+    uint32_t *ta = U32(L.ptile_a), *ga = U32(L.pgid_a), *tb = U32(L.ptile_b), *gb = U32(L.pgid_b);
+    uint32_t *to = bins.pair_tile, *go = bins.pair_gid;
+    {
+        const int blocks = (int)((n + kScanPart - 1) / kScanPart);
+        uint32_t *et = tile_passes == 0 ? to : ta, *eg = tile_passes == 0 ? go : ga;
+        prof_before("scan_emit", s);
+        k_scan_emit<<<blocks, kScanThreads, 0, s>>>(
+            (int)n, U32(L.vals_a), reinterpret_cast<const int4 *>(proj.rect), c.tiles_x, c.tiles_y,
+            et, eg, (uint64_t)bins.max_pairs, reinterpret_cast<uint64_t *>(base + L.scan_lb),
+            tickets + 4, n_pairs, status, tile_hist, tile_passes, tile_bpp);
+        prof_after(s);
+    }
+    // 4. stable pair sort on the tile bits
+    {
+        const int64_t parts = (bins.max_pairs + kSortPart - 1) / kSortPart;
+        const int blocks = (int)std::max<int64_t>(1, std::min<int64_t>(parts, (int64_t)sms * 4));
+        uint32_t *st = ta, *sg = ga;
+        for (int pass = 0; pass < tile_passes; pass++) {
+            uint32_t *dt, *dg;
+            if (pass == tile_passes - 1) { dt = to; dg = go; }
+            else if (st == ta) { dt = tb; dg = gb; }
+            else { dt = ta; dg = ga; }
+            const int sh = pass * tile_bpp;
+            const int nb = std::min(tile_bpp, tile_bits - sh);
+            prof_before("tile_sort", s);
+            k_onesweep<<<blocks, kSortThreads, 0, s>>>(
+                st, sg, dt, dg, n_pairs, 0u, (uint32_t)bins.max_pairs, sh, nb, tile_hist + pass * kRadix,
+                U32(L.tile_lb) + (size_t)pass * L.tile_parts * kRadix, tickets + 5 + pass, status, 0, 1);
+            prof_after(s);
+            st = dt; sg = dg;
+        }
+    }
+    // 5. ranges
+    {
+        const int blocks = sms * 4;
+        prof_before("ranges", s);
+        k_ranges<<<blocks, 256, 0, s>>>(bins.pair_tile, n_pairs, ranges, status);
+        prof_after(s);
+    }
+    return cudaGetLastError();
+}
+
+}  // namespace gs

@@ -1,0 +1,253 @@
+/*
+ * gs.h -- C ABI of a differentiable, tile-binned 3D Gaussian splatting
+ * rasterizer for NVIDIA B200 (sm_100a).  Library: libgs.so.
+ *
+ * The hot path is four calls, made in this order on one CUDA stream:
+ *
+ *   gs_project       raw parameters -> per-Gaussian projected records
+ *   gs_bin_and_sort  records -> (tile, Gaussian) pairs sorted by tile, then
+ *                    by depth, plus each tile's [start, end) range
+ *   gs_render_fwd    front-to-back alpha blend of every 16x16 tile
+ *   gs_render_bwd    back-to-front gradient of the blend, then the chain rule
+ *                    to the raw parameters
+ *
+ * Sources (cited by page title and section):
+ *   [GSP]  "Gaussian splatting in PyTorch" (coderigor.dev), s1-s8
+ *   [WEEK] "SplatRs: The Week the Gap Closed", "Throughput: the tile
+ *          rasterizer" (project, count, emit, sort, range, blend)
+ *   [PIX4] "SplatRs: We Gave the Model 4x More Pixels and It Got Worse",
+ *          "Lesson 2 -- Your GPU will lie by omission" (pair-list size,
+ *          pre-flight guards, errors that must not be silent)
+ *   [BLOG] 3D Gaussian Splatting course blog index (a backward pass that
+ *          recomputes the blend weights instead of storing them)
+ *
+ * Conventions shared by every call
+ *   - All floating point is IEEE single precision.
+ *   - Every pointer inside gs_params, gs_grads, gs_projected and gs_bins,
+ *     and every array argument, is DEVICE memory owned by the caller, unless
+ *     the comment says "host".  The library never allocates or frees device
+ *     memory; size queries tell the caller how much to allocate.
+ *   - Arrays of 4-vectors must be 16-byte aligned; all others 4-byte aligned
+ *     (GS_ERR_ALIGNMENT otherwise).
+ *   - `stream` is a cudaStream_t (NULL = the legacy default stream).  Every
+ *     call only enqueues work on it and returns, except where a comment says
+ *     it synchronizes.
+ *   - Return value: GS_OK (0), or a negative GS_ERR_* code.  No call aborts
+ *     the process, throws, or fails silently ([PIX4] Lesson 2).  Arguments
+ *     are checked before anything is launched; on an argument error nothing
+ *     is enqueued.
+ *   - The library holds no per-call state between calls; calls on different
+ *     streams with disjoint buffers may run concurrently.
+ */
+#ifndef GS_H_
+#define GS_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#define GS_TILE 16 /* tile edge in pixels */
+
+enum {
+    GS_OK = 0,
+    GS_ERR_INVALID_ARG = -1,    /* a size, pointer or camera value is out of range */
+    GS_ERR_CAPACITY = -2,       /* the pair list needs more than max_pairs entries */
+    GS_ERR_TOO_LARGE = -3,      /* N or max_pairs at or above 2^30 */
+    GS_ERR_ALIGNMENT = -4,      /* a pointer is not aligned as documented */
+    GS_ERR_CUDA = -5,           /* a CUDA runtime call or launch failed */
+    GS_ERR_DEVICE_TIMEOUT = -6  /* a bounded device-side wait gave up */
+};
+
+/* Pinhole camera ([GSP] s3).  Host struct, passed by pointer. */
+typedef struct gs_camera {
+    float viewmat[16];    /* row-major 4x4 world-to-camera [R | t; 0 0 0 1], OpenCV
+                             axes: +x right, +y down, +z forward */
+    float fx, fy, cx, cy; /* intrinsics in pixels; pixel (row i, col j) is sampled
+                             at (j + 0.5, i + 0.5) ([GSP] s5) */
+    int32_t width, height;/* image size in pixels, each in [1, 65536] */
+    float near_z;         /* Gaussians with camera z <= near_z are culled (0.01,
+                             [GSP] s6) */
+    float bg[3];          /* background colour, weighted by the final
+                             transmittance ([GSP] s5) */
+} gs_camera;
+
+/* Raw (unconstrained) parameters of N Gaussians ([GSP] s1), fp32, C-contiguous. */
+typedef struct gs_params {
+    const float *means;          /* [N][3] world-space centres */
+    const float *log_scales;     /* [N][3] scale = exp(log_scale) per axis */
+    const float *quats;          /* [N][4] (w, x, y, z), any norm; normalised with
+                                    max(|q|, 1e-12) so zero gives the identity */
+    const float *opacity_logits; /* [N]    opacity = sigmoid(logit) */
+    const float *colors;         /* [N][3] RGB used directly (SH degree 0) */
+} gs_params;
+
+/* Gradients of a scalar loss with respect to gs_params, same layouts.
+ * Overwritten (not accumulated) by gs_render_bwd. */
+typedef struct gs_grads {
+    float *means, *log_scales, *quats, *opacity_logits, *colors;
+} gs_grads;
+
+/* Projected records of N Gaussians, written by gs_project ([GSP] s1-s4).
+ * The layout is public so that records computed elsewhere can be binned and
+ * rendered.  gs_projected_carve lays all arrays out in one buffer. */
+typedef struct gs_projected {
+    float *xy_opacity_depth; /* [N][4]: mean2d x, y (px); opacity in (0,1); camera z */
+    float *conic_radius;     /* [N][4]: A, B, C with sigma = 1/2 (A dx^2 + C dy^2) + B dx dy
+                                ([GSP] s4); radius in px (an integer value) */
+    float *rgb;              /* [N][4]: r, g, b, 0 */
+    int32_t *rect;           /* [N][4]: tile x0, y0, x1, y1, inclusive, clamped to the
+                                tile grid; x0 > x1 or y0 > y1 when nothing is touched */
+    uint32_t *count;         /* [N]: tiles touched = rectangle area; 0 when culled */
+} gs_projected;
+
+/* Bytes of one buffer holding every gs_projected array for n Gaussians. */
+size_t gs_projected_bytes(int64_t n);
+/* Points the fields of *out into `base` (device, 256-byte aligned, at least
+ * gs_projected_bytes(n) bytes).  Host-only arithmetic; launches nothing. */
+int gs_projected_carve(void *base, int64_t n, gs_projected *out);
+
+/* Binning state: the sorted pair list, per-tile ranges, status words and the
+ * sort's scratch, all in one caller-owned device buffer carved by
+ * gs_bins_carve.  A gs_bins carved for (n, max_pairs, width, height) serves
+ * any call with at most n Gaussians and an image of at most that many tiles. */
+typedef struct gs_bins {
+    uint32_t *pair_tile;  /* [max_pairs] tile id (ty * tiles_x + tx) of each pair, ascending */
+    uint32_t *pair_gid;   /* [max_pairs] Gaussian id of each pair; within a tile, ordered by
+                             (float bits of camera z, id): the order of the 64-bit key
+                             (tile << 32 | depth bits) of [WEEK] with ties by id */
+    uint32_t *ranges;     /* [tiles][2] start, end of each tile's pairs; [0, 0) when empty */
+    uint64_t *n_pairs;    /* [1] total pairs K of the last gs_bin_and_sort (also when
+                             K > max_pairs) */
+    int32_t *status;      /* [1] 0, or the GS_ERR_* code a kernel of the last
+                             gs_bin_and_sort recorded (GS_ERR_CAPACITY,
+                             GS_ERR_DEVICE_TIMEOUT) */
+    int64_t max_pairs;    /* capacity of pair_tile / pair_gid */
+    int64_t max_n;        /* largest N this buffer was carved for */
+    int32_t max_tiles;    /* largest tile count this buffer was carved for */
+    int32_t reserved;
+    void *scratch;        /* sort and scan scratch (internal layout) */
+    size_t scratch_bytes;
+} gs_bins;
+
+/* Bytes of one buffer holding a gs_bins for at most n Gaussians, max_pairs
+ * pairs and a width x height image.  [PIX4] Lesson 2: 400k Gaussians at full
+ * resolution needed > 16.7M pairs; size max_pairs from a first call's K. */
+size_t gs_bins_bytes(int64_t n, int64_t max_pairs, int32_t width, int32_t height);
+/* Carves *out from `base` (device, 256-byte aligned, gs_bins_bytes bytes).
+ * Host-only arithmetic.  GS_ERR_TOO_LARGE if n or max_pairs >= 2^30. */
+int gs_bins_carve(void *base, int64_t n, int64_t max_pairs, int32_t width, int32_t height,
+                  gs_bins *out);
+
+/* Projection ([GSP] s1-s4, s6), one thread per Gaussian: activations;
+ * Sigma = R S S^T R^T; t = W mu + tv; cull if z <= near_z or any projected
+ * value is not finite; J from x/z, y/z clamped to the frustum widened by 0.3
+ * of the half-FoV tangent; Sigma' = J W Sigma W^T J^T + 0.3 I; det clamped
+ * at 1e-10; conic = (c, -b, a)/det; radius = ceil(3 sqrt(lambda_max)) with
+ * the root term floored at 0.1; mean2d = (fx x/z + cx, fy y/z + cy);
+ * tile rectangle per axis floor((m -+ r)/16) in single precision, clamped
+ * to the grid.  Culled Gaussians get count 0 and an empty rectangle.
+ * n may be 0.  Errors: INVALID_ARG (n < 0, null pointer with n > 0, bad
+ * camera), TOO_LARGE (n >= 2^30), ALIGNMENT, CUDA. */
+int gs_project(const gs_camera *cam, int64_t n, const gs_params *params, const gs_projected *out,
+               void *stream);
+
+/* Binning and sorting ([WEEK] count, emit, sort, range): sorts the drawable
+ * Gaussians by depth (LSD radix over the 31 used bits of camera z), scans
+ * their tile counts in that order, emits one (tile, id) pair per touched
+ * tile at the scanned offsets, sorts the pairs stably by tile (LSD radix over
+ * the used tile-id bits only), and writes each tile's range.  The result is
+ * the pair order of the 64-bit key (tile << 32 | depth bits) with ties by id.
+ * Uses `proj` from gs_project (or any records in that layout): binning reads
+ * each record's depth and its rectangle (clamped to the tile grid; `count` is
+ * not read), so no record can produce a tile id outside the grid.
+ * If n_pairs_host (HOST pointer) is non-NULL the call synchronizes `stream`,
+ * stores K there, and returns GS_ERR_CAPACITY if K > bins->max_pairs (the
+ * caller may regrow and retry) or the status a kernel recorded.  If it is
+ * NULL nothing synchronizes: K and any error land in bins->n_pairs and
+ * bins->status (read them with gs_read_status); on an error every tile's
+ * range is left empty, so the render draws only background.
+ * Errors: INVALID_ARG, TOO_LARGE, ALIGNMENT, CUDA, CAPACITY, DEVICE_TIMEOUT. */
+int gs_bin_and_sort(const gs_camera *cam, int64_t n, const gs_projected *proj,
+                    const gs_bins *bins, int64_t *n_pairs_host, void *stream);
+
+/* Forward blend ([GSP] s5; [WEEK] blend), one CTA per 16x16 tile: for each
+ * pixel, its tile's pairs in order, sigma as above at (j + 0.5, i + 0.5),
+ * alpha = min(0.99, o exp(-sigma)); skip if sigma < 0 or alpha < 1/255;
+ * stop (without adding) once T (1 - alpha) < 1e-4; C += c alpha T.
+ * Outputs (device, caller-owned, fully overwritten):
+ *   image   [H][W][3]  C + T_final bg
+ *   T_final [H][W]     final transmittance
+ *   last    [H][W]     one past the index (into pair_gid) of the last entry the
+ *                      pixel added; the tile's start when it added none
+ * Errors: INVALID_ARG, ALIGNMENT, CUDA. */
+int gs_render_fwd(const gs_camera *cam, int64_t n, const gs_projected *proj, const gs_bins *bins,
+                  float *image, float *T_final, uint32_t *last, void *stream);
+
+/* Backward ([GSP] s6; [BLOG]): one CTA per tile walks each pixel's added
+ * entries back to front from `last`, recovering T_i = T_{i+1} / (1 - alpha_i)
+ * instead of storing weights; dL/dalpha_i = T_i <c_i - R_i, g> with
+ * R_last = bg, R_{i-1} = alpha_i c_i + (1 - alpha_i) R_i; no gradient through
+ * a capped alpha; per-pixel terms are reduced across the warp before global
+ * atomics.  Then the chain rule to the raw parameters, one thread per
+ * Gaussian.  Culled Gaussians get exact zeros.
+ *   dL_dimage [H][W][3]  gradient of the loss with respect to `image`
+ *   grad2d    [N][12]    caller scratch, 16-byte aligned; overwritten.  On
+ *                        return holds per Gaussian dL/d(mean2d x, y), dL/dA,
+ *                        dL/dB, dL/dC, dL/dopacity, dL/d(r, g, b), 0, 0, 0
+ *   grads                raw-parameter gradients, overwritten
+ * `proj`, `bins`, T_final and last must be those of the forward call.
+ * Errors: INVALID_ARG, ALIGNMENT, CUDA. */
+int gs_render_bwd(const gs_camera *cam, int64_t n, const gs_params *params,
+                  const gs_projected *proj, const gs_bins *bins, const float *T_final,
+                  const uint32_t *last, const float *dL_dimage, float *grad2d,
+                  const gs_grads *grads, void *stream);
+
+/* Work counts of one forward frame, for roofline arithmetic (not part of the
+ * rendering path; it re-walks the blend with counters and is slower).
+ * counts (device, [4] uint64, overwritten):
+ *   [0] entries visited by the forward: per pixel, its tile's entries up to
+ *       and including the one that stopped it (all of them if none did)
+ *   [1] entries added (contributing) over all pixels
+ *   [2] entries the backward walks: per pixel, last - tile start
+ *   [3] pixels
+ * `last` must be the forward's output for the same proj and bins.
+ * Errors: INVALID_ARG, ALIGNMENT, CUDA. */
+int gs_render_stats(const gs_camera *cam, int64_t n, const gs_projected *proj,
+                    const gs_bins *bins, const uint32_t *last, uint64_t *counts, void *stream);
+
+/* L1 photometric loss of the training step: loss = mean |image - target| over
+ * `count` values; dL_dimage = sign(image - target) / count (sign(0) = 0).
+ * loss (device, nullable) receives the mean.  Errors: INVALID_ARG, CUDA. */
+int gs_l1_loss_grad(const float *image, const float *target, int64_t count, float *dL_dimage,
+                    float *loss, void *stream);
+
+/* Synchronizes `stream`, then returns bins->status and stores K in
+ * *n_pairs_host (HOST, nullable).  GS_ERR_CUDA if the copy fails. */
+int gs_read_status(const gs_bins *bins, int64_t *n_pairs_host, void *stream);
+
+/* Static, human-readable text for a return code. */
+const char *gs_error_string(int code);
+
+/* Per-kernel timing.  Between gs_profile_begin and gs_profile_end the library
+ * records a CUDA event pair around each kernel it launches, on the stream it
+ * launches it on.  gs_profile_end synchronizes those events and fills at
+ * most max_stats entries (one per kernel name); returns how many.  Not
+ * thread-safe; meant for benchmarks. */
+typedef struct gs_profile_stat {
+    char name[32];
+    int32_t launches;
+    float total_ms;
+} gs_profile_stat;
+int gs_profile_begin(int32_t max_launches);
+int gs_profile_end(gs_profile_stat *out, int32_t max_stats);
+
+/* ABI version of this header. */
+int gs_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* GS_H_ */

@@ -1,0 +1,140 @@
+"""Helpers shared by the GPU parity tests (imported by tests only).
+
+The CUDA path is driven through the binding (the C-ABI of include/gs.h); the
+oracle supplies every expected value.  Stage-fed checks give the CUDA stage
+under test the oracle's own single-precision records, so that a comparison
+isolates one stage.
+
+Tolerances (stated by the rasterizer's specification):
+  images and final transmittance  |delta| <= 1e-4 absolute
+  gradients                       |delta| <= 1e-6, or <= 1e-3 |ref|; elements
+                                  that fail both are re-tested against 1e-3 x
+                                  the sum of the absolute values of the terms
+                                  the element sums (fp32 atomics reorder the
+                                  sums, so cancellation is excused, and
+                                  reported), and none may fail that.
+Decisions taken on floats within a stated relative margin of their threshold
+(alpha vs 1/255, T vs 1e-4, o G vs 0.99, a tile edge, the radius ceiling,
+depth order) may flip between fp32 and fp64; the pixels they touch are listed
+as ambiguous and excluded, and their number is bounded.
+"""
+from __future__ import annotations
+
+import numpy as np
+import torch
+
+import gaussian_splatting_differentiable_tile_b200 as G
+import oracle as O
+
+IMG_TOL = 1e-4
+GRAD_ABS, GRAD_REL = 1e-6, 1e-3
+MARGIN_IMG = 1e-3     # relative margin of an alpha / transmittance decision
+MARGIN_CLAMP = 1e-3   # relative margin of o G against the 0.99 cap
+MARGIN_TILE = 1e-4    # tiles, distance of (m -+ r)/16 to an integer
+MARGIN_RADIUS = 2e-4  # px, distance of 3 sqrt(lambda) to an integer
+
+
+def cuda_params(params: dict) -> dict:
+    return {k: torch.from_numpy(np.ascontiguousarray(v, dtype=np.float32)).cuda() for k, v in params.items()}
+
+
+def fill_projected(rec: dict, n: int) -> G.Projected:
+    """Device records in the public gs_projected layout, from oracle records."""
+    proj = G.Projected(n)
+    if n == 0:
+        return proj
+    xyod = np.zeros((n, 4), np.float32)
+    xyod[:, :2] = rec["mean2d"]
+    xyod[:, 2] = rec["opacity"]
+    xyod[:, 3] = rec["depth32"]
+    conr = np.zeros((n, 4), np.float32)
+    conr[:, :3] = rec["conic"]
+    conr[:, 3] = rec["radius"]
+    rgb = np.zeros((n, 4), np.float32)
+    rgb[:, :3] = rec["color"]
+    proj.xy_opacity_depth.copy_(torch.from_numpy(xyod))
+    proj.conic_radius.copy_(torch.from_numpy(conr))
+    proj.rgb.copy_(torch.from_numpy(rgb))
+    proj.rect.copy_(torch.from_numpy(np.ascontiguousarray(rec["rect"], np.int32)))
+    proj.count.copy_(torch.from_numpy(np.ascontiguousarray(rec["count"], np.int32)))
+    return proj
+
+
+def oracle_records(params: dict, cam) -> dict:
+    """Oracle projection rounded once to fp32 (the stage-fed input)."""
+    p = O.project(params, cam)
+    r = O.records_f32(p, cam.width, cam.height)
+    return r
+
+
+def gpu_bin(cam, n, proj, max_pairs=None):
+    bins = G.Bins(n, max_pairs if max_pairs is not None else max(64, 64 * max(n, 1)), cam.width, cam.height)
+    K = G.gs_bin_and_sort(cam, n, proj, bins, sync=True)
+    return bins, K
+
+
+def gpu_render(cam, n, proj, bins):
+    H, W = cam.height, cam.width
+    image = torch.full((H, W, 3), float("nan"), device="cuda")
+    T = torch.full((H, W), float("nan"), device="cuda")
+    last = torch.full((H, W), -1, dtype=torch.int32, device="cuda")
+    G.gs_render_fwd(cam, n, proj, bins, image, T, last)
+    torch.cuda.synchronize()
+    return image, T, last
+
+
+def ambiguous_pixels(orc_fwd: dict, with_clamp: bool = False) -> np.ndarray:
+    amb = orc_fwd["margin_img"] < MARGIN_IMG
+    if with_clamp:
+        amb |= orc_fwd["margin_clamp"] < MARGIN_CLAMP
+    return amb
+
+
+def ambiguous_gaussian_tiles(p: dict, cam) -> np.ndarray:
+    """Tiles whose list may differ between an fp32 and an fp64 projection:
+    those within one tile of a Gaussian whose radius ceiling or rectangle
+    edge sits within the stated margin of flipping, or whose depth is within
+    4 float ulps of another drawable Gaussian's."""
+    v = p["valid"].astype(bool)
+    bad = v & ((p["radius_margin"] < MARGIN_RADIUS) | (p["rect_margin"] < MARGIN_TILE))
+    d = p["depth"]
+    idx = np.nonzero(v & (p["count"] > 0))[0]
+    if idx.size > 1:
+        order = idx[np.argsort(d[idx], kind="stable")]
+        ds = d[order]
+        ulp = np.spacing(ds.astype(np.float32)).astype(np.float64)
+        close = np.diff(ds) <= 4 * ulp[1:]
+        bad[order[1:][close]] = True
+        bad[order[:-1][close]] = True
+    tiles = np.zeros((cam.tiles_y, cam.tiles_x), bool)
+    for g in np.nonzero(bad)[0]:
+        x0, y0, x1, y1 = p["rect"][g]
+        if x0 > x1 or y0 > y1:
+            # a flip could make an empty rectangle non-empty at the border
+            x0, y0, x1, y1 = 0, 0, -1, -1
+            m = p["mean2d"][g]
+            r = float(p["radius"][g])
+            x0 = int(np.floor((m[0] - r) / 16)) - 1
+            x1 = int(np.floor((m[0] + r) / 16)) + 1
+            y0 = int(np.floor((m[1] - r) / 16)) - 1
+            y1 = int(np.floor((m[1] + r) / 16)) + 1
+        tiles[max(y0 - 1, 0):min(y1 + 2, cam.tiles_y), max(x0 - 1, 0):min(x1 + 2, cam.tiles_x)] = True
+    return tiles
+
+
+def tiles_to_pixels(tiles: np.ndarray, cam) -> np.ndarray:
+    px = np.repeat(np.repeat(tiles, 16, axis=0), 16, axis=1)
+    return px[:cam.height, :cam.width]
+
+
+def grad_compare(gpu: np.ndarray, ref: np.ndarray, bound: np.ndarray, name: str):
+    """Returns (n_excused); raises AssertionError on an unexcused element."""
+    d = np.abs(gpu.astype(np.float64) - ref)
+    ok = (d <= GRAD_ABS) | (d <= GRAD_REL * np.abs(ref))
+    excused = ~ok & (d <= GRAD_REL * bound + GRAD_ABS)
+    bad = ~ok & ~excused
+    if bad.any():
+        i = np.argwhere(bad)[0]
+        raise AssertionError(f"{name}: {int(bad.sum())} gradient elements out of tolerance; first at "
+                             f"{tuple(i)}: gpu={gpu[tuple(i)]!r} ref={ref[tuple(i)]!r} bound={bound[tuple(i)]!r}")
+    return int(excused.sum())

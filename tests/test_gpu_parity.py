@@ -1,0 +1,371 @@
+"""Parity of the CUDA path (through the C ABI) with the CPU oracle.
+
+Integer stages (tile counts, the sorted pair list, tile ranges) must match bit
+for bit when fed the same records; images within 1e-4; gradients within
+1e-6 absolute or 1e-3 relative (cancellation excused against the sum of
+absolute terms).  Sizes span several tiles with ragged edges and run on the
+oracle in seconds.
+"""
+import numpy as np
+import pytest
+import torch
+
+import gaussian_splatting_differentiable_tile_b200 as G
+import oracle as O
+from scenes import Camera, make_cameras, make_scene, make_target, tiny_camera
+
+from gpu_common import (IMG_TOL, MARGIN_RADIUS, MARGIN_TILE, ambiguous_gaussian_tiles, ambiguous_pixels, cuda_params, fill_projected,
+                        gpu_bin, gpu_render, grad_compare, oracle_records, tiles_to_pixels)
+
+pytestmark = pytest.mark.gpu
+
+
+def _student_subset(n, seed=2):
+    cam = make_cameras("student", count=60)[7]
+    params = make_scene("student", n=n, seed=seed)
+    return cam, params
+
+
+def _ragged_cam():
+    # 200 x 150 px: 13 x 10 tiles, last column 8 px wide and last row 6 px tall
+    return tiny_camera(200, 150, 180.0, distance=3.0)
+
+
+SCENES = {
+    "tiny": lambda: (tiny_camera(), make_scene("tiny")),
+    "ragged": lambda: (_ragged_cam(), make_scene("tiny", n=1537, seed=9)),
+    "student3k": lambda: _student_subset(3000),
+}
+
+
+# ------------------------------------------------------------------ project
+@pytest.mark.parametrize("scene", list(SCENES))
+def test_project_matches_oracle(scene):
+    cam, params = SCENES[scene]()
+    n = params["means"].shape[0]
+    proj = G.Projected(n)
+    G.gs_project(cam, cuda_params(params), proj)
+    torch.cuda.synchronize()
+    p = O.project(params, cam)
+    xyod = proj.xy_opacity_depth.cpu().numpy().astype(np.float64)
+    conr = proj.conic_radius.cpu().numpy().astype(np.float64)
+    rgb = proj.rgb.cpu().numpy()
+    rect = proj.rect.cpu().numpy()
+    count = proj.count.cpu().numpy()
+    v = p["valid"].astype(bool)
+    np.testing.assert_array_equal(rgb[:, :3], params["colors"])
+    np.testing.assert_allclose(xyod[:, 3], p["depth"], rtol=1e-6, atol=1e-6)
+    np.testing.assert_allclose(xyod[:, 2], p["opacity"], rtol=1e-6, atol=1e-7)
+    np.testing.assert_allclose(xyod[v, :2], p["mean2d"][v], rtol=2e-6, atol=2e-3)
+    scale = np.maximum(np.abs(p["conic"][v, 0]), np.abs(p["conic"][v, 2]))[:, None]
+    np.testing.assert_array_less(np.abs(conr[v, :3] - p["conic"][v]), 1e-3 * scale + 1e-9)
+    # integer decisions: equal unless the oracle says the decision was within
+    # its stated margin of flipping
+    amb = v & ((p["radius_margin"] < MARGIN_RADIUS) | (p["rect_margin"] < MARGIN_TILE))
+    diff_r = conr[:, 3] != p["radius"]
+    diff_rect = np.any(rect != p["rect"], axis=1) | (count != p["count"])
+    assert not np.any(diff_r & ~amb), np.nonzero(diff_r & ~amb)[0][:10]
+    assert not np.any(diff_rect & ~amb), np.nonzero(diff_rect & ~amb)[0][:10]
+    assert amb.sum() <= max(2, 1e-3 * n)
+
+
+# ---------------------------------------------------- bin and sort (stage-fed)
+def _check_bins(cam, rec, n, bins, K):
+    ob = O.bin_pairs(rec["rect"], rec["valid"], rec["depth32"], cam.width, cam.height)
+    assert K == ob["n_pairs"]
+    tile = bins.pair_tile[:K].cpu().numpy().astype(np.uint32)
+    gid = bins.pair_gid[:K].cpu().numpy().astype(np.uint32)
+    np.testing.assert_array_equal(tile.astype(np.uint64), ob["keys"] >> np.uint64(32))
+    np.testing.assert_array_equal(gid, ob["gids"])
+    # the 64-bit keys of the emitted pairs: tile << 32 | depth bits
+    key = (tile.astype(np.uint64) << np.uint64(32)) | rec["depth32"].view(np.uint32)[gid].astype(np.uint64)
+    np.testing.assert_array_equal(key, ob["keys"])
+    np.testing.assert_array_equal(bins.ranges.cpu().numpy().astype(np.uint32)[:cam.tiles], ob["ranges"])
+    assert int(bins.status.item()) == 0
+
+
+@pytest.mark.parametrize("scene", list(SCENES))
+def test_bin_and_sort_bit_exact(scene):
+    cam, params = SCENES[scene]()
+    n = params["means"].shape[0]
+    rec = oracle_records(params, cam)
+    proj = fill_projected(rec, n)
+    bins, K = gpu_bin(cam, n, proj)
+    _check_bins(cam, rec, n, bins, K)
+
+
+def test_bin_and_sort_depth_ties_and_many_partitions():
+    """Equal depth keys keep Gaussian-id order; N spans several sort and scan
+    partitions with a ragged last one."""
+    cam, params = _student_subset(30_000)
+    n = 30_000
+    rec = oracle_records(params, cam)
+    rec["depth32"] = (np.round(rec["depth32"] * 4) / 4).astype(np.float32)
+    proj = fill_projected(rec, n)
+    bins, K = gpu_bin(cam, n, proj)
+    _check_bins(cam, rec, n, bins, K)
+
+
+@pytest.mark.parametrize("W,H", [(16, 16), (1, 1), (17, 1), (4112, 4112)])
+def test_bin_and_sort_tile_bit_widths(W, H):
+    """0 tile bits (one tile, no pair sort), 1 and 2 tiles, and 257 x 257
+    tiles (17 bits: three sort passes)."""
+    cam = Camera(np.eye(4), W * 0.5, W * 0.5, W / 2.0, H / 2.0, W, H)
+    rng = np.random.default_rng(W + H)
+    n = 700
+    params = {"means": np.column_stack([rng.uniform(-1, 1, n), rng.uniform(-1, 1, n), rng.uniform(2, 4, n)]),
+              "log_scales": rng.normal(-2.5, 0.7, (n, 3)), "quats": rng.normal(size=(n, 4)),
+              "opacity_logits": rng.normal(0, 1, n), "colors": rng.uniform(0, 1, (n, 3))}
+    rec = oracle_records(params, cam)
+    proj = fill_projected(rec, n)
+    bins, K = gpu_bin(cam, n, proj, max_pairs=int(rec["count"].sum()) + 16)
+    _check_bins(cam, rec, n, bins, K)
+
+
+def test_bin_and_sort_capacity_error_and_async_status():
+    cam, params = SCENES["tiny"]()
+    n = params["means"].shape[0]
+    rec = oracle_records(params, cam)
+    need = int(rec["count"].sum())
+    proj = fill_projected(rec, n)
+    bins = G.Bins(n, need - 1, cam.width, cam.height)
+    with pytest.raises(G.GSError) as ei:
+        G.gs_bin_and_sort(cam, n, proj, bins, sync=True)
+    assert ei.value.code == G.GS_ERR_CAPACITY and ei.value.n_pairs == need
+    # asynchronous mode: nothing raised, the status word says so, ranges are
+    # empty, and the render draws background only
+    G.gs_bin_and_sort(cam, n, proj, bins, sync=False)
+    st, K = G.gs_read_status(bins)
+    assert st == G.GS_ERR_CAPACITY and K == need
+    assert int(bins.ranges.abs().sum().item()) == 0
+    image, T, _ = gpu_render(cam, n, proj, bins)
+    assert torch.all(image == 0) and torch.all(T == 1)
+    # regrown to the reported need, the same call succeeds
+    bins2 = G.Bins(n, need, cam.width, cam.height)
+    assert G.gs_bin_and_sort(cam, n, proj, bins2) == need
+
+
+def test_argument_errors_launch_nothing():
+    cam = tiny_camera()
+    proj = G.Projected(10)
+    bins = G.Bins(10, 100, cam.width, cam.height)
+    bad = tiny_camera()
+    bad.near_z = 0.0
+    with pytest.raises(G.GSError) as ei:
+        G.gs_bin_and_sort(bad, 10, proj, bins)
+    assert ei.value.code == G.GS_ERR_INVALID_ARG
+    with pytest.raises(G.GSError) as ei:
+        G.gs_bin_and_sort(cam, 11, proj, bins)  # more Gaussians than carved for
+    assert ei.value.code == G.GS_ERR_INVALID_ARG
+    big = tiny_camera(512, 512)
+    with pytest.raises(G.GSError):
+        G.gs_render_fwd(big, 10, proj, bins, torch.empty(512, 512, 3, device="cuda"),
+                        torch.empty(512, 512, device="cuda"),
+                        torch.empty(512, 512, dtype=torch.int32, device="cuda"))
+
+
+# ------------------------------------------------------- forward (stage-fed)
+def _fwd_stage_fed(cam, params, tile_mask=None):
+    n = params["means"].shape[0]
+    rec = oracle_records(params, cam)
+    proj = fill_projected(rec, n)
+    bins, K = gpu_bin(cam, n, proj)
+    image, T, last = gpu_render(cam, n, proj, bins)
+    ref = O.render(rec, cam, tile_mask=tile_mask)
+    return rec, proj, bins, K, image.cpu().numpy(), T.cpu().numpy(), last.cpu().numpy(), ref
+
+
+def _assert_fwd(cam, bins, image, T, last, ref, sel):
+    amb = ambiguous_pixels(ref) & sel
+    ok = sel & ~amb
+    assert amb.sum() <= max(3, 2e-3 * sel.sum()), f"{amb.sum()} ambiguous pixels"
+    d_img = np.abs(image - ref["image"]).max(axis=2)
+    assert d_img[ok].max(initial=0) <= IMG_TOL, d_img[ok].max()
+    assert np.abs(T - ref["T_final"])[ok].max(initial=0) <= IMG_TOL
+    ranges = bins.ranges.cpu().numpy()
+    ty, tx = np.mgrid[0:cam.height, 0:cam.width]
+    start = ranges[(ty // 16) * cam.tiles_x + tx // 16, 0]
+    np.testing.assert_array_equal((last - start)[ok], ref["n_walk"][ok])
+    assert np.all(np.isfinite(image)) and np.all(T > 0) and np.all(T <= 1)
+
+
+@pytest.mark.parametrize("scene", list(SCENES))
+def test_render_fwd_matches_oracle(scene):
+    cam, params = SCENES[scene]()
+    rec, proj, bins, K, image, T, last, ref = _fwd_stage_fed(cam, params)
+    _assert_fwd(cam, bins, image, T, last, ref, np.ones((cam.height, cam.width), bool))
+
+
+def test_render_fwd_student_sampled_tiles():
+    """The 30k-Gaussian student at 980 x 545 on 120 sampled tiles."""
+    cam, params = _student_subset(30_000)
+    rng = np.random.default_rng(0)
+    mask = np.zeros(cam.tiles, np.uint8)
+    mask[rng.choice(cam.tiles, 120, replace=False)] = 1
+    mask[-1] = 1  # ragged corner tile
+    rec, proj, bins, K, image, T, last, ref = _fwd_stage_fed(cam, params, tile_mask=mask)
+    sel = tiles_to_pixels(mask.reshape(cam.tiles_y, cam.tiles_x).astype(bool), cam)
+    _assert_fwd(cam, bins, image, T, last, ref, sel)
+
+
+def test_render_fwd_background_and_white_invariant():
+    cam, params = SCENES["ragged"]()
+    cam.bg = (0.2, 0.4, 0.6)
+    params = dict(params)
+    params["colors"] = np.ones_like(params["colors"])
+    rec, proj, bins, K, image, T, last, ref = _fwd_stage_fed(cam, params)
+    _assert_fwd(cam, bins, image, T, last, ref, np.ones((cam.height, cam.width), bool))
+    # white splats: C = 1 - T, so image = (1 - T) + T bg
+    np.testing.assert_allclose(image, (1 - T)[..., None] + T[..., None] * np.array(cam.bg), atol=2e-6)
+
+
+# ------------------------------------------------------ backward (stage-fed)
+def _bwd_stage_fed(cam, params, seed=0, tile_mask=None):
+    n = params["means"].shape[0]
+    rec, proj, bins, K, image, T, last, ref = _fwd_stage_fed(cam, params, tile_mask=tile_mask)
+    rng = np.random.default_rng(seed)
+    dl = rng.normal(size=(cam.height, cam.width, 3))
+    keep = ~ambiguous_pixels(ref, with_clamp=True)
+    if tile_mask is not None:
+        keep &= tiles_to_pixels(tile_mask.reshape(cam.tiles_y, cam.tiles_x).astype(bool), cam)
+    dl = np.where(keep[..., None], dl, 0.0).astype(np.float32)
+    P = cuda_params(params)
+    grads = {k: torch.full_like(v, float("nan")) for k, v in P.items()}
+    grad2d = torch.full((n, 12), float("nan"), device="cuda")
+    G.gs_render_bwd(cam, n, P, proj, bins, torch.from_numpy(T).cuda(), torch.from_numpy(last).cuda(),
+                    torch.from_numpy(dl).cuda(), grad2d, grads)
+    torch.cuda.synchronize()
+    g2_ref, g2_abs = O.render_bwd(rec, cam, dl.astype(np.float64), tile_mask=tile_mask)
+    return rec, grad2d.cpu().numpy(), {k: v.cpu().numpy() for k, v in grads.items()}, g2_ref, g2_abs, params
+
+
+@pytest.mark.parametrize("scene", list(SCENES))
+def test_render_bwd_matches_oracle(scene):
+    cam, params = SCENES[scene]()
+    rec, g2, grads, g2_ref, g2_abs, params = _bwd_stage_fed(cam, params)
+    assert np.all(g2[:, 9:] == 0)
+    grad_compare(g2[:, :9], g2_ref, g2_abs, "grad2d")
+    raw_ref = O.project_bwd(params, cam, g2_ref)
+    bound = O.grad_bound(params, cam, g2_abs)
+    for k in G.PARAM_KEYS:
+        grad_compare(grads[k], raw_ref[k], bound[k], k)
+        assert np.all(np.isfinite(grads[k]))
+
+
+def test_render_bwd_student_sampled_tiles():
+    cam, params = _student_subset(30_000)
+    rng = np.random.default_rng(1)
+    mask = np.zeros(cam.tiles, np.uint8)
+    mask[rng.choice(cam.tiles, 80, replace=False)] = 1
+    rec, g2, grads, g2_ref, g2_abs, params = _bwd_stage_fed(cam, params, tile_mask=mask)
+    grad_compare(g2[:, :9], g2_ref, g2_abs, "grad2d")
+
+
+# ------------------------------------------------------------ end to end
+def test_end_to_end_from_raw_parameters():
+    """Raw parameters through all four calls vs the oracle from the same raw
+    parameters in double precision, L1 loss against a seeded target."""
+    cam, params = SCENES["ragged"]()
+    n = params["means"].shape[0]
+    P = cuda_params(params)
+    r = G.Rasterizer(n, cam.width, cam.height)
+    image = r.forward(cam, P).clone()
+    target = torch.from_numpy(make_target(cam.width, cam.height)).cuda()
+    dl = torch.empty_like(image)
+    loss = torch.zeros(1, device="cuda")
+    G.gs_l1_loss_grad(image, target, dl, loss)
+    torch.cuda.synchronize()
+    p = O.project(params, cam)
+    ref = O.render(p, cam)
+    sel = ~(ambiguous_pixels(ref, with_clamp=True) | tiles_to_pixels(ambiguous_gaussian_tiles(p, cam), cam))
+    assert sel.mean() > 0.9
+    img = image.cpu().numpy()
+    assert np.abs(img - ref["image"]).max(axis=2)[sel].max() <= IMG_TOL
+    tgt = target.cpu().numpy().astype(np.float64)
+    assert abs(loss.item() - np.abs(img - tgt).mean()) <= 1e-5
+    # gradient of L1 with ambiguous pixels masked out
+    dlm = torch.where(torch.from_numpy(sel[..., None]).cuda(), dl, torch.zeros_like(dl))
+    grads = r.backward(cam, P, dlm)
+    torch.cuda.synchronize()
+    g2_ref, g2_abs = O.render_bwd(p, cam, dlm.cpu().numpy().astype(np.float64))
+    raw_ref = O.project_bwd(params, cam, g2_ref)
+    bound = O.grad_bound(params, cam, g2_abs)
+    for k in G.PARAM_KEYS:
+        grad_compare(grads[k].cpu().numpy(), raw_ref[k], bound[k], k)
+
+
+# --------------------------------------------------------------- edge cases
+def test_empty_scene_renders_background():
+    cam = tiny_camera(40, 24, bg=(0.1, 0.2, 0.3))
+    r = G.Rasterizer(0, cam.width, cam.height)
+    P = {k: torch.zeros((0,) + s, device="cuda") for k, s in
+         (("means", (3,)), ("log_scales", (3,)), ("quats", (4,)), ("opacity_logits", ()), ("colors", (3,)))}
+    img = r.forward(cam, P)
+    torch.cuda.synchronize()
+    assert r.n_pairs == 0
+    np.testing.assert_array_equal(img.cpu().numpy(), np.broadcast_to(np.float32([0.1, 0.2, 0.3]), (24, 40, 3)))
+    grads = r.backward(cam, P, torch.ones_like(img))
+    assert all(v.numel() == 0 for v in grads.values())
+
+
+def test_culled_nan_and_zero_quaternion_inputs():
+    """Gaussians behind the camera, on the near plane, with a NaN parameter:
+    no tiles, exactly zero gradient, and the others are unaffected.  A zero
+    quaternion renders as the identity rotation."""
+    cam = tiny_camera(64, 48, 60.0)
+    rng = np.random.default_rng(4)
+    n = 40
+    params = {"means": np.column_stack([rng.uniform(-.5, .5, n), rng.uniform(-.5, .5, n), rng.uniform(-.5, .5, n)]),
+              "log_scales": rng.normal(-2.3, 0.3, (n, 3)), "quats": rng.normal(size=(n, 4)),
+              "opacity_logits": rng.normal(0, 1, n), "colors": rng.uniform(0, 1, (n, 3))}
+    params["means"][0, 2] = -4.0            # z_cam = 0: culled
+    params["means"][1, 2] = -10.0           # behind the camera
+    params["means"][2] = [0.3, 0.3, -3.995]  # in front of the near plane
+    params["log_scales"][3, 1] = np.nan     # NaN parameter
+    params["quats"][4] = 0.0                # zero quaternion
+    params = {k: v.astype(np.float32) for k, v in params.items()}
+    P = cuda_params(params)
+    r = G.Rasterizer(n, cam.width, cam.height)
+    r.forward(cam, P)
+    cnt = r.proj.count.cpu().numpy()
+    assert cnt[0] == 0 and cnt[1] == 0 and cnt[2] == 0 and cnt[3] == 0 and cnt[4] > 0
+    grads = r.backward(cam, P, torch.ones(cam.height, cam.width, 3, device="cuda"))
+    torch.cuda.synchronize()
+    for k, v in grads.items():
+        v = v.cpu().numpy()
+        assert np.all(np.isfinite(v)), k
+        assert np.all(v[:4] == 0), k
+    p = O.project(params, cam)
+    assert p["count"][:4].tolist() == [0, 0, 0, 0]
+    assert np.all(np.isfinite(r.image.cpu().numpy()))
+
+
+def test_huge_splat_covers_every_tile():
+    cam = _ragged_cam()
+    params = {"means": np.zeros((2, 3), np.float32), "log_scales": np.full((2, 3), 1.0, np.float32),
+              "quats": np.tile(np.float32([1, 0, 0, 0]), (2, 1)), "opacity_logits": np.float32([2.0, -1.0]),
+              "colors": np.float32([[1, 0, 0], [0, 1, 0]])}
+    rec = oracle_records(params, cam)
+    assert rec["count"][0] == cam.tiles
+    proj = fill_projected(rec, 2)
+    bins, K = gpu_bin(cam, 2, proj)
+    _check_bins(cam, rec, 2, bins, K)
+    image, T, last = gpu_render(cam, 2, proj, bins)
+    ref = O.render(rec, cam)
+    _assert_fwd(cam, bins, image.cpu().numpy(), T.cpu().numpy(), last.cpu().numpy(), ref,
+                np.ones((cam.height, cam.width), bool))
+
+
+def test_saturating_stack_terminates_early():
+    """Many opaque splats: every pixel stops at T < 1e-4 long before the end
+    of its list, as in the pages' termination example."""
+    cam = tiny_camera(48, 40, 60.0)
+    n = 300
+    rng = np.random.default_rng(8)
+    params = {"means": np.column_stack([rng.uniform(-.2, .2, n), rng.uniform(-.2, .2, n), rng.uniform(-.5, .5, n)]),
+              "log_scales": np.full((n, 3), -0.5), "quats": rng.normal(size=(n, 4)),
+              "opacity_logits": np.full(n, 3.0), "colors": rng.uniform(0, 1, (n, 3))}
+    params = {k: v.astype(np.float32) for k, v in params.items()}
+    rec, proj, bins, K, image, T, last, ref = _fwd_stage_fed(cam, params)
+    _assert_fwd(cam, bins, image, T, last, ref, np.ones((cam.height, cam.width), bool))
+    assert (ref["e_visit"] < n).mean() > 0.9 and (T < 1e-3).mean() > 0.9
