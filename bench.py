@@ -315,8 +315,8 @@ def run_native(args, spec, rank, world, local):
         host_loss.copy_(loss, non_blocking=True)
 
     e2e_ms, _ = timed(step_e2e, args.steps, args.warmup)
-    h2d = sum(v.numel() * 4 for v in params_np.values()) + H * W * 3 * 4
-    d2h = sum(v.numel() * 4 for v in params_np.values()) + 4
+    h2d = sum(v.size * 4 for v in params_np.values()) + H * W * 3 * 4
+    d2h = sum(v.size * 4 for v in params_np.values()) + 4
 
     t = torch.tensor([full_ms, fwd_ms, e2e_ms], dtype=torch.float64, device=dev)
     if world > 1:

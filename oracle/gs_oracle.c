@@ -494,7 +494,7 @@ typedef struct {
     double *image, *T_final;
     int32_t *n_walk;
     int64_t *e_visit, *e_contrib;
-    double *margin_img, *margin_clamp;
+    double *margin_alpha, *margin_T, *margin_clamp;
     /* backward */
     const double *dL_dimage;
     double *grad2d, *grad2d_abs; /* per-thread slices, [nthreads][n][9] */
@@ -513,7 +513,8 @@ static double rel_margin(double v, double thr) { return fabs(v - thr) / thr; }
  * buffer as needed).  Returns the number of added entries. */
 static int64_t walk_pixel(const orc_render_ctx *c, int32_t i, int32_t j, orc_hit **hits,
                           int64_t *cap, double rgb[3], double *T_out, int32_t *n_walk,
-                          int64_t *e_visit, int64_t *e_contrib, double *m_img, double *m_clamp)
+                          int64_t *e_visit, int64_t *e_contrib, double *m_alpha, double *m_T,
+                          double *m_clamp)
 {
     const double x = j + 0.5, y = i + 0.5;
     const int32_t tx = j / ORC_TILE, ty = i / ORC_TILE;
@@ -521,7 +522,7 @@ static int64_t walk_pixel(const orc_render_ctx *c, int32_t i, int32_t j, orc_hit
     rgb[0] = rgb[1] = rgb[2] = 0.0;
     int32_t pos = 0, last_pos = 0;
     int64_t visits = 0, nh = 0;
-    double mi = INFINITY, mc = INFINITY;
+    double ma_min = INFINITY, mt_min = INFINITY, mc = INFINITY;
     for (int64_t k = 0; k < c->n_order; k++) {
         int64_t g = c->order[k];
         const int32_t *r = c->rect + 4 * g;
@@ -538,13 +539,13 @@ static int64_t walk_pixel(const orc_render_ctx *c, int32_t i, int32_t j, orc_hit
         double alpha = clamped ? (double)ORC_ALPHA_CAP_F : oG;
         if (sigma < 0.0) continue;
         double ma = rel_margin(alpha, (double)ORC_ALPHA_MIN_F);
-        if (ma < mi) mi = ma;
+        if (ma < ma_min) ma_min = ma;
         if ((float)alpha < ORC_ALPHA_MIN_F) continue;
         double mcl = rel_margin(oG, (double)ORC_ALPHA_CAP_F);
         if (mcl < mc) mc = mcl;
         double next_T = T * (1.0 - alpha);
         double mt = rel_margin(next_T, (double)ORC_T_MIN_F);
-        if (mt < mi) mi = mt;
+        if (mt < mt_min) mt_min = mt;
         if ((float)next_T < ORC_T_MIN_F) break;
         for (int ch = 0; ch < 3; ch++) rgb[ch] += c->color[3 * g + ch] * alpha * T;
         if (hits) {
@@ -564,7 +565,8 @@ static int64_t walk_pixel(const orc_render_ctx *c, int32_t i, int32_t j, orc_hit
     *n_walk = last_pos;
     *e_visit = visits;
     *e_contrib = nh;
-    *m_img = mi;
+    *m_alpha = ma_min;
+    *m_T = mt_min;
     *m_clamp = mc;
     return nh;
 }
@@ -586,7 +588,7 @@ static void *render_worker(void *arg)
             int64_t p = (int64_t)i * cam->width + j;
             double rgb[3], T;
             walk_pixel(c, i, j, NULL, NULL, rgb, &T, &c->n_walk[p], &c->e_visit[p],
-                       &c->e_contrib[p], &c->margin_img[p], &c->margin_clamp[p]);
+                       &c->e_contrib[p], &c->margin_alpha[p], &c->margin_T[p], &c->margin_clamp[p]);
             for (int ch = 0; ch < 3; ch++) c->image[3 * p + ch] = rgb[ch] + T * cam->bg[ch];
             c->T_final[p] = T;
         }
@@ -615,14 +617,15 @@ static int run_threads(orc_render_ctx *c, void *(*fn)(void *))
  * the selected tiles; other pixels are left untouched.
  * Outputs per pixel: image[3], T_final, n_walk (position in the pixel's tile
  * list one past the last added entry), e_visit (entries visited, up to and
- * including the stopping one), e_contrib (entries added), margin_img (least
- * relative distance of an alpha or transmittance test to its threshold),
- * margin_clamp (least relative distance of o G to the 0.99 cap). */
+ * including the stopping one), e_contrib (entries added), margin_alpha (least
+ * relative distance of an alpha to 1/255), margin_T (least relative distance
+ * of a next_T to 1e-4), margin_clamp (least relative distance of o G to the
+ * 0.99 cap). */
 int orc_render(int64_t n, const double *mean2d, const double *conic, const double *opacity,
                const double *color, const float *depth32, const int32_t *rect,
                const uint8_t *valid, const orc_camera *cam, const uint8_t *tile_mask, int nthreads,
                double *image, double *T_final, int32_t *n_walk, int64_t *e_visit,
-               int64_t *e_contrib, double *margin_img, double *margin_clamp)
+               int64_t *e_contrib, double *margin_alpha, double *margin_T, double *margin_clamp)
 {
     if (n < 0 || cam->width <= 0 || cam->height <= 0) return -1;
     int64_t *order = (int64_t *)malloc(sizeof(int64_t) * (size_t)(n > 0 ? n : 1));
@@ -635,7 +638,8 @@ int orc_render(int64_t n, const double *mean2d, const double *conic, const doubl
     c.cam = cam; c.tile_mask = tile_mask;
     c.tiles_x = (cam->width + ORC_TILE - 1) / ORC_TILE;
     c.image = image; c.T_final = T_final; c.n_walk = n_walk; c.e_visit = e_visit;
-    c.e_contrib = e_contrib; c.margin_img = margin_img; c.margin_clamp = margin_clamp;
+    c.e_contrib = e_contrib; c.margin_alpha = margin_alpha; c.margin_T = margin_T;
+    c.margin_clamp = margin_clamp;
     c.n = n;
     c.nthreads = nthreads;
     int rc = run_threads(&c, render_worker);
@@ -667,10 +671,10 @@ static void *backward_worker(void *arg)
         for (int32_t j = 0; j < cam->width; j++) {
             if (!pixel_selected(c, i, j)) continue;
             int64_t p = (int64_t)i * cam->width + j;
-            double rgb[3], T, mi, mc;
+            double rgb[3], T, ma, mt, mc;
             int32_t nw;
             int64_t ev, ec;
-            int64_t nh = walk_pixel(c, i, j, &hits, &cap, rgb, &T, &nw, &ev, &ec, &mi, &mc);
+            int64_t nh = walk_pixel(c, i, j, &hits, &cap, rgb, &T, &nw, &ev, &ec, &ma, &mt, &mc);
             const double *gp = c->dL_dimage + 3 * p;
             double R[3] = {cam->bg[0], cam->bg[1], cam->bg[2]};
             for (int64_t h = nh - 1; h >= 0; h--) {

@@ -74,7 +74,7 @@ def lib() -> ctypes.CDLL:
         L.orc_render.argtypes = [ctypes.c_int64, _c_double_p, _c_double_p, _c_double_p, _c_double_p,
                                  _c_float_p, _c_int32_p, _c_uint8_p, ctypes.POINTER(OrcCamera),
                                  _c_uint8_p, ctypes.c_int, _c_double_p, _c_double_p, _c_int32_p,
-                                 _c_int64_p, _c_int64_p, _c_double_p, _c_double_p]
+                                 _c_int64_p, _c_int64_p, _c_double_p, _c_double_p, _c_double_p]
         L.orc_render_bwd.argtypes = [ctypes.c_int64, _c_double_p, _c_double_p, _c_double_p,
                                      _c_double_p, _c_float_p, _c_int32_p, _c_uint8_p,
                                      ctypes.POINTER(OrcCamera), _c_uint8_p, ctypes.c_int, _c_double_p,
@@ -264,7 +264,8 @@ def render(proj: dict, cam, tile_mask=None, nthreads: int | None = None) -> dict
     out = {"image": np.zeros((H, W, 3)), "T_final": np.zeros((H, W)),
            "n_walk": np.zeros((H, W), dtype=np.int32), "e_visit": np.zeros((H, W), dtype=np.int64),
            "e_contrib": np.zeros((H, W), dtype=np.int64),
-           "margin_img": np.full((H, W), np.inf), "margin_clamp": np.full((H, W), np.inf)}
+           "margin_alpha": np.full((H, W), np.inf), "margin_T": np.full((H, W), np.inf),
+           "margin_clamp": np.full((H, W), np.inf)}
     c = _cam(cam)
     mk, mkp = _mask(cam, tile_mask)
     rc = lib().orc_render(
@@ -273,8 +274,8 @@ def render(proj: dict, cam, tile_mask=None, nthreads: int | None = None) -> dict
         _ptr(valid, _c_uint8_p), ctypes.byref(c), mkp, int(nthreads or default_threads()),
         _ptr(out["image"], _c_double_p), _ptr(out["T_final"], _c_double_p),
         _ptr(out["n_walk"], _c_int32_p), _ptr(out["e_visit"], _c_int64_p),
-        _ptr(out["e_contrib"], _c_int64_p), _ptr(out["margin_img"], _c_double_p),
-        _ptr(out["margin_clamp"], _c_double_p))
+        _ptr(out["e_contrib"], _c_int64_p), _ptr(out["margin_alpha"], _c_double_p),
+        _ptr(out["margin_T"], _c_double_p), _ptr(out["margin_clamp"], _c_double_p))
     if rc != 0:
         raise ValueError("orc_render failed")
     return out

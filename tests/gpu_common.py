@@ -28,8 +28,9 @@ import oracle as O
 
 IMG_TOL = 1e-4
 GRAD_ABS, GRAD_REL = 1e-6, 1e-3
-MARGIN_IMG = 1e-3     # relative margin of an alpha / transmittance decision
-MARGIN_CLAMP = 1e-3   # relative margin of o G against the 0.99 cap
+MARGIN_ALPHA = 5e-5   # relative margin of alpha against 1/255
+MARGIN_T = 1e-3       # relative margin of T (1 - alpha) against 1e-4
+MARGIN_CLAMP = 1e-4   # relative margin of o G against the 0.99 cap
 MARGIN_TILE = 1e-4    # tiles, distance of (m -+ r)/16 to an integer
 MARGIN_RADIUS = 2e-4  # px, distance of 3 sqrt(lambda) to an integer
 
@@ -68,7 +69,9 @@ def oracle_records(params: dict, cam) -> dict:
 
 
 def gpu_bin(cam, n, proj, max_pairs=None):
-    bins = G.Bins(n, max_pairs if max_pairs is not None else max(64, 64 * max(n, 1)), cam.width, cam.height)
+    if max_pairs is None:
+        max_pairs = 64 * n + cam.tiles + 4096
+    bins = G.Bins(n, max_pairs, cam.width, cam.height)
     K = G.gs_bin_and_sort(cam, n, proj, bins, sync=True)
     return bins, K
 
@@ -84,17 +87,17 @@ def gpu_render(cam, n, proj, bins):
 
 
 def ambiguous_pixels(orc_fwd: dict, with_clamp: bool = False) -> np.ndarray:
-    amb = orc_fwd["margin_img"] < MARGIN_IMG
+    amb = (orc_fwd["margin_alpha"] < MARGIN_ALPHA) | (orc_fwd["margin_T"] < MARGIN_T)
     if with_clamp:
         amb |= orc_fwd["margin_clamp"] < MARGIN_CLAMP
     return amb
 
 
-def ambiguous_gaussian_tiles(p: dict, cam) -> np.ndarray:
-    """Tiles whose list may differ between an fp32 and an fp64 projection:
-    those within one tile of a Gaussian whose radius ceiling or rectangle
-    edge sits within the stated margin of flipping, or whose depth is within
-    4 float ulps of another drawable Gaussian's."""
+def ambiguous_gaussians(p: dict) -> np.ndarray:
+    """Gaussians whose binning may differ between an fp32 and an fp64
+    projection: radius ceiling or a rectangle edge within the stated margin
+    of an integer, or a depth within 4 float ulps of another drawable
+    Gaussian's (their order may swap)."""
     v = p["valid"].astype(bool)
     bad = v & ((p["radius_margin"] < MARGIN_RADIUS) | (p["rect_margin"] < MARGIN_TILE))
     d = p["depth"]
@@ -105,21 +108,7 @@ def ambiguous_gaussian_tiles(p: dict, cam) -> np.ndarray:
         ulp = np.spacing(ds.astype(np.float32)).astype(np.float64)
         close = np.diff(ds) <= 4 * ulp[1:]
         bad[order[1:][close]] = True
-        bad[order[:-1][close]] = True
-    tiles = np.zeros((cam.tiles_y, cam.tiles_x), bool)
-    for g in np.nonzero(bad)[0]:
-        x0, y0, x1, y1 = p["rect"][g]
-        if x0 > x1 or y0 > y1:
-            # a flip could make an empty rectangle non-empty at the border
-            x0, y0, x1, y1 = 0, 0, -1, -1
-            m = p["mean2d"][g]
-            r = float(p["radius"][g])
-            x0 = int(np.floor((m[0] - r) / 16)) - 1
-            x1 = int(np.floor((m[0] + r) / 16)) + 1
-            y0 = int(np.floor((m[1] - r) / 16)) - 1
-            y1 = int(np.floor((m[1] + r) / 16)) + 1
-        tiles[max(y0 - 1, 0):min(y1 + 2, cam.tiles_y), max(x0 - 1, 0):min(x1 + 2, cam.tiles_x)] = True
-    return tiles
+    return bad
 
 
 def tiles_to_pixels(tiles: np.ndarray, cam) -> np.ndarray:

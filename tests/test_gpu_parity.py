@@ -14,8 +14,9 @@ import gaussian_splatting_differentiable_tile_b200 as G
 import oracle as O
 from scenes import Camera, make_cameras, make_scene, make_target, tiny_camera
 
-from gpu_common import (IMG_TOL, MARGIN_RADIUS, MARGIN_TILE, ambiguous_gaussian_tiles, ambiguous_pixels, cuda_params, fill_projected,
-                        gpu_bin, gpu_render, grad_compare, oracle_records, tiles_to_pixels)
+from gpu_common import (IMG_TOL, MARGIN_RADIUS, MARGIN_TILE, ambiguous_gaussians, ambiguous_pixels,
+                        cuda_params, fill_projected, gpu_bin, gpu_render, grad_compare, oracle_records,
+                        tiles_to_pixels)
 
 pytestmark = pytest.mark.gpu
 
@@ -58,7 +59,7 @@ def test_project_matches_oracle(scene):
     np.testing.assert_allclose(xyod[:, 2], p["opacity"], rtol=1e-6, atol=1e-7)
     np.testing.assert_allclose(xyod[v, :2], p["mean2d"][v], rtol=2e-6, atol=2e-3)
     scale = np.maximum(np.abs(p["conic"][v, 0]), np.abs(p["conic"][v, 2]))[:, None]
-    np.testing.assert_array_less(np.abs(conr[v, :3] - p["conic"][v]), 1e-3 * scale + 1e-9)
+    assert np.all(np.abs(conr[v, :3] - p["conic"][v]) <= 1e-4 * scale + 1e-9)
     # integer decisions: equal unless the oracle says the decision was within
     # its stated margin of flipping
     amb = v & ((p["radius_margin"] < MARGIN_RADIUS) | (p["rect_margin"] < MARGIN_TILE))
@@ -176,16 +177,20 @@ def _fwd_stage_fed(cam, params, tile_mask=None):
 
 
 def _assert_fwd(cam, bins, image, T, last, ref, sel):
+    """Every selected pixel matches (image and T within 1e-4, the same last
+    entry) unless one of its threshold decisions sat within the stated margin
+    of flipping; such actual flips must be rare."""
     amb = ambiguous_pixels(ref) & sel
-    ok = sel & ~amb
-    assert amb.sum() <= max(3, 2e-3 * sel.sum()), f"{amb.sum()} ambiguous pixels"
     d_img = np.abs(image - ref["image"]).max(axis=2)
-    assert d_img[ok].max(initial=0) <= IMG_TOL, d_img[ok].max()
-    assert np.abs(T - ref["T_final"])[ok].max(initial=0) <= IMG_TOL
+    d_T = np.abs(T - ref["T_final"])
     ranges = bins.ranges.cpu().numpy()
     ty, tx = np.mgrid[0:cam.height, 0:cam.width]
     start = ranges[(ty // 16) * cam.tiles_x + tx // 16, 0]
-    np.testing.assert_array_equal((last - start)[ok], ref["n_walk"][ok])
+    differs = sel & ((d_img > IMG_TOL) | (d_T > IMG_TOL) | ((last - start) != ref["n_walk"]))
+    unexplained = differs & ~amb
+    assert not unexplained.any(), (f"{int(unexplained.sum())} pixels differ away from any threshold; max "
+                                   f"|d image| {d_img[unexplained].max():.3e}")
+    assert differs.sum() <= max(2, 1e-4 * sel.sum()), f"{int(differs.sum())} flipped pixels"
     assert np.all(np.isfinite(image)) and np.all(T > 0) and np.all(T <= 1)
 
 
@@ -262,10 +267,24 @@ def test_render_bwd_student_sampled_tiles():
 
 
 # ------------------------------------------------------------ end to end
+def _without_ambiguous(params, cam):
+    """The scene with every Gaussian whose projection sits within the stated
+    margin of an integer decision (radius ceiling, tile edge, depth order)
+    moved behind the camera, so that fp32 and fp64 bin it the same way."""
+    p = O.project(params, cam)
+    bad = ambiguous_gaussians(p)
+    out = {k: v.copy() for k, v in params.items()}
+    out["means"][bad] = np.linalg.inv(cam.viewmat.astype(np.float64))[:3, :3] @ [0.0, 0.0, -50.0] + \
+        np.linalg.inv(cam.viewmat.astype(np.float64))[:3, 3]
+    return out, int(bad.sum())
+
+
 def test_end_to_end_from_raw_parameters():
     """Raw parameters through all four calls vs the oracle from the same raw
     parameters in double precision, L1 loss against a seeded target."""
     cam, params = SCENES["ragged"]()
+    params, removed = _without_ambiguous(params, cam)
+    assert removed <= 20
     n = params["means"].shape[0]
     P = cuda_params(params)
     r = G.Rasterizer(n, cam.width, cam.height)
@@ -276,9 +295,10 @@ def test_end_to_end_from_raw_parameters():
     G.gs_l1_loss_grad(image, target, dl, loss)
     torch.cuda.synchronize()
     p = O.project(params, cam)
+    assert not ambiguous_gaussians(p).any()
     ref = O.render(p, cam)
-    sel = ~(ambiguous_pixels(ref, with_clamp=True) | tiles_to_pixels(ambiguous_gaussian_tiles(p, cam), cam))
-    assert sel.mean() > 0.9
+    sel = ~ambiguous_pixels(ref, with_clamp=True)
+    assert sel.mean() > 0.99
     img = image.cpu().numpy()
     assert np.abs(img - ref["image"]).max(axis=2)[sel].max() <= IMG_TOL
     tgt = target.cpu().numpy().astype(np.float64)
@@ -368,4 +388,4 @@ def test_saturating_stack_terminates_early():
     params = {k: v.astype(np.float32) for k, v in params.items()}
     rec, proj, bins, K, image, T, last, ref = _fwd_stage_fed(cam, params)
     _assert_fwd(cam, bins, image, T, last, ref, np.ones((cam.height, cam.width), bool))
-    assert (ref["e_visit"] < n).mean() > 0.9 and (T < 1e-3).mean() > 0.9
+    assert (ref["e_visit"] < n).mean() > 0.75 and (T < 1e-3).mean() > 0.75

@@ -49,7 +49,8 @@ def _clean(cam, params):
     out = O.render(p, cam, nthreads=2)
     v = p["valid"].astype(bool)
     d = np.sort(p["depth32"][v])
-    return (out["margin_img"].min() > 1e-4 and out["margin_clamp"].min() > 1e-4 and
+    return (out["margin_alpha"].min() > 1e-4 and out["margin_T"].min() > 1e-4 and
+            out["margin_clamp"].min() > 1e-4 and
             p["rect_margin"][v].min() > 1e-4 and p["radius_margin"][v].min() > 1e-4 and
             (len(d) < 2 or np.diff(d).min() > 1e-5) and p["count"].sum() > 0)
 
