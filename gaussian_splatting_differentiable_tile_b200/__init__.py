@@ -28,7 +28,8 @@ from ._abi import (GS_ERR_ALIGNMENT, GS_ERR_CAPACITY, GS_ERR_CUDA, GS_ERR_DEVICE
                    GS_ERR_INVALID_ARG, GS_ERR_TOO_LARGE, GS_OK, GS_TILE)
 
 __all__ = [
-    "GSError", "Projected", "Bins", "make_camera", "gs_project", "gs_bin_and_sort", "gs_render_fwd",
+    "GSError", "Projected", "Bins", "make_camera", "gs_project", "gs_bin_and_sort",
+    "gs_bin_and_sort_static", "gs_render_fwd",
     "gs_render_bwd", "gs_render_stats", "gs_l1_loss_grad", "gs_read_status", "gs_error_string", "profile_begin",
     "profile_end", "lib", "PARAM_KEYS",
 ]
@@ -167,6 +168,26 @@ def gs_bin_and_sort(cam, n: int, proj: Projected, bins: Bins, sync: bool = True,
         err.n_pairs = int(k.value)
         raise err
     return int(k.value) if sync else None
+
+
+def gs_bin_and_sort_static(cam, n: int, proj: Projected, pair_tile: torch.Tensor, pair_gid: torch.Tensor,
+                           ranges: torch.Tensor, stream=None) -> int:
+    """gs_bin_and_sort without a caller scratch buffer (the library's fixed
+    array holds it; see include/gs.h).  Writes the sorted pairs and ranges into
+    the given int32 CUDA tensors and returns K; raises GSError on any error
+    (with .n_pairs set for GS_ERR_CAPACITY)."""
+    c = make_camera(cam)
+    k = ctypes.c_int64(0)
+    rc = lib().gs_bin_and_sort_static(ctypes.byref(c), int(n), ctypes.byref(proj.struct),
+                                      _dev(pair_tile, "pair_tile", torch.int32),
+                                      _dev(pair_gid, "pair_gid", torch.int32),
+                                      _dev(ranges, "ranges", torch.int32), int(pair_tile.numel()),
+                                      ctypes.byref(k), _stream(stream))
+    if rc < 0:
+        err = GSError(rc, "gs_bin_and_sort_static")
+        err.n_pairs = int(k.value)
+        raise err
+    return int(k.value)
 
 
 def gs_render_fwd(cam, n: int, proj: Projected, bins: Bins, image: torch.Tensor, T_final: torch.Tensor,

@@ -75,6 +75,10 @@ PROTOTYPES = {
     "gs_bin_and_sort": (ctypes.c_int, [ctypes.POINTER(GsCamera), ctypes.c_int64, ctypes.POINTER(GsProjected),
                                        ctypes.POINTER(GsBins), ctypes.POINTER(ctypes.c_int64),
                                        ctypes.c_void_p]),
+    "gs_bin_and_sort_static": (ctypes.c_int, [ctypes.POINTER(GsCamera), ctypes.c_int64,
+                                              ctypes.POINTER(GsProjected), ctypes.c_void_p, ctypes.c_void_p,
+                                              ctypes.c_void_p, ctypes.c_int64, ctypes.POINTER(ctypes.c_int64),
+                                              ctypes.c_void_p]),
     "gs_render_fwd": (ctypes.c_int, [ctypes.POINTER(GsCamera), ctypes.c_int64, ctypes.POINTER(GsProjected),
                                      ctypes.POINTER(GsBins), ctypes.c_void_p, ctypes.c_void_p,
                                      ctypes.c_void_p, ctypes.c_void_p]),

@@ -3,6 +3,7 @@
 #include <cmath>
 #include <cstdio>
 #include <cstring>
+#include <mutex>
 #include <vector>
 
 #include "gs_internal.cuh"
@@ -349,3 +350,80 @@ int gs_profile_end(gs_profile_stat *out, int32_t max_stats) {
 }
 
 }  // extern "C"
+
+// ------------------------------------------------------------------------
+// gs_bin_and_sort_static: the binning scratch of gs_bin_and_sort held in one
+// fixed-size device array of this library, for callers that cannot allocate.
+namespace {
+
+constexpr int64_t kStaticMaxN = int64_t(1) << 18;       // Gaussians
+constexpr int64_t kStaticMaxPairs = int64_t(1) << 20;   // pairs
+constexpr int32_t kStaticMaxTiles = 65536;              // tiles
+constexpr BinsLayout kStaticLayout = bins_layout(kStaticMaxN, kStaticMaxPairs, kStaticMaxTiles);
+// Everything the layout holds before its own result arrays: the variant
+// writes its results straight into the caller's arrays.
+constexpr size_t kStaticBytes = kStaticLayout.pair_tile;
+
+static __device__ __align__(256) unsigned char g_static_scratch[kStaticBytes];
+
+// Host-side device address of g_static_scratch, per device.  The array's name
+// in host code is only a stand-in for the symbol, never an address a kernel
+// may be given.
+constexpr int kMaxDevices = 128;
+void *g_static_ptr[kMaxDevices] = {};
+std::mutex g_static_mutex;
+
+int static_scratch(void **out) {
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return GS_ERR_CUDA;
+    std::lock_guard<std::mutex> lock(g_static_mutex);
+    if (!g_static_ptr[dev]) {
+        void *p = nullptr;
+        if (cudaGetSymbolAddress(&p, g_static_scratch) != cudaSuccess || !p) return GS_ERR_CUDA;
+        g_static_ptr[dev] = p;
+    }
+    *out = g_static_ptr[dev];
+    return GS_OK;
+}
+
+}  // namespace
+
+extern "C" int gs_bin_and_sort_static(const gs_camera *cam, int64_t n, const gs_projected *proj,
+                                      uint32_t *pair_tile, uint32_t *pair_gid, uint32_t *ranges,
+                                      int64_t max_pairs, int64_t *n_pairs_host, void *stream) {
+    CamConst c;
+    int rc = make_cam(cam, &c);
+    if (rc) return rc;
+    if (n < 0 || max_pairs < 0 || !n_pairs_host || !pair_tile || !pair_gid || !ranges)
+        return GS_ERR_INVALID_ARG;
+    const int64_t tiles = (int64_t)c.tiles_x * c.tiles_y;
+    if (n > kStaticMaxN || max_pairs > kStaticMaxPairs || tiles > kStaticMaxTiles)
+        return GS_ERR_TOO_LARGE;
+    if ((rc = check_projected(proj, n))) return rc;
+    if (!aligned(pair_tile, 4) || !aligned(pair_gid, 4) || !aligned(ranges, 8)) return GS_ERR_ALIGNMENT;
+    void *base = nullptr;
+    if ((rc = static_scratch(&base))) return rc;
+    char *b = static_cast<char *>(base);
+    gs_bins bins;
+    std::memset(&bins, 0, sizeof(bins));
+    bins.pair_tile = pair_tile;
+    bins.pair_gid = pair_gid;
+    bins.ranges = reinterpret_cast<uint32_t *>(b + kStaticLayout.ranges);
+    bins.n_pairs = reinterpret_cast<uint64_t *>(b + kStaticLayout.n_pairs);
+    bins.status = reinterpret_cast<int32_t *>(b + kStaticLayout.status);
+    bins.max_pairs = max_pairs;
+    bins.max_n = kStaticMaxN;
+    bins.max_tiles = kStaticMaxTiles;
+    bins.scratch = base;
+    bins.scratch_bytes = kStaticBytes;
+    cudaStream_t s = as_stream(stream);
+    // The launcher clears the status, count, ticket, histogram, range and
+    // look-back words at its start, so nothing of the previous call leaks in.
+    if (launch_bin_and_sort(c, n, *proj, bins, kStaticLayout, s) != cudaSuccess) return GS_ERR_CUDA;
+    if (cudaMemcpyAsync(ranges, bins.ranges, (size_t)tiles * 2 * sizeof(uint32_t),
+                        cudaMemcpyDeviceToDevice, s) != cudaSuccess)
+        return GS_ERR_CUDA;
+    rc = gs_read_status(&bins, n_pairs_host, stream);
+    if (rc == GS_OK && *n_pairs_host > max_pairs) rc = GS_ERR_CAPACITY;
+    return rc;
+}

@@ -66,9 +66,9 @@ struct BinsLayout {
     int64_t depth_parts, scan_parts, tile_parts;
 };
 
-inline size_t align_up(size_t v, size_t a) { return (v + a - 1) / a * a; }
+constexpr size_t align_up(size_t v, size_t a) { return (v + a - 1) / a * a; }
 
-inline BinsLayout bins_layout(int64_t max_n, int64_t max_pairs, int32_t max_tiles) {
+constexpr BinsLayout bins_layout(int64_t max_n, int64_t max_pairs, int32_t max_tiles) {
     BinsLayout L{};
     size_t off = 0;
     L.status = off;       off += 8;

@@ -224,6 +224,42 @@ int gs_render_stats(const gs_camera *cam, int64_t n, const gs_projected *proj,
 int gs_l1_loss_grad(const float *image, const float *target, int64_t count, float *dL_dimage,
                     float *loss, void *stream);
 
+/* gs_bin_and_sort for callers that cannot allocate device memory.
+ *
+ * There is no counterpart in the source pages: this is a deployment variant.
+ * gs_bin_and_sort needs a caller-allocated scratch buffer (gs_bins) for its
+ * depth sort, scan look-back and pair sort.  Some callers cannot allocate it:
+ * a real-time viewer's frame loop that must never call cudaMalloc/cudaFree
+ * (both can synchronize the whole device and stall a frame), or a plug-in
+ * whose host application owns all device memory and hands it no allocator.
+ * This call keeps that scratch in one fixed-size array inside libgs.so
+ * instead, so the caller passes only its inputs and outputs.
+ *
+ * Limits (GS_ERR_TOO_LARGE beyond them, nothing launched): n <= 262,144
+ * Gaussians, max_pairs <= 1,048,576 pairs, at most 65,536 tiles.  The array
+ * (about 21 MB) is part of the library's device image: every GPU on which
+ * the library is used holds it until the process exits.
+ *
+ * Inputs: cam, n, proj as for gs_bin_and_sort.  Outputs (device, caller-owned):
+ *   pair_tile [max_pairs], pair_gid [max_pairs]  the sorted pair list, the same
+ *                                                values gs_bin_and_sort writes
+ *   ranges    [tiles][2]                         each tile's [start, end)
+ *   *n_pairs_host (HOST, required)               K, the total pair count
+ * The call synchronizes `stream` to read K and the kernels' status back, and
+ * returns GS_ERR_CAPACITY when K > max_pairs (only the first max_pairs pairs
+ * are then defined, ranges are empty) or GS_ERR_DEVICE_TIMEOUT, as
+ * gs_bin_and_sort does.  It calls no allocating routine.
+ *
+ * The first call on each device looks up the array's device address
+ * (cudaGetSymbolAddress) with that device current; make that first call
+ * before any stream capture.  Every call, on every stream, shares the one
+ * array per device and clears the parts that must start at zero itself;
+ * calls whose work overlaps on the GPU (two streams, or two host threads)
+ * race on it and must be serialized by the caller. */
+int gs_bin_and_sort_static(const gs_camera *cam, int64_t n, const gs_projected *proj,
+                           uint32_t *pair_tile, uint32_t *pair_gid, uint32_t *ranges,
+                           int64_t max_pairs, int64_t *n_pairs_host, void *stream);
+
 /* Synchronizes `stream`, then returns bins->status and stores K in
  * *n_pairs_host (HOST, nullable).  GS_ERR_CUDA if the copy fails. */
 int gs_read_status(const gs_bins *bins, int64_t *n_pairs_host, void *stream);
