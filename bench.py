@@ -66,7 +66,8 @@ OPS_BWD_ADD = 32
 #   project      56 B/G raw parameters read + 68 B/G records written
 #   depth_keys   8 B/G read (depth, count) + 4 B/G written
 #   depth_sort   16 B/G per pass (key + value read and written)
-#   scan_emit    24 B/G read (sorted id, count, rectangle) + 8 B/P written
+#   scan         20 B/G read (sorted id, rectangle) + 12 B/G records written
+#   emit         16 B/G records read + 8 B/P written
 #   tile_sort    16 B/P per pass
 #   ranges       4 B/P read
 #   project_bwd  56 B/G raw parameters + 48 B/G 2D gradients read,
@@ -75,7 +76,8 @@ BYTES = {
     "project": lambda G, P: 124 * G,
     "depth_keys": lambda G, P: 12 * G,
     "depth_sort": lambda G, P: 16 * G,
-    "scan_emit": lambda G, P: 24 * G + 8 * P,
+    "scan": lambda G, P: 32 * G,
+    "emit": lambda G, P: 16 * G + 8 * P,
     "tile_sort": lambda G, P: 16 * P,
     "ranges": lambda G, P: 4 * P,
     "project_bwd": lambda G, P: 160 * G,

@@ -26,6 +26,10 @@ constexpr int kScanThreads = 256;
 constexpr int kScanItems = 8;
 constexpr int kScanPart = kScanThreads * kScanItems;  // 2048 Gaussians
 
+// Pair emit: 256 threads per block, 2048 pairs per block.
+constexpr int kEmitThreads = 256;
+constexpr int kEmitPairs = 2048;
+
 // Bounded device-side waits: a decoupled look-back poll gives up after this
 // many polls, records GS_ERR_DEVICE_TIMEOUT and lets the kernel finish.
 constexpr uint32_t kSpinLimit = 1u << 21;

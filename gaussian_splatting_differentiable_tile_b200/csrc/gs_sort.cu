@@ -55,6 +55,72 @@ __device__ __forceinline__ uint32_t block_exclusive_scan_256(uint32_t v, uint32_
     return wpre + x - v;
 }
 
+// Decoupled look-back for one digit: the sum of the digit's counts over
+// partitions [0, q0], read from the partitions' published words back to the
+// nearest inclusive one.  Eight words are requested at a time so a chain of
+// aggregates costs one L2 round trip per eight partitions.  A word that stays
+// unpublished for kSpinLimit polls records GS_ERR_DEVICE_TIMEOUT and counts
+// as zero, so the kernel always finishes.
+__device__ __forceinline__ uint32_t lookback_digit(const uint32_t *lookback, int d, int64_t q0,
+                                                   int32_t *status) {
+    constexpr int kWindow = 8;
+    uint32_t excl = 0;
+    uint32_t spins = 0;
+    for (int64_t q = q0; q >= 0; q -= kWindow) {
+        uint32_t w[kWindow];
+#pragma unroll
+        for (int k = 0; k < kWindow; k++)
+            w[k] = (q - k >= 0) ? ld_relaxed(lookback + (size_t)(q - k) * kRadix + d) : kFlagInclusive;
+#pragma unroll
+        for (int k = 0; k < kWindow; k++) {
+            while ((w[k] & ~kValueMask) == 0u) {
+                if (++spins > kSpinLimit) {
+                    set_status(status, GS_ERR_DEVICE_TIMEOUT);
+                    return excl;
+                }
+                w[k] = ld_relaxed(lookback + (size_t)(q - k) * kRadix + d);
+            }
+            excl += w[k] & kValueMask;
+            if ((w[k] & ~kValueMask) == kFlagInclusive) return excl;
+        }
+    }
+    return excl;
+}
+
+// Decoupled look-back over 64-bit partition words, by one full warp: lane l
+// reads partition q0 - l, so each L2 round trip covers 32 partitions.
+// Returns the inclusive prefix of partitions [0, q0] (to every lane).
+__device__ __forceinline__ uint64_t lookback_warp64(const uint64_t *lookback, int64_t q0,
+                                                    int32_t *status) {
+    const int lane = threadIdx.x & 31;
+    uint64_t prefix = 0;
+    uint32_t spins = 0;
+    for (int64_t base = q0; base >= 0; base -= 32) {
+        const int64_t q = base - lane;
+        uint64_t w = q >= 0 ? ld_relaxed64(lookback + q) : kFlag64Inclusive;
+        bool timed_out = false;
+        while (__any_sync(0xffffffffu, (w & ~kValue64Mask) == 0ull)) {
+            if (++spins > kSpinLimit) {
+                timed_out = true;
+                break;
+            }
+            if ((w & ~kValue64Mask) == 0ull) w = ld_relaxed64(lookback + q);
+        }
+        if (timed_out) {
+            if (lane == 0) set_status(status, GS_ERR_DEVICE_TIMEOUT);
+            if ((w & ~kValue64Mask) == 0ull) w = kFlag64Inclusive;
+        }
+        const uint32_t incl = __ballot_sync(0xffffffffu, (w & ~kValue64Mask) == kFlag64Inclusive);
+        const int first = incl ? __ffs(incl) - 1 : 31;
+        uint64_t v = lane <= first ? (w & kValue64Mask) : 0ull;
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+        prefix += v;
+        if (incl) break;
+    }
+    return prefix;
+}
+
 // Depth keys of the drawable Gaussians and the four digit histograms of the
 // depth sort.
 __global__ void __launch_bounds__(256)
@@ -178,22 +244,7 @@ k_onesweep(const uint32_t *__restrict__ keys_in, const uint32_t *__restrict__ va
                     st_relaxed(lb, kFlagInclusive | block_count);
                 } else {
                     st_relaxed(lb, kFlagAggregate | block_count);
-                    int64_t q = (int64_t)p - 1;
-                    uint32_t spins = 0;
-                    while (q >= 0) {
-                        const uint32_t w = ld_relaxed(lookback + (size_t)q * kRadix + d);
-                        const uint32_t flag = w & ~kValueMask;
-                        if (flag == 0u) {
-                            if (++spins > kSpinLimit) {
-                                set_status(status, GS_ERR_DEVICE_TIMEOUT);
-                                break;
-                            }
-                            continue;
-                        }
-                        excl += w & kValueMask;
-                        if (flag == kFlagInclusive) break;
-                        --q;
-                    }
+                    excl = lookback_digit(lookback, d, (int64_t)p - 1, status);
                     st_relaxed(lb, kFlagInclusive | ((excl + block_count) & kValueMask));
                 }
             }
@@ -232,120 +283,190 @@ k_onesweep(const uint32_t *__restrict__ keys_in, const uint32_t *__restrict__ va
     }
 }
 
-// Fused exclusive scan of the tile counts (in depth order) and pair emit.
+// Exclusive block-wide scan of one 64-bit value per thread (blockDim = 256).
+__device__ __forceinline__ uint64_t block_exclusive_scan64_256(uint64_t v, uint64_t *s_warp,
+                                                               uint64_t *total) {
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    uint64_t x = v;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+        const uint64_t y = __shfl_up_sync(0xffffffffu, x, o);
+        if (lane >= o) x += y;
+    }
+    if (lane == 31) s_warp[warp] = x;
+    __syncthreads();
+    uint64_t wpre = 0, tot = 0;
+#pragma unroll
+    for (int w = 0; w < 8; w++) {
+        const uint64_t t = s_warp[w];
+        if (w < warp) wpre += t;
+        tot += t;
+    }
+    __syncthreads();
+    *total = tot;
+    return wpre + x - v;
+}
+
+// Scan of the tile counts in depth order ("count" of the tile rasterizer).
 // One block per 2048 Gaussians of the depth order; the block's offset comes
-// from a decoupled look-back over 64-bit inclusive prefixes.  Each pair is
-// (tile, Gaussian id), written at its scanned offset; a Gaussian's tiles are
-// emitted row by row.  The digit histograms of the tile sort are gathered on
-// the way.  Pairs past max_pairs are not written: the block records
-// GS_ERR_CAPACITY, and n_pairs still receives the full count.
+// from a decoupled look-back over 64-bit inclusive prefixes.  For each depth
+// position i it writes the inclusive pair offset incl[i], the Gaussian's
+// packed first tile (x0 | y0 << 16) and its rectangle width, next to the
+// Gaussian id the depth sort left in sorted_gid: the emit reads these four
+// contiguous arrays.  The last block stores K; K > max_pairs records
+// GS_ERR_CAPACITY.
 __global__ void __launch_bounds__(kScanThreads)
-k_scan_emit(int n, const uint32_t *__restrict__ sorted_gid, const int4 *__restrict__ rect,
-            int tiles_x, int tiles_y, uint32_t *__restrict__ ptile,
-            uint32_t *__restrict__ pgid, uint64_t max_pairs, uint64_t *__restrict__ lookback,
-            uint32_t *__restrict__ ticket, uint64_t *__restrict__ n_pairs,
-            int32_t *__restrict__ status, uint32_t *__restrict__ tile_hist, int tile_passes,
-            int tile_bpp) {
-    __shared__ uint32_t s_incl[kScanPart];
-    __shared__ uint32_t s_gid[kScanPart];
-    __shared__ uint2 s_rect[kScanPart];
-    __shared__ uint32_t s_hist[kMaxTilePasses * kRadix];
-    __shared__ uint32_t s_scan[8];
+k_scan(int n, const uint32_t *__restrict__ sorted_gid, const int4 *__restrict__ rect, int tiles_x,
+       int tiles_y, uint32_t *__restrict__ incl, uint32_t *__restrict__ rpack,
+       uint32_t *__restrict__ width, uint64_t max_pairs, uint64_t *__restrict__ lookback,
+       uint32_t *__restrict__ ticket, uint64_t *__restrict__ n_pairs, int32_t *__restrict__ status) {
+    __shared__ uint64_t s_scan[8];
     __shared__ uint32_t s_part;
     __shared__ unsigned long long s_prefix;
-
     const int tid = threadIdx.x;
-    for (int i = tid; i < kMaxTilePasses * kRadix; i += kScanThreads) s_hist[i] = 0;
     if (tid == 0) s_part = atomicAdd(ticket, 1u);
     __syncthreads();
     const uint32_t p = s_part;
     const int64_t base = (int64_t)p * kScanPart;
 
-    uint32_t c[kScanItems], gid[kScanItems];
-    uint2 rc[kScanItems];
-    uint32_t tsum = 0;
+    uint32_t c[kScanItems];
+    uint64_t tsum = 0;
 #pragma unroll
     for (int i = 0; i < kScanItems; i++) {
         const int64_t idx = base + tid * kScanItems + i;
-        gid[i] = 0;
         c[i] = 0;
-        rc[i] = make_uint2(0u, 0u);
         if (idx < n) {
-            gid[i] = sorted_gid[idx];
             int x0, y0, w;
-            c[i] = rect_tiles(rect[gid[i]], tiles_x, tiles_y, x0, y0, w);
-            rc[i] = make_uint2((uint32_t)x0 | ((uint32_t)y0 << 16), (uint32_t)w);
+            c[i] = rect_tiles(rect[sorted_gid[idx]], tiles_x, tiles_y, x0, y0, w);
+            rpack[idx] = (uint32_t)x0 | ((uint32_t)y0 << 16);
+            width[idx] = (uint32_t)w;
         }
         tsum += c[i];
     }
-    uint32_t block_total;
-    const uint32_t toff = block_exclusive_scan_256(tsum, s_scan, &block_total);
-    uint32_t run = toff;
+    uint64_t block_total;
+    const uint64_t toff = block_exclusive_scan64_256(tsum, s_scan, &block_total);
+    if (tid < 32) {  // warp 0 publishes and looks back
+        uint64_t *lb = lookback + p;
+        uint64_t prefix = 0;
+        if (p == 0) {
+            if (tid == 0) st_relaxed64(lb, kFlag64Inclusive | (block_total & kValue64Mask));
+        } else {
+            if (tid == 0) st_relaxed64(lb, kFlag64Aggregate | (block_total & kValue64Mask));
+            prefix = lookback_warp64(lookback, (int64_t)p - 1, status);
+            if (tid == 0) st_relaxed64(lb, kFlag64Inclusive | ((prefix + block_total) & kValue64Mask));
+        }
+        if (tid == 0) {
+            s_prefix = prefix;
+            if (base + kScanPart >= n) {
+                const uint64_t K = prefix + block_total;
+                *n_pairs = K;
+                if (K > max_pairs) set_status(status, GS_ERR_CAPACITY);
+            }
+        }
+    }
+    __syncthreads();
+    uint64_t run = s_prefix + toff;
 #pragma unroll
     for (int i = 0; i < kScanItems; i++) {
-        const int k = tid * kScanItems + i;
+        const int64_t idx = base + tid * kScanItems + i;
         run += c[i];
-        s_incl[k] = run;
-        s_gid[k] = gid[i];
-        s_rect[k] = rc[i];
+        if (idx < n) incl[idx] = (uint32_t)run;  // meaningful while K <= max_pairs < 2^30
     }
-    if (tid == 0) {
-        uint64_t prefix = 0;
-        uint64_t *lb = lookback + p;
-        if (p == 0) {
-            st_relaxed64(lb, kFlag64Inclusive | (uint64_t)block_total);
+}
+
+// First index i in [lo, hi] with a[i] > t, for a non-decreasing array with
+// a[hi] > t, by one full warp: each round probes 32 evenly spaced entries,
+// so a search over N entries costs about log32(N) L2 round trips.
+__device__ __forceinline__ uint32_t warp_upper_bound(const uint32_t *a, uint32_t lo, uint32_t hi,
+                                                     uint32_t t) {
+    const int lane = threadIdx.x & 31;
+    while (hi - lo + 1 > 32) {
+        const uint32_t stride = (hi - lo + 32) / 32;
+        const uint32_t x = min(lo + lane * stride, hi);
+        const uint32_t m = __ballot_sync(0xffffffffu, a[x] > t);
+        if (m == 0) {
+            lo = min(lo + 31 * stride, hi) + 1;
         } else {
-            st_relaxed64(lb, kFlag64Aggregate | (uint64_t)block_total);
-            int64_t q = (int64_t)p - 1;
-            uint32_t spins = 0;
-            while (q >= 0) {
-                const uint64_t w = ld_relaxed64(lookback + q);
-                const uint64_t flag = w & ~kValue64Mask;
-                if (flag == 0ull) {
-                    if (++spins > kSpinLimit) {
-                        set_status(status, GS_ERR_DEVICE_TIMEOUT);
-                        break;
-                    }
-                    continue;
-                }
-                prefix += w & kValue64Mask;
-                if (flag == kFlag64Inclusive) break;
-                --q;
-            }
-            st_relaxed64(lb, kFlag64Inclusive | ((prefix + block_total) & kValue64Mask));
+            const int f = __ffs(m) - 1;
+            const uint32_t xf = min(lo + f * stride, hi);
+            lo = f == 0 ? lo : min(lo + (f - 1) * stride, hi) + 1;
+            hi = xf;
         }
-        s_prefix = prefix;
-        if (base + kScanPart >= n) *n_pairs = prefix + block_total;
     }
-    __syncthreads();
-    const uint64_t prefix = s_prefix;
+    const uint32_t x = min(lo + lane, hi);
+    const uint32_t m = __ballot_sync(0xffffffffu, a[x] > t);
+    return lo + (__ffs(m) - 1);
+}
+
+// Pair emit ("emit" of the tile rasterizer), balanced by pairs: block b writes
+// pairs [2048 b, 2048 b + 2048).  Warps 0 and 1 find the depth positions of
+// the Gaussians holding its first and last pair; the block stages that span
+// (at most 2048 Gaussians, since every drawable Gaussian has at least one
+// pair and the undrawable ones sort last) in shared memory, and each thread
+// finds its pair's Gaussian there by binary search.  A Gaussian's tiles are
+// emitted row by row; the digit histograms of the tile sort are gathered on
+// the way.  Nothing is emitted after a recorded error.
+__global__ void __launch_bounds__(kEmitThreads)
+k_emit(int n, const uint32_t *__restrict__ incl, const uint32_t *__restrict__ sorted_gid,
+       const uint32_t *__restrict__ rpack, const uint32_t *__restrict__ width, int tiles_x,
+       const uint64_t *__restrict__ n_pairs, const int32_t *__restrict__ status,
+       uint32_t *__restrict__ ptile, uint32_t *__restrict__ pgid, uint32_t *__restrict__ tile_hist,
+       int tile_passes, int tile_bpp) {
+    __shared__ uint32_t s_incl[kEmitPairs];
+    __shared__ uint32_t s_gid[kEmitPairs];
+    __shared__ uint32_t s_rp[kEmitPairs];
+    __shared__ uint32_t s_w[kEmitPairs];
+    __shared__ uint32_t s_hist[kMaxTilePasses * kRadix];
+    __shared__ uint32_t s_span[3];  // g0, g1, pairs before g0
+    if (*(volatile const int32_t *)status != 0 || n == 0) return;
+    const uint64_t K = *n_pairs;
+    const int tid = threadIdx.x, warp = tid >> 5;
+    for (int i = tid; i < kMaxTilePasses * kRadix; i += kEmitThreads) s_hist[i] = 0;
     const uint32_t dmask = (1u << tile_bpp) - 1u;
-    bool overflow = false;
-    for (uint32_t j = tid; j < block_total; j += kScanThreads) {
-        // item k: the first whose inclusive prefix exceeds j
-        int lo = 0, hi = kScanPart - 1;
-        while (lo < hi) {
-            const int mid = (lo + hi) >> 1;
-            if (s_incl[mid] > j) hi = mid; else lo = mid + 1;
+    for (uint64_t b = blockIdx.x; b * kEmitPairs < K; b += gridDim.x) {
+        const uint32_t p0 = (uint32_t)(b * kEmitPairs);
+        const uint64_t pe = (uint64_t)p0 + kEmitPairs;
+        const uint32_t p1 = (uint32_t)(K < pe ? K : pe);  // exclusive
+        __syncthreads();
+        if (warp == 0) {
+            const uint32_t g0 = warp_upper_bound(incl, 0, (uint32_t)n - 1, p0);
+            if (tid == 0) {
+                s_span[0] = g0;
+                s_span[2] = g0 == 0 ? 0u : incl[g0 - 1];
+            }
+        } else if (warp == 1) {
+            const uint32_t g1 = warp_upper_bound(incl, 0, (uint32_t)n - 1, p1 - 1);
+            if ((tid & 31) == 0) s_span[1] = g1;
         }
-        const uint32_t li = j - (lo == 0 ? 0u : s_incl[lo - 1]);
-        const uint2 r = s_rect[lo];
-        const uint32_t w = r.y;
-        const uint32_t row = li / w;
-        const uint32_t tile = ((r.x >> 16) + row) * (uint32_t)tiles_x + (r.x & 0xFFFFu) + (li - row * w);
-        const uint64_t pos = prefix + j;
-        if (pos < max_pairs) {
-            ptile[pos] = tile;
-            pgid[pos] = s_gid[lo];
+        __syncthreads();
+        const uint32_t g0 = s_span[0], g1 = s_span[1], before = s_span[2];
+        const uint32_t span = g1 - g0 + 1;
+        for (uint32_t k = tid; k < span && k < (uint32_t)kEmitPairs; k += kEmitThreads) {
+            s_incl[k] = incl[g0 + k];
+            s_gid[k] = sorted_gid[g0 + k];
+            s_rp[k] = rpack[g0 + k];
+            s_w[k] = width[g0 + k];
+        }
+        __syncthreads();
+        const int last = (int)min(span, (uint32_t)kEmitPairs) - 1;
+        for (uint32_t j = p0 + tid; j < p1; j += kEmitThreads) {
+            int lo = 0, hi = last;
+            while (lo < hi) {
+                const int mid = (lo + hi) >> 1;
+                if (s_incl[mid] > j) hi = mid; else lo = mid + 1;
+            }
+            const uint32_t li = j - (lo == 0 ? before : s_incl[lo - 1]);
+            const uint32_t w = s_w[lo], rp = s_rp[lo];
+            const uint32_t row = li / w;
+            const uint32_t tile = ((rp >> 16) + row) * (uint32_t)tiles_x + (rp & 0xFFFFu) + (li - row * w);
+            ptile[j] = tile;
+            pgid[j] = s_gid[lo];
             for (int k = 0; k < tile_passes; k++)
                 atomicAdd(&s_hist[k * kRadix + ((tile >> (k * tile_bpp)) & dmask)], 1u);
-        } else {
-            overflow = true;
         }
     }
-    if (overflow) set_status(status, GS_ERR_CAPACITY);
     __syncthreads();
-    for (int i = tid; i < tile_passes * kRadix; i += kScanThreads)
+    for (int i = tid; i < tile_passes * kRadix; i += kEmitThreads)
         if (s_hist[i]) atomicAdd(&tile_hist[i], s_hist[i]);
 }
 
@@ -421,7 +542,10 @@ cudaError_t launch_bin_and_sort(const CamConst &c, int64_t n, const gs_projected
             prof_after(s);
         }
     }
-    // 3. scan + emit, in depth order
+    // 3. scan of the counts in depth order, then the pair emit.  The scan's
+    //    per-Gaussian records reuse the depth sort's spare buffers: keys_b
+    //    (inclusive offsets), vals_b (packed first tile), keys_a (widths);
+    //    the sorted ids stay in vals_a.
     int tile_bits = 0;
     while ((1 << tile_bits) < tiles) tile_bits++;
     const int tile_passes = (tile_bits + kRadixBits - 1) / kRadixBits;
@@ -430,12 +554,22 @@ cudaError_t launch_bin_and_sort(const CamConst &c, int64_t n, const gs_projected
     uint32_t *to = bins.pair_tile, *go = bins.pair_gid;
     {
         const int blocks = (int)((n + kScanPart - 1) / kScanPart);
+        prof_before("scan", s);
+        k_scan<<<blocks, kScanThreads, 0, s>>>((int)n, U32(L.vals_a), reinterpret_cast<const int4 *>(proj.rect),
+                                              c.tiles_x, c.tiles_y, U32(L.keys_b), U32(L.vals_b),
+                                              U32(L.keys_a), (uint64_t)bins.max_pairs,
+                                              reinterpret_cast<uint64_t *>(base + L.scan_lb), tickets + 4,
+                                              n_pairs, status);
+        prof_after(s);
+    }
+    {
+        const int64_t chunks = (bins.max_pairs + kEmitPairs - 1) / kEmitPairs;
+        const int blocks = (int)std::max<int64_t>(1, std::min<int64_t>(chunks, (int64_t)sms * 4));
         uint32_t *et = tile_passes == 0 ? to : ta, *eg = tile_passes == 0 ? go : ga;
-        prof_before("scan_emit", s);
-        k_scan_emit<<<blocks, kScanThreads, 0, s>>>(
-            (int)n, U32(L.vals_a), reinterpret_cast<const int4 *>(proj.rect), c.tiles_x, c.tiles_y,
-            et, eg, (uint64_t)bins.max_pairs, reinterpret_cast<uint64_t *>(base + L.scan_lb),
-            tickets + 4, n_pairs, status, tile_hist, tile_passes, tile_bpp);
+        prof_before("emit", s);
+        k_emit<<<blocks, kEmitThreads, 0, s>>>((int)n, U32(L.keys_b), U32(L.vals_a), U32(L.vals_b),
+                                               U32(L.keys_a), c.tiles_x, n_pairs, status, et, eg, tile_hist,
+                                               tile_passes, tile_bpp);
         prof_after(s);
     }
     // 4. stable pair sort on the tile bits

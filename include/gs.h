@@ -246,8 +246,8 @@ int gs_l1_loss_grad(const float *image, const float *target, int64_t count, floa
  *   ranges    [tiles][2]                         each tile's [start, end)
  *   *n_pairs_host (HOST, required)               K, the total pair count
  * The call synchronizes `stream` to read K and the kernels' status back, and
- * returns GS_ERR_CAPACITY when K > max_pairs (only the first max_pairs pairs
- * are then defined, ranges are empty) or GS_ERR_DEVICE_TIMEOUT, as
+ * returns GS_ERR_CAPACITY when K > max_pairs (the pair arrays are then left
+ * undefined and the ranges empty) or GS_ERR_DEVICE_TIMEOUT, as
  * gs_bin_and_sort does.  It calls no allocating routine.
  *
  * The first call on each device looks up the array's device address
