@@ -2,6 +2,8 @@
 
     python -m gaussian_splatting_differentiable_tile_b200.build [--force] [--verbose]
 
+GS_EXTRA_NVCC_FLAGS in the environment adds compiler flags (tuning builds).
+
 Each translation unit under csrc/ is compiled to an object in _build/ (in
 parallel), then linked into libgs.so beside this file.  --verbose passes
 -Xptxas -v so the register, spill and shared-memory figures of every kernel
@@ -50,11 +52,14 @@ def up_to_date() -> bool:
 
 
 def build(force: bool = False, verbose: bool = False) -> str:
-    if not force and not verbose and up_to_date():
+    if not force and not verbose and not os.environ.get("GS_EXTRA_NVCC_FLAGS") and up_to_date():
         return LIB
     nvcc = _nvcc()
     os.makedirs(BUILD, exist_ok=True)
     extra = ["-Xptxas", "-v"] if verbose else []
+    # extra compiler flags, e.g. GS_EXTRA_NVCC_FLAGS="-DGS_ROWS_PER_LANE=2" for
+    # a variant of the blend's pixels-per-lane layout
+    extra += os.environ.get("GS_EXTRA_NVCC_FLAGS", "").split()
 
     def compile_one(src):
         obj = os.path.join(BUILD, os.path.basename(src) + ".o")

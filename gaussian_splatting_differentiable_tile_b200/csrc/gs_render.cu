@@ -1,34 +1,67 @@
 // gs_render.cu -- per-tile alpha blending (forward) and its back-to-front
-// gradient (backward), plus the L1 photometric loss of a training step.
+// gradient (backward), the frame's work counts, and the L1 loss of a training
+// step.
 //
 // Source: "Gaussian splatting in PyTorch" s5 (the per-pixel loop:
 // sigma = 1/2 (A dx^2 + C dy^2) + B dx dy, alpha = min(0.99, o exp(-sigma)),
 // skip sigma < 0 or alpha < 1/255, stop once T (1 - alpha) < 1e-4,
 // C += c alpha T; pixel centres at +0.5; background weighted by the final T),
-// s6 (the CUDA backward recovers T_i by dividing by 1 - alpha_j back to front;
+// s6 (the CUDA backward recovers T_i by dividing by 1 - alpha back to front;
 // no gradient through the 0.99 cap) and s8 (16 x 16 tiles, each pixel walks
 // only its tile's list); the course blog index (a backward that recomputes
 // the blend weights rather than storing them).
 //
-// One CTA per tile, one thread per pixel.  The tile's list is staged through
-// shared memory in batches of 256 entries, each entry converted once per tile
-// to the form the inner loop wants: the conic pre-scaled by -log2(e)/2 (and
-// -log2(e) for B) and log2(opacity), so that
-//     log2(o exp(-sigma)) = log2 o + cA dx^2 + cB dx dy + cC dy^2
-// costs five FP32 instructions and one MUFU ex2.  The forward and backward
-// share that evaluation code and use explicitly rounded intrinsics, so the
-// backward re-takes every skip decision bit-identically.
+// Work layout.  One CTA per tile.  Each lane owns RPL vertically adjacent
+// pixels of one column: lanes 0-15 the upper RPL rows of the warp's strip,
+// lanes 16-31 the lower RPL rows, so a warp covers a 16 x 2RPL strip and a
+// tile takes 8 / RPL warps.  The tile's list is staged through shared memory
+// in batches of 256 entries, each entry converted once per tile to
+//     geo  = (mx, my, cA, cB),  geo2 = (cC, log2 o, kx, ky)
+// with cA = -log2(e) A / 2, cB = -log2(e) B, cC = -log2(e) C / 2, so that
+//     log2(o exp(-sigma)) = log2 o + cA dx^2 + cB dx dy + cC dy^2.
+// The terms that depend only on the column (dx) are computed once per entry
+// and shared by the lane's RPL pixels.
+//
+// Exact culling per warp.  kx = cA - cB^2 / (4 cC) and ky = cC - cB^2 / (4 cA)
+// are the quadratic form's minima along a row and a column: over a strip of
+// pixel centres no closer than dy_min (rows) and dx_min (columns) to the mean,
+// -sigma log2(e) <= min(kx dx_min^2, ky dy_min^2).  When that bound keeps
+// alpha below 1/255 with a 1 % margin at every pixel of the warp, the entry is
+// skipped for the warp; each of its pixels would have skipped it anyway, so
+// the result is unchanged.
+//
+// The forward and backward share the evaluation code and use explicitly
+// rounded intrinsics, so the backward re-takes every skip decision
+// bit-identically.
 #include "gs_internal.cuh"
+
+// Pixels per lane and per-warp culling of the two blend kernels (tuning
+// knobs; the defaults are the fastest measured on B200).
+#ifndef GS_FWD_RPL
+#define GS_FWD_RPL 1
+#endif
+#ifndef GS_FWD_CULL
+#define GS_FWD_CULL 0
+#endif
+#ifndef GS_BWD_RPL
+#define GS_BWD_RPL 2
+#endif
+#ifndef GS_BWD_CULL
+#define GS_BWD_CULL 1
+#endif
 
 namespace gs {
 namespace {
 
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr float kAlphaCap = 0.99f;
-constexpr float kAlphaMin = 1.f / 255.f;
 constexpr float kTMin = 1e-4f;
-constexpr int kBlendThreads = kTilePixels;  // 256
-constexpr int kBatch = kBlendThreads;
+// log2(1/255) minus a margin of 0.0145 (1 % in alpha).
+constexpr float kCullLog2 = -7.994353436858858f - 0.0145f;
+// log2(1/255) in single precision: the alpha >= 1/255 test is taken on the
+// exponent, log2(o exp(-sigma)) >= this, before the exponential.
+constexpr float kLog2AlphaMin = -7.994353436858858f;
+constexpr int kBatch = 256;
 
 // PTX ex2.approx / rcp.approx (MUFU instructions).
 __device__ __forceinline__ float ex2_approx(float x) {
@@ -42,90 +75,220 @@ __device__ __forceinline__ float rcp_approx(float x) {
     return y;
 }
 
-// Per-tile staged form of one list entry.
-struct __align__(16) Staged {
-    float4 geo;   // mean2d x, y; cA = -log2e A / 2; cB = -log2e B
-    float2 geo2;  // cC = -log2e C / 2; log2(opacity)
+__device__ __forceinline__ void stage_entry(const float4 xyod, const float4 conr, float4 &geo,
+                                            float4 &geo2) {
+    const float cA = (-0.5f * kLog2e) * conr.x;
+    const float cB = -kLog2e * conr.y;
+    const float cC = (-0.5f * kLog2e) * conr.z;
+    const float kx = cA - cB * cB / (4.f * cC);
+    const float ky = cC - cB * cB / (4.f * cA);
+    geo = make_float4(xyod.x, xyod.y, cA, cB);
+    geo2 = make_float4(cC, log2f(xyod.z), kx, ky);
+}
+
+// Geometry of a lane: its column centre, its first row's centre, and the
+// centre and half extents of its warp's strip.
+struct LaneGeom {
+    float fx, fy0;
+    float sx, sy, hx, hy;
+    int px, py0;
 };
 
-__device__ __forceinline__ void stage_entry(const float4 xyod, const float4 conr, float4 &geo,
-                                            float2 &geo2) {
-    geo = make_float4(xyod.x, xyod.y, (-0.5f * kLog2e) * conr.x, -kLog2e * conr.y);
-    geo2 = make_float2((-0.5f * kLog2e) * conr.z, log2f(xyod.z));
+template <int kRPL>
+__device__ __forceinline__ LaneGeom lane_geom(const CamConst &cam, int tile) {
+    const int tx = tile % cam.tiles_x, ty = tile / cam.tiles_x;
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    LaneGeom L;
+    L.px = tx * kTile + (lane & 15);
+    L.py0 = ty * kTile + warp * 2 * kRPL + (lane >> 4) * kRPL;
+    L.fx = (float)L.px + 0.5f;
+    L.fy0 = (float)L.py0 + 0.5f;
+    L.sx = (float)(tx * kTile) + 8.f;
+    L.hx = 7.5f;
+    L.sy = (float)(ty * kTile + warp * 2 * kRPL + kRPL);
+    L.hy = (float)kRPL - 0.5f;
+    return L;
 }
 
-// Alpha of one entry at pixel centre (px, py).  Returns false when the entry
-// is skipped (sigma < 0 or alpha < 1/255).  dx, dy = mean - pixel.
-__device__ __forceinline__ bool eval_alpha(const float4 geo, const float2 geo2, float px, float py,
-                                           float &dx, float &dy, float &alpha, bool &capped) {
-    dx = __fsub_rn(geo.x, px);
-    dy = __fsub_rn(geo.y, py);
-    const float t = __fmaf_rn(geo.z, dx, __fmul_rn(geo.w, dy));          // cA dx + cB dy
-    const float q = __fmaf_rn(t, dx, __fmul_rn(__fmul_rn(geo2.x, dy), dy));  // -sigma log2 e
-    const float a = ex2_approx(__fadd_rn(q, geo2.y));                    // o exp(-sigma)
+// True when the entry cannot reach alpha >= 1/255 anywhere in the warp's strip.
+__device__ __forceinline__ bool culled(const float4 geo, const float4 geo2, const LaneGeom &L) {
+    const float dxm = fmaxf(fabsf(geo.x - L.sx) - L.hx, 0.f);
+    const float dym = fmaxf(fabsf(geo.y - L.sy) - L.hy, 0.f);
+    const float qb = fminf(geo2.z * dxm * dxm, geo2.w * dym * dym);
+    return geo2.y + qb < kCullLog2;
+}
+
+// Per-entry, per-lane terms shared by the lane's rows.
+struct ColTerms {
+    float dx, bdx, a0;  // mean - pixel x; cB dx; cA dx^2
+};
+__device__ __forceinline__ ColTerms col_terms(const float4 geo, float fx) {
+    ColTerms t;
+    t.dx = __fsub_rn(geo.x, fx);
+    t.bdx = __fmul_rn(geo.w, t.dx);
+    t.a0 = __fmul_rn(__fmul_rn(geo.z, t.dx), t.dx);
+    return t;
+}
+
+// Alpha at one pixel.  q = -sigma log2(e) = cA dx^2 + dy (cB dx + cC dy);
+// the entry is skipped there when sigma < 0 (q > 0) or alpha < 1/255
+// (log2 o + q below log2(1/255)), both decided before the exponential.
+// Returns false when skipped.  dy = mean y - pixel y.
+__device__ __forceinline__ bool eval_alpha(const float4 geo, const float4 geo2, const ColTerms &c,
+                                           float fy, float &dy, float &alpha, bool &capped) {
+    dy = __fsub_rn(geo.y, fy);
+    const float u = __fmaf_rn(geo2.x, dy, c.bdx);
+    const float q = __fmaf_rn(dy, u, c.a0);
+    const float p = __fadd_rn(q, geo2.y);              // log2(o exp(-sigma))
+    if (q > 0.f || p < kLog2AlphaMin) return false;
+    const float a = ex2_approx(p);
     capped = a > kAlphaCap;
     alpha = fminf(a, kAlphaCap);
-    return !(q > 0.f) && alpha >= kAlphaMin;
+    return true;
 }
 
-__global__ void __launch_bounds__(kBlendThreads)
+// Stages entries [0, cnt) of a batch into shared memory: slot i holds list
+// entry idx(i).  Each thread gathers two entries per round (ids first, then
+// records), so the dependent loads overlap without holding many registers.
+template <int kThreads, bool kRaw, typename Idx>
+__device__ __forceinline__ void stage_batch(uint32_t cnt, Idx idx, const uint32_t *__restrict__ pair_gid,
+                                            const float4 *__restrict__ xyod,
+                                            const float4 *__restrict__ conr,
+                                            const float4 *__restrict__ rgb, float4 *s_geo,
+                                            float4 *s_geo2, float4 *s_col, float4 *s_raw,
+                                            uint32_t *s_gid) {
+    for (uint32_t i0 = threadIdx.x; i0 < cnt; i0 += 2 * kThreads) {
+        const uint32_t i1 = i0 + kThreads;
+        const uint32_t g0 = pair_gid[idx(i0)];
+        const uint32_t g1 = i1 < cnt ? pair_gid[idx(i1)] : g0;
+        const float4 x0 = xyod[g0], c0 = conr[g0], r0 = rgb[g0];
+        const float4 x1 = xyod[g1], c1 = conr[g1], r1 = rgb[g1];
+        float4 geo, geo2;
+        stage_entry(x0, c0, geo, geo2);
+        s_geo[i0] = geo;
+        s_geo2[i0] = geo2;
+        s_col[i0] = r0;
+        if (kRaw) {
+            s_raw[i0] = make_float4(c0.x, c0.y, c0.z, 1.f / x0.z);
+            s_gid[i0] = g0;
+        }
+        if (i1 < cnt) {
+            stage_entry(x1, c1, geo, geo2);
+            s_geo[i1] = geo;
+            s_geo2[i1] = geo2;
+            s_col[i1] = r1;
+            if (kRaw) {
+                s_raw[i1] = make_float4(c1.x, c1.y, c1.z, 1.f / x1.z);
+                s_gid[i1] = g1;
+            }
+        }
+    }
+}
+
+template <int kRPL, bool kCull>
+__global__ void __launch_bounds__(kTilePixels / kRPL)
 k_render_fwd(CamConst cam, const float4 *__restrict__ xyod, const float4 *__restrict__ conr,
              const float4 *__restrict__ rgb, const uint32_t *__restrict__ pair_gid,
              const uint2 *__restrict__ ranges, float *__restrict__ image,
              float *__restrict__ T_final, uint32_t *__restrict__ last) {
+    constexpr int kThreads = kTilePixels / kRPL;
     __shared__ float4 s_geo[kBatch];
-    __shared__ float2 s_geo2[kBatch];
+    __shared__ float4 s_geo2[kBatch];
     __shared__ float4 s_col[kBatch];
 
     const int tile = blockIdx.x;
-    const int tx = tile % cam.tiles_x, ty = tile / cam.tiles_x;
-    const int px = tx * kTile + (threadIdx.x & (kTile - 1));
-    const int py = ty * kTile + (threadIdx.x >> 4);
-    const bool inside = px < cam.width && py < cam.height;
-    const float fx = (float)px + 0.5f, fy = (float)py + 0.5f;
+    const LaneGeom L = lane_geom<kRPL>(cam, tile);
     const uint2 range = ranges[tile];
+    const bool col_in = L.px < cam.width;
 
-    float T = 1.f, C0 = 0.f, C1 = 0.f, C2 = 0.f;
-    uint32_t last_idx = range.x;
-    bool done = !inside;
+    float T[kRPL], C0[kRPL], C1[kRPL], C2[kRPL];
+    uint32_t lst[kRPL];
+    bool done[kRPL];
+#pragma unroll
+    for (int r = 0; r < kRPL; r++) {
+        T[r] = 1.f; C0[r] = 0.f; C1[r] = 0.f; C2[r] = 0.f;
+        lst[r] = range.x;
+        done[r] = !(col_in && L.py0 + r < cam.height);
+    }
     for (uint32_t b = range.x; b < range.y; b += kBatch) {
-        if (__syncthreads_count(done) == kBlendThreads) break;
-        const uint32_t j = b + threadIdx.x;
-        if (j < range.y) {
-            const uint32_t g = pair_gid[j];
-            float4 geo;
-            float2 geo2;
-            stage_entry(xyod[g], conr[g], geo, geo2);
-            s_geo[threadIdx.x] = geo;
-            s_geo2[threadIdx.x] = geo2;
-            s_col[threadIdx.x] = rgb[g];
-        }
+        bool all_done = true;
+#pragma unroll
+        for (int r = 0; r < kRPL; r++) all_done &= done[r];
+        if (__syncthreads_count(all_done) == kThreads) break;
+        const uint32_t cnt = min((uint32_t)kBatch, range.y - b);
+        stage_batch<kThreads, false>(cnt, [b](uint32_t i) { return b + i; }, pair_gid, xyod, conr, rgb,
+                                     s_geo, s_geo2, s_col, nullptr, nullptr);
         __syncthreads();
-        const int cnt = (int)min((uint32_t)kBatch, range.y - b);
-        if (!done) {
-            for (int k = 0; k < cnt; k++) {
-                float dx, dy, a;
-                bool capped;
-                if (!eval_alpha(s_geo[k], s_geo2[k], fx, fy, dx, dy, a, capped)) continue;
-                const float nT = __fmaf_rn(-T, a, T);
-                if (nT < kTMin) { done = true; break; }
-                const float w = __fmul_rn(a, T);
-                const float4 c = s_col[k];
-                C0 = __fmaf_rn(w, c.x, C0);
-                C1 = __fmaf_rn(w, c.y, C1);
-                C2 = __fmaf_rn(w, c.z, C2);
-                T = nT;
-                last_idx = b + k + 1;
+        // A lane leaves the batch loop as soon as all its pixels have stopped
+        // (a per-lane exit, not a per-entry warp vote: measured faster).  The
+        // cull test depends only on the warp's strip, so it stays uniform
+        // among the lanes still in the loop.
+        if (kRPL == 1 && !kCull) {
+            // one pixel per lane: the lane breaks out at its stopping entry
+            if (!done[0]) {
+                for (uint32_t k = 0; k < cnt; k++) {
+                    const float4 geo = s_geo[k], geo2 = s_geo2[k];
+                    const ColTerms ct = col_terms(geo, L.fx);
+                    float dy, a;
+                    bool capped;
+                    if (!eval_alpha(geo, geo2, ct, L.fy0, dy, a, capped)) continue;
+                    const float nT = __fmaf_rn(-T[0], a, T[0]);
+                    if (nT < kTMin) {
+                        done[0] = true;
+                        break;
+                    }
+                    const float4 c = s_col[k];
+                    const float w = __fmul_rn(a, T[0]);
+                    C0[0] = __fmaf_rn(w, c.x, C0[0]);
+                    C1[0] = __fmaf_rn(w, c.y, C1[0]);
+                    C2[0] = __fmaf_rn(w, c.z, C2[0]);
+                    T[0] = nT;
+                    lst[0] = b + k + 1;
+                }
+            }
+        } else if (!all_done) {
+            for (uint32_t k = 0; k < cnt; k++) {
+                const float4 geo = s_geo[k], geo2 = s_geo2[k];
+                if (kCull && culled(geo, geo2, L)) continue;
+                const ColTerms ct = col_terms(geo, L.fx);
+                bool lane_done = true;
+#pragma unroll
+                for (int r = 0; r < kRPL; r++) {
+                    if (done[r]) continue;
+                    float dy, a;
+                    bool capped;
+                    if (eval_alpha(geo, geo2, ct, L.fy0 + (float)r, dy, a, capped)) {
+                        const float nT = __fmaf_rn(-T[r], a, T[r]);
+                        if (nT < kTMin) {
+                            done[r] = true;
+                            continue;
+                        }
+                        const float4 c = s_col[k];
+                        const float w = __fmul_rn(a, T[r]);
+                        C0[r] = __fmaf_rn(w, c.x, C0[r]);
+                        C1[r] = __fmaf_rn(w, c.y, C1[r]);
+                        C2[r] = __fmaf_rn(w, c.z, C2[r]);
+                        T[r] = nT;
+                        lst[r] = b + k + 1;
+                    }
+                    lane_done = false;
+                }
+                if (lane_done) break;
             }
         }
     }
-    if (inside) {
-        const size_t p = (size_t)py * cam.width + px;
-        image[3 * p] = __fmaf_rn(T, cam.bg[0], C0);
-        image[3 * p + 1] = __fmaf_rn(T, cam.bg[1], C1);
-        image[3 * p + 2] = __fmaf_rn(T, cam.bg[2], C2);
-        T_final[p] = T;
-        last[p] = last_idx;
+    if (col_in) {
+#pragma unroll
+        for (int r = 0; r < kRPL; r++) {
+            const int py = L.py0 + r;
+            if (py >= cam.height) continue;
+            const size_t p = (size_t)py * cam.width + L.px;
+            image[3 * p] = __fmaf_rn(T[r], cam.bg[0], C0[r]);
+            image[3 * p + 1] = __fmaf_rn(T[r], cam.bg[1], C1[r]);
+            image[3 * p + 2] = __fmaf_rn(T[r], cam.bg[2], C2[r]);
+            T_final[p] = T[r];
+            last[p] = lst[r];
+        }
     }
 }
 
@@ -135,99 +298,108 @@ __device__ __forceinline__ float warp_sum(float v) {
     return v;
 }
 
-__global__ void __launch_bounds__(kBlendThreads)
+template <int kRPL, bool kCull>
+__global__ void __launch_bounds__(kTilePixels / kRPL)
 k_render_bwd(CamConst cam, const float4 *__restrict__ xyod, const float4 *__restrict__ conr,
              const float4 *__restrict__ rgb, const uint32_t *__restrict__ pair_gid,
              const uint2 *__restrict__ ranges, const float *__restrict__ T_final,
              const uint32_t *__restrict__ last, const float *__restrict__ dL_dimage,
              float *__restrict__ grad2d) {
+    constexpr int kThreads = kTilePixels / kRPL;
     __shared__ float4 s_geo[kBatch];
-    __shared__ float2 s_geo2[kBatch];
+    __shared__ float4 s_geo2[kBatch];
     __shared__ float4 s_col[kBatch];
     __shared__ float4 s_raw[kBatch];  // A, B, C, 1/opacity
     __shared__ uint32_t s_gid[kBatch];
     __shared__ uint32_t s_max_last;
 
     const int tile = blockIdx.x;
-    const int tx = tile % cam.tiles_x, ty = tile / cam.tiles_x;
-    const int px = tx * kTile + (threadIdx.x & (kTile - 1));
-    const int py = ty * kTile + (threadIdx.x >> 4);
-    const bool inside = px < cam.width && py < cam.height;
-    const float fx = (float)px + 0.5f, fy = (float)py + 0.5f;
+    const LaneGeom L = lane_geom<kRPL>(cam, tile);
     const uint2 range = ranges[tile];
+    const bool col_in = L.px < cam.width;
     const int lane = threadIdx.x & 31;
 
-    float T = 1.f, g0 = 0.f, g1 = 0.f, g2 = 0.f;
-    uint32_t my_last = range.x;
-    if (inside) {
-        const size_t p = (size_t)py * cam.width + px;
-        T = T_final[p];
-        my_last = min(max(last[p], range.x), range.y);  // never walk outside the tile's list
-        g0 = dL_dimage[3 * p];
-        g1 = dL_dimage[3 * p + 1];
-        g2 = dL_dimage[3 * p + 2];
+    float T[kRPL], R0[kRPL], R1[kRPL], R2[kRPL], g0[kRPL], g1[kRPL], g2[kRPL];
+    uint32_t lst[kRPL];
+    uint32_t lane_max = range.x;
+#pragma unroll
+    for (int r = 0; r < kRPL; r++) {
+        T[r] = 1.f; g0[r] = 0.f; g1[r] = 0.f; g2[r] = 0.f;
+        R0[r] = cam.bg[0]; R1[r] = cam.bg[1]; R2[r] = cam.bg[2];
+        lst[r] = range.x;
+        const int py = L.py0 + r;
+        if (col_in && py < cam.height) {
+            const size_t p = (size_t)py * cam.width + L.px;
+            T[r] = T_final[p];
+            lst[r] = min(max(last[p], range.x), range.y);  // never walk outside the tile's list
+            g0[r] = dL_dimage[3 * p];
+            g1[r] = dL_dimage[3 * p + 1];
+            g2[r] = dL_dimage[3 * p + 2];
+        }
+        lane_max = max(lane_max, lst[r]);
     }
-    float R0 = cam.bg[0], R1 = cam.bg[1], R2 = cam.bg[2];
+    // entries at or past every pixel's last are not walked: per warp and per CTA
+    uint32_t warp_max = lane_max;
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) warp_max = max(warp_max, __shfl_xor_sync(0xffffffffu, warp_max, o));
     if (threadIdx.x == 0) s_max_last = range.x;
     __syncthreads();
-    atomicMax(&s_max_last, my_last);
+    if (lane == 0) atomicMax(&s_max_last, warp_max);
     __syncthreads();
     const uint32_t max_last = s_max_last;
 
     for (uint32_t bend = max_last; bend > range.x;) {
         const uint32_t bstart = bend - range.x > (uint32_t)kBatch ? bend - kBatch : range.x;
         const uint32_t cnt = bend - bstart;
-        if (threadIdx.x < cnt) {
-            const uint32_t j = bend - 1 - threadIdx.x;  // slot 0 = back-most entry
-            const uint32_t g = pair_gid[j];
-            const float4 xo = xyod[g], cr = conr[g];
-            float4 geo;
-            float2 geo2;
-            stage_entry(xo, cr, geo, geo2);
-            s_geo[threadIdx.x] = geo;
-            s_geo2[threadIdx.x] = geo2;
-            s_col[threadIdx.x] = rgb[g];
-            s_raw[threadIdx.x] = make_float4(cr.x, cr.y, cr.z, 1.f / xo.z);
-            s_gid[threadIdx.x] = g;
-        }
+        // slot i holds list entry bend - 1 - i (slot 0 = back-most)
+        stage_batch<kThreads, true>(cnt, [bend](uint32_t i) { return bend - 1 - i; }, pair_gid, xyod,
+                                    conr, rgb, s_geo, s_geo2, s_col, s_raw, s_gid);
         __syncthreads();
-        for (uint32_t k = 0; k < cnt; k++) {
+        // skip the slots this warp's pixels never reached
+        const uint32_t k0 = bend > warp_max ? min(bend - warp_max, cnt) : 0u;
+        for (uint32_t k = k0; k < cnt; k++) {
             const uint32_t j = bend - 1 - k;
-            float v = 0.f, gx = 0.f, gy = 0.f, gxx = 0.f, gxy = 0.f, gyy = 0.f;
-            float cr0 = 0.f, cr1 = 0.f, cr2 = 0.f;
+            const float4 geo = s_geo[k], geo2 = s_geo2[k];
+            if (kCull && culled(geo, geo2, L)) continue;
+            const ColTerms ct = col_terms(geo, L.fx);
+            const float4 c = s_col[k];
+            float sv = 0.f, sgy = 0.f, sgyy = 0.f, cr0 = 0.f, cr1 = 0.f, cr2 = 0.f;
             bool contrib = false;
-            if (j < my_last) {
-                float dx, dy, a;
+#pragma unroll
+            for (int r = 0; r < kRPL; r++) {
+                if (j >= lst[r]) continue;
+                float dy, a;
                 bool capped;
-                if (eval_alpha(s_geo[k], s_geo2[k], fx, fy, dx, dy, a, capped)) {
-                    contrib = true;
-                    const float Ti = __fmul_rn(T, rcp_approx(__fsub_rn(1.f, a)));
-                    const float w = __fmul_rn(a, Ti);
-                    const float4 c = s_col[k];
-                    cr0 = w * g0;
-                    cr1 = w * g1;
-                    cr2 = w * g2;
-                    const float d0 = c.x - R0, d1 = c.y - R1, d2 = c.z - R2;
-                    const float dLda = Ti * (d0 * g0 + d1 * g1 + d2 * g2);
-                    R0 = __fmaf_rn(a, d0, R0);
-                    R1 = __fmaf_rn(a, d1, R1);
-                    R2 = __fmaf_rn(a, d2, R2);
-                    v = capped ? 0.f : dLda * a;  // dL/dsigma = -v, dL/do = v / o
-                    gx = v * dx;
-                    gy = v * dy;
-                    gxx = gx * dx;
-                    gxy = gx * dy;
-                    gyy = gy * dy;
-                    T = Ti;
-                }
+                if (!eval_alpha(geo, geo2, ct, L.fy0 + (float)r, dy, a, capped)) continue;
+                contrib = true;
+                const float Ti = __fmul_rn(T[r], rcp_approx(__fsub_rn(1.f, a)));
+                const float w = __fmul_rn(a, Ti);
+                cr0 = __fmaf_rn(w, g0[r], cr0);
+                cr1 = __fmaf_rn(w, g1[r], cr1);
+                cr2 = __fmaf_rn(w, g2[r], cr2);
+                const float d0 = c.x - R0[r], d1 = c.y - R1[r], d2 = c.z - R2[r];
+                const float dLda = Ti * (d0 * g0[r] + d1 * g1[r] + d2 * g2[r]);
+                R0[r] = __fmaf_rn(a, d0, R0[r]);
+                R1[r] = __fmaf_rn(a, d1, R1[r]);
+                R2[r] = __fmaf_rn(a, d2, R2[r]);
+                const float v = capped ? 0.f : dLda * a;  // dL/dsigma = -v, dL/do = v / o
+                sv += v;
+                const float vy = v * dy;
+                sgy += vy;
+                sgyy = __fmaf_rn(vy, dy, sgyy);
+                T[r] = Ti;
             }
             if (__any_sync(0xffffffffu, contrib)) {
-                v = warp_sum(v);
-                gx = warp_sum(gx);
-                gy = warp_sum(gy);
-                gxx = warp_sum(gxx);
-                gxy = warp_sum(gxy);
-                gyy = warp_sum(gyy);
+                // per lane: sum v dx = dx sum v, sum v dx^2, sum v dx dy
+                float sgx = sv * ct.dx;
+                float sgxx = sgx * ct.dx;
+                float sgxy = sgy * ct.dx;
+                sv = warp_sum(sv);
+                sgx = warp_sum(sgx);
+                sgy = warp_sum(sgy);
+                sgxx = warp_sum(sgxx);
+                sgxy = warp_sum(sgxy);
+                sgyy = warp_sum(sgyy);
                 cr0 = warp_sum(cr0);
                 cr1 = warp_sum(cr1);
                 cr2 = warp_sum(cr2);
@@ -235,10 +407,10 @@ k_render_bwd(CamConst cam, const float4 *__restrict__ xyod, const float4 *__rest
                     const float4 raw = s_raw[k];
                     float *dst = grad2d + 12 * (size_t)s_gid[k];
                     atomicAdd(reinterpret_cast<float4 *>(dst),
-                              make_float4(-(raw.x * gx + raw.y * gy), -(raw.y * gx + raw.z * gy),
-                                          -0.5f * gxx, -gxy));
+                              make_float4(-(raw.x * sgx + raw.y * sgy), -(raw.y * sgx + raw.z * sgy),
+                                          -0.5f * sgxx, -sgxy));
                     atomicAdd(reinterpret_cast<float4 *>(dst + 4),
-                              make_float4(-0.5f * gyy, v * raw.w, cr0, cr1));
+                              make_float4(-0.5f * sgyy, sv * raw.w, cr0, cr1));
                     atomicAdd(dst + 8, cr2);
                 }
             }
@@ -248,13 +420,14 @@ k_render_bwd(CamConst cam, const float4 *__restrict__ xyod, const float4 *__rest
     }
 }
 
-// Same walk as k_render_fwd, counting instead of blending.
-__global__ void __launch_bounds__(kBlendThreads)
+// The forward's walk with counters instead of blending (no culling, one pixel
+// per thread): the work the method must do.
+__global__ void __launch_bounds__(kTilePixels)
 k_render_stats(CamConst cam, const float4 *__restrict__ xyod, const float4 *__restrict__ conr,
                const uint32_t *__restrict__ pair_gid, const uint2 *__restrict__ ranges,
                const uint32_t *__restrict__ last, unsigned long long *__restrict__ counts) {
     __shared__ float4 s_geo[kBatch];
-    __shared__ float2 s_geo2[kBatch];
+    __shared__ float4 s_geo2[kBatch];
     __shared__ unsigned long long s_c[3];
     const int tile = blockIdx.x;
     const int tx = tile % cam.tiles_x, ty = tile / cam.tiles_x;
@@ -268,12 +441,11 @@ k_render_stats(CamConst cam, const float4 *__restrict__ xyod, const float4 *__re
     unsigned long long visits = 0, adds = 0;
     bool done = !inside;
     for (uint32_t b = range.x; b < range.y; b += kBatch) {
-        if (__syncthreads_count(done) == kBlendThreads) break;
+        if (__syncthreads_count(done) == kTilePixels) break;
         const uint32_t j = b + threadIdx.x;
         if (j < range.y) {
             const uint32_t g = pair_gid[j];
-            float4 geo;
-            float2 geo2;
+            float4 geo, geo2;
             stage_entry(xyod[g], conr[g], geo, geo2);
             s_geo[threadIdx.x] = geo;
             s_geo2[threadIdx.x] = geo2;
@@ -282,10 +454,12 @@ k_render_stats(CamConst cam, const float4 *__restrict__ xyod, const float4 *__re
         const int cnt = (int)min((uint32_t)kBatch, range.y - b);
         if (!done) {
             for (int k = 0; k < cnt; k++) {
-                float dx, dy, a;
+                float dy, a;
                 bool capped;
                 visits++;
-                if (!eval_alpha(s_geo[k], s_geo2[k], fx, fy, dx, dy, a, capped)) continue;
+                const float4 geo = s_geo[k], geo2 = s_geo2[k];
+                const ColTerms ct = col_terms(geo, fx);
+                if (!eval_alpha(geo, geo2, ct, fy, dy, a, capped)) continue;
                 const float nT = __fmaf_rn(-T, a, T);
                 if (nT < kTMin) { done = true; break; }
                 adds++;
@@ -336,7 +510,7 @@ cudaError_t launch_render_fwd(const CamConst &c, const gs_projected &proj, const
                               float *image, float *T_final, uint32_t *last, cudaStream_t s) {
     const int tiles = c.tiles_x * c.tiles_y;
     prof_before("render_fwd", s);
-    k_render_fwd<<<tiles, kBlendThreads, 0, s>>>(
+    k_render_fwd<GS_FWD_RPL, GS_FWD_CULL != 0><<<tiles, kTilePixels / GS_FWD_RPL, 0, s>>>(
         c, reinterpret_cast<const float4 *>(proj.xy_opacity_depth),
         reinterpret_cast<const float4 *>(proj.conic_radius), reinterpret_cast<const float4 *>(proj.rgb),
         bins.pair_gid, reinterpret_cast<const uint2 *>(bins.ranges), image, T_final, last);
@@ -349,7 +523,7 @@ cudaError_t launch_render_bwd(const CamConst &c, const gs_projected &proj, const
                               float *grad2d, cudaStream_t s) {
     const int tiles = c.tiles_x * c.tiles_y;
     prof_before("render_bwd", s);
-    k_render_bwd<<<tiles, kBlendThreads, 0, s>>>(
+    k_render_bwd<GS_BWD_RPL, GS_BWD_CULL != 0><<<tiles, kTilePixels / GS_BWD_RPL, 0, s>>>(
         c, reinterpret_cast<const float4 *>(proj.xy_opacity_depth),
         reinterpret_cast<const float4 *>(proj.conic_radius), reinterpret_cast<const float4 *>(proj.rgb),
         bins.pair_gid, reinterpret_cast<const uint2 *>(bins.ranges), T_final, last, dL_dimage,
@@ -364,7 +538,7 @@ cudaError_t launch_render_stats(const CamConst &c, const gs_projected &proj, con
     if (e != cudaSuccess) return e;
     const int tiles = c.tiles_x * c.tiles_y;
     prof_before("render_stats", s);
-    k_render_stats<<<tiles, kBlendThreads, 0, s>>>(
+    k_render_stats<<<tiles, kTilePixels, 0, s>>>(
         c, reinterpret_cast<const float4 *>(proj.xy_opacity_depth),
         reinterpret_cast<const float4 *>(proj.conic_radius), bins.pair_gid,
         reinterpret_cast<const uint2 *>(bins.ranges), last,
