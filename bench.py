@@ -70,8 +70,8 @@ OPS_BWD_ADD = 32
 #   emit         16 B/G records read + 8 B/P written
 #   tile_sort    16 B/P per pass
 #   ranges       4 B/P read
-#   project_bwd  56 B/G raw parameters + 48 B/G 2D gradients read,
-#                56 B/G raw gradients written
+#   project_bwd  56 B/G raw parameters + 48 B/G 2D sums + 32 B/G records read,
+#                48 B/G 2D gradients + 56 B/G raw gradients written
 BYTES = {
     "project": lambda G, P: 124 * G,
     "depth_keys": lambda G, P: 12 * G,
@@ -80,7 +80,7 @@ BYTES = {
     "emit": lambda G, P: 16 * G + 8 * P,
     "tile_sort": lambda G, P: 16 * P,
     "ranges": lambda G, P: 4 * P,
-    "project_bwd": lambda G, P: 160 * G,
+    "project_bwd": lambda G, P: 240 * G,
 }
 ALU_KERNELS = ("render_fwd", "render_bwd")
 

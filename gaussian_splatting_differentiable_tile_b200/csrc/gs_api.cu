@@ -275,7 +275,7 @@ int gs_render_bwd(const gs_camera *cam, int64_t n, const gs_params *params,
         return GS_ERR_CUDA;
     if (launch_render_bwd(c, *proj, *bins, T_final, last, dL_dimage, grad2d, s) != cudaSuccess)
         return GS_ERR_CUDA;
-    if (launch_project_bwd(c, n, *params, grad2d, *grads, s) != cudaSuccess) return GS_ERR_CUDA;
+    if (launch_project_bwd(c, n, *params, *proj, grad2d, *grads, s) != cudaSuccess) return GS_ERR_CUDA;
     return GS_OK;
 }
 

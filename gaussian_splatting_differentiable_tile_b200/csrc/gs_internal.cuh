@@ -155,7 +155,8 @@ __device__ __forceinline__ void set_status(int32_t *status, int32_t code) {
 cudaError_t launch_project(const CamConst &c, int64_t n, const gs_params &p, const gs_projected &o,
                            cudaStream_t s);
 cudaError_t launch_project_bwd(const CamConst &c, int64_t n, const gs_params &p,
-                               const float *grad2d, const gs_grads &g, cudaStream_t s);
+                               const gs_projected &proj, float *grad2d, const gs_grads &g,
+                               cudaStream_t s);
 cudaError_t launch_bin_and_sort(const CamConst &c, int64_t n, const gs_projected &proj,
                                 const gs_bins &bins, const BinsLayout &L, cudaStream_t s);
 cudaError_t launch_render_fwd(const CamConst &c, const gs_projected &proj, const gs_bins &bins,

@@ -172,11 +172,19 @@ __device__ __forceinline__ void rotmat_vjp(const float *qh, const float *G, floa
                    x * G[6] + y * G[7]);
 }
 
-// grad2d per Gaussian: dL/d(mx, my, A, B, C, opacity, r, g, b, -, -, -).
+// grad2d per Gaussian arrives holding the blend backward's sums over pixels:
+//   sum v, sum v dx, sum v dy, sum v dx^2, sum v dx dy, sum v dy^2, dL/d(r, g, b)
+// with v = alpha dL/dalpha and dx, dy = mean - pixel.  With sigma =
+// 1/2 (A dx^2 + C dy^2) + B dx dy and dL/dsigma = -v, dL/do = v / o:
+//   dL/dmx = -(A sum v dx + B sum v dy), dL/dmy = -(B sum v dx + C sum v dy),
+//   dL/dA = -sum v dx^2 / 2, dL/dB = -sum v dx dy, dL/dC = -sum v dy^2 / 2.
+// Those values are written back: on return grad2d holds
+// dL/d(mx, my, A, B, C, opacity, r, g, b, 0, 0, 0).
 __global__ void __launch_bounds__(256)
 k_project_bwd(CamConst cam, int n, const float *__restrict__ means,
               const float *__restrict__ log_scales, const float *__restrict__ quats,
-              const float *__restrict__ logits, const float4 *__restrict__ grad2d,
+              const float *__restrict__ logits, const float4 *__restrict__ xyod,
+              const float4 *__restrict__ conr, float4 *__restrict__ grad2d,
               float *__restrict__ d_means, float *__restrict__ d_log_scales,
               float *__restrict__ d_quats, float *__restrict__ d_logits,
               float *__restrict__ d_colors) {
@@ -188,7 +196,17 @@ k_project_bwd(CamConst cam, int n, const float *__restrict__ means,
     float q[4] = {q4.x, q4.y, q4.z, q4.w};
     Proj P;
     project_one(cam, mu, ls, q, logits[g], P);
-    const float4 g0 = grad2d[3 * g], g1 = grad2d[3 * g + 1], g2 = grad2d[3 * g + 2];
+    const float4 s0 = grad2d[3 * g], s1 = grad2d[3 * g + 1], s2 = grad2d[3 * g + 2];
+    // Conic and opacity as the blend used them: the projected records.
+    const float4 cr = conr[g];
+    const float op = xyod[g].z;
+    const float4 g0 = make_float4(-(cr.x * s0.y + cr.y * s0.z), -(cr.y * s0.y + cr.z * s0.z),
+                                  -0.5f * s0.w, -s1.x);
+    const float4 g1 = make_float4(-0.5f * s1.y, op > 0.f ? s0.x / op : 0.f, s1.z, s1.w);
+    const float4 g2 = make_float4(s2.x, 0.f, 0.f, 0.f);
+    grad2d[3 * g] = g0;
+    grad2d[3 * g + 1] = g1;
+    grad2d[3 * g + 2] = g2;
     if (!P.valid) {  // [GSP] s6: culled Gaussians get exact zeros
         for (int k = 0; k < 3; k++) {
             d_means[3 * g + k] = 0.f;
@@ -322,14 +340,17 @@ cudaError_t launch_project(const CamConst &c, int64_t n, const gs_params &p, con
 }
 
 cudaError_t launch_project_bwd(const CamConst &c, int64_t n, const gs_params &p,
-                               const float *grad2d, const gs_grads &g, cudaStream_t s) {
+                               const gs_projected &proj, float *grad2d, const gs_grads &g,
+                               cudaStream_t s) {
     if (n == 0) return cudaSuccess;
     const int threads = 256;
     const int blocks = (int)((n + threads - 1) / threads);
     prof_before("project_bwd", s);
     k_project_bwd<<<blocks, threads, 0, s>>>(c, (int)n, p.means, p.log_scales, p.quats,
                                              p.opacity_logits,
-                                             reinterpret_cast<const float4 *>(grad2d), g.means,
+                                             reinterpret_cast<const float4 *>(proj.xy_opacity_depth),
+                                             reinterpret_cast<const float4 *>(proj.conic_radius),
+                                             reinterpret_cast<float4 *>(grad2d), g.means,
                                              g.log_scales, g.quats, g.opacity_logits, g.colors);
     prof_after(s);
     return cudaGetLastError();

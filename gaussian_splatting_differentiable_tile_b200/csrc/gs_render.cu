@@ -44,7 +44,7 @@
 #define GS_FWD_CULL 0
 #endif
 #ifndef GS_BWD_RPL
-#define GS_BWD_RPL 2
+#define GS_BWD_RPL 4
 #endif
 #ifndef GS_BWD_CULL
 #define GS_BWD_CULL 1
@@ -148,15 +148,14 @@ __device__ __forceinline__ bool eval_alpha(const float4 geo, const float4 geo2, 
 }
 
 // Stages entries [0, cnt) of a batch into shared memory: slot i holds list
-// entry idx(i).  Each thread gathers two entries per round (ids first, then
+// entry idx(i) (and, for the backward, its Gaussian id).  Each thread gathers two entries per round (ids first, then
 // records), so the dependent loads overlap without holding many registers.
-template <int kThreads, bool kRaw, typename Idx>
+template <int kThreads, bool kGid, typename Idx>
 __device__ __forceinline__ void stage_batch(uint32_t cnt, Idx idx, const uint32_t *__restrict__ pair_gid,
                                             const float4 *__restrict__ xyod,
                                             const float4 *__restrict__ conr,
                                             const float4 *__restrict__ rgb, float4 *s_geo,
-                                            float4 *s_geo2, float4 *s_col, float4 *s_raw,
-                                            uint32_t *s_gid) {
+                                            float4 *s_geo2, float4 *s_col, uint32_t *s_gid) {
     for (uint32_t i0 = threadIdx.x; i0 < cnt; i0 += 2 * kThreads) {
         const uint32_t i1 = i0 + kThreads;
         const uint32_t g0 = pair_gid[idx(i0)];
@@ -168,19 +167,13 @@ __device__ __forceinline__ void stage_batch(uint32_t cnt, Idx idx, const uint32_
         s_geo[i0] = geo;
         s_geo2[i0] = geo2;
         s_col[i0] = r0;
-        if (kRaw) {
-            s_raw[i0] = make_float4(c0.x, c0.y, c0.z, 1.f / x0.z);
-            s_gid[i0] = g0;
-        }
+        if (kGid) s_gid[i0] = g0;
         if (i1 < cnt) {
             stage_entry(x1, c1, geo, geo2);
             s_geo[i1] = geo;
             s_geo2[i1] = geo2;
             s_col[i1] = r1;
-            if (kRaw) {
-                s_raw[i1] = make_float4(c1.x, c1.y, c1.z, 1.f / x1.z);
-                s_gid[i1] = g1;
-            }
+            if (kGid) s_gid[i1] = g1;
         }
     }
 }
@@ -217,7 +210,7 @@ k_render_fwd(CamConst cam, const float4 *__restrict__ xyod, const float4 *__rest
         if (__syncthreads_count(all_done) == kThreads) break;
         const uint32_t cnt = min((uint32_t)kBatch, range.y - b);
         stage_batch<kThreads, false>(cnt, [b](uint32_t i) { return b + i; }, pair_gid, xyod, conr, rgb,
-                                     s_geo, s_geo2, s_col, nullptr, nullptr);
+                                     s_geo, s_geo2, s_col, nullptr);
         __syncthreads();
         // A lane leaves the batch loop as soon as all its pixels have stopped
         // (a per-lane exit, not a per-entry warp vote: measured faster).  The
@@ -298,6 +291,51 @@ __device__ __forceinline__ float warp_sum(float v) {
     return v;
 }
 
+// Warp reduce-scatter of nine values per lane.  Five xor levels (16, 8, 4, 2,
+// 1); at each level a lane keeps one half of its values and sends the other
+// half to its partner, which keeps that half: 46 instructions instead of the
+// 90 of nine full butterflies.  On return every even lane whose *idx is in
+// [0, 9) holds the warp total of value *idx (one lane per value).
+__device__ __forceinline__ float reduce_scatter9(const float (&v)[9], int lane, int *idx) {
+    const bool b4 = lane & 16, b3 = lane & 8, b2 = lane & 4, b1 = lane & 2;
+    float k[5];
+#pragma unroll
+    for (int i = 0; i < 5; i++) {
+        const float lo = v[i], hi = i < 4 ? v[5 + i] : 0.f;
+        k[i] = (b4 ? hi : lo) + __shfl_xor_sync(0xffffffffu, b4 ? lo : hi, 16);
+    }
+    float m[3];
+#pragma unroll
+    for (int i = 0; i < 3; i++) {
+        const float lo = k[i], hi = i < 2 ? k[3 + i] : 0.f;
+        m[i] = (b3 ? hi : lo) + __shfl_xor_sync(0xffffffffu, b3 ? lo : hi, 8);
+    }
+    float n[2];
+#pragma unroll
+    for (int i = 0; i < 2; i++) {
+        const float lo = m[i], hi = i == 0 ? m[2] : 0.f;
+        n[i] = (b2 ? hi : lo) + __shfl_xor_sync(0xffffffffu, b2 ? lo : hi, 4);
+    }
+    float x = (b1 ? n[1] : n[0]) + __shfl_xor_sync(0xffffffffu, b1 ? n[0] : n[1], 2);
+    x += __shfl_xor_sync(0xffffffffu, x, 1);
+    const int q = 2 * (int)b2 + (int)b1, p = 3 * (int)b3 + q;
+    *idx = (q <= 2 && p <= 4 && !(lane & 1)) ? 5 * (int)b4 + p : 9;
+    return x;
+}
+
+// Backward of the blend.  Per pixel, from the last added entry back to the
+// first: with T the transmittance after entry i, r = 1 / (1 - alpha_i),
+// T_i = T r, and sg = <S_i, g> where S_i = T_{i+1} R_i is the colour already
+// composited behind i (S_last = T_final bg),
+//     dL/dalpha_i = T_i <c_i, g> - sg / (1 - alpha_i),
+//     sg <- sg + alpha_i T_i <c_i, g>,   dL/dc_i = alpha_i T_i g.
+// (the same quantities as T_i <c_i - R_i, g> with R the normalised colour
+// behind, carried as one scalar instead of a colour).  The nine sums
+// per entry, over the warp's pixels, are
+//     sum v, sum v dx, sum v dy, sum v dx^2, sum v dx dy, sum v dy^2, sum w g
+// with v = alpha dL/dalpha (0 when alpha was capped), w = alpha T_i; they are
+// added into grad2d, and k_project_bwd maps them to dL/d(mean2d, conic,
+// opacity) with the Gaussian's own A, B, C, o.
 template <int kRPL, bool kCull>
 __global__ void __launch_bounds__(kTilePixels / kRPL)
 k_render_bwd(CamConst cam, const float4 *__restrict__ xyod, const float4 *__restrict__ conr,
@@ -309,7 +347,6 @@ k_render_bwd(CamConst cam, const float4 *__restrict__ xyod, const float4 *__rest
     __shared__ float4 s_geo[kBatch];
     __shared__ float4 s_geo2[kBatch];
     __shared__ float4 s_col[kBatch];
-    __shared__ float4 s_raw[kBatch];  // A, B, C, 1/opacity
     __shared__ uint32_t s_gid[kBatch];
     __shared__ uint32_t s_max_last;
 
@@ -319,13 +356,12 @@ k_render_bwd(CamConst cam, const float4 *__restrict__ xyod, const float4 *__rest
     const bool col_in = L.px < cam.width;
     const int lane = threadIdx.x & 31;
 
-    float T[kRPL], R0[kRPL], R1[kRPL], R2[kRPL], g0[kRPL], g1[kRPL], g2[kRPL];
+    float T[kRPL], sg[kRPL], g0[kRPL], g1[kRPL], g2[kRPL];
     uint32_t lst[kRPL];
     uint32_t lane_max = range.x;
 #pragma unroll
     for (int r = 0; r < kRPL; r++) {
         T[r] = 1.f; g0[r] = 0.f; g1[r] = 0.f; g2[r] = 0.f;
-        R0[r] = cam.bg[0]; R1[r] = cam.bg[1]; R2[r] = cam.bg[2];
         lst[r] = range.x;
         const int py = L.py0 + r;
         if (col_in && py < cam.height) {
@@ -336,6 +372,7 @@ k_render_bwd(CamConst cam, const float4 *__restrict__ xyod, const float4 *__rest
             g1[r] = dL_dimage[3 * p + 1];
             g2[r] = dL_dimage[3 * p + 2];
         }
+        sg[r] = T[r] * (cam.bg[0] * g0[r] + cam.bg[1] * g1[r] + cam.bg[2] * g2[r]);
         lane_max = max(lane_max, lst[r]);
     }
     // entries at or past every pixel's last are not walked: per warp and per CTA
@@ -353,7 +390,7 @@ k_render_bwd(CamConst cam, const float4 *__restrict__ xyod, const float4 *__rest
         const uint32_t cnt = bend - bstart;
         // slot i holds list entry bend - 1 - i (slot 0 = back-most)
         stage_batch<kThreads, true>(cnt, [bend](uint32_t i) { return bend - 1 - i; }, pair_gid, xyod,
-                                    conr, rgb, s_geo, s_geo2, s_col, s_raw, s_gid);
+                                    conr, rgb, s_geo, s_geo2, s_col, s_gid);
         __syncthreads();
         // skip the slots this warp's pixels never reached
         const uint32_t k0 = bend > warp_max ? min(bend - warp_max, cnt) : 0u;
@@ -372,16 +409,15 @@ k_render_bwd(CamConst cam, const float4 *__restrict__ xyod, const float4 *__rest
                 bool capped;
                 if (!eval_alpha(geo, geo2, ct, L.fy0 + (float)r, dy, a, capped)) continue;
                 contrib = true;
-                const float Ti = __fmul_rn(T[r], rcp_approx(__fsub_rn(1.f, a)));
+                const float ri = rcp_approx(__fsub_rn(1.f, a));
+                const float Ti = __fmul_rn(T[r], ri);
                 const float w = __fmul_rn(a, Ti);
+                const float cg = __fmaf_rn(c.z, g2[r], __fmaf_rn(c.y, g1[r], c.x * g0[r]));
+                const float dLda = ri * __fmaf_rn(T[r], cg, -sg[r]);
+                sg[r] = __fmaf_rn(w, cg, sg[r]);
                 cr0 = __fmaf_rn(w, g0[r], cr0);
                 cr1 = __fmaf_rn(w, g1[r], cr1);
                 cr2 = __fmaf_rn(w, g2[r], cr2);
-                const float d0 = c.x - R0[r], d1 = c.y - R1[r], d2 = c.z - R2[r];
-                const float dLda = Ti * (d0 * g0[r] + d1 * g1[r] + d2 * g2[r]);
-                R0[r] = __fmaf_rn(a, d0, R0[r]);
-                R1[r] = __fmaf_rn(a, d1, R1[r]);
-                R2[r] = __fmaf_rn(a, d2, R2[r]);
                 const float v = capped ? 0.f : dLda * a;  // dL/dsigma = -v, dL/do = v / o
                 sv += v;
                 const float vy = v * dy;
@@ -390,29 +426,11 @@ k_render_bwd(CamConst cam, const float4 *__restrict__ xyod, const float4 *__rest
                 T[r] = Ti;
             }
             if (__any_sync(0xffffffffu, contrib)) {
-                // per lane: sum v dx = dx sum v, sum v dx^2, sum v dx dy
-                float sgx = sv * ct.dx;
-                float sgxx = sgx * ct.dx;
-                float sgxy = sgy * ct.dx;
-                sv = warp_sum(sv);
-                sgx = warp_sum(sgx);
-                sgy = warp_sum(sgy);
-                sgxx = warp_sum(sgxx);
-                sgxy = warp_sum(sgxy);
-                sgyy = warp_sum(sgyy);
-                cr0 = warp_sum(cr0);
-                cr1 = warp_sum(cr1);
-                cr2 = warp_sum(cr2);
-                if (lane == 0) {
-                    const float4 raw = s_raw[k];
-                    float *dst = grad2d + 12 * (size_t)s_gid[k];
-                    atomicAdd(reinterpret_cast<float4 *>(dst),
-                              make_float4(-(raw.x * sgx + raw.y * sgy), -(raw.y * sgx + raw.z * sgy),
-                                          -0.5f * sgxx, -sgxy));
-                    atomicAdd(reinterpret_cast<float4 *>(dst + 4),
-                              make_float4(-0.5f * sgyy, sv * raw.w, cr0, cr1));
-                    atomicAdd(dst + 8, cr2);
-                }
+                const float sgx = sv * ct.dx;
+                const float vals[9] = {sv, sgx, sgy, sgx * ct.dx, sgy * ct.dx, sgyy, cr0, cr1, cr2};
+                int idx;
+                const float tot = reduce_scatter9(vals, lane, &idx);
+                if (idx < 9) atomicAdd(grad2d + 12 * (size_t)s_gid[k] + idx, tot);
             }
         }
         __syncthreads();
