@@ -15,7 +15,7 @@
 // ceil(43..45 / 8) passes of 12 bytes.
 //
 // Both sorts are LSD radix sorts built from one "onesweep" pass kernel:
-// a block ranks its 4096 keys with warp-level match/popc, publishes its digit
+// a block ranks its 4096 keys with warp ballots and popc, publishes its digit
 // counts, and resolves its global offsets by a decoupled look-back over the
 // preceding partitions (bounded: a poll loop that runs out sets
 // GS_ERR_DEVICE_TIMEOUT and the kernel still finishes).  Partitions are taken
@@ -29,6 +29,24 @@ __device__ __forceinline__ uint32_t lanemask_lt() {
     uint32_t m;
     asm("mov.u32 %0, %%lanemask_lt;" : "=r"(m));
     return m;
+}
+
+// Lanes of the warp holding the same digit as this lane, for digits of
+// `bits` (<= 8) bits or the sentinel kRadix: one ballot per digit bit (and one
+// for the sentinel), each lane keeping the lanes that agree with it.  Cheaper
+// than a match instruction on this hardware.
+__device__ __forceinline__ uint32_t digit_peers(uint32_t d, int bits) {
+    const uint32_t valid = __ballot_sync(0xffffffffu, d < kRadix);
+    uint32_t peers = d < kRadix ? valid : ~valid;
+#pragma unroll
+    for (int b = 0; b < kRadixBits; b++) {
+        if (b < bits) {
+            const bool set = (d >> b) & 1u;
+            const uint32_t bal = __ballot_sync(0xffffffffu, set);
+            peers &= set ? bal : ~bal;
+        }
+    }
+    return peers;
 }
 
 // Exclusive block-wide scan of one value per thread (blockDim = 256).
@@ -57,13 +75,13 @@ __device__ __forceinline__ uint32_t block_exclusive_scan_256(uint32_t v, uint32_
 
 // Decoupled look-back for one digit: the sum of the digit's counts over
 // partitions [0, q0], read from the partitions' published words back to the
-// nearest inclusive one.  Eight words are requested at a time so a chain of
-// aggregates costs one L2 round trip per eight partitions.  A word that stays
+// nearest inclusive one.  32 words are requested at a time, so a chain of
+// aggregates costs one L2 round trip per 32 partitions.  A word that stays
 // unpublished for kSpinLimit polls records GS_ERR_DEVICE_TIMEOUT and counts
 // as zero, so the kernel always finishes.
 __device__ __forceinline__ uint32_t lookback_digit(const uint32_t *lookback, int d, int64_t q0,
                                                    int32_t *status) {
-    constexpr int kWindow = 8;
+    constexpr int kWindow = 32;
     uint32_t excl = 0;
     uint32_t spins = 0;
     for (int64_t q = q0; q >= 0; q -= kWindow) {
@@ -196,23 +214,43 @@ k_onesweep(const uint32_t *__restrict__ keys_in, const uint32_t *__restrict__ va
         // (warp, item, lane), which the ranking below preserves (stable).
         const uint32_t base = p * kSortPart + warp * (32 * kSortItems);
         uint32_t key[kSortItems], val[kSortItems], dig[kSortItems], rank[kSortItems];
+        if (base + 32 * kSortItems <= n) {
+            // a full slice: every load is issued before any is used (a
+            // per-item guard and value select keep them from overlapping)
 #pragma unroll
-        for (int i = 0; i < kSortItems; i++) {
-            const uint32_t idx = base + i * 32 + lane;
-            if (idx < n) {
-                key[i] = keys_in[idx];
-                val[i] = iota_vals ? idx : vals_in[idx];
-                dig[i] = (key[i] >> shift) & mask;
+            for (int i = 0; i < kSortItems; i++) key[i] = __ldcg(keys_in + base + i * 32 + lane);
+            if (iota_vals) {
+#pragma unroll
+                for (int i = 0; i < kSortItems; i++) val[i] = base + i * 32 + lane;
             } else {
-                key[i] = 0; val[i] = 0;
-                dig[i] = kRadix;  // sentinel: not counted
+#pragma unroll
+                for (int i = 0; i < kSortItems; i++) val[i] = __ldcg(vals_in + base + i * 32 + lane);
+            }
+#pragma unroll
+            for (int i = 0; i < kSortItems; i++) dig[i] = (key[i] >> shift) & mask;
+        } else {
+#pragma unroll
+            for (int i = 0; i < kSortItems; i++) {
+                const uint32_t idx = base + i * 32 + lane;
+                if (idx < n) {
+                    key[i] = keys_in[idx];
+                    val[i] = iota_vals ? idx : vals_in[idx];
+                    dig[i] = (key[i] >> shift) & mask;
+                } else {
+                    key[i] = 0; val[i] = 0;
+                    dig[i] = kRadix;  // sentinel: not counted
+                }
             }
         }
-        // Warp-level ranking of each item among equal digits.
+        // Warp-level ranking of each item among equal digits: the peer masks
+        // first (independent ballots), then the per-digit counters in order.
+        uint32_t peer[kSortItems];
+#pragma unroll
+        for (int i = 0; i < kSortItems; i++) peer[i] = digit_peers(dig[i], bits);
 #pragma unroll
         for (int i = 0; i < kSortItems; i++) {
             const uint32_t d = dig[i];
-            const uint32_t peers = __match_any_sync(0xffffffffu, d);
+            const uint32_t peers = peer[i];
             const int leader = __ffs(peers) - 1;
             uint32_t b = 0;
             if (d < kRadix) b = s_warp_hist[warp][d];
@@ -223,7 +261,8 @@ k_onesweep(const uint32_t *__restrict__ keys_in, const uint32_t *__restrict__ va
         }
         __syncthreads();
 
-        // Per digit (thread = digit): warp offsets and the block's count.
+        // Per digit (thread = digit): warp offsets, the block's count, and
+        // where the digit's run starts in the partition's local order.
         uint32_t block_count = 0;
         {
             const int d = tid;
@@ -232,6 +271,20 @@ k_onesweep(const uint32_t *__restrict__ keys_in, const uint32_t *__restrict__ va
                 const uint32_t c = s_warp_hist[w][d];
                 s_warp_hist[w][d] = block_count;
                 block_count += c;
+            }
+            uint32_t tot;
+            s_digit_start[d] = block_exclusive_scan_256(d < radix ? block_count : 0u, s_scan, &tot);
+        }
+        __syncthreads();
+        // Local reorder through shared memory first, so the look-back below
+        // runs with the keys out of registers.
+#pragma unroll
+        for (int i = 0; i < kSortItems; i++) {
+            const uint32_t d = dig[i];
+            if (d < kRadix) {
+                const uint32_t loc = s_digit_start[d] + s_warp_hist[warp][d] + rank[i];
+                s_keys[loc] = key[i];
+                s_vals[loc] = val[i];
             }
         }
         // Publish this partition's count for the digit, then look back.
@@ -249,22 +302,8 @@ k_onesweep(const uint32_t *__restrict__ keys_in, const uint32_t *__restrict__ va
                 }
             }
             s_global_base[d] = s_hist_excl[d] + excl;
-            uint32_t tot;
-            s_digit_start[d] = block_exclusive_scan_256(d < radix ? block_count : 0u, s_scan, &tot);
         }
-        __syncthreads();
-
-        // Local reorder through shared memory, then coalesced-run stores.
-        uint32_t valid_count = 0;
-#pragma unroll
-        for (int i = 0; i < kSortItems; i++) {
-            const uint32_t d = dig[i];
-            if (d < kRadix) {
-                const uint32_t loc = s_digit_start[d] + s_warp_hist[warp][d] + rank[i];
-                s_keys[loc] = key[i];
-                s_vals[loc] = val[i];
-            }
-        }
+        uint32_t valid_count;
         {
             const uint64_t rem = (uint64_t)n - (uint64_t)p * kSortPart;
             valid_count = rem < (uint64_t)kSortPart ? (uint32_t)rem : (uint32_t)kSortPart;
