@@ -39,6 +39,10 @@
  *     A pixel is considered by a splat only if its tile is inside this
  *     rectangle: this is the tiled method's cutoff, applied to the naive
  *     render so that both compute the same function.
+ *   - optional opacity-aware tile cut ([GSP] s4, gsplat's extent of
+ *     sqrt(2 ln(255 o)) standard deviations), taken per tile column and row
+ *     against pixel centres so that it only removes tiles in which no pixel
+ *     can pass the alpha >= 1/255 test (see opacity_cut)
  *   - colour parameter used directly as RGB (SH degree 0, no offset)
  *   - a Gaussian is culled (no tiles, exactly zero gradient) if its camera
  *     z <= near_z, or if any projected value is not finite       [GSP] s6
@@ -60,6 +64,7 @@ typedef struct {
     int32_t width, height;
     double near_z;
     double bg[3];
+    int32_t tight_tiles;  /* 1: narrow each tile rectangle by the opacity-aware cut */
 } orc_camera;
 
 /* Single-precision decision constants, as the [GSP] s5 listing writes them. */
@@ -256,16 +261,84 @@ static void project_one(const double *mean, const double *log_scale, const doubl
                isfinite(P->opacity);
 }
 
+static double dist_to_int(double v) { return fabs(v - nearbyint(v)); }
+
+/* Slack of the opacity-aware cut, in ln(alpha): a tile is cut only where
+ * every pixel has alpha below e^-0.01 / 255 (1 % under the threshold). */
+#define ORC_CUT_SLACK    0.01
+/* Largest A C / (A C - B^2) at which the cut is taken. */
+#define ORC_CUT_MAX_COND 1024.0
+
+/* Opacity-aware tile cut ([GSP] s4: gsplat shrinks a splat's extent to where
+ * it fades below 1/255, sqrt(2 ln(255 o)) standard deviations).  Taken per
+ * tile column and row against pixel centres:
+ *   on the vertical line at horizontal offset dx from the mean, sigma is
+ *   smallest at dy = -B dx / C, where it is dx^2 (A C - B^2) / (2 C); so every
+ *   pixel of a tile column whose nearest centre is farther than
+ *   D_x = sqrt(2 ell C / (A C - B^2)), ell = ln(255 o) + slack, from mx has
+ *   alpha < e^-slack / 255 and fails the 1/255 test.  Rows likewise with
+ *   D_y = sqrt(2 ell A / (A C - B^2)).
+ * Column tx holds centres 16 tx + 0.5 ... 16 tx + 15.5, so it is kept iff
+ *   16 tx + 0.5 <= mx + D_x and 16 tx + 15.5 >= mx - D_x,
+ * i.e. tx in [ceil((mx - D_x - 15.5)/16), floor((mx + D_x - 0.5)/16)].
+ * ell <= 0 (o <= e^-slack / 255): no pixel can pass, nothing is kept.
+ * Not taken (all four bounds infinite) when A C - B^2 <= 0 or
+ * A C > 1024 (A C - B^2): there the rounding of a single-precision sigma
+ * near the threshold can exceed the slack.
+ * Writes cut = {lo x, hi x, lo y, hi y} (tiles, integral or infinite).
+ * Returns the smallest distance of its decisions from flipping, each
+ * relative to its own scale: |cond / 1024 - 1|, |ell|, and for each of the
+ * four bounds the distance in pixels of (m -+ D - ...)/16 from an integer
+ * divided by (1 + D). */
+static double opacity_cut(double mx, double my, double A, double B, double C, double o,
+                          double cut[4])
+{
+    cut[0] = cut[2] = -INFINITY;
+    cut[1] = cut[3] = INFINITY;
+    double q = A * C - B * B;
+    if (!(q > 0.0)) return INFINITY;
+    double cond = A * C / q;
+    double margin = fabs(cond / ORC_CUT_MAX_COND - 1.0);
+    if (!(cond <= ORC_CUT_MAX_COND)) return margin;
+    double ell = log(255.0 * o) + ORC_CUT_SLACK;
+    if (fabs(ell) < margin) margin = fabs(ell);
+    if (ell <= 0.0) {
+        cut[0] = cut[2] = INFINITY;
+        cut[1] = cut[3] = -INFINITY;
+        return margin;
+    }
+    const double D[2] = {sqrt(2.0 * ell * C / q), sqrt(2.0 * ell * A / q)};
+    const double m[2] = {mx, my};
+    for (int axis = 0; axis < 2; axis++) {
+        double lo = (m[axis] - D[axis] - (ORC_TILE - 0.5)) / ORC_TILE;
+        double hi = (m[axis] + D[axis] - 0.5) / ORC_TILE;
+        cut[2 * axis] = ceil(lo);
+        cut[2 * axis + 1] = floor(hi);
+        double d0 = ORC_TILE * dist_to_int(lo) / (1.0 + D[axis]);
+        double d1 = ORC_TILE * dist_to_int(hi) / (1.0 + D[axis]);
+        if (d0 < margin) margin = d0;
+        if (d1 < margin) margin = d1;
+    }
+    return margin;
+}
+
 /* Tile rectangle of a splat, in float (a pixel grid decision taken in single
- * precision).  Returns the tile count; writes x0, y0, x1, y1 (inclusive),
- * with x0 > x1 or y0 > y1 when nothing is touched. */
+ * precision).  With cut (from opacity_cut) the bounds are narrowed to it
+ * before clamping.  Returns the tile count; writes x0, y0, x1, y1
+ * (inclusive), with x0 > x1 or y0 > y1 when nothing is touched. */
 static int32_t tile_rect_f32(float mx, float my, float r, int32_t tiles_x, int32_t tiles_y,
-                             int32_t *rect)
+                             const double *cut, int32_t *rect)
 {
     float lx = floorf((mx - r) * (1.0f / ORC_TILE));
     float hx = floorf((mx + r) * (1.0f / ORC_TILE));
     float ly = floorf((my - r) * (1.0f / ORC_TILE));
     float hy = floorf((my + r) * (1.0f / ORC_TILE));
+    if (cut) {
+        lx = fmaxf(lx, (float)cut[0]);
+        hx = fminf(hx, (float)cut[1]);
+        ly = fmaxf(ly, (float)cut[2]);
+        hy = fminf(hy, (float)cut[3]);
+    }
     lx = fminf(fmaxf(lx, 0.0f), (float)tiles_x);
     ly = fminf(fmaxf(ly, 0.0f), (float)tiles_y);
     hx = fmaxf(fminf(hx, (float)(tiles_x - 1)), -1.0f);
@@ -278,7 +351,6 @@ static int32_t tile_rect_f32(float mx, float my, float r, int32_t tiles_x, int32
     return (rect[2] - rect[0] + 1) * (rect[3] - rect[1] + 1);
 }
 
-static double dist_to_int(double v) { return fabs(v - nearbyint(v)); }
 
 /* Projection of n Gaussians ([GSP] s1-s4, s6).  Outputs, per Gaussian:
  *   mean2d[2], conic[3] (A, B, C), cov2d[3] (dilated a, b, c), opacity,
@@ -286,13 +358,14 @@ static double dist_to_int(double v) { return fabs(v - nearbyint(v)); }
  *   rect[4] (tile x0, y0, x1, y1), count (tiles touched), valid (0/1),
  *   radius_margin (|3 sqrt(lambda) - nearest integer|, px),
  *   rect_margin (min over the four rectangle edges of |(m +- r)/16 - nearest
- *   integer|, in tiles).  The margins say how close an integer decision came
- *   to flipping.  Returns 0, or -1 on bad arguments. */
+ *   integer|, in tiles), cut_margin (what opacity_cut returns when
+ *   cam->tight_tiles is set, else infinity).  The margins say how close an
+ *   integer decision came to flipping.  Returns 0, or -1 on bad arguments. */
 int orc_project(int64_t n, const double *means, const double *log_scales, const double *quats,
                 const double *opacity_logits, const double *colors, const orc_camera *cam,
                 double *mean2d, double *conic, double *cov2d, double *opacity, double *depth,
                 double *color, float *radius, int32_t *rect, int32_t *count, uint8_t *valid,
-                double *radius_margin, double *rect_margin)
+                double *radius_margin, double *rect_margin, double *cut_margin)
 {
     if (n < 0 || cam->width <= 0 || cam->height <= 0) return -1;
     int32_t tiles_x = (cam->width + ORC_TILE - 1) / ORC_TILE;
@@ -313,6 +386,7 @@ int orc_project(int64_t n, const double *means, const double *log_scales, const 
             count[g] = 0;
             radius_margin[g] = INFINITY;
             rect_margin[g] = INFINITY;
+            cut_margin[g] = INFINITY;
             continue;
         }
         mean2d[2 * g] = P.mean2d[0];
@@ -325,8 +399,13 @@ int orc_project(int64_t n, const double *means, const double *log_scales, const 
         float r = ceilf((float)P.radius_value);
         radius[g] = r;
         radius_margin[g] = dist_to_int(P.radius_value);
+        double cut[4];
+        cut_margin[g] = INFINITY;
+        if (cam->tight_tiles)
+            cut_margin[g] = opacity_cut(P.mean2d[0], P.mean2d[1], P.conic[0], P.conic[1],
+                                        P.conic[2], P.opacity, cut);
         count[g] = tile_rect_f32((float)P.mean2d[0], (float)P.mean2d[1], r, tiles_x, tiles_y,
-                                 rect + 4 * g);
+                                 cam->tight_tiles ? cut : NULL, rect + 4 * g);
         double m = INFINITY;
         for (int axis = 0; axis < 2; axis++) {
             double e0 = (P.mean2d[axis] - (double)r) / ORC_TILE;
@@ -340,10 +419,13 @@ int orc_project(int64_t n, const double *means, const double *log_scales, const 
     return 0;
 }
 
-/* Rectangle rule alone, for callers that already hold float mean2d and radius
- * (used to bin records that are given in single precision). */
-int orc_tile_rects(int64_t n, const float *mean2d, const float *radius, const uint8_t *valid,
-                   int32_t width, int32_t height, int32_t *rect, int32_t *count)
+/* Rectangle rule alone, for callers that already hold float records (used
+ * to bin records that are given in single precision).  conic [n][3] and
+ * opacity [n] are read only when tight_tiles is set; the cut is then taken
+ * on their values as given. */
+int orc_tile_rects(int64_t n, const float *mean2d, const float *radius, const float *conic,
+                   const float *opacity, const uint8_t *valid, int32_t width, int32_t height,
+                   int32_t tight_tiles, int32_t *rect, int32_t *count)
 {
     if (n < 0 || width <= 0 || height <= 0) return -1;
     int32_t tiles_x = (width + ORC_TILE - 1) / ORC_TILE;
@@ -354,8 +436,12 @@ int orc_tile_rects(int64_t n, const float *mean2d, const float *radius, const ui
             count[g] = 0;
             continue;
         }
+        double cut[4];
+        if (tight_tiles)
+            (void)opacity_cut(mean2d[2 * g], mean2d[2 * g + 1], conic[3 * g], conic[3 * g + 1],
+                              conic[3 * g + 2], opacity[g], cut);
         count[g] = tile_rect_f32(mean2d[2 * g], mean2d[2 * g + 1], radius[g], tiles_x, tiles_y,
-                                 rect + 4 * g);
+                                 tight_tiles ? cut : NULL, rect + 4 * g);
     }
     return 0;
 }

@@ -22,12 +22,15 @@ import numpy as np
 from . import build as _build
 
 __all__ = [
-    "TILE", "OrcCamera", "lib", "quat_to_rotmat", "covariance3d", "project_debug", "project", "tile_rects",
+    "TILE", "TIGHT_TILES", "OrcCamera", "lib", "quat_to_rotmat", "covariance3d", "project_debug", "project", "tile_rects",
     "records_f32", "bin_pairs", "depth_order", "render", "render_bwd", "project_bwd",
     "grad_bound", "default_threads",
 ]
 
 TILE = 16
+# Camera flag bit that selects the opacity-aware tile cut (the value the
+# library's camera struct uses for the same option).
+TIGHT_TILES = 1
 
 _c_double_p = ctypes.POINTER(ctypes.c_double)
 _c_float_p = ctypes.POINTER(ctypes.c_float)
@@ -46,6 +49,7 @@ class OrcCamera(ctypes.Structure):
         ("width", ctypes.c_int32), ("height", ctypes.c_int32),
         ("near_z", ctypes.c_double),
         ("bg", ctypes.c_double * 3),
+        ("tight_tiles", ctypes.c_int32),
     ]
 
 
@@ -61,10 +65,12 @@ def lib() -> ctypes.CDLL:
         L.orc_quat_to_rotmat.argtypes = [_c_double_p, _c_double_p]
         L.orc_covariance3d.argtypes = [_c_double_p, _c_double_p, _c_double_p]
         L.orc_project.argtypes = [ctypes.c_int64] + [_c_double_p] * 5 + [ctypes.POINTER(OrcCamera)] + \
-            [_c_double_p] * 6 + [_c_float_p, _c_int32_p, _c_int32_p, _c_uint8_p, _c_double_p, _c_double_p]
+            [_c_double_p] * 6 + [_c_float_p, _c_int32_p, _c_int32_p, _c_uint8_p, _c_double_p, _c_double_p,
+                                 _c_double_p]
         L.orc_project.restype = ctypes.c_int
-        L.orc_tile_rects.argtypes = [ctypes.c_int64, _c_float_p, _c_float_p, _c_uint8_p,
-                                     ctypes.c_int32, ctypes.c_int32, _c_int32_p, _c_int32_p]
+        L.orc_tile_rects.argtypes = [ctypes.c_int64, _c_float_p, _c_float_p, _c_float_p, _c_float_p,
+                                     _c_uint8_p, ctypes.c_int32, ctypes.c_int32, ctypes.c_int32,
+                                     _c_int32_p, _c_int32_p]
         L.orc_bin.argtypes = [ctypes.c_int64, _c_int32_p, _c_uint8_p, _c_float_p, ctypes.c_int32,
                               ctypes.c_int32, ctypes.c_int64, _c_int32_p, _c_uint64_p, _c_uint32_p,
                               _c_uint32_p]
@@ -110,6 +116,7 @@ def _cam(cam) -> OrcCamera:
     bg = np.asarray(cam.bg, dtype=np.float64).reshape(3)
     for k in range(3):
         c.bg[k] = float(bg[k])
+    c.tight_tiles = 1 if int(getattr(cam, "flags", 0)) & TIGHT_TILES else 0
     return c
 
 
@@ -159,7 +166,7 @@ def project(params: dict, cam) -> dict:
         "opacity": np.zeros(n), "depth": np.zeros(n), "color": np.zeros((n, 3)),
         "radius": np.zeros(n, dtype=np.float32), "rect": np.zeros((n, 4), dtype=np.int32),
         "count": np.zeros(n, dtype=np.int32), "valid": np.zeros(n, dtype=np.uint8),
-        "radius_margin": np.zeros(n), "rect_margin": np.zeros(n),
+        "radius_margin": np.zeros(n), "rect_margin": np.zeros(n), "cut_margin": np.zeros(n),
     }
     c = _cam(cam)
     rc = lib().orc_project(
@@ -170,37 +177,47 @@ def project(params: dict, cam) -> dict:
         _ptr(out["depth"], _c_double_p), _ptr(out["color"], _c_double_p),
         _ptr(out["radius"], _c_float_p), _ptr(out["rect"], _c_int32_p),
         _ptr(out["count"], _c_int32_p), _ptr(out["valid"], _c_uint8_p),
-        _ptr(out["radius_margin"], _c_double_p), _ptr(out["rect_margin"], _c_double_p))
+        _ptr(out["radius_margin"], _c_double_p), _ptr(out["rect_margin"], _c_double_p),
+        _ptr(out["cut_margin"], _c_double_p))
     if rc != 0:
         raise ValueError("orc_project: bad arguments")
     out["depth32"] = out["depth"].astype(np.float32)
     return out
 
 
-def tile_rects(mean2d32, radius32, valid, width: int, height: int):
-    """The tile-rectangle rule alone, on single-precision mean2d and radius."""
+def tile_rects(mean2d32, radius32, valid, width: int, height: int, conic32=None, opacity32=None,
+               tight: bool = False):
+    """The tile-rectangle rule alone, on single-precision records; with
+    ``tight`` the opacity-aware cut is taken on conic32 and opacity32."""
     m = np.ascontiguousarray(mean2d32, dtype=np.float32).reshape(-1, 2)
     n = m.shape[0]
     r = np.ascontiguousarray(radius32, dtype=np.float32).reshape(n)
     v = np.ascontiguousarray(valid, dtype=np.uint8).reshape(n)
+    cn = np.ascontiguousarray(np.zeros((n, 3)) if conic32 is None else conic32, dtype=np.float32).reshape(n, 3)
+    op = np.ascontiguousarray(np.zeros(n) if opacity32 is None else opacity32, dtype=np.float32).reshape(n)
+    if tight and (conic32 is None or opacity32 is None):
+        raise ValueError("tile_rects: the opacity-aware cut needs conic32 and opacity32")
     rect = np.zeros((n, 4), dtype=np.int32)
     count = np.zeros(n, dtype=np.int32)
-    lib().orc_tile_rects(n, _ptr(m, _c_float_p), _ptr(r, _c_float_p), _ptr(v, _c_uint8_p),
-                         int(width), int(height), _ptr(rect, _c_int32_p), _ptr(count, _c_int32_p))
+    lib().orc_tile_rects(n, _ptr(m, _c_float_p), _ptr(r, _c_float_p), _ptr(cn, _c_float_p),
+                         _ptr(op, _c_float_p), _ptr(v, _c_uint8_p), int(width), int(height),
+                         1 if tight else 0, _ptr(rect, _c_int32_p), _ptr(count, _c_int32_p))
     return rect, count
 
 
-def records_f32(proj: dict, width: int, height: int) -> dict:
+def records_f32(proj: dict, width: int, height: int, tight: bool = False) -> dict:
     """Rounds projected records once to single precision (the precision the
     CUDA path stores them in) and re-derives the rectangles from the rounded
-    mean2d and radius.  Rendering these records in double with ``render``
-    isolates the blend from the projection."""
+    mean2d and radius (and, with ``tight``, the opacity-aware cut from the
+    rounded conic and opacity).  Rendering these records in double with
+    ``render`` isolates the blend from the projection."""
     out = dict(proj)
     for k in ("mean2d", "conic", "opacity", "color", "depth"):
         out[k] = np.asarray(proj[k], dtype=np.float32).astype(np.float64)
     out["depth32"] = np.asarray(proj["depth"], dtype=np.float32)
     rect, count = tile_rects(out["mean2d"].astype(np.float32), proj["radius"], proj["valid"],
-                             width, height)
+                             width, height, out["conic"].astype(np.float32),
+                             out["opacity"].astype(np.float32), tight)
     out["rect"], out["count"] = rect, count
     return out
 

@@ -30,7 +30,8 @@ class Camera:
     """Pinhole camera.  ``viewmat`` is the row-major 4x4 world-to-camera
     matrix [R | t; 0 0 0 1] in OpenCV axes (+x right, +y down, +z forward);
     fx, fy, cx, cy are in pixels; pixel (row i, col j) is sampled at
-    (j + 0.5, i + 0.5).  All values are single precision."""
+    (j + 0.5, i + 0.5).  All values are single precision.  ``flags`` holds
+    option bits of the renderer (bit 0: the opacity-aware tile cut)."""
     viewmat: np.ndarray
     fx: float
     fy: float
@@ -40,6 +41,7 @@ class Camera:
     height: int
     near_z: float = 0.01
     bg: tuple = (0.0, 0.0, 0.0)
+    flags: int = 0
 
     def __post_init__(self):
         self.viewmat = np.asarray(self.viewmat, dtype=np.float32).reshape(4, 4)
@@ -47,6 +49,7 @@ class Camera:
             float(np.float32(v)) for v in (self.fx, self.fy, self.cx, self.cy, self.near_z))
         self.bg = tuple(float(np.float32(v)) for v in self.bg)
         self.width, self.height = int(self.width), int(self.height)
+        self.flags = int(self.flags)
 
     @property
     def tiles_x(self) -> int:

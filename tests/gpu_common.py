@@ -33,6 +33,7 @@ MARGIN_T = 1e-3       # relative margin of T (1 - alpha) against 1e-4
 MARGIN_CLAMP = 1e-4   # relative margin of o G against the 0.99 cap
 MARGIN_TILE = 1e-4    # tiles, distance of (m -+ r)/16 to an integer
 MARGIN_RADIUS = 2e-4  # px, distance of 3 sqrt(lambda) to an integer
+MARGIN_CUT = 1e-3     # relative distance of an opacity-cut decision from flipping
 
 
 def cuda_params(params: dict) -> dict:
@@ -64,7 +65,7 @@ def fill_projected(rec: dict, n: int) -> G.Projected:
 def oracle_records(params: dict, cam) -> dict:
     """Oracle projection rounded once to fp32 (the stage-fed input)."""
     p = O.project(params, cam)
-    r = O.records_f32(p, cam.width, cam.height)
+    r = O.records_f32(p, cam.width, cam.height, tight=bool(cam.flags & O.TIGHT_TILES))
     return r
 
 
@@ -95,11 +96,12 @@ def ambiguous_pixels(orc_fwd: dict, with_clamp: bool = False) -> np.ndarray:
 
 def ambiguous_gaussians(p: dict) -> np.ndarray:
     """Gaussians whose binning may differ between an fp32 and an fp64
-    projection: radius ceiling or a rectangle edge within the stated margin
-    of an integer, or a depth within 4 float ulps of another drawable
+    projection: radius ceiling, a rectangle edge or an opacity-cut decision
+    within the stated margin of flipping, or a depth within 4 float ulps of another drawable
     Gaussian's (their order may swap)."""
     v = p["valid"].astype(bool)
-    bad = v & ((p["radius_margin"] < MARGIN_RADIUS) | (p["rect_margin"] < MARGIN_TILE))
+    bad = v & ((p["radius_margin"] < MARGIN_RADIUS) | (p["rect_margin"] < MARGIN_TILE) |
+               (p["cut_margin"] < MARGIN_CUT))
     d = p["depth"]
     idx = np.nonzero(v & (p["count"] > 0))[0]
     if idx.size > 1:

@@ -14,7 +14,7 @@ import gaussian_splatting_differentiable_tile_b200 as G
 import oracle as O
 from scenes import Camera, make_cameras, make_scene, make_target, tiny_camera
 
-from gpu_common import (IMG_TOL, MARGIN_RADIUS, MARGIN_TILE, ambiguous_gaussians, ambiguous_pixels,
+from gpu_common import (IMG_TOL, MARGIN_CUT, MARGIN_RADIUS, MARGIN_TILE, ambiguous_gaussians, ambiguous_pixels,
                         cuda_params, fill_projected, gpu_bin, gpu_render, grad_compare, oracle_records,
                         tiles_to_pixels)
 
@@ -62,7 +62,8 @@ def test_project_matches_oracle(scene):
     assert np.all(np.abs(conr[v, :3] - p["conic"][v]) <= 1e-4 * scale + 1e-9)
     # integer decisions: equal unless the oracle says the decision was within
     # its stated margin of flipping
-    amb = v & ((p["radius_margin"] < MARGIN_RADIUS) | (p["rect_margin"] < MARGIN_TILE))
+    amb = v & ((p["radius_margin"] < MARGIN_RADIUS) | (p["rect_margin"] < MARGIN_TILE) |
+               (p["cut_margin"] < MARGIN_CUT))
     diff_r = conr[:, 3] != p["radius"]
     diff_rect = np.any(rect != p["rect"], axis=1) | (count != p["count"])
     assert not np.any(diff_r & ~amb), np.nonzero(diff_r & ~amb)[0][:10]
