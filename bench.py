@@ -43,6 +43,8 @@ sys.path.insert(0, ROOT)
 
 from scenes import SPECS, make_cameras, make_scene, make_target  # noqa: E402
 
+TIGHT_TILES = 1  # gs_camera.flags bit of the opacity-aware tile cut (GS_FLAG_TIGHT_TILES)
+
 DEFAULT_WORKLOAD = "train400k_half"
 METRIC = "fwd and fwd+bwd frames/s at 400k Gaussians, 980x545; tile-pairs/s; % roofline"
 
@@ -184,11 +186,18 @@ def cpu_frame_time(params_np, cam, sample_tiles: int, seed: int = 0) -> dict:
             "threads": O.default_threads()}
 
 
+def _cameras(spec, args):
+    cams = make_cameras(spec)
+    for c in cams:
+        c.flags = TIGHT_TILES if args.tiles == "cut" else 0
+    return cams
+
+
 def run_reference(args, spec, rank, world):
     if rank != 0:
         return
     params = make_scene(spec)
-    cams = make_cameras(spec)
+    cams = _cameras(spec, args)
     for i in range(args.warmup):
         cpu_frame_time(params, cams[i % len(cams)], args.ref_sample_tiles, seed=i)
     times = []
@@ -203,16 +212,18 @@ def run_reference(args, spec, rank, world):
     out = {"impl": "reference", "metric": METRIC, "value": fps, "unit": "frames/s", "n_gpus": world,
            "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1000.0 * statistics.mean(times),
            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
-           "data": "synthetic", "config": _config(spec, None, False),
+           "data": "synthetic", "config": _config(spec, None, args.tiles, False),
            "cpu_baseline": {"value": fps, "unit": "frames/s", "cores": info["threads"], "kind": "oracle",
                             "sample": sample},
            "e2e": {"value": fps, "unit": "frames/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
     print(json.dumps(out), flush=True)
 
 
-def _config(spec, pairs, graphs=True):
+def _config(spec, pairs, tiles, graphs=True):
     return {"workload": spec.name, "n_gaussians": spec.n, "width": spec.width, "height": spec.height,
             "focal": spec.focal, "cameras": f"{spec.n_cameras} {spec.cameras}", "pairs_per_frame": pairs,
+            "tiles": ("3-sigma rectangle narrowed by the opacity-aware cut (same image)" if tiles == "cut"
+                      else "3-sigma rectangle"),
             "l2": "flushed between timed steps (256 MB write outside the timed events)",
             "launch": "one CUDA graph per camera, replayed" if graphs else "eager launches",
             "parallelism": "replicas (cameras split across ranks)"}
@@ -228,7 +239,7 @@ def run_native(args, spec, rank, world, local):
     torch.cuda.set_device(local)
     dev = torch.device("cuda", local)
     params_np = make_scene(spec)
-    cams = make_cameras(spec)
+    cams = _cameras(spec, args)
     mine = [c for i, c in enumerate(cams) if i % world == rank] or cams[:1]
     n = spec.n
     P = {k: torch.from_numpy(v).to(dev) for k, v in params_np.items()}
@@ -416,7 +427,7 @@ def run_native(args, spec, rank, world, local):
         "vs_baseline": None,
         "dtype": "f32",
         "data": "synthetic",
-        "config": _config(spec, int(mean_pairs), not args.no_graphs),
+        "config": _config(spec, int(mean_pairs), args.tiles, not args.no_graphs),
         "fwd_frames_per_s": frames / (fwd_ms * 1e-3),
         "fwd_ms_per_frame": fwd_ms / args.steps,
         "tile_pairs_per_s": mean_pairs * frames / (fwd_ms * 1e-3),
@@ -443,6 +454,8 @@ def main():
     ap.add_argument("--ref-sample-tiles", type=int, default=8)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-graphs", action="store_true", help="launch every kernel eagerly")
+    ap.add_argument("--tiles", choices=("cut", "3sigma"), default="cut",
+                    help="tile rectangles: 3-sigma narrowed by the opacity-aware cut, or plain 3-sigma")
     args = ap.parse_args()
     rank = int(os.environ.get("RANK", 0))
     world = int(os.environ.get("WORLD_SIZE", 1))

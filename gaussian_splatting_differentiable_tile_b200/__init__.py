@@ -25,7 +25,7 @@ import torch
 
 from . import _abi
 from ._abi import (GS_ERR_ALIGNMENT, GS_ERR_CAPACITY, GS_ERR_CUDA, GS_ERR_DEVICE_TIMEOUT,  # noqa: F401
-                   GS_ERR_INVALID_ARG, GS_ERR_TOO_LARGE, GS_OK, GS_TILE)
+                   GS_ERR_INVALID_ARG, GS_ERR_TOO_LARGE, GS_FLAG_TIGHT_TILES, GS_OK, GS_TILE)
 
 __all__ = [
     "GSError", "Projected", "Bins", "make_camera", "gs_project", "gs_bin_and_sort",
@@ -87,6 +87,7 @@ def make_camera(cam) -> _abi.GsCamera:
     c.near_z = float(cam.near_z)
     for k in range(3):
         c.bg[k] = float(cam.bg[k])
+    c.flags = int(getattr(cam, "flags", 0))
     return c
 
 

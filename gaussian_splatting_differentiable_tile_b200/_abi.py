@@ -20,6 +20,7 @@ GS_ERR_TOO_LARGE = -3
 GS_ERR_ALIGNMENT = -4
 GS_ERR_CUDA = -5
 GS_ERR_DEVICE_TIMEOUT = -6
+GS_FLAG_TIGHT_TILES = 1
 
 c_float_p = ctypes.c_void_p  # device pointers travel as plain addresses
 
@@ -31,6 +32,7 @@ class GsCamera(ctypes.Structure):
         ("width", ctypes.c_int32), ("height", ctypes.c_int32),
         ("near_z", ctypes.c_float),
         ("bg", ctypes.c_float * 3),
+        ("flags", ctypes.c_uint32),
     ]
 
 

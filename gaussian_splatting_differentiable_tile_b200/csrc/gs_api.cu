@@ -30,6 +30,7 @@ int make_cam(const gs_camera *cam, CamConst *out) {
         if (!std::isfinite(cam->viewmat[k])) return GS_ERR_INVALID_ARG;
     for (int k = 0; k < 3; k++)
         if (!std::isfinite(cam->bg[k])) return GS_ERR_INVALID_ARG;
+    if (cam->flags & ~GS_FLAG_TIGHT_TILES) return GS_ERR_INVALID_ARG;
     CamConst c{};
     for (int i = 0; i < 3; i++) {
         for (int j = 0; j < 3; j++) c.R[3 * i + j] = cam->viewmat[4 * i + j];
@@ -49,6 +50,7 @@ int make_cam(const gs_camera *cam, CamConst *out) {
     c.height = cam->height;
     c.tiles_x = (cam->width + kTile - 1) / kTile;
     c.tiles_y = (cam->height + kTile - 1) / kTile;
+    c.flags = cam->flags;
     *out = c;
     return GS_OK;
 }

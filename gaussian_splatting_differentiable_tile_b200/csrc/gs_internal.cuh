@@ -55,6 +55,7 @@ struct CamConst {
     float near_z;
     float bg[3];
     int32_t width, height, tiles_x, tiles_y;
+    uint32_t flags;     // GS_FLAG_* of the camera
 };
 
 // Byte layout of a gs_bins buffer.  The first `zero_bytes` bytes are cleared

@@ -16,6 +16,12 @@ constexpr float kEps2d = 0.3f;        // [GSP] s4 low-pass dilation, px^2
 constexpr float kDetMin = 1e-10f;     // [GSP] s3 det clamp
 constexpr float kLambdaFloor = 0.1f;  // [GSP] s4 floor under the root
 constexpr float kRadiusSigmas = 3.f;  // [GSP] s4 3DGS radius rule
+// Opacity-aware tile cut: slack in ln(alpha) (cut tiles stay below
+// e^-0.01 / 255) and the largest conic condition A C / (A C - B^2) it is
+// taken at (beyond it single-precision sigma near the threshold can stray
+// by more than the slack).
+constexpr float kCutSlack = 0.01f;
+constexpr float kCutMaxCond = 1024.f;
 
 // Everything the forward computes for one Gaussian; the backward re-derives
 // it from the raw parameters instead of storing it.
@@ -146,11 +152,39 @@ k_project(CamConst cam, int n, const float *__restrict__ means, const float *__r
     const float r = ceilf(kRadiusSigmas * sqrtf(P.lambda));
     xyod[g] = make_float4(P.mx, P.my, P.opacity, P.t[2]);
     conr[g] = make_float4(P.A, P.B, P.C, r);
-    // Tile rectangle: floor((m -+ r) / 16) per axis, clamped to the grid in
-    // float before any integer conversion.
+    // Tile rectangle: floor((m -+ r) / 16) per axis, optionally narrowed by
+    // the opacity-aware cut, clamped to the grid in float before any integer
+    // conversion.
     const float inv_tile = 1.f / kTile;
     float lx = floorf((P.mx - r) * inv_tile), hx = floorf((P.mx + r) * inv_tile);
     float ly = floorf((P.my - r) * inv_tile), hy = floorf((P.my + r) * inv_tile);
+    if (cam.flags & GS_FLAG_TIGHT_TILES) {
+        // Opacity-aware cut ([GSP] s4, gsplat's sqrt(2 ln(255 o)) extent),
+        // per pixel-centre column and row.  On the column at horizontal
+        // offset dx from the mean, sigma is smallest at dy = -B dx / C, where
+        // it is dx^2 q / (2 C), q = A C - B^2: columns whose nearest centre is
+        // farther than D_x = sqrt(2 ell C / q), ell = ln(255 o) + slack, hold
+        // no pixel that passes alpha >= 1/255.  Column tx (centres 16 tx + 0.5
+        // ... 16 tx + 15.5) is kept iff tx lies in
+        // [ceil((mx - D_x - 15.5) / 16), floor((mx + D_x - 0.5) / 16)].
+        const float q = P.A * P.C - P.B * P.B;
+        if (q > 0.f && P.A * P.C <= kCutMaxCond * q) {
+            const float ell = logf(255.f * P.opacity) + kCutSlack;
+            if (ell <= 0.f) {  // o too small for any pixel to pass
+                lx = (float)cam.tiles_x;
+                hx = -1.f;
+                ly = (float)cam.tiles_y;
+                hy = -1.f;
+            } else {
+                const float s2 = 2.f * ell / q;
+                const float dx = sqrtf(s2 * P.C), dy = sqrtf(s2 * P.A);
+                lx = fmaxf(lx, ceilf((P.mx - dx - 15.5f) * inv_tile));
+                hx = fminf(hx, floorf((P.mx + dx - 0.5f) * inv_tile));
+                ly = fmaxf(ly, ceilf((P.my - dy - 15.5f) * inv_tile));
+                hy = fminf(hy, floorf((P.my + dy - 0.5f) * inv_tile));
+            }
+        }
+    }
     lx = fminf(fmaxf(lx, 0.f), (float)cam.tiles_x);
     ly = fminf(fmaxf(ly, 0.f), (float)cam.tiles_y);
     hx = fmaxf(fminf(hx, (float)(cam.tiles_x - 1)), -1.f);

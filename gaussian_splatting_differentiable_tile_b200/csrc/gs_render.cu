@@ -80,8 +80,14 @@ __device__ __forceinline__ void stage_entry(const float4 xyod, const float4 conr
     const float cA = (-0.5f * kLog2e) * conr.x;
     const float cB = -kLog2e * conr.y;
     const float cC = (-0.5f * kLog2e) * conr.z;
-    const float kx = cA - cB * cB / (4.f * cC);
-    const float ky = cC - cB * cB / (4.f * cA);
+    // Separable bound of the exponent: max over dy of the quadratic at fixed
+    // dx is kx dx^2, and likewise ky dy^2.  Not used (zero) for conics with
+    // condition A C / (A C - B^2) above 1024, where single-precision rounding
+    // of the exponent near the alpha threshold can exceed the cull margin.
+    const float acx4 = 4.f * cA * cC, det4 = acx4 - cB * cB;  // log2(e)^2 (A C - B^2)
+    const bool bounded = det4 > 0.f && acx4 <= 1024.f * det4;
+    const float kx = bounded ? cA - cB * cB / (4.f * cC) : 0.f;
+    const float ky = bounded ? cC - cB * cB / (4.f * cA) : 0.f;
     geo = make_float4(xyod.x, xyod.y, cA, cB);
     geo2 = make_float4(cC, log2f(xyod.z), kx, ky);
 }

@@ -72,7 +72,26 @@ typedef struct gs_camera {
                              [GSP] s6) */
     float bg[3];          /* background colour, weighted by the final
                              transmittance ([GSP] s5) */
+    uint32_t flags;       /* GS_FLAG_* bits; 0 = the pages' plain method.
+                             Unknown bits are rejected (GS_ERR_INVALID_ARG). */
 } gs_camera;
+
+/* gs_camera.flags: opacity-aware tile cut ([GSP] s4, gsplat's extent of
+ * sqrt(2 ln(255 o)) standard deviations).  gs_project narrows each tile
+ * rectangle to the tile columns and rows where some pixel centre can still
+ * pass the alpha >= 1/255 test of the blend: with the record's conic
+ * (A, B, C) and opacity o, ell = ln(255 o) + 0.01 and q = A C - B^2, the
+ * largest alpha on the pixel-centre column at horizontal offset dx is
+ * o exp(-dx^2 q / (2 C)), so columns whose nearest centre is farther than
+ * D_x = sqrt(2 ell C / q) from the mean are cut (rows likewise with
+ * D_y = sqrt(2 ell A / q)); ell <= 0 cuts everything.  The cut is skipped
+ * when A C > 1024 q (an ill-conditioned conic).  Every pixel of a cut tile
+ * has alpha below 0.99 / 255, so the image, the final transmittance and the
+ * gradients are those of the 3-sigma rectangle (up to alpha tests that
+ * single-precision rounding leaves undecided within that 1 %), while the
+ * pair count, the sort and the blend work shrink.  `last` (an index into a
+ * tile's list) refers to the shorter lists. */
+#define GS_FLAG_TIGHT_TILES 1u
 
 /* Raw (unconstrained) parameters of N Gaussians ([GSP] s1), fp32, C-contiguous. */
 typedef struct gs_params {
@@ -148,7 +167,8 @@ int gs_bins_carve(void *base, int64_t n, int64_t max_pairs, int32_t width, int32
  * at 1e-10; conic = (c, -b, a)/det; radius = ceil(3 sqrt(lambda_max)) with
  * the root term floored at 0.1; mean2d = (fx x/z + cx, fy y/z + cy);
  * tile rectangle per axis floor((m -+ r)/16) in single precision, clamped
- * to the grid.  Culled Gaussians get count 0 and an empty rectangle.
+ * to the grid, narrowed by the opacity-aware cut when cam->flags has
+ * GS_FLAG_TIGHT_TILES.  Culled Gaussians get count 0 and an empty rectangle.
  * n may be 0.  Errors: INVALID_ARG (n < 0, null pointer with n > 0, bad
  * camera), TOO_LARGE (n >= 2^30), ALIGNMENT, CUDA. */
 int gs_project(const gs_camera *cam, int64_t n, const gs_params *params, const gs_projected *out,

@@ -286,10 +286,13 @@ static double dist_to_int(double v) { return fabs(v - nearbyint(v)); }
  * A C > 1024 (A C - B^2): there the rounding of a single-precision sigma
  * near the threshold can exceed the slack.
  * Writes cut = {lo x, hi x, lo y, hi y} (tiles, integral or infinite).
- * Returns the smallest distance of its decisions from flipping, each
- * relative to its own scale: |cond / 1024 - 1|, |ell|, and for each of the
- * four bounds the distance in pixels of (m -+ D - ...)/16 from an integer
- * divided by (1 + D). */
+ * Returns how far its decisions sit from flipping, as the smallest relative
+ * perturbation of the conic (or, for ell, of the opacity) that could flip
+ * one, to first order: |cond - 1024| / (2 cond^2) for the condition test
+ * (cond moves by about 2 cond^2 per unit relative change of A, B, C), |ell|
+ * for the ell test, and for each of the four bounds the pixel distance of
+ * m -+ D from the nearest flip divided by (1 + D cond) (D moves by about
+ * D cond). */
 static double opacity_cut(double mx, double my, double A, double B, double C, double o,
                           double cut[4])
 {
@@ -298,7 +301,7 @@ static double opacity_cut(double mx, double my, double A, double B, double C, do
     double q = A * C - B * B;
     if (!(q > 0.0)) return INFINITY;
     double cond = A * C / q;
-    double margin = fabs(cond / ORC_CUT_MAX_COND - 1.0);
+    double margin = fabs(cond - ORC_CUT_MAX_COND) / (2.0 * cond * cond);
     if (!(cond <= ORC_CUT_MAX_COND)) return margin;
     double ell = log(255.0 * o) + ORC_CUT_SLACK;
     if (fabs(ell) < margin) margin = fabs(ell);
@@ -314,8 +317,8 @@ static double opacity_cut(double mx, double my, double A, double B, double C, do
         double hi = (m[axis] + D[axis] - 0.5) / ORC_TILE;
         cut[2 * axis] = ceil(lo);
         cut[2 * axis + 1] = floor(hi);
-        double d0 = ORC_TILE * dist_to_int(lo) / (1.0 + D[axis]);
-        double d1 = ORC_TILE * dist_to_int(hi) / (1.0 + D[axis]);
+        double d0 = ORC_TILE * dist_to_int(lo) / (1.0 + D[axis] * cond);
+        double d1 = ORC_TILE * dist_to_int(hi) / (1.0 + D[axis] * cond);
         if (d0 < margin) margin = d0;
         if (d1 < margin) margin = d1;
     }

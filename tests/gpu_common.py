@@ -33,7 +33,7 @@ MARGIN_T = 1e-3       # relative margin of T (1 - alpha) against 1e-4
 MARGIN_CLAMP = 1e-4   # relative margin of o G against the 0.99 cap
 MARGIN_TILE = 1e-4    # tiles, distance of (m -+ r)/16 to an integer
 MARGIN_RADIUS = 2e-4  # px, distance of 3 sqrt(lambda) to an integer
-MARGIN_CUT = 1e-3     # relative distance of an opacity-cut decision from flipping
+MARGIN_CUT = 2e-5     # relative conic (opacity) change that flips an opacity-cut decision
 
 
 def cuda_params(params: dict) -> dict:

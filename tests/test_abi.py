@@ -39,7 +39,7 @@ def test_binding_declares_exactly_the_header(lib):
 
 def test_struct_sizes_match_header_layout():
     from gaussian_splatting_differentiable_tile_b200 import _abi
-    assert ctypes.sizeof(_abi.GsCamera) == 4 * (16 + 4 + 2 + 1 + 3)
+    assert ctypes.sizeof(_abi.GsCamera) == 4 * (16 + 4 + 2 + 1 + 3 + 1)
     assert ctypes.sizeof(_abi.GsProjected) == 5 * 8
     assert ctypes.sizeof(_abi.GsBins) == 5 * 8 + 8 + 8 + 4 + 4 + 8 + 8
 

@@ -40,9 +40,11 @@ SCENES = {
 
 
 # ------------------------------------------------------------------ project
+@pytest.mark.parametrize("flags", [0, G.GS_FLAG_TIGHT_TILES])
 @pytest.mark.parametrize("scene", list(SCENES))
-def test_project_matches_oracle(scene):
+def test_project_matches_oracle(scene, flags):
     cam, params = SCENES[scene]()
+    cam.flags = flags
     n = params["means"].shape[0]
     proj = G.Projected(n)
     G.gs_project(cam, cuda_params(params), proj)
@@ -68,7 +70,7 @@ def test_project_matches_oracle(scene):
     diff_rect = np.any(rect != p["rect"], axis=1) | (count != p["count"])
     assert not np.any(diff_r & ~amb), np.nonzero(diff_r & ~amb)[0][:10]
     assert not np.any(diff_rect & ~amb), np.nonzero(diff_rect & ~amb)[0][:10]
-    assert amb.sum() <= max(2, 1e-3 * n)
+    assert amb.sum() <= max(4, 2e-3 * n)
 
 
 # ---------------------------------------------------- bin and sort (stage-fed)
@@ -267,6 +269,50 @@ def test_render_bwd_student_sampled_tiles():
     grad_compare(g2[:, :9], g2_ref, g2_abs, "grad2d")
 
 
+# --------------------------------------------- opacity-aware tile cut
+@pytest.mark.parametrize("scene", ["ragged", "student3k"])
+def test_tight_tiles_stage_fed(scene):
+    """Forward and backward on the oracle's cut rectangles."""
+    cam, params = SCENES[scene]()
+    cam.flags = G.GS_FLAG_TIGHT_TILES
+    rec, proj, bins, K, image, T, last, ref = _fwd_stage_fed(cam, params)
+    _assert_fwd(cam, bins, image, T, last, ref, np.ones((cam.height, cam.width), bool))
+    rec, g2, grads, g2_ref, g2_abs, params = _bwd_stage_fed(cam, params)
+    grad_compare(g2[:, :9], g2_ref, g2_abs, "grad2d")
+    raw_ref = O.project_bwd(params, cam, g2_ref)
+    bound = O.grad_bound(params, cam, g2_abs)
+    for k in G.PARAM_KEYS:
+        grad_compare(grads[k], raw_ref[k], bound[k], k)
+
+
+def test_tight_tiles_leave_image_and_gradients_unchanged():
+    """The 30k student at 980 x 545 through the CUDA path with and without
+    the cut: the same entries pass the alpha test in the same order, so the
+    image and transmittance are equal bit for bit, with fewer pairs."""
+    cam, params = _student_subset(30_000)
+    n = params["means"].shape[0]
+    P = cuda_params(params)
+    target = torch.from_numpy(make_target(cam.width, cam.height)).cuda()
+    out = {}
+    for flags in (0, G.GS_FLAG_TIGHT_TILES):
+        cam.flags = flags
+        r = G.Rasterizer(n, cam.width, cam.height)
+        image = r.forward(cam, P).clone()
+        T = r.T_final.clone()
+        dl = torch.empty_like(image)
+        G.gs_l1_loss_grad(image, target, dl, torch.zeros(1, device="cuda"))
+        grads = {k: v.clone() for k, v in r.backward(cam, P, dl).items()}
+        torch.cuda.synchronize()
+        out[flags] = (image.cpu().numpy(), T.cpu().numpy(), grads, r.n_pairs)
+    (i0, t0, g0, k0), (i1, t1, g1, k1) = out[0], out[G.GS_FLAG_TIGHT_TILES]
+    assert k1 < 0.85 * k0
+    np.testing.assert_array_equal(i1, i0)
+    np.testing.assert_array_equal(t1, t0)
+    for k in G.PARAM_KEYS:  # same sums, atomics in another order
+        a, b = g1[k].cpu().numpy(), g0[k].cpu().numpy()
+        assert np.abs(a - b).max() <= 1e-5 * max(np.abs(b).max(), 1e-30), k
+
+
 # ------------------------------------------------------------ end to end
 def _without_ambiguous(params, cam):
     """The scene with every Gaussian whose projection sits within the stated
@@ -280,10 +326,12 @@ def _without_ambiguous(params, cam):
     return out, int(bad.sum())
 
 
-def test_end_to_end_from_raw_parameters():
+@pytest.mark.parametrize("flags", [0, G.GS_FLAG_TIGHT_TILES])
+def test_end_to_end_from_raw_parameters(flags):
     """Raw parameters through all four calls vs the oracle from the same raw
     parameters in double precision, L1 loss against a seeded target."""
     cam, params = SCENES["ragged"]()
+    cam.flags = flags
     params, removed = _without_ambiguous(params, cam)
     assert removed <= 20
     n = params["means"].shape[0]
