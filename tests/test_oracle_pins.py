@@ -311,3 +311,22 @@ def test_culled_gaussians_get_exact_zero_gradient():
             if not g["contributes"][k]:
                 assert np.all(v[k] == 0.0), (name, k)
     assert np.abs(grads["means"][0]).sum() > 0 and np.abs(grads["colors"][0]).sum() > 0
+
+
+def test_non_finite_colour_is_culled():
+    """s6: a Gaussian whose colour is not finite never enters the blend; the
+    image of the others is unchanged and its gradients are exactly 0."""
+    cam = _identity_cam(32, 32, 40.0, 40.0, 16.0, 16.0)
+    params = {"means": np.array([[0.0, 0.0, 2.0], [0.05, 0.0, 2.5]]),
+              "log_scales": np.full((2, 3), -2.0), "quats": np.tile([1.0, 0, 0, 0], (2, 1)),
+              "opacity_logits": np.zeros(2), "colors": np.array([[0.5, 0.5, 0.5], [0.2, np.nan, 0.1]])}
+    p = O.project(params, cam)
+    assert p["valid"].tolist() == [1, 0] and p["count"][1] == 0
+    one = {k: v[:1] for k, v in params.items()}
+    np.testing.assert_array_equal(O.render(p, cam, nthreads=1)["image"],
+                                  O.render(O.project(one, cam), cam, nthreads=1)["image"])
+    g2, _ = O.render_bwd(p, cam, np.ones((32, 32, 3)), nthreads=1)
+    grads = O.project_bwd(params, cam, g2)
+    for name, v in grads.items():
+        assert np.all(v[1] == 0.0), name
+    assert np.abs(grads["means"][0]).sum() > 0 and np.abs(grads["colors"][0]).sum() > 0
