@@ -154,20 +154,6 @@ __device__ __forceinline__ bool eval_alpha(const float4 geo, const float4 geo2, 
     return true;
 }
 
-// eval_alpha without control flow: alpha = 0 where the entry is skipped
-// (the same decisions, the exponential taken unconditionally).
-__device__ __forceinline__ float eval_alpha_nb(const float4 geo, const float4 geo2, const ColTerms &c,
-                                               float fy, bool walk, float &dy, bool &capped) {
-    dy = __fsub_rn(geo.y, fy);
-    const float u = __fmaf_rn(geo2.x, dy, c.bdx);
-    const float q = __fmaf_rn(dy, u, c.a0);
-    const float p = __fadd_rn(q, geo2.y);
-    const bool hit = walk && !(q > 0.f) && !(p < kLog2AlphaMin);
-    const float a = ex2_approx(p);
-    capped = hit && a > kAlphaCap;
-    return hit ? fminf(a, kAlphaCap) : 0.f;
-}
-
 // Stages entries [0, cnt) of a batch into shared memory: slot i holds list
 // entry idx(i) (and, for the backward, its Gaussian id).  Each thread gathers two entries per round (ids first, then
 // records), so the dependent loads overlap without holding many registers.
@@ -364,7 +350,9 @@ k_render_bwd(CamConst cam, const float4 *__restrict__ xyod, const float4 *__rest
              const uint2 *__restrict__ ranges, const float *__restrict__ T_final,
              const uint32_t *__restrict__ last, const float *__restrict__ dL_dimage,
              float *__restrict__ grad2d) {
+    static_assert(kRPL % 2 == 0, "the backward works on pairs of rows");
     constexpr int kThreads = kTilePixels / kRPL;
+    constexpr int kPairs = kRPL / 2;
     constexpr int kB = kBwdBatch;
     __shared__ float4 s_geo[kB];
     __shared__ float4 s_geo2[kB];
@@ -378,23 +366,32 @@ k_render_bwd(CamConst cam, const float4 *__restrict__ xyod, const float4 *__rest
     const bool col_in = L.px < cam.width;
     const int lane = threadIdx.x & 31;
 
-    float T[kRPL], sg[kRPL], g0[kRPL], g1[kRPL], g2[kRPL];
+    // Per pixel state, two rows per float2 (x: row 2i, y: row 2i + 1).
+    float2 T[kPairs], sg[kPairs], g0[kPairs], g1[kPairs], g2[kPairs], nfy[kPairs];
     uint32_t lst[kRPL];
     uint32_t lane_max = range.x;
 #pragma unroll
     for (int r = 0; r < kRPL; r++) {
-        T[r] = 1.f; g0[r] = 0.f; g1[r] = 0.f; g2[r] = 0.f;
+        float t = 1.f, d0 = 0.f, d1 = 0.f, d2 = 0.f;
         lst[r] = range.x;
         const int py = L.py0 + r;
         if (col_in && py < cam.height) {
             const size_t p = (size_t)py * cam.width + L.px;
-            T[r] = T_final[p];
+            t = T_final[p];
             lst[r] = min(max(last[p], range.x), range.y);  // never walk outside the tile's list
-            g0[r] = dL_dimage[3 * p];
-            g1[r] = dL_dimage[3 * p + 1];
-            g2[r] = dL_dimage[3 * p + 2];
+            d0 = dL_dimage[3 * p];
+            d1 = dL_dimage[3 * p + 1];
+            d2 = dL_dimage[3 * p + 2];
         }
-        sg[r] = T[r] * (cam.bg[0] * g0[r] + cam.bg[1] * g1[r] + cam.bg[2] * g2[r]);
+        const float s0 = t * (cam.bg[0] * d0 + cam.bg[1] * d1 + cam.bg[2] * d2);
+        const float nf = -(L.fy0 + (float)r);
+        if (r & 1) {
+            T[r / 2].y = t; g0[r / 2].y = d0; g1[r / 2].y = d1; g2[r / 2].y = d2; sg[r / 2].y = s0;
+            nfy[r / 2].y = nf;
+        } else {
+            T[r / 2].x = t; g0[r / 2].x = d0; g1[r / 2].x = d1; g2[r / 2].x = d2; sg[r / 2].x = s0;
+            nfy[r / 2].x = nf;
+        }
         lane_max = max(lane_max, lst[r]);
     }
     // entries at or past every pixel's last are not walked: per warp and per CTA
@@ -421,42 +418,64 @@ k_render_bwd(CamConst cam, const float4 *__restrict__ xyod, const float4 *__rest
             const float4 geo = s_geo[k], geo2 = s_geo2[k];
             if (kCull && culled(geo, geo2, L)) continue;
             const ColTerms ct = col_terms(geo, L.fx);
-            const float4 c = s_col[k];
-            float sv = 0.f, sgy = 0.f, sgyy = 0.f, cr0 = 0.f, cr1 = 0.f, cr2 = 0.f;
-            bool contrib = false;
-            // Branch-free over the lane's rows (measured 16 % faster than
-            // skipping per row): where the entry is skipped alpha is 0, so
-            // w, v and every sum get exact zeros (colours of drawn Gaussians
-            // are finite), and T is kept by a select.
+            // The exponent at the lane's rows, two rows per paired instruction
+            // (each half rounded exactly as the forward's scalar evaluation,
+            // so every skip decision is the same), and which rows pass.
+            float2 dy[kPairs], p[kPairs];
+            bool hit[kRPL];
+            bool any = false;
 #pragma unroll
-            for (int r = 0; r < kRPL; r++) {
-                float dy;
-                bool capped;
-                const float a = eval_alpha_nb(geo, geo2, ct, L.fy0 + (float)r, j < lst[r], dy, capped);
-                contrib |= a > 0.f;
-                const float ri = rcp_approx(__fsub_rn(1.f, a));
-                const float Ti = __fmul_rn(T[r], ri);
-                const float w = __fmul_rn(a, Ti);
-                const float cg = __fmaf_rn(c.z, g2[r], __fmaf_rn(c.y, g1[r], c.x * g0[r]));
-                const float dLda = ri * __fmaf_rn(T[r], cg, -sg[r]);
-                sg[r] = __fmaf_rn(w, cg, sg[r]);
-                cr0 = __fmaf_rn(w, g0[r], cr0);
-                cr1 = __fmaf_rn(w, g1[r], cr1);
-                cr2 = __fmaf_rn(w, g2[r], cr2);
-                const float v = capped ? 0.f : dLda * a;
-                sv += v;
-                const float vy = v * dy;
-                sgy += vy;
-                sgyy = __fmaf_rn(vy, dy, sgyy);
-                T[r] = a > 0.f ? Ti : T[r];
+            for (int i = 0; i < kPairs; i++) {
+                dy[i] = __fadd2_rn(make_float2(geo.y, geo.y), nfy[i]);
+                const float2 u = __ffma2_rn(make_float2(geo2.x, geo2.x), dy[i], make_float2(ct.bdx, ct.bdx));
+                const float2 q = __ffma2_rn(dy[i], u, make_float2(ct.a0, ct.a0));
+                p[i] = __fadd2_rn(q, make_float2(geo2.y, geo2.y));
+                hit[2 * i] = j < lst[2 * i] && !(q.x > 0.f) && !(p[i].x < kLog2AlphaMin);
+                hit[2 * i + 1] = j < lst[2 * i + 1] && !(q.y > 0.f) && !(p[i].y < kLog2AlphaMin);
+                any |= hit[2 * i] | hit[2 * i + 1];
             }
-            if (__any_sync(0xffffffffu, contrib)) {
-                const float sgx = sv * ct.dx;
-                const float vals[9] = {sv, sgx, sgy, sgx * ct.dx, sgy * ct.dx, sgyy, cr0, cr1, cr2};
-                int idx;
-                const float tot = reduce_scatter9(vals, lane, &idx);
-                if (idx < 9) atomicAdd(grad2d + 12 * (size_t)s_gid[k] + idx, tot);
+            if (!__any_sync(0xffffffffu, any)) continue;
+            // Contributions, branch-free (measured faster than skipping per
+            // row): a skipped row has alpha 0, which zeroes w, v and every
+            // sum exactly (colours of drawn Gaussians are finite); T is kept
+            // by a select.
+            const float4 c = s_col[k];
+            float2 sv = make_float2(0.f, 0.f), sgy = sv, sgyy = sv, cr0 = sv, cr1 = sv, cr2 = sv;
+#pragma unroll
+            for (int i = 0; i < kPairs; i++) {
+                const bool h0 = hit[2 * i], h1 = hit[2 * i + 1];
+                const float e0 = ex2_approx(p[i].x), e1 = ex2_approx(p[i].y);
+                const float2 a = make_float2(h0 ? fminf(e0, kAlphaCap) : 0.f, h1 ? fminf(e1, kAlphaCap) : 0.f);
+                const bool cap0 = h0 && e0 > kAlphaCap, cap1 = h1 && e1 > kAlphaCap;
+                const float2 om = __fadd2_rn(make_float2(1.f, 1.f), make_float2(-a.x, -a.y));
+                const float2 ri = make_float2(rcp_approx(om.x), rcp_approx(om.y));
+                const float2 Ti = __fmul2_rn(T[i], ri);
+                const float2 w = __fmul2_rn(a, Ti);
+                const float2 cg = __ffma2_rn(make_float2(c.z, c.z), g2[i],
+                                             __ffma2_rn(make_float2(c.y, c.y), g1[i],
+                                                        __fmul2_rn(make_float2(c.x, c.x), g0[i])));
+                const float2 dLda = __fmul2_rn(ri, __ffma2_rn(T[i], cg, make_float2(-sg[i].x, -sg[i].y)));
+                sg[i] = __ffma2_rn(w, cg, sg[i]);
+                cr0 = __ffma2_rn(w, g0[i], cr0);
+                cr1 = __ffma2_rn(w, g1[i], cr1);
+                cr2 = __ffma2_rn(w, g2[i], cr2);
+                float2 v = __fmul2_rn(dLda, a);  // dL/dsigma = -v, dL/do = v / o
+                v.x = cap0 ? 0.f : v.x;
+                v.y = cap1 ? 0.f : v.y;
+                sv = __fadd2_rn(sv, v);
+                const float2 vy = __fmul2_rn(v, dy[i]);
+                sgy = __fadd2_rn(sgy, vy);
+                sgyy = __ffma2_rn(vy, dy[i], sgyy);
+                T[i].x = h0 ? Ti.x : T[i].x;
+                T[i].y = h1 ? Ti.y : T[i].y;
             }
+            const float svs = sv.x + sv.y, sgys = sgy.x + sgy.y;
+            const float sgx = svs * ct.dx;
+            const float vals[9] = {svs, sgx, sgys, sgx * ct.dx, sgys * ct.dx, sgyy.x + sgyy.y,
+                                   cr0.x + cr0.y, cr1.x + cr1.y, cr2.x + cr2.y};
+            int idx;
+            const float tot = reduce_scatter9(vals, lane, &idx);
+            if (idx < 9) atomicAdd(grad2d + 12 * (size_t)s_gid[k] + idx, tot);
         }
         __syncthreads();
         bend = bstart;
