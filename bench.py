@@ -229,6 +229,25 @@ def _config(spec, pairs, tiles, graphs=True):
             "parallelism": "replicas (cameras split across ranks)"}
 
 
+# ------------------------------------------------------------ rank logic
+def my_cameras(cams, rank: int, world: int):
+    """Replicas: rank r renders cameras r, r + world, ... (at least one, so
+    that every rank takes the same collective steps)."""
+    return [c for i, c in enumerate(cams) if i % world == rank] or cams[:1]
+
+
+def max_over_ranks(values, world: int, device):
+    """Elementwise max over ranks of per-rank timings (the whole job ends when
+    the slowest rank does)."""
+    import torch
+    import torch.distributed as dist
+
+    t = torch.tensor([float(v) for v in values], dtype=torch.float64, device=device)
+    if world > 1:
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return t.tolist()
+
+
 # ------------------------------------------------------------------ GPU side
 def run_profile_frame(args, spec):
     """One eager frame (forward, L1 gradient, backward) of one camera for a
@@ -262,7 +281,7 @@ def run_native(args, spec, rank, world, local):
     dev = torch.device("cuda", local)
     params_np = make_scene(spec)
     cams = _cameras(spec, args)
-    mine = [c for i, c in enumerate(cams) if i % world == rank] or cams[:1]
+    mine = my_cameras(cams, rank, world)
     n = spec.n
     P = {k: torch.from_numpy(v).to(dev) for k, v in params_np.items()}
     targets = [torch.from_numpy(make_target(spec.width, spec.height, seed=i)).to(dev) for i in range(len(mine))]
@@ -382,10 +401,7 @@ def run_native(args, spec, rank, world, local):
     h2d = sum(v.size * 4 for v in params_np.values()) + H * W * 3 * 4
     d2h = sum(v.size * 4 for v in params_np.values()) + 4
 
-    t = torch.tensor([full_ms, fwd_ms, e2e_ms], dtype=torch.float64, device=dev)
-    if world > 1:
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-    full_ms, fwd_ms, e2e_ms = t.tolist()
+    full_ms, fwd_ms, e2e_ms = max_over_ranks([full_ms, fwd_ms, e2e_ms], world, dev)
     frames = args.steps * world
     if rank != 0:
         return
