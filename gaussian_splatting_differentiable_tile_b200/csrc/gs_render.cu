@@ -14,8 +14,9 @@
 // Work layout.  One CTA per tile.  Each lane owns RPL vertically adjacent
 // pixels of one column: lanes 0-15 the upper RPL rows of the warp's strip,
 // lanes 16-31 the lower RPL rows, so a warp covers a 16 x 2RPL strip and a
-// tile takes 8 / RPL warps.  The tile's list is staged through shared memory
-// in batches of 256 entries, each entry converted once per tile to
+// tile takes 8 / RPL warps (forward: RPL = 1, eight warps; backward: RPL = 4,
+// two warps).  The tile's list is staged through shared memory in batches
+// (forward 256 entries, backward 128), each entry converted once per tile to
 //     geo  = (mx, my, cA, cB),  geo2 = (cC, log2 o, kx, ky)
 // with cA = -log2(e) A / 2, cB = -log2(e) B, cC = -log2(e) C / 2, so that
 //     log2(o exp(-sigma)) = log2 o + cA dx^2 + cB dx dy + cC dy^2.
@@ -28,21 +29,17 @@
 // -sigma log2(e) <= min(kx dx_min^2, ky dy_min^2).  When that bound keeps
 // alpha below 1/255 with a 1 % margin at every pixel of the warp, the entry is
 // skipped for the warp; each of its pixels would have skipped it anyway, so
-// the result is unchanged.
+// the result is unchanged.  The forward takes the test for all eight strips
+// while staging and lets each warp walk a compacted list of its slots; the
+// backward takes it per entry.
 //
 // The forward and backward share the evaluation code and use explicitly
 // rounded intrinsics, so the backward re-takes every skip decision
 // bit-identically.
 #include "gs_internal.cuh"
 
-// Pixels per lane and per-warp culling of the two blend kernels (tuning
-// knobs; the defaults are the fastest measured on B200).
-#ifndef GS_FWD_RPL
-#define GS_FWD_RPL 1
-#endif
-#ifndef GS_FWD_CULL
-#define GS_FWD_CULL 0
-#endif
+// Pixels per lane and per-warp culling of the backward (tuning knobs; the
+// defaults are the fastest measured on B200).
 #ifndef GS_BWD_RPL
 #define GS_BWD_RPL 4
 #endif
@@ -185,110 +182,100 @@ __device__ __forceinline__ void stage_batch(uint32_t cnt, Idx idx, const uint32_
     }
 }
 
-template <int kRPL, bool kCull>
-__global__ void __launch_bounds__(kTilePixels / kRPL)
+
+// Forward, one pixel per thread, eight warps per tile (warp w owns the
+// 16 x 2 strip of rows 2w, 2w + 1).  While a batch is staged, each entry's
+// per-strip cull test (the separable bound above, taken for the eight strips
+// at once) yields an 8-bit mask; each warp then compacts the batch to the
+// slots whose bit it holds, in order, and walks only those.  A culled slot
+// could not have passed the alpha test at any pixel of the strip, so the
+// sequence of contributions, the stopping entry and `last` are unchanged.
+__global__ void __launch_bounds__(kTilePixels, 6)
 k_render_fwd(CamConst cam, const float4 *__restrict__ xyod, const float4 *__restrict__ conr,
              const float4 *__restrict__ rgb, const uint32_t *__restrict__ pair_gid,
-             const uint2 *__restrict__ ranges, float *__restrict__ image,
-             float *__restrict__ T_final, uint32_t *__restrict__ last) {
-    constexpr int kThreads = kTilePixels / kRPL;
+             const uint2 *__restrict__ ranges, float *__restrict__ image, float *__restrict__ T_final,
+             uint32_t *__restrict__ last) {
+    constexpr int kWarps = kTilePixels / 32;
     __shared__ float4 s_geo[kBatch];
     __shared__ float4 s_geo2[kBatch];
     __shared__ float4 s_col[kBatch];
+    __shared__ uint8_t s_mask[kBatch];
+    __shared__ uint8_t s_list[kWarps][kBatch];
 
     const int tile = blockIdx.x;
-    const LaneGeom L = lane_geom<kRPL>(cam, tile);
+    const LaneGeom L = lane_geom<1>(cam, tile);
     const uint2 range = ranges[tile];
-    const bool col_in = L.px < cam.width;
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    const uint32_t lt = (1u << lane) - 1u;
+    // strip geometry for the staging threads' mask: x as the lane's strip,
+    // y centre of strip w = tile top + 2 w + 1, half extent 0.5
+    const float strip_y0 = (float)((tile / cam.tiles_x) * kTile) + 1.f;
 
-    float T[kRPL], C0[kRPL], C1[kRPL], C2[kRPL];
-    uint32_t lst[kRPL];
-    bool done[kRPL];
-#pragma unroll
-    for (int r = 0; r < kRPL; r++) {
-        T[r] = 1.f; C0[r] = 0.f; C1[r] = 0.f; C2[r] = 0.f;
-        lst[r] = range.x;
-        done[r] = !(col_in && L.py0 + r < cam.height);
-    }
+    float T = 1.f, C0 = 0.f, C1 = 0.f, C2 = 0.f;
+    uint32_t lst = range.x;
+    bool done = !(L.px < cam.width && L.py0 < cam.height);
     for (uint32_t b = range.x; b < range.y; b += kBatch) {
-        bool all_done = true;
-#pragma unroll
-        for (int r = 0; r < kRPL; r++) all_done &= done[r];
-        if (__syncthreads_count(all_done) == kThreads) break;
+        if (__syncthreads_count(done) == kTilePixels) break;
         const uint32_t cnt = min((uint32_t)kBatch, range.y - b);
-        stage_batch<kThreads, false>(cnt, [b](uint32_t i) { return b + i; }, pair_gid, xyod, conr, rgb,
-                                     s_geo, s_geo2, s_col, nullptr);
-        __syncthreads();
-        // A lane leaves the batch loop as soon as all its pixels have stopped
-        // (a per-lane exit, not a per-entry warp vote: measured faster).  The
-        // cull test depends only on the warp's strip, so it stays uniform
-        // among the lanes still in the loop.
-        if (kRPL == 1 && !kCull) {
-            // one pixel per lane: the lane breaks out at its stopping entry
-            if (!done[0]) {
-                for (uint32_t k = 0; k < cnt; k++) {
-                    const float4 geo = s_geo[k], geo2 = s_geo2[k];
-                    const ColTerms ct = col_terms(geo, L.fx);
-                    float dy, a;
-                    bool capped;
-                    if (!eval_alpha(geo, geo2, ct, L.fy0, dy, a, capped)) continue;
-                    const float nT = __fmaf_rn(-T[0], a, T[0]);
-                    if (nT < kTMin) {
-                        done[0] = true;
-                        break;
-                    }
-                    const float4 c = s_col[k];
-                    const float w = __fmul_rn(a, T[0]);
-                    C0[0] = __fmaf_rn(w, c.x, C0[0]);
-                    C1[0] = __fmaf_rn(w, c.y, C1[0]);
-                    C2[0] = __fmaf_rn(w, c.z, C2[0]);
-                    T[0] = nT;
-                    lst[0] = b + k + 1;
-                }
-            }
-        } else if (!all_done) {
-            for (uint32_t k = 0; k < cnt; k++) {
-                const float4 geo = s_geo[k], geo2 = s_geo2[k];
-                if (kCull && culled(geo, geo2, L)) continue;
-                const ColTerms ct = col_terms(geo, L.fx);
-                bool lane_done = true;
+        if (threadIdx.x < cnt) {
+            const uint32_t g = pair_gid[b + threadIdx.x];
+            float4 geo, geo2;
+            stage_entry(xyod[g], conr[g], geo, geo2);
+            s_geo[threadIdx.x] = geo;
+            s_geo2[threadIdx.x] = geo2;
+            s_col[threadIdx.x] = rgb[g];
+            const float dxm = fmaxf(fabsf(geo.x - L.sx) - L.hx, 0.f);
+            const float qx = geo2.z * dxm * dxm;
+            uint32_t m = 0;
 #pragma unroll
-                for (int r = 0; r < kRPL; r++) {
-                    if (done[r]) continue;
-                    float dy, a;
-                    bool capped;
-                    if (eval_alpha(geo, geo2, ct, L.fy0 + (float)r, dy, a, capped)) {
-                        const float nT = __fmaf_rn(-T[r], a, T[r]);
-                        if (nT < kTMin) {
-                            done[r] = true;
-                            continue;
-                        }
-                        const float4 c = s_col[k];
-                        const float w = __fmul_rn(a, T[r]);
-                        C0[r] = __fmaf_rn(w, c.x, C0[r]);
-                        C1[r] = __fmaf_rn(w, c.y, C1[r]);
-                        C2[r] = __fmaf_rn(w, c.z, C2[r]);
-                        T[r] = nT;
-                        lst[r] = b + k + 1;
-                    }
-                    lane_done = false;
+            for (int w = 0; w < kWarps; w++) {
+                const float dym = fmaxf(fabsf(geo.y - (strip_y0 + 2.f * w)) - 0.5f, 0.f);
+                const float qb = fminf(qx, geo2.w * dym * dym);
+                m |= (geo2.y + qb < kCullLog2 ? 0u : 1u) << w;
+            }
+            s_mask[threadIdx.x] = (uint8_t)m;
+        }
+        __syncthreads();
+        uint32_t n = 0;
+#pragma unroll
+        for (int c = 0; c < kBatch / 32; c++) {
+            const uint32_t i = c * 32 + lane;
+            const bool f = i < cnt && ((s_mask[i] >> warp) & 1u);
+            const uint32_t bal = __ballot_sync(0xffffffffu, f);
+            if (f) s_list[warp][n + __popc(bal & lt)] = (uint8_t)i;
+            n += __popc(bal);
+        }
+        __syncwarp();
+        if (!done) {
+            for (uint32_t k = 0; k < n; k++) {
+                const uint32_t i = s_list[warp][k];
+                const float4 geo = s_geo[i], geo2 = s_geo2[i];
+                const ColTerms ct = col_terms(geo, L.fx);
+                float dy, a;
+                bool capped;
+                if (!eval_alpha(geo, geo2, ct, L.fy0, dy, a, capped)) continue;
+                const float nT = __fmaf_rn(-T, a, T);
+                if (nT < kTMin) {
+                    done = true;
+                    break;
                 }
-                if (lane_done) break;
+                const float4 c = s_col[i];
+                const float w = __fmul_rn(a, T);
+                C0 = __fmaf_rn(w, c.x, C0);
+                C1 = __fmaf_rn(w, c.y, C1);
+                C2 = __fmaf_rn(w, c.z, C2);
+                T = nT;
+                lst = b + i + 1;
             }
         }
     }
-    if (col_in) {
-#pragma unroll
-        for (int r = 0; r < kRPL; r++) {
-            const int py = L.py0 + r;
-            if (py >= cam.height) continue;
-            const size_t p = (size_t)py * cam.width + L.px;
-            image[3 * p] = __fmaf_rn(T[r], cam.bg[0], C0[r]);
-            image[3 * p + 1] = __fmaf_rn(T[r], cam.bg[1], C1[r]);
-            image[3 * p + 2] = __fmaf_rn(T[r], cam.bg[2], C2[r]);
-            T_final[p] = T[r];
-            last[p] = lst[r];
-        }
+    if (L.px < cam.width && L.py0 < cam.height) {
+        const size_t p = (size_t)L.py0 * cam.width + L.px;
+        image[3 * p] = __fmaf_rn(T, cam.bg[0], C0);
+        image[3 * p + 1] = __fmaf_rn(T, cam.bg[1], C1);
+        image[3 * p + 2] = __fmaf_rn(T, cam.bg[2], C2);
+        T_final[p] = T;
+        last[p] = lst;
     }
 }
 
@@ -572,7 +559,7 @@ cudaError_t launch_render_fwd(const CamConst &c, const gs_projected &proj, const
                               float *image, float *T_final, uint32_t *last, cudaStream_t s) {
     const int tiles = c.tiles_x * c.tiles_y;
     prof_before("render_fwd", s);
-    k_render_fwd<GS_FWD_RPL, GS_FWD_CULL != 0><<<tiles, kTilePixels / GS_FWD_RPL, 0, s>>>(
+    k_render_fwd<<<tiles, kTilePixels, 0, s>>>(
         c, reinterpret_cast<const float4 *>(proj.xy_opacity_depth),
         reinterpret_cast<const float4 *>(proj.conic_radius), reinterpret_cast<const float4 *>(proj.rgb),
         bins.pair_gid, reinterpret_cast<const uint2 *>(bins.ranges), image, T_final, last);
