@@ -38,13 +38,10 @@
 // bit-identically.
 #include "gs_internal.cuh"
 
-// Pixels per lane and per-warp culling of the backward (tuning knobs; the
-// defaults are the fastest measured on B200).
+// Pixels per lane of the backward (a tuning knob; the default is the fastest
+// measured on B200).
 #ifndef GS_BWD_RPL
 #define GS_BWD_RPL 4
-#endif
-#ifndef GS_BWD_CULL
-#define GS_BWD_CULL 1
 #endif
 
 namespace gs {
@@ -90,11 +87,12 @@ __device__ __forceinline__ void stage_entry(const float4 xyod, const float4 conr
     geo2 = make_float4(cC, log2f(xyod.z), kx, ky);
 }
 
-// Geometry of a lane: its column centre, its first row's centre, and the
-// centre and half extents of its warp's strip.
+// Geometry of a lane: its column centre and first row's centre; and the
+// tile's strips (2 RPL rows each): x centre and half width, y centre of the
+// first strip, half height.
 struct LaneGeom {
     float fx, fy0;
-    float sx, sy, hx, hy;
+    float sx, hx, sy0, hy;
     int px, py0;
 };
 
@@ -109,17 +107,46 @@ __device__ __forceinline__ LaneGeom lane_geom(const CamConst &cam, int tile) {
     L.fy0 = (float)L.py0 + 0.5f;
     L.sx = (float)(tx * kTile) + 8.f;
     L.hx = 7.5f;
-    L.sy = (float)(ty * kTile + warp * 2 * kRPL + kRPL);
+    L.sy0 = (float)(ty * kTile + kRPL);
     L.hy = (float)kRPL - 0.5f;
     return L;
 }
 
-// True when the entry cannot reach alpha >= 1/255 anywhere in the warp's strip.
-__device__ __forceinline__ bool culled(const float4 geo, const float4 geo2, const LaneGeom &L) {
-    const float dxm = fmaxf(fabsf(geo.x - L.sx) - L.hx, 0.f);
-    const float dym = fmaxf(fabsf(geo.y - L.sy) - L.hy, 0.f);
-    const float qb = fminf(geo2.z * dxm * dxm, geo2.w * dym * dym);
-    return geo2.y + qb < kCullLog2;
+// Bit w set unless the entry cannot reach alpha >= 1/255 anywhere in strip w
+// of kStrips horizontal strips (x centre sx, half width hx; y centre
+// sy0 + w step, half height hy).
+template <int kStrips>
+__device__ __forceinline__ uint32_t strip_mask(const float4 geo, const float4 geo2, float sx, float hx,
+                                               float sy0, float step, float hy) {
+    const float dxm = fmaxf(fabsf(geo.x - sx) - hx, 0.f);
+    const float qx = geo2.z * dxm * dxm;
+    uint32_t m = 0;
+#pragma unroll
+    for (int w = 0; w < kStrips; w++) {
+        const float dym = fmaxf(fabsf(geo.y - (sy0 + step * (float)w)) - hy, 0.f);
+        const float qb = fminf(qx, geo2.w * dym * dym);
+        m |= (geo2.y + qb < kCullLog2 ? 0u : 1u) << w;
+    }
+    return m;
+}
+
+// Compacts the slots [k0, cnt) of a staged batch whose mask holds this
+// warp's bit into list[0, n), in order (one ballot per 32 slots).  Returns n.
+template <int kSlots>
+__device__ __forceinline__ uint32_t compact_slots(const uint8_t *mask, uint32_t k0, uint32_t cnt, int warp,
+                                                  int lane, uint8_t *list) {
+    const uint32_t lt = (1u << lane) - 1u;
+    uint32_t n = 0;
+#pragma unroll
+    for (int c = 0; c < kSlots / 32; c++) {
+        const uint32_t i = c * 32 + lane;
+        const bool f = i >= k0 && i < cnt && ((mask[i] >> warp) & 1u);
+        const uint32_t bal = __ballot_sync(0xffffffffu, f);
+        if (f) list[n + __popc(bal & lt)] = (uint8_t)i;
+        n += __popc(bal);
+    }
+    __syncwarp();
+    return n;
 }
 
 // Per-entry, per-lane terms shared by the lane's rows.
@@ -151,38 +178,6 @@ __device__ __forceinline__ bool eval_alpha(const float4 geo, const float4 geo2, 
     return true;
 }
 
-// Stages entries [0, cnt) of a batch into shared memory: slot i holds list
-// entry idx(i) (and, for the backward, its Gaussian id).  Each thread gathers two entries per round (ids first, then
-// records), so the dependent loads overlap without holding many registers.
-template <int kThreads, bool kGid, typename Idx>
-__device__ __forceinline__ void stage_batch(uint32_t cnt, Idx idx, const uint32_t *__restrict__ pair_gid,
-                                            const float4 *__restrict__ xyod,
-                                            const float4 *__restrict__ conr,
-                                            const float4 *__restrict__ rgb, float4 *s_geo,
-                                            float4 *s_geo2, float4 *s_col, uint32_t *s_gid) {
-    for (uint32_t i0 = threadIdx.x; i0 < cnt; i0 += 2 * kThreads) {
-        const uint32_t i1 = i0 + kThreads;
-        const uint32_t g0 = pair_gid[idx(i0)];
-        const uint32_t g1 = i1 < cnt ? pair_gid[idx(i1)] : g0;
-        const float4 x0 = xyod[g0], c0 = conr[g0], r0 = rgb[g0];
-        const float4 x1 = xyod[g1], c1 = conr[g1], r1 = rgb[g1];
-        float4 geo, geo2;
-        stage_entry(x0, c0, geo, geo2);
-        s_geo[i0] = geo;
-        s_geo2[i0] = geo2;
-        s_col[i0] = r0;
-        if (kGid) s_gid[i0] = g0;
-        if (i1 < cnt) {
-            stage_entry(x1, c1, geo, geo2);
-            s_geo[i1] = geo;
-            s_geo2[i1] = geo2;
-            s_col[i1] = r1;
-            if (kGid) s_gid[i1] = g1;
-        }
-    }
-}
-
-
 // Forward, one pixel per thread, eight warps per tile (warp w owns the
 // 16 x 2 strip of rows 2w, 2w + 1).  While a batch is staged, each entry's
 // per-strip cull test (the separable bound above, taken for the eight strips
@@ -206,10 +201,6 @@ k_render_fwd(CamConst cam, const float4 *__restrict__ xyod, const float4 *__rest
     const LaneGeom L = lane_geom<1>(cam, tile);
     const uint2 range = ranges[tile];
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-    const uint32_t lt = (1u << lane) - 1u;
-    // strip geometry for the staging threads' mask: x as the lane's strip,
-    // y centre of strip w = tile top + 2 w + 1, half extent 0.5
-    const float strip_y0 = (float)((tile / cam.tiles_x) * kTile) + 1.f;
 
     float T = 1.f, C0 = 0.f, C1 = 0.f, C2 = 0.f;
     uint32_t lst = range.x;
@@ -224,28 +215,11 @@ k_render_fwd(CamConst cam, const float4 *__restrict__ xyod, const float4 *__rest
             s_geo[threadIdx.x] = geo;
             s_geo2[threadIdx.x] = geo2;
             s_col[threadIdx.x] = rgb[g];
-            const float dxm = fmaxf(fabsf(geo.x - L.sx) - L.hx, 0.f);
-            const float qx = geo2.z * dxm * dxm;
-            uint32_t m = 0;
-#pragma unroll
-            for (int w = 0; w < kWarps; w++) {
-                const float dym = fmaxf(fabsf(geo.y - (strip_y0 + 2.f * w)) - 0.5f, 0.f);
-                const float qb = fminf(qx, geo2.w * dym * dym);
-                m |= (geo2.y + qb < kCullLog2 ? 0u : 1u) << w;
-            }
+            const uint32_t m = strip_mask<kWarps>(geo, geo2, L.sx, L.hx, L.sy0, 2.f, L.hy);
             s_mask[threadIdx.x] = (uint8_t)m;
         }
         __syncthreads();
-        uint32_t n = 0;
-#pragma unroll
-        for (int c = 0; c < kBatch / 32; c++) {
-            const uint32_t i = c * 32 + lane;
-            const bool f = i < cnt && ((s_mask[i] >> warp) & 1u);
-            const uint32_t bal = __ballot_sync(0xffffffffu, f);
-            if (f) s_list[warp][n + __popc(bal & lt)] = (uint8_t)i;
-            n += __popc(bal);
-        }
-        __syncwarp();
+        const uint32_t n = compact_slots<kBatch>(s_mask, 0, cnt, warp, lane, s_list[warp]);
         if (!done) {
             for (uint32_t k = 0; k < n; k++) {
                 const uint32_t i = s_list[warp][k];
@@ -330,7 +304,7 @@ __device__ __forceinline__ float reduce_scatter9(const float (&v)[9], int lane, 
 // with v = alpha dL/dalpha (0 when alpha was capped), w = alpha T_i; they are
 // added into grad2d, and k_project_bwd maps them to dL/d(mean2d, conic,
 // opacity) with the Gaussian's own A, B, C, o.
-template <int kRPL, bool kCull>
+template <int kRPL>
 __global__ void __launch_bounds__(kTilePixels / kRPL, 56 / kRPL)
 k_render_bwd(CamConst cam, const float4 *__restrict__ xyod, const float4 *__restrict__ conr,
              const float4 *__restrict__ rgb, const uint32_t *__restrict__ pair_gid,
@@ -339,19 +313,22 @@ k_render_bwd(CamConst cam, const float4 *__restrict__ xyod, const float4 *__rest
              float *__restrict__ grad2d) {
     static_assert(kRPL % 2 == 0, "the backward works on pairs of rows");
     constexpr int kThreads = kTilePixels / kRPL;
+    constexpr int kWarps = kThreads / 32;
     constexpr int kPairs = kRPL / 2;
     constexpr int kB = kBwdBatch;
     __shared__ float4 s_geo[kB];
     __shared__ float4 s_geo2[kB];
     __shared__ float4 s_col[kB];
     __shared__ uint32_t s_gid[kB];
+    __shared__ uint8_t s_mask[kB];
+    __shared__ uint8_t s_list[kWarps][kB];
     __shared__ uint32_t s_max_last;
 
     const int tile = blockIdx.x;
     const LaneGeom L = lane_geom<kRPL>(cam, tile);
     const uint2 range = ranges[tile];
     const bool col_in = L.px < cam.width;
-    const int lane = threadIdx.x & 31;
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
 
     // Per pixel state, two rows per float2 (x: row 2i, y: row 2i + 1).
     float2 T[kPairs], sg[kPairs], g0[kPairs], g1[kPairs], g2[kPairs], nfy[kPairs];
@@ -394,16 +371,40 @@ k_render_bwd(CamConst cam, const float4 *__restrict__ xyod, const float4 *__rest
     for (uint32_t bend = max_last; bend > range.x;) {
         const uint32_t bstart = bend - range.x > (uint32_t)kB ? bend - kB : range.x;
         const uint32_t cnt = bend - bstart;
-        // slot i holds list entry bend - 1 - i (slot 0 = back-most)
-        stage_batch<kThreads, true>(cnt, [bend](uint32_t i) { return bend - 1 - i; }, pair_gid, xyod,
-                                    conr, rgb, s_geo, s_geo2, s_col, s_gid);
+        // slot i holds list entry bend - 1 - i (slot 0 = back-most); each
+        // thread stages two entries per round (ids first, then records), so
+        // the dependent loads overlap
+        for (uint32_t i0 = threadIdx.x; i0 < cnt; i0 += 2 * kThreads) {
+            const uint32_t i1 = i0 + kThreads;
+            const uint32_t ga = pair_gid[bend - 1 - i0];
+            const uint32_t gb = i1 < cnt ? pair_gid[bend - 1 - i1] : ga;
+            const float4 xa = xyod[ga], ca = conr[ga], ra = rgb[ga];
+            const float4 xb = xyod[gb], cb = conr[gb], rb = rgb[gb];
+            float4 geo, geo2;
+            stage_entry(xa, ca, geo, geo2);
+            s_geo[i0] = geo;
+            s_geo2[i0] = geo2;
+            s_col[i0] = ra;
+            s_gid[i0] = ga;
+            s_mask[i0] = (uint8_t)strip_mask<kWarps>(geo, geo2, L.sx, L.hx, L.sy0, 2.f * kRPL, L.hy);
+            if (i1 < cnt) {
+                stage_entry(xb, cb, geo, geo2);
+                s_geo[i1] = geo;
+                s_geo2[i1] = geo2;
+                s_col[i1] = rb;
+                s_gid[i1] = gb;
+                s_mask[i1] = (uint8_t)strip_mask<kWarps>(geo, geo2, L.sx, L.hx, L.sy0, 2.f * kRPL, L.hy);
+            }
+        }
         __syncthreads();
-        // skip the slots this warp's pixels never reached
+        // this warp's slots: reached by one of its pixels (entry below
+        // warp_max) and not culled for its strip
         const uint32_t k0 = bend > warp_max ? min(bend - warp_max, cnt) : 0u;
-        for (uint32_t k = k0; k < cnt; k++) {
+        const uint32_t n = compact_slots<kB>(s_mask, k0, cnt, warp, lane, s_list[warp]);
+        for (uint32_t t = 0; t < n; t++) {
+            const uint32_t k = s_list[warp][t];
             const uint32_t j = bend - 1 - k;
             const float4 geo = s_geo[k], geo2 = s_geo2[k];
-            if (kCull && culled(geo, geo2, L)) continue;
             const ColTerms ct = col_terms(geo, L.fx);
             // The exponent at the lane's rows, two rows per paired instruction
             // (each half rounded exactly as the forward's scalar evaluation,
@@ -572,7 +573,7 @@ cudaError_t launch_render_bwd(const CamConst &c, const gs_projected &proj, const
                               float *grad2d, cudaStream_t s) {
     const int tiles = c.tiles_x * c.tiles_y;
     prof_before("render_bwd", s);
-    k_render_bwd<GS_BWD_RPL, GS_BWD_CULL != 0><<<tiles, kTilePixels / GS_BWD_RPL, 0, s>>>(
+    k_render_bwd<GS_BWD_RPL><<<tiles, kTilePixels / GS_BWD_RPL, 0, s>>>(
         c, reinterpret_cast<const float4 *>(proj.xy_opacity_depth),
         reinterpret_cast<const float4 *>(proj.conic_radius), reinterpret_cast<const float4 *>(proj.rgb),
         bins.pair_gid, reinterpret_cast<const uint2 *>(bins.ranges), T_final, last, dL_dimage,
