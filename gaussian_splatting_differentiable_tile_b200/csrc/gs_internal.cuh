@@ -64,6 +64,7 @@ struct BinsLayout {
     size_t status, n_pairs, tickets, depth_hist, tile_hist;
     size_t ranges, depth_lb, scan_lb, tile_lb;
     size_t zero_bytes;
+    size_t tile_order;                              // [max_tiles] tiles, longest list first
     size_t keys_a, vals_a, keys_b, vals_b;          // depth sort, [max_n]
     size_t ptile_a, pgid_a, ptile_b, pgid_b;        // pair sort ping-pong, [max_pairs]
     size_t pair_tile, pair_gid;                     // result, [max_pairs]
@@ -95,6 +96,7 @@ constexpr BinsLayout bins_layout(int64_t max_n, int64_t max_pairs, int32_t max_t
     L.tile_lb = off;
     off = align_up(off + (size_t)kMaxTilePasses * L.tile_parts * kRadix * sizeof(uint32_t), 256);
     L.zero_bytes = off;
+    L.tile_order = off;   off = align_up(off + (size_t)max_tiles * sizeof(uint32_t), 256);
     size_t nb = align_up((size_t)max_n * sizeof(uint32_t), 256);
     size_t pb = align_up((size_t)max_pairs * sizeof(uint32_t), 256);
     L.keys_a = off;  off += nb;

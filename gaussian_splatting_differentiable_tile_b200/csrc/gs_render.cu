@@ -188,8 +188,8 @@ __device__ __forceinline__ bool eval_alpha(const float4 geo, const float4 geo2, 
 __global__ void __launch_bounds__(kTilePixels, 6)
 k_render_fwd(CamConst cam, const float4 *__restrict__ xyod, const float4 *__restrict__ conr,
              const float4 *__restrict__ rgb, const uint32_t *__restrict__ pair_gid,
-             const uint2 *__restrict__ ranges, float *__restrict__ image, float *__restrict__ T_final,
-             uint32_t *__restrict__ last) {
+             const uint2 *__restrict__ ranges, const uint32_t *__restrict__ order,
+             float *__restrict__ image, float *__restrict__ T_final, uint32_t *__restrict__ last) {
     constexpr int kWarps = kTilePixels / 32;
     __shared__ float4 s_geo[kBatch];
     __shared__ float4 s_geo2[kBatch];
@@ -197,7 +197,7 @@ k_render_fwd(CamConst cam, const float4 *__restrict__ xyod, const float4 *__rest
     __shared__ uint8_t s_mask[kBatch];
     __shared__ uint8_t s_list[kWarps][kBatch];
 
-    const int tile = blockIdx.x;
+    const int tile = (int)order[blockIdx.x];  // longest lists first
     const LaneGeom L = lane_geom<1>(cam, tile);
     const uint2 range = ranges[tile];
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
@@ -308,7 +308,8 @@ template <int kRPL>
 __global__ void __launch_bounds__(kTilePixels / kRPL, 56 / kRPL)
 k_render_bwd(CamConst cam, const float4 *__restrict__ xyod, const float4 *__restrict__ conr,
              const float4 *__restrict__ rgb, const uint32_t *__restrict__ pair_gid,
-             const uint2 *__restrict__ ranges, const float *__restrict__ T_final,
+             const uint2 *__restrict__ ranges, const uint32_t *__restrict__ order,
+             const float *__restrict__ T_final,
              const uint32_t *__restrict__ last, const float *__restrict__ dL_dimage,
              float *__restrict__ grad2d) {
     static_assert(kRPL % 2 == 0, "the backward works on pairs of rows");
@@ -324,7 +325,7 @@ k_render_bwd(CamConst cam, const float4 *__restrict__ xyod, const float4 *__rest
     __shared__ uint8_t s_list[kWarps][kB];
     __shared__ uint32_t s_max_last;
 
-    const int tile = blockIdx.x;
+    const int tile = (int)order[blockIdx.x];  // longest lists first
     const LaneGeom L = lane_geom<kRPL>(cam, tile);
     const uint2 range = ranges[tile];
     const bool col_in = L.px < cam.width;
@@ -556,6 +557,12 @@ k_l1(const float *__restrict__ image, const float *__restrict__ target, int64_t 
 
 }  // namespace
 
+// The tile order gs_bin_and_sort left in the bins' scratch.
+static const uint32_t *tile_order(const gs_bins &bins) {
+    const BinsLayout L = bins_layout(bins.max_n, bins.max_pairs, bins.max_tiles);
+    return reinterpret_cast<const uint32_t *>(static_cast<const char *>(bins.scratch) + L.tile_order);
+}
+
 cudaError_t launch_render_fwd(const CamConst &c, const gs_projected &proj, const gs_bins &bins,
                               float *image, float *T_final, uint32_t *last, cudaStream_t s) {
     const int tiles = c.tiles_x * c.tiles_y;
@@ -563,7 +570,8 @@ cudaError_t launch_render_fwd(const CamConst &c, const gs_projected &proj, const
     k_render_fwd<<<tiles, kTilePixels, 0, s>>>(
         c, reinterpret_cast<const float4 *>(proj.xy_opacity_depth),
         reinterpret_cast<const float4 *>(proj.conic_radius), reinterpret_cast<const float4 *>(proj.rgb),
-        bins.pair_gid, reinterpret_cast<const uint2 *>(bins.ranges), image, T_final, last);
+        bins.pair_gid, reinterpret_cast<const uint2 *>(bins.ranges), tile_order(bins), image, T_final,
+        last);
     prof_after(s);
     return cudaGetLastError();
 }
@@ -576,8 +584,8 @@ cudaError_t launch_render_bwd(const CamConst &c, const gs_projected &proj, const
     k_render_bwd<GS_BWD_RPL><<<tiles, kTilePixels / GS_BWD_RPL, 0, s>>>(
         c, reinterpret_cast<const float4 *>(proj.xy_opacity_depth),
         reinterpret_cast<const float4 *>(proj.conic_radius), reinterpret_cast<const float4 *>(proj.rgb),
-        bins.pair_gid, reinterpret_cast<const uint2 *>(bins.ranges), T_final, last, dL_dimage,
-        grad2d);
+        bins.pair_gid, reinterpret_cast<const uint2 *>(bins.ranges), tile_order(bins), T_final, last,
+        dL_dimage, grad2d);
     prof_after(s);
     return cudaGetLastError();
 }

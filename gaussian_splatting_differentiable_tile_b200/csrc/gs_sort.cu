@@ -524,6 +524,50 @@ k_ranges(const uint32_t *__restrict__ ptile, const uint64_t *__restrict__ n_pair
     }
 }
 
+// Order in which the blend kernels take the tiles: longest list first, so
+// that the heaviest tiles do not start last and leave SMs idle at the end
+// (a counting sort on list length in steps of 4 entries, one CTA; the order
+// within a bucket is arbitrary).
+constexpr int kOrderBuckets = 1024;
+__global__ void __launch_bounds__(kOrderBuckets)
+k_tile_order(const uint32_t *__restrict__ ranges, int tiles, uint32_t *__restrict__ order) {
+    __shared__ uint32_t s_off[kOrderBuckets];
+    __shared__ uint32_t s_warp[kOrderBuckets / 32];
+    const int t = threadIdx.x;
+    auto bucket = [&](int i) {
+        const uint32_t len = ranges[2 * (size_t)i + 1] - ranges[2 * (size_t)i];
+        return kOrderBuckets - 1 - (int)min(len >> 2, (uint32_t)(kOrderBuckets - 1));
+    };
+    s_off[t] = 0;
+    __syncthreads();
+    for (int i = t; i < tiles; i += kOrderBuckets) atomicAdd(&s_off[bucket(i)], 1u);
+    __syncthreads();
+    // exclusive scan of the bucket counts
+    const uint32_t v = s_off[t];
+    uint32_t x = v;
+    const int lane = t & 31, w = t >> 5;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+        const uint32_t y = __shfl_up_sync(0xffffffffu, x, o);
+        if (lane >= o) x += y;
+    }
+    if (lane == 31) s_warp[w] = x;
+    __syncthreads();
+    if (w == 0) {
+        uint32_t z = s_warp[lane];
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+            const uint32_t y = __shfl_up_sync(0xffffffffu, z, o);
+            if (lane >= o) z += y;
+        }
+        s_warp[lane] = z;
+    }
+    __syncthreads();
+    s_off[t] = x - v + (w > 0 ? s_warp[w - 1] : 0u);
+    __syncthreads();
+    for (int i = t; i < tiles; i += kOrderBuckets) order[atomicAdd(&s_off[bucket(i)], 1u)] = (uint32_t)i;
+}
+
 int num_sms() {
     static int sms = 0;
     if (sms == 0) {
@@ -549,9 +593,15 @@ cudaError_t launch_bin_and_sort(const CamConst &c, int64_t n, const gs_projected
     uint32_t *ranges = U32(L.ranges);
     const int tiles = c.tiles_x * c.tiles_y;
 
+    auto tile_order = [&]() {
+        prof_before("tile_order", s);
+        k_tile_order<<<1, kOrderBuckets, 0, s>>>(ranges, tiles, U32(L.tile_order));
+        prof_after(s);
+        return cudaGetLastError();
+    };
     cudaError_t e = cudaMemsetAsync(base, 0, L.zero_bytes, s);
     if (e != cudaSuccess) return e;
-    if (n == 0) return cudaSuccess;  // K = 0, all ranges empty
+    if (n == 0) return tile_order();  // K = 0, all ranges empty
 
     const int sms = num_sms();
     const uint32_t nn = (uint32_t)n;
@@ -638,7 +688,8 @@ cudaError_t launch_bin_and_sort(const CamConst &c, int64_t n, const gs_projected
         k_ranges<<<blocks, 256, 0, s>>>(bins.pair_tile, n_pairs, ranges, status);
         prof_after(s);
     }
-    return cudaGetLastError();
+    // 6. the blend kernels' tile order
+    return tile_order();
 }
 
 }  // namespace gs

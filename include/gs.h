@@ -181,6 +181,9 @@ int gs_project(const gs_camera *cam, int64_t n, const gs_params *params, const g
  * tile at the scanned offsets, sorts the pairs stably by tile (LSD radix over
  * the used tile-id bits only), and writes each tile's range.  The result is
  * the pair order of the 64-bit key (tile << 32 | depth bits) with ties by id.
+ * It also leaves in bins->scratch the order in which the blend kernels take
+ * the tiles (longest list first); the render calls need bins filled by this
+ * call.
  * Uses `proj` from gs_project (or any records in that layout): binning reads
  * each record's depth and its rectangle (clamped to the tile grid; `count` is
  * not read), so no record can produce a tile id outside the grid.
@@ -194,7 +197,8 @@ int gs_project(const gs_camera *cam, int64_t n, const gs_params *params, const g
 int gs_bin_and_sort(const gs_camera *cam, int64_t n, const gs_projected *proj,
                     const gs_bins *bins, int64_t *n_pairs_host, void *stream);
 
-/* Forward blend ([GSP] s5; [WEEK] blend), one CTA per 16x16 tile: for each
+/* Forward blend ([GSP] s5; [WEEK] blend), one CTA per 16x16 tile (tiles
+ * taken in the order gs_bin_and_sort left in bins->scratch): for each
  * pixel, its tile's pairs in order, sigma as above at (j + 0.5, i + 0.5),
  * alpha = min(0.99, o exp(-sigma)); skip if sigma < 0 or alpha < 1/255;
  * stop (without adding) once T (1 - alpha) < 1e-4; C += c alpha T.
