@@ -216,6 +216,25 @@ def test_render_fwd_student_sampled_tiles():
     _assert_fwd(cam, bins, image, T, last, ref, sel)
 
 
+@pytest.mark.parametrize("scene", ["ragged", "student3k"])
+def test_render_stats_match_oracle_counts(scene):
+    """gs_render_stats counts the work the method must do: entries visited up
+    to and including each pixel's stopping entry, entries added, and the
+    backward's walk [start, last).  The oracle counts the same per pixel;
+    pixels whose decisions sit within the stated margins may differ."""
+    cam, params = SCENES[scene]()
+    rec, proj, bins, K, image, T, last, ref = _fwd_stage_fed(cam, params)
+    n = params["means"].shape[0]
+    st = G.gs_render_stats(cam, n, proj, bins, torch.from_numpy(last).cuda())
+    amb = ambiguous_pixels(ref)
+    slack = int(ref["e_visit"][amb].sum()) + int(amb.sum())
+    assert st["pixels"] == cam.width * cam.height
+    assert abs(st["fwd_visits"] - int(ref["e_visit"].sum())) <= slack
+    assert abs(st["contributions"] - int(ref["e_contrib"].sum())) <= slack
+    assert abs(st["bwd_visits"] - int(ref["n_walk"].sum())) <= slack
+    assert st["contributions"] > 0 and st["fwd_visits"] >= st["contributions"]
+
+
 def test_render_fwd_background_and_white_invariant():
     cam, params = SCENES["ragged"]()
     cam.bg = (0.2, 0.4, 0.6)
