@@ -62,9 +62,11 @@ struct CamConst {
 // by one memset at the start of every gs_bin_and_sort.
 struct BinsLayout {
     size_t status, n_pairs, tickets, depth_hist, tile_hist;
+    size_t tile_count;                              // [max_tiles] pairs per tile, then emit cursors
     size_t ranges, depth_lb, scan_lb, tile_lb;
     size_t zero_bytes;
     size_t tile_order;                              // [max_tiles] tiles, longest list first
+    size_t bin_hist;                                // per-CTA tile counts, then offsets
     size_t keys_a, vals_a, keys_b, vals_b;          // depth sort, [max_n]
     size_t ptile_a, pgid_a, ptile_b, pgid_b;        // pair sort ping-pong, [max_pairs]
     size_t pair_tile, pair_gid;                     // result, [max_pairs]
@@ -85,6 +87,7 @@ constexpr BinsLayout bins_layout(int64_t max_n, int64_t max_pairs, int32_t max_t
     L.depth_hist = off;   off += kMaxDepthPasses * kRadix * sizeof(uint32_t);
     L.tile_hist = off;    off += kMaxTilePasses * kRadix * sizeof(uint32_t);
     off = align_up(off, 256);
+    L.tile_count = off;   off = align_up(off + (size_t)max_tiles * sizeof(uint32_t), 256);
     L.ranges = off;       off = align_up(off + (size_t)max_tiles * 2 * sizeof(uint32_t), 256);
     L.depth_parts = (max_n + kSortPart - 1) / kSortPart;
     L.scan_parts = (max_n + kScanPart - 1) / kScanPart;
@@ -97,6 +100,11 @@ constexpr BinsLayout bins_layout(int64_t max_n, int64_t max_pairs, int32_t max_t
     off = align_up(off + (size_t)kMaxTilePasses * L.tile_parts * kRadix * sizeof(uint32_t), 256);
     L.zero_bytes = off;
     L.tile_order = off;   off = align_up(off + (size_t)max_tiles * sizeof(uint32_t), 256);
+    L.bin_hist = off;
+    {
+        const int64_t h = (int64_t)160 * max_tiles, cap = (int64_t)1 << 22;  // per-CTA tile counts
+        off = align_up(off + (size_t)(h < cap ? h : cap) * sizeof(uint32_t), 256);
+    }
     size_t nb = align_up((size_t)max_n * sizeof(uint32_t), 256);
     size_t pb = align_up((size_t)max_pairs * sizeof(uint32_t), 256);
     L.keys_a = off;  off += nb;

@@ -568,6 +568,433 @@ k_tile_order(const uint32_t *__restrict__ ranges, int tiles, uint32_t *__restric
     for (int i = t; i < tiles; i += kOrderBuckets) order[atomicAdd(&s_off[bucket(i)], 1u)] = (uint32_t)i;
 }
 
+// ---------------------------------------------------------------------
+// Per-tile binning.  A fixed set of CTAs splits the Gaussians into
+// contiguous ranges; each CTA counts its pairs per tile in shared memory and
+// writes its row of a [CTA][tile] count matrix (no contended global
+// atomics).  A column scan gives every (CTA, tile) its offset inside the
+// tile, a one-CTA scan gives the tile ranges, K and the tile order; each CTA
+// then emits its pairs at its offsets through shared-memory cursors (in
+// arbitrary order within the tile), and each tile's list is sorted by the
+// 64-bit key (depth bits << 32 | Gaussian id).  Keys are unique, so the
+// result is exactly the pair order of the global sort on
+// (tile << 32 | depth bits) with ties by id.
+
+#ifndef GS_BIN_LOCAL
+#define GS_BIN_LOCAL 1
+#endif
+
+constexpr int kBinThreads = 512;
+// The count matrix holds at most kBinHistCap entries: min(SMs, kBinCTAsMax,
+// kBinHistCap / tiles) CTAs share the Gaussians.
+constexpr int kBinCTAsMax = 160;
+constexpr int64_t kBinHistCap = 1 << 22;
+// Rectangles of at most this many tiles are handled by their own lane; larger
+// ones by the whole warp, one at a time.
+constexpr uint32_t kLaneTiles = 16;
+// Tile grids up to this size count in shared memory; larger ones in their
+// CTA's row of the global matrix.
+constexpr int kSmemTiles = 16384;
+// Size classes of the per-tile sort (256 keys per warp): up to
+// kTileSortShort keys (4 warps, two 8 KB shared-memory buffers), up to
+// kTileSortMid (32 warps, two 64 KB buffers), and longer lists in global
+// memory.
+constexpr int kShortWarps = 4, kMidWarps = 32;
+constexpr uint32_t kTileSortShort = 256u * kShortWarps;
+constexpr uint32_t kTileSortMid = 256u * kMidWarps;
+
+// Calls f(g, tile) for every pair of the Gaussians [g_begin, g_end), the
+// CTA's warps striding through the range 32 Gaussians at a time.
+template <typename F>
+__device__ __forceinline__ void for_each_pair(int g_begin, int g_end, const int4 *__restrict__ rect,
+                                              int tiles_x, int tiles_y, F f) {
+    const int lane = threadIdx.x & 31;
+    for (int g0 = g_begin + (int)(threadIdx.x & ~31u); g0 < g_end; g0 += (int)blockDim.x) {
+        const int g = g0 + lane;
+        int x0 = 0, y0 = 0, w = 1;
+        const uint32_t c = g < g_end ? rect_tiles(rect[g], tiles_x, tiles_y, x0, y0, w) : 0u;
+        if (c <= kLaneTiles) {
+            for (uint32_t k = 0; k < c; k++) {
+                const uint32_t dy = k / (uint32_t)w;
+                f(g, (y0 + (int)dy) * tiles_x + x0 + (int)(k - dy * (uint32_t)w));
+            }
+        }
+        uint32_t big = __ballot_sync(0xffffffffu, c > kLaneTiles);
+        while (big) {
+            const int src = __ffs(big) - 1;
+            big &= big - 1;
+            const int gb = __shfl_sync(0xffffffffu, g, src);
+            const uint32_t cb = __shfl_sync(0xffffffffu, c, src);
+            const int xb = __shfl_sync(0xffffffffu, x0, src), yb = __shfl_sync(0xffffffffu, y0, src);
+            const uint32_t wb = (uint32_t)__shfl_sync(0xffffffffu, w, src);
+            for (uint32_t k = lane; k < cb; k += 32) {
+                const uint32_t dy = k / wb;
+                f(gb, (yb + (int)dy) * tiles_x + xb + (int)(k - dy * wb));
+            }
+        }
+    }
+}
+
+__device__ __forceinline__ void cta_range(int n, int &g_begin, int &g_end) {
+    const int chunk = (n + (int)gridDim.x - 1) / (int)gridDim.x;
+    g_begin = min((int)blockIdx.x * chunk, n);
+    g_end = min(g_begin + chunk, n);
+}
+
+// Row blockIdx of the count matrix H[CTA][tile].
+__global__ void __launch_bounds__(kBinThreads)
+k_bin_count(int n, const int4 *__restrict__ rect, int tiles_x, int tiles_y, uint32_t *__restrict__ H) {
+    extern __shared__ uint32_t s_cnt[];
+    const int tiles = tiles_x * tiles_y;
+    uint32_t *row = H + (size_t)blockIdx.x * tiles;
+    const bool smem = tiles <= kSmemTiles;
+    uint32_t *cnt = smem ? s_cnt : row;
+    for (int t = threadIdx.x; t < tiles; t += kBinThreads) cnt[t] = 0;
+    __syncthreads();
+    int g_begin, g_end;
+    cta_range(n, g_begin, g_end);
+    for_each_pair(g_begin, g_end, rect, tiles_x, tiles_y, [&](int, int t) { atomicAdd(&cnt[t], 1u); });
+    __syncthreads();
+    if (smem)
+        for (int t = threadIdx.x; t < tiles; t += kBinThreads) row[t] = s_cnt[t];
+}
+
+// Per tile: exclusive scan down its column of H (in place) and the total.
+// A CTA takes 32 tiles (lane = tile, so every row access is coalesced) and
+// splits the rows among its 8 warps; each warp loads its rows at once.
+constexpr int kColRows = (kBinCTAsMax + 7) / 8;
+__global__ void __launch_bounds__(256)
+k_bin_colscan(int tiles, int ctas, uint32_t *__restrict__ H, uint32_t *__restrict__ totals) {
+    __shared__ uint32_t s_part[8][32];
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    const int t = blockIdx.x * 32 + lane;
+    const int per = (ctas + 7) / 8;
+    const int c0 = warp * per;
+    uint32_t v[kColRows];
+#pragma unroll
+    for (int k = 0; k < kColRows; k++) {
+        const int c = c0 + k;
+        v[k] = (k < per && c < ctas && t < tiles) ? H[(size_t)c * tiles + t] : 0u;
+    }
+    uint32_t sum = 0;
+#pragma unroll
+    for (int k = 0; k < kColRows; k++) {
+        const uint32_t x = v[k];
+        v[k] = sum;
+        sum += x;
+    }
+    s_part[warp][lane] = sum;
+    __syncthreads();
+    uint32_t base = 0, total = 0;
+#pragma unroll
+    for (int w = 0; w < 8; w++) {
+        const uint32_t x = s_part[w][lane];
+        base += w < warp ? x : 0u;
+        total += x;
+    }
+#pragma unroll
+    for (int k = 0; k < kColRows; k++) {
+        const int c = c0 + k;
+        if (k < per && c < ctas && t < tiles) H[(size_t)c * tiles + t] = base + v[k];
+    }
+    if (warp == 0 && t < tiles) totals[t] = total;
+}
+
+// One CTA: ranges from the exclusive scan of the tile totals (all empty if K
+// exceeds the capacity, with GS_ERR_CAPACITY recorded), K, and the tile
+// order (longest list first, by a counting sort on length in steps of 4).
+constexpr int kScanTilesThreads = 1024;
+__global__ void __launch_bounds__(kScanTilesThreads)
+k_tile_scan(int tiles, const uint32_t *__restrict__ totals, uint64_t max_pairs,
+            uint32_t *__restrict__ ranges, uint32_t *__restrict__ order, uint64_t *__restrict__ n_pairs,
+            int32_t *__restrict__ status) {
+    __shared__ uint64_t s_w64[kScanTilesThreads / 32];
+    __shared__ uint32_t s_off[kScanTilesThreads];
+    __shared__ uint32_t s_w32[kScanTilesThreads / 32];
+    __shared__ int s_ok;
+    const int t = threadIdx.x, lane = t & 31, w = t >> 5;
+    const int chunk = (tiles + kScanTilesThreads - 1) / kScanTilesThreads;
+    const int lo = min(t * chunk, tiles), hi = min(lo + chunk, tiles);
+    uint64_t sum = 0;
+    for (int i = lo; i < hi; i++) sum += totals[i];
+    uint64_t x = sum;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+        const uint64_t y = __shfl_up_sync(0xffffffffu, x, o);
+        if (lane >= o) x += y;
+    }
+    if (lane == 31) s_w64[w] = x;
+    __syncthreads();
+    if (w == 0) {
+        uint64_t z = s_w64[lane];
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+            const uint64_t y = __shfl_up_sync(0xffffffffu, z, o);
+            if (lane >= o) z += y;
+        }
+        s_w64[lane] = z;
+        if (lane == 31) {
+            *n_pairs = z;
+            const bool ok = z <= max_pairs;
+            if (!ok) set_status(status, GS_ERR_CAPACITY);
+            s_ok = ok && *(volatile int32_t *)status == 0;
+        }
+    }
+    __syncthreads();
+    uint64_t off = x - sum + (w > 0 ? s_w64[w - 1] : 0ull);
+    const bool ok = s_ok;
+    for (int i = lo; i < hi; i++) {
+        const uint32_t c = totals[i];
+        const bool some = ok && c > 0;  // empty tiles are [0, 0)
+        ranges[2 * (size_t)i] = some ? (uint32_t)off : 0u;
+        ranges[2 * (size_t)i + 1] = some ? (uint32_t)(off + c) : 0u;
+        off += c;
+    }
+    auto bucket = [&](int i) {
+        const uint32_t len = ranges[2 * (size_t)i + 1] - ranges[2 * (size_t)i];
+        return kScanTilesThreads - 1 - (int)min(len >> 2, (uint32_t)(kScanTilesThreads - 1));
+    };
+    s_off[t] = 0;
+    __syncthreads();
+    for (int i = lo; i < hi; i++) atomicAdd(&s_off[bucket(i)], 1u);
+    __syncthreads();
+    const uint32_t v = s_off[t];
+    uint32_t y = v;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+        const uint32_t z = __shfl_up_sync(0xffffffffu, y, o);
+        if (lane >= o) y += z;
+    }
+    if (lane == 31) s_w32[w] = y;
+    __syncthreads();
+    if (w == 0) {
+        uint32_t z = s_w32[lane];
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+            const uint32_t q = __shfl_up_sync(0xffffffffu, z, o);
+            if (lane >= o) z += q;
+        }
+        s_w32[lane] = z;
+    }
+    __syncthreads();
+    s_off[t] = y - v + (w > 0 ? s_w32[w - 1] : 0u);
+    __syncthreads();
+    for (int i = lo; i < hi; i++) order[atomicAdd(&s_off[bucket(i)], 1u)] = (uint32_t)i;
+}
+
+// Each CTA emits the pairs of its Gaussians: cursor = tile start + the CTA's
+// column offset, advanced by shared-memory atomics.  Nothing is written once
+// an error has been recorded.
+__global__ void __launch_bounds__(kBinThreads)
+k_bin_emit(int n, const int4 *__restrict__ rect, int tiles_x, int tiles_y, const uint32_t *__restrict__ ranges,
+           uint32_t *__restrict__ H, uint32_t *__restrict__ pair_gid, const int32_t *__restrict__ status) {
+    extern __shared__ uint32_t s_cur[];
+    if (*(volatile const int32_t *)status != 0) return;
+    const int tiles = tiles_x * tiles_y;
+    uint32_t *row = H + (size_t)blockIdx.x * tiles;
+    const bool smem = tiles <= kSmemTiles;
+    uint32_t *cur = smem ? s_cur : row;
+    for (int t = threadIdx.x; t < tiles; t += kBinThreads) cur[t] = ranges[2 * (size_t)t] + row[t];
+    __syncthreads();
+    int g_begin, g_end;
+    cta_range(n, g_begin, g_end);
+    for_each_pair(g_begin, g_end, rect, tiles_x, tiles_y,
+                  [&](int g, int t) { pair_gid[atomicAdd(&cur[t], 1u)] = (uint32_t)g; });
+}
+
+__device__ __forceinline__ uint64_t pair_key(const float4 *__restrict__ xyod, uint32_t g) {
+    return ((uint64_t)__float_as_uint(xyod[g].w) << 32) | g;
+}
+
+__device__ __forceinline__ uint32_t order_bucket(uint32_t len) {
+    return min(len >> 2, (uint32_t)(kScanTilesThreads - 1));
+}
+
+// Sorts the 256 keys of a warp ascending in registers: lane l holds
+// elements 8l .. 8l + 7 in k[0..7].  Bitonic network: strides below 8 swap
+// within the lane, larger strides exchange with lane ^ (stride / 8).
+__device__ __forceinline__ void warp_bitonic_256(uint64_t (&k)[8], int lane) {
+#pragma unroll
+    for (int kk = 2; kk <= 256; kk <<= 1) {
+#pragma unroll
+        for (int j = kk >> 1; j > 0; j >>= 1) {
+            if (j >= 8) {
+#pragma unroll
+                for (int r = 0; r < 8; r++) {
+                    const int i = lane * 8 + r;
+                    const uint64_t o = __shfl_xor_sync(0xffffffffu, k[r], j >> 3);
+                    const bool take_min = ((i & j) == 0) == ((i & kk) == 0);
+                    k[r] = take_min ? (k[r] < o ? k[r] : o) : (k[r] < o ? o : k[r]);
+                }
+            } else {
+#pragma unroll
+                for (int r = 0; r < 8; r++) {
+                    if (r & j) continue;
+                    const int i = lane * 8 + r;
+                    const uint64_t x = k[r], y = k[r | j];
+                    if ((x > y) == ((i & kk) == 0)) {
+                        k[r] = y;
+                        k[r | j] = x;
+                    }
+                }
+            }
+        }
+    }
+}
+
+// Number of keys in the sorted run a[0, n) below x (strictly, or at most x).
+template <bool kInclusive>
+__device__ __forceinline__ int run_rank(const uint64_t *a, int n, uint64_t x) {
+    int lo = 0, hi = n;
+    while (lo < hi) {
+        const int mid = (lo + hi) >> 1;
+        const bool left = kInclusive ? a[mid] <= x : a[mid] < x;
+        if (left) lo = mid + 1;
+        else hi = mid;
+    }
+    return lo;
+}
+
+// Tile lists in (lo, hi], hi = 256 kWarps: sorted by one CTA each.  Warp w
+// sorts keys [256 w, 256 w + 256) in registers; the runs are then merged
+// pairwise in shared memory (each key's output position is its index plus
+// its rank in the other run).  With `persistent` a small grid walks the tile
+// order (longest first) and stops at the first tile whose length bucket
+// lies below lo's; otherwise CTA b takes the b-th tile of the order.
+template <int kWarps>
+__global__ void __launch_bounds__(kWarps * 32)
+k_tile_sort(const uint32_t *__restrict__ ranges, const uint32_t *__restrict__ order, int tiles,
+            const float4 *__restrict__ xyod, uint32_t *__restrict__ pair_gid,
+            uint32_t *__restrict__ pair_tile, uint32_t lo, int persistent) {
+    constexpr int kThreads = kWarps * 32;
+    constexpr uint32_t kHi = 256u * kWarps;
+    extern __shared__ uint64_t s_buf[];
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    const int step = persistent ? (int)gridDim.x : tiles;
+    for (int b = blockIdx.x; b < tiles; b += step) {
+        const uint32_t tile = order[b];
+        const uint32_t start = ranges[2 * (size_t)tile], end = ranges[2 * (size_t)tile + 1];
+        const uint32_t L = end - start;
+        if (persistent && order_bucket(L) < order_bucket(lo)) break;
+        if (L <= lo || L > kHi) continue;
+        const int chunks = (int)((L + 255) / 256);
+        int runs = 1;
+        while (runs < chunks) runs <<= 1;
+        if (warp < runs) {
+            uint64_t k[8];
+#pragma unroll
+            for (int r = 0; r < 8; r++) {
+                const uint32_t idx = (uint32_t)(warp * 256 + lane * 8 + r);
+                k[r] = idx < L ? pair_key(xyod, pair_gid[start + idx]) : ~0ull;
+            }
+            if (warp < chunks) warp_bitonic_256(k, lane);
+#pragma unroll
+            for (int r = 0; r < 8; r++) s_buf[warp * 256 + lane * 8 + r] = k[r];
+        }
+        __syncthreads();
+        uint64_t *src = s_buf, *dst = s_buf + kHi;
+        const int total = runs * 256;
+        for (int run = 256; run < total; run <<= 1) {
+            for (int i = threadIdx.x; i < total; i += kThreads) {
+                const int base = i & ~(2 * run - 1), off = i - base;
+                const uint64_t x = src[i];
+                const int pos = off < run ? off + run_rank<false>(src + base + run, run, x)
+                                          : (off - run) + run_rank<true>(src + base, run, x);
+                dst[base + pos] = x;
+            }
+            __syncthreads();
+            uint64_t *t = src;
+            src = dst;
+            dst = t;
+        }
+        for (uint32_t i = threadIdx.x; i < L; i += kThreads) {
+            pair_gid[start + i] = (uint32_t)src[i];
+            pair_tile[start + i] = tile;
+        }
+        __syncthreads();
+    }
+}
+
+// Tiles longer than the shared-memory sort holds: one CTA per tile runs an
+// LSD radix sort of the tile's keys in global memory (8-bit digits: four
+// passes over the id, then four over the depth bits; each pass stable, in
+// chunks of 256 ranked with warp ballots), through scratch arrays at the
+// same offsets as the tile's range.
+__global__ void __launch_bounds__(256)
+k_tile_sort_long(const uint32_t *__restrict__ ranges, const uint32_t *__restrict__ order, int tiles,
+                 const float4 *__restrict__ xyod, uint32_t *__restrict__ pair_gid,
+                 uint32_t *__restrict__ pair_tile, uint32_t lo, uint32_t *__restrict__ ka,
+                 uint32_t *__restrict__ va, uint32_t *__restrict__ kb, uint32_t *__restrict__ vb) {
+    __shared__ uint32_t s_base[kRadix];
+    __shared__ uint32_t s_wc[8][kRadix];
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    for (int b = blockIdx.x; b < tiles; b += gridDim.x) {
+        const uint32_t tile = order[b];
+        const uint32_t start = ranges[2 * (size_t)tile], end = ranges[2 * (size_t)tile + 1];
+        if (order_bucket(end - start) < order_bucket(lo)) break;
+        if (end - start <= lo) continue;
+        for (uint32_t i = start + tid; i < end; i += 256) {
+            const uint32_t g = pair_gid[i];
+            ka[i] = __float_as_uint(xyod[g].w);
+            va[i] = g;
+        }
+        __syncthreads();
+        uint32_t *sk = ka, *sv = va, *dk = kb, *dv = vb;
+        for (int pass = 0; pass < 8; pass++) {
+            const bool on_id = pass < 4;
+            const int shift = 8 * (pass & 3);
+            s_base[tid] = 0;
+            __syncthreads();
+            for (uint32_t i = start + tid; i < end; i += 256)
+                atomicAdd(&s_base[((on_id ? sv[i] : sk[i]) >> shift) & 0xFFu], 1u);
+            __syncthreads();
+            if (tid == 0) {  // exclusive scan, in place
+                uint32_t acc = start;
+                for (int d = 0; d < kRadix; d++) {
+                    const uint32_t c = s_base[d];
+                    s_base[d] = acc;
+                    acc += c;
+                }
+            }
+            __syncthreads();
+            for (uint32_t c0 = start; c0 < end; c0 += 256) {
+                const uint32_t i = c0 + tid;
+                const bool in = i < end;
+                const uint32_t key = in ? sk[i] : 0u, val = in ? sv[i] : 0u;
+                const uint32_t d = in ? ((on_id ? val : key) >> shift) & 0xFFu : (uint32_t)kRadix;
+                for (int k = tid; k < 8 * kRadix; k += 256) (&s_wc[0][0])[k] = 0;
+                __syncthreads();
+                const uint32_t peers = digit_peers(d, 8);
+                if (in && lane == __ffs(peers) - 1) s_wc[warp][d] = __popc(peers);
+                __syncthreads();
+                uint32_t acc = 0;  // per digit (thread = digit): exclusive over warps
+                for (int ww = 0; ww < 8; ww++) {
+                    const uint32_t c = s_wc[ww][tid];
+                    s_wc[ww][tid] = acc;
+                    acc += c;
+                }
+                __syncthreads();
+                if (in) {
+                    const uint32_t pos = s_base[d] + s_wc[warp][d] + __popc(peers & lanemask_lt());
+                    dk[pos] = key;
+                    dv[pos] = val;
+                }
+                __syncthreads();
+                s_base[tid] += acc;
+                __syncthreads();
+            }
+            uint32_t *t0 = sk, *t1 = sv;
+            sk = dk; sv = dv; dk = t0; dv = t1;
+            __syncthreads();
+        }
+        for (uint32_t i = start + tid; i < end; i += 256) {
+            pair_gid[i] = sv[i];
+            pair_tile[i] = tile;
+        }
+        __syncthreads();
+    }
+}
+
 int num_sms() {
     static int sms = 0;
     if (sms == 0) {
@@ -601,6 +1028,55 @@ cudaError_t launch_bin_and_sort(const CamConst &c, int64_t n, const gs_projected
     };
     cudaError_t e = cudaMemsetAsync(base, 0, L.zero_bytes, s);
     if (e != cudaSuccess) return e;
+#if GS_BIN_LOCAL
+    {
+        const int sms = num_sms();
+        uint32_t *H = U32(L.bin_hist);
+        uint32_t *totals = U32(L.tile_count);
+        const int4 *rect = reinterpret_cast<const int4 *>(proj.rect);
+        const float4 *xyod = reinterpret_cast<const float4 *>(proj.xy_opacity_depth);
+        uint32_t *order = U32(L.tile_order);
+        int64_t ctas64 = std::min<int64_t>((int64_t)sms, (int64_t)kBinCTAsMax);
+        ctas64 = std::min<int64_t>(ctas64, kBinHistCap / tiles);
+        const int ctas = (int)std::max<int64_t>(1, ctas64);
+        const size_t cnt_smem = tiles <= kSmemTiles ? (size_t)tiles * sizeof(uint32_t) : 0;
+        static bool attr = [] {
+            cudaFuncSetAttribute(k_bin_count, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 (int)(kSmemTiles * sizeof(uint32_t)));
+            cudaFuncSetAttribute(k_bin_emit, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 (int)(kSmemTiles * sizeof(uint32_t)));
+            cudaFuncSetAttribute(k_tile_sort<kMidWarps>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 (int)(2 * kTileSortMid * sizeof(uint64_t)));
+            return true;
+        }();
+        (void)attr;
+        prof_before("bin_count", s);
+        k_bin_count<<<ctas, kBinThreads, cnt_smem, s>>>((int)n, rect, c.tiles_x, c.tiles_y, H);
+        k_bin_colscan<<<(tiles + 31) / 32, 256, 0, s>>>(tiles, ctas, H, totals);
+        prof_after(s);
+        prof_before("tile_scan", s);
+        k_tile_scan<<<1, kScanTilesThreads, 0, s>>>(tiles, totals, (uint64_t)bins.max_pairs, ranges, order,
+                                                    n_pairs, status);
+        prof_after(s);
+        if (n > 0) {
+            prof_before("emit", s);
+            k_bin_emit<<<ctas, kBinThreads, cnt_smem, s>>>((int)n, rect, c.tiles_x, c.tiles_y, ranges, H,
+                                                           bins.pair_gid, status);
+            prof_after(s);
+            const int few = std::min(tiles, sms);
+            prof_before("tile_sort", s);
+            k_tile_sort<kShortWarps><<<tiles, kShortWarps * 32, 2 * kTileSortShort * sizeof(uint64_t), s>>>(
+                ranges, order, tiles, xyod, bins.pair_gid, bins.pair_tile, 0u, 0);
+            k_tile_sort<kMidWarps><<<few, kMidWarps * 32, 2 * kTileSortMid * sizeof(uint64_t), s>>>(
+                ranges, order, tiles, xyod, bins.pair_gid, bins.pair_tile, kTileSortShort, 1);
+            k_tile_sort_long<<<few, 256, 0, s>>>(ranges, order, tiles, xyod, bins.pair_gid, bins.pair_tile,
+                                                 kTileSortMid, U32(L.ptile_a), U32(L.pgid_a),
+                                                 U32(L.ptile_b), U32(L.pgid_b));
+            prof_after(s);
+        }
+        return cudaGetLastError();
+    }
+#endif
     if (n == 0) return tile_order();  // K = 0, all ranges empty
 
     const int sms = num_sms();

@@ -126,6 +126,27 @@ def test_bin_and_sort_tile_bit_widths(W, H):
     _check_bins(cam, rec, n, bins, K)
 
 
+@pytest.mark.parametrize("n", [900, 5000, 20000])
+def test_bin_and_sort_long_tile_lists(n):
+    """Every Gaussian covers the few tiles of a 48 x 32 image, so each tile's
+    list has about n entries: the shared-memory sort of short and of long
+    lists, and the global-memory sort beyond 16384 entries; a quarter of the
+    depths tie."""
+    cam = Camera(np.eye(4), 20.0, 20.0, 24.0, 16.0, 48, 32)
+    rng = np.random.default_rng(n)
+    params = {"means": np.column_stack([rng.uniform(-.3, .3, n), rng.uniform(-.3, .3, n), rng.uniform(2, 4, n)]),
+              "log_scales": rng.normal(-0.5, 0.2, (n, 3)), "quats": rng.normal(size=(n, 4)),
+              "opacity_logits": rng.normal(0, 1, n), "colors": rng.uniform(0, 1, (n, 3))}
+    rec = oracle_records(params, cam)
+    tie = rng.random(n) < 0.25
+    rec["depth32"] = np.where(tie, np.float32(3.0), rec["depth32"]).astype(np.float32)
+    proj = fill_projected(rec, n)
+    bins, K = gpu_bin(cam, n, proj, max_pairs=int(rec["count"].sum()) + 16)
+    r = bins.ranges.cpu().numpy()[:cam.tiles]
+    assert (r[:, 1] - r[:, 0]).max() > 0.8 * n
+    _check_bins(cam, rec, n, bins, K)
+
+
 def test_bin_and_sort_capacity_error_and_async_status():
     cam, params = SCENES["tiny"]()
     n = params["means"].shape[0]
