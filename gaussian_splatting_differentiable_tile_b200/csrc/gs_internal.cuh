@@ -102,7 +102,7 @@ constexpr BinsLayout bins_layout(int64_t max_n, int64_t max_pairs, int32_t max_t
     L.tile_order = off;   off = align_up(off + (size_t)max_tiles * sizeof(uint32_t), 256);
     L.bin_hist = off;
     {
-        const int64_t h = (int64_t)160 * max_tiles, cap = (int64_t)1 << 22;  // per-CTA tile counts
+        const int64_t h = (int64_t)320 * max_tiles, cap = (int64_t)1 << 22;  // per-CTA tile counts
         off = align_up(off + (size_t)(h < cap ? h : cap) * sizeof(uint32_t), 256);
     }
     size_t nb = align_up((size_t)max_n * sizeof(uint32_t), 256);

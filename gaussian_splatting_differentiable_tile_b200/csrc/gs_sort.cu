@@ -587,7 +587,7 @@ k_tile_order(const uint32_t *__restrict__ ranges, int tiles, uint32_t *__restric
 constexpr int kBinThreads = 512;
 // The count matrix holds at most kBinHistCap entries: min(SMs, kBinCTAsMax,
 // kBinHistCap / tiles) CTAs share the Gaussians.
-constexpr int kBinCTAsMax = 160;
+constexpr int kBinCTAsMax = 320;
 constexpr int64_t kBinHistCap = 1 << 22;
 // Rectangles of at most this many tiles are handled by their own lane; larger
 // ones by the whole warp, one at a time.
@@ -596,40 +596,50 @@ constexpr uint32_t kLaneTiles = 16;
 // CTA's row of the global matrix.
 constexpr int kSmemTiles = 16384;
 // Size classes of the per-tile sort (256 keys per warp): up to
-// kTileSortShort keys (4 warps, two 8 KB shared-memory buffers), up to
-// kTileSortMid (32 warps, two 64 KB buffers), and longer lists in global
-// memory.
+// kTileSortShort keys (4 warps), up to kTileSortMid (32 warps, two 64 KB
+// shared-memory buffers), and longer lists in global memory.
 constexpr int kShortWarps = 4, kMidWarps = 32;
 constexpr uint32_t kTileSortShort = 256u * kShortWarps;
 constexpr uint32_t kTileSortMid = 256u * kMidWarps;
 
 // Calls f(g, tile) for every pair of the Gaussians [g_begin, g_end), the
-// CTA's warps striding through the range 32 Gaussians at a time.
+// CTA's warps striding through the range 32 Gaussians at a time, four
+// groups per round (their rectangles loaded together).
 template <typename F>
 __device__ __forceinline__ void for_each_pair(int g_begin, int g_end, const int4 *__restrict__ rect,
                                               int tiles_x, int tiles_y, F f) {
+    constexpr int kGroups = 4;
     const int lane = threadIdx.x & 31;
-    for (int g0 = g_begin + (int)(threadIdx.x & ~31u); g0 < g_end; g0 += (int)blockDim.x) {
-        const int g = g0 + lane;
-        int x0 = 0, y0 = 0, w = 1;
-        const uint32_t c = g < g_end ? rect_tiles(rect[g], tiles_x, tiles_y, x0, y0, w) : 0u;
-        if (c <= kLaneTiles) {
-            for (uint32_t k = 0; k < c; k++) {
-                const uint32_t dy = k / (uint32_t)w;
-                f(g, (y0 + (int)dy) * tiles_x + x0 + (int)(k - dy * (uint32_t)w));
-            }
+    for (int g0 = g_begin + (int)(threadIdx.x & ~31u); g0 < g_end; g0 += kGroups * (int)blockDim.x) {
+        int4 rc[kGroups];
+#pragma unroll
+        for (int u = 0; u < kGroups; u++) {
+            const int g = g0 + u * (int)blockDim.x + lane;
+            rc[u] = g < g_end ? rect[g] : make_int4(0, 0, -1, -1);
         }
-        uint32_t big = __ballot_sync(0xffffffffu, c > kLaneTiles);
-        while (big) {
-            const int src = __ffs(big) - 1;
-            big &= big - 1;
-            const int gb = __shfl_sync(0xffffffffu, g, src);
-            const uint32_t cb = __shfl_sync(0xffffffffu, c, src);
-            const int xb = __shfl_sync(0xffffffffu, x0, src), yb = __shfl_sync(0xffffffffu, y0, src);
-            const uint32_t wb = (uint32_t)__shfl_sync(0xffffffffu, w, src);
-            for (uint32_t k = lane; k < cb; k += 32) {
-                const uint32_t dy = k / wb;
-                f(gb, (yb + (int)dy) * tiles_x + xb + (int)(k - dy * wb));
+#pragma unroll
+        for (int u = 0; u < kGroups; u++) {
+            const int g = g0 + u * (int)blockDim.x + lane;
+            int x0 = 0, y0 = 0, w = 1;
+            const uint32_t c = rect_tiles(rc[u], tiles_x, tiles_y, x0, y0, w);
+            if (c <= kLaneTiles) {
+                for (uint32_t k = 0; k < c; k++) {
+                    const uint32_t dy = k / (uint32_t)w;
+                    f(g, (y0 + (int)dy) * tiles_x + x0 + (int)(k - dy * (uint32_t)w));
+                }
+            }
+            uint32_t big = __ballot_sync(0xffffffffu, c > kLaneTiles);
+            while (big) {
+                const int src = __ffs(big) - 1;
+                big &= big - 1;
+                const int gb = __shfl_sync(0xffffffffu, g, src);
+                const uint32_t cb = __shfl_sync(0xffffffffu, c, src);
+                const int xb = __shfl_sync(0xffffffffu, x0, src), yb = __shfl_sync(0xffffffffu, y0, src);
+                const uint32_t wb = (uint32_t)__shfl_sync(0xffffffffu, w, src);
+                for (uint32_t k = lane; k < cb; k += 32) {
+                    const uint32_t dy = k / wb;
+                    f(gb, (yb + (int)dy) * tiles_x + xb + (int)(k - dy * wb));
+                }
             }
         }
     }
@@ -642,7 +652,7 @@ __device__ __forceinline__ void cta_range(int n, int &g_begin, int &g_end) {
 }
 
 // Row blockIdx of the count matrix H[CTA][tile].
-__global__ void __launch_bounds__(kBinThreads)
+__global__ void __launch_bounds__(kBinThreads, 2)
 k_bin_count(int n, const int4 *__restrict__ rect, int tiles_x, int tiles_y, uint32_t *__restrict__ H) {
     extern __shared__ uint32_t s_cnt[];
     const int tiles = tiles_x * tiles_y;
@@ -782,12 +792,18 @@ k_tile_scan(int tiles, const uint32_t *__restrict__ totals, uint64_t max_pairs,
     for (int i = lo; i < hi; i++) order[atomicAdd(&s_off[bucket(i)], 1u)] = (uint32_t)i;
 }
 
-// Each CTA emits the pairs of its Gaussians: cursor = tile start + the CTA's
-// column offset, advanced by shared-memory atomics.  Nothing is written once
-// an error has been recorded.
-__global__ void __launch_bounds__(kBinThreads)
-k_bin_emit(int n, const int4 *__restrict__ rect, int tiles_x, int tiles_y, const uint32_t *__restrict__ ranges,
-           uint32_t *__restrict__ H, uint32_t *__restrict__ pair_gid, const int32_t *__restrict__ status) {
+__device__ __forceinline__ uint64_t pair_key(const float4 *__restrict__ xyod, uint32_t g) {
+    return ((uint64_t)__float_as_uint(xyod[g].w) << 32) | g;
+}
+
+// Each CTA emits the pairs of its Gaussians as sort keys (depth bits << 32 |
+// id): cursor = tile start + the CTA's column offset, advanced by
+// shared-memory atomics.  Nothing is written once an error has been
+// recorded.
+__global__ void __launch_bounds__(kBinThreads, 2)
+k_bin_emit(int n, const int4 *__restrict__ rect, const float4 *__restrict__ xyod, int tiles_x, int tiles_y,
+           const uint32_t *__restrict__ ranges, uint32_t *__restrict__ H, uint64_t *__restrict__ keys,
+           const int32_t *__restrict__ status) {
     extern __shared__ uint32_t s_cur[];
     if (*(volatile const int32_t *)status != 0) return;
     const int tiles = tiles_x * tiles_y;
@@ -799,43 +815,43 @@ k_bin_emit(int n, const int4 *__restrict__ rect, int tiles_x, int tiles_y, const
     int g_begin, g_end;
     cta_range(n, g_begin, g_end);
     for_each_pair(g_begin, g_end, rect, tiles_x, tiles_y,
-                  [&](int g, int t) { pair_gid[atomicAdd(&cur[t], 1u)] = (uint32_t)g; });
-}
-
-__device__ __forceinline__ uint64_t pair_key(const float4 *__restrict__ xyod, uint32_t g) {
-    return ((uint64_t)__float_as_uint(xyod[g].w) << 32) | g;
+                  [&](int g, int t) { keys[atomicAdd(&cur[t], 1u)] = pair_key(xyod, (uint32_t)g); });
 }
 
 __device__ __forceinline__ uint32_t order_bucket(uint32_t len) {
     return min(len >> 2, (uint32_t)(kScanTilesThreads - 1));
 }
 
-// Sorts the 256 keys of a warp ascending in registers: lane l holds
-// elements 8l .. 8l + 7 in k[0..7].  Bitonic network: strides below 8 swap
-// within the lane, larger strides exchange with lane ^ (stride / 8).
-__device__ __forceinline__ void warp_bitonic_256(uint64_t (&k)[8], int lane) {
+// Sorts the keys of a warp ascending in registers: lane l holds elements
+// 8l .. 8l + 7 in k[0..7].  Bitonic network: strides below 8 swap within the
+// lane, larger strides exchange with lane ^ (stride / 8).  Stopping after
+// blocks of P (a power of two) sorts the first P keys, which is all that is
+// needed when the others are padding.
+__device__ __forceinline__ void warp_bitonic_256(uint64_t (&k)[8], int lane, int P = 256) {
+    const int l8 = lane << 3;  // element index of k[0]; k[r] is element l8 | r
 #pragma unroll
     for (int kk = 2; kk <= 256; kk <<= 1) {
+        if (kk > P) continue;  // the first P keys are sorted (the rest are padding)
 #pragma unroll
         for (int j = kk >> 1; j > 0; j >>= 1) {
             if (j >= 8) {
+                // partner in lane ^ (j / 8); directions depend on the lane only
+                const bool keep_min = ((l8 & j) == 0) == ((l8 & kk) == 0);
 #pragma unroll
                 for (int r = 0; r < 8; r++) {
-                    const int i = lane * 8 + r;
                     const uint64_t o = __shfl_xor_sync(0xffffffffu, k[r], j >> 3);
-                    const bool take_min = ((i & j) == 0) == ((i & kk) == 0);
-                    k[r] = take_min ? (k[r] < o ? k[r] : o) : (k[r] < o ? o : k[r]);
+                    k[r] = ((k[r] > o) == keep_min) ? o : k[r];
                 }
             } else {
 #pragma unroll
                 for (int r = 0; r < 8; r++) {
                     if (r & j) continue;
-                    const int i = lane * 8 + r;
+                    // ascending block unless bit kk of the element index is set
+                    const bool asc = kk >= 8 ? (l8 & kk) == 0 : (r & kk) == 0;
                     const uint64_t x = k[r], y = k[r | j];
-                    if ((x > y) == ((i & kk) == 0)) {
-                        k[r] = y;
-                        k[r | j] = x;
-                    }
+                    const bool sw = (x > y) == asc;
+                    k[r] = sw ? y : x;
+                    k[r | j] = sw ? x : y;
                 }
             }
         }
@@ -855,6 +871,38 @@ __device__ __forceinline__ int run_rank(const uint64_t *a, int n, uint64_t x) {
     return lo;
 }
 
+// Tile lists of at most 256 entries: one warp each, in registers (CTA b,
+// warp w take the (4 b + w)-th tile of the order).
+__global__ void __launch_bounds__(128)
+k_tile_sort_warp(const uint32_t *__restrict__ ranges, const uint32_t *__restrict__ order, int tiles,
+                 const uint64_t *__restrict__ keys, uint32_t *__restrict__ pair_gid,
+                 uint32_t *__restrict__ pair_tile) {
+    const int lane = threadIdx.x & 31;
+    const int b = blockIdx.x * 4 + (threadIdx.x >> 5);
+    if (b >= tiles) return;
+    const uint32_t tile = order[b];
+    const uint32_t start = ranges[2 * (size_t)tile], end = ranges[2 * (size_t)tile + 1];
+    const uint32_t L = end - start;
+    if (L == 0 || L > 256) return;
+    uint64_t k[8];
+#pragma unroll
+    for (int r = 0; r < 8; r++) {
+        const uint32_t idx = (uint32_t)(lane * 8 + r);
+        k[r] = idx < L ? keys[start + idx] : ~0ull;
+    }
+    int P = 2;
+    while ((uint32_t)P < L) P <<= 1;
+    warp_bitonic_256(k, lane, P);
+#pragma unroll
+    for (int r = 0; r < 8; r++) {
+        const uint32_t idx = (uint32_t)(lane * 8 + r);
+        if (idx < L) {
+            pair_gid[start + idx] = (uint32_t)k[r];
+            pair_tile[start + idx] = tile;
+        }
+    }
+}
+
 // Tile lists in (lo, hi], hi = 256 kWarps: sorted by one CTA each.  Warp w
 // sorts keys [256 w, 256 w + 256) in registers; the runs are then merged
 // pairwise in shared memory (each key's output position is its index plus
@@ -864,7 +912,7 @@ __device__ __forceinline__ int run_rank(const uint64_t *a, int n, uint64_t x) {
 template <int kWarps>
 __global__ void __launch_bounds__(kWarps * 32)
 k_tile_sort(const uint32_t *__restrict__ ranges, const uint32_t *__restrict__ order, int tiles,
-            const float4 *__restrict__ xyod, uint32_t *__restrict__ pair_gid,
+            const uint64_t *__restrict__ keys, uint32_t *__restrict__ pair_gid,
             uint32_t *__restrict__ pair_tile, uint32_t lo, int persistent) {
     constexpr int kThreads = kWarps * 32;
     constexpr uint32_t kHi = 256u * kWarps;
@@ -885,9 +933,14 @@ k_tile_sort(const uint32_t *__restrict__ ranges, const uint32_t *__restrict__ or
 #pragma unroll
             for (int r = 0; r < 8; r++) {
                 const uint32_t idx = (uint32_t)(warp * 256 + lane * 8 + r);
-                k[r] = idx < L ? pair_key(xyod, pair_gid[start + idx]) : ~0ull;
+                k[r] = idx < L ? keys[start + idx] : ~0ull;
             }
-            if (warp < chunks) warp_bitonic_256(k, lane);
+            if (warp < chunks) {
+                const uint32_t m = min(L - (uint32_t)warp * 256u, 256u);  // real keys of the chunk
+                int P = 2;
+                while ((uint32_t)P < m) P <<= 1;
+                warp_bitonic_256(k, lane, P);
+            }
 #pragma unroll
             for (int r = 0; r < 8; r++) s_buf[warp * 256 + lane * 8 + r] = k[r];
         }
@@ -918,11 +971,11 @@ k_tile_sort(const uint32_t *__restrict__ ranges, const uint32_t *__restrict__ or
 // Tiles longer than the shared-memory sort holds: one CTA per tile runs an
 // LSD radix sort of the tile's keys in global memory (8-bit digits: four
 // passes over the id, then four over the depth bits; each pass stable, in
-// chunks of 256 ranked with warp ballots), through scratch arrays at the
-// same offsets as the tile's range.
+// chunks of 256 ranked with warp ballots), ping-ponging between (ka, va) and
+// (kb, vb) at the same offsets as the tile's range.
 __global__ void __launch_bounds__(256)
 k_tile_sort_long(const uint32_t *__restrict__ ranges, const uint32_t *__restrict__ order, int tiles,
-                 const float4 *__restrict__ xyod, uint32_t *__restrict__ pair_gid,
+                 const uint64_t *__restrict__ keys, uint32_t *__restrict__ pair_gid,
                  uint32_t *__restrict__ pair_tile, uint32_t lo, uint32_t *__restrict__ ka,
                  uint32_t *__restrict__ va, uint32_t *__restrict__ kb, uint32_t *__restrict__ vb) {
     __shared__ uint32_t s_base[kRadix];
@@ -934,9 +987,9 @@ k_tile_sort_long(const uint32_t *__restrict__ ranges, const uint32_t *__restrict
         if (order_bucket(end - start) < order_bucket(lo)) break;
         if (end - start <= lo) continue;
         for (uint32_t i = start + tid; i < end; i += 256) {
-            const uint32_t g = pair_gid[i];
-            ka[i] = __float_as_uint(xyod[g].w);
-            va[i] = g;
+            const uint64_t key = keys[i];
+            ka[i] = (uint32_t)(key >> 32);
+            va[i] = (uint32_t)key;
         }
         __syncthreads();
         uint32_t *sk = ka, *sv = va, *dk = kb, *dv = vb;
@@ -1036,7 +1089,9 @@ cudaError_t launch_bin_and_sort(const CamConst &c, int64_t n, const gs_projected
         const int4 *rect = reinterpret_cast<const int4 *>(proj.rect);
         const float4 *xyod = reinterpret_cast<const float4 *>(proj.xy_opacity_depth);
         uint32_t *order = U32(L.tile_order);
-        int64_t ctas64 = std::min<int64_t>((int64_t)sms, (int64_t)kBinCTAsMax);
+        // the emitted sort keys, u64[max_pairs], over the (ptile_a, pgid_a) scratch
+        uint64_t *keys = reinterpret_cast<uint64_t *>(base + L.ptile_a);
+        int64_t ctas64 = std::min<int64_t>((int64_t)2 * sms, (int64_t)kBinCTAsMax);
         ctas64 = std::min<int64_t>(ctas64, kBinHistCap / tiles);
         const int ctas = (int)std::max<int64_t>(1, ctas64);
         const size_t cnt_smem = tiles <= kSmemTiles ? (size_t)tiles * sizeof(uint32_t) : 0;
@@ -1060,18 +1115,20 @@ cudaError_t launch_bin_and_sort(const CamConst &c, int64_t n, const gs_projected
         prof_after(s);
         if (n > 0) {
             prof_before("emit", s);
-            k_bin_emit<<<ctas, kBinThreads, cnt_smem, s>>>((int)n, rect, c.tiles_x, c.tiles_y, ranges, H,
-                                                           bins.pair_gid, status);
+            k_bin_emit<<<ctas, kBinThreads, cnt_smem, s>>>((int)n, rect, xyod, c.tiles_x, c.tiles_y, ranges, H,
+                                                           keys, status);
             prof_after(s);
-            const int few = std::min(tiles, sms);
             prof_before("tile_sort", s);
+            k_tile_sort_warp<<<(tiles + 3) / 4, 128, 0, s>>>(ranges, order, tiles, keys, bins.pair_gid,
+                                                              bins.pair_tile);
             k_tile_sort<kShortWarps><<<tiles, kShortWarps * 32, 2 * kTileSortShort * sizeof(uint64_t), s>>>(
-                ranges, order, tiles, xyod, bins.pair_gid, bins.pair_tile, 0u, 0);
-            k_tile_sort<kMidWarps><<<few, kMidWarps * 32, 2 * kTileSortMid * sizeof(uint64_t), s>>>(
-                ranges, order, tiles, xyod, bins.pair_gid, bins.pair_tile, kTileSortShort, 1);
-            k_tile_sort_long<<<few, 256, 0, s>>>(ranges, order, tiles, xyod, bins.pair_gid, bins.pair_tile,
-                                                 kTileSortMid, U32(L.ptile_a), U32(L.pgid_a),
-                                                 U32(L.ptile_b), U32(L.pgid_b));
+                ranges, order, tiles, keys, bins.pair_gid, bins.pair_tile, 256u, 0);
+            k_tile_sort<kMidWarps><<<std::min(tiles, sms), kMidWarps * 32, 2 * kTileSortMid * sizeof(uint64_t),
+                                     s>>>(ranges, order, tiles, keys, bins.pair_gid, bins.pair_tile,
+                                          kTileSortShort, 1);
+            k_tile_sort_long<<<std::min(tiles, sms), 256, 0, s>>>(
+                ranges, order, tiles, keys, bins.pair_gid, bins.pair_tile, kTileSortMid, U32(L.ptile_b),
+                U32(L.pgid_b), bins.pair_tile, bins.pair_gid);
             prof_after(s);
         }
         return cudaGetLastError();
