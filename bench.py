@@ -67,31 +67,21 @@ OPS_VISIT = 12
 OPS_FWD_ADD = 6
 OPS_BWD_ADD = 32
 
-# Algorithmic HBM bytes of the streaming kernels (per Gaussian G, pair P):
+# Algorithmic HBM bytes of the streaming stages (per Gaussian G, pair P):
 #   project      56 B/G raw parameters read + 68 B/G records written
-#   depth_keys   8 B/G read (depth, count) + 4 B/G written
-#   depth_sort   16 B/G per pass (key + value read and written)
-#   scan         20 B/G read (sorted id, rectangle) + 12 B/G records written
-#   emit         16 B/G records read + 8 B/P written
-#   tile_sort    16 B/P per pass
-#   ranges       4 B/P read
+#   bin_count    16 B/G rectangles read (the count matrix is 4 B per CTA and
+#                tile, small beside them)
+#   emit         16 B/G rectangle + 16 B/G depth record read, 8 B/P keys written
+#   tile_sort    8 B/P keys read, 8 B/P (id, tile) written
 #   project_bwd  56 B/G raw parameters + 48 B/G 2D sums + 32 B/G records read,
 #                48 B/G 2D gradients + 56 B/G raw gradients written
 BYTES = {
     "project": lambda G, P: 124 * G,
-    "depth_keys": lambda G, P: 12 * G,
-    "depth_sort": lambda G, P: 16 * G,
-    "scan": lambda G, P: 32 * G,
-    "emit": lambda G, P: 16 * G + 8 * P,
+    "bin_count": lambda G, P: 16 * G,
+    "emit": lambda G, P: 32 * G + 8 * P,
     "tile_sort": lambda G, P: 16 * P,
-    "ranges": lambda G, P: 4 * P,
     "project_bwd": lambda G, P: 240 * G,
 }
-ALU_KERNELS = ("render_fwd", "render_bwd")
-
-# DRAM traffic per launch of render_bwd measured by ncu
-# (dram__bytes_read.sum + dram__bytes_write.sum), valid only for the kernel
-# source it was taken on.
 TRAFFIC = {}  # {"render_bwd": {"src_sha": ..., "bytes_per_pair": ...}}
 
 
@@ -421,9 +411,8 @@ def run_native(args, spec, rank, world, local):
         gpu_launches += launches
         entry = {"launches": launches, "ms_total": ms, "ms_per_step": ms / args.steps}
         if name in BYTES:
-            passes = launches / args.steps
             per_step = [BYTES[name](n, pairs[i]) for i in sel]
-            total_bytes = sum(per_step) * (passes if name in ("depth_sort", "tile_sort") else 1)
+            total_bytes = sum(per_step)
             ach = total_bytes / (ms * 1e-3) / 1e9
             entry.update(bound="hbm", achieved=ach, peak=hbm_peak, unit="GB/s", frac=ach / hbm_peak)
         elif name in ALU_KERNELS:

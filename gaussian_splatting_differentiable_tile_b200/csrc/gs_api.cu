@@ -94,6 +94,7 @@ inline cudaStream_t as_stream(void *s) { return reinterpret_cast<cudaStream_t>(s
 struct ProfRec {
     const char *name;
     cudaEvent_t a, b;
+    int kernels;  // kernel launches between the two events
 };
 std::vector<ProfRec> g_prof;
 std::vector<cudaEvent_t> g_pool;
@@ -118,14 +119,15 @@ namespace gs {
 void prof_before(const char *name, cudaStream_t s) {
     g_prof_pending = false;
     if (!g_prof_on || (int32_t)g_prof.size() >= g_prof_max) return;
-    ProfRec r{name, pool_event(), pool_event()};
+    ProfRec r{name, pool_event(), pool_event(), 1};
     if (!r.a || !r.b) return;
     cudaEventRecord(r.a, s);
     g_prof.push_back(r);
     g_prof_pending = true;
 }
-void prof_after(cudaStream_t s) {
+void prof_after(cudaStream_t s, int kernels) {
     if (!g_prof_pending) return;
+    g_prof.back().kernels = kernels;
     cudaEventRecord(g_prof.back().b, s);
     g_prof_pending = false;
 }
@@ -337,7 +339,7 @@ int gs_profile_end(gs_profile_stat *out, int32_t max_stats) {
             stats.push_back(s);
             hit = &stats.back();
         }
-        hit->launches += 1;
+        hit->launches += r.kernels;
         hit->total_ms += ms;
     }
     for (auto &r : g_prof) {

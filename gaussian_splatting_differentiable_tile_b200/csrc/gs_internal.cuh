@@ -12,39 +12,14 @@ namespace gs {
 constexpr int kTile = GS_TILE;            // 16 x 16 pixel tiles
 constexpr int kTilePixels = kTile * kTile;
 
-// Radix sort: 8-bit digits, 256 threads x 16 keys per partition.
+// Radix digits of the long-list sort: 8 bits.
 constexpr int kRadixBits = 8;
 constexpr int kRadix = 1 << kRadixBits;
-constexpr int kSortThreads = 256;
-constexpr int kSortItems = 16;
-constexpr int kSortPart = kSortThreads * kSortItems;  // 4096 keys
-constexpr int kMaxDepthPasses = 4;                    // 31 depth bits
-constexpr int kMaxTilePasses = 3;                     // up to 24 tile-id bits
 
-// Scan + emit: 256 threads x 8 Gaussians per partition.
-constexpr int kScanThreads = 256;
-constexpr int kScanItems = 8;
-constexpr int kScanPart = kScanThreads * kScanItems;  // 2048 Gaussians
-
-// Pair emit: 256 threads per block, 2048 pairs per block.
-constexpr int kEmitThreads = 256;
-constexpr int kEmitPairs = 2048;
-
-// Bounded device-side waits: a decoupled look-back poll gives up after this
-// many polls, records GS_ERR_DEVICE_TIMEOUT and lets the kernel finish.
-constexpr uint32_t kSpinLimit = 1u << 21;
-
-// Look-back words: 2 flag bits + 30 value bits (partition aggregate or
-// inclusive prefix).  N and max_pairs are kept below 2^30 so values fit.
-constexpr uint32_t kFlagAggregate = 1u << 30;
-constexpr uint32_t kFlagInclusive = 2u << 30;
-constexpr uint32_t kValueMask = (1u << 30) - 1;
-constexpr uint64_t kFlag64Aggregate = 1ull << 62;
-constexpr uint64_t kFlag64Inclusive = 2ull << 62;
-constexpr uint64_t kValue64Mask = (1ull << 62) - 1;
-
-// Key given to Gaussians that draw nothing: sorts after every positive float.
-constexpr uint32_t kInvalidDepthKey = 0x7FFFFFFFu;
+// Binning: the count matrix [CTA][tile] holds at most kBinHistCap entries
+// and is split among at most kBinCTAsMax CTAs.
+constexpr int kBinCTAsMax = 320;
+constexpr int64_t kBinHistCap = (int64_t)1 << 22;
 
 // Camera constants derived once on the host.
 struct CamConst {
@@ -61,60 +36,41 @@ struct CamConst {
 // Byte layout of a gs_bins buffer.  The first `zero_bytes` bytes are cleared
 // by one memset at the start of every gs_bin_and_sort.
 struct BinsLayout {
-    size_t status, n_pairs, tickets, depth_hist, tile_hist;
-    size_t tile_count;                              // [max_tiles] pairs per tile, then emit cursors
-    size_t ranges, depth_lb, scan_lb, tile_lb;
+    size_t status, n_pairs;     // the status word and K
     size_t zero_bytes;
-    size_t tile_order;                              // [max_tiles] tiles, longest list first
-    size_t bin_hist;                                // per-CTA tile counts, then offsets
-    size_t keys_a, vals_a, keys_b, vals_b;          // depth sort, [max_n]
-    size_t ptile_a, pgid_a, ptile_b, pgid_b;        // pair sort ping-pong, [max_pairs]
-    size_t pair_tile, pair_gid;                     // result, [max_pairs]
+    size_t tile_total;          // [max_tiles] pairs per tile
+    size_t ranges;              // [max_tiles][2]
+    size_t tile_order;          // [max_tiles] tiles, longest list first
+    size_t bin_hist;            // count matrix: per-CTA tile counts, then offsets
+    size_t keys;                // u64[max_pairs] emitted sort keys
+    size_t long_keys, long_ids; // u32[max_pairs] each: scratch of the long-list sort
+    size_t pair_tile, pair_gid; // u32[max_pairs] each: the result
     size_t total;
-    int64_t depth_parts, scan_parts, tile_parts;
 };
 
 constexpr size_t align_up(size_t v, size_t a) { return (v + a - 1) / a * a; }
 
 constexpr BinsLayout bins_layout(int64_t max_n, int64_t max_pairs, int32_t max_tiles) {
+    (void)max_n;
     BinsLayout L{};
     size_t off = 0;
     L.status = off;       off += 8;
     L.n_pairs = off;      off += 8;
-    off = align_up(off, 64);
-    L.tickets = off;      off += 16 * sizeof(uint32_t);
     off = align_up(off, 256);
-    L.depth_hist = off;   off += kMaxDepthPasses * kRadix * sizeof(uint32_t);
-    L.tile_hist = off;    off += kMaxTilePasses * kRadix * sizeof(uint32_t);
-    off = align_up(off, 256);
-    L.tile_count = off;   off = align_up(off + (size_t)max_tiles * sizeof(uint32_t), 256);
-    L.ranges = off;       off = align_up(off + (size_t)max_tiles * 2 * sizeof(uint32_t), 256);
-    L.depth_parts = (max_n + kSortPart - 1) / kSortPart;
-    L.scan_parts = (max_n + kScanPart - 1) / kScanPart;
-    L.tile_parts = (max_pairs + kSortPart - 1) / kSortPart;
-    L.depth_lb = off;
-    off = align_up(off + (size_t)kMaxDepthPasses * L.depth_parts * kRadix * sizeof(uint32_t), 256);
-    L.scan_lb = off;
-    off = align_up(off + (size_t)L.scan_parts * sizeof(uint64_t), 256);
-    L.tile_lb = off;
-    off = align_up(off + (size_t)kMaxTilePasses * L.tile_parts * kRadix * sizeof(uint32_t), 256);
     L.zero_bytes = off;
-    L.tile_order = off;   off = align_up(off + (size_t)max_tiles * sizeof(uint32_t), 256);
+    const size_t tb = align_up((size_t)max_tiles * sizeof(uint32_t), 256);
+    L.tile_total = off;   off += tb;
+    L.ranges = off;       off += 2 * tb;
+    L.tile_order = off;   off += tb;
     L.bin_hist = off;
     {
-        const int64_t h = (int64_t)320 * max_tiles, cap = (int64_t)1 << 22;  // per-CTA tile counts
-        off = align_up(off + (size_t)(h < cap ? h : cap) * sizeof(uint32_t), 256);
+        const int64_t h = (int64_t)kBinCTAsMax * max_tiles;
+        off = align_up(off + (size_t)(h < kBinHistCap ? h : kBinHistCap) * sizeof(uint32_t), 256);
     }
-    size_t nb = align_up((size_t)max_n * sizeof(uint32_t), 256);
-    size_t pb = align_up((size_t)max_pairs * sizeof(uint32_t), 256);
-    L.keys_a = off;  off += nb;
-    L.vals_a = off;  off += nb;
-    L.keys_b = off;  off += nb;
-    L.vals_b = off;  off += nb;
-    L.ptile_a = off; off += pb;
-    L.pgid_a = off;  off += pb;
-    L.ptile_b = off; off += pb;
-    L.pgid_b = off;  off += pb;
+    const size_t pb = align_up((size_t)max_pairs * sizeof(uint32_t), 256);
+    L.keys = off;      off += 2 * pb;
+    L.long_keys = off; off += pb;
+    L.long_ids = off;  off += pb;
     L.pair_tile = off; off += pb;
     L.pair_gid = off;  off += pb;
     L.total = off;
@@ -123,22 +79,6 @@ constexpr BinsLayout bins_layout(int64_t max_n, int64_t max_pairs, int32_t max_t
 
 // ---------------------------------------------------------------- device
 #ifdef __CUDACC__
-__device__ __forceinline__ uint32_t ld_relaxed(const uint32_t *p) {
-    uint32_t v;
-    asm volatile("ld.relaxed.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
-    return v;
-}
-__device__ __forceinline__ void st_relaxed(uint32_t *p, uint32_t v) {
-    asm volatile("st.relaxed.gpu.global.u32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
-}
-__device__ __forceinline__ uint64_t ld_relaxed64(const uint64_t *p) {
-    uint64_t v;
-    asm volatile("ld.relaxed.gpu.global.u64 %0, [%1];" : "=l"(v) : "l"(p) : "memory");
-    return v;
-}
-__device__ __forceinline__ void st_relaxed64(uint64_t *p, uint64_t v) {
-    asm volatile("st.relaxed.gpu.global.u64 [%0], %1;" ::"l"(p), "l"(v) : "memory");
-}
 // A splat's tile rectangle clamped to the grid: returns the number of tiles
 // it covers (0 when empty) and its first column, row and width.  Binning
 // derives everything from the rectangle, so records from any source can
@@ -182,6 +122,6 @@ cudaError_t launch_l1(const float *image, const float *target, int64_t count, fl
 
 // Profiling hooks used around every launch (gs_api.cu).
 void prof_before(const char *name, cudaStream_t s);
-void prof_after(cudaStream_t s);
+void prof_after(cudaStream_t s, int kernels = 1);  // kernels launched since prof_before
 
 }  // namespace gs

@@ -1,25 +1,30 @@
-// gs_sort.cu -- tile binning: depth sort, count scan, pair emit, pair sort,
-// per-tile ranges.
+// gs_sort.cu -- tile binning: count, scan, emit, per-tile sort, ranges.
 //
 // Source: "SplatRs: The Week the Gap Closed", "Throughput: the tile
-// rasterizer" (project, count, emit, sort, range, blend) and "Gaussian
-// splatting in PyTorch" s5 (one global depth sort replaces per-tile sorts).
+// rasterizer" (project, count, emit, sort, range, blend).
 //
 // The pages key each (tile, Gaussian) pair by (tile << 32 | depth bits) and
-// radix-sort the pairs on that key.  Here the depth half of the key is sorted
-// once per Gaussian instead of once per pair: Gaussians are first sorted by
-// depth (31 used bits of the positive float), their pairs are emitted in that
-// order, and a stable sort on the tile bits alone finishes the job.  The pair
-// order is identical (ties in depth by Gaussian id), while each pair passes
-// through ceil(tile_bits / 8) sort passes of 8 bytes instead of
-// ceil(43..45 / 8) passes of 12 bytes.
+// radix-sort all pairs on that key.  The same order is reached here without
+// a global sort: pairs are grouped by tile through counts and scans, and
+// each tile's short list is sorted on its own by the 64-bit key
+// (depth bits << 32 | Gaussian id), which is unique, so the order inside a
+// tile is by depth with ties by id -- exactly the global key order.
 //
-// Both sorts are LSD radix sorts built from one "onesweep" pass kernel:
-// a block ranks its 4096 keys with warp ballots and popc, publishes its digit
-// counts, and resolves its global offsets by a decoupled look-back over the
-// preceding partitions (bounded: a poll loop that runs out sets
-// GS_ERR_DEVICE_TIMEOUT and the kernel still finishes).  Partitions are taken
-// in ticket order so every block waits only on blocks already running.
+//   k_bin_count    a fixed set of CTAs splits the Gaussians into contiguous
+//                  ranges; each counts its pairs per tile in shared memory
+//                  and writes its row of a [CTA][tile] count matrix
+//   k_bin_colscan  offsets down each tile's column, and each tile's total
+//   k_tile_scan    one CTA: ranges, K (capacity check), and the order in
+//                  which the sorts and the blend take the tiles (longest
+//                  list first)
+//   k_bin_emit     each CTA writes the keys of its pairs at its offsets,
+//                  advancing shared-memory cursors
+//   k_tile_sort*   per tile: one warp sorts up to 256 keys in registers; a
+//                  CTA sorts up to 1024 (and a wide CTA up to 8192) as warp
+//                  runs merged in shared memory; longer lists are radix
+//                  sorted in global memory by one CTA each
+//
+// No kernel waits on another CTA, and no global atomic is contended.
 #include "gs_internal.cuh"
 
 namespace gs {
@@ -49,525 +54,6 @@ __device__ __forceinline__ uint32_t digit_peers(uint32_t d, int bits) {
     return peers;
 }
 
-// Exclusive block-wide scan of one value per thread (blockDim = 256).
-__device__ __forceinline__ uint32_t block_exclusive_scan_256(uint32_t v, uint32_t *s_warp,
-                                                             uint32_t *total) {
-    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-    uint32_t x = v;
-#pragma unroll
-    for (int o = 1; o < 32; o <<= 1) {
-        uint32_t y = __shfl_up_sync(0xffffffffu, x, o);
-        if (lane >= o) x += y;
-    }
-    if (lane == 31) s_warp[warp] = x;
-    __syncthreads();
-    uint32_t wpre = 0, tot = 0;
-#pragma unroll
-    for (int w = 0; w < 8; w++) {
-        uint32_t t = s_warp[w];
-        if (w < warp) wpre += t;
-        tot += t;
-    }
-    __syncthreads();
-    *total = tot;
-    return wpre + x - v;
-}
-
-// Decoupled look-back for one digit: the sum of the digit's counts over
-// partitions [0, q0], read from the partitions' published words back to the
-// nearest inclusive one.  32 words are requested at a time, so a chain of
-// aggregates costs one L2 round trip per 32 partitions.  A word that stays
-// unpublished for kSpinLimit polls records GS_ERR_DEVICE_TIMEOUT and counts
-// as zero, so the kernel always finishes.
-__device__ __forceinline__ uint32_t lookback_digit(const uint32_t *lookback, int d, int64_t q0,
-                                                   int32_t *status) {
-    constexpr int kWindow = 32;
-    uint32_t excl = 0;
-    uint32_t spins = 0;
-    for (int64_t q = q0; q >= 0; q -= kWindow) {
-        uint32_t w[kWindow];
-#pragma unroll
-        for (int k = 0; k < kWindow; k++)
-            w[k] = (q - k >= 0) ? ld_relaxed(lookback + (size_t)(q - k) * kRadix + d) : kFlagInclusive;
-#pragma unroll
-        for (int k = 0; k < kWindow; k++) {
-            while ((w[k] & ~kValueMask) == 0u) {
-                if (++spins > kSpinLimit) {
-                    set_status(status, GS_ERR_DEVICE_TIMEOUT);
-                    return excl;
-                }
-                w[k] = ld_relaxed(lookback + (size_t)(q - k) * kRadix + d);
-            }
-            excl += w[k] & kValueMask;
-            if ((w[k] & ~kValueMask) == kFlagInclusive) return excl;
-        }
-    }
-    return excl;
-}
-
-// Decoupled look-back over 64-bit partition words, by one full warp: lane l
-// reads partition q0 - l, so each L2 round trip covers 32 partitions.
-// Returns the inclusive prefix of partitions [0, q0] (to every lane).
-__device__ __forceinline__ uint64_t lookback_warp64(const uint64_t *lookback, int64_t q0,
-                                                    int32_t *status) {
-    const int lane = threadIdx.x & 31;
-    uint64_t prefix = 0;
-    uint32_t spins = 0;
-    for (int64_t base = q0; base >= 0; base -= 32) {
-        const int64_t q = base - lane;
-        uint64_t w = q >= 0 ? ld_relaxed64(lookback + q) : kFlag64Inclusive;
-        bool timed_out = false;
-        while (__any_sync(0xffffffffu, (w & ~kValue64Mask) == 0ull)) {
-            if (++spins > kSpinLimit) {
-                timed_out = true;
-                break;
-            }
-            if ((w & ~kValue64Mask) == 0ull) w = ld_relaxed64(lookback + q);
-        }
-        if (timed_out) {
-            if (lane == 0) set_status(status, GS_ERR_DEVICE_TIMEOUT);
-            if ((w & ~kValue64Mask) == 0ull) w = kFlag64Inclusive;
-        }
-        const uint32_t incl = __ballot_sync(0xffffffffu, (w & ~kValue64Mask) == kFlag64Inclusive);
-        const int first = incl ? __ffs(incl) - 1 : 31;
-        uint64_t v = lane <= first ? (w & kValue64Mask) : 0ull;
-#pragma unroll
-        for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
-        prefix += v;
-        if (incl) break;
-    }
-    return prefix;
-}
-
-// Depth keys of the drawable Gaussians and the four digit histograms of the
-// depth sort.
-__global__ void __launch_bounds__(256)
-k_depth_keys(int n, const float4 *__restrict__ xyod, const int4 *__restrict__ rect, int tiles_x,
-             int tiles_y, uint32_t *__restrict__ keys, uint32_t *__restrict__ hist) {
-    __shared__ uint32_t s_h[kMaxDepthPasses * kRadix];
-    for (int i = threadIdx.x; i < kMaxDepthPasses * kRadix; i += blockDim.x) s_h[i] = 0;
-    __syncthreads();
-    for (int g = blockIdx.x * blockDim.x + threadIdx.x; g < n; g += gridDim.x * blockDim.x) {
-        int x0, y0, w;
-        const uint32_t c = rect_tiles(rect[g], tiles_x, tiles_y, x0, y0, w);
-        const uint32_t key = c > 0 ? __float_as_uint(xyod[g].w) : kInvalidDepthKey;
-        keys[g] = key;
-#pragma unroll
-        for (int k = 0; k < kMaxDepthPasses; k++) atomicAdd(&s_h[k * kRadix + ((key >> (8 * k)) & 0xFF)], 1u);
-    }
-    __syncthreads();
-    for (int i = threadIdx.x; i < kMaxDepthPasses * kRadix; i += blockDim.x)
-        if (s_h[i]) atomicAdd(&hist[i], s_h[i]);
-}
-
-// One LSD radix pass over bits [shift, shift + bits) of 32-bit keys with
-// 32-bit values.  n = min(*n_dev, n_cap) when n_dev is given, else n_host.
-// With iota_vals the values are the input indices (first pass of a sort).
-// When check_status is set the pass does nothing if *status is non-zero.
-__global__ void __launch_bounds__(kSortThreads)
-k_onesweep(const uint32_t *__restrict__ keys_in, const uint32_t *__restrict__ vals_in,
-           uint32_t *__restrict__ keys_out, uint32_t *__restrict__ vals_out,
-           const uint64_t *__restrict__ n_dev, uint32_t n_host, uint32_t n_cap, int shift, int bits,
-           const uint32_t *__restrict__ hist, uint32_t *__restrict__ lookback,
-           uint32_t *__restrict__ ticket, int32_t *__restrict__ status, int iota_vals,
-           int check_status) {
-    __shared__ uint32_t s_warp_hist[kSortThreads / 32][kRadix];
-    __shared__ uint32_t s_digit_start[kRadix];
-    __shared__ uint32_t s_global_base[kRadix];
-    __shared__ uint32_t s_hist_excl[kRadix];
-    __shared__ uint32_t s_keys[kSortPart];
-    __shared__ uint32_t s_vals[kSortPart];
-    __shared__ uint32_t s_scan[8];
-    __shared__ uint32_t s_part;
-    __shared__ int s_skip;
-
-    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-    if (tid == 0) s_skip = check_status ? (*(volatile int32_t *)status != 0) : 0;
-    __syncthreads();
-    if (s_skip) return;
-    uint32_t n = n_host;
-    if (n_dev) {
-        const uint64_t nd = *n_dev;
-        n = nd < (uint64_t)n_cap ? (uint32_t)nd : n_cap;
-    }
-    const uint32_t mask = (1u << bits) - 1u;
-    const int radix = 1 << bits;
-
-    // Exclusive scan of the global digit histogram: where each digit starts.
-    {
-        uint32_t tot;
-        const uint32_t h = tid < radix ? hist[tid] : 0u;
-        s_hist_excl[tid] = block_exclusive_scan_256(h, s_scan, &tot);
-    }
-
-    for (;;) {
-        if (tid == 0) s_part = atomicAdd(ticket, 1u);
-        __syncthreads();
-        const uint32_t p = s_part;
-        if ((uint64_t)p * kSortPart >= n) break;
-        for (int i = tid; i < (kSortThreads / 32) * kRadix; i += kSortThreads)
-            (&s_warp_hist[0][0])[i] = 0;
-        __syncthreads();
-
-        // Load: warp w owns keys [w*32*ITEMS, (w+1)*32*ITEMS) of the partition,
-        // item i of lane l at offset i*32 + l: coalesced, and index order is
-        // (warp, item, lane), which the ranking below preserves (stable).
-        const uint32_t base = p * kSortPart + warp * (32 * kSortItems);
-        uint32_t key[kSortItems], val[kSortItems], dig[kSortItems], rank[kSortItems];
-        if (base + 32 * kSortItems <= n) {
-            // a full slice: every load is issued before any is used (a
-            // per-item guard and value select keep them from overlapping)
-#pragma unroll
-            for (int i = 0; i < kSortItems; i++) key[i] = __ldcg(keys_in + base + i * 32 + lane);
-            if (iota_vals) {
-#pragma unroll
-                for (int i = 0; i < kSortItems; i++) val[i] = base + i * 32 + lane;
-            } else {
-#pragma unroll
-                for (int i = 0; i < kSortItems; i++) val[i] = __ldcg(vals_in + base + i * 32 + lane);
-            }
-#pragma unroll
-            for (int i = 0; i < kSortItems; i++) dig[i] = (key[i] >> shift) & mask;
-        } else {
-#pragma unroll
-            for (int i = 0; i < kSortItems; i++) {
-                const uint32_t idx = base + i * 32 + lane;
-                if (idx < n) {
-                    key[i] = keys_in[idx];
-                    val[i] = iota_vals ? idx : vals_in[idx];
-                    dig[i] = (key[i] >> shift) & mask;
-                } else {
-                    key[i] = 0; val[i] = 0;
-                    dig[i] = kRadix;  // sentinel: not counted
-                }
-            }
-        }
-        // Warp-level ranking of each item among equal digits: the peer masks
-        // first (independent ballots), then the per-digit counters in order.
-        uint32_t peer[kSortItems];
-#pragma unroll
-        for (int i = 0; i < kSortItems; i++) peer[i] = digit_peers(dig[i], bits);
-#pragma unroll
-        for (int i = 0; i < kSortItems; i++) {
-            const uint32_t d = dig[i];
-            const uint32_t peers = peer[i];
-            const int leader = __ffs(peers) - 1;
-            uint32_t b = 0;
-            if (d < kRadix) b = s_warp_hist[warp][d];
-            __syncwarp();
-            if (d < kRadix && lane == leader) s_warp_hist[warp][d] = b + __popc(peers);
-            __syncwarp();
-            rank[i] = b + __popc(peers & lanemask_lt());
-        }
-        __syncthreads();
-
-        // Per digit (thread = digit): warp offsets, the block's count, and
-        // where the digit's run starts in the partition's local order.
-        uint32_t block_count = 0;
-        {
-            const int d = tid;
-#pragma unroll
-            for (int w = 0; w < kSortThreads / 32; w++) {
-                const uint32_t c = s_warp_hist[w][d];
-                s_warp_hist[w][d] = block_count;
-                block_count += c;
-            }
-            uint32_t tot;
-            s_digit_start[d] = block_exclusive_scan_256(d < radix ? block_count : 0u, s_scan, &tot);
-        }
-        __syncthreads();
-        // Local reorder through shared memory first, so the look-back below
-        // runs with the keys out of registers.
-#pragma unroll
-        for (int i = 0; i < kSortItems; i++) {
-            const uint32_t d = dig[i];
-            if (d < kRadix) {
-                const uint32_t loc = s_digit_start[d] + s_warp_hist[warp][d] + rank[i];
-                s_keys[loc] = key[i];
-                s_vals[loc] = val[i];
-            }
-        }
-        // Publish this partition's count for the digit, then look back.
-        {
-            const int d = tid;
-            uint32_t *lb = lookback + (size_t)p * kRadix + d;
-            uint32_t excl = 0;
-            if (d < radix) {
-                if (p == 0) {
-                    st_relaxed(lb, kFlagInclusive | block_count);
-                } else {
-                    st_relaxed(lb, kFlagAggregate | block_count);
-                    excl = lookback_digit(lookback, d, (int64_t)p - 1, status);
-                    st_relaxed(lb, kFlagInclusive | ((excl + block_count) & kValueMask));
-                }
-            }
-            s_global_base[d] = s_hist_excl[d] + excl;
-        }
-        uint32_t valid_count;
-        {
-            const uint64_t rem = (uint64_t)n - (uint64_t)p * kSortPart;
-            valid_count = rem < (uint64_t)kSortPart ? (uint32_t)rem : (uint32_t)kSortPart;
-        }
-        __syncthreads();
-        for (uint32_t j = tid; j < valid_count; j += kSortThreads) {
-            const uint32_t k = s_keys[j];
-            const uint32_t d = (k >> shift) & mask;
-            const uint32_t pos = s_global_base[d] + (j - s_digit_start[d]);
-            if (pos < n) {
-                keys_out[pos] = k;
-                vals_out[pos] = s_vals[j];
-            }
-        }
-        __syncthreads();
-    }
-}
-
-// Exclusive block-wide scan of one 64-bit value per thread (blockDim = 256).
-__device__ __forceinline__ uint64_t block_exclusive_scan64_256(uint64_t v, uint64_t *s_warp,
-                                                               uint64_t *total) {
-    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-    uint64_t x = v;
-#pragma unroll
-    for (int o = 1; o < 32; o <<= 1) {
-        const uint64_t y = __shfl_up_sync(0xffffffffu, x, o);
-        if (lane >= o) x += y;
-    }
-    if (lane == 31) s_warp[warp] = x;
-    __syncthreads();
-    uint64_t wpre = 0, tot = 0;
-#pragma unroll
-    for (int w = 0; w < 8; w++) {
-        const uint64_t t = s_warp[w];
-        if (w < warp) wpre += t;
-        tot += t;
-    }
-    __syncthreads();
-    *total = tot;
-    return wpre + x - v;
-}
-
-// Scan of the tile counts in depth order ("count" of the tile rasterizer).
-// One block per 2048 Gaussians of the depth order; the block's offset comes
-// from a decoupled look-back over 64-bit inclusive prefixes.  For each depth
-// position i it writes the inclusive pair offset incl[i], the Gaussian's
-// packed first tile (x0 | y0 << 16) and its rectangle width, next to the
-// Gaussian id the depth sort left in sorted_gid: the emit reads these four
-// contiguous arrays.  The last block stores K; K > max_pairs records
-// GS_ERR_CAPACITY.
-__global__ void __launch_bounds__(kScanThreads)
-k_scan(int n, const uint32_t *__restrict__ sorted_gid, const int4 *__restrict__ rect, int tiles_x,
-       int tiles_y, uint32_t *__restrict__ incl, uint32_t *__restrict__ rpack,
-       uint32_t *__restrict__ width, uint64_t max_pairs, uint64_t *__restrict__ lookback,
-       uint32_t *__restrict__ ticket, uint64_t *__restrict__ n_pairs, int32_t *__restrict__ status) {
-    __shared__ uint64_t s_scan[8];
-    __shared__ uint32_t s_part;
-    __shared__ unsigned long long s_prefix;
-    const int tid = threadIdx.x;
-    if (tid == 0) s_part = atomicAdd(ticket, 1u);
-    __syncthreads();
-    const uint32_t p = s_part;
-    const int64_t base = (int64_t)p * kScanPart;
-
-    uint32_t c[kScanItems];
-    uint64_t tsum = 0;
-#pragma unroll
-    for (int i = 0; i < kScanItems; i++) {
-        const int64_t idx = base + tid * kScanItems + i;
-        c[i] = 0;
-        if (idx < n) {
-            int x0, y0, w;
-            c[i] = rect_tiles(rect[sorted_gid[idx]], tiles_x, tiles_y, x0, y0, w);
-            rpack[idx] = (uint32_t)x0 | ((uint32_t)y0 << 16);
-            width[idx] = (uint32_t)w;
-        }
-        tsum += c[i];
-    }
-    uint64_t block_total;
-    const uint64_t toff = block_exclusive_scan64_256(tsum, s_scan, &block_total);
-    if (tid < 32) {  // warp 0 publishes and looks back
-        uint64_t *lb = lookback + p;
-        uint64_t prefix = 0;
-        if (p == 0) {
-            if (tid == 0) st_relaxed64(lb, kFlag64Inclusive | (block_total & kValue64Mask));
-        } else {
-            if (tid == 0) st_relaxed64(lb, kFlag64Aggregate | (block_total & kValue64Mask));
-            prefix = lookback_warp64(lookback, (int64_t)p - 1, status);
-            if (tid == 0) st_relaxed64(lb, kFlag64Inclusive | ((prefix + block_total) & kValue64Mask));
-        }
-        if (tid == 0) {
-            s_prefix = prefix;
-            if (base + kScanPart >= n) {
-                const uint64_t K = prefix + block_total;
-                *n_pairs = K;
-                if (K > max_pairs) set_status(status, GS_ERR_CAPACITY);
-            }
-        }
-    }
-    __syncthreads();
-    uint64_t run = s_prefix + toff;
-#pragma unroll
-    for (int i = 0; i < kScanItems; i++) {
-        const int64_t idx = base + tid * kScanItems + i;
-        run += c[i];
-        if (idx < n) incl[idx] = (uint32_t)run;  // meaningful while K <= max_pairs < 2^30
-    }
-}
-
-// First index i in [lo, hi] with a[i] > t, for a non-decreasing array with
-// a[hi] > t, by one full warp: each round probes 32 evenly spaced entries,
-// so a search over N entries costs about log32(N) L2 round trips.
-__device__ __forceinline__ uint32_t warp_upper_bound(const uint32_t *a, uint32_t lo, uint32_t hi,
-                                                     uint32_t t) {
-    const int lane = threadIdx.x & 31;
-    while (hi - lo + 1 > 32) {
-        const uint32_t stride = (hi - lo + 32) / 32;
-        const uint32_t x = min(lo + lane * stride, hi);
-        const uint32_t m = __ballot_sync(0xffffffffu, a[x] > t);
-        if (m == 0) {
-            lo = min(lo + 31 * stride, hi) + 1;
-        } else {
-            const int f = __ffs(m) - 1;
-            const uint32_t xf = min(lo + f * stride, hi);
-            lo = f == 0 ? lo : min(lo + (f - 1) * stride, hi) + 1;
-            hi = xf;
-        }
-    }
-    const uint32_t x = min(lo + lane, hi);
-    const uint32_t m = __ballot_sync(0xffffffffu, a[x] > t);
-    return lo + (__ffs(m) - 1);
-}
-
-// Pair emit ("emit" of the tile rasterizer), balanced by pairs: block b writes
-// pairs [2048 b, 2048 b + 2048).  Warps 0 and 1 find the depth positions of
-// the Gaussians holding its first and last pair; the block stages that span
-// (at most 2048 Gaussians, since every drawable Gaussian has at least one
-// pair and the undrawable ones sort last) in shared memory, and each thread
-// finds its pair's Gaussian there by binary search.  A Gaussian's tiles are
-// emitted row by row; the digit histograms of the tile sort are gathered on
-// the way.  Nothing is emitted after a recorded error.
-__global__ void __launch_bounds__(kEmitThreads)
-k_emit(int n, const uint32_t *__restrict__ incl, const uint32_t *__restrict__ sorted_gid,
-       const uint32_t *__restrict__ rpack, const uint32_t *__restrict__ width, int tiles_x,
-       const uint64_t *__restrict__ n_pairs, const int32_t *__restrict__ status,
-       uint32_t *__restrict__ ptile, uint32_t *__restrict__ pgid, uint32_t *__restrict__ tile_hist,
-       int tile_passes, int tile_bpp) {
-    __shared__ uint32_t s_incl[kEmitPairs];
-    __shared__ uint32_t s_gid[kEmitPairs];
-    __shared__ uint32_t s_rp[kEmitPairs];
-    __shared__ uint32_t s_w[kEmitPairs];
-    __shared__ uint32_t s_hist[kMaxTilePasses * kRadix];
-    __shared__ uint32_t s_span[3];  // g0, g1, pairs before g0
-    if (*(volatile const int32_t *)status != 0 || n == 0) return;
-    const uint64_t K = *n_pairs;
-    const int tid = threadIdx.x, warp = tid >> 5;
-    for (int i = tid; i < kMaxTilePasses * kRadix; i += kEmitThreads) s_hist[i] = 0;
-    const uint32_t dmask = (1u << tile_bpp) - 1u;
-    for (uint64_t b = blockIdx.x; b * kEmitPairs < K; b += gridDim.x) {
-        const uint32_t p0 = (uint32_t)(b * kEmitPairs);
-        const uint64_t pe = (uint64_t)p0 + kEmitPairs;
-        const uint32_t p1 = (uint32_t)(K < pe ? K : pe);  // exclusive
-        __syncthreads();
-        if (warp == 0) {
-            const uint32_t g0 = warp_upper_bound(incl, 0, (uint32_t)n - 1, p0);
-            if (tid == 0) {
-                s_span[0] = g0;
-                s_span[2] = g0 == 0 ? 0u : incl[g0 - 1];
-            }
-        } else if (warp == 1) {
-            const uint32_t g1 = warp_upper_bound(incl, 0, (uint32_t)n - 1, p1 - 1);
-            if ((tid & 31) == 0) s_span[1] = g1;
-        }
-        __syncthreads();
-        const uint32_t g0 = s_span[0], g1 = s_span[1], before = s_span[2];
-        const uint32_t span = g1 - g0 + 1;
-        for (uint32_t k = tid; k < span && k < (uint32_t)kEmitPairs; k += kEmitThreads) {
-            s_incl[k] = incl[g0 + k];
-            s_gid[k] = sorted_gid[g0 + k];
-            s_rp[k] = rpack[g0 + k];
-            s_w[k] = width[g0 + k];
-        }
-        __syncthreads();
-        const int last = (int)min(span, (uint32_t)kEmitPairs) - 1;
-        for (uint32_t j = p0 + tid; j < p1; j += kEmitThreads) {
-            int lo = 0, hi = last;
-            while (lo < hi) {
-                const int mid = (lo + hi) >> 1;
-                if (s_incl[mid] > j) hi = mid; else lo = mid + 1;
-            }
-            const uint32_t li = j - (lo == 0 ? before : s_incl[lo - 1]);
-            const uint32_t w = s_w[lo], rp = s_rp[lo];
-            const uint32_t row = li / w;
-            const uint32_t tile = ((rp >> 16) + row) * (uint32_t)tiles_x + (rp & 0xFFFFu) + (li - row * w);
-            ptile[j] = tile;
-            pgid[j] = s_gid[lo];
-            for (int k = 0; k < tile_passes; k++)
-                atomicAdd(&s_hist[k * kRadix + ((tile >> (k * tile_bpp)) & dmask)], 1u);
-        }
-    }
-    __syncthreads();
-    for (int i = tid; i < tile_passes * kRadix; i += kEmitThreads)
-        if (s_hist[i]) atomicAdd(&tile_hist[i], s_hist[i]);
-}
-
-// [start, end) of each tile in the sorted pair list.  Ranges were zeroed
-// beforehand, so empty tiles stay [0, 0); on a recorded error all stay empty.
-__global__ void __launch_bounds__(256)
-k_ranges(const uint32_t *__restrict__ ptile, const uint64_t *__restrict__ n_pairs,
-         uint32_t *__restrict__ ranges, const int32_t *__restrict__ status) {
-    if (*(volatile const int32_t *)status != 0) return;
-    const uint64_t K = *n_pairs;
-    for (uint64_t j = (uint64_t)blockIdx.x * blockDim.x + threadIdx.x; j < K;
-         j += (uint64_t)gridDim.x * blockDim.x) {
-        const uint32_t t = ptile[j];
-        if (j == 0 || ptile[j - 1] != t) ranges[2 * (size_t)t] = (uint32_t)j;
-        if (j == K - 1 || ptile[j + 1] != t) ranges[2 * (size_t)t + 1] = (uint32_t)(j + 1);
-    }
-}
-
-// Order in which the blend kernels take the tiles: longest list first, so
-// that the heaviest tiles do not start last and leave SMs idle at the end
-// (a counting sort on list length in steps of 4 entries, one CTA; the order
-// within a bucket is arbitrary).
-constexpr int kOrderBuckets = 1024;
-__global__ void __launch_bounds__(kOrderBuckets)
-k_tile_order(const uint32_t *__restrict__ ranges, int tiles, uint32_t *__restrict__ order) {
-    __shared__ uint32_t s_off[kOrderBuckets];
-    __shared__ uint32_t s_warp[kOrderBuckets / 32];
-    const int t = threadIdx.x;
-    auto bucket = [&](int i) {
-        const uint32_t len = ranges[2 * (size_t)i + 1] - ranges[2 * (size_t)i];
-        return kOrderBuckets - 1 - (int)min(len >> 2, (uint32_t)(kOrderBuckets - 1));
-    };
-    s_off[t] = 0;
-    __syncthreads();
-    for (int i = t; i < tiles; i += kOrderBuckets) atomicAdd(&s_off[bucket(i)], 1u);
-    __syncthreads();
-    // exclusive scan of the bucket counts
-    const uint32_t v = s_off[t];
-    uint32_t x = v;
-    const int lane = t & 31, w = t >> 5;
-#pragma unroll
-    for (int o = 1; o < 32; o <<= 1) {
-        const uint32_t y = __shfl_up_sync(0xffffffffu, x, o);
-        if (lane >= o) x += y;
-    }
-    if (lane == 31) s_warp[w] = x;
-    __syncthreads();
-    if (w == 0) {
-        uint32_t z = s_warp[lane];
-#pragma unroll
-        for (int o = 1; o < 32; o <<= 1) {
-            const uint32_t y = __shfl_up_sync(0xffffffffu, z, o);
-            if (lane >= o) z += y;
-        }
-        s_warp[lane] = z;
-    }
-    __syncthreads();
-    s_off[t] = x - v + (w > 0 ? s_warp[w - 1] : 0u);
-    __syncthreads();
-    for (int i = t; i < tiles; i += kOrderBuckets) order[atomicAdd(&s_off[bucket(i)], 1u)] = (uint32_t)i;
-}
-
 // ---------------------------------------------------------------------
 // Per-tile binning.  A fixed set of CTAs splits the Gaussians into
 // contiguous ranges; each CTA counts its pairs per tile in shared memory and
@@ -580,15 +66,8 @@ k_tile_order(const uint32_t *__restrict__ ranges, int tiles, uint32_t *__restric
 // result is exactly the pair order of the global sort on
 // (tile << 32 | depth bits) with ties by id.
 
-#ifndef GS_BIN_LOCAL
-#define GS_BIN_LOCAL 1
-#endif
-
 constexpr int kBinThreads = 512;
-// The count matrix holds at most kBinHistCap entries: min(SMs, kBinCTAsMax,
-// kBinHistCap / tiles) CTAs share the Gaussians.
-constexpr int kBinCTAsMax = 320;
-constexpr int64_t kBinHistCap = 1 << 22;
+
 // Rectangles of at most this many tiles are handled by their own lane; larger
 // ones by the whole warp, one at a time.
 constexpr uint32_t kLaneTiles = 16;
@@ -1067,162 +546,60 @@ cudaError_t launch_bin_and_sort(const CamConst &c, int64_t n, const gs_projected
     auto U32 = [&](size_t off) { return reinterpret_cast<uint32_t *>(base + off); };
     int32_t *status = reinterpret_cast<int32_t *>(base + L.status);
     uint64_t *n_pairs = reinterpret_cast<uint64_t *>(base + L.n_pairs);
-    uint32_t *tickets = U32(L.tickets);
-    uint32_t *depth_hist = U32(L.depth_hist);
-    uint32_t *tile_hist = U32(L.tile_hist);
     uint32_t *ranges = U32(L.ranges);
+    uint32_t *totals = U32(L.tile_total);
+    uint32_t *order = U32(L.tile_order);
+    uint32_t *H = U32(L.bin_hist);
+    uint64_t *keys = reinterpret_cast<uint64_t *>(base + L.keys);
+    const int4 *rect = reinterpret_cast<const int4 *>(proj.rect);
     const int tiles = c.tiles_x * c.tiles_y;
+    const int sms = num_sms();
+    // CTAs sharing the Gaussians: two per SM, within the count matrix's size
+    int64_t ctas64 = std::min<int64_t>((int64_t)2 * sms, (int64_t)kBinCTAsMax);
+    ctas64 = std::min<int64_t>(ctas64, kBinHistCap / tiles);
+    const int ctas = (int)std::max<int64_t>(1, ctas64);
+    const size_t cnt_smem = tiles <= kSmemTiles ? (size_t)tiles * sizeof(uint32_t) : 0;
+    static bool attr = [] {
+        cudaFuncSetAttribute(k_bin_count, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             (int)(kSmemTiles * sizeof(uint32_t)));
+        cudaFuncSetAttribute(k_bin_emit, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             (int)(kSmemTiles * sizeof(uint32_t)));
+        cudaFuncSetAttribute(k_tile_sort<kMidWarps>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             (int)(2 * kTileSortMid * sizeof(uint64_t)));
+        return true;
+    }();
+    (void)attr;
 
-    auto tile_order = [&]() {
-        prof_before("tile_order", s);
-        k_tile_order<<<1, kOrderBuckets, 0, s>>>(ranges, tiles, U32(L.tile_order));
-        prof_after(s);
-        return cudaGetLastError();
-    };
     cudaError_t e = cudaMemsetAsync(base, 0, L.zero_bytes, s);
     if (e != cudaSuccess) return e;
-#if GS_BIN_LOCAL
-    {
-        const int sms = num_sms();
-        uint32_t *H = U32(L.bin_hist);
-        uint32_t *totals = U32(L.tile_count);
-        const int4 *rect = reinterpret_cast<const int4 *>(proj.rect);
-        const float4 *xyod = reinterpret_cast<const float4 *>(proj.xy_opacity_depth);
-        uint32_t *order = U32(L.tile_order);
-        // the emitted sort keys, u64[max_pairs], over the (ptile_a, pgid_a) scratch
-        uint64_t *keys = reinterpret_cast<uint64_t *>(base + L.ptile_a);
-        int64_t ctas64 = std::min<int64_t>((int64_t)2 * sms, (int64_t)kBinCTAsMax);
-        ctas64 = std::min<int64_t>(ctas64, kBinHistCap / tiles);
-        const int ctas = (int)std::max<int64_t>(1, ctas64);
-        const size_t cnt_smem = tiles <= kSmemTiles ? (size_t)tiles * sizeof(uint32_t) : 0;
-        static bool attr = [] {
-            cudaFuncSetAttribute(k_bin_count, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                 (int)(kSmemTiles * sizeof(uint32_t)));
-            cudaFuncSetAttribute(k_bin_emit, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                 (int)(kSmemTiles * sizeof(uint32_t)));
-            cudaFuncSetAttribute(k_tile_sort<kMidWarps>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                 (int)(2 * kTileSortMid * sizeof(uint64_t)));
-            return true;
-        }();
-        (void)attr;
-        prof_before("bin_count", s);
-        k_bin_count<<<ctas, kBinThreads, cnt_smem, s>>>((int)n, rect, c.tiles_x, c.tiles_y, H);
-        k_bin_colscan<<<(tiles + 31) / 32, 256, 0, s>>>(tiles, ctas, H, totals);
-        prof_after(s);
-        prof_before("tile_scan", s);
-        k_tile_scan<<<1, kScanTilesThreads, 0, s>>>(tiles, totals, (uint64_t)bins.max_pairs, ranges, order,
-                                                    n_pairs, status);
-        prof_after(s);
-        if (n > 0) {
-            prof_before("emit", s);
-            k_bin_emit<<<ctas, kBinThreads, cnt_smem, s>>>((int)n, rect, xyod, c.tiles_x, c.tiles_y, ranges, H,
-                                                           keys, status);
-            prof_after(s);
-            prof_before("tile_sort", s);
-            k_tile_sort_warp<<<(tiles + 3) / 4, 128, 0, s>>>(ranges, order, tiles, keys, bins.pair_gid,
-                                                              bins.pair_tile);
-            k_tile_sort<kShortWarps><<<tiles, kShortWarps * 32, 2 * kTileSortShort * sizeof(uint64_t), s>>>(
-                ranges, order, tiles, keys, bins.pair_gid, bins.pair_tile, 256u, 0);
-            k_tile_sort<kMidWarps><<<std::min(tiles, sms), kMidWarps * 32, 2 * kTileSortMid * sizeof(uint64_t),
-                                     s>>>(ranges, order, tiles, keys, bins.pair_gid, bins.pair_tile,
-                                          kTileSortShort, 1);
-            k_tile_sort_long<<<std::min(tiles, sms), 256, 0, s>>>(
-                ranges, order, tiles, keys, bins.pair_gid, bins.pair_tile, kTileSortMid, U32(L.ptile_b),
-                U32(L.pgid_b), bins.pair_tile, bins.pair_gid);
-            prof_after(s);
-        }
-        return cudaGetLastError();
-    }
-#endif
-    if (n == 0) return tile_order();  // K = 0, all ranges empty
-
-    const int sms = num_sms();
-    const uint32_t nn = (uint32_t)n;
-    // 1. depth keys + histograms
-    {
-        const int blocks = (int)std::min<int64_t>((n + 255) / 256, (int64_t)sms * 4);
-        prof_before("depth_keys", s);
-        k_depth_keys<<<blocks, 256, 0, s>>>((int)n, reinterpret_cast<const float4 *>(proj.xy_opacity_depth),
-                                             reinterpret_cast<const int4 *>(proj.rect), c.tiles_x, c.tiles_y,
-                                             U32(L.keys_a), depth_hist);
-        prof_after(s);
-    }
-    // 2. depth sort: 31 bits in four passes, A -> B -> A -> B -> A
-    {
-        const int shifts[4] = {0, 8, 16, 24}, bits[4] = {8, 8, 8, 7};
-        uint32_t *ka = U32(L.keys_a), *va = U32(L.vals_a), *kb = U32(L.keys_b), *vb = U32(L.vals_b);
-        const int64_t parts = (n + kSortPart - 1) / kSortPart;
-        const int blocks = (int)std::min<int64_t>(parts, (int64_t)sms * 4);
-        for (int pass = 0; pass < 4; pass++) {
-            const bool even = (pass % 2) == 0;
-            prof_before("depth_sort", s);
-            k_onesweep<<<blocks, kSortThreads, 0, s>>>(
-                even ? ka : kb, even ? va : vb, even ? kb : ka, even ? vb : va, nullptr, nn, nn,
-                shifts[pass], bits[pass], depth_hist + pass * kRadix,
-                U32(L.depth_lb) + (size_t)pass * L.depth_parts * kRadix, tickets + pass, status,
-                pass == 0 ? 1 : 0, 0);
-            prof_after(s);
-        }
-    }
-    // 3. scan of the counts in depth order, then the pair emit.  The scan's
-    //    per-Gaussian records reuse the depth sort's spare buffers: keys_b
-    //    (inclusive offsets), vals_b (packed first tile), keys_a (widths);
-    //    the sorted ids stay in vals_a.
-    int tile_bits = 0;
-    while ((1 << tile_bits) < tiles) tile_bits++;
-    const int tile_passes = (tile_bits + kRadixBits - 1) / kRadixBits;
-    const int tile_bpp = tile_passes ? (tile_bits + tile_passes - 1) / tile_passes : 1;
-    uint32_t *ta = U32(L.ptile_a), *ga = U32(L.pgid_a), *tb = U32(L.ptile_b), *gb = U32(L.pgid_b);
-    uint32_t *to = bins.pair_tile, *go = bins.pair_gid;
-    {
-        const int blocks = (int)((n + kScanPart - 1) / kScanPart);
-        prof_before("scan", s);
-        k_scan<<<blocks, kScanThreads, 0, s>>>((int)n, U32(L.vals_a), reinterpret_cast<const int4 *>(proj.rect),
-                                              c.tiles_x, c.tiles_y, U32(L.keys_b), U32(L.vals_b),
-                                              U32(L.keys_a), (uint64_t)bins.max_pairs,
-                                              reinterpret_cast<uint64_t *>(base + L.scan_lb), tickets + 4,
-                                              n_pairs, status);
-        prof_after(s);
-    }
-    {
-        const int64_t chunks = (bins.max_pairs + kEmitPairs - 1) / kEmitPairs;
-        const int blocks = (int)std::max<int64_t>(1, std::min<int64_t>(chunks, (int64_t)sms * 4));
-        uint32_t *et = tile_passes == 0 ? to : ta, *eg = tile_passes == 0 ? go : ga;
-        prof_before("emit", s);
-        k_emit<<<blocks, kEmitThreads, 0, s>>>((int)n, U32(L.keys_b), U32(L.vals_a), U32(L.vals_b),
-                                               U32(L.keys_a), c.tiles_x, n_pairs, status, et, eg, tile_hist,
-                                               tile_passes, tile_bpp);
-        prof_after(s);
-    }
-    // 4. stable pair sort on the tile bits
-    {
-        const int64_t parts = (bins.max_pairs + kSortPart - 1) / kSortPart;
-        const int blocks = (int)std::max<int64_t>(1, std::min<int64_t>(parts, (int64_t)sms * 4));
-        uint32_t *st = ta, *sg = ga;
-        for (int pass = 0; pass < tile_passes; pass++) {
-            uint32_t *dt, *dg;
-            if (pass == tile_passes - 1) { dt = to; dg = go; }
-            else if (st == ta) { dt = tb; dg = gb; }
-            else { dt = ta; dg = ga; }
-            const int sh = pass * tile_bpp;
-            const int nb = std::min(tile_bpp, tile_bits - sh);
-            prof_before("tile_sort", s);
-            k_onesweep<<<blocks, kSortThreads, 0, s>>>(
-                st, sg, dt, dg, n_pairs, 0u, (uint32_t)bins.max_pairs, sh, nb, tile_hist + pass * kRadix,
-                U32(L.tile_lb) + (size_t)pass * L.tile_parts * kRadix, tickets + 5 + pass, status, 0, 1);
-            prof_after(s);
-            st = dt; sg = dg;
-        }
-    }
-    // 5. ranges
-    {
-        const int blocks = sms * 4;
-        prof_before("ranges", s);
-        k_ranges<<<blocks, 256, 0, s>>>(bins.pair_tile, n_pairs, ranges, status);
-        prof_after(s);
-    }
-    // 6. the blend kernels' tile order
-    return tile_order();
+    // 1. per-CTA tile counts, 2. offsets down each tile's column
+    prof_before("bin_count", s);
+    k_bin_count<<<ctas, kBinThreads, cnt_smem, s>>>((int)n, rect, c.tiles_x, c.tiles_y, H);
+    k_bin_colscan<<<(tiles + 31) / 32, 256, 0, s>>>(tiles, ctas, H, totals);
+    prof_after(s, 2);
+    // 3. ranges, K, capacity check, tile order
+    prof_before("tile_scan", s);
+    k_tile_scan<<<1, kScanTilesThreads, 0, s>>>(tiles, totals, (uint64_t)bins.max_pairs, ranges, order,
+                                                n_pairs, status);
+    prof_after(s);
+    if (n == 0) return cudaGetLastError();  // K = 0, all ranges empty
+    // 4. emit the sort keys
+    prof_before("emit", s);
+    k_bin_emit<<<ctas, kBinThreads, cnt_smem, s>>>((int)n, rect, reinterpret_cast<const float4 *>(proj.xy_opacity_depth),
+                                                   c.tiles_x, c.tiles_y, ranges, H, keys, status);
+    prof_after(s);
+    // 5. sort each tile's list, by size class
+    prof_before("tile_sort", s);
+    k_tile_sort_warp<<<(tiles + 3) / 4, 128, 0, s>>>(ranges, order, tiles, keys, bins.pair_gid, bins.pair_tile);
+    k_tile_sort<kShortWarps><<<tiles, kShortWarps * 32, 2 * kTileSortShort * sizeof(uint64_t), s>>>(
+        ranges, order, tiles, keys, bins.pair_gid, bins.pair_tile, 256u, 0);
+    k_tile_sort<kMidWarps><<<std::min(tiles, sms), kMidWarps * 32, 2 * kTileSortMid * sizeof(uint64_t), s>>>(
+        ranges, order, tiles, keys, bins.pair_gid, bins.pair_tile, kTileSortShort, 1);
+    k_tile_sort_long<<<std::min(tiles, sms), 256, 0, s>>>(ranges, order, tiles, keys, bins.pair_gid,
+                                                          bins.pair_tile, kTileSortMid, U32(L.long_keys),
+                                                          U32(L.long_ids), bins.pair_tile, bins.pair_gid);
+    prof_after(s, 4);
+    return cudaGetLastError();
 }
 
 }  // namespace gs

@@ -58,7 +58,8 @@ enum {
     GS_ERR_TOO_LARGE = -3,      /* N or max_pairs at or above 2^30 */
     GS_ERR_ALIGNMENT = -4,      /* a pointer is not aligned as documented */
     GS_ERR_CUDA = -5,           /* a CUDA runtime call or launch failed */
-    GS_ERR_DEVICE_TIMEOUT = -6  /* a bounded device-side wait gave up */
+    GS_ERR_DEVICE_TIMEOUT = -6  /* a bounded device-side wait gave up (reserved:
+                                   no kernel of this version waits on another) */
 };
 
 /* Pinhole camera ([GSP] s3).  Host struct, passed by pointer. */
@@ -141,8 +142,7 @@ typedef struct gs_bins {
     uint64_t *n_pairs;    /* [1] total pairs K of the last gs_bin_and_sort (also when
                              K > max_pairs) */
     int32_t *status;      /* [1] 0, or the GS_ERR_* code a kernel of the last
-                             gs_bin_and_sort recorded (GS_ERR_CAPACITY,
-                             GS_ERR_DEVICE_TIMEOUT) */
+                             gs_bin_and_sort recorded (GS_ERR_CAPACITY) */
     int64_t max_pairs;    /* capacity of pair_tile / pair_gid */
     int64_t max_n;        /* largest N this buffer was carved for */
     int32_t max_tiles;    /* largest tile count this buffer was carved for */
@@ -175,12 +175,11 @@ int gs_bins_carve(void *base, int64_t n, int64_t max_pairs, int32_t width, int32
 int gs_project(const gs_camera *cam, int64_t n, const gs_params *params, const gs_projected *out,
                void *stream);
 
-/* Binning and sorting ([WEEK] count, emit, sort, range): sorts the drawable
- * Gaussians by depth (LSD radix over the 31 used bits of camera z), scans
- * their tile counts in that order, emits one (tile, id) pair per touched
- * tile at the scanned offsets, sorts the pairs stably by tile (LSD radix over
- * the used tile-id bits only), and writes each tile's range.  The result is
- * the pair order of the 64-bit key (tile << 32 | depth bits) with ties by id.
+/* Binning and sorting ([WEEK] count, emit, sort, range): counts the pairs
+ * of every tile, scans the counts into per-tile ranges, emits one entry per
+ * (tile, drawable Gaussian) at its tile's range, and sorts each tile's list
+ * by (float bits of camera z, Gaussian id).  The result is the pair order of
+ * the 64-bit key (tile << 32 | depth bits) with ties by id.
  * It also leaves in bins->scratch the order in which the blend kernels take
  * the tiles (longest list first); the render calls need bins filled by this
  * call.
@@ -193,7 +192,7 @@ int gs_project(const gs_camera *cam, int64_t n, const gs_params *params, const g
  * NULL nothing synchronizes: K and any error land in bins->n_pairs and
  * bins->status (read them with gs_read_status); on an error every tile's
  * range is left empty, so the render draws only background.
- * Errors: INVALID_ARG, TOO_LARGE, ALIGNMENT, CUDA, CAPACITY, DEVICE_TIMEOUT. */
+ * Errors: INVALID_ARG, TOO_LARGE, ALIGNMENT, CUDA, CAPACITY. */
 int gs_bin_and_sort(const gs_camera *cam, int64_t n, const gs_projected *proj,
                     const gs_bins *bins, int64_t *n_pairs_host, void *stream);
 
@@ -262,7 +261,7 @@ int gs_l1_loss_grad(const float *image, const float *target, int64_t count, floa
  *
  * Limits (GS_ERR_TOO_LARGE beyond them, nothing launched): n <= 262,144
  * Gaussians, max_pairs <= 1,048,576 pairs, at most 65,536 tiles.  The array
- * (about 21 MB) is part of the library's device image: every GPU on which
+ * (about 33 MB) is part of the library's device image: every GPU on which
  * the library is used holds it until the process exits.
  *
  * Inputs: cam, n, proj as for gs_bin_and_sort.  Outputs (device, caller-owned):
@@ -272,8 +271,7 @@ int gs_l1_loss_grad(const float *image, const float *target, int64_t count, floa
  *   *n_pairs_host (HOST, required)               K, the total pair count
  * The call synchronizes `stream` to read K and the kernels' status back, and
  * returns GS_ERR_CAPACITY when K > max_pairs (the pair arrays are then left
- * undefined and the ranges empty) or GS_ERR_DEVICE_TIMEOUT, as
- * gs_bin_and_sort does.  It calls no allocating routine.
+ * undefined and the ranges empty), as gs_bin_and_sort does.  It calls no allocating routine.
  *
  * The first call on each device looks up the array's device address
  * (cudaGetSymbolAddress) with that device current; make that first call
@@ -292,11 +290,13 @@ int gs_read_status(const gs_bins *bins, int64_t *n_pairs_host, void *stream);
 /* Static, human-readable text for a return code. */
 const char *gs_error_string(int code);
 
-/* Per-kernel timing.  Between gs_profile_begin and gs_profile_end the library
- * records a CUDA event pair around each kernel it launches, on the stream it
- * launches it on.  gs_profile_end synchronizes those events and fills at
- * most max_stats entries (one per kernel name); returns how many.  Not
- * thread-safe; meant for benchmarks. */
+/* Per-stage timing.  Between gs_profile_begin and gs_profile_end the library
+ * records a CUDA event pair around each stage it launches (one kernel, or a
+ * few back to back: the count and column scan of binning, the per-tile
+ * sorts), on the stream it launches it on.  gs_profile_end synchronizes
+ * those events and fills at most max_stats entries (one per stage name:
+ * `launches` counts the kernels, `total_ms` the time); returns how many.
+ * Not thread-safe; meant for benchmarks. */
 typedef struct gs_profile_stat {
     char name[32];
     int32_t launches;

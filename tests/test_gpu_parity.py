@@ -112,8 +112,8 @@ def test_bin_and_sort_depth_ties_and_many_partitions():
 
 @pytest.mark.parametrize("W,H", [(16, 16), (1, 1), (17, 1), (4112, 4112)])
 def test_bin_and_sort_tile_bit_widths(W, H):
-    """0 tile bits (one tile, no pair sort), 1 and 2 tiles, and 257 x 257
-    tiles (17 bits: three sort passes)."""
+    """One tile, 1 x 2 tiles, and 257 x 257 tiles (66049: the count matrix
+    then takes fewer CTAs and rows longer than shared memory)."""
     cam = Camera(np.eye(4), W * 0.5, W * 0.5, W / 2.0, H / 2.0, W, H)
     rng = np.random.default_rng(W + H)
     n = 700
