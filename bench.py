@@ -82,6 +82,11 @@ BYTES = {
     "tile_sort": lambda G, P: 16 * P,
     "project_bwd": lambda G, P: 240 * G,
 }
+ALU_KERNELS = ("render_fwd", "render_bwd")
+
+# DRAM traffic per launch of render_bwd measured by ncu
+# (dram__bytes_read.sum + dram__bytes_write.sum), valid only for the kernel
+# source it was taken on.
 TRAFFIC = {}  # {"render_bwd": {"src_sha": ..., "bytes_per_pair": ...}}
 
 

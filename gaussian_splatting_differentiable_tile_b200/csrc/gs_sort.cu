@@ -240,7 +240,7 @@ k_tile_scan(int tiles, const uint32_t *__restrict__ totals, uint64_t max_pairs,
         off += c;
     }
     auto bucket = [&](int i) {
-        const uint32_t len = ranges[2 * (size_t)i + 1] - ranges[2 * (size_t)i];
+        const uint32_t len = ok ? totals[i] : 0u;
         return kScanTilesThreads - 1 - (int)min(len >> 2, (uint32_t)(kScanTilesThreads - 1));
     };
     s_off[t] = 0;
@@ -382,20 +382,101 @@ k_tile_sort_warp(const uint32_t *__restrict__ ranges, const uint32_t *__restrict
     }
 }
 
+// A tile list too long for the shared-memory sort: LSD radix sort of its
+// keys in global memory by the whole CTA (8-bit digits: four passes over the
+// id, then four over the depth bits; each pass stable, in chunks of kThreads
+// ranked with warp ballots), ping-ponging between (ka, va) and (kb, vb) at
+// the same offsets as the tile's range.  Writes the result to pair_gid and
+// pair_tile.  s_wc holds kThreads / 32 rows of 256 counters.
+template <int kThreads>
+__device__ void global_radix_sort_tile(uint32_t start, uint32_t end, uint32_t tile,
+                                       const uint64_t *__restrict__ keys, uint32_t *ka, uint32_t *va,
+                                       uint32_t *kb, uint32_t *vb, uint32_t *__restrict__ pair_gid,
+                                       uint32_t *__restrict__ pair_tile, uint32_t *s_base, uint32_t *s_tot,
+                                       uint32_t (*s_wc)[kRadix]) {
+    constexpr int kWarps = kThreads / 32;
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    for (uint32_t i = start + tid; i < end; i += kThreads) {
+        const uint64_t key = keys[i];
+        ka[i] = (uint32_t)(key >> 32);
+        va[i] = (uint32_t)key;
+    }
+    __syncthreads();
+    uint32_t *sk = ka, *sv = va, *dk = kb, *dv = vb;
+    for (int pass = 0; pass < 8; pass++) {
+        const bool on_id = pass < 4;
+        const int shift = 8 * (pass & 3);
+        for (int d = tid; d < kRadix; d += kThreads) s_base[d] = 0;
+        __syncthreads();
+        for (uint32_t i = start + tid; i < end; i += kThreads)
+            atomicAdd(&s_base[((on_id ? sv[i] : sk[i]) >> shift) & 0xFFu], 1u);
+        __syncthreads();
+        if (tid == 0) {  // exclusive scan, in place
+            uint32_t acc = start;
+            for (int d = 0; d < kRadix; d++) {
+                const uint32_t c = s_base[d];
+                s_base[d] = acc;
+                acc += c;
+            }
+        }
+        __syncthreads();
+        for (uint32_t c0 = start; c0 < end; c0 += kThreads) {
+            const uint32_t i = c0 + tid;
+            const bool in = i < end;
+            const uint32_t key = in ? sk[i] : 0u, val = in ? sv[i] : 0u;
+            const uint32_t d = in ? ((on_id ? val : key) >> shift) & 0xFFu : (uint32_t)kRadix;
+            for (int k = tid; k < kWarps * kRadix; k += kThreads) (&s_wc[0][0])[k] = 0;
+            __syncthreads();
+            const uint32_t peers = digit_peers(d, 8);
+            if (in && lane == __ffs(peers) - 1) s_wc[warp][d] = __popc(peers);
+            __syncthreads();
+            for (int dd = tid; dd < kRadix; dd += kThreads) {  // exclusive over warps
+                uint32_t acc = 0;
+                for (int ww = 0; ww < kWarps; ww++) {
+                    const uint32_t c = s_wc[ww][dd];
+                    s_wc[ww][dd] = acc;
+                    acc += c;
+                }
+                s_tot[dd] = acc;
+            }
+            __syncthreads();
+            if (in) {
+                const uint32_t pos = s_base[d] + s_wc[warp][d] + __popc(peers & lanemask_lt());
+                dk[pos] = key;
+                dv[pos] = val;
+            }
+            __syncthreads();
+            for (int dd = tid; dd < kRadix; dd += kThreads) s_base[dd] += s_tot[dd];
+            __syncthreads();
+        }
+        uint32_t *t0 = sk, *t1 = sv;
+        sk = dk; sv = dv; dk = t0; dv = t1;
+        __syncthreads();
+    }
+    for (uint32_t i = start + tid; i < end; i += kThreads) {
+        pair_gid[i] = sv[i];
+        pair_tile[i] = tile;
+    }
+    __syncthreads();
+}
+
 // Tile lists in (lo, hi], hi = 256 kWarps: sorted by one CTA each.  Warp w
 // sorts keys [256 w, 256 w + 256) in registers; the runs are then merged
 // pairwise in shared memory (each key's output position is its index plus
-// its rank in the other run).  With `persistent` a small grid walks the tile
+// its rank in the other run).  With kLong the CTA also takes lists above hi,
+// by a radix sort in global memory.  With `persistent` a small grid walks the tile
 // order (longest first) and stops at the first tile whose length bucket
 // lies below lo's; otherwise CTA b takes the b-th tile of the order.
-template <int kWarps>
+template <int kWarps, bool kLong>
 __global__ void __launch_bounds__(kWarps * 32)
 k_tile_sort(const uint32_t *__restrict__ ranges, const uint32_t *__restrict__ order, int tiles,
             const uint64_t *__restrict__ keys, uint32_t *__restrict__ pair_gid,
-            uint32_t *__restrict__ pair_tile, uint32_t lo, int persistent) {
+            uint32_t *__restrict__ pair_tile, uint32_t lo, int persistent, uint32_t *ka, uint32_t *va) {
     constexpr int kThreads = kWarps * 32;
     constexpr uint32_t kHi = 256u * kWarps;
     extern __shared__ uint64_t s_buf[];
+    __shared__ uint32_t s_base[kLong ? kRadix : 1], s_tot[kLong ? kRadix : 1];
+    __shared__ uint32_t s_wc[kLong ? kWarps : 1][kRadix];
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
     const int step = persistent ? (int)gridDim.x : tiles;
     for (int b = blockIdx.x; b < tiles; b += step) {
@@ -403,7 +484,15 @@ k_tile_sort(const uint32_t *__restrict__ ranges, const uint32_t *__restrict__ or
         const uint32_t start = ranges[2 * (size_t)tile], end = ranges[2 * (size_t)tile + 1];
         const uint32_t L = end - start;
         if (persistent && order_bucket(L) < order_bucket(lo)) break;
-        if (L <= lo || L > kHi) continue;
+        if (L <= lo) continue;
+        if (L > kHi) {
+            // longer than shared memory holds: sorted in global memory, with
+            // (pair_tile, pair_gid) as the second ping-pong buffer
+            if (kLong)
+                global_radix_sort_tile<kThreads>(start, end, tile, keys, ka, va, pair_tile, pair_gid, pair_gid,
+                                                 pair_tile, s_base, s_tot, s_wc);
+            continue;
+        }
         const int chunks = (int)((L + 255) / 256);
         int runs = 1;
         while (runs < chunks) runs <<= 1;
@@ -447,86 +536,6 @@ k_tile_sort(const uint32_t *__restrict__ ranges, const uint32_t *__restrict__ or
     }
 }
 
-// Tiles longer than the shared-memory sort holds: one CTA per tile runs an
-// LSD radix sort of the tile's keys in global memory (8-bit digits: four
-// passes over the id, then four over the depth bits; each pass stable, in
-// chunks of 256 ranked with warp ballots), ping-ponging between (ka, va) and
-// (kb, vb) at the same offsets as the tile's range.
-__global__ void __launch_bounds__(256)
-k_tile_sort_long(const uint32_t *__restrict__ ranges, const uint32_t *__restrict__ order, int tiles,
-                 const uint64_t *__restrict__ keys, uint32_t *__restrict__ pair_gid,
-                 uint32_t *__restrict__ pair_tile, uint32_t lo, uint32_t *__restrict__ ka,
-                 uint32_t *__restrict__ va, uint32_t *__restrict__ kb, uint32_t *__restrict__ vb) {
-    __shared__ uint32_t s_base[kRadix];
-    __shared__ uint32_t s_wc[8][kRadix];
-    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-    for (int b = blockIdx.x; b < tiles; b += gridDim.x) {
-        const uint32_t tile = order[b];
-        const uint32_t start = ranges[2 * (size_t)tile], end = ranges[2 * (size_t)tile + 1];
-        if (order_bucket(end - start) < order_bucket(lo)) break;
-        if (end - start <= lo) continue;
-        for (uint32_t i = start + tid; i < end; i += 256) {
-            const uint64_t key = keys[i];
-            ka[i] = (uint32_t)(key >> 32);
-            va[i] = (uint32_t)key;
-        }
-        __syncthreads();
-        uint32_t *sk = ka, *sv = va, *dk = kb, *dv = vb;
-        for (int pass = 0; pass < 8; pass++) {
-            const bool on_id = pass < 4;
-            const int shift = 8 * (pass & 3);
-            s_base[tid] = 0;
-            __syncthreads();
-            for (uint32_t i = start + tid; i < end; i += 256)
-                atomicAdd(&s_base[((on_id ? sv[i] : sk[i]) >> shift) & 0xFFu], 1u);
-            __syncthreads();
-            if (tid == 0) {  // exclusive scan, in place
-                uint32_t acc = start;
-                for (int d = 0; d < kRadix; d++) {
-                    const uint32_t c = s_base[d];
-                    s_base[d] = acc;
-                    acc += c;
-                }
-            }
-            __syncthreads();
-            for (uint32_t c0 = start; c0 < end; c0 += 256) {
-                const uint32_t i = c0 + tid;
-                const bool in = i < end;
-                const uint32_t key = in ? sk[i] : 0u, val = in ? sv[i] : 0u;
-                const uint32_t d = in ? ((on_id ? val : key) >> shift) & 0xFFu : (uint32_t)kRadix;
-                for (int k = tid; k < 8 * kRadix; k += 256) (&s_wc[0][0])[k] = 0;
-                __syncthreads();
-                const uint32_t peers = digit_peers(d, 8);
-                if (in && lane == __ffs(peers) - 1) s_wc[warp][d] = __popc(peers);
-                __syncthreads();
-                uint32_t acc = 0;  // per digit (thread = digit): exclusive over warps
-                for (int ww = 0; ww < 8; ww++) {
-                    const uint32_t c = s_wc[ww][tid];
-                    s_wc[ww][tid] = acc;
-                    acc += c;
-                }
-                __syncthreads();
-                if (in) {
-                    const uint32_t pos = s_base[d] + s_wc[warp][d] + __popc(peers & lanemask_lt());
-                    dk[pos] = key;
-                    dv[pos] = val;
-                }
-                __syncthreads();
-                s_base[tid] += acc;
-                __syncthreads();
-            }
-            uint32_t *t0 = sk, *t1 = sv;
-            sk = dk; sv = dv; dk = t0; dv = t1;
-            __syncthreads();
-        }
-        for (uint32_t i = start + tid; i < end; i += 256) {
-            pair_gid[i] = sv[i];
-            pair_tile[i] = tile;
-        }
-        __syncthreads();
-    }
-}
-
 int num_sms() {
     static int sms = 0;
     if (sms == 0) {
@@ -564,7 +573,7 @@ cudaError_t launch_bin_and_sort(const CamConst &c, int64_t n, const gs_projected
                              (int)(kSmemTiles * sizeof(uint32_t)));
         cudaFuncSetAttribute(k_bin_emit, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              (int)(kSmemTiles * sizeof(uint32_t)));
-        cudaFuncSetAttribute(k_tile_sort<kMidWarps>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+        cudaFuncSetAttribute(k_tile_sort<kMidWarps, true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              (int)(2 * kTileSortMid * sizeof(uint64_t)));
         return true;
     }();
@@ -591,14 +600,12 @@ cudaError_t launch_bin_and_sort(const CamConst &c, int64_t n, const gs_projected
     // 5. sort each tile's list, by size class
     prof_before("tile_sort", s);
     k_tile_sort_warp<<<(tiles + 3) / 4, 128, 0, s>>>(ranges, order, tiles, keys, bins.pair_gid, bins.pair_tile);
-    k_tile_sort<kShortWarps><<<tiles, kShortWarps * 32, 2 * kTileSortShort * sizeof(uint64_t), s>>>(
-        ranges, order, tiles, keys, bins.pair_gid, bins.pair_tile, 256u, 0);
-    k_tile_sort<kMidWarps><<<std::min(tiles, sms), kMidWarps * 32, 2 * kTileSortMid * sizeof(uint64_t), s>>>(
-        ranges, order, tiles, keys, bins.pair_gid, bins.pair_tile, kTileSortShort, 1);
-    k_tile_sort_long<<<std::min(tiles, sms), 256, 0, s>>>(ranges, order, tiles, keys, bins.pair_gid,
-                                                          bins.pair_tile, kTileSortMid, U32(L.long_keys),
-                                                          U32(L.long_ids), bins.pair_tile, bins.pair_gid);
-    prof_after(s, 4);
+    k_tile_sort<kShortWarps, false><<<tiles, kShortWarps * 32, 2 * kTileSortShort * sizeof(uint64_t), s>>>(
+        ranges, order, tiles, keys, bins.pair_gid, bins.pair_tile, 256u, 0, nullptr, nullptr);
+    k_tile_sort<kMidWarps, true><<<std::min(tiles, sms), kMidWarps * 32, 2 * kTileSortMid * sizeof(uint64_t), s>>>(
+        ranges, order, tiles, keys, bins.pair_gid, bins.pair_tile, kTileSortShort, 1, U32(L.long_keys),
+        U32(L.long_ids));
+    prof_after(s, 3);
     return cudaGetLastError();
 }
 
