@@ -65,8 +65,21 @@ typedef struct {
     int32_t width, height;
     double near_z;
     double bg[3];
-    int32_t tight_tiles;  /* 1: narrow each tile rectangle by the opacity-aware cut */
+    int32_t flags;        /* ORC_FLAG_* bits: the variants below */
 } orc_camera;
+
+/* Variants of the method the pages describe, as camera flag bits (the values
+ * the library's camera uses for the same options). */
+#define ORC_FLAG_TIGHT_TILES    1  /* opacity-aware tile cut (opacity_cut)            */
+#define ORC_FLAG_ANTIALIASED    2  /* [GSP] s4: opacity x sqrt(det S' / det S'')      */
+#define ORC_FLAG_STOP_INCLUSIVE 4  /* [GSP] s5, gsplat: stop once next_T <= 1e-4      */
+#define ORC_FLAG_CAP_0999       8  /* [GSP] s6, older gsplat: alpha cap 0.999         */
+#define ORC_FLAG_RADII_AXIS    16  /* [GSP] s4, gsplat: radii ceil(3.33 sqrt(S''_xx)), */
+                                   /* ceil(3.33 sqrt(S''_yy)) per axis                */
+#define ORC_FLAG_RADII_OPACITY 32  /* with RADII_AXIS: min(3.33, sqrt(2 ln(255 o)))   */
+                                   /* standard deviations; 255 o <= 1 touches nothing */
+#define ORC_GSPLAT_SIGMAS 3.33
+#define ORC_ALPHA_CAP_0999_F 0.999f
 
 /* Single-precision decision constants, as the [GSP] s5 listing writes them. */
 #define ORC_ALPHA_CAP_F   0.99f
@@ -137,6 +150,11 @@ typedef struct {
     double opacity;
     double lambda_max;
     double radius_value;   /* 3 sqrt(lambda) before the ceiling */
+    double opacity_raw;    /* sigmoid(logit) */
+    double det_orig;       /* det of the undilated 2D covariance */
+    double comp;           /* antialiasing compensation (1 without the flag) */
+    double rx_value, ry_value;  /* per-axis radii before the ceiling */
+    int extent_empty;      /* RADII_OPACITY and 255 o <= 1: no tiles */
 } orc_proj;
 
 static void project_one(const double *mean, const double *log_scale, const double *quat,
@@ -152,6 +170,8 @@ static void project_one(const double *mean, const double *log_scale, const doubl
     orc_quat_to_rotmat(quat, P->R);
     for (int j = 0; j < 3; j++) P->s[j] = exp(log_scale[j]);
     P->opacity = 1.0 / (1.0 + exp(-opacity_logit));
+    P->opacity_raw = P->opacity;
+    P->comp = 1.0;
 
     /* [GSP] s2: Sigma = (R S)(R S)^T. */
     for (int i = 0; i < 3; i++)
@@ -253,6 +273,35 @@ static void project_one(const double *mean, const double *log_scale, const doubl
     P->lambda_max = mid + sqrt(disc);
     P->radius_value = ORC_RADIUS_SIGMAS * sqrt(P->lambda_max);
 
+    /* [GSP] s4, antialiased mode: the opacity is scaled by
+     * sqrt(det Sigma' / det Sigma'') (0 when det Sigma' <= 0), which keeps a
+     * small splat's total energy instead of fattening it. */
+    P->det_orig = cov[0] * cov[3] - cov[1] * cov[1];
+    if (cam->flags & ORC_FLAG_ANTIALIASED) {
+        P->comp = P->det_orig > 0.0 ? sqrt(P->det_orig / det) : 0.0;
+        P->opacity = P->opacity_raw * P->comp;
+    }
+    /* [GSP] s4, gsplat radii: the 3.33-sigma extent of the ellipse along x
+     * and y, optionally shrunk to where the (compensated) opacity fades
+     * below 1/255. */
+    P->rx_value = P->ry_value = P->radius_value;
+    P->extent_empty = 0;
+    if (cam->flags & ORC_FLAG_RADII_AXIS) {
+        double e = ORC_GSPLAT_SIGMAS;
+        if (cam->flags & ORC_FLAG_RADII_OPACITY) {
+            double l = log(255.0 * P->opacity);
+            if (l > 0.0) {
+                double ee = sqrt(2.0 * l);
+                if (ee < e) e = ee;
+            } else {
+                e = 0.0;
+                P->extent_empty = 1;
+            }
+        }
+        P->rx_value = e * sqrt(P->a);
+        P->ry_value = e * sqrt(P->c);
+    }
+
     /* [GSP] s3: the 2D mean is not clamped. */
     P->mean2d[0] = cam->fx * tx / tz + cam->cx;
     P->mean2d[1] = cam->fy * ty / tz + cam->cy;
@@ -327,16 +376,16 @@ static double opacity_cut(double mx, double my, double A, double B, double C, do
 }
 
 /* Tile rectangle of a splat, in float (a pixel grid decision taken in single
- * precision).  With cut (from opacity_cut) the bounds are narrowed to it
- * before clamping.  Returns the tile count; writes x0, y0, x1, y1
+ * precision), from per-axis radii (equal under the 3DGS rule).  With cut
+ * (from opacity_cut) the bounds are narrowed to it before clamping.  Returns the tile count; writes x0, y0, x1, y1
  * (inclusive), with x0 > x1 or y0 > y1 when nothing is touched. */
-static int32_t tile_rect_f32(float mx, float my, float r, int32_t tiles_x, int32_t tiles_y,
+static int32_t tile_rect_f32(float mx, float my, float rx, float ry, int32_t tiles_x, int32_t tiles_y,
                              const double *cut, int32_t *rect)
 {
-    float lx = floorf((mx - r) * (1.0f / ORC_TILE));
-    float hx = floorf((mx + r) * (1.0f / ORC_TILE));
-    float ly = floorf((my - r) * (1.0f / ORC_TILE));
-    float hy = floorf((my + r) * (1.0f / ORC_TILE));
+    float lx = floorf((mx - rx) * (1.0f / ORC_TILE));
+    float hx = floorf((mx + rx) * (1.0f / ORC_TILE));
+    float ly = floorf((my - ry) * (1.0f / ORC_TILE));
+    float hy = floorf((my + ry) * (1.0f / ORC_TILE));
     if (cut) {
         lx = fmaxf(lx, (float)cut[0]);
         hx = fminf(hx, (float)cut[1]);
@@ -358,18 +407,21 @@ static int32_t tile_rect_f32(float mx, float my, float r, int32_t tiles_x, int32
 
 /* Projection of n Gaussians ([GSP] s1-s4, s6).  Outputs, per Gaussian:
  *   mean2d[2], conic[3] (A, B, C), cov2d[3] (dilated a, b, c), opacity,
- *   depth (camera z), color[3] (passed through), radius (float, integral),
- *   rect[4] (tile x0, y0, x1, y1), count (tiles touched), valid (0/1),
- *   radius_margin (|3 sqrt(lambda) - nearest integer|, px),
+ *   depth (camera z), color[3] (passed through), radius (float, integral:
+ *   the larger of the two radii), radius_xy[2] (per-axis radii, equal under
+ *   the 3DGS rule), rect[4] (tile x0, y0, x1, y1), count (tiles touched),
+ *   valid (0/1), radius_margin (smallest |radius before the ceiling -
+ *   nearest integer|, px),
  *   rect_margin (min over the four rectangle edges of |(m +- r)/16 - nearest
- *   integer|, in tiles), cut_margin (what opacity_cut returns when
- *   cam->tight_tiles is set, else infinity).  The margins say how close an
+ *   integer|, in tiles), cut_margin (what opacity_cut returns with
+ *   ORC_FLAG_TIGHT_TILES, and |ln(255 o)| with the opacity-aware radii;
+ *   else infinity).  The margins say how close an
  *   integer decision came to flipping.  Returns 0, or -1 on bad arguments. */
 int orc_project(int64_t n, const double *means, const double *log_scales, const double *quats,
                 const double *opacity_logits, const double *colors, const orc_camera *cam,
                 double *mean2d, double *conic, double *cov2d, double *opacity, double *depth,
-                double *color, float *radius, int32_t *rect, int32_t *count, uint8_t *valid,
-                double *radius_margin, double *rect_margin, double *cut_margin)
+                double *color, float *radius, float *radius_xy, int32_t *rect, int32_t *count,
+                uint8_t *valid, double *radius_margin, double *rect_margin, double *cut_margin)
 {
     if (n < 0 || cam->width <= 0 || cam->height <= 0) return -1;
     int32_t tiles_x = (cam->width + ORC_TILE - 1) / ORC_TILE;
@@ -389,6 +441,7 @@ int orc_project(int64_t n, const double *means, const double *log_scales, const 
             conic[3 * g] = conic[3 * g + 1] = conic[3 * g + 2] = 0.0;
             cov2d[3 * g] = cov2d[3 * g + 1] = cov2d[3 * g + 2] = 0.0;
             radius[g] = 0.0f;
+            radius_xy[2 * g] = radius_xy[2 * g + 1] = 0.0f;
             rect[4 * g] = 0; rect[4 * g + 1] = 0; rect[4 * g + 2] = -1; rect[4 * g + 3] = -1;
             count[g] = 0;
             radius_margin[g] = INFINITY;
@@ -402,21 +455,33 @@ int orc_project(int64_t n, const double *means, const double *log_scales, const 
         cov2d[3 * g] = P.a;
         cov2d[3 * g + 1] = P.b;
         cov2d[3 * g + 2] = P.c;
-        /* radius: ceiling taken on the float-rounded value */
-        float r = ceilf((float)P.radius_value);
-        radius[g] = r;
-        radius_margin[g] = dist_to_int(P.radius_value);
+        /* radii: ceiling taken on the float-rounded values */
+        const float rxy[2] = {ceilf((float)P.rx_value), ceilf((float)P.ry_value)};
+        radius[g] = rxy[0] > rxy[1] ? rxy[0] : rxy[1];
+        radius_xy[2 * g] = rxy[0];
+        radius_xy[2 * g + 1] = rxy[1];
+        radius_margin[g] = fmin(dist_to_int(P.rx_value), dist_to_int(P.ry_value));
+        const int tight = (cam->flags & ORC_FLAG_TIGHT_TILES) != 0;
         double cut[4];
         cut_margin[g] = INFINITY;
-        if (cam->tight_tiles)
+        if (tight)
             cut_margin[g] = opacity_cut(P.mean2d[0], P.mean2d[1], P.conic[0], P.conic[1],
                                         P.conic[2], P.opacity, cut);
-        count[g] = tile_rect_f32((float)P.mean2d[0], (float)P.mean2d[1], r, tiles_x, tiles_y,
-                                 cam->tight_tiles ? cut : NULL, rect + 4 * g);
+        if (cam->flags & ORC_FLAG_RADII_OPACITY && cam->flags & ORC_FLAG_RADII_AXIS) {
+            double l = fabs(log(255.0 * P.opacity));
+            if (l < cut_margin[g]) cut_margin[g] = l;
+        }
+        if (P.extent_empty) {
+            rect[4 * g] = 0; rect[4 * g + 1] = 0; rect[4 * g + 2] = -1; rect[4 * g + 3] = -1;
+            count[g] = 0;
+        } else {
+            count[g] = tile_rect_f32((float)P.mean2d[0], (float)P.mean2d[1], rxy[0], rxy[1], tiles_x,
+                                     tiles_y, tight ? cut : NULL, rect + 4 * g);
+        }
         double m = INFINITY;
         for (int axis = 0; axis < 2; axis++) {
-            double e0 = (P.mean2d[axis] - (double)r) / ORC_TILE;
-            double e1 = (P.mean2d[axis] + (double)r) / ORC_TILE;
+            double e0 = (P.mean2d[axis] - (double)rxy[axis]) / ORC_TILE;
+            double e1 = (P.mean2d[axis] + (double)rxy[axis]) / ORC_TILE;
             double d0 = dist_to_int(e0), d1 = dist_to_int(e1);
             if (d0 < m) m = d0;
             if (d1 < m) m = d1;
@@ -427,10 +492,12 @@ int orc_project(int64_t n, const double *means, const double *log_scales, const 
 }
 
 /* Rectangle rule alone, for callers that already hold float records (used
- * to bin records that are given in single precision).  conic [n][3] and
- * opacity [n] are read only when tight_tiles is set; the cut is then taken
- * on their values as given. */
-int orc_tile_rects(int64_t n, const float *mean2d, const float *radius, const float *conic,
+ * to bin records that are given in single precision): radius_xy [n][2] per
+ * axis.  conic [n][3] and opacity [n] are read only when tight_tiles is set;
+ * the cut is then taken on their values as given.  Records whose radii are
+ * both 0 and whose opacity-aware extent was empty must be marked invalid by
+ * the caller. */
+int orc_tile_rects(int64_t n, const float *mean2d, const float *radius_xy, const float *conic,
                    const float *opacity, const uint8_t *valid, int32_t width, int32_t height,
                    int32_t tight_tiles, int32_t *rect, int32_t *count)
 {
@@ -447,8 +514,8 @@ int orc_tile_rects(int64_t n, const float *mean2d, const float *radius, const fl
         if (tight_tiles)
             (void)opacity_cut(mean2d[2 * g], mean2d[2 * g + 1], conic[3 * g], conic[3 * g + 1],
                               conic[3 * g + 2], opacity[g], cut);
-        count[g] = tile_rect_f32(mean2d[2 * g], mean2d[2 * g + 1], radius[g], tiles_x, tiles_y,
-                                 tight_tiles ? cut : NULL, rect + 4 * g);
+        count[g] = tile_rect_f32(mean2d[2 * g], mean2d[2 * g + 1], radius_xy[2 * g], radius_xy[2 * g + 1],
+                                 tiles_x, tiles_y, tight_tiles ? cut : NULL, rect + 4 * g);
     }
     return 0;
 }
@@ -628,18 +695,22 @@ static int64_t walk_pixel(const orc_render_ctx *c, int32_t i, int32_t j, orc_hit
         double sigma = 0.5 * (A * dx * dx + C * dy * dy) + B * dx * dy;
         double G = exp(-sigma);
         double oG = c->opacity[g] * G;
-        int clamped = (float)oG > ORC_ALPHA_CAP_F;
-        double alpha = clamped ? (double)ORC_ALPHA_CAP_F : oG;
+        const float acap = (c->cam->flags & ORC_FLAG_CAP_0999) ? ORC_ALPHA_CAP_0999_F : ORC_ALPHA_CAP_F;
+        int clamped = (float)oG > acap;
+        double alpha = clamped ? (double)acap : oG;
         if (sigma < 0.0) continue;
         double ma = rel_margin(alpha, (double)ORC_ALPHA_MIN_F);
         if (ma < ma_min) ma_min = ma;
         if ((float)alpha < ORC_ALPHA_MIN_F) continue;
-        double mcl = rel_margin(oG, (double)ORC_ALPHA_CAP_F);
+        double mcl = rel_margin(oG, (double)acap);
         if (mcl < mc) mc = mcl;
         double next_T = T * (1.0 - alpha);
         double mt = rel_margin(next_T, (double)ORC_T_MIN_F);
         if (mt < mt_min) mt_min = mt;
-        if ((float)next_T < ORC_T_MIN_F) break;
+        /* 3DGS stops when next_T < 1e-4; gsplat when next_T <= 1e-4 */
+        if ((c->cam->flags & ORC_FLAG_STOP_INCLUSIVE) ? (float)next_T <= ORC_T_MIN_F
+                                                      : (float)next_T < ORC_T_MIN_F)
+            break;
         for (int ch = 0; ch < 3; ch++) rgb[ch] += c->color[3 * g + ch] * alpha * T;
         if (hits) {
             if (nh == *cap) {
@@ -881,8 +952,10 @@ int orc_project_bwd(int64_t n, const double *means, const double *log_scales, co
         double d_mx = gg[0], d_my = gg[1], d_A = gg[2], d_B = gg[3], d_C = gg[4], d_o = gg[5];
         /* colour passes through */
         for (int k = 0; k < 3; k++) dc[k] = gg[6 + k];
-        /* sigmoid */
-        d_opacity_logits[g] = d_o * P.opacity * (1.0 - P.opacity);
+        /* opacity = sigmoid(logit) x comp; comp = sqrt(D1 / D2) with D1 the
+         * undilated and D2 the dilated determinant (antialiased mode) */
+        d_opacity_logits[g] = d_o * P.comp * P.opacity_raw * (1.0 - P.opacity_raw);
+        double d_comp = (cam->flags & ORC_FLAG_ANTIALIASED) && P.det_orig > 0.0 ? d_o * P.opacity_raw : 0.0;
 
         /* conic (A, B, C) = (c, -b, a) / det, det = a c - b^2 (no gradient
          * through det when it was clamped) */
@@ -893,6 +966,15 @@ int orc_project_bwd(int64_t n, const double *means, const double *log_scales, co
         double d_a = d_C / det + dl_ddet * P.c;
         double d_b = -d_B / det + dl_ddet * (-2.0 * P.b);
         double d_c = d_A / det + dl_ddet * P.a;
+        if (d_comp != 0.0) {
+            /* d comp = comp/2 (dD1/D1 - dD2/D2); D1 = (a - e)(c - e) - b^2,
+             * D2 = a c - b^2 (no D2 term when the det was clamped) */
+            const double h = 0.5 * P.comp * d_comp, D1 = P.det_orig;
+            const double k2 = P.det_clamped ? 0.0 : 1.0 / det;
+            d_a += h * ((P.c - ORC_EPS2D) / D1 - k2 * P.c);
+            d_c += h * ((P.a - ORC_EPS2D) / D1 - k2 * P.a);
+            d_b += h * (-2.0 * P.b / D1 + k2 * 2.0 * P.b);
+        }
         /* Sigma' = Sigma'' - 0.3 I has the same gradient; Sigma' = J Sc J^T */
         double Gp[4] = {d_a, 0.5 * d_b, 0.5 * d_b, d_c};
         /* dL/dSc = J^T Gp J */

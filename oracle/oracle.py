@@ -22,15 +22,21 @@ import numpy as np
 from . import build as _build
 
 __all__ = [
-    "TILE", "TIGHT_TILES", "OrcCamera", "lib", "quat_to_rotmat", "covariance3d", "project_debug", "project", "tile_rects",
+    "TILE", "TIGHT_TILES", "ANTIALIASED", "STOP_INCLUSIVE", "CAP_0999", "RADII_AXIS",
+    "RADII_OPACITY", "OrcCamera", "lib", "quat_to_rotmat", "covariance3d", "project_debug", "project", "tile_rects",
     "records_f32", "bin_pairs", "depth_order", "render", "render_bwd", "project_bwd",
     "grad_bound", "default_threads",
 ]
 
 TILE = 16
-# Camera flag bit that selects the opacity-aware tile cut (the value the
-# library's camera struct uses for the same option).
-TIGHT_TILES = 1
+# Camera flag bits of the variants (the values the library's camera struct
+# uses for the same options).
+TIGHT_TILES = 1       # opacity-aware tile cut
+ANTIALIASED = 2       # opacity x sqrt(det S' / det S'')
+STOP_INCLUSIVE = 4    # stop once next_T <= 1e-4 (gsplat)
+CAP_0999 = 8          # alpha cap 0.999 (older gsplat)
+RADII_AXIS = 16       # gsplat per-axis 3.33-sigma radii
+RADII_OPACITY = 32    # with RADII_AXIS: min(3.33, sqrt(2 ln(255 o))) sigmas
 
 _c_double_p = ctypes.POINTER(ctypes.c_double)
 _c_float_p = ctypes.POINTER(ctypes.c_float)
@@ -49,7 +55,7 @@ class OrcCamera(ctypes.Structure):
         ("width", ctypes.c_int32), ("height", ctypes.c_int32),
         ("near_z", ctypes.c_double),
         ("bg", ctypes.c_double * 3),
-        ("tight_tiles", ctypes.c_int32),
+        ("flags", ctypes.c_int32),
     ]
 
 
@@ -65,8 +71,8 @@ def lib() -> ctypes.CDLL:
         L.orc_quat_to_rotmat.argtypes = [_c_double_p, _c_double_p]
         L.orc_covariance3d.argtypes = [_c_double_p, _c_double_p, _c_double_p]
         L.orc_project.argtypes = [ctypes.c_int64] + [_c_double_p] * 5 + [ctypes.POINTER(OrcCamera)] + \
-            [_c_double_p] * 6 + [_c_float_p, _c_int32_p, _c_int32_p, _c_uint8_p, _c_double_p, _c_double_p,
-                                 _c_double_p]
+            [_c_double_p] * 6 + [_c_float_p, _c_float_p, _c_int32_p, _c_int32_p, _c_uint8_p, _c_double_p,
+                                 _c_double_p, _c_double_p]
         L.orc_project.restype = ctypes.c_int
         L.orc_tile_rects.argtypes = [ctypes.c_int64, _c_float_p, _c_float_p, _c_float_p, _c_float_p,
                                      _c_uint8_p, ctypes.c_int32, ctypes.c_int32, ctypes.c_int32,
@@ -116,7 +122,7 @@ def _cam(cam) -> OrcCamera:
     bg = np.asarray(cam.bg, dtype=np.float64).reshape(3)
     for k in range(3):
         c.bg[k] = float(bg[k])
-    c.tight_tiles = 1 if int(getattr(cam, "flags", 0)) & TIGHT_TILES else 0
+    c.flags = int(getattr(cam, "flags", 0))
     return c
 
 
@@ -164,7 +170,8 @@ def project(params: dict, cam) -> dict:
     out = {
         "mean2d": np.zeros((n, 2)), "conic": np.zeros((n, 3)), "cov2d": np.zeros((n, 3)),
         "opacity": np.zeros(n), "depth": np.zeros(n), "color": np.zeros((n, 3)),
-        "radius": np.zeros(n, dtype=np.float32), "rect": np.zeros((n, 4), dtype=np.int32),
+        "radius": np.zeros(n, dtype=np.float32), "radius_xy": np.zeros((n, 2), dtype=np.float32),
+        "rect": np.zeros((n, 4), dtype=np.int32),
         "count": np.zeros(n, dtype=np.int32), "valid": np.zeros(n, dtype=np.uint8),
         "radius_margin": np.zeros(n), "rect_margin": np.zeros(n), "cut_margin": np.zeros(n),
     }
@@ -175,7 +182,7 @@ def project(params: dict, cam) -> dict:
         _ptr(out["mean2d"], _c_double_p), _ptr(out["conic"], _c_double_p),
         _ptr(out["cov2d"], _c_double_p), _ptr(out["opacity"], _c_double_p),
         _ptr(out["depth"], _c_double_p), _ptr(out["color"], _c_double_p),
-        _ptr(out["radius"], _c_float_p), _ptr(out["rect"], _c_int32_p),
+        _ptr(out["radius"], _c_float_p), _ptr(out["radius_xy"], _c_float_p), _ptr(out["rect"], _c_int32_p),
         _ptr(out["count"], _c_int32_p), _ptr(out["valid"], _c_uint8_p),
         _ptr(out["radius_margin"], _c_double_p), _ptr(out["rect_margin"], _c_double_p),
         _ptr(out["cut_margin"], _c_double_p))
@@ -187,11 +194,13 @@ def project(params: dict, cam) -> dict:
 
 def tile_rects(mean2d32, radius32, valid, width: int, height: int, conic32=None, opacity32=None,
                tight: bool = False):
-    """The tile-rectangle rule alone, on single-precision records; with
-    ``tight`` the opacity-aware cut is taken on conic32 and opacity32."""
+    """The tile-rectangle rule alone, on single-precision records: radius32 is
+    one radius per Gaussian (n,) or per-axis radii (n, 2); with ``tight`` the
+    opacity-aware cut is taken on conic32 and opacity32."""
     m = np.ascontiguousarray(mean2d32, dtype=np.float32).reshape(-1, 2)
     n = m.shape[0]
-    r = np.ascontiguousarray(radius32, dtype=np.float32).reshape(n)
+    r = np.asarray(radius32, dtype=np.float32)
+    r = np.ascontiguousarray(np.repeat(r.reshape(n, 1), 2, axis=1) if r.ndim == 1 else r.reshape(n, 2))
     v = np.ascontiguousarray(valid, dtype=np.uint8).reshape(n)
     cn = np.ascontiguousarray(np.zeros((n, 3)) if conic32 is None else conic32, dtype=np.float32).reshape(n, 3)
     op = np.ascontiguousarray(np.zeros(n) if opacity32 is None else opacity32, dtype=np.float32).reshape(n)
@@ -215,9 +224,10 @@ def records_f32(proj: dict, width: int, height: int, tight: bool = False) -> dic
     for k in ("mean2d", "conic", "opacity", "color", "depth"):
         out[k] = np.asarray(proj[k], dtype=np.float32).astype(np.float64)
     out["depth32"] = np.asarray(proj["depth"], dtype=np.float32)
-    rect, count = tile_rects(out["mean2d"].astype(np.float32), proj["radius"], proj["valid"],
-                             width, height, out["conic"].astype(np.float32),
-                             out["opacity"].astype(np.float32), tight)
+    rxy = np.asarray(proj["radius_xy"], dtype=np.float32)
+    draws = proj["valid"].astype(bool) & np.any(rxy > 0, axis=1)  # an empty opacity extent draws nothing
+    rect, count = tile_rects(out["mean2d"].astype(np.float32), rxy, draws, width, height,
+                             out["conic"].astype(np.float32), out["opacity"].astype(np.float32), tight)
     out["rect"], out["count"] = rect, count
     return out
 

@@ -24,10 +24,11 @@ from scenes import Camera, tiny_camera
 H_STEP = 1e-6
 
 
-def _scene(seed, n=6, clamp_case=False, bg=(0.0, 0.0, 0.0)):
+def _scene(seed, n=6, clamp_case=False, bg=(0.0, 0.0, 0.0), flags=0):
     rng = np.random.default_rng(seed)
     W, H, f = 40, 36, 60.0
     cam = tiny_camera(W, H, f, distance=4.0, bg=bg)
+    cam.flags = flags
     means = np.column_stack([rng.uniform(-0.4, 0.4, n), rng.uniform(-0.4, 0.4, n),
                              rng.uniform(-0.5, 0.5, n)])
     params = {"means": means, "log_scales": rng.normal(-2.2, 0.3, (n, 3)),
@@ -104,9 +105,15 @@ def test_blend_backward_matches_finite_differences(bg):
     assert np.all(g2abs >= np.abs(g2) - 1e-15)
 
 
-@pytest.mark.parametrize("clamp_case", [False, True])
-def test_raw_parameter_gradients_match_finite_differences(clamp_case):
-    cam, params = _find_clean(300, clamp_case=clamp_case, bg=(0.1, 0.2, 0.3))
+ALL_VARIANTS = O.ANTIALIASED | O.RADII_AXIS | O.RADII_OPACITY | O.CAP_0999 | O.STOP_INCLUSIVE
+
+
+@pytest.mark.parametrize("clamp_case,flags", [(False, 0), (True, 0), (False, O.ANTIALIASED),
+                                              (True, ALL_VARIANTS)])
+def test_raw_parameter_gradients_match_finite_differences(clamp_case, flags):
+    """With the antialiased flag the chain also runs through the
+    compensation sqrt(det S' / det S'') into S' and the sigmoid."""
+    cam, params = _find_clean(300, clamp_case=clamp_case, bg=(0.1, 0.2, 0.3), flags=flags)
     if clamp_case:
         d = O.project_debug(params["means"][-1], params["log_scales"][-1], params["quats"][-1],
                             params["opacity_logits"][-1], cam)
