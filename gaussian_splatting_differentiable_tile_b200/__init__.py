@@ -25,7 +25,9 @@ import torch
 
 from . import _abi
 from ._abi import (GS_ERR_ALIGNMENT, GS_ERR_CAPACITY, GS_ERR_CUDA, GS_ERR_DEVICE_TIMEOUT,  # noqa: F401
-                   GS_ERR_INVALID_ARG, GS_ERR_TOO_LARGE, GS_FLAG_TIGHT_TILES, GS_OK, GS_TILE)
+                   GS_ERR_INVALID_ARG, GS_ERR_TOO_LARGE, GS_FLAG_ANTIALIASED, GS_FLAG_CAP_0999,
+                   GS_FLAG_RADII_AXIS, GS_FLAG_RADII_OPACITY, GS_FLAG_STOP_INCLUSIVE, GS_FLAG_TIGHT_TILES, GS_OK,
+                   GS_TILE)
 
 __all__ = [
     "GSError", "Projected", "Bins", "make_camera", "gs_project", "gs_bin_and_sort",

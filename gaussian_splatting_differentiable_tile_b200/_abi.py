@@ -21,6 +21,11 @@ GS_ERR_ALIGNMENT = -4
 GS_ERR_CUDA = -5
 GS_ERR_DEVICE_TIMEOUT = -6
 GS_FLAG_TIGHT_TILES = 1
+GS_FLAG_ANTIALIASED = 2
+GS_FLAG_STOP_INCLUSIVE = 4
+GS_FLAG_CAP_0999 = 8
+GS_FLAG_RADII_AXIS = 16
+GS_FLAG_RADII_OPACITY = 32
 
 c_float_p = ctypes.c_void_p  # device pointers travel as plain addresses
 

@@ -30,7 +30,7 @@ int make_cam(const gs_camera *cam, CamConst *out) {
         if (!std::isfinite(cam->viewmat[k])) return GS_ERR_INVALID_ARG;
     for (int k = 0; k < 3; k++)
         if (!std::isfinite(cam->bg[k])) return GS_ERR_INVALID_ARG;
-    if (cam->flags & ~GS_FLAG_TIGHT_TILES) return GS_ERR_INVALID_ARG;
+    if (cam->flags & ~GS_FLAGS_ALL) return GS_ERR_INVALID_ARG;
     CamConst c{};
     for (int i = 0; i < 3; i++) {
         for (int j = 0; j < 3; j++) c.R[3 * i + j] = cam->viewmat[4 * i + j];
@@ -51,6 +51,11 @@ int make_cam(const gs_camera *cam, CamConst *out) {
     c.tiles_x = (cam->width + kTile - 1) / kTile;
     c.tiles_y = (cam->height + kTile - 1) / kTile;
     c.flags = cam->flags;
+    // [GSP] s5/s6: alpha cap 0.99 (3DGS) or 0.999 (older gsplat); the stop
+    // test next_T < 1e-4 (3DGS) or <= 1e-4 (gsplat), the latter as
+    // next_T < the float after 1e-4.
+    c.alpha_cap = (cam->flags & GS_FLAG_CAP_0999) ? 0.999f : 0.99f;
+    c.t_stop = (cam->flags & GS_FLAG_STOP_INCLUSIVE) ? std::nextafter(1e-4f, 1.f) : 1e-4f;
     *out = c;
     return GS_OK;
 }

@@ -31,6 +31,8 @@ struct CamConst {
     float bg[3];
     int32_t width, height, tiles_x, tiles_y;
     uint32_t flags;     // GS_FLAG_* of the camera
+    float alpha_cap;    // 0.99, or 0.999 with GS_FLAG_CAP_0999
+    float t_stop;       // a pixel stops once T (1 - alpha) < t_stop
 };
 
 // Byte layout of a gs_bins buffer.  The first `zero_bytes` bytes are cleared

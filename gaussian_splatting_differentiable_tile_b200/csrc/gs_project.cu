@@ -16,6 +16,7 @@ constexpr float kEps2d = 0.3f;        // [GSP] s4 low-pass dilation, px^2
 constexpr float kDetMin = 1e-10f;     // [GSP] s3 det clamp
 constexpr float kLambdaFloor = 0.1f;  // [GSP] s4 floor under the root
 constexpr float kRadiusSigmas = 3.f;  // [GSP] s4 3DGS radius rule
+constexpr float kGsplatSigmas = 3.33f;  // [GSP] s4 gsplat per-axis radii
 // Opacity-aware tile cut: slack in ln(alpha) (cut tiles stay below
 // e^-0.01 / 255) and the largest conic condition A C / (A C - B^2) it is
 // taken at (beyond it single-precision sigma near the threshold can stray
@@ -37,7 +38,10 @@ struct Proj {
     bool det_clamped, clamped_x, clamped_y;
     float A, B, C;       // conic
     float mx, my;
-    float opacity;
+    float opacity;       // the opacity the blend uses (compensated in antialiased mode)
+    float opacity_raw;   // sigmoid(logit)
+    float det_orig;      // det of the undilated 2D covariance
+    float comp;          // antialiasing compensation, 1 without the flag
     float lambda;
     bool valid;
 };
@@ -61,6 +65,8 @@ __device__ __forceinline__ void project_one(const CamConst &cam, const float *mu
     P.R[8] = 1.f - 2.f * (x * x + y * y);
     P.s[0] = expf(ls[0]); P.s[1] = expf(ls[1]); P.s[2] = expf(ls[2]);
     P.opacity = 1.f / (1.f + expf(-logit));
+    P.opacity_raw = P.opacity;
+    P.comp = 1.f;
 
     // [GSP] s2: M = R diag(s); Sigma = M M^T.  Then [GSP] s3: the camera
     // sees V = W M, and Sigma_c = V V^T = W Sigma W^T.
@@ -108,9 +114,12 @@ __device__ __forceinline__ void project_one(const CamConst &cam, const float *mu
     const float r0z = P.J[0] * P.Sc[2] + P.J[1] * P.Sc[5];
     const float r1y = P.J[2] * P.Sc[3] + P.J[3] * P.Sc[4];
     const float r1z = P.J[2] * P.Sc[4] + P.J[3] * P.Sc[5];
-    P.a = r0x * P.J[0] + r0z * P.J[1] + kEps2d;  // [GSP] s4 dilation
+    const float a0 = r0x * P.J[0] + r0z * P.J[1];  // undilated
+    const float c0 = r1y * P.J[2] + r1z * P.J[3];
+    P.a = a0 + kEps2d;  // [GSP] s4 dilation
     P.b = r0y * P.J[2] + r0z * P.J[3];
-    P.c = r1y * P.J[2] + r1z * P.J[3] + kEps2d;
+    P.c = c0 + kEps2d;
+    P.det_orig = a0 * c0 - P.b * P.b;
     float det = P.a * P.c - P.b * P.b;
     P.det_clamped = det < kDetMin;
     det = fmaxf(det, kDetMin);
@@ -118,6 +127,11 @@ __device__ __forceinline__ void project_one(const CamConst &cam, const float *mu
     P.A = P.c / det;
     P.B = -P.b / det;
     P.C = P.a / det;
+    if (cam.flags & GS_FLAG_ANTIALIASED) {
+        // [GSP] s4, antialiased mode: opacity x sqrt(det S' / det S'')
+        P.comp = P.det_orig > 0.f ? sqrtf(P.det_orig / det) : 0.f;
+        P.opacity = P.opacity_raw * P.comp;
+    }
     const float mid = 0.5f * (P.a + P.c);
     P.lambda = mid + sqrtf(fmaxf(mid * mid - det, kLambdaFloor));
     P.mx = cam.fx * tx * inv_z + cam.cx;
@@ -151,15 +165,34 @@ k_project(CamConst cam, int n, const float *__restrict__ means, const float *__r
         count[g] = 0;
         return;
     }
-    const float r = ceilf(kRadiusSigmas * sqrtf(P.lambda));
+    // radii: 3DGS ceil(3 sqrt(lambda_max)); gsplat per axis ceil(e sqrt(S''_ii)),
+    // e = 3.33 or min(3.33, sqrt(2 ln(255 o))) ([GSP] s4)
+    float rx = ceilf(kRadiusSigmas * sqrtf(P.lambda)), ry = rx;
+    bool none = false;
+    if (cam.flags & GS_FLAG_RADII_AXIS) {
+        float e = kGsplatSigmas;
+        if (cam.flags & GS_FLAG_RADII_OPACITY) {
+            const float l = logf(255.f * P.opacity);
+            none = !(l > 0.f);
+            e = none ? 0.f : fminf(e, sqrtf(2.f * l));
+        }
+        rx = ceilf(e * sqrtf(P.a));
+        ry = ceilf(e * sqrtf(P.c));
+    }
+    const float r = fmaxf(rx, ry);
     xyod[g] = make_float4(P.mx, P.my, P.opacity, P.t[2]);
     conr[g] = make_float4(P.A, P.B, P.C, r);
+    if (none) {  // fades below 1/255 everywhere: no tiles
+        rect[g] = make_int4(0, 0, -1, -1);
+        count[g] = 0;
+        return;
+    }
     // Tile rectangle: floor((m -+ r) / 16) per axis, optionally narrowed by
     // the opacity-aware cut, clamped to the grid in float before any integer
     // conversion.
     const float inv_tile = 1.f / kTile;
-    float lx = floorf((P.mx - r) * inv_tile), hx = floorf((P.mx + r) * inv_tile);
-    float ly = floorf((P.my - r) * inv_tile), hy = floorf((P.my + r) * inv_tile);
+    float lx = floorf((P.mx - rx) * inv_tile), hx = floorf((P.mx + rx) * inv_tile);
+    float ly = floorf((P.my - ry) * inv_tile), hy = floorf((P.my + ry) * inv_tile);
     if (cam.flags & GS_FLAG_TIGHT_TILES) {
         // Opacity-aware cut ([GSP] s4, gsplat's sqrt(2 ln(255 o)) extent),
         // per pixel-centre column and row.  On the column at horizontal
@@ -258,15 +291,25 @@ k_project_bwd(CamConst cam, int n, const float *__restrict__ means,
     d_colors[3 * g] = g1.z;
     d_colors[3 * g + 1] = g1.w;
     d_colors[3 * g + 2] = g2.x;
-    d_logits[g] = d_o * P.opacity * (1.f - P.opacity);
+    // opacity = sigmoid(logit) x comp
+    d_logits[g] = d_o * P.comp * P.opacity_raw * (1.f - P.opacity_raw);
 
     // conic = (c, -b, a) / det; no gradient through a clamped det
     const float inv_det = 1.f / P.det;
     float dl_ddet = 0.f;
     if (!P.det_clamped) dl_ddet = -(d_A * P.c - d_B * P.b + d_C * P.a) * inv_det * inv_det;
-    const float d_a = d_C * inv_det + dl_ddet * P.c;
-    const float d_b = -d_B * inv_det - 2.f * dl_ddet * P.b;
-    const float d_c = d_A * inv_det + dl_ddet * P.a;
+    float d_a = d_C * inv_det + dl_ddet * P.c;
+    float d_b = -d_B * inv_det - 2.f * dl_ddet * P.b;
+    float d_c = d_A * inv_det + dl_ddet * P.a;
+    if ((cam.flags & GS_FLAG_ANTIALIASED) && P.det_orig > 0.f) {
+        // comp = sqrt(D1 / D2), D1 = (a - e)(c - e) - b^2, D2 = a c - b^2:
+        // d comp = comp / 2 (dD1 / D1 - dD2 / D2)
+        const float h = 0.5f * P.comp * d_o * P.opacity_raw, i1 = 1.f / P.det_orig;
+        const float i2 = P.det_clamped ? 0.f : inv_det;
+        d_a += h * ((P.c - kEps2d) * i1 - P.c * i2);
+        d_c += h * ((P.a - kEps2d) * i1 - P.a * i2);
+        d_b += h * 2.f * P.b * (i2 - i1);
+    }
     // Sigma' (undilated) has the same gradient.  Sigma' = J Sc J^T:
     //   dL/dSc = J^T Gp J,  dL/dJ = 2 Gp J Sc,  Gp = [[d_a, d_b/2], [d_b/2, d_c]]
     const float hb = 0.5f * d_b;

@@ -4,7 +4,8 @@
 //
 // Source: "Gaussian splatting in PyTorch" s5 (the per-pixel loop:
 // sigma = 1/2 (A dx^2 + C dy^2) + B dx dy, alpha = min(0.99, o exp(-sigma)),
-// skip sigma < 0 or alpha < 1/255, stop once T (1 - alpha) < 1e-4,
+// skip sigma < 0 or alpha < 1/255, stop once T (1 - alpha) < 1e-4 -- the
+// cap 0.999 and the stop test <= 1e-4 of gsplat as camera flags,
 // C += c alpha T; pixel centres at +0.5; background weighted by the final T),
 // s6 (the CUDA backward recovers T_i by dividing by 1 - alpha back to front;
 // no gradient through the 0.99 cap) and s8 (16 x 16 tiles, each pixel walks
@@ -48,8 +49,6 @@ namespace gs {
 namespace {
 
 constexpr float kLog2e = 1.4426950408889634f;
-constexpr float kAlphaCap = 0.99f;
-constexpr float kTMin = 1e-4f;
 // log2(1/255) minus a margin of 0.0145 (1 % in alpha).
 constexpr float kCullLog2 = -7.994353436858858f - 0.0145f;
 // log2(1/255) in single precision: the alpha >= 1/255 test is taken on the
@@ -164,8 +163,9 @@ __device__ __forceinline__ ColTerms col_terms(const float4 geo, float fx) {
 // Alpha at one pixel.  q = -sigma log2(e) = cA dx^2 + dy (cB dx + cC dy);
 // the entry is skipped there when sigma < 0 (q > 0) or alpha < 1/255
 // (log2 o + q below log2(1/255)), both decided before the exponential.
-// Returns false when skipped.  dy = mean y - pixel y.
-__device__ __forceinline__ bool eval_alpha(const float4 geo, const float4 geo2, const ColTerms &c,
+// Returns false when skipped; else alpha = min(cap, o exp(-sigma)) and
+// whether the cap applied.  dy = mean y - pixel y.
+__device__ __forceinline__ bool eval_alpha(const float4 geo, const float4 geo2, const ColTerms &c, float cap,
                                            float fy, float &dy, float &alpha, bool &capped) {
     dy = __fsub_rn(geo.y, fy);
     const float u = __fmaf_rn(geo2.x, dy, c.bdx);
@@ -173,8 +173,8 @@ __device__ __forceinline__ bool eval_alpha(const float4 geo, const float4 geo2, 
     const float p = __fadd_rn(q, geo2.y);              // log2(o exp(-sigma))
     if (q > 0.f || p < kLog2AlphaMin) return false;
     const float a = ex2_approx(p);
-    capped = a > kAlphaCap;
-    alpha = fminf(a, kAlphaCap);
+    capped = a > cap;
+    alpha = fminf(a, cap);
     return true;
 }
 
@@ -227,9 +227,9 @@ k_render_fwd(CamConst cam, const float4 *__restrict__ xyod, const float4 *__rest
                 const ColTerms ct = col_terms(geo, L.fx);
                 float dy, a;
                 bool capped;
-                if (!eval_alpha(geo, geo2, ct, L.fy0, dy, a, capped)) continue;
+                if (!eval_alpha(geo, geo2, ct, cam.alpha_cap, L.fy0, dy, a, capped)) continue;
                 const float nT = __fmaf_rn(-T, a, T);
-                if (nT < kTMin) {
+                if (nT < cam.t_stop) {
                     done = true;
                     break;
                 }
@@ -434,8 +434,8 @@ k_render_bwd(CamConst cam, const float4 *__restrict__ xyod, const float4 *__rest
             for (int i = 0; i < kPairs; i++) {
                 const bool h0 = hit[2 * i], h1 = hit[2 * i + 1];
                 const float e0 = ex2_approx(p[i].x), e1 = ex2_approx(p[i].y);
-                const float2 a = make_float2(h0 ? fminf(e0, kAlphaCap) : 0.f, h1 ? fminf(e1, kAlphaCap) : 0.f);
-                const bool cap0 = h0 && e0 > kAlphaCap, cap1 = h1 && e1 > kAlphaCap;
+                const float2 a = make_float2(h0 ? fminf(e0, cam.alpha_cap) : 0.f, h1 ? fminf(e1, cam.alpha_cap) : 0.f);
+                const bool cap0 = h0 && e0 > cam.alpha_cap, cap1 = h1 && e1 > cam.alpha_cap;
                 const float2 om = __fadd2_rn(make_float2(1.f, 1.f), make_float2(-a.x, -a.y));
                 const float2 ri = make_float2(rcp_approx(om.x), rcp_approx(om.y));
                 const float2 Ti = __fmul2_rn(T[i], ri);
@@ -510,9 +510,9 @@ k_render_stats(CamConst cam, const float4 *__restrict__ xyod, const float4 *__re
                 visits++;
                 const float4 geo = s_geo[k], geo2 = s_geo2[k];
                 const ColTerms ct = col_terms(geo, fx);
-                if (!eval_alpha(geo, geo2, ct, fy, dy, a, capped)) continue;
+                if (!eval_alpha(geo, geo2, ct, cam.alpha_cap, fy, dy, a, capped)) continue;
                 const float nT = __fmaf_rn(-T, a, T);
-                if (nT < kTMin) { done = true; break; }
+                if (nT < cam.t_stop) { done = true; break; }
                 adds++;
                 T = nT;
             }

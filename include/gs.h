@@ -94,6 +94,28 @@ typedef struct gs_camera {
  * tile's list) refers to the shorter lists. */
 #define GS_FLAG_TIGHT_TILES 1u
 
+/* gs_camera.flags: variants of the method the pages describe ([GSP] s4-s6).
+ * GS_FLAG_ANTIALIASED: gs_project multiplies the opacity by
+ *   sqrt(det S' / det S'') (0 when det S' <= 0), S' the 2D covariance before
+ *   and S'' after the 0.3 dilation; gs_render_bwd differentiates through it.
+ * GS_FLAG_STOP_INCLUSIVE: a pixel stops once T (1 - alpha) <= 1e-4 (gsplat)
+ *   instead of < 1e-4 (3DGS).
+ * GS_FLAG_CAP_0999: alpha = min(0.999, o G) (older gsplat) instead of 0.99.
+ * GS_FLAG_RADII_AXIS: the tile rectangle uses gsplat's per-axis radii
+ *   ceil(3.33 sqrt(S''_xx)), ceil(3.33 sqrt(S''_yy)) instead of 3DGS's
+ *   ceil(3 sqrt(lambda_max)); the record's radius is the larger one.
+ * GS_FLAG_RADII_OPACITY (with GS_FLAG_RADII_AXIS): the extent is
+ *   min(3.33, sqrt(2 ln(255 o))) standard deviations (o the opacity the
+ *   blend uses); a Gaussian with 255 o <= 1 touches no tile.
+ * The render calls take the flags of the camera they are given, which must
+ * be the camera the records were projected with. */
+#define GS_FLAG_ANTIALIASED 2u
+#define GS_FLAG_STOP_INCLUSIVE 4u
+#define GS_FLAG_CAP_0999 8u
+#define GS_FLAG_RADII_AXIS 16u
+#define GS_FLAG_RADII_OPACITY 32u
+#define GS_FLAGS_ALL 63u
+
 /* Raw (unconstrained) parameters of N Gaussians ([GSP] s1), fp32, C-contiguous. */
 typedef struct gs_params {
     const float *means;          /* [N][3] world-space centres */

@@ -40,7 +40,11 @@ SCENES = {
 
 
 # ------------------------------------------------------------------ project
-@pytest.mark.parametrize("flags", [0, G.GS_FLAG_TIGHT_TILES])
+VARIANTS = (G.GS_FLAG_ANTIALIASED | G.GS_FLAG_RADII_AXIS | G.GS_FLAG_RADII_OPACITY | G.GS_FLAG_CAP_0999 |
+            G.GS_FLAG_STOP_INCLUSIVE)
+
+
+@pytest.mark.parametrize("flags", [0, G.GS_FLAG_TIGHT_TILES, VARIANTS, VARIANTS | G.GS_FLAG_TIGHT_TILES])
 @pytest.mark.parametrize("scene", list(SCENES))
 def test_project_matches_oracle(scene, flags):
     cam, params = SCENES[scene]()
@@ -70,7 +74,7 @@ def test_project_matches_oracle(scene, flags):
     diff_rect = np.any(rect != p["rect"], axis=1) | (count != p["count"])
     assert not np.any(diff_r & ~amb), np.nonzero(diff_r & ~amb)[0][:10]
     assert not np.any(diff_rect & ~amb), np.nonzero(diff_rect & ~amb)[0][:10]
-    assert amb.sum() <= max(4, 2e-3 * n)
+    assert amb.sum() <= max(10, 1e-2 * n)
 
 
 # ---------------------------------------------------- bin and sort (stage-fed)
@@ -325,6 +329,22 @@ def test_tight_tiles_stage_fed(scene):
         grad_compare(grads[k], raw_ref[k], bound[k], k)
 
 
+@pytest.mark.parametrize("flags", [G.GS_FLAG_CAP_0999 | G.GS_FLAG_STOP_INCLUSIVE, VARIANTS])
+def test_variants_stage_fed(flags):
+    """The pages' variants (antialiased compensation, gsplat radii, inclusive
+    stop test, 0.999 cap): forward and backward on the oracle's records."""
+    cam, params = SCENES["student3k"]()
+    cam.flags = flags
+    rec, proj, bins, K, image, T, last, ref = _fwd_stage_fed(cam, params)
+    _assert_fwd(cam, bins, image, T, last, ref, np.ones((cam.height, cam.width), bool))
+    rec, g2, grads, g2_ref, g2_abs, params = _bwd_stage_fed(cam, params)
+    grad_compare(g2[:, :9], g2_ref, g2_abs, "grad2d")
+    raw_ref = O.project_bwd(params, cam, g2_ref)
+    bound = O.grad_bound(params, cam, g2_abs)
+    for k in G.PARAM_KEYS:
+        grad_compare(grads[k], raw_ref[k], bound[k], k)
+
+
 def test_tight_tiles_leave_image_and_gradients_unchanged():
     """The 30k student at 980 x 545 through the CUDA path with and without
     the cut: the same entries pass the alpha test in the same order, so the
@@ -366,7 +386,7 @@ def _without_ambiguous(params, cam):
     return out, int(bad.sum())
 
 
-@pytest.mark.parametrize("flags", [0, G.GS_FLAG_TIGHT_TILES])
+@pytest.mark.parametrize("flags", [0, G.GS_FLAG_TIGHT_TILES, VARIANTS])
 def test_end_to_end_from_raw_parameters(flags):
     """Raw parameters through all four calls vs the oracle from the same raw
     parameters in double precision, L1 loss against a seeded target."""
