@@ -183,10 +183,16 @@ def cpu_frame_time(params_np, cam, sample_tiles: int, seed: int = 0) -> dict:
             "threads": O.default_threads()}
 
 
+# gs_camera.flags bits of the pages' variants (GS_FLAG_* in include/gs.h)
+VARIANT_FLAGS = {"3dgs": 0,
+                 "gsplat": 4 | 16 | 32,           # inclusive stop test, per-axis opacity-aware radii
+                 "gsplat-antialiased": 2 | 4 | 16 | 32}
+
+
 def _cameras(spec, args):
     cams = make_cameras(spec)
     for c in cams:
-        c.flags = TIGHT_TILES if args.tiles == "cut" else 0
+        c.flags = (TIGHT_TILES if args.tiles == "cut" else 0) | VARIANT_FLAGS[args.variant]
     return cams
 
 
@@ -209,15 +215,16 @@ def run_reference(args, spec, rank, world):
     out = {"impl": "reference", "metric": METRIC, "value": fps, "unit": "frames/s", "n_gpus": world,
            "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1000.0 * statistics.mean(times),
            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
-           "data": "synthetic", "config": _config(spec, None, args.tiles, False),
+           "data": "synthetic", "config": _config(spec, None, args.tiles, False, args.variant),
            "cpu_baseline": {"value": fps, "unit": "frames/s", "cores": info["threads"], "kind": "oracle",
                             "sample": sample},
            "e2e": {"value": fps, "unit": "frames/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
     print(json.dumps(out), flush=True)
 
 
-def _config(spec, pairs, tiles, graphs=True):
+def _config(spec, pairs, tiles, graphs=True, variant="3dgs"):
     return {"workload": spec.name, "n_gaussians": spec.n, "width": spec.width, "height": spec.height,
+            "variant": variant,
             "focal": spec.focal, "cameras": f"{spec.n_cameras} {spec.cameras}", "pairs_per_frame": pairs,
             "tiles": ("3-sigma rectangle narrowed by the opacity-aware cut (same image)" if tiles == "cut"
                       else "3-sigma rectangle"),
@@ -461,7 +468,7 @@ def run_native(args, spec, rank, world, local):
         "vs_baseline": None,
         "dtype": "f32",
         "data": "synthetic",
-        "config": _config(spec, int(mean_pairs), args.tiles, not args.no_graphs),
+        "config": _config(spec, int(mean_pairs), args.tiles, not args.no_graphs, args.variant),
         "fwd_frames_per_s": frames / (fwd_ms * 1e-3),
         "fwd_ms_per_frame": fwd_ms / args.steps,
         "tile_pairs_per_s": mean_pairs * frames / (fwd_ms * 1e-3),
@@ -490,6 +497,8 @@ def main():
     ap.add_argument("--no-graphs", action="store_true", help="launch every kernel eagerly")
     ap.add_argument("--tiles", choices=("cut", "3sigma"), default="cut",
                     help="tile rectangles: 3-sigma narrowed by the opacity-aware cut, or plain 3-sigma")
+    ap.add_argument("--variant", choices=sorted(VARIANT_FLAGS), default="3dgs",
+                    help="the method's conventions: 3DGS (default), gsplat, or gsplat with antialiasing")
     ap.add_argument("--profile-frame", action="store_true",
                     help="run one eager frame of one camera and exit (for ncu); prints no bench line")
     ap.add_argument("--profile-camera", type=int, default=0)
