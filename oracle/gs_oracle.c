@@ -78,7 +78,12 @@ typedef struct {
                                    /* ceil(3.33 sqrt(S''_yy)) per axis                */
 #define ORC_FLAG_RADII_OPACITY 32  /* with RADII_AXIS: min(3.33, sqrt(2 ln(255 o)))   */
                                    /* standard deviations; 255 o <= 1 touches nothing */
+#define ORC_FLAG_DEPTH         64  /* [GSP] s5: a fourth channel, camera z, blended */
+                                   /* with the colours' weights ("C channels of any */
+                                   /* kind cost the same"); no background term      */
 #define ORC_GSPLAT_SIGMAS 3.33
+#define ORC_MAX_CH 4
+static int orc_channels(const orc_camera *cam) { return (cam->flags & ORC_FLAG_DEPTH) ? 4 : 3; }
 #define ORC_ALPHA_CAP_0999_F 0.999f
 
 /* Single-precision decision constants, as the [GSP] s5 listing writes them. */
@@ -429,7 +434,9 @@ int orc_project(int64_t n, const double *means, const double *log_scales, const 
     for (int64_t g = 0; g < n; g++) {
         orc_proj P;
         project_one(means + 3 * g, log_scales + 3 * g, quats + 4 * g, opacity_logits[g], cam, &P);
-        for (int k = 0; k < 3; k++) color[3 * g + k] = colors[3 * g + k];
+        const int nc = orc_channels(cam);
+        for (int k = 0; k < 3; k++) color[nc * g + k] = colors[3 * g + k];
+        if (nc == 4) color[4 * g + 3] = P.t[2];  /* the depth channel: camera z */
         depth[g] = P.t[2];
         opacity[g] = P.opacity;
         /* the colour is a projected value too: not finite -> culled ([GSP] s6) */
@@ -672,14 +679,15 @@ static double rel_margin(double v, double thr) { return fabs(v - thr) / thr; }
 /* Walks one pixel.  If hits != NULL, records every added entry (growing the
  * buffer as needed).  Returns the number of added entries. */
 static int64_t walk_pixel(const orc_render_ctx *c, int32_t i, int32_t j, orc_hit **hits,
-                          int64_t *cap, double rgb[3], double *T_out, int32_t *n_walk,
+                          int64_t *cap, double rgb[ORC_MAX_CH], double *T_out, int32_t *n_walk,
                           int64_t *e_visit, int64_t *e_contrib, double *m_alpha, double *m_T,
                           double *m_clamp)
 {
     const double x = j + 0.5, y = i + 0.5;
     const int32_t tx = j / ORC_TILE, ty = i / ORC_TILE;
     double T = 1.0;
-    rgb[0] = rgb[1] = rgb[2] = 0.0;
+    const int nc = orc_channels(c->cam);
+    for (int ch = 0; ch < ORC_MAX_CH; ch++) rgb[ch] = 0.0;
     int32_t pos = 0, last_pos = 0;
     int64_t visits = 0, nh = 0;
     double ma_min = INFINITY, mt_min = INFINITY, mc = INFINITY;
@@ -711,7 +719,7 @@ static int64_t walk_pixel(const orc_render_ctx *c, int32_t i, int32_t j, orc_hit
         if ((c->cam->flags & ORC_FLAG_STOP_INCLUSIVE) ? (float)next_T <= ORC_T_MIN_F
                                                       : (float)next_T < ORC_T_MIN_F)
             break;
-        for (int ch = 0; ch < 3; ch++) rgb[ch] += c->color[3 * g + ch] * alpha * T;
+        for (int ch = 0; ch < nc; ch++) rgb[ch] += c->color[nc * g + ch] * alpha * T;
         if (hits) {
             if (nh == *cap) {
                 *cap = *cap ? 2 * *cap : 64;
@@ -750,10 +758,12 @@ static void *render_worker(void *arg)
         for (int32_t j = 0; j < cam->width; j++) {
             if (!pixel_selected(c, i, j)) continue;
             int64_t p = (int64_t)i * cam->width + j;
-            double rgb[3], T;
+            double rgb[ORC_MAX_CH], T;
             walk_pixel(c, i, j, NULL, NULL, rgb, &T, &c->n_walk[p], &c->e_visit[p],
                        &c->e_contrib[p], &c->margin_alpha[p], &c->margin_T[p], &c->margin_clamp[p]);
-            for (int ch = 0; ch < 3; ch++) c->image[3 * p + ch] = rgb[ch] + T * cam->bg[ch];
+            const int nc = orc_channels(cam);
+            for (int ch = 0; ch < nc; ch++)  /* the depth channel has no background */
+                c->image[nc * p + ch] = rgb[ch] + (ch < 3 ? T * cam->bg[ch] : 0.0);
             c->T_final[p] = T;
         }
     }
@@ -820,42 +830,44 @@ int orc_render(int64_t n, const double *mean2d, const double *conic, const doubl
  *   dsigma/dA = dx^2/2, dsigma/dB = dx dy, dsigma/dC = dy^2/2,
  *   dsigma/dmx = A dx + B dy, dsigma/dmy = B dx + C dy.
  * The pixel's own T_i are those of its forward walk.  Per Gaussian the nine
- * sums (dmx, dmy, dA, dB, dC, dopacity, dr, dg, db) and the sums of their
- * absolute contributions are accumulated. */
+ * sums (dmx, dmy, dA, dB, dC, dopacity, dr, dg, db, and d of the depth
+ * channel when it is on) and the sums of their absolute contributions are
+ * accumulated. */
 static void *backward_worker(void *arg)
 {
     orc_thread_arg *a = (orc_thread_arg *)arg;
     orc_render_ctx *c = a->ctx;
     const orc_camera *cam = c->cam;
-    double *acc = c->grad2d + (size_t)a->tid * (size_t)c->n * 9;
-    double *acc_abs = c->grad2d_abs + (size_t)a->tid * (size_t)c->n * 9;
+    const int nc = orc_channels(cam), ng = 6 + nc;
+    double *acc = c->grad2d + (size_t)a->tid * (size_t)c->n * ng;
+    double *acc_abs = c->grad2d_abs + (size_t)a->tid * (size_t)c->n * ng;
     orc_hit *hits = NULL;
     int64_t cap = 0;
     for (int32_t i = a->tid; i < cam->height; i += c->nthreads) {
         for (int32_t j = 0; j < cam->width; j++) {
             if (!pixel_selected(c, i, j)) continue;
             int64_t p = (int64_t)i * cam->width + j;
-            double rgb[3], T, ma, mt, mc;
+            double rgb[ORC_MAX_CH], T, ma, mt, mc;
             int32_t nw;
             int64_t ev, ec;
             int64_t nh = walk_pixel(c, i, j, &hits, &cap, rgb, &T, &nw, &ev, &ec, &ma, &mt, &mc);
-            const double *gp = c->dL_dimage + 3 * p;
-            double R[3] = {cam->bg[0], cam->bg[1], cam->bg[2]};
+            const double *gp = c->dL_dimage + nc * p;
+            double R[ORC_MAX_CH] = {cam->bg[0], cam->bg[1], cam->bg[2], 0.0};
             for (int64_t h = nh - 1; h >= 0; h--) {
                 const orc_hit *e = &hits[h];
                 int64_t g = e->g;
-                double *d = acc + 9 * g, *da = acc_abs + 9 * g;
-                const double *col = c->color + 3 * g;
+                double *d = acc + ng * g, *da = acc_abs + ng * g;
+                const double *col = c->color + nc * g;
                 double w = e->alpha * e->T;
                 double dl_dalpha = 0.0;
-                for (int ch = 0; ch < 3; ch++) {
+                for (int ch = 0; ch < nc; ch++) {
                     double v = w * gp[ch];
                     d[6 + ch] += v;
                     da[6 + ch] += fabs(v);
                     dl_dalpha += (col[ch] - R[ch]) * gp[ch];
                 }
                 dl_dalpha *= e->T;
-                for (int ch = 0; ch < 3; ch++) R[ch] = e->alpha * col[ch] + (1.0 - e->alpha) * R[ch];
+                for (int ch = 0; ch < nc; ch++) R[ch] = e->alpha * col[ch] + (1.0 - e->alpha) * R[ch];
                 if (e->clamped) continue;
                 double o = c->opacity[g];
                 double dl_dsigma = dl_dalpha * (-o * e->G);
@@ -886,9 +898,10 @@ int orc_render_bwd(int64_t n, const double *mean2d, const double *conic, const d
 {
     if (n < 0 || cam->width <= 0 || cam->height <= 0) return -1;
     int nt = nthreads < 1 ? 1 : (nthreads > 256 ? 256 : nthreads);
+    const int ng = 6 + orc_channels(cam);
     int64_t *order = (int64_t *)malloc(sizeof(int64_t) * (size_t)(n > 0 ? n : 1));
-    double *acc = (double *)calloc((size_t)nt * (size_t)(n > 0 ? n : 1) * 9, sizeof(double));
-    double *acc_abs = (double *)calloc((size_t)nt * (size_t)(n > 0 ? n : 1) * 9, sizeof(double));
+    double *acc = (double *)calloc((size_t)nt * (size_t)(n > 0 ? n : 1) * ng, sizeof(double));
+    double *acc_abs = (double *)calloc((size_t)nt * (size_t)(n > 0 ? n : 1) * ng, sizeof(double));
     if (!order || !acc || !acc_abs) { free(order); free(acc); free(acc_abs); return -2; }
     int64_t m = orc_depth_order(n, depth32, rect, valid, order);
     orc_render_ctx c;
@@ -903,11 +916,11 @@ int orc_render_bwd(int64_t n, const double *mean2d, const double *conic, const d
     c.nthreads = nt;
     int rc = run_threads(&c, backward_worker);
     /* sum the per-thread partials in thread order */
-    for (int64_t k = 0; k < n * 9; k++) {
+    for (int64_t k = 0; k < n * ng; k++) {
         double s = 0.0, sa = 0.0;
         for (int t = 0; t < nt; t++) {
-            s += acc[(size_t)t * (size_t)n * 9 + (size_t)k];
-            sa += acc_abs[(size_t)t * (size_t)n * 9 + (size_t)k];
+            s += acc[(size_t)t * (size_t)n * ng + (size_t)k];
+            sa += acc_abs[(size_t)t * (size_t)n * ng + (size_t)k];
         }
         grad2d[k] = s;
         grad2d_abs[k] = sa;
@@ -948,7 +961,8 @@ int orc_project_bwd(int64_t n, const double *means, const double *log_scales, co
         orc_proj P;
         project_one(means + 3 * g, log_scales + 3 * g, quats + 4 * g, opacity_logits[g], cam, &P);
         if (!P.valid) continue;
-        const double *gg = grad2d + 9 * g;
+        const int ng = 6 + orc_channels(cam);
+        const double *gg = grad2d + ng * g;
         double d_mx = gg[0], d_my = gg[1], d_A = gg[2], d_B = gg[3], d_C = gg[4], d_o = gg[5];
         /* colour passes through */
         for (int k = 0; k < 3; k++) dc[k] = gg[6 + k];
@@ -1014,6 +1028,8 @@ int orc_project_bwd(int64_t n, const double *means, const double *log_scales, co
             double lim = P.jy / tz;
             dt[2] += dJ[5] * (fy * lim / (tz * tz));
         }
+        /* the depth channel's colour is the camera z */
+        if (ng == 10) dt[2] += gg[9];
         /* mean2d = (fx x/z + cx, fy y/z + cy) */
         dt[0] += d_mx * fx / tz;
         dt[1] += d_my * fy / tz;

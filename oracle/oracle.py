@@ -23,7 +23,7 @@ from . import build as _build
 
 __all__ = [
     "TILE", "TIGHT_TILES", "ANTIALIASED", "STOP_INCLUSIVE", "CAP_0999", "RADII_AXIS",
-    "RADII_OPACITY", "OrcCamera", "lib", "quat_to_rotmat", "covariance3d", "project_debug", "project", "tile_rects",
+    "RADII_OPACITY", "DEPTH", "channels", "OrcCamera", "lib", "quat_to_rotmat", "covariance3d", "project_debug", "project", "tile_rects",
     "records_f32", "bin_pairs", "depth_order", "render", "render_bwd", "project_bwd",
     "grad_bound", "default_threads",
 ]
@@ -37,6 +37,12 @@ STOP_INCLUSIVE = 4    # stop once next_T <= 1e-4 (gsplat)
 CAP_0999 = 8          # alpha cap 0.999 (older gsplat)
 RADII_AXIS = 16       # gsplat per-axis 3.33-sigma radii
 RADII_OPACITY = 32    # with RADII_AXIS: min(3.33, sqrt(2 ln(255 o))) sigmas
+DEPTH = 64            # a fourth channel, camera z, blended with the colours' weights
+
+
+def channels(cam) -> int:
+    """Channels of the rendered image: RGB, plus depth with the DEPTH flag."""
+    return 4 if int(getattr(cam, "flags", 0)) & DEPTH else 3
 
 _c_double_p = ctypes.POINTER(ctypes.c_double)
 _c_float_p = ctypes.POINTER(ctypes.c_float)
@@ -169,7 +175,7 @@ def project(params: dict, cam) -> dict:
     colors = _f64(params["colors"]).reshape(n, 3)
     out = {
         "mean2d": np.zeros((n, 2)), "conic": np.zeros((n, 3)), "cov2d": np.zeros((n, 3)),
-        "opacity": np.zeros(n), "depth": np.zeros(n), "color": np.zeros((n, 3)),
+        "opacity": np.zeros(n), "depth": np.zeros(n), "color": np.zeros((n, channels(cam))),
         "radius": np.zeros(n, dtype=np.float32), "radius_xy": np.zeros((n, 2), dtype=np.float32),
         "rect": np.zeros((n, 4), dtype=np.int32),
         "count": np.zeros(n, dtype=np.int32), "valid": np.zeros(n, dtype=np.uint8),
@@ -267,10 +273,10 @@ def depth_order(depth32, rect, valid) -> np.ndarray:
     return order[:m]
 
 
-def _render_inputs(proj: dict):
+def _render_inputs(proj: dict, nc: int = 3):
     n = np.asarray(proj["mean2d"]).reshape(-1, 2).shape[0]
     return (n, _f64(proj["mean2d"]).reshape(n, 2), _f64(proj["conic"]).reshape(n, 3),
-            _f64(proj["opacity"]).reshape(n), _f64(proj["color"]).reshape(n, 3),
+            _f64(proj["opacity"]).reshape(n), _f64(proj["color"]).reshape(n, nc),
             np.ascontiguousarray(proj["depth32"], dtype=np.float32).reshape(n),
             np.ascontiguousarray(proj["rect"], dtype=np.int32).reshape(n, 4),
             np.ascontiguousarray(proj["valid"], dtype=np.uint8).reshape(n))
@@ -286,9 +292,10 @@ def _mask(cam, tile_mask):
 
 def render(proj: dict, cam, tile_mask=None, nthreads: int | None = None) -> dict:
     """[WEEK] naive renderer with the tile-rectangle cutoff; [GSP] s5 loop."""
-    n, m2, con, op, col, d32, rect, valid = _render_inputs(proj)
+    nc = channels(cam)
+    n, m2, con, op, col, d32, rect, valid = _render_inputs(proj, nc)
     H, W = int(cam.height), int(cam.width)
-    out = {"image": np.zeros((H, W, 3)), "T_final": np.zeros((H, W)),
+    out = {"image": np.zeros((H, W, nc)), "T_final": np.zeros((H, W)),
            "n_walk": np.zeros((H, W), dtype=np.int32), "e_visit": np.zeros((H, W), dtype=np.int64),
            "e_contrib": np.zeros((H, W), dtype=np.int64),
            "margin_alpha": np.full((H, W), np.inf), "margin_T": np.full((H, W), np.inf),
@@ -311,12 +318,14 @@ def render(proj: dict, cam, tile_mask=None, nthreads: int | None = None) -> dict
 def render_bwd(proj: dict, cam, dL_dimage, tile_mask=None, nthreads: int | None = None):
     """[GSP] s6 back-to-front analytic backward of the blend.  Returns
     (grad2d, grad2d_abs), each (n, 9): dmean2d x/y, dA, dB, dC, dopacity,
-    dr, dg, db, and the sums of absolute contributions."""
-    n, m2, con, op, col, d32, rect, valid = _render_inputs(proj)
+    dr, dg, db (and a tenth column, the depth channel, with the DEPTH flag),
+    and the sums of absolute contributions."""
+    nc = channels(cam)
+    n, m2, con, op, col, d32, rect, valid = _render_inputs(proj, nc)
     H, W = int(cam.height), int(cam.width)
-    g = _f64(dL_dimage).reshape(H, W, 3)
-    grad2d = np.zeros((n, 9))
-    grad_abs = np.zeros((n, 9))
+    g = _f64(dL_dimage).reshape(H, W, nc)
+    grad2d = np.zeros((n, 6 + nc))
+    grad_abs = np.zeros((n, 6 + nc))
     c = _cam(cam)
     mk, mkp = _mask(cam, tile_mask)
     rc = lib().orc_render_bwd(
@@ -336,7 +345,7 @@ def project_bwd(params: dict, cam, grad2d) -> dict:
     log_scales = _f64(params["log_scales"]).reshape(n, 3)
     quats = _f64(params["quats"]).reshape(n, 4)
     logits = _f64(params["opacity_logits"]).reshape(n)
-    g2 = _f64(grad2d).reshape(n, 9)
+    g2 = _f64(grad2d).reshape(n, 6 + channels(cam))
     out = {"means": np.zeros((n, 3)), "log_scales": np.zeros((n, 3)), "quats": np.zeros((n, 4)),
            "opacity_logits": np.zeros(n), "colors": np.zeros((n, 3))}
     c = _cam(cam)
@@ -355,10 +364,11 @@ def grad_bound(params: dict, cam, grad2d_abs) -> dict:
     gradient element a bound on the magnitude of the terms it sums.  Used for
     the cancellation-aware gradient tolerance."""
     n = np.asarray(params["means"]).reshape(-1, 3).shape[0]
-    ga = _f64(grad2d_abs).reshape(n, 9)
-    total = {k: np.zeros_like(v) for k, v in project_bwd(params, cam, np.zeros((n, 9))).items()}
-    for k in range(9):
-        e = np.zeros((n, 9))
+    ng = 6 + channels(cam)
+    ga = _f64(grad2d_abs).reshape(n, ng)
+    total = {k: np.zeros_like(v) for k, v in project_bwd(params, cam, np.zeros((n, ng))).items()}
+    for k in range(ng):
+        e = np.zeros((n, ng))
         e[:, k] = 1.0
         col = project_bwd(params, cam, e)
         for name, v in col.items():

@@ -65,7 +65,7 @@ def _find_clean(seed0, **kw):
 
 
 def _loss_weights(cam, seed=99):
-    return np.random.default_rng(seed).normal(size=(cam.height, cam.width, 3))
+    return np.random.default_rng(seed).normal(size=(cam.height, cam.width, O.channels(cam)))
 
 
 def _loss_from_records(rec, cam, w):
@@ -76,13 +76,15 @@ def _loss_from_params(params, cam, w):
     return _loss_from_records(O.project(params, cam), cam, w)
 
 
-@pytest.mark.parametrize("bg", [(0.0, 0.0, 0.0), (0.3, 0.2, 0.1)])
-def test_blend_backward_matches_finite_differences(bg):
-    cam, params = _find_clean(100, bg=bg)
+@pytest.mark.parametrize("bg,flags", [((0.0, 0.0, 0.0), 0), ((0.3, 0.2, 0.1), 0), ((0.3, 0.2, 0.1), O.DEPTH)])
+def test_blend_backward_matches_finite_differences(bg, flags):
+    cam, params = _find_clean(100, bg=bg, flags=flags)
     w = _loss_weights(cam)
     rec = O.project(params, cam)
     g2, g2abs = O.render_bwd(rec, cam, w, nthreads=2)
-    fields = [("mean2d", 2, [0, 1]), ("conic", 3, [2, 3, 4]), ("opacity", 1, [5]), ("color", 3, [6, 7, 8])]
+    nc = O.channels(cam)
+    fields = [("mean2d", 2, [0, 1]), ("conic", 3, [2, 3, 4]), ("opacity", 1, [5]),
+              ("color", nc, list(range(6, 6 + nc)))]
     checked = 0
     for g in range(len(rec["opacity"])):
         if rec["count"][g] == 0:
@@ -109,7 +111,8 @@ ALL_VARIANTS = O.ANTIALIASED | O.RADII_AXIS | O.RADII_OPACITY | O.CAP_0999 | O.S
 
 
 @pytest.mark.parametrize("clamp_case,flags", [(False, 0), (True, 0), (False, O.ANTIALIASED),
-                                              (True, ALL_VARIANTS)])
+                                              (True, ALL_VARIANTS), (False, O.DEPTH),
+                                              (True, ALL_VARIANTS | O.DEPTH)])
 def test_raw_parameter_gradients_match_finite_differences(clamp_case, flags):
     """With the antialiased flag the chain also runs through the
     compensation sqrt(det S' / det S'') into S' and the sigmoid."""

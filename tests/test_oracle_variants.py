@@ -108,3 +108,28 @@ def test_gsplat_radii_page_values_and_opacity_extent():
     params["opacity_logits"] = np.array([math.log(0.0035 / (1 - 0.0035))])  # 255 o < 1
     p = O.project(params, cam)
     assert p["count"][0] == 0 and p["radius_xy"][0].tolist() == [0, 0]
+
+
+def test_depth_channel():
+    """s5: "C channels of any kind cost the same": with the depth flag each
+    record carries its camera z as a fourth colour, blended with the same
+    weights and no background (image[..., 3] = sum_i w_i z_i)."""
+    rec = _records([[0.5, 0.5], [0.5, 0.5]], [[1.0, 0.0, 1.0]] * 2, [0.6, 0.5],
+                   [[1.0, 0.0, 0.0], [0.0, 1.0, 0.0]], [2.0, 3.0], [[0, 0, 0, 0]] * 2)
+    rec["color"] = np.array([[1.0, 0.0, 0.0, 2.0], [0.0, 1.0, 0.0, 3.0]])
+    cam = _one_pixel_cam(O.DEPTH)
+    cam.bg = (0.25, 0.25, 0.25)
+    img = O.render(rec, cam, nthreads=1)["image"][0, 0]
+    T1 = 1.0 - 0.6
+    np.testing.assert_allclose(img, [0.6 + T1 * 0.5 * 0 + T1 * 0.5 * 0.25, T1 * 0.5 + T1 * 0.5 * 0.25,
+                                     T1 * 0.5 * 0.25, 0.6 * 2.0 + T1 * 0.5 * 3.0], rtol=1e-12)
+    # the projection fills the fourth colour with the camera z
+    cam2 = _identity_cam(64, 64, 50.0, 50.0, 32.0, 32.0)
+    cam2.flags = O.DEPTH
+    params = {"means": np.array([[0.1, -0.2, 3.0], [0.0, 0.1, 5.0]]), "log_scales": np.full((2, 3), -2.0),
+              "quats": np.tile([1.0, 0, 0, 0], (2, 1)), "opacity_logits": np.zeros(2),
+              "colors": np.array([[0.1, 0.2, 0.3], [0.4, 0.5, 0.6]])}
+    p = O.project(params, cam2)
+    np.testing.assert_array_equal(p["color"][:, :3], params["colors"])
+    np.testing.assert_array_equal(p["color"][:, 3], p["depth"])
+    assert O.render(p, cam2, nthreads=1)["image"].shape == (64, 64, 4)
