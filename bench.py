@@ -87,9 +87,9 @@ ALU_KERNELS = ("render_fwd", "render_bwd")
 # DRAM traffic per launch of render_bwd measured by ncu
 # (dram__bytes_read.sum + dram__bytes_write.sum), valid only for the kernel
 # source it was taken on.
-# Taken on one frame of this workload (camera 0, 644,012 pairs): 42,362,368 B
-# read + 430,336 B written; scaled to a launch by its pair count.
-TRAFFIC = {"render_bwd": {"src_sha": "50f7093f06b735ee", "bytes_per_pair": 66.447}}
+# Taken on one frame of this workload (camera 0, 644,012 pairs): 42,370,048 B
+# read + 213,504 B written; scaled to a launch by its pair count.
+TRAFFIC = {"render_bwd": {"src_sha": "7892df41a2ba539e", "bytes_per_pair": 66.122}}
 
 
 def _peaks():
@@ -169,7 +169,8 @@ def cpu_frame_time(params_np, cam, sample_tiles: int, seed: int = 0) -> dict:
     t0 = time.perf_counter()
     O.render(p, cam, tile_mask=mask)
     t["render_sample"] = time.perf_counter() - t0
-    dl = np.random.default_rng(seed + 1).normal(size=(cam.height, cam.width, 3)) / (3 * cam.pixels)
+    nc = O.channels(cam)
+    dl = np.random.default_rng(seed + 1).normal(size=(cam.height, cam.width, nc)) / (nc * cam.pixels)
     t0 = time.perf_counter()
     g2, _ = O.render_bwd(p, cam, dl, tile_mask=mask)
     t["render_bwd_sample"] = time.perf_counter() - t0
@@ -186,7 +187,8 @@ def cpu_frame_time(params_np, cam, sample_tiles: int, seed: int = 0) -> dict:
 # gs_camera.flags bits of the pages' variants (GS_FLAG_* in include/gs.h)
 VARIANT_FLAGS = {"3dgs": 0,
                  "gsplat": 4 | 16 | 32,           # inclusive stop test, per-axis opacity-aware radii
-                 "gsplat-antialiased": 2 | 4 | 16 | 32}
+                 "gsplat-antialiased": 2 | 4 | 16 | 32,
+                 "3dgs-depth": 64}                # a fourth channel: blended camera depth
 
 
 def _cameras(spec, args):
@@ -265,7 +267,7 @@ def run_profile_frame(args, spec):
     cam = _cameras(spec, args)[args.profile_camera]
     r = G.Rasterizer(spec.n, spec.width, spec.height, max_pairs=24 * spec.n)
     image = r.forward(cam, params, sync=True)
-    target = torch.from_numpy(make_target(spec.width, spec.height)).cuda()
+    target = torch.from_numpy(make_target(spec.width, spec.height, channels=G.channels(cam))).cuda()
     dl = torch.empty_like(image)
     loss = torch.zeros(1, device="cuda")
     G.gs_l1_loss_grad(image, target, dl, loss)
@@ -288,7 +290,9 @@ def run_native(args, spec, rank, world, local):
     mine = my_cameras(cams, rank, world)
     n = spec.n
     P = {k: torch.from_numpy(v).to(dev) for k, v in params_np.items()}
-    targets = [torch.from_numpy(make_target(spec.width, spec.height, seed=i)).to(dev) for i in range(len(mine))]
+    nc = G.channels(cams[0])
+    targets = [torch.from_numpy(make_target(spec.width, spec.height, seed=i, channels=nc)).to(dev)
+               for i in range(len(mine))]
     ccams = [G.make_camera(c) for c in mine]
 
     # size the pair list from the cameras this rank renders
@@ -301,7 +305,7 @@ def run_native(args, spec, rank, world, local):
     bins = G.Bins(n, int(max(pairs) * 1.05) + 4096, spec.width, spec.height, device=dev)
     proj = r.proj
     H, W = spec.height, spec.width
-    image = torch.empty((H, W, 3), device=dev)
+    image = torch.empty((H, W, nc), device=dev)
     T = torch.empty((H, W), device=dev)
     last = torch.empty((H, W), dtype=torch.int32, device=dev)
     dl = torch.empty_like(image)
@@ -561,7 +565,7 @@ def main():
     ap.add_argument("--tiles", choices=("cut", "3sigma"), default="cut",
                     help="tile rectangles: 3-sigma narrowed by the opacity-aware cut, or plain 3-sigma")
     ap.add_argument("--variant", choices=sorted(VARIANT_FLAGS), default="3dgs",
-                    help="the method's conventions: 3DGS (default), gsplat, or gsplat with antialiasing")
+                    help="the method's conventions: 3DGS (default), gsplat, gsplat with antialiasing, or 3DGS with a depth channel")
     ap.add_argument("--profile-frame", action="store_true",
                     help="run one eager frame of one camera and exit (for ncu); prints no bench line")
     ap.add_argument("--profile-camera", type=int, default=0)

@@ -25,12 +25,12 @@ import torch
 
 from . import _abi
 from ._abi import (GS_ERR_ALIGNMENT, GS_ERR_CAPACITY, GS_ERR_CUDA, GS_ERR_DEVICE_TIMEOUT,  # noqa: F401
-                   GS_ERR_INVALID_ARG, GS_ERR_TOO_LARGE, GS_FLAG_ANTIALIASED, GS_FLAG_CAP_0999,
+                   GS_ERR_INVALID_ARG, GS_ERR_TOO_LARGE, GS_FLAG_ANTIALIASED, GS_FLAG_CAP_0999, GS_FLAG_DEPTH,
                    GS_FLAG_RADII_AXIS, GS_FLAG_RADII_OPACITY, GS_FLAG_STOP_INCLUSIVE, GS_FLAG_TIGHT_TILES, GS_OK,
                    GS_TILE)
 
 __all__ = [
-    "GSError", "Projected", "Bins", "make_camera", "gs_project", "gs_bin_and_sort",
+    "GSError", "Projected", "Bins", "make_camera", "channels", "gs_project", "gs_bin_and_sort",
     "gs_bin_and_sort_static", "gs_render_fwd",
     "gs_render_bwd", "gs_render_stats", "gs_l1_loss_grad", "gs_read_status", "gs_error_string", "profile_begin",
     "profile_end", "lib", "PARAM_KEYS",
@@ -74,6 +74,11 @@ def _dev(t: torch.Tensor | None, name: str, dtype=None) -> ctypes.c_void_p:
 def _stream(stream) -> ctypes.c_void_p:
     s = torch.cuda.current_stream() if stream is None else stream
     return ctypes.c_void_p(s.cuda_stream)
+
+
+def channels(cam) -> int:
+    """Image channels for a camera: RGB, plus depth with GS_FLAG_DEPTH."""
+    return 4 if int(getattr(cam, "flags", 0)) & GS_FLAG_DEPTH else 3
 
 
 def make_camera(cam) -> _abi.GsCamera:
@@ -196,8 +201,9 @@ def gs_bin_and_sort_static(cam, n: int, proj: Projected, pair_tile: torch.Tensor
 def gs_render_fwd(cam, n: int, proj: Projected, bins: Bins, image: torch.Tensor, T_final: torch.Tensor,
                   last: torch.Tensor, stream=None) -> None:
     H, W = int(cam.height), int(cam.width)
-    if image.numel() != H * W * 3 or T_final.numel() != H * W or last.numel() != H * W:
-        raise ValueError("output tensors must be [H,W,3], [H,W], [H,W]")
+    ch = channels(cam)
+    if image.numel() != H * W * ch or T_final.numel() != H * W or last.numel() != H * W:
+        raise ValueError(f"output tensors must be [H,W,{ch}], [H,W], [H,W]")
     c = make_camera(cam)
     _check(lib().gs_render_fwd(ctypes.byref(c), int(n), ctypes.byref(proj.struct), ctypes.byref(bins.struct),
                                _dev(image, "image", torch.float32), _dev(T_final, "T_final", torch.float32),
@@ -209,6 +215,8 @@ def gs_render_bwd(cam, n: int, params: dict, proj: Projected, bins: Bins, T_fina
                   stream=None) -> None:
     if grad2d.numel() < 12 * int(n):
         raise ValueError("grad2d must hold [N,12] floats")
+    if dL_dimage.numel() != int(cam.height) * int(cam.width) * channels(cam):
+        raise ValueError(f"dL_dimage must be [H,W,{channels(cam)}]")
     c = make_camera(cam)
     p = _params_struct(params)
     g = _params_struct(grads, _abi.GsGrads)

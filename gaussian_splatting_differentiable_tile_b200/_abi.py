@@ -26,6 +26,7 @@ GS_FLAG_STOP_INCLUSIVE = 4
 GS_FLAG_CAP_0999 = 8
 GS_FLAG_RADII_AXIS = 16
 GS_FLAG_RADII_OPACITY = 32
+GS_FLAG_DEPTH = 64
 
 c_float_p = ctypes.c_void_p  # device pointers travel as plain addresses
 

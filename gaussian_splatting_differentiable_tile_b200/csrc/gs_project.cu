@@ -155,7 +155,9 @@ k_project(CamConst cam, int n, const float *__restrict__ means, const float *__r
     float q[4] = {q4.x, q4.y, q4.z, q4.w};
     Proj P;
     project_one(cam, mu, ls, q, logits[g], P);
-    const float4 col = make_float4(colors[3 * g], colors[3 * g + 1], colors[3 * g + 2], 0.f);
+    // with GS_FLAG_DEPTH the fourth colour is the camera z ([GSP] s5: any channel blends alike)
+    const float4 col = make_float4(colors[3 * g], colors[3 * g + 1], colors[3 * g + 2],
+                                   (cam.flags & GS_FLAG_DEPTH) ? P.t[2] : 0.f);
     rgb[g] = col;
     // the colour is a projected value too: not finite -> culled ([GSP] s6)
     if (!P.valid || !isfinite(col.x) || !isfinite(col.y) || !isfinite(col.z)) {
@@ -248,7 +250,8 @@ __device__ __forceinline__ void rotmat_vjp(const float *qh, const float *G, floa
 //   dL/dmx = -(A sum v dx + B sum v dy), dL/dmy = -(B sum v dx + C sum v dy),
 //   dL/dA = -sum v dx^2 / 2, dL/dB = -sum v dx dy, dL/dC = -sum v dy^2 / 2.
 // Those values are written back: on return grad2d holds
-// dL/d(mx, my, A, B, C, opacity, r, g, b, 0, 0, 0).
+// dL/d(mx, my, A, B, C, opacity, r, g, b, depth channel, 0, 0) (the depth
+// channel's entry is 0 without GS_FLAG_DEPTH).
 __global__ void __launch_bounds__(256)
 k_project_bwd(CamConst cam, int n, const float *__restrict__ means,
               const float *__restrict__ log_scales, const float *__restrict__ quats,
@@ -272,7 +275,7 @@ k_project_bwd(CamConst cam, int n, const float *__restrict__ means,
     const float4 g0 = make_float4(-(cr.x * s0.y + cr.y * s0.z), -(cr.y * s0.y + cr.z * s0.z),
                                   -0.5f * s0.w, -s1.x);
     const float4 g1 = make_float4(-0.5f * s1.y, op > 0.f ? s0.x / op : 0.f, s1.z, s1.w);
-    const float4 g2 = make_float4(s2.x, 0.f, 0.f, 0.f);
+    const float4 g2 = make_float4(s2.x, s2.y, 0.f, 0.f);  // b, depth channel
     grad2d[3 * g] = g0;
     grad2d[3 * g + 1] = g1;
     grad2d[3 * g + 2] = g2;
@@ -347,6 +350,8 @@ k_project_bwd(CamConst cam, int n, const float *__restrict__ means,
         const float lim = ty * iz < cam.lim_y_lo ? cam.lim_y_lo : cam.lim_y_hi;
         dt2 += dJ12 * cam.fy * lim * iz2;
     }
+    // the depth channel's colour is the camera z
+    if (cam.flags & GS_FLAG_DEPTH) dt2 += g2.y;
     // mean2d = (fx x/z + cx, fy y/z + cy)
     dt0 += d_mx * cam.fx * iz;
     dt1 += d_my * cam.fy * iz;

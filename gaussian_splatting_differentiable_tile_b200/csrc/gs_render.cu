@@ -185,6 +185,7 @@ __device__ __forceinline__ bool eval_alpha(const float4 geo, const float4 geo2, 
 // slots whose bit it holds, in order, and walks only those.  A culled slot
 // could not have passed the alpha test at any pixel of the strip, so the
 // sequence of contributions, the stopping entry and `last` are unchanged.
+template <bool kDepth>
 __global__ void __launch_bounds__(kTilePixels, 6)
 k_render_fwd(CamConst cam, const float4 *__restrict__ xyod, const float4 *__restrict__ conr,
              const float4 *__restrict__ rgb, const uint32_t *__restrict__ pair_gid,
@@ -202,7 +203,7 @@ k_render_fwd(CamConst cam, const float4 *__restrict__ xyod, const float4 *__rest
     const uint2 range = ranges[tile];
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
 
-    float T = 1.f, C0 = 0.f, C1 = 0.f, C2 = 0.f;
+    float T = 1.f, C0 = 0.f, C1 = 0.f, C2 = 0.f, C3 = 0.f;
     uint32_t lst = range.x;
     bool done = !(L.px < cam.width && L.py0 < cam.height);
     for (uint32_t b = range.x; b < range.y; b += kBatch) {
@@ -238,6 +239,7 @@ k_render_fwd(CamConst cam, const float4 *__restrict__ xyod, const float4 *__rest
                 C0 = __fmaf_rn(w, c.x, C0);
                 C1 = __fmaf_rn(w, c.y, C1);
                 C2 = __fmaf_rn(w, c.z, C2);
+                if (kDepth) C3 = __fmaf_rn(w, c.w, C3);
                 T = nT;
                 lst = b + i + 1;
             }
@@ -245,9 +247,11 @@ k_render_fwd(CamConst cam, const float4 *__restrict__ xyod, const float4 *__rest
     }
     if (L.px < cam.width && L.py0 < cam.height) {
         const size_t p = (size_t)L.py0 * cam.width + L.px;
-        image[3 * p] = __fmaf_rn(T, cam.bg[0], C0);
-        image[3 * p + 1] = __fmaf_rn(T, cam.bg[1], C1);
-        image[3 * p + 2] = __fmaf_rn(T, cam.bg[2], C2);
+        constexpr int kC = kDepth ? 4 : 3;
+        image[kC * p] = __fmaf_rn(T, cam.bg[0], C0);
+        image[kC * p + 1] = __fmaf_rn(T, cam.bg[1], C1);
+        image[kC * p + 2] = __fmaf_rn(T, cam.bg[2], C2);
+        if (kDepth) image[kC * p + 3] = C3;  // the depth channel has no background
         T_final[p] = T;
         last[p] = lst;
     }
@@ -259,35 +263,58 @@ __device__ __forceinline__ float warp_sum(float v) {
     return v;
 }
 
-// Warp reduce-scatter of nine values per lane.  Five xor levels (16, 8, 4, 2,
-// 1); at each level a lane keeps one half of its values and sends the other
-// half to its partner, which keeps that half: 46 instructions instead of the
-// 90 of nine full butterflies.  On return every even lane whose *idx is in
-// [0, 9) holds the warp total of value *idx (one lane per value).
-__device__ __forceinline__ float reduce_scatter9(const float (&v)[9], int lane, int *idx) {
-    const bool b4 = lane & 16, b3 = lane & 8, b2 = lane & 4, b1 = lane & 2;
-    float k[5];
-#pragma unroll
-    for (int i = 0; i < 5; i++) {
-        const float lo = v[i], hi = i < 4 ? v[5 + i] : 0.f;
-        k[i] = (b4 ? hi : lo) + __shfl_xor_sync(0xffffffffu, b4 ? lo : hi, 16);
+// Size of the kept half at xor level `level` (0: 16, 1: 8, 2: 4, 3: 2) of a
+// reduce-scatter of n values.
+__host__ __device__ constexpr int rs_half(int n, int level) {
+    for (int i = 0; i < level; i++) n = (n + 1) / 2;
+    return (n + 1) / 2;
+}
+// Even lanes that end a reduce-scatter of n values holding a real value (not
+// the zero padding of an odd half).
+__host__ __device__ constexpr uint32_t rs_valid_lanes(int n) {
+    uint32_t mask = 0;
+    for (int lane = 0; lane < 32; lane += 2) {
+        int real = n;
+        for (int level = 0; level < 4; level++) {
+            const int h = rs_half(n, level);
+            real = (lane & (16 >> level)) ? (real > h ? real - h : 0) : (real < h ? real : h);
+        }
+        if (real > 0) mask |= 1u << lane;
     }
-    float m[3];
+    return mask;
+}
+
+// Warp reduce-scatter of N <= 16 values per lane.  At each xor level (16,
+// 8, 4, 2) a lane keeps one half of its values and sends the other half to
+// its partner, which keeps that half; the last level (1) sums the one value
+// left.  A 9-value reduce takes 46 instructions instead of the 90 of nine
+// full butterflies.  On return every even lane whose *idx is in [0, N)
+// holds the warp total of value *idx (one lane per value).
+template <int N>
+__device__ __forceinline__ float reduce_scatter(const float (&v)[N], int lane, int *idx) {
+    static_assert(N >= 2 && N <= 16, "2 to 16 values");
+    float a[16];
 #pragma unroll
-    for (int i = 0; i < 3; i++) {
-        const float lo = k[i], hi = i < 2 ? k[3 + i] : 0.f;
-        m[i] = (b3 ? hi : lo) + __shfl_xor_sync(0xffffffffu, b3 ? lo : hi, 8);
-    }
-    float n[2];
+    for (int i = 0; i < 16; i++) a[i] = i < N ? v[i] : 0.f;
+    int m = N;  // values left per lane
 #pragma unroll
-    for (int i = 0; i < 2; i++) {
-        const float lo = m[i], hi = i == 0 ? m[2] : 0.f;
-        n[i] = (b2 ? hi : lo) + __shfl_xor_sync(0xffffffffu, b2 ? lo : hi, 4);
+    for (int off = 16; off >= 2; off >>= 1) {
+        const int h = (m + 1) / 2;
+        const bool up = lane & off;
+#pragma unroll
+        for (int i = 0; i < 8; i++) {
+            if (i >= h) break;
+            const float lo = a[i], hi = h + i < m ? a[h + i] : 0.f;
+            a[i] = (up ? hi : lo) + __shfl_xor_sync(0xffffffffu, up ? lo : hi, off);
+        }
+        m = h;
     }
-    float x = (b1 ? n[1] : n[0]) + __shfl_xor_sync(0xffffffffu, b1 ? n[0] : n[1], 2);
-    x += __shfl_xor_sync(0xffffffffu, x, 1);
-    const int q = 2 * (int)b2 + (int)b1, p = 3 * (int)b3 + q;
-    *idx = (q <= 2 && p <= 4 && !(lane & 1)) ? 5 * (int)b4 + p : 9;
+    const float x = a[0] + __shfl_xor_sync(0xffffffffu, a[0], 1);
+    // which value the lane ended with: the halves it kept, level by level
+    constexpr uint32_t kValid = rs_valid_lanes(N);
+    const int base = ((lane & 16) ? rs_half(N, 0) : 0) + ((lane & 8) ? rs_half(N, 1) : 0) +
+                     ((lane & 4) ? rs_half(N, 2) : 0) + ((lane & 2) ? rs_half(N, 3) : 0);
+    *idx = ((kValid >> lane) & 1u) ? base : N;
     return x;
 }
 
@@ -304,7 +331,7 @@ __device__ __forceinline__ float reduce_scatter9(const float (&v)[9], int lane, 
 // with v = alpha dL/dalpha (0 when alpha was capped), w = alpha T_i; they are
 // added into grad2d, and k_project_bwd maps them to dL/d(mean2d, conic,
 // opacity) with the Gaussian's own A, B, C, o.
-template <int kRPL>
+template <int kRPL, bool kDepth>
 __global__ void __launch_bounds__(kTilePixels / kRPL, 56 / kRPL)
 k_render_bwd(CamConst cam, const float4 *__restrict__ xyod, const float4 *__restrict__ conr,
              const float4 *__restrict__ rgb, const uint32_t *__restrict__ pair_gid,
@@ -332,30 +359,32 @@ k_render_bwd(CamConst cam, const float4 *__restrict__ xyod, const float4 *__rest
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
 
     // Per pixel state, two rows per float2 (x: row 2i, y: row 2i + 1).
-    float2 T[kPairs], sg[kPairs], g0[kPairs], g1[kPairs], g2[kPairs], nfy[kPairs];
+    constexpr int kC = kDepth ? 4 : 3;  // image channels
+    float2 T[kPairs], sg[kPairs], g0[kPairs], g1[kPairs], g2[kPairs], g3[kPairs], nfy[kPairs];
     uint32_t lst[kRPL];
     uint32_t lane_max = range.x;
 #pragma unroll
     for (int r = 0; r < kRPL; r++) {
-        float t = 1.f, d0 = 0.f, d1 = 0.f, d2 = 0.f;
+        float t = 1.f, d0 = 0.f, d1 = 0.f, d2 = 0.f, d3 = 0.f;
         lst[r] = range.x;
         const int py = L.py0 + r;
         if (col_in && py < cam.height) {
             const size_t p = (size_t)py * cam.width + L.px;
             t = T_final[p];
             lst[r] = min(max(last[p], range.x), range.y);  // never walk outside the tile's list
-            d0 = dL_dimage[3 * p];
-            d1 = dL_dimage[3 * p + 1];
-            d2 = dL_dimage[3 * p + 2];
+            d0 = dL_dimage[kC * p];
+            d1 = dL_dimage[kC * p + 1];
+            d2 = dL_dimage[kC * p + 2];
+            if (kDepth) d3 = dL_dimage[kC * p + 3];
         }
-        const float s0 = t * (cam.bg[0] * d0 + cam.bg[1] * d1 + cam.bg[2] * d2);
+        const float s0 = t * (cam.bg[0] * d0 + cam.bg[1] * d1 + cam.bg[2] * d2);  // depth: no background
         const float nf = -(L.fy0 + (float)r);
         if (r & 1) {
-            T[r / 2].y = t; g0[r / 2].y = d0; g1[r / 2].y = d1; g2[r / 2].y = d2; sg[r / 2].y = s0;
-            nfy[r / 2].y = nf;
+            T[r / 2].y = t; g0[r / 2].y = d0; g1[r / 2].y = d1; g2[r / 2].y = d2; g3[r / 2].y = d3;
+            sg[r / 2].y = s0; nfy[r / 2].y = nf;
         } else {
-            T[r / 2].x = t; g0[r / 2].x = d0; g1[r / 2].x = d1; g2[r / 2].x = d2; sg[r / 2].x = s0;
-            nfy[r / 2].x = nf;
+            T[r / 2].x = t; g0[r / 2].x = d0; g1[r / 2].x = d1; g2[r / 2].x = d2; g3[r / 2].x = d3;
+            sg[r / 2].x = s0; nfy[r / 2].x = nf;
         }
         lane_max = max(lane_max, lst[r]);
     }
@@ -429,7 +458,7 @@ k_render_bwd(CamConst cam, const float4 *__restrict__ xyod, const float4 *__rest
             // sum exactly (colours of drawn Gaussians are finite); T is kept
             // by a select.
             const float4 c = s_col[k];
-            float2 sv = make_float2(0.f, 0.f), sgy = sv, sgyy = sv, cr0 = sv, cr1 = sv, cr2 = sv;
+            float2 sv = make_float2(0.f, 0.f), sgy = sv, sgyy = sv, cr0 = sv, cr1 = sv, cr2 = sv, cr3 = sv;
 #pragma unroll
             for (int i = 0; i < kPairs; i++) {
                 const bool h0 = hit[2 * i], h1 = hit[2 * i + 1];
@@ -440,14 +469,16 @@ k_render_bwd(CamConst cam, const float4 *__restrict__ xyod, const float4 *__rest
                 const float2 ri = make_float2(rcp_approx(om.x), rcp_approx(om.y));
                 const float2 Ti = __fmul2_rn(T[i], ri);
                 const float2 w = __fmul2_rn(a, Ti);
-                const float2 cg = __ffma2_rn(make_float2(c.z, c.z), g2[i],
-                                             __ffma2_rn(make_float2(c.y, c.y), g1[i],
-                                                        __fmul2_rn(make_float2(c.x, c.x), g0[i])));
+                float2 cg = __ffma2_rn(make_float2(c.z, c.z), g2[i],
+                                       __ffma2_rn(make_float2(c.y, c.y), g1[i],
+                                                  __fmul2_rn(make_float2(c.x, c.x), g0[i])));
+                if (kDepth) cg = __ffma2_rn(make_float2(c.w, c.w), g3[i], cg);
                 const float2 dLda = __fmul2_rn(ri, __ffma2_rn(T[i], cg, make_float2(-sg[i].x, -sg[i].y)));
                 sg[i] = __ffma2_rn(w, cg, sg[i]);
                 cr0 = __ffma2_rn(w, g0[i], cr0);
                 cr1 = __ffma2_rn(w, g1[i], cr1);
                 cr2 = __ffma2_rn(w, g2[i], cr2);
+                if (kDepth) cr3 = __ffma2_rn(w, g3[i], cr3);
                 float2 v = __fmul2_rn(dLda, a);  // dL/dsigma = -v, dL/do = v / o
                 v.x = cap0 ? 0.f : v.x;
                 v.y = cap1 ? 0.f : v.y;
@@ -460,11 +491,19 @@ k_render_bwd(CamConst cam, const float4 *__restrict__ xyod, const float4 *__rest
             }
             const float svs = sv.x + sv.y, sgys = sgy.x + sgy.y;
             const float sgx = svs * ct.dx;
-            const float vals[9] = {svs, sgx, sgys, sgx * ct.dx, sgys * ct.dx, sgyy.x + sgyy.y,
-                                   cr0.x + cr0.y, cr1.x + cr1.y, cr2.x + cr2.y};
+            constexpr int kV = 6 + kC;
             int idx;
-            const float tot = reduce_scatter9(vals, lane, &idx);
-            if (idx < 9) atomicAdd(grad2d + 12 * (size_t)s_gid[k] + idx, tot);
+            float tot;
+            if (kDepth) {
+                const float vals[10] = {svs, sgx, sgys, sgx * ct.dx, sgys * ct.dx, sgyy.x + sgyy.y,
+                                        cr0.x + cr0.y, cr1.x + cr1.y, cr2.x + cr2.y, cr3.x + cr3.y};
+                tot = reduce_scatter<10>(vals, lane, &idx);
+            } else {
+                const float vals[9] = {svs, sgx, sgys, sgx * ct.dx, sgys * ct.dx, sgyy.x + sgyy.y,
+                                       cr0.x + cr0.y, cr1.x + cr1.y, cr2.x + cr2.y};
+                tot = reduce_scatter<9>(vals, lane, &idx);
+            }
+            if (idx < kV) atomicAdd(grad2d + 12 * (size_t)s_gid[k] + idx, tot);
         }
         __syncthreads();
         bend = bstart;
@@ -567,7 +606,14 @@ cudaError_t launch_render_fwd(const CamConst &c, const gs_projected &proj, const
                               float *image, float *T_final, uint32_t *last, cudaStream_t s) {
     const int tiles = c.tiles_x * c.tiles_y;
     prof_before("render_fwd", s);
-    k_render_fwd<<<tiles, kTilePixels, 0, s>>>(
+    if (c.flags & GS_FLAG_DEPTH)
+        k_render_fwd<true><<<tiles, kTilePixels, 0, s>>>(
+        c, reinterpret_cast<const float4 *>(proj.xy_opacity_depth),
+        reinterpret_cast<const float4 *>(proj.conic_radius), reinterpret_cast<const float4 *>(proj.rgb),
+        bins.pair_gid, reinterpret_cast<const uint2 *>(bins.ranges), tile_order(bins), image, T_final,
+        last);
+    else
+        k_render_fwd<false><<<tiles, kTilePixels, 0, s>>>(
         c, reinterpret_cast<const float4 *>(proj.xy_opacity_depth),
         reinterpret_cast<const float4 *>(proj.conic_radius), reinterpret_cast<const float4 *>(proj.rgb),
         bins.pair_gid, reinterpret_cast<const uint2 *>(bins.ranges), tile_order(bins), image, T_final,
@@ -581,7 +627,14 @@ cudaError_t launch_render_bwd(const CamConst &c, const gs_projected &proj, const
                               float *grad2d, cudaStream_t s) {
     const int tiles = c.tiles_x * c.tiles_y;
     prof_before("render_bwd", s);
-    k_render_bwd<GS_BWD_RPL><<<tiles, kTilePixels / GS_BWD_RPL, 0, s>>>(
+    if (c.flags & GS_FLAG_DEPTH)
+        k_render_bwd<GS_BWD_RPL, true><<<tiles, kTilePixels / GS_BWD_RPL, 0, s>>>(
+        c, reinterpret_cast<const float4 *>(proj.xy_opacity_depth),
+        reinterpret_cast<const float4 *>(proj.conic_radius), reinterpret_cast<const float4 *>(proj.rgb),
+        bins.pair_gid, reinterpret_cast<const uint2 *>(bins.ranges), tile_order(bins), T_final, last,
+        dL_dimage, grad2d);
+    else
+        k_render_bwd<GS_BWD_RPL, false><<<tiles, kTilePixels / GS_BWD_RPL, 0, s>>>(
         c, reinterpret_cast<const float4 *>(proj.xy_opacity_depth),
         reinterpret_cast<const float4 *>(proj.conic_radius), reinterpret_cast<const float4 *>(proj.rgb),
         bins.pair_gid, reinterpret_cast<const uint2 *>(bins.ranges), tile_order(bins), T_final, last,

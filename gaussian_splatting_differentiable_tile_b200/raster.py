@@ -7,7 +7,7 @@ import math
 
 import torch
 
-from . import (GS_ERR_CAPACITY, Bins, GSError, Projected, gs_bin_and_sort, gs_project, gs_render_bwd,
+from . import (GS_ERR_CAPACITY, Bins, GSError, Projected, channels, gs_bin_and_sort, gs_project, gs_render_bwd,
                gs_render_fwd)
 
 
@@ -52,6 +52,9 @@ class Rasterizer:
                 self.n_pairs = gs_bin_and_sort(cam, n, self.proj, self.bins, sync=True)
         else:
             gs_bin_and_sort(cam, n, self.proj, self.bins, sync=False)
+        ch = channels(cam)
+        if self.image.shape[-1] != ch:  # RGB, or RGB + depth with GS_FLAG_DEPTH
+            self.image = torch.empty((self.height, self.width, ch), dtype=torch.float32, device=self.device)
         gs_render_fwd(cam, n, self.proj, self.bins, self.image, self.T_final, self.last)
         return self.image
 

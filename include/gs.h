@@ -114,7 +114,14 @@ typedef struct gs_camera {
 #define GS_FLAG_CAP_0999 8u
 #define GS_FLAG_RADII_AXIS 16u
 #define GS_FLAG_RADII_OPACITY 32u
-#define GS_FLAGS_ALL 63u
+/* GS_FLAG_DEPTH ([GSP] s5: channels of any kind blend alike): a fourth
+ * channel, each Gaussian's camera z, blended with the colours' weights and
+ * no background term: image and dL_dimage are [H][W][4] (R, G, B,
+ * sum_i w_i z_i; divide by 1 - T_final for the expected depth), and the
+ * backward carries the fourth channel's gradient into the means.  rgb[3] of
+ * the projected record holds z. */
+#define GS_FLAG_DEPTH 64u
+#define GS_FLAGS_ALL 127u
 
 /* Raw (unconstrained) parameters of N Gaussians ([GSP] s1), fp32, C-contiguous. */
 typedef struct gs_params {
@@ -222,9 +229,10 @@ int gs_bin_and_sort(const gs_camera *cam, int64_t n, const gs_projected *proj,
  * taken in the order gs_bin_and_sort left in bins->scratch): for each
  * pixel, its tile's pairs in order, sigma as above at (j + 0.5, i + 0.5),
  * alpha = min(0.99, o exp(-sigma)); skip if sigma < 0 or alpha < 1/255;
- * stop (without adding) once T (1 - alpha) < 1e-4; C += c alpha T.
+ * stop (without adding) once T (1 - alpha) < 1e-4; C += c alpha T (the cap,
+ * the stop test and a depth channel per the camera's flags).
  * Outputs (device, caller-owned, fully overwritten):
- *   image   [H][W][3]  C + T_final bg
+ *   image   [H][W][3]  C + T_final bg ([H][W][4] with GS_FLAG_DEPTH)
  *   T_final [H][W]     final transmittance
  *   last    [H][W]     one past the index (into pair_gid) of the last entry the
  *                      pixel added; the tile's start when it added none
@@ -240,9 +248,11 @@ int gs_render_fwd(const gs_camera *cam, int64_t n, const gs_projected *proj, con
  * atomics.  Then the chain rule to the raw parameters, one thread per
  * Gaussian.  Culled Gaussians get exact zeros.
  *   dL_dimage [H][W][3]  gradient of the loss with respect to `image`
+ *                        ([H][W][4] with GS_FLAG_DEPTH)
  *   grad2d    [N][12]    caller scratch, 16-byte aligned; overwritten.  On
  *                        return holds per Gaussian dL/d(mean2d x, y), dL/dA,
- *                        dL/dB, dL/dC, dL/dopacity, dL/d(r, g, b), 0, 0, 0
+ *                        dL/dB, dL/dC, dL/dopacity, dL/d(r, g, b), dL/d of
+ *                        the depth channel's value (0 without the flag), 0, 0
  *   grads                raw-parameter gradients, overwritten
  * `proj`, `bins`, T_final and last must be those of the forward call.
  * Errors: INVALID_ARG, ALIGNMENT, CUDA. */

@@ -204,7 +204,14 @@ def make_cameras(spec: SceneSpec | str, count: int | None = None) -> list:
     return cams
 
 
-def make_target(width: int, height: int, seed: int = 0) -> np.ndarray:
-    """A seeded U(0, 1) target image, (H, W, 3) float32."""
+def make_target(width: int, height: int, seed: int = 0, channels: int = 3) -> np.ndarray:
+    """A seeded U(0, 1) target image, (H, W, 3) float32; with channels=4 a
+    fourth, depth channel U(2, 8) follows (drawn after the colours, so the
+    colours do not depend on it)."""
     rng = np.random.default_rng(10_000 + seed)
-    return np.ascontiguousarray(rng.uniform(0.0, 1.0, size=(height, width, 3)), dtype=np.float32)
+    rgb = rng.uniform(0.0, 1.0, size=(height, width, 3))
+    if channels == 4:
+        rgb = np.concatenate([rgb, rng.uniform(2.0, 8.0, size=(height, width, 1))], axis=2)
+    elif channels != 3:
+        raise ValueError("channels must be 3 or 4")
+    return np.ascontiguousarray(rgb, dtype=np.float32)

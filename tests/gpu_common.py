@@ -53,7 +53,8 @@ def fill_projected(rec: dict, n: int) -> G.Projected:
     conr[:, :3] = rec["conic"]
     conr[:, 3] = rec["radius"]
     rgb = np.zeros((n, 4), np.float32)
-    rgb[:, :3] = rec["color"]
+    col = np.asarray(rec["color"])
+    rgb[:, :col.shape[1]] = col  # a fourth column is the depth channel
     proj.xy_opacity_depth.copy_(torch.from_numpy(xyod))
     proj.conic_radius.copy_(torch.from_numpy(conr))
     proj.rgb.copy_(torch.from_numpy(rgb))
@@ -79,7 +80,7 @@ def gpu_bin(cam, n, proj, max_pairs=None):
 
 def gpu_render(cam, n, proj, bins):
     H, W = cam.height, cam.width
-    image = torch.full((H, W, 3), float("nan"), device="cuda")
+    image = torch.full((H, W, G.channels(cam)), float("nan"), device="cuda")
     T = torch.full((H, W), float("nan"), device="cuda")
     last = torch.full((H, W), -1, dtype=torch.int32, device="cuda")
     G.gs_render_fwd(cam, n, proj, bins, image, T, last)

@@ -86,7 +86,7 @@ def test_fullsize_binning_blend_and_backward(scene):
     g2 = grad2d.cpu().numpy()
     touched = np.abs(g2_ref).sum(axis=1) > 0
     assert touched.sum() > 1000
-    grad_compare(g2[:, :9], g2_ref, g2_abs, "grad2d")
+    grad_compare(g2[:, :g2_ref.shape[1]], g2_ref, g2_abs, "grad2d")
     raw_ref = O.project_bwd(params, cam, g2_ref)
     bound = O.grad_bound(params, cam, g2_abs)
     for k in G.PARAM_KEYS:

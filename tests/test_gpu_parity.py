@@ -276,7 +276,7 @@ def _bwd_stage_fed(cam, params, seed=0, tile_mask=None):
     n = params["means"].shape[0]
     rec, proj, bins, K, image, T, last, ref = _fwd_stage_fed(cam, params, tile_mask=tile_mask)
     rng = np.random.default_rng(seed)
-    dl = rng.normal(size=(cam.height, cam.width, 3))
+    dl = rng.normal(size=(cam.height, cam.width, G.channels(cam)))
     keep = ~ambiguous_pixels(ref, with_clamp=True)
     if tile_mask is not None:
         keep &= tiles_to_pixels(tile_mask.reshape(cam.tiles_y, cam.tiles_x).astype(bool), cam)
@@ -296,7 +296,7 @@ def test_render_bwd_matches_oracle(scene):
     cam, params = SCENES[scene]()
     rec, g2, grads, g2_ref, g2_abs, params = _bwd_stage_fed(cam, params)
     assert np.all(g2[:, 9:] == 0)
-    grad_compare(g2[:, :9], g2_ref, g2_abs, "grad2d")
+    grad_compare(g2[:, :g2_ref.shape[1]], g2_ref, g2_abs, "grad2d")
     raw_ref = O.project_bwd(params, cam, g2_ref)
     bound = O.grad_bound(params, cam, g2_abs)
     for k in G.PARAM_KEYS:
@@ -310,7 +310,7 @@ def test_render_bwd_student_sampled_tiles():
     mask = np.zeros(cam.tiles, np.uint8)
     mask[rng.choice(cam.tiles, 80, replace=False)] = 1
     rec, g2, grads, g2_ref, g2_abs, params = _bwd_stage_fed(cam, params, tile_mask=mask)
-    grad_compare(g2[:, :9], g2_ref, g2_abs, "grad2d")
+    grad_compare(g2[:, :g2_ref.shape[1]], g2_ref, g2_abs, "grad2d")
 
 
 # --------------------------------------------- opacity-aware tile cut
@@ -322,14 +322,15 @@ def test_tight_tiles_stage_fed(scene):
     rec, proj, bins, K, image, T, last, ref = _fwd_stage_fed(cam, params)
     _assert_fwd(cam, bins, image, T, last, ref, np.ones((cam.height, cam.width), bool))
     rec, g2, grads, g2_ref, g2_abs, params = _bwd_stage_fed(cam, params)
-    grad_compare(g2[:, :9], g2_ref, g2_abs, "grad2d")
+    grad_compare(g2[:, :g2_ref.shape[1]], g2_ref, g2_abs, "grad2d")
     raw_ref = O.project_bwd(params, cam, g2_ref)
     bound = O.grad_bound(params, cam, g2_abs)
     for k in G.PARAM_KEYS:
         grad_compare(grads[k], raw_ref[k], bound[k], k)
 
 
-@pytest.mark.parametrize("flags", [G.GS_FLAG_CAP_0999 | G.GS_FLAG_STOP_INCLUSIVE, VARIANTS])
+@pytest.mark.parametrize("flags", [G.GS_FLAG_CAP_0999 | G.GS_FLAG_STOP_INCLUSIVE, VARIANTS, G.GS_FLAG_DEPTH,
+                                   VARIANTS | G.GS_FLAG_DEPTH | G.GS_FLAG_TIGHT_TILES])
 def test_variants_stage_fed(flags):
     """The pages' variants (antialiased compensation, gsplat radii, inclusive
     stop test, 0.999 cap): forward and backward on the oracle's records."""
@@ -338,7 +339,7 @@ def test_variants_stage_fed(flags):
     rec, proj, bins, K, image, T, last, ref = _fwd_stage_fed(cam, params)
     _assert_fwd(cam, bins, image, T, last, ref, np.ones((cam.height, cam.width), bool))
     rec, g2, grads, g2_ref, g2_abs, params = _bwd_stage_fed(cam, params)
-    grad_compare(g2[:, :9], g2_ref, g2_abs, "grad2d")
+    grad_compare(g2[:, :g2_ref.shape[1]], g2_ref, g2_abs, "grad2d")
     raw_ref = O.project_bwd(params, cam, g2_ref)
     bound = O.grad_bound(params, cam, g2_abs)
     for k in G.PARAM_KEYS:
@@ -386,7 +387,7 @@ def _without_ambiguous(params, cam):
     return out, int(bad.sum())
 
 
-@pytest.mark.parametrize("flags", [0, G.GS_FLAG_TIGHT_TILES, VARIANTS])
+@pytest.mark.parametrize("flags", [0, G.GS_FLAG_TIGHT_TILES, VARIANTS, VARIANTS | G.GS_FLAG_DEPTH])
 def test_end_to_end_from_raw_parameters(flags):
     """Raw parameters through all four calls vs the oracle from the same raw
     parameters in double precision, L1 loss against a seeded target."""
@@ -398,7 +399,10 @@ def test_end_to_end_from_raw_parameters(flags):
     P = cuda_params(params)
     r = G.Rasterizer(n, cam.width, cam.height)
     image = r.forward(cam, P).clone()
-    target = torch.from_numpy(make_target(cam.width, cam.height)).cuda()
+    tgt = make_target(cam.width, cam.height)
+    if G.channels(cam) == 4:  # a target depth channel as well
+        tgt = np.concatenate([tgt, np.random.default_rng(5).uniform(2, 5, tgt.shape[:2] + (1,))], axis=2)
+    target = torch.from_numpy(np.ascontiguousarray(tgt, np.float32)).cuda()
     dl = torch.empty_like(image)
     loss = torch.zeros(1, device="cuda")
     G.gs_l1_loss_grad(image, target, dl, loss)
