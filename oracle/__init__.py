@@ -5,3 +5,4 @@ the CPU-baseline leg of ``bench.py`` may import this package.  The CUDA
 library and its Python binding never import it, and it never imports them.
 """
 from .oracle import *  # noqa: F401,F403
+from . import train  # noqa: F401
