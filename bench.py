@@ -471,7 +471,34 @@ def run_native(args, spec, rank, world, local):
     h2d = in_bytes
     d2h = out_bytes
 
-    full_ms, fwd_ms, e2e_ms = max_over_ranks([full_ms, fwd_ms, e2e_ms], world, dev)
+    # the batched training step: B cameras per gs_train_step (lanes run
+    # concurrently), then Adam on the mean gradient; one graph per camera group
+    train = None
+    if args.train_cams > 0:
+        B = min(args.train_cams, len(mine))
+        groups = [[(g * B + j) % len(mine) for j in range(B)] for g in range(max(1, len(mine) // B))]
+        tr = G.Trainer(n, W, H, lanes=args.lanes, channels=nc, max_pairs=int(max(pairs) * 1.05) + 4096,
+                       device=dev)
+        Pt = {k: v.clone() for k, v in P.items()}  # Adam moves these, not the frames' parameters
+        tcams = [[mine[j] for j in grp] for grp in groups]
+        ttg = [torch.stack([targets[j] for j in grp]) for grp in groups]
+
+        def step_train(i):
+            tr.step(tcams[i % len(groups)], Pt, ttg[i % len(groups)])
+
+        t_steps = max(1, args.steps // B)
+        _, tprof = timed(step_train, t_steps, args.warmup, profile=True)
+        g_train = graphed(step_train, len(groups))
+        train_ms, _ = timed(g_train, t_steps, args.warmup)
+        st = tr.cam_stats.cpu()
+        if int(st[:, 0].abs().max()) != 0:
+            raise RuntimeError(f"training step: pair list overflow {st.tolist()}")
+        train = {"cameras_per_step": B, "lanes": args.lanes, "steps": t_steps, "ms": train_ms, "prof": tprof,
+                 "slots": min(args.lanes, B)}
+    else:
+        train_ms = 0.0
+
+    full_ms, fwd_ms, e2e_ms, train_ms = max_over_ranks([full_ms, fwd_ms, e2e_ms, train_ms], world, dev)
     frames = args.steps * world
     if rank != 0:
         return
@@ -521,6 +548,23 @@ def run_native(args, spec, rank, world, local):
                           f"extrapolated by tile count ({info['frame_s']:.1f} s/frame)"),
                "fwd_frames_per_s": 1.0 / info["fwd_s"]}
     mean_pairs = statistics.mean(pairs_steps)
+    train_out = None
+    if train is not None:
+        B, t_steps = train["cameras_per_step"], train["steps"]
+        train_out = {"frames_per_s": B * t_steps * world / (train_ms * 1e-3), "ms_per_step": train_ms / t_steps,
+                     "cameras_per_step": B, "lanes": train["lanes"],
+                     "step": "gs_train_step: per camera project, bin, blend, L1, backward into the lane's "
+                             "gradient slot; Adam on the mean gradient; one CUDA graph per camera group"}
+        ad = (train["prof"] or {}).get("adam")
+        if ad:
+            launches, ms = ad
+            # per value: p, m, v and each slot read; p, m, v and the mean gradient written
+            abytes = 14 * n * 4 * (3 + train["slots"] + 4)
+            kernels_per_step = launches / t_steps
+            ach = abytes * t_steps / (ms * 1e-3) / 1e9
+            train_out["adam"] = {"ms_per_step": ms / t_steps, "kernels_per_step": kernels_per_step,
+                                 "bound": "hbm", "achieved": ach, "peak": hbm_peak, "unit": "GB/s",
+                                 "frac": ach / hbm_peak, "bytes_per_step": abytes}
     out = {
         "metric": METRIC,
         "value": frames / (full_ms * 1e-3),
@@ -547,6 +591,7 @@ def run_native(args, spec, rank, world, local):
                 "pipeline": "copy-in, compute and copy-out streams, two buffer slots; L2 flushed every step"},
         "gpu_launches": gpu_launches,
         "clocks": clocks,
+        "train_step": train_out,
     }
     print(json.dumps(out), flush=True)
 
@@ -561,6 +606,9 @@ def main():
     ap.add_argument("--cpu-sample-tiles", type=int, default=48)
     ap.add_argument("--ref-sample-tiles", type=int, default=8)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--train-cams", type=int, default=4,
+                    help="cameras per batched training step (0: do not measure the training step)")
+    ap.add_argument("--lanes", type=int, default=4, help="concurrent camera chains of the training step")
     ap.add_argument("--no-graphs", action="store_true", help="launch every kernel eagerly")
     ap.add_argument("--tiles", choices=("cut", "3sigma"), default="cut",
                     help="tile rectangles: 3-sigma narrowed by the opacity-aware cut, or plain 3-sigma")

@@ -267,6 +267,103 @@ def profile_end(max_stats: int = 64) -> dict:
     return {arr[i].name.decode(): (int(arr[i].launches), float(arr[i].total_ms)) for i in range(m)}
 
 
-from .raster import Rasterizer, rasterize  # noqa: E402,F401
+# ------------------------------------------------------------------ training
+def adam_config(lr: dict, beta1: float = 0.9, beta2: float = 0.999, eps: float = 1e-8) -> _abi.GsAdamConfig:
+    """gs_adam_config from a {group: learning rate} dict over PARAM_KEYS."""
+    c = _abi.GsAdamConfig()
+    for i, k in enumerate(PARAM_KEYS):
+        c.lr[i] = float(lr[k])
+    c.beta1, c.beta2, c.eps = float(beta1), float(beta2), float(eps)
+    return c
 
-__all__ += ["Rasterizer", "rasterize"]
+
+def _set_struct(d: dict | None):
+    return None if d is None else ctypes.byref(_params_struct(d, _abi.GsGrads))
+
+
+def gs_adam_step(params: dict, slots: list, m: dict, v: dict, cfg: _abi.GsAdamConfig, step: torch.Tensor,
+                 grad_scale: float = 1.0, grad_out: dict | None = None, stream=None) -> None:
+    """One Adam step, in place, with g = grad_scale * sum of the slots' gradients;
+    `step` is a CUDA int64 tensor of one element (steps taken), advanced by one."""
+    n = int(params["means"].shape[0])
+    arr = (_abi.GsGrads * max(1, len(slots)))()
+    for i, sl in enumerate(slots):
+        arr[i] = _params_struct(sl, _abi.GsGrads)
+    _check(lib().gs_adam_step(n, _set_struct(params), arr, len(slots), float(grad_scale), _set_struct(m),
+                              _set_struct(v), ctypes.byref(cfg), _dev(step, "step", torch.int64),
+                              _set_struct(grad_out), _stream(stream)), "gs_adam_step")
+
+
+class TrainLane:
+    """The buffers of one camera chain of gs_train_step (include/gs.h
+    gs_train_lane): records, pair list, image state and a gradient slot.
+    `stream` None runs the lane on the step's own stream; otherwise a
+    torch.cuda.Stream of its own, joined through an event."""
+
+    def __init__(self, n: int, width: int, height: int, channels: int, max_pairs: int, own_stream: bool,
+                 device="cuda"):
+        self.n, self.width, self.height = int(n), int(width), int(height)
+        self.device = device
+        self.proj = Projected(self.n, device)
+        self.bins = Bins(self.n, max_pairs, width, height, device)
+        self.image = torch.empty((height, width, channels), dtype=torch.float32, device=device)
+        self.dL_dimage = torch.empty_like(self.image)
+        self.T_final = torch.empty((height, width), dtype=torch.float32, device=device)
+        self.last = torch.empty((height, width), dtype=torch.int32, device=device)
+        self.grad2d = torch.empty((max(self.n, 1), 12), dtype=torch.float32, device=device)
+        self.grads = {k: torch.empty(sh, dtype=torch.float32, device=device)
+                      for k, sh in _param_shapes(self.n).items()}
+        self.stream = torch.cuda.Stream(device=device) if own_stream else None
+        self.done = torch.cuda.Event()
+        self.done.record()  # creates the event
+
+    def regrow(self, max_pairs: int) -> None:
+        self.bins = Bins(self.n, int(max_pairs), self.width, self.height, self.device)
+
+    def struct(self, step_stream) -> _abi.GsTrainLane:
+        ln = _abi.GsTrainLane()
+        ln.proj = self.proj.struct
+        ln.bins = self.bins.struct
+        ln.image = self.image.data_ptr()
+        ln.T_final = self.T_final.data_ptr()
+        ln.last = self.last.data_ptr()
+        ln.dL_dimage = self.dL_dimage.data_ptr()
+        ln.grad2d = self.grad2d.data_ptr()
+        ln.grads = _params_struct(self.grads, _abi.GsGrads)
+        ln.stream = (self.stream.cuda_stream if self.stream is not None else step_stream.value) or None
+        ln.done = self.done.cuda_event
+        return ln
+
+
+def _param_shapes(n: int) -> dict:
+    return {"means": (n, 3), "log_scales": (n, 3), "quats": (n, 4), "opacity_logits": (n,), "colors": (n, 3)}
+
+
+def gs_train_step(cams, params: dict, targets: torch.Tensor, lanes: list, fork: torch.cuda.Event,
+                  m: dict | None, v: dict | None, cfg: _abi.GsAdamConfig | None, step: torch.Tensor | None,
+                  losses: torch.Tensor | None = None, cam_stats: torch.Tensor | None = None,
+                  grad_out: dict | None = None, stream=None) -> None:
+    """One training step over the cameras (include/gs.h gs_train_step): camera
+    b on lane b mod len(lanes), Adam on the mean gradient (cfg None: only
+    grad_out).  targets is [B, H, W, C]; losses [B] float32 and cam_stats
+    [B, 2] int64 (status, K) are optional outputs."""
+    B = len(cams)
+    n = int(params["means"].shape[0])
+    if targets.dim() != 4 or targets.shape[0] != B:
+        raise ValueError("targets must be [B, H, W, C]")
+    carr = (_abi.GsCamera * B)(*[make_camera(c) for c in cams])
+    s = _stream(stream)
+    larr = (_abi.GsTrainLane * len(lanes))(*[ln.struct(s) for ln in lanes])
+    _check(lib().gs_train_step(carr, B, n, _set_struct(params), _dev(targets, "targets", torch.float32), larr,
+                               len(lanes), ctypes.c_void_p(fork.cuda_event), _set_struct(m), _set_struct(v),
+                               None if cfg is None else ctypes.byref(cfg),
+                               _dev(step, "step", torch.int64) if step is not None else None,
+                               _dev(losses, "losses", torch.float32), _dev(cam_stats, "cam_stats", torch.int64),
+                               _set_struct(grad_out), s), "gs_train_step")
+
+
+__all__ += ["adam_config", "gs_adam_step", "TrainLane", "gs_train_step"]
+
+from .raster import Rasterizer, Trainer, rasterize  # noqa: E402,F401
+
+__all__ += ["Rasterizer", "Trainer", "rasterize"]

@@ -67,6 +67,20 @@ class GsBins(ctypes.Structure):
     ]
 
 
+GsParamSet = GsGrads  # gs_param_set: writable arrays in the gs_params layout
+
+
+class GsAdamConfig(ctypes.Structure):
+    _fields_ = [("lr", ctypes.c_float * 5), ("eps", ctypes.c_float), ("beta1", ctypes.c_double),
+                ("beta2", ctypes.c_double)]
+
+
+class GsTrainLane(ctypes.Structure):
+    _fields_ = [("proj", GsProjected), ("bins", GsBins), ("image", ctypes.c_void_p), ("T_final", ctypes.c_void_p),
+                ("last", ctypes.c_void_p), ("dL_dimage", ctypes.c_void_p), ("grad2d", ctypes.c_void_p),
+                ("grads", GsGrads), ("stream", ctypes.c_void_p), ("done", ctypes.c_void_p)]
+
+
 class GsProfileStat(ctypes.Structure):
     _fields_ = [("name", ctypes.c_char * 32), ("launches", ctypes.c_int32), ("total_ms", ctypes.c_float)]
 
@@ -99,6 +113,15 @@ PROTOTYPES = {
                                        ctypes.c_void_p]),
     "gs_l1_loss_grad": (ctypes.c_int, [ctypes.c_void_p, ctypes.c_void_p, ctypes.c_int64, ctypes.c_void_p,
                                        ctypes.c_void_p, ctypes.c_void_p]),
+    "gs_adam_step": (ctypes.c_int, [ctypes.c_int64, ctypes.POINTER(GsGrads), ctypes.POINTER(GsGrads), ctypes.c_int32,
+                                    ctypes.c_float, ctypes.POINTER(GsGrads), ctypes.POINTER(GsGrads),
+                                    ctypes.POINTER(GsAdamConfig), ctypes.c_void_p, ctypes.POINTER(GsGrads),
+                                    ctypes.c_void_p]),
+    "gs_train_step": (ctypes.c_int, [ctypes.POINTER(GsCamera), ctypes.c_int32, ctypes.c_int64,
+                                     ctypes.POINTER(GsGrads), ctypes.c_void_p, ctypes.POINTER(GsTrainLane),
+                                     ctypes.c_int32, ctypes.c_void_p, ctypes.POINTER(GsGrads),
+                                     ctypes.POINTER(GsGrads), ctypes.POINTER(GsAdamConfig), ctypes.c_void_p,
+                                     ctypes.c_void_p, ctypes.c_void_p, ctypes.POINTER(GsGrads), ctypes.c_void_p]),
     "gs_read_status": (ctypes.c_int, [ctypes.POINTER(GsBins), ctypes.POINTER(ctypes.c_int64),
                                       ctypes.c_void_p]),
     "gs_error_string": (ctypes.c_char_p, [ctypes.c_int]),

@@ -311,6 +311,190 @@ int gs_l1_loss_grad(const float *image, const float *target, int64_t count, floa
                : GS_ERR_CUDA;
 }
 
+// ---------------------------------------------------------------- training
+namespace {
+
+bool set_complete(const gs_param_set *p) {
+    return p && p->means && p->log_scales && p->quats && p->opacity_logits && p->colors;
+}
+
+int check_adam_cfg(const gs_adam_config *cfg) {
+    if (!cfg) return GS_ERR_INVALID_ARG;
+    for (float lr : cfg->lr)
+        if (!std::isfinite(lr) || lr < 0.f) return GS_ERR_INVALID_ARG;
+    if (!(cfg->beta1 >= 0.0 && cfg->beta1 < 1.0) || !(cfg->beta2 >= 0.0 && cfg->beta2 < 1.0) ||
+        !(cfg->eps > 0.f) || !std::isfinite(cfg->eps))
+        return GS_ERR_INVALID_ARG;
+    return GS_OK;
+}
+
+AdamBetas adam_betas(const gs_adam_config *cfg) {
+    AdamBetas b{};
+    if (!cfg) return b;
+    b.b1 = cfg->beta1;
+    b.b2 = cfg->beta2;
+    b.b1f = (float)cfg->beta1;
+    b.b2f = (float)cfg->beta2;
+    b.omb1 = (float)(1.0 - cfg->beta1);
+    b.omb2 = (float)(1.0 - cfg->beta2);
+    return b;
+}
+
+// Adam's launch description from the parameter, moment, slot and output sets.
+// M and V are null for a gradient sum without update.
+int adam_groups(int64_t n, const gs_param_set &P, const gs_param_set *slots, int n_slots,
+                const gs_param_set *M, const gs_param_set *V, const gs_param_set *out,
+                const gs_adam_config *cfg, AdamGroups *G) {
+    float *gs_param_set::*field[5] = {&gs_param_set::means, &gs_param_set::log_scales, &gs_param_set::quats,
+                                      &gs_param_set::opacity_logits, &gs_param_set::colors};
+    const int64_t width[5] = {3, 3, 4, 1, 3};
+    for (int k = 0; k < 5; k++) {
+        AdamGroup &A = G->g[k];
+        A = AdamGroup{};
+        A.p = P.*field[k];
+        A.m = M ? M->*field[k] : nullptr;
+        A.v = V ? V->*field[k] : nullptr;
+        A.out = out ? out->*field[k] : nullptr;
+        A.count = n * width[k];
+        A.lr = cfg ? cfg->lr[k] : 0.f;
+        bool vec = aligned(A.p, 16) && aligned(A.m, 16) && aligned(A.v, 16) && aligned(A.out, 16);
+        for (int s = 0; s < n_slots; s++) {
+            A.slot[s] = slots[s].*field[k];
+            vec = vec && aligned(A.slot[s], 16);
+        }
+        A.vec = vec ? 1 : 0;
+        if (k == 2 && !vec) return GS_ERR_ALIGNMENT;  // quaternion arrays are float4
+        if (!aligned(A.p, 4) || !aligned(A.m, 4) || !aligned(A.v, 4) || !aligned(A.out, 4))
+            return GS_ERR_ALIGNMENT;
+        for (int s = 0; s < n_slots; s++)
+            if (!aligned(A.slot[s], 4)) return GS_ERR_ALIGNMENT;
+    }
+    return GS_OK;
+}
+
+}  // namespace
+
+int gs_adam_step(int64_t n, const gs_param_set *params, const gs_param_set *slots, int32_t n_slots,
+                 float grad_scale, const gs_param_set *m, const gs_param_set *v,
+                 const gs_adam_config *cfg, int64_t *step, const gs_param_set *grad_out,
+                 void *stream) {
+    if (n < 0 || n_slots < 1 || n_slots > kAdamMaxSlots || !step || !params || !slots || !m || !v ||
+        !std::isfinite(grad_scale))
+        return GS_ERR_INVALID_ARG;
+    if (n > kMaxCount) return GS_ERR_TOO_LARGE;
+    int rc = check_adam_cfg(cfg);
+    if (rc) return rc;
+    if (!aligned(step, 8)) return GS_ERR_ALIGNMENT;
+    if (n > 0) {
+        if (!set_complete(params) || !set_complete(m) || !set_complete(v) ||
+            (grad_out && !set_complete(grad_out)))
+            return GS_ERR_INVALID_ARG;
+        for (int s = 0; s < n_slots; s++)
+            if (!set_complete(&slots[s])) return GS_ERR_INVALID_ARG;
+    }
+    AdamGroups G;
+    if (n > 0 && (rc = adam_groups(n, *params, slots, n_slots, m, v, grad_out, cfg, &G))) return rc;
+    return launch_adam(G, n > 0 ? 4 * n : 0, adam_betas(cfg), cfg->eps, grad_scale, n_slots, step,
+                       as_stream(stream)) == cudaSuccess
+               ? GS_OK
+               : GS_ERR_CUDA;
+}
+
+int gs_train_step(const gs_camera *cams, int32_t n_cams, int64_t n, const gs_param_set *params,
+                  const float *targets, const gs_train_lane *lanes, int32_t n_lanes, void *fork,
+                  const gs_param_set *m, const gs_param_set *v, const gs_adam_config *cfg,
+                  int64_t *step, float *losses, int64_t *cam_stats, const gs_param_set *grad_out,
+                  void *stream) {
+    if (!cams || n_cams < 1 || !lanes || n_lanes < 1 || n_lanes > kAdamMaxSlots || n < 0 || !params ||
+        !targets)
+        return GS_ERR_INVALID_ARG;
+    if (n > kMaxCount) return GS_ERR_TOO_LARGE;
+    if (!cfg && !grad_out) return GS_ERR_INVALID_ARG;
+    int rc;
+    if (cfg && ((rc = check_adam_cfg(cfg)) || !m || !v || !step)) return rc ? rc : GS_ERR_INVALID_ARG;
+    if (cfg && !aligned(step, 8)) return GS_ERR_ALIGNMENT;
+    if (!aligned(targets, 4) || (losses && !aligned(losses, 4)) || (cam_stats && !aligned(cam_stats, 8)))
+        return GS_ERR_ALIGNMENT;
+    if (n > 0 && (!set_complete(params) || (cfg && (!set_complete(m) || !set_complete(v))) ||
+                  (grad_out && !set_complete(grad_out))))
+        return GS_ERR_INVALID_ARG;
+    // cameras: valid, one image size and channel count
+    std::vector<CamConst> cc((size_t)n_cams);
+    for (int b = 0; b < n_cams; b++) {
+        if ((rc = make_cam(&cams[b], &cc[b]))) return rc;
+        if (cc[b].width != cc[0].width || cc[b].height != cc[0].height ||
+            ((cc[b].flags ^ cc[0].flags) & GS_FLAG_DEPTH))
+            return GS_ERR_INVALID_ARG;
+    }
+    const int64_t pixels = (int64_t)cc[0].width * cc[0].height;
+    const int64_t values = pixels * ((cc[0].flags & GS_FLAG_DEPTH) ? 4 : 3);
+    gs_params pc{params->means, params->log_scales, params->quats, params->opacity_logits, params->colors};
+    if ((rc = check_params(&pc, n))) return rc;
+    // lanes: complete buffers for this camera size and N
+    const int used = std::min(n_lanes, n_cams);
+    std::vector<BinsLayout> L((size_t)used);
+    for (int l = 0; l < used; l++) {
+        const gs_train_lane &ln = lanes[l];
+        if ((rc = check_projected(&ln.proj, n)) || (rc = check_bins(&ln.bins, n, cc[0], &L[l]))) return rc;
+        if (!ln.image || !ln.T_final || !ln.last || !ln.dL_dimage || (n > 0 && !ln.grad2d))
+            return GS_ERR_INVALID_ARG;
+        if (n > 0 && !set_complete(&ln.grads)) return GS_ERR_INVALID_ARG;
+        if (!aligned(ln.image, 4) || !aligned(ln.T_final, 4) || !aligned(ln.last, 4) ||
+            !aligned(ln.dL_dimage, 4) || !aligned(ln.grad2d, 16) || !aligned(ln.grads.quats, 16))
+            return GS_ERR_ALIGNMENT;
+        if (ln.stream != stream && (!fork || !ln.done)) return GS_ERR_INVALID_ARG;
+    }
+    // the Adam (or gradient-sum) launch is described before anything runs
+    std::vector<gs_param_set> slots((size_t)used);
+    for (int l = 0; l < used; l++) slots[l] = lanes[l].grads;
+    AdamGroups G;
+    if (n > 0 && (rc = adam_groups(n, *params, slots.data(), used, cfg ? m : nullptr, cfg ? v : nullptr,
+                                   grad_out, cfg, &G)))
+        return rc;
+
+    cudaStream_t s = as_stream(stream);
+    bool forked = false;
+    for (int l = 0; l < used; l++)
+        if (lanes[l].stream != stream) forked = true;
+    if (forked && cudaEventRecord(reinterpret_cast<cudaEvent_t>(fork), s) != cudaSuccess) return GS_ERR_CUDA;
+    for (int l = 0; l < used; l++) {
+        const gs_train_lane &ln = lanes[l];
+        cudaStream_t ls = as_stream(ln.stream);
+        if (ln.stream != stream && cudaStreamWaitEvent(ls, reinterpret_cast<cudaEvent_t>(fork), 0) != cudaSuccess)
+            return GS_ERR_CUDA;
+        for (int b = l; b < n_cams; b += n_lanes) {
+            const CamConst &c = cc[b];
+            const gs_params &pp = pc;
+            if (launch_project(c, n, pp, ln.proj, ls) != cudaSuccess ||
+                launch_bin_and_sort(c, n, ln.proj, ln.bins, L[l], ls) != cudaSuccess ||
+                launch_render_fwd(c, ln.proj, ln.bins, ln.image, ln.T_final, ln.last, ls) != cudaSuccess ||
+                launch_l1_train(ln.image, targets + (size_t)b * values, values, ln.dL_dimage,
+                                losses ? losses + b : nullptr, ln.bins, cam_stats ? cam_stats + 2 * b : nullptr,
+                                ls) != cudaSuccess)
+                return GS_ERR_CUDA;
+            if (n > 0 && cudaMemsetAsync(ln.grad2d, 0, (size_t)n * 12 * sizeof(float), ls) != cudaSuccess)
+                return GS_ERR_CUDA;
+            if (launch_render_bwd(c, ln.proj, ln.bins, ln.T_final, ln.last, ln.dL_dimage, ln.grad2d, ls) !=
+                    cudaSuccess ||
+                launch_project_bwd(c, n, pp, ln.proj, ln.grad2d, ln.grads, ls, b >= n_lanes) != cudaSuccess)
+                return GS_ERR_CUDA;
+        }
+        if (ln.stream != stream &&
+            (cudaEventRecord(reinterpret_cast<cudaEvent_t>(ln.done), ls) != cudaSuccess ||
+             cudaStreamWaitEvent(s, reinterpret_cast<cudaEvent_t>(ln.done), 0) != cudaSuccess))
+            return GS_ERR_CUDA;
+    }
+    const float scale = 1.f / (float)n_cams;
+    if (cfg)
+        return launch_adam(G, n > 0 ? 4 * n : 0, adam_betas(cfg), cfg->eps, scale, used, step, s) ==
+                       cudaSuccess
+                   ? GS_OK
+                   : GS_ERR_CUDA;
+    return launch_adam(G, n > 0 ? 4 * n : 0, adam_betas(nullptr), 1.f, scale, used, nullptr, s, false) == cudaSuccess
+               ? GS_OK
+               : GS_ERR_CUDA;
+}
+
 int gs_profile_begin(int32_t max_launches) {
     if (max_launches < 0) return GS_ERR_INVALID_ARG;
     for (auto &r : g_prof) {

@@ -5,6 +5,8 @@
 #include <cuda_runtime.h>
 #include <stdint.h>
 
+#include <algorithm>
+
 #include "gs.h"
 
 namespace gs {
@@ -103,13 +105,28 @@ __device__ __forceinline__ void set_status(int32_t *status, int32_t code) {
 }
 #endif
 
+// Adam over the five parameter groups (gs_train.cu).
+constexpr int kAdamMaxSlots = 16;
+struct AdamGroup {
+    float *p, *m, *v;                    // parameters and moments, updated in place
+    float *out;                          // nullable: the summed, scaled gradient
+    const float *slot[kAdamMaxSlots];    // gradient slots, summed in order
+    int64_t count;                       // values in the group
+    float lr;
+    int vec;                             // every array 16-byte aligned: float4 path
+};
+struct AdamGroups {
+    AdamGroup g[5];  // means, log_scales, quats, opacity_logits, colors
+};
+
 // ------------------------------------------------------------- launchers
 // Each returns cudaGetLastError() of its launches.
 cudaError_t launch_project(const CamConst &c, int64_t n, const gs_params &p, const gs_projected &o,
                            cudaStream_t s);
+// accumulate: add the raw-parameter gradients into g instead of writing them
 cudaError_t launch_project_bwd(const CamConst &c, int64_t n, const gs_params &p,
                                const gs_projected &proj, float *grad2d, const gs_grads &g,
-                               cudaStream_t s);
+                               cudaStream_t s, bool accumulate = false);
 cudaError_t launch_bin_and_sort(const CamConst &c, int64_t n, const gs_projected &proj,
                                 const gs_bins &bins, const BinsLayout &L, cudaStream_t s);
 cudaError_t launch_render_fwd(const CamConst &c, const gs_projected &proj, const gs_bins &bins,
@@ -121,6 +138,17 @@ cudaError_t launch_render_stats(const CamConst &c, const gs_projected &proj, con
                                 const uint32_t *last, uint64_t *counts, cudaStream_t s);
 cudaError_t launch_l1(const float *image, const float *target, int64_t count, float *dL_dimage,
                       float *loss, cudaStream_t s);
+cudaError_t launch_l1_train(const float *image, const float *target, int64_t count, float *dL_dimage,
+                            float *loss, const gs_bins &bins, int64_t *stats, cudaStream_t s);
+// update: k_adam_tick (advances *step), then k_adam when max_count > 0;
+// otherwise only the scaled slot sum is written to each group's `out`
+struct AdamBetas {
+    double b1, b2;   // for the bias corrections
+    float b1f, b2f;  // beta rounded once, for the moment updates
+    float omb1, omb2;  // 1 - beta computed in double, rounded once
+};
+cudaError_t launch_adam(const AdamGroups &G, int64_t max_count, const AdamBetas &betas, float eps,
+                        float grad_scale, int n_slots, int64_t *step, cudaStream_t s, bool update = true);
 
 // Profiling hooks used around every launch (gs_api.cu).
 void prof_before(const char *name, cudaStream_t s);

@@ -252,6 +252,14 @@ __device__ __forceinline__ void rotmat_vjp(const float *qh, const float *G, floa
 // Those values are written back: on return grad2d holds
 // dL/d(mx, my, A, B, C, opacity, r, g, b, depth channel, 0, 0) (the depth
 // channel's entry is 0 without GS_FLAG_DEPTH).
+// Stores (or, with kAcc, adds) one raw-parameter gradient value.
+template <bool kAcc>
+__device__ __forceinline__ void put(float *a, int i, float x) {
+    if (kAcc) a[i] += x;
+    else a[i] = x;
+}
+
+template <bool kAcc>
 __global__ void __launch_bounds__(256)
 k_project_bwd(CamConst cam, int n, const float *__restrict__ means,
               const float *__restrict__ log_scales, const float *__restrict__ quats,
@@ -280,6 +288,7 @@ k_project_bwd(CamConst cam, int n, const float *__restrict__ means,
     grad2d[3 * g + 1] = g1;
     grad2d[3 * g + 2] = g2;
     if (!P.valid) {  // [GSP] s6: culled Gaussians get exact zeros
+        if (kAcc) return;
         for (int k = 0; k < 3; k++) {
             d_means[3 * g + k] = 0.f;
             d_log_scales[3 * g + k] = 0.f;
@@ -291,11 +300,11 @@ k_project_bwd(CamConst cam, int n, const float *__restrict__ means,
     }
     const float d_mx = g0.x, d_my = g0.y, d_A = g0.z, d_B = g0.w;
     const float d_C = g1.x, d_o = g1.y;
-    d_colors[3 * g] = g1.z;
-    d_colors[3 * g + 1] = g1.w;
-    d_colors[3 * g + 2] = g2.x;
+    put<kAcc>(d_colors, 3 * g, g1.z);
+    put<kAcc>(d_colors, 3 * g + 1, g1.w);
+    put<kAcc>(d_colors, 3 * g + 2, g2.x);
     // opacity = sigmoid(logit) x comp
-    d_logits[g] = d_o * P.comp * P.opacity_raw * (1.f - P.opacity_raw);
+    put<kAcc>(d_logits, g, d_o * P.comp * P.opacity_raw * (1.f - P.opacity_raw));
 
     // conic = (c, -b, a) / det; no gradient through a clamped det
     const float inv_det = 1.f / P.det;
@@ -359,7 +368,7 @@ k_project_bwd(CamConst cam, int n, const float *__restrict__ means,
     // t = W mu + tv
 #pragma unroll
     for (int j = 0; j < 3; j++)
-        d_means[3 * g + j] = cam.R[j] * dt0 + cam.R[3 + j] * dt1 + cam.R[6 + j] * dt2;
+        put<kAcc>(d_means, 3 * g + j, cam.R[j] * dt0 + cam.R[3 + j] * dt1 + cam.R[6 + j] * dt2);
     // Sc = W Sigma W^T -> dSigma = W^T dSc W
     float T1[9], dS[9];
 #pragma unroll
@@ -388,8 +397,8 @@ k_project_bwd(CamConst cam, int n, const float *__restrict__ means,
         for (int j = 0; j < 3; j++) dR[3 * i + j] = dM[3 * i + j] * P.s[j];
 #pragma unroll
     for (int j = 0; j < 3; j++)
-        d_log_scales[3 * g + j] =
-            (dM[j] * P.R[j] + dM[3 + j] * P.R[3 + j] + dM[6 + j] * P.R[6 + j]) * P.s[j];
+        put<kAcc>(d_log_scales, 3 * g + j,
+                  (dM[j] * P.R[j] + dM[3 + j] * P.R[3 + j] + dM[6 + j] * P.R[6 + j]) * P.s[j]);
     // R(q_hat) -> q_hat -> q through the normalisation with its clamp
     float dqh[4];
     rotmat_vjp(P.qh, dR, dqh);
@@ -402,6 +411,10 @@ k_project_bwd(CamConst cam, int n, const float *__restrict__ means,
     } else {
         const float iq = 1.f / kQuatEps;
         dq = make_float4(dqh[0] * iq, dqh[1] * iq, dqh[2] * iq, dqh[3] * iq);
+    }
+    if (kAcc) {
+        const float4 o = reinterpret_cast<const float4 *>(d_quats)[g];
+        dq = make_float4(o.x + dq.x, o.y + dq.y, o.z + dq.z, o.w + dq.w);
     }
     reinterpret_cast<float4 *>(d_quats)[g] = dq;
 }
@@ -425,12 +438,12 @@ cudaError_t launch_project(const CamConst &c, int64_t n, const gs_params &p, con
 
 cudaError_t launch_project_bwd(const CamConst &c, int64_t n, const gs_params &p,
                                const gs_projected &proj, float *grad2d, const gs_grads &g,
-                               cudaStream_t s) {
+                               cudaStream_t s, bool accumulate) {
     if (n == 0) return cudaSuccess;
     const int threads = 256;
     const int blocks = (int)((n + threads - 1) / threads);
     prof_before("project_bwd", s);
-    k_project_bwd<<<blocks, threads, 0, s>>>(c, (int)n, p.means, p.log_scales, p.quats,
+    (accumulate ? k_project_bwd<true> : k_project_bwd<false>)<<<blocks, threads, 0, s>>>(c, (int)n, p.means, p.log_scales, p.quats,
                                              p.opacity_logits,
                                              reinterpret_cast<const float4 *>(proj.xy_opacity_depth),
                                              reinterpret_cast<const float4 *>(proj.conic_radius),

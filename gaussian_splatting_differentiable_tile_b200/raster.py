@@ -7,8 +7,8 @@ import math
 
 import torch
 
-from . import (GS_ERR_CAPACITY, Bins, GSError, Projected, channels, gs_bin_and_sort, gs_project, gs_render_bwd,
-               gs_render_fwd)
+from . import (GS_ERR_CAPACITY, PARAM_KEYS, Bins, GSError, Projected, TrainLane, adam_config, channels,
+               gs_bin_and_sort, gs_project, gs_render_bwd, gs_render_fwd, gs_train_step)
 
 
 class Rasterizer:
@@ -89,3 +89,80 @@ def rasterize(means, log_scales, quats, opacity_logits, colors, cam, rasterizer:
     rasterizer's buffers hold the forward state until backward runs, so one
     rasterizer serves one forward/backward pair at a time."""
     return _RasterizeFn.apply(means, log_scales, quats, opacity_logits, colors, cam, rasterizer)
+
+
+# Learning rates of "Gaussian splatting in PyTorch" s7 (3DGS's latest code):
+# means 1.6e-4 x the scene extent (decayed over training; the caller scales
+# it), scales 5e-3, opacities 2.5e-2, quaternions 1e-3.  The pages give none
+# for colours; 2.5e-3 is used.
+DEFAULT_LR = {"means": 1.6e-4, "log_scales": 5e-3, "quats": 1e-3, "opacity_logits": 2.5e-2, "colors": 2.5e-3}
+
+
+class Trainer:
+    """A batched multi-camera training step with Adam ("Gaussian splatting in
+    PyTorch" s7; "Training a smaller scene": one model fitted to renders from
+    many cameras).  Owns `lanes` camera chains that run concurrently (lane 0
+    on the caller's stream, the others on streams of their own), Adam's
+    moments and its device step counter.  Every step is one gs_train_step
+    call, so it can be captured in a CUDA graph."""
+
+    def __init__(self, n: int, width: int, height: int, lanes: int = 2, channels: int = 3,
+                 max_pairs: int | None = None, lr: dict | None = None, betas=(0.9, 0.999), eps: float = 1e-8,
+                 device="cuda"):
+        self.n, self.width, self.height, self.channels = int(n), int(width), int(height), int(channels)
+        self.device = device
+        mp = int(max_pairs) if max_pairs else max(1024, 16 * self.n)
+        self.lanes = [TrainLane(self.n, width, height, channels, mp, own_stream=(i > 0), device=device)
+                      for i in range(int(lanes))]
+        self.cfg = adam_config(lr or DEFAULT_LR, betas[0], betas[1], eps)
+        shapes = {k: v.shape for k, v in self.lanes[0].grads.items()}
+        self.m = {k: torch.zeros(shapes[k], dtype=torch.float32, device=device) for k in PARAM_KEYS}
+        self.v = {k: torch.zeros(shapes[k], dtype=torch.float32, device=device) for k in PARAM_KEYS}
+        self.step_count = torch.zeros(1, dtype=torch.int64, device=device)
+        self.fork = torch.cuda.Event()
+        self.fork.record()
+        self.grads = {k: torch.empty(shapes[k], dtype=torch.float32, device=device) for k in PARAM_KEYS}
+        self.losses = None
+        self.cam_stats = None
+
+    def fit_pairs(self, cams, params: dict) -> int:
+        """Sizes every lane's pair list for these cameras (one synchronizing
+        binning per camera); returns the largest K."""
+        need = 0
+        lane = self.lanes[0]
+        n = int(params["means"].shape[0])
+        for c in cams:
+            gs_project(c, params, lane.proj)
+            try:
+                k = gs_bin_and_sort(c, n, lane.proj, lane.bins, sync=True)
+            except GSError as e:
+                if e.code != GS_ERR_CAPACITY:
+                    raise
+                k = e.n_pairs
+            need = max(need, k)
+        if need > self.lanes[0].bins.max_pairs:
+            for ln in self.lanes:
+                ln.regrow(int(math.ceil(need * 1.25)) + 1024)
+        return need
+
+    def step(self, cams, params: dict, targets, check: bool = False, adam: bool = True, stream=None):
+        """One step over the cameras (targets [B, H, W, C]); updates params in
+        place (adam=True) and returns the per-camera losses (a device tensor).
+        self.grads receives the mean gradient.  check=True synchronizes and
+        raises GSError(GS_ERR_CAPACITY) if a camera overflowed its pair list
+        (its image was then background only; Adam has already run)."""
+        B = len(cams)
+        if self.losses is None or self.losses.numel() != B:
+            self.losses = torch.zeros(B, dtype=torch.float32, device=self.device)
+            self.cam_stats = torch.zeros((B, 2), dtype=torch.int64, device=self.device)
+        gs_train_step(cams, params, targets, self.lanes, self.fork, self.m if adam else None,
+                      self.v if adam else None, self.cfg if adam else None, self.step_count if adam else None,
+                      self.losses, self.cam_stats, self.grads, stream)
+        if check:
+            st = self.cam_stats.cpu()
+            bad = [b for b in range(B) if int(st[b, 0]) != 0]
+            if bad:
+                err = GSError(int(st[bad[0], 0]), f"gs_train_step (cameras {bad})")
+                err.n_pairs = int(st[:, 1].max())
+                raise err
+        return self.losses

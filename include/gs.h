@@ -20,6 +20,9 @@
  *          pre-flight guards, errors that must not be silent)
  *   [BLOG] 3D Gaussian Splatting course blog index (a backward pass that
  *          recomputes the blend weights instead of storing them)
+ *   [DIST] "The backward pass I deleted trained the model the Nano runs",
+ *          "Training a smaller scene" (a student optimised against the
+ *          teacher's renders from sixty cameras)
  *
  * Conventions shared by every call
  *   - All floating point is IEEE single precision.
@@ -279,6 +282,105 @@ int gs_render_stats(const gs_camera *cam, int64_t n, const gs_projected *proj,
  * loss (device, nullable) receives the mean.  Errors: INVALID_ARG, CUDA. */
 int gs_l1_loss_grad(const float *image, const float *target, int64_t count, float *dL_dimage,
                     float *loss, void *stream);
+
+/* ------------------------------------------------------------- training
+ * The optimisation loop of [GSP] s7 (render, L1 loss against the target,
+ * backward, one Adam step over the raw parameters with a learning rate per
+ * parameter group), batched over several cameras as in [DIST] (a student
+ * fitted to the teacher's renders from sixty cameras, so that it becomes a
+ * 3D model rather than one memorised view). */
+
+/* Five writable arrays in the gs_params layout: the parameters Adam
+ * updates, its two moments, a gradient slot. */
+typedef gs_grads gs_param_set;
+
+/* Adam hyperparameters ([GSP] s7: torch.optim.Adam with per-parameter
+ * learning rates; the pages name 1.6e-4 x scene extent for means (decayed),
+ * 5e-3 for scales, 2.5e-2 for opacities and 1e-3 for quaternions). */
+typedef struct gs_adam_config {
+    float lr[5];   /* means, log_scales, quats, opacity_logits, colors; finite, >= 0 */
+    float eps;     /* > 0, usually 1e-8 (Kingma & Ba; torch's default) */
+    double beta1;  /* [0, 1), usually 0.9 */
+    double beta2;  /* [0, 1), usually 0.999.  The bias corrections use the
+                      betas in double precision; the moment updates use
+                      beta and 1 - beta each rounded once to single */
+} gs_adam_config;
+
+/* One Adam step over the raw parameters, fused with the sum of gradient
+ * slots (Kingma & Ba's algorithm in the form torch.optim.Adam evaluates it):
+ *   g = grad_scale * sum_s slots[s]      (summed in slot order)
+ *   t = *step + 1
+ *   m = beta1 m + (1 - beta1) g
+ *   v = beta2 v + (1 - beta2) g^2
+ *   p = p - (lr / (1 - beta1^t)) m / (sqrt(v) / sqrt(1 - beta2^t) + eps)
+ * with lr the learning rate of p's group; then *step = t.  The step count
+ * lives on the device so that a captured CUDA graph replays correctly; the
+ * bias corrections are evaluated in double precision.
+ *   params    parameters, updated in place
+ *   slots     HOST array of n_slots (1..16) gradient sets (device arrays)
+ *   m, v      moments, updated in place (zero before the first step)
+ *   step      DEVICE int64: steps taken so far; incremented by the call
+ *   grad_out  nullable: receives g
+ * Arrays of quaternions must be 16-byte aligned.  n may be 0 (only the
+ * counter moves).  Errors: INVALID_ARG (n < 0, n_slots out of range, a null
+ * array with n > 0, a learning rate or beta out of range), TOO_LARGE,
+ * ALIGNMENT, CUDA. */
+int gs_adam_step(int64_t n, const gs_param_set *params, const gs_param_set *slots, int32_t n_slots,
+                 float grad_scale, const gs_param_set *m, const gs_param_set *v,
+                 const gs_adam_config *cfg, int64_t *step, const gs_param_set *grad_out,
+                 void *stream);
+
+/* The buffers one camera chain of gs_train_step runs in: the render state of
+ * its current camera, and the lane's gradient slot (the sum of its
+ * cameras' raw-parameter gradients).  All device arrays are caller-owned. */
+typedef struct gs_train_lane {
+    gs_projected proj;   /* records of N Gaussians */
+    gs_bins bins;        /* pair list: max_pairs must hold every camera's K */
+    float *image;        /* [H][W][C] */
+    float *T_final;      /* [H][W] */
+    uint32_t *last;      /* [H][W] */
+    float *dL_dimage;    /* [H][W][C] */
+    float *grad2d;       /* [N][12], 16-byte aligned */
+    gs_param_set grads;  /* gradient slot, overwritten */
+    void *stream;        /* cudaStream_t the lane's cameras run on; may be the
+                            step's own stream (then no event is needed) */
+    void *done;          /* cudaEvent_t recorded on the lane's stream after its
+                            last camera (ignored when stream is the step's) */
+} gs_train_lane;
+
+/* One training step over n_cams cameras.  Camera b runs on lane
+ * b mod n_lanes, after the lane's previous camera: gs_project,
+ * gs_bin_and_sort (asynchronous), gs_render_fwd, the L1 loss of camera b's
+ * image against targets[b] (loss_b = mean |image - target| over H W C values),
+ * and gs_render_bwd, whose raw-parameter gradients are written (first camera
+ * of the lane) or added (the others) into the lane's slot.  Lanes run
+ * concurrently: each waits on `fork` (recorded on `stream` by the call) and
+ * `stream` waits on each lane's `done`.  Then, on `stream`, gs_adam_step
+ * with the lanes' slots and grad_scale = 1 / n_cams, i.e. the gradient of
+ * the mean of the cameras' losses.
+ *   cams      HOST array; all of one width, height and channel count (C = 3,
+ *             or 4 with GS_FLAG_DEPTH)
+ *   params    raw parameters, updated in place by Adam
+ *   targets   [n_cams][H][W][C]
+ *   lanes     HOST array of n_lanes (1..16) lanes with disjoint buffers
+ *   fork      cudaEvent_t (needed when a lane has its own stream)
+ *   cfg       Adam hyperparameters; NULL skips Adam (and `m`, `v`, `step`):
+ *             the step then only writes the mean gradient to grad_out,
+ *             e.g. for an all-reduce across GPUs before gs_adam_step
+ *   losses    nullable, DEVICE [n_cams] float: loss_b
+ *   cam_stats nullable, DEVICE [n_cams][2] int64: camera b's binning status
+ *             (GS_OK or GS_ERR_CAPACITY, the pair list then left empty and
+ *             the camera's image background only) and its pair count K
+ *   grad_out  nullable (required when cfg is NULL): the mean gradient
+ * Nothing synchronizes; read cam_stats to detect an overflowed pair list.
+ * The call may be captured in a CUDA graph (the lanes' streams join the
+ * capture through `fork`).  Errors: INVALID_ARG, TOO_LARGE, ALIGNMENT,
+ * CUDA. */
+int gs_train_step(const gs_camera *cams, int32_t n_cams, int64_t n, const gs_param_set *params,
+                  const float *targets, const gs_train_lane *lanes, int32_t n_lanes, void *fork,
+                  const gs_param_set *m, const gs_param_set *v, const gs_adam_config *cfg,
+                  int64_t *step, float *losses, int64_t *cam_stats, const gs_param_set *grad_out,
+                  void *stream);
 
 /* gs_bin_and_sort for callers that cannot allocate device memory.
  *

@@ -12,6 +12,7 @@ import torch
 
 import gaussian_splatting_differentiable_tile_b200 as G
 import oracle as O
+from oracle import train as OT
 from scenes import Camera, make_cameras, make_scene, make_target, tiny_camera
 
 from gpu_common import (IMG_TOL, MARGIN_CUT, MARGIN_RADIUS, MARGIN_TILE, ambiguous_gaussians, ambiguous_pixels,
@@ -415,12 +416,18 @@ def test_end_to_end_from_raw_parameters(flags):
     img = image.cpu().numpy()
     assert np.abs(img - ref["image"]).max(axis=2)[sel].max() <= IMG_TOL
     tgt = target.cpu().numpy().astype(np.float64)
-    assert abs(loss.item() - np.abs(img - tgt).mean()) <= 1e-5
-    # gradient of L1 with ambiguous pixels masked out
+    # the L1 gradient of each side from its own image; pixels whose sign of
+    # image - target the fp32 image could flip are masked out with the
+    # ambiguous ones
+    loss_ref, dl_ref = OT.l1_loss_grad(ref["image"], tgt)
+    assert abs(loss.item() - loss_ref) <= 1e-5
+    sel &= ~(np.abs(ref["image"] - tgt) <= IMG_TOL).any(axis=2)
+    dl_gpu = dl.cpu().numpy().astype(np.float64)
+    np.testing.assert_allclose(dl_gpu[sel], dl_ref[sel], rtol=1e-7, atol=0)
     dlm = torch.where(torch.from_numpy(sel[..., None]).cuda(), dl, torch.zeros_like(dl))
     grads = r.backward(cam, P, dlm)
     torch.cuda.synchronize()
-    g2_ref, g2_abs = O.render_bwd(p, cam, dlm.cpu().numpy().astype(np.float64))
+    g2_ref, g2_abs = O.render_bwd(p, cam, np.where(sel[..., None], dl_ref, 0.0))
     raw_ref = O.project_bwd(params, cam, g2_ref)
     bound = O.grad_bound(params, cam, g2_abs)
     for k in G.PARAM_KEYS:
