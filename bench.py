@@ -488,13 +488,15 @@ def run_native(args, spec, rank, world, local):
 
         t_steps = max(1, args.steps // B)
         _, tprof = timed(step_train, t_steps, args.warmup, profile=True)
-        g_train = graphed(step_train, len(groups))
+        # with several ranks the step all-reduces the gradient (data parallel)
+        # and runs eagerly: no NCCL call inside a captured graph
+        g_train = graphed(step_train, len(groups)) if world == 1 else step_train
         train_ms, _ = timed(g_train, t_steps, args.warmup)
         st = tr.cam_stats.cpu()
         if int(st[:, 0].abs().max()) != 0:
             raise RuntimeError(f"training step: pair list overflow {st.tolist()}")
         train = {"cameras_per_step": B, "lanes": args.lanes, "steps": t_steps, "ms": train_ms, "prof": tprof,
-                 "slots": min(args.lanes, B)}
+                 "slots": min(args.lanes, B) if world == 1 else 1}
     else:
         train_ms = 0.0
 
@@ -553,8 +555,11 @@ def run_native(args, spec, rank, world, local):
         B, t_steps = train["cameras_per_step"], train["steps"]
         train_out = {"frames_per_s": B * t_steps * world / (train_ms * 1e-3), "ms_per_step": train_ms / t_steps,
                      "cameras_per_step": B, "lanes": train["lanes"],
-                     "step": "gs_train_step: per camera project, bin, blend, L1, backward into the lane's "
-                             "gradient slot; Adam on the mean gradient; one CUDA graph per camera group"}
+                     "step": ("gs_train_step: per camera project, bin, blend, L1, backward into the lane's "
+                              "gradient slot; Adam on the mean gradient; one CUDA graph per camera group"
+                              if world == 1 else
+                              "data parallel: each rank's gs_train_step (no Adam) over its cameras, one NCCL "
+                              "all-reduce of the mean gradient, gs_adam_step; eager launches")}
         ad = (train["prof"] or {}).get("adam")
         if ad:
             launches, ms = ad

@@ -8,7 +8,7 @@ import math
 import torch
 
 from . import (GS_ERR_CAPACITY, PARAM_KEYS, Bins, GSError, Projected, TrainLane, adam_config, channels,
-               gs_bin_and_sort, gs_project, gs_render_bwd, gs_render_fwd, gs_train_step)
+               gs_adam_step, gs_bin_and_sort, gs_project, gs_render_bwd, gs_render_fwd, gs_train_step)
 
 
 class Rasterizer:
@@ -121,7 +121,9 @@ class Trainer:
         self.step_count = torch.zeros(1, dtype=torch.int64, device=device)
         self.fork = torch.cuda.Event()
         self.fork.record()
-        self.grads = {k: torch.empty(shapes[k], dtype=torch.float32, device=device) for k in PARAM_KEYS}
+        # the mean gradient, one flat buffer (one all-reduce across GPUs);
+        # each group starts on a 16-byte boundary
+        self.grads_flat, self.grads = _flat_views(shapes, device)
         self.losses = None
         self.cam_stats = None
 
@@ -145,19 +147,34 @@ class Trainer:
                 ln.regrow(int(math.ceil(need * 1.25)) + 1024)
         return need
 
-    def step(self, cams, params: dict, targets, check: bool = False, adam: bool = True, stream=None):
+    def step(self, cams, params: dict, targets, check: bool = False, adam: bool = True, stream=None,
+             group=None):
         """One step over the cameras (targets [B, H, W, C]); updates params in
         place (adam=True) and returns the per-camera losses (a device tensor).
         self.grads receives the mean gradient.  check=True synchronizes and
         raises GSError(GS_ERR_CAPACITY) if a camera overflowed its pair list
-        (its image was then background only; Adam has already run)."""
+        (its image was then background only; Adam has already run).
+
+        With a torch.distributed process group of several ranks (data
+        parallel: every rank its own B cameras, the same parameters), the
+        ranks' mean gradients are summed by one all-reduce and Adam applies
+        their mean, so every rank takes the same step."""
         B = len(cams)
         if self.losses is None or self.losses.numel() != B:
             self.losses = torch.zeros(B, dtype=torch.float32, device=self.device)
             self.cam_stats = torch.zeros((B, 2), dtype=torch.int64, device=self.device)
-        gs_train_step(cams, params, targets, self.lanes, self.fork, self.m if adam else None,
-                      self.v if adam else None, self.cfg if adam else None, self.step_count if adam else None,
-                      self.losses, self.cam_stats, self.grads, stream)
+        world = _world(group)
+        if world > 1 and adam:
+            data_parallel_step(
+                lambda: gs_train_step(cams, params, targets, self.lanes, self.fork, None, None, None, None,
+                                      self.losses, self.cam_stats, self.grads, stream),
+                lambda scale: gs_adam_step(params, [self.grads], self.m, self.v, self.cfg, self.step_count,
+                                           grad_scale=scale, stream=stream),
+                self.grads_flat, group)
+        else:
+            gs_train_step(cams, params, targets, self.lanes, self.fork, self.m if adam else None,
+                          self.v if adam else None, self.cfg if adam else None,
+                          self.step_count if adam else None, self.losses, self.cam_stats, self.grads, stream)
         if check:
             st = self.cam_stats.cpu()
             bad = [b for b in range(B) if int(st[b, 0]) != 0]
@@ -166,3 +183,32 @@ class Trainer:
                 err.n_pairs = int(st[:, 1].max())
                 raise err
         return self.losses
+
+
+def _flat_views(shapes: dict, device):
+    """One float32 buffer holding an array per group, each starting on a
+    16-byte boundary; returns (buffer, {group: view})."""
+    offs, off = {}, 0
+    for k in PARAM_KEYS:
+        offs[k] = off
+        off += (math.prod(shapes[k]) + 3) // 4 * 4
+    flat = torch.zeros(max(off, 4), dtype=torch.float32, device=device)
+    return flat, {k: flat[offs[k]:offs[k] + math.prod(shapes[k])].view(shapes[k]) for k in PARAM_KEYS}
+
+
+def _world(group) -> int:
+    import torch.distributed as dist
+    if not dist.is_available() or not dist.is_initialized():
+        return 1
+    return dist.get_world_size(group)
+
+
+def data_parallel_step(local_step, adam_step, grads_flat, group=None) -> None:
+    """Data-parallel training step: local_step() writes this rank's mean
+    gradient into grads_flat; one all-reduce sums the ranks' gradients; then
+    adam_step(1 / world) applies their mean.  Every rank makes the same
+    collective call in the same order."""
+    import torch.distributed as dist
+    local_step()
+    dist.all_reduce(grads_flat, op=dist.ReduceOp.SUM, group=group)
+    adam_step(1.0 / dist.get_world_size(group))
