@@ -454,9 +454,11 @@ k_render_bwd(CamConst cam, const float4 *__restrict__ xyod, const float4 *__rest
             }
             if (!__any_sync(0xffffffffu, any)) continue;
             // Contributions, branch-free (measured faster than skipping per
-            // row): a skipped row has alpha 0, which zeroes w, v and every
-            // sum exactly (colours of drawn Gaussians are finite); T is kept
-            // by a select.
+            // row, and than skipping the cap for entries that cannot reach
+            // it): a skipped row has alpha 0, which zeroes w, v and every sum
+            // exactly (colours of drawn Gaussians are finite) and leaves T as
+            // it is (T / (1 - 0) with the approximate reciprocal of 1, which
+            // is exact).
             const float4 c = s_col[k];
             float2 sv = make_float2(0.f, 0.f), sgy = sv, sgyy = sv, cr0 = sv, cr1 = sv, cr2 = sv, cr3 = sv;
 #pragma unroll
@@ -486,8 +488,7 @@ k_render_bwd(CamConst cam, const float4 *__restrict__ xyod, const float4 *__rest
                 const float2 vy = __fmul2_rn(v, dy[i]);
                 sgy = __fadd2_rn(sgy, vy);
                 sgyy = __ffma2_rn(vy, dy[i], sgyy);
-                T[i].x = h0 ? Ti.x : T[i].x;
-                T[i].y = h1 ? Ti.y : T[i].y;
+                T[i] = Ti;  // a skipped row: alpha 0, rcp.approx(1) = 1 exactly, so Ti = T
             }
             const float svs = sv.x + sv.y, sgys = sgy.x + sgy.y;
             const float sgx = svs * ct.dx;
