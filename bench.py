@@ -500,7 +500,37 @@ def run_native(args, spec, rank, world, local):
     else:
         train_ms = 0.0
 
-    full_ms, fwd_ms, e2e_ms, train_ms = max_over_ranks([full_ms, fwd_ms, e2e_ms, train_ms], world, dev)
+    # feature channels: F per-Gaussian values blended with the forward's
+    # weights and their backward, per frame after that camera's forward
+    feat = None
+    if args.features > 0:
+        F = args.features
+        fts = torch.from_numpy(np.random.default_rng(5).uniform(-1, 1, (n, F)).astype(np.float32)).to(dev)
+        fout = torch.empty((H, W, F), device=dev)
+        fdl = torch.from_numpy(np.random.default_rng(6).normal(size=(H, W, F)).astype(np.float32) / (H * W * F)).to(dev)
+        dfts = torch.empty_like(fts)
+        f_fwd = f_bwd = 0.0
+        f_steps = max(1, args.steps // 4)
+        for i in range(args.warmup + f_steps):
+            step_full(i)
+            c = ccams[i % len(ccams)]
+            e0, e1, e2 = (torch.cuda.Event(enable_timing=True) for _ in range(3))
+            flush.zero_()
+            e0.record()
+            G.gs_render_features_fwd(c, n, proj, bins, fts, fout)
+            e1.record()
+            G.gs_render_features_bwd(c, n, P, proj, bins, T, last, fts, fdl, grad2d, dfts, grads)
+            e2.record()
+            torch.cuda.synchronize()
+            if i >= args.warmup:
+                f_fwd += e0.elapsed_time(e1)
+                f_bwd += e1.elapsed_time(e2)
+        feat = {"F": F, "frames": f_steps, "fwd_ms": f_fwd, "bwd_ms": f_bwd}
+    feat_fwd_ms = feat["fwd_ms"] if feat else 0.0
+    feat_bwd_ms = feat["bwd_ms"] if feat else 0.0
+
+    full_ms, fwd_ms, e2e_ms, train_ms, feat_fwd_ms, feat_bwd_ms = max_over_ranks(
+        [full_ms, fwd_ms, e2e_ms, train_ms, feat_fwd_ms, feat_bwd_ms], world, dev)
     frames = args.steps * world
     if rank != 0:
         return
@@ -570,6 +600,13 @@ def run_native(args, spec, rank, world, local):
             train_out["adam"] = {"ms_per_step": ms / t_steps, "kernels_per_step": kernels_per_step,
                                  "bound": "hbm", "achieved": ach, "peak": hbm_peak, "unit": "GB/s",
                                  "frac": ach / hbm_peak, "bytes_per_step": abytes}
+    feat_out = None
+    if feat is not None:
+        fr = feat["frames"]
+        feat_out = {"channels": feat["F"], "fwd_ms_per_frame": feat_fwd_ms / fr, "bwd_ms_per_frame": feat_bwd_ms / fr,
+                    "fwd_bwd_frames_per_s": fr * world / ((feat_fwd_ms + feat_bwd_ms) * 1e-3),
+                    "passes": f"{feat['F'] // 4} blend passes of four channels each way (forward weights recomputed, "
+                              "no background); backward adds into the frame's raw-parameter gradients"}
     out = {
         "metric": METRIC,
         "value": frames / (full_ms * 1e-3),
@@ -597,6 +634,7 @@ def run_native(args, spec, rank, world, local):
         "gpu_launches": gpu_launches,
         "clocks": clocks,
         "train_step": train_out,
+        "features": feat_out,
     }
     print(json.dumps(out), flush=True)
 
@@ -614,6 +652,8 @@ def main():
     ap.add_argument("--train-cams", type=int, default=4,
                     help="cameras per batched training step (0: do not measure the training step)")
     ap.add_argument("--lanes", type=int, default=4, help="concurrent camera chains of the training step")
+    ap.add_argument("--features", type=int, default=8,
+                    help="feature channels per Gaussian to time (a multiple of 4; 0: skip)")
     ap.add_argument("--no-graphs", action="store_true", help="launch every kernel eagerly")
     ap.add_argument("--tiles", choices=("cut", "3sigma"), default="cut",
                     help="tile rectangles: 3-sigma narrowed by the opacity-aware cut, or plain 3-sigma")

@@ -31,7 +31,7 @@ from ._abi import (GS_ERR_ALIGNMENT, GS_ERR_CAPACITY, GS_ERR_CUDA, GS_ERR_DEVICE
 
 __all__ = [
     "GSError", "Projected", "Bins", "make_camera", "channels", "gs_project", "gs_bin_and_sort",
-    "gs_bin_and_sort_static", "gs_render_fwd",
+    "gs_bin_and_sort_static", "gs_render_fwd", "gs_render_features_fwd", "gs_render_features_bwd",
     "gs_render_bwd", "gs_render_stats", "gs_l1_loss_grad", "gs_read_status", "gs_error_string", "profile_begin",
     "profile_end", "lib", "PARAM_KEYS",
 ]
@@ -225,6 +225,41 @@ def gs_render_bwd(cam, n: int, params: dict, proj: Projected, bins: Bins, T_fina
                                _dev(last, "last", torch.int32), _dev(dL_dimage, "dL_dimage", torch.float32),
                                _dev(grad2d, "grad2d", torch.float32), ctypes.byref(g), _stream(stream)),
            "gs_render_bwd")
+
+
+def gs_render_features_fwd(cam, n: int, proj: Projected, bins: Bins, features: torch.Tensor, out: torch.Tensor,
+                           stream=None) -> None:
+    """Blends features [N, F] (F a multiple of 4) with the forward's weights
+    into out [H, W, F] (no background)."""
+    F = int(features.shape[-1]) if features.dim() == 2 else -1
+    if F < 0 or out.numel() != int(cam.height) * int(cam.width) * F:
+        raise ValueError("features must be [N, F] and out [H, W, F]")
+    c = make_camera(cam)
+    _check(lib().gs_render_features_fwd(ctypes.byref(c), int(n), ctypes.byref(proj.struct), ctypes.byref(bins.struct),
+                                        _dev(features, "features", torch.float32), F,
+                                        _dev(out, "out", torch.float32), _stream(stream)), "gs_render_features_fwd")
+
+
+def gs_render_features_bwd(cam, n: int, params: dict, proj: Projected, bins: Bins, T_final: torch.Tensor,
+                           last: torch.Tensor, features: torch.Tensor, dL_dout: torch.Tensor, grad2d: torch.Tensor,
+                           dL_dfeatures: torch.Tensor, grads: dict, stream=None) -> None:
+    """dL/dfeatures (overwritten) and the features' share of the raw-parameter
+    gradients, added into grads (call after gs_render_bwd)."""
+    F = int(features.shape[-1]) if features.dim() == 2 else -1
+    if F < 0 or dL_dout.numel() != int(cam.height) * int(cam.width) * F or dL_dfeatures.shape != features.shape:
+        raise ValueError("features [N, F], dL_dout [H, W, F], dL_dfeatures [N, F]")
+    if grad2d.numel() < 12 * int(n):
+        raise ValueError("grad2d must hold [N,12] floats")
+    c = make_camera(cam)
+    p = _params_struct(params)
+    g = _params_struct(grads, _abi.GsGrads)
+    _check(lib().gs_render_features_bwd(ctypes.byref(c), int(n), ctypes.byref(p), ctypes.byref(proj.struct),
+                                        ctypes.byref(bins.struct), _dev(T_final, "T_final", torch.float32),
+                                        _dev(last, "last", torch.int32), _dev(features, "features", torch.float32),
+                                        F, _dev(dL_dout, "dL_dout", torch.float32),
+                                        _dev(grad2d, "grad2d", torch.float32),
+                                        _dev(dL_dfeatures, "dL_dfeatures", torch.float32), ctypes.byref(g),
+                                        _stream(stream)), "gs_render_features_bwd")
 
 
 def gs_render_stats(cam, n: int, proj: Projected, bins: Bins, last: torch.Tensor, stream=None) -> dict:

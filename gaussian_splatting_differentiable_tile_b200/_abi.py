@@ -108,6 +108,14 @@ PROTOTYPES = {
                                      ctypes.POINTER(GsProjected), ctypes.POINTER(GsBins), ctypes.c_void_p,
                                      ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p,
                                      ctypes.POINTER(GsGrads), ctypes.c_void_p]),
+    "gs_render_features_fwd": (ctypes.c_int, [ctypes.POINTER(GsCamera), ctypes.c_int64, ctypes.POINTER(GsProjected),
+                                              ctypes.POINTER(GsBins), ctypes.c_void_p, ctypes.c_int32, ctypes.c_void_p,
+                                              ctypes.c_void_p]),
+    "gs_render_features_bwd": (ctypes.c_int, [ctypes.POINTER(GsCamera), ctypes.c_int64, ctypes.POINTER(GsParams),
+                                              ctypes.POINTER(GsProjected), ctypes.POINTER(GsBins), ctypes.c_void_p,
+                                              ctypes.c_void_p, ctypes.c_void_p, ctypes.c_int32, ctypes.c_void_p,
+                                              ctypes.c_void_p, ctypes.c_void_p, ctypes.POINTER(GsGrads),
+                                              ctypes.c_void_p]),
     "gs_render_stats": (ctypes.c_int, [ctypes.POINTER(GsCamera), ctypes.c_int64, ctypes.POINTER(GsProjected),
                                        ctypes.POINTER(GsBins), ctypes.c_void_p, ctypes.c_void_p,
                                        ctypes.c_void_p]),

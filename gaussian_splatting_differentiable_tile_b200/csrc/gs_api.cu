@@ -288,6 +288,57 @@ int gs_render_bwd(const gs_camera *cam, int64_t n, const gs_params *params,
     return GS_OK;
 }
 
+namespace {
+constexpr int32_t kMaxFeatures = 1024;
+}
+
+int gs_render_features_fwd(const gs_camera *cam, int64_t n, const gs_projected *proj, const gs_bins *bins,
+                           const float *features, int32_t F, float *out, void *stream) {
+    CamConst c;
+    int rc = make_cam(cam, &c);
+    if (rc) return rc;
+    if (n < 0 || F < 4 || F > kMaxFeatures || F % 4 != 0 || !out || (n > 0 && !features))
+        return GS_ERR_INVALID_ARG;
+    BinsLayout L;
+    if ((rc = check_projected(proj, n)) || (rc = check_bins(bins, n, c, &L))) return rc;
+    if (!aligned(features, 16) || !aligned(out, 4)) return GS_ERR_ALIGNMENT;
+    return launch_render_features_fwd(c, *proj, *bins, features, F, out, as_stream(stream)) == cudaSuccess
+               ? GS_OK
+               : GS_ERR_CUDA;
+}
+
+int gs_render_features_bwd(const gs_camera *cam, int64_t n, const gs_params *params, const gs_projected *proj,
+                           const gs_bins *bins, const float *T_final, const uint32_t *last,
+                           const float *features, int32_t F, const float *dL_dout, float *grad2d,
+                           float *dL_dfeatures, const gs_grads *grads, void *stream) {
+    CamConst c;
+    int rc = make_cam(cam, &c);
+    if (rc) return rc;
+    if (n < 0 || F < 4 || F > kMaxFeatures || F % 4 != 0) return GS_ERR_INVALID_ARG;
+    BinsLayout L;
+    if ((rc = check_params(params, n)) || (rc = check_projected(proj, n)) ||
+        (rc = check_bins(bins, n, c, &L)))
+        return rc;
+    if (!T_final || !last || !dL_dout || !grads) return GS_ERR_INVALID_ARG;
+    if (n > 0 && (!features || !grad2d || !dL_dfeatures || !grads->means || !grads->log_scales ||
+                  !grads->quats || !grads->opacity_logits || !grads->colors))
+        return GS_ERR_INVALID_ARG;
+    if (!aligned(features, 16) || !aligned(grad2d, 16) || !aligned(grads->quats, 16) || !aligned(T_final, 4) ||
+        !aligned(last, 4) || !aligned(dL_dout, 4) || !aligned(dL_dfeatures, 4))
+        return GS_ERR_ALIGNMENT;
+    if (n == 0) return GS_OK;
+    cudaStream_t s = as_stream(stream);
+    if (cudaMemsetAsync(grad2d, 0, (size_t)n * 12 * sizeof(float), s) != cudaSuccess ||
+        cudaMemsetAsync(dL_dfeatures, 0, (size_t)n * F * sizeof(float), s) != cudaSuccess)
+        return GS_ERR_CUDA;
+    if (launch_render_features_bwd(c, *proj, *bins, T_final, last, features, F, dL_dout, grad2d, dL_dfeatures,
+                                   s) != cudaSuccess)
+        return GS_ERR_CUDA;
+    // the features' share of dL/d(mean2d, conic, opacity), added into grads
+    if (launch_project_bwd(c, n, *params, *proj, grad2d, *grads, s, true) != cudaSuccess) return GS_ERR_CUDA;
+    return GS_OK;
+}
+
 int gs_render_stats(const gs_camera *cam, int64_t n, const gs_projected *proj, const gs_bins *bins,
                     const uint32_t *last, uint64_t *counts, void *stream) {
     CamConst c;

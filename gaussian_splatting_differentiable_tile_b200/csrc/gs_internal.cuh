@@ -134,6 +134,15 @@ cudaError_t launch_render_fwd(const CamConst &c, const gs_projected &proj, const
 cudaError_t launch_render_bwd(const CamConst &c, const gs_projected &proj, const gs_bins &bins,
                               const float *T_final, const uint32_t *last, const float *dL_dimage,
                               float *grad2d, cudaStream_t s);
+// Feature channels: F / 4 passes of the blend over chunks of four channels
+// (no background).  The backward adds the geometric sums into grad2d and
+// the feature gradients into dL_dfeatures (both zeroed by the caller).
+cudaError_t launch_render_features_fwd(const CamConst &c, const gs_projected &proj, const gs_bins &bins,
+                                       const float *features, int F, float *out, cudaStream_t s);
+cudaError_t launch_render_features_bwd(const CamConst &c, const gs_projected &proj, const gs_bins &bins,
+                                       const float *T_final, const uint32_t *last, const float *features,
+                                       int F, const float *dL_dout, float *grad2d, float *dL_dfeatures,
+                                       cudaStream_t s);
 cudaError_t launch_render_stats(const CamConst &c, const gs_projected &proj, const gs_bins &bins,
                                 const uint32_t *last, uint64_t *counts, cudaStream_t s);
 cudaError_t launch_l1(const float *image, const float *target, int64_t count, float *dL_dimage,

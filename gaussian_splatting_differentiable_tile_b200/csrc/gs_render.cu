@@ -86,6 +86,17 @@ __device__ __forceinline__ void stage_entry(const float4 xyod, const float4 conr
     geo2 = make_float4(cC, log2f(xyod.z), kx, ky);
 }
 
+// Where a blend kernel reads its per-Gaussian channel values and writes its
+// per-pixel and per-Gaussian channel outputs: the records' colours, or a
+// chunk of four feature channels.
+struct ChannelIO {
+    const float4 *col;  // channel values of Gaussian g at col[g * col_stride]
+    int col_stride;     // in float4s
+    int img_stride;     // floats per pixel of the image (forward) or dL/dimage (backward)
+    float *cgrad;       // backward: the channel-gradient sums of Gaussian g at cgrad[g * cgrad_stride]
+    int cgrad_stride;   // in floats
+};
+
 // Geometry of a lane: its column centre and first row's centre; and the
 // tile's strips (2 RPL rows each): x centre and half width, y centre of the
 // first strip, half height.
@@ -185,10 +196,10 @@ __device__ __forceinline__ bool eval_alpha(const float4 geo, const float4 geo2, 
 // slots whose bit it holds, in order, and walks only those.  A culled slot
 // could not have passed the alpha test at any pixel of the strip, so the
 // sequence of contributions, the stopping entry and `last` are unchanged.
-template <bool kDepth>
+template <bool kDepth, bool kFeat = false>
 __global__ void __launch_bounds__(kTilePixels, 6)
 k_render_fwd(CamConst cam, const float4 *__restrict__ xyod, const float4 *__restrict__ conr,
-             const float4 *__restrict__ rgb, const uint32_t *__restrict__ pair_gid,
+             const ChannelIO io, const uint32_t *__restrict__ pair_gid,
              const uint2 *__restrict__ ranges, const uint32_t *__restrict__ order,
              float *__restrict__ image, float *__restrict__ T_final, uint32_t *__restrict__ last) {
     constexpr int kWarps = kTilePixels / 32;
@@ -215,7 +226,7 @@ k_render_fwd(CamConst cam, const float4 *__restrict__ xyod, const float4 *__rest
             stage_entry(xyod[g], conr[g], geo, geo2);
             s_geo[threadIdx.x] = geo;
             s_geo2[threadIdx.x] = geo2;
-            s_col[threadIdx.x] = rgb[g];
+            s_col[threadIdx.x] = io.col[kFeat ? (size_t)g * io.col_stride : (size_t)g];
             const uint32_t m = strip_mask<kWarps>(geo, geo2, L.sx, L.hx, L.sy0, 2.f, L.hy);
             s_mask[threadIdx.x] = (uint8_t)m;
         }
@@ -247,13 +258,13 @@ k_render_fwd(CamConst cam, const float4 *__restrict__ xyod, const float4 *__rest
     }
     if (L.px < cam.width && L.py0 < cam.height) {
         const size_t p = (size_t)L.py0 * cam.width + L.px;
-        constexpr int kC = kDepth ? 4 : 3;
-        image[kC * p] = __fmaf_rn(T, cam.bg[0], C0);
-        image[kC * p + 1] = __fmaf_rn(T, cam.bg[1], C1);
-        image[kC * p + 2] = __fmaf_rn(T, cam.bg[2], C2);
-        if (kDepth) image[kC * p + 3] = C3;  // the depth channel has no background
-        T_final[p] = T;
-        last[p] = lst;
+        float *px = image + (size_t)(kFeat ? io.img_stride : (kDepth ? 4 : 3)) * p;
+        px[0] = __fmaf_rn(T, cam.bg[0], C0);
+        px[1] = __fmaf_rn(T, cam.bg[1], C1);
+        px[2] = __fmaf_rn(T, cam.bg[2], C2);
+        if (kDepth) px[3] = C3;  // the fourth channel has no background
+        if (T_final) T_final[p] = T;
+        if (last) last[p] = lst;
     }
 }
 
@@ -331,10 +342,10 @@ __device__ __forceinline__ float reduce_scatter(const float (&v)[N], int lane, i
 // with v = alpha dL/dalpha (0 when alpha was capped), w = alpha T_i; they are
 // added into grad2d, and k_project_bwd maps them to dL/d(mean2d, conic,
 // opacity) with the Gaussian's own A, B, C, o.
-template <int kRPL, bool kDepth>
+template <int kRPL, bool kDepth, bool kFeat = false>
 __global__ void __launch_bounds__(kTilePixels / kRPL, 56 / kRPL)
 k_render_bwd(CamConst cam, const float4 *__restrict__ xyod, const float4 *__restrict__ conr,
-             const float4 *__restrict__ rgb, const uint32_t *__restrict__ pair_gid,
+             const ChannelIO io, const uint32_t *__restrict__ pair_gid,
              const uint2 *__restrict__ ranges, const uint32_t *__restrict__ order,
              const float *__restrict__ T_final,
              const uint32_t *__restrict__ last, const float *__restrict__ dL_dimage,
@@ -372,10 +383,11 @@ k_render_bwd(CamConst cam, const float4 *__restrict__ xyod, const float4 *__rest
             const size_t p = (size_t)py * cam.width + L.px;
             t = T_final[p];
             lst[r] = min(max(last[p], range.x), range.y);  // never walk outside the tile's list
-            d0 = dL_dimage[kC * p];
-            d1 = dL_dimage[kC * p + 1];
-            d2 = dL_dimage[kC * p + 2];
-            if (kDepth) d3 = dL_dimage[kC * p + 3];
+            const float *dp = dL_dimage + (size_t)(kFeat ? io.img_stride : kC) * p;
+            d0 = dp[0];
+            d1 = dp[1];
+            d2 = dp[2];
+            if (kDepth) d3 = dp[3];
         }
         const float s0 = t * (cam.bg[0] * d0 + cam.bg[1] * d1 + cam.bg[2] * d2);  // depth: no background
         const float nf = -(L.fy0 + (float)r);
@@ -408,8 +420,8 @@ k_render_bwd(CamConst cam, const float4 *__restrict__ xyod, const float4 *__rest
             const uint32_t i1 = i0 + kThreads;
             const uint32_t ga = pair_gid[bend - 1 - i0];
             const uint32_t gb = i1 < cnt ? pair_gid[bend - 1 - i1] : ga;
-            const float4 xa = xyod[ga], ca = conr[ga], ra = rgb[ga];
-            const float4 xb = xyod[gb], cb = conr[gb], rb = rgb[gb];
+            const float4 xa = xyod[ga], ca = conr[ga], ra = io.col[kFeat ? (size_t)ga * io.col_stride : (size_t)ga];
+            const float4 xb = xyod[gb], cb = conr[gb], rb = io.col[kFeat ? (size_t)gb * io.col_stride : (size_t)gb];
             float4 geo, geo2;
             stage_entry(xa, ca, geo, geo2);
             s_geo[i0] = geo;
@@ -504,7 +516,13 @@ k_render_bwd(CamConst cam, const float4 *__restrict__ xyod, const float4 *__rest
                                        cr0.x + cr0.y, cr1.x + cr1.y, cr2.x + cr2.y};
                 tot = reduce_scatter<9>(vals, lane, &idx);
             }
-            if (idx < kV) atomicAdd(grad2d + 12 * (size_t)s_gid[k] + idx, tot);
+            // the six geometric sums into grad2d; the channel sums follow them
+            // in grad2d (colours), or go to io.cgrad (a feature chunk)
+            if (idx < kV) {
+                float *dst = grad2d + 12 * (size_t)s_gid[k] + idx;
+                if (kFeat && idx >= 6) dst = io.cgrad + (size_t)io.cgrad_stride * s_gid[k] + (idx - 6);
+                atomicAdd(dst, tot);
+            }
         }
         __syncthreads();
         bend = bstart;
@@ -606,20 +624,37 @@ static const uint32_t *tile_order(const gs_bins &bins) {
 cudaError_t launch_render_fwd(const CamConst &c, const gs_projected &proj, const gs_bins &bins,
                               float *image, float *T_final, uint32_t *last, cudaStream_t s) {
     const int tiles = c.tiles_x * c.tiles_y;
+    const bool depth = c.flags & GS_FLAG_DEPTH;
+    const ChannelIO io{reinterpret_cast<const float4 *>(proj.rgb), 1, depth ? 4 : 3, nullptr, 0};
     prof_before("render_fwd", s);
-    if (c.flags & GS_FLAG_DEPTH)
+    if (depth)
         k_render_fwd<true><<<tiles, kTilePixels, 0, s>>>(
-        c, reinterpret_cast<const float4 *>(proj.xy_opacity_depth),
-        reinterpret_cast<const float4 *>(proj.conic_radius), reinterpret_cast<const float4 *>(proj.rgb),
-        bins.pair_gid, reinterpret_cast<const uint2 *>(bins.ranges), tile_order(bins), image, T_final,
-        last);
+            c, reinterpret_cast<const float4 *>(proj.xy_opacity_depth),
+            reinterpret_cast<const float4 *>(proj.conic_radius), io, bins.pair_gid,
+            reinterpret_cast<const uint2 *>(bins.ranges), tile_order(bins), image, T_final, last);
     else
         k_render_fwd<false><<<tiles, kTilePixels, 0, s>>>(
-        c, reinterpret_cast<const float4 *>(proj.xy_opacity_depth),
-        reinterpret_cast<const float4 *>(proj.conic_radius), reinterpret_cast<const float4 *>(proj.rgb),
-        bins.pair_gid, reinterpret_cast<const uint2 *>(bins.ranges), tile_order(bins), image, T_final,
-        last);
+            c, reinterpret_cast<const float4 *>(proj.xy_opacity_depth),
+            reinterpret_cast<const float4 *>(proj.conic_radius), io, bins.pair_gid,
+            reinterpret_cast<const uint2 *>(bins.ranges), tile_order(bins), image, T_final, last);
     prof_after(s);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_render_features_fwd(const CamConst &c, const gs_projected &proj, const gs_bins &bins,
+                                       const float *features, int F, float *out, cudaStream_t s) {
+    const int tiles = c.tiles_x * c.tiles_y;
+    CamConst cf = c;  // features blend without a background
+    cf.bg[0] = cf.bg[1] = cf.bg[2] = 0.f;
+    prof_before("render_features_fwd", s);
+    for (int k = 0; k < F / 4; k++) {
+        const ChannelIO io{reinterpret_cast<const float4 *>(features) + k, F / 4, F, nullptr, 0};
+        k_render_fwd<true, true><<<tiles, kTilePixels, 0, s>>>(
+            cf, reinterpret_cast<const float4 *>(proj.xy_opacity_depth),
+            reinterpret_cast<const float4 *>(proj.conic_radius), io, bins.pair_gid,
+            reinterpret_cast<const uint2 *>(bins.ranges), tile_order(bins), out + 4 * k, nullptr, nullptr);
+    }
+    prof_after(s, F / 4);
     return cudaGetLastError();
 }
 
@@ -627,20 +662,40 @@ cudaError_t launch_render_bwd(const CamConst &c, const gs_projected &proj, const
                               const float *T_final, const uint32_t *last, const float *dL_dimage,
                               float *grad2d, cudaStream_t s) {
     const int tiles = c.tiles_x * c.tiles_y;
+    const bool depth = c.flags & GS_FLAG_DEPTH;
+    const ChannelIO io{reinterpret_cast<const float4 *>(proj.rgb), 1, depth ? 4 : 3, grad2d + 6, 12};
     prof_before("render_bwd", s);
-    if (c.flags & GS_FLAG_DEPTH)
+    if (depth)
         k_render_bwd<GS_BWD_RPL, true><<<tiles, kTilePixels / GS_BWD_RPL, 0, s>>>(
-        c, reinterpret_cast<const float4 *>(proj.xy_opacity_depth),
-        reinterpret_cast<const float4 *>(proj.conic_radius), reinterpret_cast<const float4 *>(proj.rgb),
-        bins.pair_gid, reinterpret_cast<const uint2 *>(bins.ranges), tile_order(bins), T_final, last,
-        dL_dimage, grad2d);
+            c, reinterpret_cast<const float4 *>(proj.xy_opacity_depth),
+            reinterpret_cast<const float4 *>(proj.conic_radius), io, bins.pair_gid,
+            reinterpret_cast<const uint2 *>(bins.ranges), tile_order(bins), T_final, last, dL_dimage, grad2d);
     else
         k_render_bwd<GS_BWD_RPL, false><<<tiles, kTilePixels / GS_BWD_RPL, 0, s>>>(
-        c, reinterpret_cast<const float4 *>(proj.xy_opacity_depth),
-        reinterpret_cast<const float4 *>(proj.conic_radius), reinterpret_cast<const float4 *>(proj.rgb),
-        bins.pair_gid, reinterpret_cast<const uint2 *>(bins.ranges), tile_order(bins), T_final, last,
-        dL_dimage, grad2d);
+            c, reinterpret_cast<const float4 *>(proj.xy_opacity_depth),
+            reinterpret_cast<const float4 *>(proj.conic_radius), io, bins.pair_gid,
+            reinterpret_cast<const uint2 *>(bins.ranges), tile_order(bins), T_final, last, dL_dimage, grad2d);
     prof_after(s);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_render_features_bwd(const CamConst &c, const gs_projected &proj, const gs_bins &bins,
+                                       const float *T_final, const uint32_t *last, const float *features,
+                                       int F, const float *dL_dout, float *grad2d, float *dL_dfeatures,
+                                       cudaStream_t s) {
+    const int tiles = c.tiles_x * c.tiles_y;
+    CamConst cf = c;  // features blend without a background
+    cf.bg[0] = cf.bg[1] = cf.bg[2] = 0.f;
+    prof_before("render_features_bwd", s);
+    for (int k = 0; k < F / 4; k++) {
+        const ChannelIO io{reinterpret_cast<const float4 *>(features) + k, F / 4, F, dL_dfeatures + 4 * k, F};
+        k_render_bwd<GS_BWD_RPL, true, true><<<tiles, kTilePixels / GS_BWD_RPL, 0, s>>>(
+            cf, reinterpret_cast<const float4 *>(proj.xy_opacity_depth),
+            reinterpret_cast<const float4 *>(proj.conic_radius), io, bins.pair_gid,
+            reinterpret_cast<const uint2 *>(bins.ranges), tile_order(bins), T_final, last, dL_dout + 4 * k,
+            grad2d);
+    }
+    prof_after(s, F / 4);
     return cudaGetLastError();
 }
 

@@ -264,6 +264,37 @@ int gs_render_bwd(const gs_camera *cam, int64_t n, const gs_params *params,
                   const uint32_t *last, const float *dL_dimage, float *grad2d,
                   const gs_grads *grads, void *stream);
 
+/* Feature channels ([GSP] s5: the final weighted sum costs the same for
+ * channels of any kind, RGB, depth or features).  Each Gaussian carries F
+ * feature values; the forward's weights w_i = alpha_i T_i blend them with
+ * no background: out[p][f] = sum_i w_i features[g_i][f].  The walk is the
+ * forward's (same tests, same stop, same rounding), run once per chunk of
+ * four channels.
+ *   features [N][F]  F a positive multiple of 4 (at most 1024), 16-byte aligned
+ *   out      [H][W][F], overwritten
+ * `proj` and `bins` must be those gs_render_fwd used for this camera.
+ * Errors: INVALID_ARG, ALIGNMENT, CUDA. */
+int gs_render_features_fwd(const gs_camera *cam, int64_t n, const gs_projected *proj,
+                           const gs_bins *bins, const float *features, int32_t F, float *out,
+                           void *stream);
+
+/* Backward of the feature channels: dL/dfeatures, and the features' share
+ * of the blend gradient (through alpha: dL/dalpha_i = T_i <f_i - R_i, g>,
+ * the colours' formula with the features' dL/dout as g and no background)
+ * mapped to the raw parameters and ADDED into grads.  Call it after
+ * gs_render_bwd (which overwrites grads with the colours' share).
+ *   dL_dout      [H][W][F]  gradient of the loss with respect to out
+ *   grad2d       [N][12]    caller scratch, 16-byte aligned
+ *   dL_dfeatures [N][F]     overwritten
+ *   grads                   raw-parameter gradients, accumulated into
+ * T_final and last must be gs_render_fwd's for the same proj and bins.
+ * Errors: INVALID_ARG, ALIGNMENT, CUDA. */
+int gs_render_features_bwd(const gs_camera *cam, int64_t n, const gs_params *params,
+                           const gs_projected *proj, const gs_bins *bins, const float *T_final,
+                           const uint32_t *last, const float *features, int32_t F,
+                           const float *dL_dout, float *grad2d, float *dL_dfeatures,
+                           const gs_grads *grads, void *stream);
+
 /* Work counts of one forward frame, for roofline arithmetic (not part of the
  * rendering path; it re-walks the blend with counters and is slower).
  * counts (device, [4] uint64, overwritten):

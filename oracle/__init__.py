@@ -6,3 +6,4 @@ library and its Python binding never import it, and it never imports them.
 """
 from .oracle import *  # noqa: F401,F403
 from . import train  # noqa: F401
+from . import features  # noqa: F401,E402
