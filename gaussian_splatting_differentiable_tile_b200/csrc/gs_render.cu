@@ -44,6 +44,14 @@
 #ifndef GS_BWD_RPL
 #define GS_BWD_RPL 4
 #endif
+// Backward: entries staged per round (at most 128) and resident CTAs per SM
+// the register allocation targets (tuning knobs; defaults measured fastest).
+#ifndef GS_BWD_BATCH
+#define GS_BWD_BATCH 128
+#endif
+#ifndef GS_BWD_MINB
+#define GS_BWD_MINB (56 / GS_BWD_RPL)
+#endif
 
 namespace gs {
 namespace {
@@ -55,7 +63,7 @@ constexpr float kCullLog2 = -7.994353436858858f - 0.0145f;
 // exponent, log2(o exp(-sigma)) >= this, before the exponential.
 constexpr float kLog2AlphaMin = -7.994353436858858f;
 constexpr int kBatch = 256;     // forward batch (entries staged per round)
-constexpr int kBwdBatch = 128;  // backward batch: less shared memory, more CTAs per SM
+constexpr int kBwdBatch = GS_BWD_BATCH;  // backward batch: less shared memory, more CTAs per SM
 
 // PTX ex2.approx / rcp.approx (MUFU instructions).
 __device__ __forceinline__ float ex2_approx(float x) {
@@ -343,7 +351,7 @@ __device__ __forceinline__ float reduce_scatter(const float (&v)[N], int lane, i
 // added into grad2d, and k_project_bwd maps them to dL/d(mean2d, conic,
 // opacity) with the Gaussian's own A, B, C, o.
 template <int kRPL, bool kDepth, bool kFeat = false>
-__global__ void __launch_bounds__(kTilePixels / kRPL, 56 / kRPL)
+__global__ void __launch_bounds__(kTilePixels / kRPL, GS_BWD_MINB)
 k_render_bwd(CamConst cam, const float4 *__restrict__ xyod, const float4 *__restrict__ conr,
              const ChannelIO io, const uint32_t *__restrict__ pair_gid,
              const uint2 *__restrict__ ranges, const uint32_t *__restrict__ order,
