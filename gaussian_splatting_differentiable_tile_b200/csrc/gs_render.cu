@@ -20,7 +20,9 @@
 // (forward 256 entries, backward 128), each entry converted once per tile to
 //     geo  = (mx, my, cA, cB),  geo2 = (cC, log2 o, kx, ky)
 // with cA = -log2(e) A / 2, cB = -log2(e) B, cC = -log2(e) C / 2, so that
-//     log2(o exp(-sigma)) = log2 o + cA dx^2 + cB dx dy + cC dy^2.
+//     log2(o exp(-sigma)) = log2 o + cA dx^2 + cB dx dy + cC dy^2;
+// kx, ky serve the cull masks while staging, and geo2.z then holds the
+// centre c of the range test below.
 // The terms that depend only on the column (dx) are computed once per entry
 // and shared by the lane's RPL pixels.
 //
@@ -104,6 +106,14 @@ struct ChannelIO {
     float *cgrad;       // backward: the channel-gradient sums of Gaussian g at cgrad[g * cgrad_stride]
     int cgrad_stride;   // in floats
 };
+
+// The blend's two skip tests (sigma < 0, alpha < 1/255) on the exponent
+// q = -sigma log2(e) as one range test: a pixel takes the entry iff
+// log2(1/255) - log2 o <= q <= 0, i.e. |q - c| <= -c with
+// c = (log2(1/255) - log2 o) / 2, computed once per entry while staging
+// (c > 0 when o < 1/255: then no pixel passes).  Every kernel that walks
+// the lists stages c the same way, so their decisions agree bit for bit.
+__device__ __forceinline__ float hit_center(float log2o) { return 0.5f * (kLog2AlphaMin - log2o); }
 
 // Geometry of a lane: its column centre and first row's centre; and the
 // tile's strips (2 RPL rows each): x centre and half width, y centre of the
@@ -189,8 +199,8 @@ __device__ __forceinline__ bool eval_alpha(const float4 geo, const float4 geo2, 
     dy = __fsub_rn(geo.y, fy);
     const float u = __fmaf_rn(geo2.x, dy, c.bdx);
     const float q = __fmaf_rn(dy, u, c.a0);
+    if (!(fabsf(__fsub_rn(q, geo2.z)) <= -geo2.z)) return false;  // the range test above
     const float p = __fadd_rn(q, geo2.y);              // log2(o exp(-sigma))
-    if (q > 0.f || p < kLog2AlphaMin) return false;
     const float a = ex2_approx(p);
     capped = a > cap;
     alpha = fminf(a, cap);
@@ -237,6 +247,7 @@ k_render_fwd(CamConst cam, const float4 *__restrict__ xyod, const float4 *__rest
             s_col[threadIdx.x] = io.col[kFeat ? (size_t)g * io.col_stride : (size_t)g];
             const uint32_t m = strip_mask<kWarps>(geo, geo2, L.sx, L.hx, L.sy0, 2.f, L.hy);
             s_mask[threadIdx.x] = (uint8_t)m;
+            s_geo2[threadIdx.x].z = hit_center(geo2.y);  // kx, ky are only needed for the mask
         }
         __syncthreads();
         const uint32_t n = compact_slots<kBatch>(s_mask, 0, cnt, warp, lane, s_list[warp]);
@@ -437,6 +448,7 @@ k_render_bwd(CamConst cam, const float4 *__restrict__ xyod, const float4 *__rest
             s_col[i0] = ra;
             s_gid[i0] = ga;
             s_mask[i0] = (uint8_t)strip_mask<kWarps>(geo, geo2, L.sx, L.hx, L.sy0, 2.f * kRPL, L.hy);
+            s_geo2[i0].z = hit_center(geo2.y);
             if (i1 < cnt) {
                 stage_entry(xb, cb, geo, geo2);
                 s_geo[i1] = geo;
@@ -444,6 +456,7 @@ k_render_bwd(CamConst cam, const float4 *__restrict__ xyod, const float4 *__rest
                 s_col[i1] = rb;
                 s_gid[i1] = gb;
                 s_mask[i1] = (uint8_t)strip_mask<kWarps>(geo, geo2, L.sx, L.hx, L.sy0, 2.f * kRPL, L.hy);
+                s_geo2[i1].z = hit_center(geo2.y);
             }
         }
         __syncthreads();
@@ -468,8 +481,9 @@ k_render_bwd(CamConst cam, const float4 *__restrict__ xyod, const float4 *__rest
                 const float2 u = __ffma2_rn(make_float2(geo2.x, geo2.x), dy[i], make_float2(ct.bdx, ct.bdx));
                 const float2 q = __ffma2_rn(dy[i], u, make_float2(ct.a0, ct.a0));
                 p[i] = __fadd2_rn(q, make_float2(geo2.y, geo2.y));
-                hit[2 * i] = j < lst[2 * i] && !(q.x > 0.f) && !(p[i].x < kLog2AlphaMin);
-                hit[2 * i + 1] = j < lst[2 * i + 1] && !(q.y > 0.f) && !(p[i].y < kLog2AlphaMin);
+                const float2 t = __fadd2_rn(q, make_float2(-geo2.z, -geo2.z));  // q - c, as the forward
+                hit[2 * i] = j < lst[2 * i] && fabsf(t.x) <= -geo2.z;
+                hit[2 * i + 1] = j < lst[2 * i + 1] && fabsf(t.y) <= -geo2.z;
                 any |= hit[2 * i] | hit[2 * i + 1];
             }
             if (!__any_sync(0xffffffffu, any)) continue;
@@ -564,6 +578,7 @@ k_render_stats(CamConst cam, const float4 *__restrict__ xyod, const float4 *__re
             const uint32_t g = pair_gid[j];
             float4 geo, geo2;
             stage_entry(xyod[g], conr[g], geo, geo2);
+            geo2.z = hit_center(geo2.y);
             s_geo[threadIdx.x] = geo;
             s_geo2[threadIdx.x] = geo2;
         }
