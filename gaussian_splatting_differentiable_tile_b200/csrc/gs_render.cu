@@ -48,11 +48,16 @@
 #endif
 // Backward: entries staged per round (at most 128) and resident CTAs per SM
 // the register allocation targets (tuning knobs; defaults measured fastest).
+// Forward: resident CTAs per SM the register allocation targets (a tuning
+// knob; the default is the fastest measured).
+#ifndef GS_FWD_MINB
+#define GS_FWD_MINB 6
+#endif
 #ifndef GS_BWD_BATCH
 #define GS_BWD_BATCH 128
 #endif
 #ifndef GS_BWD_MINB
-#define GS_BWD_MINB (56 / GS_BWD_RPL)
+#define GS_BWD_MINB (48 / GS_BWD_RPL)
 #endif
 
 namespace gs {
@@ -215,7 +220,7 @@ __device__ __forceinline__ bool eval_alpha(const float4 geo, const float4 geo2, 
 // could not have passed the alpha test at any pixel of the strip, so the
 // sequence of contributions, the stopping entry and `last` are unchanged.
 template <bool kDepth, bool kFeat = false>
-__global__ void __launch_bounds__(kTilePixels, 6)
+__global__ void __launch_bounds__(kTilePixels, GS_FWD_MINB)
 k_render_fwd(CamConst cam, const float4 *__restrict__ xyod, const float4 *__restrict__ conr,
              const ChannelIO io, const uint32_t *__restrict__ pair_gid,
              const uint2 *__restrict__ ranges, const uint32_t *__restrict__ order,
