@@ -94,8 +94,11 @@ SPECS = {
                          -4.0, 0.6, 1.0, 1.5, 980, 545, 1000.0, "ring", 60, 2),
     "teacher": SceneSpec("teacher: 742k Gaussians, 200 clusters, 980x545, f=1000", 742_000, 200,
                          -5.0, 0.7, 0.0, 2.0, 980, 545, 1000.0, "orbit", 16, 3),
-    "train400k": SceneSpec("train400k: 400k Gaussians, 120 clusters, 1960x1090, f=2000", 400_000,
-                           120, -4.0, 0.6, 1.0, 1.5, 1960, 1090, 2000.0, "ring", 16, 4),
+    # full resolution, the log-scale mean raised from -4.0 in steps of 0.25
+    # until a frame's pair list (opacity-aware cut) exceeds 2^24 entries
+    "train400k": SceneSpec("train400k: 400k Gaussians, 120 clusters, log-scales N(-2.5,0.6), 1960x1090, "
+                           "f=2000, > 2^24 pairs", 400_000, 120, -2.5, 0.6, 1.0, 1.5, 1960, 1090, 2000.0,
+                           "ring", 16, 4),
     "train400k_half": SceneSpec("train400k_half: 400k Gaussians, 120 clusters, 980x545, f=1000",
                                 400_000, 120, -4.0, 0.6, 1.0, 1.5, 980, 545, 1000.0, "ring", 16, 4),
     "large_splats": SceneSpec("large_splats: 30k Gaussians, log-scales N(-2.5,0.6), 1960x1090",

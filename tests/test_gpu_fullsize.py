@@ -1,6 +1,9 @@
 """Parity at the benchmark's own size and launch configuration: 400k
 Gaussians at 980 x 545 (ring camera), opacity-aware tile cut on, pair list
-sized as the benchmark sizes it and binned without a host sync.
+sized as the benchmark sizes it and binned without a host sync; and the
+full-resolution 400k configuration (1960 x 1090) whose pair list exceeds
+2^24 entries ("SplatRs: We Gave the Model 4x More Pixels and It Got Worse",
+Lesson 2), where the default pair list overflows and is regrown.
 
 Integer stages are compared in full (the oracle bins all 400k Gaussians by
 brute force); the blend and its backward on seeded samples of tiles, which
@@ -20,13 +23,11 @@ from test_gpu_parity import _assert_fwd, _check_bins
 
 pytestmark = pytest.mark.gpu
 
-SPEC = SPECS["train400k_half"]
-
-
-@pytest.fixture(scope="module")
-def scene():
-    params = make_scene(SPEC)
-    cam = make_cameras(SPEC)[5]
+@pytest.fixture(scope="module", params=["train400k_half", "train400k"])
+def scene(request):
+    spec = SPECS[request.param]
+    params = make_scene(spec)
+    cam = make_cameras(spec)[5]
     cam.flags = G.GS_FLAG_TIGHT_TILES
     return cam, params
 
@@ -47,7 +48,9 @@ def test_fullsize_projection(scene):
                (p["cut_margin"] < MARGIN_CUT))
     diff = np.any(rect != p["rect"], axis=1) | (count != p["count"])
     assert not np.any(diff & ~amb), np.nonzero(diff & ~amb)[0][:10]
-    assert amb.sum() <= 2e-3 * n
+    # at most 0.5 % of the Gaussians sit that close to a decision (measured
+    # by the oracle: 0.29 % at full resolution, fewer at half resolution)
+    assert amb.sum() <= 5e-3 * n
 
 
 def test_fullsize_binning_blend_and_backward(scene):
@@ -85,9 +88,30 @@ def test_fullsize_binning_blend_and_backward(scene):
     g2_ref, g2_abs = O.render_bwd(rec, cam, dl.astype(np.float64), tile_mask=mask)
     g2 = grad2d.cpu().numpy()
     touched = np.abs(g2_ref).sum(axis=1) > 0
-    assert touched.sum() > 1000
+    assert touched.sum() > 500  # 40 tiles: about 900 Gaussians at full resolution, more at half
     grad_compare(g2[:, :g2_ref.shape[1]], g2_ref, g2_abs, "grad2d")
     raw_ref = O.project_bwd(params, cam, g2_ref)
     bound = O.grad_bound(params, cam, g2_abs)
     for k in G.PARAM_KEYS:
         grad_compare(grads[k].cpu().numpy(), raw_ref[k], bound[k], k)
+
+
+def test_fullsize_pair_list_regrows_past_2_24(scene):
+    """The rasterizer's default pair list (16 per Gaussian) overflows on the
+    full-resolution frame; the capacity error reports the need, the list is
+    regrown and the frame binned again, with K the oracle's."""
+    cam, params = scene
+    n = params["means"].shape[0]
+    K_ref = int(oracle_records(params, cam)["count"].sum())
+    r = G.Rasterizer(n, cam.width, cam.height)
+    default = r.bins.max_pairs
+    r.forward(cam, cuda_params(params))
+    torch.cuda.synchronize()
+    K = r.n_pairs
+    # K is the sum of the GPU's own tile counts, and the oracle's up to the
+    # few Gaussians whose rectangle edge sits within its margin (a raw-
+    # parameter projection in single precision)
+    assert K == int(r.proj.count.sum().item())
+    assert abs(K - K_ref) <= 1e-5 * K_ref
+    if K_ref > default:
+        assert K > 1 << 24 and r.bins.max_pairs >= K
