@@ -94,3 +94,33 @@ def test_binding_fails_loudly_without_library(tmp_path):
             _abi.load(str(tmp_path / "missing.so"))
         finally:
             _abi._LIB = saved
+
+
+def test_ctypes_layouts_match_the_c_compiler(tmp_path):
+    """Every struct of include/gs.h, as the C compiler lays it out (size and
+    the offset of every field), equals the binding's ctypes declaration."""
+    import shutil
+    import subprocess
+    from gaussian_splatting_differentiable_tile_b200 import _abi
+    cc = shutil.which("gcc") or shutil.which("cc")
+    if cc is None:
+        pytest.skip("no C compiler")
+    structs = {"gs_camera": _abi.GsCamera, "gs_params": _abi.GsParams, "gs_grads": _abi.GsGrads,
+               "gs_projected": _abi.GsProjected, "gs_bins": _abi.GsBins, "gs_profile_stat": _abi.GsProfileStat,
+               "gs_adam_config": _abi.GsAdamConfig, "gs_train_lane": _abi.GsTrainLane}
+    lines = ['#include <stddef.h>', '#include <stdio.h>', '#include "gs.h"', "int main(void) {"]
+    for cname, cls in structs.items():
+        lines.append(f'printf("{cname} size %zu\\n", sizeof({cname}));')
+        for field, _ in cls._fields_:
+            lines.append(f'printf("{cname} {field} %zu\\n", offsetof({cname}, {field}));')
+    lines += ["return 0;", "}"]
+    src = tmp_path / "layout.c"
+    src.write_text("\n".join(lines))
+    exe = tmp_path / "layout"
+    subprocess.run([cc, "-I", os.path.join(ROOT, "include"), str(src), "-o", str(exe)], check=True)
+    out = subprocess.run([str(exe)], check=True, capture_output=True, text=True).stdout.split("\n")
+    got = {tuple(line.split()[:2]): int(line.split()[2]) for line in out if line.strip()}
+    for cname, cls in structs.items():
+        assert got[(cname, "size")] == ctypes.sizeof(cls), cname
+        for field, _ in cls._fields_:
+            assert got[(cname, field)] == getattr(cls, field).offset, (cname, field)
