@@ -11,6 +11,12 @@
  *   gs_render_bwd    back-to-front gradient of the blend, then the chain rule
  *                    to the raw parameters
  *
+ * Around them: gs_render_features_fwd/bwd (feature channels blended with the
+ * forward's weights), gs_train_step (a training step over several cameras,
+ * run as concurrent lanes, ending in gs_adam_step), gs_l1_loss_grad, the
+ * work counter gs_render_stats, and host-side size, carve, status, error and
+ * profiling calls.
+ *
  * Sources (cited by page title and section):
  *   [GSP]  "Gaussian splatting in PyTorch" (coderigor.dev), s1-s8
  *   [WEEK] "SplatRs: The Week the Gap Closed", "Throughput: the tile
