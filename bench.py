@@ -66,6 +66,12 @@ METRIC = "fwd and fwd+bwd frames/s at 400k Gaussians, 980x545; tile-pairs/s; % r
 OPS_VISIT = 12
 OPS_FWD_ADD = 6
 OPS_BWD_ADD = 32
+# The survey's per-evaluation estimate charges every visited entry the whole
+# evaluation (forward about 21 FP32-pipe instructions, backward about 50),
+# whether or not the entry passes the alpha test; reported beside the split
+# above, which charges the add path only to the entries that take it.
+SURVEY_OPS_FWD = 21
+SURVEY_OPS_BWD = 50
 
 # Algorithmic HBM bytes of the streaming stages (per Gaussian G, pair P):
 #   project      56 B/G raw parameters read + 68 B/G records written
@@ -99,6 +105,18 @@ def _peaks():
         return float(d["hbm_gbs"]), "measured", float(d.get("sm_max_mhz", 1965.0))
     except Exception:
         return 6650.0, "fallback", 1965.0
+
+
+def _cpu_model() -> str:
+    try:
+        with open("/proc/cpuinfo") as f:
+            for line in f:
+                if line.startswith("model name"):
+                    return line.split(":", 1)[1].strip()
+    except OSError:
+        pass
+    import platform
+    return platform.processor() or "unknown"
 
 
 def _src_sha(name):
@@ -217,9 +235,11 @@ def run_reference(args, spec, rank, world):
         cpu_frame_time(params, cams[i % len(cams)], args.ref_sample_tiles, seed=i, bin_fraction=frac)
     times = []
     info = None
+    wall0 = time.perf_counter()
     for i in range(args.steps):
         info = cpu_frame_time(params, cams[i % len(cams)], args.ref_sample_tiles, seed=100 + i, bin_fraction=frac)
         times.append(info["frame_s"])
+    wall = time.perf_counter() - wall0
     fps = 1.0 / statistics.mean(times)
     sample = (f"per step one camera: full projection of {spec.n} Gaussians, brute-force binning of a seeded "
               f"{frac:g} of them (its time scaled by 1/{frac:g}: linear in the Gaussians binned), blend and "
@@ -229,9 +249,13 @@ def run_reference(args, spec, rank, world):
            "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1000.0 * statistics.mean(times),
            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
            "data": "synthetic", "config": _config(spec, None, args.tiles, False, args.variant),
-           "cpu_baseline": {"value": fps, "unit": "frames/s", "cores": info["threads"], "kind": "oracle",
-                            "sample": sample},
-           "e2e": {"value": fps, "unit": "frames/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+           "cpu_baseline": {"value": fps, "unit": "frames/s", "cores": info["threads"], "cpu_model": _cpu_model(),
+                            "kind": "oracle", "sample": sample},
+           "e2e": {"value": fps, "unit": "frames/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+           # ms_per_step is the extrapolated time of a whole frame; the sampled
+           # work this run actually did took wall_s
+           "measured": {"wall_s": wall, "sampled_s_per_step": wall / max(1, args.steps),
+                        "extrapolated_ms_per_step": 1000.0 * statistics.mean(times)}}
     print(json.dumps(out), flush=True)
 
 
@@ -550,11 +574,22 @@ def run_native(args, spec, rank, world, local):
     sms = torch.cuda.get_device_properties(local).multi_processor_count
     clock_mhz = clocks["sm_max_mhz"] or sm_max
     alu_peak = sms * 128 * clock_mhz * 1e6 / 1e12  # T FP32 lane-ops/s
+    # the same peak at the median SM clock sampled during the timed region
+    alu_peak_sampled = sms * 128 * (clocks["sm_mhz"] or clock_mhz) * 1e6 / 1e12
     # work per timed step (cameras cycle through `mine`)
     sel = [i % len(mine) for i in range(args.steps)]
     pairs_steps = [pairs[i] for i in sel]
-    fwd_ops = sum(OPS_VISIT * stats[i]["fwd_visits"] + OPS_FWD_ADD * stats[i]["contributions"] for i in sel)
-    bwd_ops = sum(OPS_VISIT * stats[i]["bwd_visits"] + OPS_BWD_ADD * stats[i]["contributions"] for i in sel)
+    fwd_visits = sum(stats[i]["fwd_visits"] for i in sel)
+    bwd_visits = sum(stats[i]["bwd_visits"] for i in sel)
+    contributions = sum(stats[i]["contributions"] for i in sel)
+    fwd_ops = OPS_VISIT * fwd_visits + OPS_FWD_ADD * contributions
+    bwd_ops = OPS_VISIT * bwd_visits + OPS_BWD_ADD * contributions
+    work = {"steps": args.steps, "fwd_visits": fwd_visits, "bwd_visits": bwd_visits,
+            "contributions": contributions,
+            "ops": {"visit": OPS_VISIT, "fwd_add": OPS_FWD_ADD, "bwd_add": OPS_BWD_ADD},
+            "fwd_ops": fwd_ops, "bwd_ops": bwd_ops,
+            "formula": "fwd_ops = visit*fwd_visits + fwd_add*contributions; "
+                       "bwd_ops = visit*bwd_visits + bwd_add*contributions; achieved = ops / summed kernel ms"}
     stages = {}
     gpu_launches = 0
     for name, (launches, ms) in (prof or {}).items():
@@ -568,7 +603,12 @@ def run_native(args, spec, rank, world, local):
         elif name in ALU_KERNELS:
             ops = fwd_ops if name == "render_fwd" else bwd_ops
             ach = ops / (ms * 1e-3) / 1e12
-            entry.update(bound="alu", achieved=ach, peak=alu_peak, unit="Tops/s", frac=ach / alu_peak)
+            entry.update(bound="alu", achieved=ach, peak=alu_peak, unit="Tops/s", frac=ach / alu_peak,
+                         ops=ops, frac_at_sampled_clock=ach / alu_peak_sampled)
+            # the same work counted with the survey's per-evaluation constants
+            # (every visit charged the whole forward or backward evaluation)
+            survey = (SURVEY_OPS_FWD * fwd_visits if name == "render_fwd" else SURVEY_OPS_BWD * bwd_visits)
+            entry["frac_survey_constants"] = survey / (ms * 1e-3) / 1e12 / alu_peak
         stages[name] = entry
     dom = max(stages, key=lambda k: stages[k]["ms_total"]) if stages else None
     roof = None
@@ -582,10 +622,15 @@ def run_native(args, spec, rank, world, local):
                 "unit": s["unit"], "frac": s["frac"], "traffic": traffic,
                 "peak_basis": (f"{sms} SMs x 128 FP32 lanes x {clock_mhz:.0f} MHz (FMA = 1 op)"
                                if s["bound"] == "alu" else f"{peak_kind} HBM copy bandwidth")}
+        if s["bound"] == "alu":
+            roof.update(kernel_ms_total=s["ms_total"], work=work,
+                        frac_at_sampled_clock=s["frac_at_sampled_clock"],
+                        sampled_sm_mhz=clocks["sm_mhz"])
     cpu = None
     if world == 1 and not args.no_cpu_baseline:
         info = cpu_frame_time(params_np, mine[0], args.cpu_sample_tiles)
-        cpu = {"value": 1.0 / info["frame_s"], "unit": "frames/s", "cores": info["threads"], "kind": "oracle",
+        cpu = {"value": 1.0 / info["frame_s"], "unit": "frames/s", "cores": info["threads"],
+               "cpu_model": _cpu_model(), "kind": "oracle",
                "sample": (f"one camera: full projection and brute-force binning of {n} Gaussians, blend and "
                           f"backward on {info['sampled_tiles']} of {info['tiles']} seeded tiles, frame time "
                           f"extrapolated by tile count ({info['frame_s']:.1f} s/frame)"),

@@ -32,7 +32,8 @@ from ._abi import (GS_ERR_ALIGNMENT, GS_ERR_CAPACITY, GS_ERR_CUDA, GS_ERR_DEVICE
 __all__ = [
     "GSError", "Projected", "Bins", "make_camera", "channels", "gs_project", "gs_bin_and_sort",
     "gs_bin_and_sort_static", "gs_render_fwd", "gs_render_features_fwd", "gs_render_features_bwd",
-    "gs_render_bwd", "gs_render_stats", "gs_l1_loss_grad", "gs_read_status", "gs_error_string", "profile_begin",
+    "gs_render_bwd", "gs_render_stats", "gs_l1_loss_grad", "gs_read_status", "gs_last_device_error",
+    "gs_sort_bytes", "gs_error_string", "profile_begin",
     "profile_end", "lib", "PARAM_KEYS",
 ]
 
@@ -183,7 +184,15 @@ def gs_bin_and_sort_static(cam, n: int, proj: Projected, pair_tile: torch.Tensor
     """gs_bin_and_sort without a caller scratch buffer (the library's fixed
     array holds it; see include/gs.h).  Writes the sorted pairs and ranges into
     the given int32 CUDA tensors and returns K; raises GSError on any error
-    (with .n_pairs set for GS_ERR_CAPACITY)."""
+    (with .n_pairs set for GS_ERR_CAPACITY).  The C call cannot see the
+    arrays' sizes, so they are checked here, before anything is launched:
+    pair_gid must hold as many entries as pair_tile (the capacity passed on)
+    and ranges two per tile of the camera's grid."""
+    tiles = ((int(cam.width) + GS_TILE - 1) // GS_TILE) * ((int(cam.height) + GS_TILE - 1) // GS_TILE)
+    if pair_gid.numel() < pair_tile.numel():
+        raise ValueError(f"pair_gid holds {pair_gid.numel()} entries, fewer than pair_tile's {pair_tile.numel()}")
+    if ranges.numel() < 2 * tiles:
+        raise ValueError(f"ranges holds {ranges.numel()} entries; the camera's {tiles} tiles need {2 * tiles}")
     c = make_camera(cam)
     k = ctypes.c_int64(0)
     rc = lib().gs_bin_and_sort_static(ctypes.byref(c), int(n), ctypes.byref(proj.struct),
@@ -289,6 +298,20 @@ def gs_read_status(bins: Bins, stream=None):
     if rc == GS_ERR_CUDA:
         raise GSError(rc, "gs_read_status")
     return rc, int(k.value)
+
+
+def gs_last_device_error(bins: Bins, stream=None) -> int:
+    """Synchronizes and returns the status word of the last gs_bin_and_sort
+    on these bins (GS_OK or a GS_ERR_* code)."""
+    rc = lib().gs_last_device_error(ctypes.byref(bins.struct), _stream(stream))
+    if rc == GS_ERR_CUDA:
+        raise GSError(rc, "gs_last_device_error")
+    return rc
+
+
+def gs_sort_bytes(max_pairs: int, tiles: int) -> int:
+    """Scratch bytes of one bin-and-sort for max_pairs pairs and `tiles` tiles."""
+    return int(lib().gs_sort_bytes(int(max_pairs), int(tiles)))
 
 
 def profile_begin(max_launches: int = 1 << 16) -> None:

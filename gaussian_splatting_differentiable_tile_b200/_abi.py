@@ -132,6 +132,8 @@ PROTOTYPES = {
                                      ctypes.c_void_p, ctypes.c_void_p, ctypes.POINTER(GsGrads), ctypes.c_void_p]),
     "gs_read_status": (ctypes.c_int, [ctypes.POINTER(GsBins), ctypes.POINTER(ctypes.c_int64),
                                       ctypes.c_void_p]),
+    "gs_last_device_error": (ctypes.c_int, [ctypes.POINTER(GsBins), ctypes.c_void_p]),
+    "gs_sort_bytes": (ctypes.c_size_t, [ctypes.c_int64, ctypes.c_int32]),
     "gs_error_string": (ctypes.c_char_p, [ctypes.c_int]),
     "gs_profile_begin": (ctypes.c_int, [ctypes.c_int32]),
     "gs_profile_end": (ctypes.c_int, [ctypes.POINTER(GsProfileStat), ctypes.c_int32]),

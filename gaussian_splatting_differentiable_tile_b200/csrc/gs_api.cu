@@ -229,6 +229,13 @@ int gs_read_status(const gs_bins *bins, int64_t *n_pairs_host, void *stream) {
     return st;
 }
 
+int gs_last_device_error(const gs_bins *bins, void *stream) { return gs_read_status(bins, nullptr, stream); }
+
+size_t gs_sort_bytes(int64_t max_pairs, int32_t tiles) {
+    if (max_pairs < 0 || tiles < 1) return 0;
+    return bins_layout(0, max_pairs, tiles).total;
+}
+
 int gs_bin_and_sort(const gs_camera *cam, int64_t n, const gs_projected *proj, const gs_bins *bins,
                     int64_t *n_pairs_host, void *stream) {
     CamConst c;
@@ -661,8 +668,11 @@ extern "C" int gs_bin_and_sort_static(const gs_camera *cam, int64_t n, const gs_
     bins.scratch = base;
     bins.scratch_bytes = kStaticBytes;
     cudaStream_t s = as_stream(stream);
-    // The launcher clears the status, count, ticket, histogram, range and
-    // look-back words at its start, so nothing of the previous call leaks in.
+    // Nothing of the previous call leaks in: the launcher's one memset clears
+    // the status word and K, and every other array the stages read (the
+    // [CTA][tile] count matrix, the per-tile totals, ranges and tile order,
+    // the emitted keys, the long-list sort's ping-pong arrays) is written in
+    // full, for every tile or pair of this call, before it is read.
     if (launch_bin_and_sort(c, n, *proj, bins, kStaticLayout, s) != cudaSuccess) return GS_ERR_CUDA;
     if (cudaMemcpyAsync(ranges, bins.ranges, (size_t)tiles * 2 * sizeof(uint32_t),
                         cudaMemcpyDeviceToDevice, s) != cudaSuccess)

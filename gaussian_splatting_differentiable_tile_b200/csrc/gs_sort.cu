@@ -25,6 +25,8 @@
 //                  sorted in global memory by one CTA each
 //
 // No kernel waits on another CTA, and no global atomic is contended.
+#include <mutex>
+
 #include "gs_internal.cuh"
 
 namespace gs {
@@ -536,15 +538,40 @@ k_tile_sort(const uint32_t *__restrict__ ranges, const uint32_t *__restrict__ or
     }
 }
 
-int num_sms() {
-    static int sms = 0;
-    if (sms == 0) {
-        int dev = 0;
-        cudaGetDevice(&dev);
-        cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-        if (sms <= 0) sms = 148;
+// Per-device launch set-up of the binning kernels, done once per device with
+// that device current: its SM count, and the dynamic shared memory the count,
+// emit and wide sort kernels may use beyond the default 48 KB (a function
+// attribute is a property of the device it was set on).
+constexpr int kMaxDevices = 128;
+struct DeviceSetup {
+    int sms = 0;
+    cudaError_t err = cudaSuccess;
+};
+DeviceSetup g_setup[kMaxDevices];
+std::mutex g_setup_mutex;
+
+cudaError_t device_setup(int *sms) {
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return e;
+    if (dev < 0 || dev >= kMaxDevices) return cudaErrorInvalidDevice;
+    std::lock_guard<std::mutex> lock(g_setup_mutex);
+    DeviceSetup &d = g_setup[dev];
+    if (d.sms == 0) {
+        int n = 0;
+        if ((e = cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev)) != cudaSuccess) return e;
+        const int cnt_bytes = (int)(kSmemTiles * sizeof(uint32_t));
+        if ((e = cudaFuncSetAttribute(k_bin_count, cudaFuncAttributeMaxDynamicSharedMemorySize, cnt_bytes)) !=
+                cudaSuccess ||
+            (e = cudaFuncSetAttribute(k_bin_emit, cudaFuncAttributeMaxDynamicSharedMemorySize, cnt_bytes)) !=
+                cudaSuccess ||
+            (e = cudaFuncSetAttribute(k_tile_sort<kMidWarps, true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                      (int)(2 * kTileSortMid * sizeof(uint64_t)))) != cudaSuccess)
+            return e;
+        d.sms = n > 0 ? n : 148;
     }
-    return sms;
+    *sms = d.sms;
+    return cudaSuccess;
 }
 
 }  // namespace
@@ -562,24 +589,15 @@ cudaError_t launch_bin_and_sort(const CamConst &c, int64_t n, const gs_projected
     uint64_t *keys = reinterpret_cast<uint64_t *>(base + L.keys);
     const int4 *rect = reinterpret_cast<const int4 *>(proj.rect);
     const int tiles = c.tiles_x * c.tiles_y;
-    const int sms = num_sms();
+    int sms = 0;
+    cudaError_t e = device_setup(&sms);
+    if (e != cudaSuccess) return e;
     // CTAs sharing the Gaussians: two per SM, within the count matrix's size
     int64_t ctas64 = std::min<int64_t>((int64_t)2 * sms, (int64_t)kBinCTAsMax);
     ctas64 = std::min<int64_t>(ctas64, kBinHistCap / tiles);
     const int ctas = (int)std::max<int64_t>(1, ctas64);
     const size_t cnt_smem = tiles <= kSmemTiles ? (size_t)tiles * sizeof(uint32_t) : 0;
-    static bool attr = [] {
-        cudaFuncSetAttribute(k_bin_count, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             (int)(kSmemTiles * sizeof(uint32_t)));
-        cudaFuncSetAttribute(k_bin_emit, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             (int)(kSmemTiles * sizeof(uint32_t)));
-        cudaFuncSetAttribute(k_tile_sort<kMidWarps, true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             (int)(2 * kTileSortMid * sizeof(uint64_t)));
-        return true;
-    }();
-    (void)attr;
-
-    cudaError_t e = cudaMemsetAsync(base, 0, L.zero_bytes, s);
+    e = cudaMemsetAsync(base, 0, L.zero_bytes, s);
     if (e != cudaSuccess) return e;
     // 1. per-CTA tile counts, 2. offsets down each tile's column
     prof_before("bin_count", s);

@@ -423,7 +423,9 @@ int gs_train_step(const gs_camera *cams, int32_t n_cams, int64_t n, const gs_par
  *
  * There is no counterpart in the source pages: this is a deployment variant.
  * gs_bin_and_sort needs a caller-allocated scratch buffer (gs_bins) for its
- * depth sort, scan look-back and pair sort.  Some callers cannot allocate it:
+ * per-tile binning stages: the [CTA][tile] count matrix, the per-tile totals
+ * and ranges, the tile order, the emitted sort keys and the long-list sort's
+ * ping-pong arrays.  Some callers cannot allocate it:
  * a real-time viewer's frame loop that must never call cudaMalloc/cudaFree
  * (both can synchronize the whole device and stall a frame), or a plug-in
  * whose host application owns all device memory and hands it no allocator.
@@ -457,6 +459,19 @@ int gs_bin_and_sort_static(const gs_camera *cam, int64_t n, const gs_projected *
 /* Synchronizes `stream`, then returns bins->status and stores K in
  * *n_pairs_host (HOST, nullable).  GS_ERR_CUDA if the copy fails. */
 int gs_read_status(const gs_bins *bins, int64_t *n_pairs_host, void *stream);
+
+/* Synchronizes `stream` and returns the device error word the kernels of
+ * the last gs_bin_and_sort on `bins` recorded: GS_OK, or the GS_ERR_* code
+ * (GS_ERR_CAPACITY).  The word lives in the caller's bins buffer, not in the
+ * library (which holds no per-call state), so the call takes `bins`.  Same
+ * as gs_read_status without the pair count.  GS_ERR_CUDA if the copy fails;
+ * GS_ERR_INVALID_ARG for a NULL or incomplete bins. */
+int gs_last_device_error(const gs_bins *bins, void *stream);
+
+/* Bytes of the scratch one bin-and-sort needs for max_pairs pairs and
+ * `tiles` tiles: gs_bins_bytes for any n (the layout does not depend on N)
+ * and a grid of `tiles` tiles.  0 if max_pairs < 0 or tiles < 1. */
+size_t gs_sort_bytes(int64_t max_pairs, int32_t tiles);
 
 /* Static, human-readable text for a return code. */
 const char *gs_error_string(int code);

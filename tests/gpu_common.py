@@ -119,8 +119,38 @@ def tiles_to_pixels(tiles: np.ndarray, cam) -> np.ndarray:
     return px[:cam.height, :cam.width]
 
 
+# At most this fraction of the compared gradient elements (those with a
+# non-zero value on either side) may pass only by the cancellation-aware
+# rule.  An element needs it when its terms cancel to below about 1e-4 of
+# their absolute sum, so that fp32 reordering alone exceeds 1e-3 relative:
+# for random per-pixel gradients that is rare, well under 1e-3 of the
+# elements.
+MAX_EXCUSED_FRAC = 1e-3
+# At most this fraction of the compared pixels may have a threshold decision
+# inside the stated margins (measured by the oracle: up to 1.05e-2 on the
+# dense full-size scenes, where most are T within 1e-3 of 1e-4 -- an alpha
+# just under the cap multiplies its fp32 error by alpha / (1 - alpha), about
+# 50, in T -- and under 2e-4 on the sparse ones).
+MAX_AMBIGUOUS_FRAC = 1.5e-2
+
+
+def report(what: str, **counts) -> None:
+    """One line in the pytest log (-s, or the captured output of a failure)."""
+    print(f"[parity] {what}: " + ", ".join(f"{k}={v}" for k, v in counts.items()), flush=True)
+
+
+def check_ambiguous(amb: np.ndarray, sel: np.ndarray, what: str) -> int:
+    """Counts and bounds the pixels excluded or excused as ambiguous."""
+    n_amb, n_sel = int((amb & sel).sum()), int(sel.sum())
+    report(what, ambiguous_pixels=n_amb, compared_pixels=n_sel, fraction=f"{n_amb / max(1, n_sel):.2e}")
+    assert n_amb <= MAX_AMBIGUOUS_FRAC * n_sel + 4, f"{what}: {n_amb} of {n_sel} pixels ambiguous"
+    return n_amb
+
+
 def grad_compare(gpu: np.ndarray, ref: np.ndarray, bound: np.ndarray, name: str):
-    """Returns (n_excused); raises AssertionError on an unexcused element."""
+    """Returns (n_excused); raises AssertionError on an unexcused element, or
+    when more than MAX_EXCUSED_FRAC of the compared elements needed the
+    cancellation-aware rule.  Prints the counts."""
     d = np.abs(gpu.astype(np.float64) - ref)
     ok = (d <= GRAD_ABS) | (d <= GRAD_REL * np.abs(ref))
     excused = ~ok & (d <= GRAD_REL * bound + GRAD_ABS)
@@ -129,4 +159,9 @@ def grad_compare(gpu: np.ndarray, ref: np.ndarray, bound: np.ndarray, name: str)
         i = np.argwhere(bad)[0]
         raise AssertionError(f"{name}: {int(bad.sum())} gradient elements out of tolerance; first at "
                              f"{tuple(i)}: gpu={gpu[tuple(i)]!r} ref={ref[tuple(i)]!r} bound={bound[tuple(i)]!r}")
-    return int(excused.sum())
+    compared = int(((ref != 0) | (gpu != 0)).sum())
+    n_exc = int(excused.sum())
+    report(f"gradients {name}", compared=compared, excused=n_exc,
+           worst_rel=f"{float(np.max(d / np.maximum(np.abs(ref), 1e-30), initial=0.0)):.2e}" if compared else "0")
+    assert n_exc <= MAX_EXCUSED_FRAC * compared + 2, f"{name}: {n_exc} of {compared} elements excused"
+    return n_exc

@@ -124,3 +124,31 @@ def test_ctypes_layouts_match_the_c_compiler(tmp_path):
         assert got[(cname, "size")] == ctypes.sizeof(cls), cname
         for field, _ in cls._fields_:
             assert got[(cname, field)] == getattr(cls, field).offset, (cname, field)
+
+
+def test_sort_bytes_is_the_bins_layout_for_any_n(lib):
+    """gs_sort_bytes (the size query under its plain name) equals gs_bins_bytes
+    for the same pairs and tile grid, whatever N."""
+    W, H = 1960, 1090
+    tiles = ((W + 15) // 16) * ((H + 15) // 16)
+    for n, mp in ((0, 0), (1000, 5000), (400_000, 21_000_000)):
+        assert lib.gs_sort_bytes(mp, tiles) == lib.gs_bins_bytes(n, mp, W, H)
+    assert lib.gs_sort_bytes(-1, tiles) == 0 and lib.gs_sort_bytes(10, 0) == 0
+
+
+def test_static_binding_refuses_short_arrays_before_any_launch():
+    """gs_bin_and_sort_static cannot see the sizes of its output arrays, so the
+    binding refuses a pair_gid shorter than pair_tile, or ranges with fewer
+    than two entries per tile, before anything reaches the library."""
+    import torch
+
+    import gaussian_splatting_differentiable_tile_b200 as G
+    from scenes import tiny_camera
+
+    cam = tiny_camera(100, 40)  # 7 x 3 tiles
+    pt = torch.empty(64, dtype=torch.int32)
+    with pytest.raises(ValueError, match="pair_gid"):
+        G.gs_bin_and_sort_static(cam, 8, None, pt, torch.empty(63, dtype=torch.int32),
+                                 torch.empty(21, 2, dtype=torch.int32))
+    with pytest.raises(ValueError, match="ranges"):
+        G.gs_bin_and_sort_static(cam, 8, None, pt, pt.clone(), torch.empty(20, 2, dtype=torch.int32))

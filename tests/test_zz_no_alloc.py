@@ -12,7 +12,7 @@ import pytest
 import torch
 
 import gaussian_splatting_differentiable_tile_b200 as G
-from scenes import make_cameras, make_scene, tiny_camera
+from scenes import Camera, make_cameras, make_scene, tiny_camera
 
 from gpu_common import cuda_params
 
@@ -56,6 +56,39 @@ def test_static_variant_matches_bin_and_sort_on_consecutive_calls():
         np.testing.assert_array_equal(ranges_s, ranges)
 
 
+def _synthetic(W, H, n, seed, spread, log_scale):
+    """n Gaussians in front of an identity camera looking down +z."""
+    cam = Camera(np.eye(4), W * 0.5, W * 0.5, W / 2.0, H / 2.0, W, H)
+    rng = np.random.default_rng(seed)
+    params = {"means": np.column_stack([rng.uniform(-spread, spread, n), rng.uniform(-spread, spread, n),
+                                        rng.uniform(2, 4, n)]).astype(np.float32),
+              "log_scales": rng.normal(log_scale, 0.2, (n, 3)).astype(np.float32),
+              "quats": rng.normal(size=(n, 4)).astype(np.float32),
+              "opacity_logits": rng.normal(0, 1, n).astype(np.float32),
+              "colors": rng.uniform(0, 1, (n, 3)).astype(np.float32)}
+    return cam, params
+
+
+def test_static_variant_long_lists_and_large_grids():
+    """The two paths of the shared array that short lists on small grids never
+    reach, each compared with gs_bin_and_sort: tile lists longer than 8192
+    entries (sorted by the long-list radix sort in the array's ping-pong
+    space), and a grid of more than 16384 tiles (counted in the array's
+    count matrix instead of shared memory, with fewer CTAs)."""
+    cases = [_synthetic(48, 32, 10_000, 3, 0.3, -0.5),        # 6 tiles, ~10 000 entries each
+             _synthetic(2400, 1800, 3000, 4, 1.0, -3.0)]       # 150 x 113 = 16 950 tiles
+    for cam, params in cases:
+        proj, n = _project(cam, params)
+        K, tile, gid, ranges = _reference(cam, proj, n)
+        length = ranges[:, 1] - ranges[:, 0]
+        assert length.max() > 8192 or cam.tiles > 16384
+        Ks, tile_s, gid_s, ranges_s = _static(cam, proj, n, max_pairs=K + 16)
+        assert Ks == K
+        np.testing.assert_array_equal(tile_s, tile)
+        np.testing.assert_array_equal(gid_s, gid)
+        np.testing.assert_array_equal(ranges_s, ranges)
+
+
 def test_static_variant_rejects_sizes_beyond_its_array():
     cam = tiny_camera()
     proj = G.Projected(16)
@@ -76,7 +109,10 @@ def test_static_variant_reports_capacity():
     proj, n = _project(cam, params)
     K, _, _, _ = _reference(cam, proj, n)
     pt = torch.empty(K - 1, dtype=torch.int32, device="cuda")
-    rg = torch.empty(cam.tiles, 2, dtype=torch.int32, device="cuda")
+    rg = torch.full((cam.tiles, 2), -1, dtype=torch.int32, device="cuda")
     with pytest.raises(G.GSError) as ei:
         G.gs_bin_and_sort_static(cam, n, proj, pt, pt.clone(), rg)
     assert ei.value.code == G.GS_ERR_CAPACITY and ei.value.n_pairs == K
+    # as documented: every tile's range is left empty, so a render of these
+    # ranges draws only background
+    assert int(rg.abs().sum().item()) == 0
