@@ -88,6 +88,18 @@ BYTES = {
     "tile_sort": lambda G, P: 16 * P,
     "project_bwd": lambda G, P: 240 * G,
 }
+# The same stages on the global binning path (GS_BIN_GLOBAL):
+#   depth_sort   16 B/G rectangle + 16 B/G depth record read, 8 B/G keys written;
+#                four passes of 4 B/G digit counts read + 8 B/G read, 8 B/G written
+#   emit         rank sums and offsets: 2 x (4 B/G order + 16 B/G rectangle)
+#                read, 4 B/G offsets written; the emit: 24 B/G read, 8 B/P written
+#   tile_sort    per pass over the tile id's 8-bit digits: 4 B/P counts read,
+#                8 B/P read and 8 B/P written
+BYTES_GLOBAL = {
+    "depth_sort": lambda G, P, tile_passes: 40 * G + 4 * 20 * G,
+    "emit": lambda G, P, tile_passes: 68 * G + 8 * P,
+    "tile_sort": lambda G, P, tile_passes: tile_passes * 20 * P,
+}
 ALU_KERNELS = ("render_fwd", "render_bwd")
 
 # DRAM traffic per launch of render_bwd measured by ncu
@@ -96,6 +108,14 @@ ALU_KERNELS = ("render_fwd", "render_bwd")
 # Taken on one frame of this workload (camera 0, 644,012 pairs): 42,377,472 B
 # read + 296,192 B written; scaled to a launch by its pair count.
 TRAFFIC = {"render_bwd": {"src_sha": "6ad9fbf35209d3d0", "bytes_per_pair": 66.262}}
+
+
+def _binning_used(choice, max_pairs, spec) -> str:
+    """The strategy gs_bin_and_sort takes (the automatic rule of include/gs.h)."""
+    if choice != "auto":
+        return choice
+    tiles = ((spec.width + 15) // 16) * ((spec.height + 15) // 16)
+    return "auto: " + ("global" if max_pairs >= 1024 * tiles and spec.n <= max_pairs else "per-tile")
 
 
 def _peaks():
@@ -218,6 +238,10 @@ VARIANT_FLAGS = {"3dgs": 0,
                  "3dgs-depth": 64}                # a fourth channel: blended camera depth
 
 
+# gs_bins.strategy (GS_BIN_* in include/gs.h): the same pairs either way
+BINNING = {"auto": 0, "per-tile": 1, "global": 2}
+
+
 def _cameras(spec, args):
     cams = make_cameras(spec)
     for c in cams:
@@ -259,7 +283,7 @@ def run_reference(args, spec, rank, world):
     print(json.dumps(out), flush=True)
 
 
-def _config(spec, pairs, tiles, graphs=True, variant="3dgs"):
+def _config(spec, pairs, tiles, graphs=True, variant="3dgs", binning="auto"):
     return {"workload": spec.name, "n_gaussians": spec.n, "width": spec.width, "height": spec.height,
             "variant": variant,
             "focal": spec.focal, "cameras": f"{spec.n_cameras} {spec.cameras}", "pairs_per_frame": pairs,
@@ -267,6 +291,7 @@ def _config(spec, pairs, tiles, graphs=True, variant="3dgs"):
                       else "3-sigma rectangle"),
             "l2": "flushed between timed steps (256 MB write outside the timed events)",
             "launch": "one CUDA graph per camera, replayed" if graphs else "eager launches",
+            "binning": binning,
             "parallelism": "replicas (cameras split across ranks)"}
 
 
@@ -337,7 +362,8 @@ def run_native(args, spec, rank, world, local):
         r.forward(c, P, sync=True)
         pairs.append(r.n_pairs)
         stats.append(G.gs_render_stats(c, n, r.proj, r.bins, r.last))
-    bins = G.Bins(n, int(max(pairs) * 1.05) + 4096, spec.width, spec.height, device=dev)
+    bins = G.Bins(n, int(max(pairs) * 1.05) + 4096, spec.width, spec.height, device=dev,
+                  strategy=BINNING[args.binning])
     proj = r.proj
     H, W = spec.height, spec.width
     image = torch.empty((H, W, nc), device=dev)
@@ -595,7 +621,15 @@ def run_native(args, spec, rank, world, local):
     for name, (launches, ms) in (prof or {}).items():
         gpu_launches += launches
         entry = {"launches": launches, "ms_total": ms, "ms_per_step": ms / args.steps}
-        if name in BYTES:
+        global_path = "global" in _binning_used(args.binning, bins.max_pairs, spec)
+        tiles_n = ((spec.width + 15) // 16) * ((spec.height + 15) // 16)
+        tile_passes = 1 if tiles_n <= 256 else (2 if tiles_n <= 65536 else 3)
+        if global_path and name in BYTES_GLOBAL:
+            per_step = [BYTES_GLOBAL[name](n, pairs[i], tile_passes) for i in sel]
+            total_bytes = sum(per_step)
+            ach = total_bytes / (ms * 1e-3) / 1e9
+            entry.update(bound="hbm", achieved=ach, peak=hbm_peak, unit="GB/s", frac=ach / hbm_peak)
+        elif name in BYTES:
             per_step = [BYTES[name](n, pairs[i]) for i in sel]
             total_bytes = sum(per_step)
             ach = total_bytes / (ms * 1e-3) / 1e9
@@ -676,7 +710,8 @@ def run_native(args, spec, rank, world, local):
         "vs_baseline": None,
         "dtype": "f32",
         "data": "synthetic",
-        "config": _config(spec, int(mean_pairs), args.tiles, not args.no_graphs, args.variant),
+        "config": _config(spec, int(mean_pairs), args.tiles, not args.no_graphs, args.variant,
+                          _binning_used(args.binning, bins.max_pairs, spec)),
         "fwd_frames_per_s": frames / (fwd_ms * 1e-3),
         "fwd_ms_per_frame": fwd_ms / args.steps,
         "tile_pairs_per_s": mean_pairs * frames / (fwd_ms * 1e-3),
@@ -717,6 +752,8 @@ def main():
                     help="tile rectangles: 3-sigma narrowed by the opacity-aware cut, or plain 3-sigma")
     ap.add_argument("--variant", choices=sorted(VARIANT_FLAGS), default="3dgs",
                     help="the method's conventions: 3DGS (default), gsplat, gsplat with antialiasing, or 3DGS with a depth channel")
+    ap.add_argument("--binning", choices=sorted(BINNING), default="auto",
+                    help="binning strategy: automatic, per-tile sorts, or one depth sort and tile radix passes")
     ap.add_argument("--profile-frame", action="store_true",
                     help="run one eager frame of one camera and exit (for ncu); prints no bench line")
     ap.add_argument("--profile-camera", type=int, default=0)

@@ -24,7 +24,7 @@ import ctypes
 import torch
 
 from . import _abi
-from ._abi import (GS_ERR_ALIGNMENT, GS_ERR_CAPACITY, GS_ERR_CUDA, GS_ERR_DEVICE_TIMEOUT,  # noqa: F401
+from ._abi import (GS_BIN_AUTO, GS_BIN_GLOBAL, GS_BIN_PER_TILE, GS_ERR_ALIGNMENT, GS_ERR_CAPACITY, GS_ERR_CUDA, GS_ERR_DEVICE_TIMEOUT,  # noqa: F401
                    GS_ERR_INVALID_ARG, GS_ERR_TOO_LARGE, GS_FLAG_ANTIALIASED, GS_FLAG_CAP_0999, GS_FLAG_DEPTH,
                    GS_FLAG_RADII_AXIS, GS_FLAG_RADII_OPACITY, GS_FLAG_STOP_INCLUSIVE, GS_FLAG_TIGHT_TILES, GS_OK,
                    GS_TILE)
@@ -134,9 +134,11 @@ class Projected(_Carved):
 
 
 class Bins(_Carved):
-    """gs_bins for at most n Gaussians, max_pairs pairs, a width x height image."""
+    """gs_bins for at most n Gaussians, max_pairs pairs, a width x height image.
+    strategy: GS_BIN_AUTO (default), GS_BIN_PER_TILE or GS_BIN_GLOBAL (the
+    same result; see include/gs.h)."""
 
-    def __init__(self, n: int, max_pairs: int, width: int, height: int, device="cuda"):
+    def __init__(self, n: int, max_pairs: int, width: int, height: int, device="cuda", strategy: int = 0):
         self.n, self.max_pairs = int(n), int(max_pairs)
         self.width, self.height = int(width), int(height)
         nbytes = int(lib().gs_bins_bytes(self.n, self.max_pairs, self.width, self.height))
@@ -146,6 +148,7 @@ class Bins(_Carved):
         self.struct = _abi.GsBins()
         _check(lib().gs_bins_carve(ctypes.c_void_p(self.buffer.data_ptr()), self.n, self.max_pairs,
                                    self.width, self.height, ctypes.byref(self.struct)), "gs_bins_carve")
+        self.struct.strategy = int(strategy)
         tiles = int(self.struct.max_tiles)
         self.tiles = tiles
         self.pair_tile = self._view(self.struct.pair_tile, self.max_pairs, torch.int32, (self.max_pairs,))

@@ -27,6 +27,9 @@ GS_FLAG_CAP_0999 = 8
 GS_FLAG_RADII_AXIS = 16
 GS_FLAG_RADII_OPACITY = 32
 GS_FLAG_DEPTH = 64
+GS_BIN_AUTO = 0
+GS_BIN_PER_TILE = 1
+GS_BIN_GLOBAL = 2
 
 c_float_p = ctypes.c_void_p  # device pointers travel as plain addresses
 
@@ -62,7 +65,7 @@ class GsBins(ctypes.Structure):
         ("pair_tile", ctypes.c_void_p), ("pair_gid", ctypes.c_void_p), ("ranges", ctypes.c_void_p),
         ("n_pairs", ctypes.c_void_p), ("status", ctypes.c_void_p),
         ("max_pairs", ctypes.c_int64), ("max_n", ctypes.c_int64),
-        ("max_tiles", ctypes.c_int32), ("reserved", ctypes.c_int32),
+        ("max_tiles", ctypes.c_int32), ("strategy", ctypes.c_int32),
         ("scratch", ctypes.c_void_p), ("scratch_bytes", ctypes.c_size_t),
     ]
 

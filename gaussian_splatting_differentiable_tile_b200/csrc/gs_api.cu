@@ -88,6 +88,7 @@ int check_bins(const gs_bins *b, int64_t n, const CamConst &c, BinsLayout *L) {
     if (n > b->max_n || (int64_t)c.tiles_x * c.tiles_y > b->max_tiles) return GS_ERR_INVALID_ARG;
     if (b->max_n < 0 || b->max_pairs < 0 || b->max_n > kMaxCount || b->max_pairs > kMaxCount)
         return GS_ERR_TOO_LARGE;
+    if (b->strategy < GS_BIN_AUTO || b->strategy > GS_BIN_GLOBAL) return GS_ERR_INVALID_ARG;
     *L = bins_layout(b->max_n, b->max_pairs, b->max_tiles);
     if (b->scratch_bytes < L->total || !aligned(b->scratch, 256)) return GS_ERR_INVALID_ARG;
     return GS_OK;

@@ -37,10 +37,15 @@ struct CamConst {
     float t_stop;       // a pixel stops once T (1 - alpha) < t_stop
 };
 
+// LSD passes of the global binning path: four over the depth bits, up to
+// three over the tile id (8 bits each); each has 256 digit totals.
+constexpr int kLsdMaxPasses = 7;
+
 // Byte layout of a gs_bins buffer.  The first `zero_bytes` bytes are cleared
 // by one memset at the start of every gs_bin_and_sort.
 struct BinsLayout {
     size_t status, n_pairs;     // the status word and K
+    size_t lsd_totals;          // [kLsdMaxPasses][256] digit totals of the global path
     size_t zero_bytes;
     size_t tile_total;          // [max_tiles] pairs per tile
     size_t ranges;              // [max_tiles][2]
@@ -60,6 +65,7 @@ constexpr BinsLayout bins_layout(int64_t max_n, int64_t max_pairs, int32_t max_t
     size_t off = 0;
     L.status = off;       off += 8;
     L.n_pairs = off;      off += 8;
+    L.lsd_totals = off;   off += (size_t)kLsdMaxPasses * 256 * sizeof(uint32_t);
     off = align_up(off, 256);
     L.zero_bytes = off;
     const size_t tb = align_up((size_t)max_tiles * sizeof(uint32_t), 256);

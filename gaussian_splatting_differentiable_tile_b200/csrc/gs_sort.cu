@@ -538,6 +538,277 @@ k_tile_sort(const uint32_t *__restrict__ ranges, const uint32_t *__restrict__ or
     }
 }
 
+// ---------------------------------------------------------------------
+// Global binning, for frames whose tile lists are long (a thousand entries
+// and more: 400k Gaussians at 1960 x 1090 give more than 2^24 pairs, about
+// 2 500 per tile), where sorting each tile's list on its own costs
+// L log L per tile.  The same unique order is reached with linear passes:
+//   k_depth_init + LSD passes   the Gaussians ordered by the float bits of
+//                               their depth (stable, so ties stay in id
+//                               order); Gaussians without tiles last
+//   k_rank_sums, k_rank_offsets the first pair position of each Gaussian in
+//                               that order: an exclusive scan of its tile count
+//   k_emit_ranked               every Gaussian writes (tile, id) for the tiles
+//                               of its rectangle at its position, so the pair
+//                               list comes out in (depth, id) order and is
+//                               written contiguously
+//   LSD passes on the tile id   stable, 8 bits each: the pairs grouped by
+//                               tile, the (depth, id) order kept inside every
+//                               tile; the last pass writes pair_tile and
+//                               pair_gid
+// An LSD pass is a histogram kernel (counts per CTA and digit, and the
+// digit totals by atomics) and a scatter kernel (each CTA finds its offsets
+// from the counts of the CTAs before it and the digit totals, then ranks its
+// elements in order with warp ballots).  No kernel waits on another CTA.
+// The tile ranges, K, the capacity check and the tile order come from the
+// count kernels above, as on the per-tile path.
+
+constexpr int kLsdThreads = 512;
+constexpr int kLsdWarps = kLsdThreads / 32;
+
+// The elements [lo, hi) of this CTA when `count` elements are split among
+// the grid's CTAs in contiguous chunks.
+__device__ __forceinline__ void lsd_chunk(uint64_t count, uint32_t &lo, uint32_t &hi) {
+    const uint64_t chunk = (count + gridDim.x - 1) / gridDim.x;
+    lo = (uint32_t)min((uint64_t)blockIdx.x * chunk, count);
+    hi = (uint32_t)min((uint64_t)lo + chunk, count);
+}
+
+// The Gaussians' sort keys: the float bits of the depth (positive, so their
+// order is the depth order) for Gaussians that touch a tile, all ones for
+// the others; values: the ids.
+__global__ void __launch_bounds__(256)
+k_depth_init(int n, const int4 *__restrict__ rect, const float4 *__restrict__ xyod, int tiles_x, int tiles_y,
+             uint32_t *__restrict__ keys, uint32_t *__restrict__ vals, const int32_t *__restrict__ status) {
+    if (*(volatile const int32_t *)status != 0) return;
+    const int g = blockIdx.x * blockDim.x + threadIdx.x;
+    if (g >= n) return;
+    int x0, y0, w;
+    const uint32_t c = rect_tiles(rect[g], tiles_x, tiles_y, x0, y0, w);
+    keys[g] = c ? __float_as_uint(xyod[g].w) : 0xFFFFFFFFu;
+    vals[g] = (uint32_t)g;
+}
+
+// Counts of the digit (key >> shift) & 255 over this CTA's chunk, into
+// H[CTA][256], and their totals over all CTAs into D[256] (zeroed by the
+// call's memset).  The element count is *count_dev when given (K), else
+// count_host.
+__global__ void __launch_bounds__(kLsdThreads)
+k_lsd_hist(const uint32_t *__restrict__ keys, const uint64_t *__restrict__ count_dev, uint32_t count_host,
+           int shift, uint32_t *__restrict__ H, uint32_t *__restrict__ D, const int32_t *__restrict__ status) {
+    __shared__ uint32_t s_h[kLsdWarps][kRadix];
+    if (*(volatile const int32_t *)status != 0) return;
+    const int warp = threadIdx.x >> 5;
+    for (int i = threadIdx.x; i < kLsdWarps * kRadix; i += kLsdThreads) (&s_h[0][0])[i] = 0;
+    __syncthreads();
+    uint32_t lo, hi;
+    lsd_chunk(count_dev ? *count_dev : count_host, lo, hi);
+    for (uint32_t i = lo + threadIdx.x; i < hi; i += kLsdThreads)
+        atomicAdd(&s_h[warp][(keys[i] >> shift) & 0xFFu], 1u);
+    __syncthreads();
+    for (int d = threadIdx.x; d < kRadix; d += kLsdThreads) {
+        uint32_t t = 0;
+#pragma unroll
+        for (int w = 0; w < kLsdWarps; w++) t += s_h[w][d];
+        H[(size_t)blockIdx.x * kRadix + d] = t;
+        if (t) atomicAdd(&D[d], t);
+    }
+}
+
+// Exclusive scan of 256 values in shared memory by the first 256 threads
+// (the others only meet the barriers).  Returns the total in *total when
+// given.
+__device__ __forceinline__ void scan256(uint32_t *v, uint32_t *s_w) {
+    const int t = threadIdx.x, lane = t & 31, w = t >> 5;
+    uint32_t x = 0, y = 0;
+    if (t < kRadix) {
+        x = v[t];
+        y = x;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+            const uint32_t z = __shfl_up_sync(0xffffffffu, y, o);
+            if (lane >= o) y += z;
+        }
+        if (lane == 31) s_w[w] = y;
+    }
+    __syncthreads();
+    if (t < kRadix) {
+        uint32_t base = 0;
+        for (int k = 0; k < w; k++) base += s_w[k];
+        v[t] = base + y - x;
+    }
+    __syncthreads();
+}
+
+// Stable scatter of one LSD pass: element i of this CTA's chunk goes to
+// (digit offset) + (its digit's count in the CTAs before this one) + (its
+// rank among the chunk's elements of that digit, in order).
+__global__ void __launch_bounds__(kLsdThreads)
+k_lsd_scatter(const uint32_t *__restrict__ keys_in, const uint32_t *__restrict__ vals_in,
+              const uint64_t *__restrict__ count_dev, uint32_t count_host, int shift,
+              const uint32_t *__restrict__ H, const uint32_t *__restrict__ D, uint32_t *__restrict__ keys_out,
+              uint32_t *__restrict__ vals_out, const int32_t *__restrict__ status) {
+    __shared__ uint32_t s_base[kRadix], s_tot[kRadix], s_w[kLsdWarps];
+    __shared__ uint32_t s_wc[kLsdWarps][kRadix];
+    if (*(volatile const int32_t *)status != 0) return;
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    if (tid < kRadix) {
+        uint32_t pre = 0;
+        for (int c = 0; c < (int)blockIdx.x; c++) pre += H[(size_t)c * kRadix + tid];
+        s_base[tid] = pre;
+        s_tot[tid] = D[tid];
+    }
+    __syncthreads();
+    scan256(s_tot, s_w);  // digit offsets
+    if (tid < kRadix) s_base[tid] += s_tot[tid];
+    __syncthreads();
+    uint32_t lo, hi;
+    lsd_chunk(count_dev ? *count_dev : count_host, lo, hi);
+    for (uint32_t c0 = lo; c0 < hi; c0 += kLsdThreads) {
+        const uint32_t i = c0 + tid;
+        const bool in = i < hi;
+        const uint32_t key = in ? keys_in[i] : 0u, val = in ? vals_in[i] : 0u;
+        const uint32_t d = in ? (key >> shift) & 0xFFu : (uint32_t)kRadix;
+        for (int k = tid; k < kLsdWarps * kRadix; k += kLsdThreads) (&s_wc[0][0])[k] = 0;
+        __syncthreads();
+        const uint32_t peers = digit_peers(d, 8);
+        if (in && lane == __ffs(peers) - 1) s_wc[warp][d] = __popc(peers);
+        __syncthreads();
+        if (tid < kRadix) {  // exclusive over warps, per digit
+            uint32_t acc = 0;
+#pragma unroll
+            for (int ww = 0; ww < kLsdWarps; ww++) {
+                const uint32_t cc = s_wc[ww][tid];
+                s_wc[ww][tid] = acc;
+                acc += cc;
+            }
+            s_tot[tid] = acc;
+        }
+        __syncthreads();
+        if (in) {
+            const uint32_t pos = s_base[d] + s_wc[warp][d] + __popc(peers & lanemask_lt());
+            keys_out[pos] = key;
+            vals_out[pos] = val;
+        }
+        __syncthreads();
+        if (tid < kRadix) s_base[tid] += s_tot[tid];
+        __syncthreads();
+    }
+}
+
+// Per-CTA sums of the tile counts of the Gaussians in depth order (rank r:
+// Gaussian order[r]), over contiguous chunks of ranks.
+__device__ __forceinline__ uint32_t ranked_count(const int4 *__restrict__ rect, const uint32_t *__restrict__ order,
+                                                 uint32_t r, int tiles_x, int tiles_y) {
+    int x0, y0, w;
+    return rect_tiles(rect[order[r]], tiles_x, tiles_y, x0, y0, w);
+}
+
+__device__ __forceinline__ uint32_t block_sum_512(uint32_t v, uint32_t *s_w) {
+    const int lane = threadIdx.x & 31, w = threadIdx.x >> 5;
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+    if (lane == 0) s_w[w] = v;
+    __syncthreads();
+    uint32_t t = 0;
+#pragma unroll
+    for (int k = 0; k < kLsdWarps; k++) t += s_w[k];
+    __syncthreads();
+    return t;
+}
+
+__global__ void __launch_bounds__(kLsdThreads)
+k_rank_sums(int n, const int4 *__restrict__ rect, const uint32_t *__restrict__ order, int tiles_x, int tiles_y,
+            uint32_t *__restrict__ S, const int32_t *__restrict__ status) {
+    __shared__ uint32_t s_w[kLsdWarps];
+    if (*(volatile const int32_t *)status != 0) return;
+    uint32_t lo, hi;
+    lsd_chunk((uint64_t)n, lo, hi);
+    uint32_t sum = 0;
+    for (uint32_t r = lo + threadIdx.x; r < hi; r += kLsdThreads) sum += ranked_count(rect, order, r, tiles_x, tiles_y);
+    sum = block_sum_512(sum, s_w);
+    if (threadIdx.x == 0) S[blockIdx.x] = sum;
+}
+
+// offsets[r] = pairs of the Gaussians ranked before r (exclusive scan).
+__global__ void __launch_bounds__(kLsdThreads)
+k_rank_offsets(int n, const int4 *__restrict__ rect, const uint32_t *__restrict__ order, int tiles_x, int tiles_y,
+               const uint32_t *__restrict__ S, uint32_t *__restrict__ offsets, const int32_t *__restrict__ status) {
+    __shared__ uint32_t s_w[kLsdWarps];
+    if (*(volatile const int32_t *)status != 0) return;
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    uint32_t base = 0;
+    for (int c = tid; c < (int)blockIdx.x; c += kLsdThreads) base += S[c];
+    base = block_sum_512(base, s_w);
+    uint32_t lo, hi;
+    lsd_chunk((uint64_t)n, lo, hi);
+    for (uint32_t c0 = lo; c0 < hi; c0 += kLsdThreads) {
+        const uint32_t r = c0 + tid;
+        const uint32_t v = r < hi ? ranked_count(rect, order, r, tiles_x, tiles_y) : 0u;
+        uint32_t y = v;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+            const uint32_t z = __shfl_up_sync(0xffffffffu, y, o);
+            if (lane >= o) y += z;
+        }
+        if (lane == 31) s_w[warp] = y;
+        __syncthreads();
+        uint32_t wbase = 0, total = 0;
+#pragma unroll
+        for (int k = 0; k < kLsdWarps; k++) {
+            const uint32_t x = s_w[k];
+            wbase += k < warp ? x : 0u;
+            total += x;
+        }
+        if (r < hi) offsets[r] = base + wbase + y - v;
+        base += total;
+        __syncthreads();
+    }
+}
+
+// Each Gaussian (rank r, id order[r]) writes the tile id and its id for
+// every tile of its rectangle, row by row, at offsets[r]: rectangles of at
+// most 16 tiles by their own lane, larger ones by the whole warp.
+__global__ void __launch_bounds__(256)
+k_emit_ranked(int n, const int4 *__restrict__ rect, const uint32_t *__restrict__ order,
+              const uint32_t *__restrict__ offsets, int tiles_x, int tiles_y, uint32_t *__restrict__ tile_out,
+              uint32_t *__restrict__ gid_out, const int32_t *__restrict__ status) {
+    if (*(volatile const int32_t *)status != 0) return;
+    const int lane = threadIdx.x & 31;
+    const int stride = gridDim.x * blockDim.x;
+    for (int r0 = blockIdx.x * blockDim.x + (threadIdx.x & ~31); r0 < n; r0 += stride) {
+        const int r = r0 + lane;
+        uint32_t g = 0, c = 0, off = 0;
+        int x0 = 0, y0 = 0, w = 1;
+        if (r < n) {
+            g = order[r];
+            c = rect_tiles(rect[g], tiles_x, tiles_y, x0, y0, w);
+            if (c) off = offsets[r];
+        }
+        if (c <= kLaneTiles) {
+            for (uint32_t k = 0; k < c; k++) {
+                const uint32_t dy = k / (uint32_t)w;
+                tile_out[off + k] = (uint32_t)((y0 + (int)dy) * tiles_x + x0 + (int)(k - dy * (uint32_t)w));
+                gid_out[off + k] = g;
+            }
+        }
+        uint32_t big = __ballot_sync(0xffffffffu, c > kLaneTiles);
+        while (big) {
+            const int src = __ffs(big) - 1;
+            big &= big - 1;
+            const uint32_t gb = __shfl_sync(0xffffffffu, g, src), cb = __shfl_sync(0xffffffffu, c, src);
+            const uint32_t ob = __shfl_sync(0xffffffffu, off, src);
+            const int xb = __shfl_sync(0xffffffffu, x0, src), yb = __shfl_sync(0xffffffffu, y0, src);
+            const uint32_t wb = (uint32_t)__shfl_sync(0xffffffffu, w, src);
+            for (uint32_t k = lane; k < cb; k += 32) {
+                const uint32_t dy = k / wb;
+                tile_out[ob + k] = (uint32_t)((yb + (int)dy) * tiles_x + xb + (int)(k - dy * wb));
+                gid_out[ob + k] = gb;
+            }
+        }
+    }
+}
+
 // Per-device launch set-up of the binning kernels, done once per device with
 // that device current: its SM count, and the dynamic shared memory the count,
 // emit and wide sort kernels may use beyond the default 48 KB (a function
@@ -576,6 +847,59 @@ cudaError_t device_setup(int *sms) {
 
 }  // namespace
 
+// The global path after the tile scan (see the kernels above).  ctas: CTAs
+// of the LSD, rank and emit kernels.
+cudaError_t launch_bin_global(const CamConst &c, int64_t n, const gs_projected &proj, const gs_bins &bins,
+                              const BinsLayout &L, int ctas, int sms, cudaStream_t s) {
+    char *base = static_cast<char *>(bins.scratch);
+    auto U32 = [&](size_t off) { return reinterpret_cast<uint32_t *>(base + off); };
+    const int32_t *status = reinterpret_cast<const int32_t *>(base + L.status);
+    const uint64_t *n_pairs = reinterpret_cast<const uint64_t *>(base + L.n_pairs);
+    uint32_t *D = U32(L.lsd_totals);
+    uint32_t *H = U32(L.bin_hist);
+    const size_t pb = align_up((size_t)bins.max_pairs * sizeof(uint32_t), 256);
+    uint32_t *KA = U32(L.keys), *VA = U32(L.keys + pb);  // the key array's two halves
+    uint32_t *KB = U32(L.long_keys), *VB = U32(L.long_ids);
+    const int4 *rect = reinterpret_cast<const int4 *>(proj.rect);
+    const float4 *xyod = reinterpret_cast<const float4 *>(proj.xy_opacity_depth);
+    const int tiles = c.tiles_x * c.tiles_y;
+    const uint32_t nn = (uint32_t)n;
+    // 4. the Gaussians by depth: four stable 8-bit passes, A -> B -> A -> B -> A
+    prof_before("depth_sort", s);
+    k_depth_init<<<(unsigned)((n + 255) / 256), 256, 0, s>>>((int)n, rect, xyod, c.tiles_x, c.tiles_y, KA, VA,
+                                                               status);
+    for (int p = 0; p < 4; p++) {
+        uint32_t *ki = p & 1 ? KB : KA, *vi = p & 1 ? VB : VA, *ko = p & 1 ? KA : KB, *vo = p & 1 ? VA : VB;
+        k_lsd_hist<<<ctas, kLsdThreads, 0, s>>>(ki, nullptr, nn, 8 * p, H, D + kRadix * p, status);
+        k_lsd_scatter<<<ctas, kLsdThreads, 0, s>>>(ki, vi, nullptr, nn, 8 * p, H, D + kRadix * p, ko, vo, status);
+    }
+    prof_after(s, 9);
+    // 5. each Gaussian's first pair position in depth order (into KA), then
+    // the pairs in (depth, id) order into (KB, VB)
+    prof_before("emit", s);
+    uint32_t *S = H;
+    k_rank_sums<<<ctas, kLsdThreads, 0, s>>>((int)n, rect, VA, c.tiles_x, c.tiles_y, S, status);
+    k_rank_offsets<<<ctas, kLsdThreads, 0, s>>>((int)n, rect, VA, c.tiles_x, c.tiles_y, S, KA, status);
+    const int emit_blocks = (int)std::min<int64_t>((n + 255) / 256, (int64_t)8 * sms);
+    k_emit_ranked<<<emit_blocks, 256, 0, s>>>((int)n, rect, VA, KA, c.tiles_x, c.tiles_y, KB, VB, status);
+    prof_after(s, 3);
+    // 6. stable passes over the tile id's 8-bit digits: B -> A -> B ..., the
+    // last into pair_tile / pair_gid
+    int passes = 1;
+    while (passes < 3 && (uint32_t)(tiles - 1) >> (8 * passes)) passes++;
+    prof_before("tile_sort", s);
+    for (int p = 0; p < passes; p++) {
+        const bool last = p == passes - 1;
+        uint32_t *ki = p & 1 ? KA : KB, *vi = p & 1 ? VA : VB;
+        uint32_t *ko = last ? bins.pair_tile : (p & 1 ? KB : KA), *vo = last ? bins.pair_gid : (p & 1 ? VB : VA);
+        k_lsd_hist<<<ctas, kLsdThreads, 0, s>>>(ki, n_pairs, 0u, 8 * p, H, D + kRadix * (4 + p), status);
+        k_lsd_scatter<<<ctas, kLsdThreads, 0, s>>>(ki, vi, n_pairs, 0u, 8 * p, H, D + kRadix * (4 + p), ko, vo,
+                                                   status);
+    }
+    prof_after(s, 2 * passes);
+    return cudaGetLastError();
+}
+
 cudaError_t launch_bin_and_sort(const CamConst &c, int64_t n, const gs_projected &proj,
                                 const gs_bins &bins, const BinsLayout &L, cudaStream_t s) {
     char *base = static_cast<char *>(bins.scratch);
@@ -610,6 +934,15 @@ cudaError_t launch_bin_and_sort(const CamConst &c, int64_t n, const gs_projected
                                                 n_pairs, status);
     prof_after(s);
     if (n == 0) return cudaGetLastError();  // K = 0, all ranges empty
+    // the global path's LSD passes keep per-CTA digit counts in the count
+    // matrix's space (free once the tile scan has run)
+    const int64_t hist_cap = std::min<int64_t>((int64_t)kBinCTAsMax * bins.max_tiles, kBinHistCap);
+    const int lsd_ctas = (int)std::min<int64_t>((int64_t)2 * sms, hist_cap / kRadix);
+    bool global = bins.strategy == GS_BIN_GLOBAL;
+    if (bins.strategy == GS_BIN_AUTO)
+        global = bins.max_pairs >= (int64_t)1024 * tiles;
+    global = global && n <= bins.max_pairs && lsd_ctas >= 1;
+    if (global) return launch_bin_global(c, n, proj, bins, L, lsd_ctas, sms, s);
     // 4. emit the sort keys
     prof_before("emit", s);
     k_bin_emit<<<ctas, kBinThreads, cnt_smem, s>>>((int)n, rect, reinterpret_cast<const float4 *>(proj.xy_opacity_depth),

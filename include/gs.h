@@ -184,10 +184,24 @@ typedef struct gs_bins {
     int64_t max_pairs;    /* capacity of pair_tile / pair_gid */
     int64_t max_n;        /* largest N this buffer was carved for */
     int32_t max_tiles;    /* largest tile count this buffer was carved for */
-    int32_t reserved;
+    int32_t strategy;     /* GS_BIN_*: how gs_bin_and_sort sorts (0, automatic,
+                             after gs_bins_carve); every strategy gives the same
+                             pairs, ranges and K */
     void *scratch;        /* sort and scan scratch (internal layout) */
     size_t scratch_bytes;
 } gs_bins;
+
+/* gs_bins.strategy.  GS_BIN_PER_TILE groups the pairs by tile through
+ * counts and scans and sorts every tile's list on its own by (depth bits,
+ * id); GS_BIN_GLOBAL orders the Gaussians by depth once, emits the pairs in
+ * that order and groups them by tile with stable radix passes over the tile
+ * id only; both give the order of the key (tile << 32 | depth bits) with
+ * ties by id.  GS_BIN_AUTO takes the global strategy when the capacity
+ * holds at least 1024 pairs per tile of the frame (long lists, where the
+ * per-tile sorts cost the most) and at least n, else the per-tile one. */
+#define GS_BIN_AUTO 0
+#define GS_BIN_PER_TILE 1
+#define GS_BIN_GLOBAL 2
 
 /* Bytes of one buffer holding a gs_bins for at most n Gaussians, max_pairs
  * pairs and a width x height image.  [PIX4] Lesson 2: 400k Gaussians at full

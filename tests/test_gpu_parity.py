@@ -79,8 +79,9 @@ def test_project_matches_oracle(scene, flags):
 
 
 # ---------------------------------------------------- bin and sort (stage-fed)
-def _check_bins(cam, rec, n, bins, K):
-    ob = O.bin_pairs(rec["rect"], rec["valid"], rec["depth32"], cam.width, cam.height)
+def _check_bins(cam, rec, n, bins, K, ob=None):
+    if ob is None:
+        ob = O.bin_pairs(rec["rect"], rec["valid"], rec["depth32"], cam.width, cam.height)
     assert K == ob["n_pairs"]
     tile = bins.pair_tile[:K].cpu().numpy().astype(np.uint32)
     gid = bins.pair_gid[:K].cpu().numpy().astype(np.uint32)
@@ -93,17 +94,22 @@ def _check_bins(cam, rec, n, bins, K):
     assert int(bins.status.item()) == 0
 
 
+STRATEGIES = [G.GS_BIN_PER_TILE, G.GS_BIN_GLOBAL]
+
+
+@pytest.mark.parametrize("strategy", STRATEGIES)
 @pytest.mark.parametrize("scene", list(SCENES))
-def test_bin_and_sort_bit_exact(scene):
+def test_bin_and_sort_bit_exact(scene, strategy):
     cam, params = SCENES[scene]()
     n = params["means"].shape[0]
     rec = oracle_records(params, cam)
     proj = fill_projected(rec, n)
-    bins, K = gpu_bin(cam, n, proj)
+    bins, K = gpu_bin(cam, n, proj, strategy=strategy)
     _check_bins(cam, rec, n, bins, K)
 
 
-def test_bin_and_sort_depth_ties_and_many_partitions():
+@pytest.mark.parametrize("strategy", STRATEGIES)
+def test_bin_and_sort_depth_ties_and_many_partitions(strategy):
     """Equal depth keys keep Gaussian-id order; N spans several sort and scan
     partitions with a ragged last one."""
     cam, params = _student_subset(30_000)
@@ -111,12 +117,13 @@ def test_bin_and_sort_depth_ties_and_many_partitions():
     rec = oracle_records(params, cam)
     rec["depth32"] = (np.round(rec["depth32"] * 4) / 4).astype(np.float32)
     proj = fill_projected(rec, n)
-    bins, K = gpu_bin(cam, n, proj)
+    bins, K = gpu_bin(cam, n, proj, strategy=strategy)
     _check_bins(cam, rec, n, bins, K)
 
 
+@pytest.mark.parametrize("strategy", STRATEGIES)
 @pytest.mark.parametrize("W,H", [(16, 16), (1, 1), (17, 1), (4112, 4112)])
-def test_bin_and_sort_tile_bit_widths(W, H):
+def test_bin_and_sort_tile_bit_widths(W, H, strategy):
     """One tile, 1 x 2 tiles, and 257 x 257 tiles (66049: the count matrix
     then takes fewer CTAs and rows longer than shared memory)."""
     cam = Camera(np.eye(4), W * 0.5, W * 0.5, W / 2.0, H / 2.0, W, H)
@@ -127,12 +134,13 @@ def test_bin_and_sort_tile_bit_widths(W, H):
               "opacity_logits": rng.normal(0, 1, n), "colors": rng.uniform(0, 1, (n, 3))}
     rec = oracle_records(params, cam)
     proj = fill_projected(rec, n)
-    bins, K = gpu_bin(cam, n, proj, max_pairs=int(rec["count"].sum()) + 16)
+    bins, K = gpu_bin(cam, n, proj, max_pairs=max(int(rec["count"].sum()), n) + 16, strategy=strategy)
     _check_bins(cam, rec, n, bins, K)
 
 
+@pytest.mark.parametrize("strategy", STRATEGIES)
 @pytest.mark.parametrize("n", [900, 5000, 20000])
-def test_bin_and_sort_long_tile_lists(n):
+def test_bin_and_sort_long_tile_lists(n, strategy):
     """Every Gaussian covers the few tiles of a 48 x 32 image, so each tile's
     list has about n entries: the shared-memory sort of short and of long
     lists, and the global-memory sort beyond 16384 entries; a quarter of the
@@ -146,19 +154,20 @@ def test_bin_and_sort_long_tile_lists(n):
     tie = rng.random(n) < 0.25
     rec["depth32"] = np.where(tie, np.float32(3.0), rec["depth32"]).astype(np.float32)
     proj = fill_projected(rec, n)
-    bins, K = gpu_bin(cam, n, proj, max_pairs=int(rec["count"].sum()) + 16)
+    bins, K = gpu_bin(cam, n, proj, max_pairs=int(rec["count"].sum()) + 16, strategy=strategy)
     r = bins.ranges.cpu().numpy()[:cam.tiles]
     assert (r[:, 1] - r[:, 0]).max() > 0.8 * n
     _check_bins(cam, rec, n, bins, K)
 
 
-def test_bin_and_sort_capacity_error_and_async_status():
+@pytest.mark.parametrize("strategy", STRATEGIES)
+def test_bin_and_sort_capacity_error_and_async_status(strategy):
     cam, params = SCENES["tiny"]()
     n = params["means"].shape[0]
     rec = oracle_records(params, cam)
     need = int(rec["count"].sum())
     proj = fill_projected(rec, n)
-    bins = G.Bins(n, need - 1, cam.width, cam.height)
+    bins = G.Bins(n, need - 1, cam.width, cam.height, strategy=strategy)
     with pytest.raises(G.GSError) as ei:
         G.gs_bin_and_sort(cam, n, proj, bins, sync=True)
     assert ei.value.code == G.GS_ERR_CAPACITY and ei.value.n_pairs == need

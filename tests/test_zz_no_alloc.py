@@ -27,7 +27,8 @@ def _project(cam, params):
 
 
 def _reference(cam, proj, n):
-    bins = G.Bins(n, 64 * n + cam.tiles + 4096, cam.width, cam.height)
+    need = int(proj.count[:n].sum().item()) if n else 0
+    bins = G.Bins(n, max(64 * n, need) + cam.tiles + 4096, cam.width, cam.height)
     K = G.gs_bin_and_sort(cam, n, proj, bins)
     return (K, bins.pair_tile[:K].cpu().numpy(), bins.pair_gid[:K].cpu().numpy(),
             bins.ranges.cpu().numpy()[:cam.tiles])
