@@ -10,7 +10,9 @@ import ctypes
 import os
 
 HERE = os.path.dirname(os.path.abspath(__file__))
-LIB_PATH = os.path.join(HERE, "libgs.so")
+# GS_LIBRARY names the library file beside this module: libgs.so, or the
+# checked build libgs_check.so
+LIB_PATH = os.path.join(HERE, os.environ.get("GS_LIBRARY", "libgs.so"))
 
 GS_TILE = 16
 GS_OK = 0
@@ -20,6 +22,7 @@ GS_ERR_TOO_LARGE = -3
 GS_ERR_ALIGNMENT = -4
 GS_ERR_CUDA = -5
 GS_ERR_DEVICE_TIMEOUT = -6
+GS_ERR_BOUNDS = -7
 GS_FLAG_TIGHT_TILES = 1
 GS_FLAG_ANTIALIASED = 2
 GS_FLAG_STOP_INCLUSIVE = 4

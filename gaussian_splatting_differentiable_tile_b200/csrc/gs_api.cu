@@ -152,6 +152,7 @@ const char *gs_error_string(int code) {
         case GS_ERR_ALIGNMENT: return "pointer not aligned as documented";
         case GS_ERR_CUDA: return "CUDA runtime call or kernel launch failed";
         case GS_ERR_DEVICE_TIMEOUT: return "a bounded device-side wait gave up";
+        case GS_ERR_BOUNDS: return "a kernel index was out of range and its access skipped (checked build)";
         default: return "unknown error code";
     }
 }
@@ -263,7 +264,7 @@ int gs_render_fwd(const gs_camera *cam, int64_t n, const gs_projected *proj, con
     if ((rc = check_projected(proj, n)) || (rc = check_bins(bins, n, c, &L))) return rc;
     if (!image || !T_final || !last) return GS_ERR_INVALID_ARG;
     if (!aligned(image, 4) || !aligned(T_final, 4) || !aligned(last, 4)) return GS_ERR_ALIGNMENT;
-    return launch_render_fwd(c, *proj, *bins, image, T_final, last, as_stream(stream)) == cudaSuccess
+    return launch_render_fwd(c, n, *proj, *bins, image, T_final, last, as_stream(stream)) == cudaSuccess
                ? GS_OK
                : GS_ERR_CUDA;
 }
@@ -290,7 +291,7 @@ int gs_render_bwd(const gs_camera *cam, int64_t n, const gs_params *params,
     cudaStream_t s = as_stream(stream);
     if (n > 0 && cudaMemsetAsync(grad2d, 0, (size_t)n * 12 * sizeof(float), s) != cudaSuccess)
         return GS_ERR_CUDA;
-    if (launch_render_bwd(c, *proj, *bins, T_final, last, dL_dimage, grad2d, s) != cudaSuccess)
+    if (launch_render_bwd(c, n, *proj, *bins, T_final, last, dL_dimage, grad2d, s) != cudaSuccess)
         return GS_ERR_CUDA;
     if (launch_project_bwd(c, n, *params, *proj, grad2d, *grads, s) != cudaSuccess) return GS_ERR_CUDA;
     return GS_OK;
@@ -310,7 +311,7 @@ int gs_render_features_fwd(const gs_camera *cam, int64_t n, const gs_projected *
     BinsLayout L;
     if ((rc = check_projected(proj, n)) || (rc = check_bins(bins, n, c, &L))) return rc;
     if (!aligned(features, 16) || !aligned(out, 4)) return GS_ERR_ALIGNMENT;
-    return launch_render_features_fwd(c, *proj, *bins, features, F, out, as_stream(stream)) == cudaSuccess
+    return launch_render_features_fwd(c, n, *proj, *bins, features, F, out, as_stream(stream)) == cudaSuccess
                ? GS_OK
                : GS_ERR_CUDA;
 }
@@ -339,7 +340,7 @@ int gs_render_features_bwd(const gs_camera *cam, int64_t n, const gs_params *par
     if (cudaMemsetAsync(grad2d, 0, (size_t)n * 12 * sizeof(float), s) != cudaSuccess ||
         cudaMemsetAsync(dL_dfeatures, 0, (size_t)n * F * sizeof(float), s) != cudaSuccess)
         return GS_ERR_CUDA;
-    if (launch_render_features_bwd(c, *proj, *bins, T_final, last, features, F, dL_dout, grad2d, dL_dfeatures,
+    if (launch_render_features_bwd(c, n, *proj, *bins, T_final, last, features, F, dL_dout, grad2d, dL_dfeatures,
                                    s) != cudaSuccess)
         return GS_ERR_CUDA;
     // the features' share of dL/d(mean2d, conic, opacity), added into grads
@@ -357,7 +358,7 @@ int gs_render_stats(const gs_camera *cam, int64_t n, const gs_projected *proj, c
     if ((rc = check_projected(proj, n)) || (rc = check_bins(bins, n, c, &L))) return rc;
     if (!last || !counts) return GS_ERR_INVALID_ARG;
     if (!aligned(last, 4) || !aligned(counts, 8)) return GS_ERR_ALIGNMENT;
-    return launch_render_stats(c, *proj, *bins, last, counts, as_stream(stream)) == cudaSuccess
+    return launch_render_stats(c, n, *proj, *bins, last, counts, as_stream(stream)) == cudaSuccess
                ? GS_OK
                : GS_ERR_CUDA;
 }
@@ -526,14 +527,14 @@ int gs_train_step(const gs_camera *cams, int32_t n_cams, int64_t n, const gs_par
             const gs_params &pp = pc;
             if (launch_project(c, n, pp, ln.proj, ls) != cudaSuccess ||
                 launch_bin_and_sort(c, n, ln.proj, ln.bins, L[l], ls) != cudaSuccess ||
-                launch_render_fwd(c, ln.proj, ln.bins, ln.image, ln.T_final, ln.last, ls) != cudaSuccess ||
+                launch_render_fwd(c, n, ln.proj, ln.bins, ln.image, ln.T_final, ln.last, ls) != cudaSuccess ||
                 launch_l1_train(ln.image, targets + (size_t)b * values, values, ln.dL_dimage,
                                 losses ? losses + b : nullptr, ln.bins, cam_stats ? cam_stats + 2 * b : nullptr,
                                 ls) != cudaSuccess)
                 return GS_ERR_CUDA;
             if (n > 0 && cudaMemsetAsync(ln.grad2d, 0, (size_t)n * 12 * sizeof(float), ls) != cudaSuccess)
                 return GS_ERR_CUDA;
-            if (launch_render_bwd(c, ln.proj, ln.bins, ln.T_final, ln.last, ln.dL_dimage, ln.grad2d, ls) !=
+            if (launch_render_bwd(c, n, ln.proj, ln.bins, ln.T_final, ln.last, ln.dL_dimage, ln.grad2d, ls) !=
                     cudaSuccess ||
                 launch_project_bwd(c, n, pp, ln.proj, ln.grad2d, ln.grads, ls, b >= n_lanes) != cudaSuccess)
                 return GS_ERR_CUDA;

@@ -37,15 +37,10 @@ struct CamConst {
     float t_stop;       // a pixel stops once T (1 - alpha) < t_stop
 };
 
-// LSD passes of the global binning path: four over the depth bits, up to
-// three over the tile id (8 bits each); each has 256 digit totals.
-constexpr int kLsdMaxPasses = 7;
-
 // Byte layout of a gs_bins buffer.  The first `zero_bytes` bytes are cleared
 // by one memset at the start of every gs_bin_and_sort.
 struct BinsLayout {
     size_t status, n_pairs;     // the status word and K
-    size_t lsd_totals;          // [kLsdMaxPasses][256] digit totals of the global path
     size_t zero_bytes;
     size_t tile_total;          // [max_tiles] pairs per tile
     size_t ranges;              // [max_tiles][2]
@@ -65,7 +60,6 @@ constexpr BinsLayout bins_layout(int64_t max_n, int64_t max_pairs, int32_t max_t
     size_t off = 0;
     L.status = off;       off += 8;
     L.n_pairs = off;      off += 8;
-    L.lsd_totals = off;   off += (size_t)kLsdMaxPasses * 256 * sizeof(uint32_t);
     off = align_up(off, 256);
     L.zero_bytes = off;
     const size_t tb = align_up((size_t)max_tiles * sizeof(uint32_t), 256);
@@ -111,6 +105,39 @@ __device__ __forceinline__ void set_status(int32_t *status, int32_t code) {
 }
 #endif
 
+// Checked builds (libgs_check.so, compiled with -DGS_CHECK) test the index of
+// every gather and scatter of the blend, binning and sort kernels against its
+// array's bound: an index out of range records GS_ERR_BOUNDS in the bins'
+// status word and the access is skipped (no trap).  Ordinary builds compile
+// the tests away.
+#ifdef GS_CHECK
+constexpr bool kCheck = true;
+#else
+constexpr bool kCheck = false;
+#endif
+// What a checked build tests kernel indices against.
+struct Bounds {
+    int32_t *status;  // where an index out of range is recorded
+    uint64_t n;       // Gaussians: records, gradients
+    uint64_t pairs;   // capacity of the pair list
+    uint32_t tiles;   // tiles of the frame
+};
+inline Bounds bounds_of(const gs_bins &b, int64_t n, int tiles) {
+    return Bounds{b.status, (uint64_t)n, (uint64_t)b.max_pairs, (uint32_t)tiles};
+}
+#ifdef __CUDACC__
+__device__ __forceinline__ bool in_bounds(uint64_t i, uint64_t bound, int32_t *status) {
+    if (!kCheck || i < bound) return true;
+    set_status(status, GS_ERR_BOUNDS);
+    return false;
+}
+// A tile's [start, end) lies inside the pair list.
+__device__ __forceinline__ bool range_in_bounds(uint2 r, const Bounds &bd) {
+    if (!kCheck) return true;
+    return in_bounds(r.x, (uint64_t)r.y + 1, bd.status) && in_bounds(r.y, bd.pairs + 1, bd.status);
+}
+#endif
+
 // Adam over the five parameter groups (gs_train.cu).
 constexpr int kAdamMaxSlots = 16;
 struct AdamGroup {
@@ -135,21 +162,21 @@ cudaError_t launch_project_bwd(const CamConst &c, int64_t n, const gs_params &p,
                                cudaStream_t s, bool accumulate = false);
 cudaError_t launch_bin_and_sort(const CamConst &c, int64_t n, const gs_projected &proj,
                                 const gs_bins &bins, const BinsLayout &L, cudaStream_t s);
-cudaError_t launch_render_fwd(const CamConst &c, const gs_projected &proj, const gs_bins &bins,
+cudaError_t launch_render_fwd(const CamConst &c, int64_t n, const gs_projected &proj, const gs_bins &bins,
                               float *image, float *T_final, uint32_t *last, cudaStream_t s);
-cudaError_t launch_render_bwd(const CamConst &c, const gs_projected &proj, const gs_bins &bins,
+cudaError_t launch_render_bwd(const CamConst &c, int64_t n, const gs_projected &proj, const gs_bins &bins,
                               const float *T_final, const uint32_t *last, const float *dL_dimage,
                               float *grad2d, cudaStream_t s);
 // Feature channels: F / 4 passes of the blend over chunks of four channels
 // (no background).  The backward adds the geometric sums into grad2d and
 // the feature gradients into dL_dfeatures (both zeroed by the caller).
-cudaError_t launch_render_features_fwd(const CamConst &c, const gs_projected &proj, const gs_bins &bins,
+cudaError_t launch_render_features_fwd(const CamConst &c, int64_t n, const gs_projected &proj, const gs_bins &bins,
                                        const float *features, int F, float *out, cudaStream_t s);
-cudaError_t launch_render_features_bwd(const CamConst &c, const gs_projected &proj, const gs_bins &bins,
+cudaError_t launch_render_features_bwd(const CamConst &c, int64_t n, const gs_projected &proj, const gs_bins &bins,
                                        const float *T_final, const uint32_t *last, const float *features,
                                        int F, const float *dL_dout, float *grad2d, float *dL_dfeatures,
                                        cudaStream_t s);
-cudaError_t launch_render_stats(const CamConst &c, const gs_projected &proj, const gs_bins &bins,
+cudaError_t launch_render_stats(const CamConst &c, int64_t n, const gs_projected &proj, const gs_bins &bins,
                                 const uint32_t *last, uint64_t *counts, cudaStream_t s);
 cudaError_t launch_l1(const float *image, const float *target, int64_t count, float *dL_dimage,
                       float *loss, cudaStream_t s);

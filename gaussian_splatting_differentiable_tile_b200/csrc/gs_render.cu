@@ -262,7 +262,8 @@ __global__ void __launch_bounds__(kTilePixels, GS_FWD_MINB)
 k_render_fwd(CamConst cam, const float4 *__restrict__ xyod, const float4 *__restrict__ conr,
              const ChannelIO io, const uint32_t *__restrict__ pair_gid,
              const uint2 *__restrict__ ranges, const uint32_t *__restrict__ order,
-             float *__restrict__ image, float *__restrict__ T_final, uint32_t *__restrict__ last) {
+             float *__restrict__ image, float *__restrict__ T_final, uint32_t *__restrict__ last,
+             const Bounds bd) {
     constexpr int kWarps = kTilePixels / 32;
     __shared__ float4 s_geo[kBatch];
     __shared__ float4 s_geo2[kBatch];
@@ -270,7 +271,9 @@ k_render_fwd(CamConst cam, const float4 *__restrict__ xyod, const float4 *__rest
     __shared__ uint8_t s_mask[kBatch];
     __shared__ FwdWarpBuf s_wb[kWarps];
 
-    const int tile = (int)order[blockIdx.x];  // longest lists first
+    const uint32_t tile_id = order[blockIdx.x];  // longest lists first
+    if (!in_bounds(tile_id, bd.tiles, bd.status)) return;
+    const int tile = (int)tile_id;
     const int tx = tile % cam.tiles_x, ty = tile / cam.tiles_x;
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
     const int px = tx * kTile + 8 * (warp & 1) + (lane & 7);
@@ -279,6 +282,7 @@ k_render_fwd(CamConst cam, const float4 *__restrict__ xyod, const float4 *__rest
     const float2 nfx = make_float2(-fx, -fx), nfy = make_float2(-fy, -fy);
     const float x0 = (float)(tx * kTile), y0 = (float)(ty * kTile);
     const uint2 range = ranges[tile];
+    if (!range_in_bounds(range, bd)) return;
     FwdWarpBuf &wb = s_wb[warp];
     const uint32_t lt_mask = (1u << lane) - 1u;
 
@@ -290,11 +294,12 @@ k_render_fwd(CamConst cam, const float4 *__restrict__ xyod, const float4 *__rest
         const uint32_t cnt = min((uint32_t)kBatch, range.y - b);
         if (threadIdx.x < cnt) {
             const uint32_t g = pair_gid[b + threadIdx.x];
-            float4 geo, geo2;
-            stage_entry(xyod[g], conr[g], geo, geo2);
+            const bool ok = in_bounds(g, bd.n, bd.status);  // checked builds: else a slot no warp walks
+            float4 geo = make_float4(0.f, 0.f, 0.f, 0.f), geo2 = make_float4(0.f, 0.f, 0.f, 0.f);
+            if (ok) stage_entry(xyod[g], conr[g], geo, geo2);
             s_geo[threadIdx.x] = geo;
-            s_col[threadIdx.x] = io.col[kFeat ? (size_t)g * io.col_stride : (size_t)g];
-            s_mask[threadIdx.x] = (uint8_t)block_mask(geo, geo2, x0, y0);
+            s_col[threadIdx.x] = ok ? io.col[kFeat ? (size_t)g * io.col_stride : (size_t)g] : geo;
+            s_mask[threadIdx.x] = ok ? (uint8_t)block_mask(geo, geo2, x0, y0) : (uint8_t)0;
             geo2.z = hit_center(geo2.y);  // kx, ky are only needed for the mask
             s_geo2[threadIdx.x] = geo2;
         }
@@ -482,7 +487,7 @@ k_render_bwd(CamConst cam, const float4 *__restrict__ xyod, const float4 *__rest
              const uint2 *__restrict__ ranges, const uint32_t *__restrict__ order,
              const float *__restrict__ T_final,
              const uint32_t *__restrict__ last, const float *__restrict__ dL_dimage,
-             float *__restrict__ grad2d) {
+             float *__restrict__ grad2d, const Bounds bd) {
     static_assert(kRPL % 2 == 0, "the backward works on pairs of rows");
     constexpr int kThreads = kTilePixels / kRPL;
     constexpr int kWarps = kThreads / 32;
@@ -496,9 +501,12 @@ k_render_bwd(CamConst cam, const float4 *__restrict__ xyod, const float4 *__rest
     __shared__ uint8_t s_list[kWarps][kB];
     __shared__ uint32_t s_max_last;
 
-    const int tile = (int)order[blockIdx.x];  // longest lists first
+    const uint32_t tile_id = order[blockIdx.x];  // longest lists first
+    if (!in_bounds(tile_id, bd.tiles, bd.status)) return;
+    const int tile = (int)tile_id;
     const LaneGeom L = lane_geom<kRPL>(cam, tile);
     const uint2 range = ranges[tile];
+    if (!range_in_bounds(range, bd)) return;
     const bool col_in = L.px < cam.width;
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
 
@@ -543,6 +551,15 @@ k_render_bwd(CamConst cam, const float4 *__restrict__ xyod, const float4 *__rest
     __syncthreads();
     const uint32_t max_last = s_max_last;
 
+    // Sums of an entry: the six geometric ones into grad2d, the channel sums
+    // after them (colours) or into io.cgrad (a feature chunk).
+    constexpr int kV = 6 + kC;
+    auto add_sums = [&](uint32_t g, int i, float x) {
+        float *dst = grad2d + 12 * (size_t)g + i;
+        if (kFeat && i >= 6) dst = io.cgrad + (size_t)io.cgrad_stride * g + (i - 6);
+        atomicAdd(dst, x);
+    };
+
     for (uint32_t bend = max_last; bend > range.x;) {
         const uint32_t bstart = bend - range.x > (uint32_t)kB ? bend - kB : range.x;
         const uint32_t cnt = bend - bstart;
@@ -551,8 +568,13 @@ k_render_bwd(CamConst cam, const float4 *__restrict__ xyod, const float4 *__rest
         // the dependent loads overlap
         for (uint32_t i0 = threadIdx.x; i0 < cnt; i0 += 2 * kThreads) {
             const uint32_t i1 = i0 + kThreads;
-            const uint32_t ga = pair_gid[bend - 1 - i0];
-            const uint32_t gb = i1 < cnt ? pair_gid[bend - 1 - i1] : ga;
+            uint32_t ga = pair_gid[bend - 1 - i0];
+            uint32_t gb = i1 < cnt ? pair_gid[bend - 1 - i1] : ga;
+            // checked builds: an id out of range is replaced by 0 and its slot
+            // never walked
+            const bool oka = in_bounds(ga, bd.n, bd.status), okb = i1 >= cnt || in_bounds(gb, bd.n, bd.status);
+            if (kCheck && !oka) ga = 0;
+            if (kCheck && !okb) gb = 0;
             const float4 xa = xyod[ga], ca = conr[ga], ra = io.col[kFeat ? (size_t)ga * io.col_stride : (size_t)ga];
             const float4 xb = xyod[gb], cb = conr[gb], rb = io.col[kFeat ? (size_t)gb * io.col_stride : (size_t)gb];
             float4 geo, geo2;
@@ -561,7 +583,7 @@ k_render_bwd(CamConst cam, const float4 *__restrict__ xyod, const float4 *__rest
             s_geo2[i0] = geo2;
             s_col[i0] = ra;
             s_gid[i0] = ga;
-            s_mask[i0] = (uint8_t)strip_mask<kWarps>(geo, geo2, L.sx, L.hx, L.sy0, 2.f * kRPL, L.hy);
+            s_mask[i0] = oka ? (uint8_t)strip_mask<kWarps>(geo, geo2, L.sx, L.hx, L.sy0, 2.f * kRPL, L.hy) : 0;
             s_geo2[i0].z = hit_center(geo2.y);
             if (i1 < cnt) {
                 stage_entry(xb, cb, geo, geo2);
@@ -569,7 +591,7 @@ k_render_bwd(CamConst cam, const float4 *__restrict__ xyod, const float4 *__rest
                 s_geo2[i1] = geo2;
                 s_col[i1] = rb;
                 s_gid[i1] = gb;
-                s_mask[i1] = (uint8_t)strip_mask<kWarps>(geo, geo2, L.sx, L.hx, L.sy0, 2.f * kRPL, L.hy);
+                s_mask[i1] = okb ? (uint8_t)strip_mask<kWarps>(geo, geo2, L.sx, L.hx, L.sy0, 2.f * kRPL, L.hy) : 0;
                 s_geo2[i1].z = hit_center(geo2.y);
             }
         }
@@ -614,7 +636,8 @@ k_render_bwd(CamConst cam, const float4 *__restrict__ xyod, const float4 *__rest
                 const bool h0 = hit[2 * i], h1 = hit[2 * i + 1];
                 const float e0 = ex2_approx(p[i].x), e1 = ex2_approx(p[i].y);
                 const float2 a = make_float2(h0 ? fminf(e0, cam.alpha_cap) : 0.f, h1 ? fminf(e1, cam.alpha_cap) : 0.f);
-                const bool cap0 = h0 && e0 > cam.alpha_cap, cap1 = h1 && e1 > cam.alpha_cap;
+                // alpha for the opacity and conic gradients: 0 where the cap applied
+                const float2 av = make_float2(e0 > cam.alpha_cap ? 0.f : a.x, e1 > cam.alpha_cap ? 0.f : a.y);
                 const float2 om = __fadd2_rn(make_float2(1.f, 1.f), make_float2(-a.x, -a.y));
                 const float2 ri = make_float2(rcp_approx(om.x), rcp_approx(om.y));
                 const float2 Ti = __fmul2_rn(T[i], ri);
@@ -629,9 +652,7 @@ k_render_bwd(CamConst cam, const float4 *__restrict__ xyod, const float4 *__rest
                 cr1 = __ffma2_rn(w, g1[i], cr1);
                 cr2 = __ffma2_rn(w, g2[i], cr2);
                 if (kDepth) cr3 = __ffma2_rn(w, g3[i], cr3);
-                float2 v = __fmul2_rn(dLda, a);  // dL/dsigma = -v, dL/do = v / o
-                v.x = cap0 ? 0.f : v.x;
-                v.y = cap1 ? 0.f : v.y;
+                const float2 v = __fmul2_rn(dLda, av);  // dL/dsigma = -v, dL/do = v / o
                 sv = __fadd2_rn(sv, v);
                 const float2 vy = __fmul2_rn(v, dy[i]);
                 sgy = __fadd2_rn(sgy, vy);
@@ -640,25 +661,20 @@ k_render_bwd(CamConst cam, const float4 *__restrict__ xyod, const float4 *__rest
             }
             const float svs = sv.x + sv.y, sgys = sgy.x + sgy.y;
             const float sgx = svs * ct.dx;
-            constexpr int kV = 6 + kC;
+            float vals[kV];
+            vals[0] = svs;
+            vals[1] = sgx;
+            vals[2] = sgys;
+            vals[3] = sgx * ct.dx;
+            vals[4] = sgys * ct.dx;
+            vals[5] = sgyy.x + sgyy.y;
+            vals[6] = cr0.x + cr0.y;
+            vals[7] = cr1.x + cr1.y;
+            vals[8] = cr2.x + cr2.y;
+            if (kDepth) vals[kV - 1] = cr3.x + cr3.y;
             int idx;
-            float tot;
-            if (kDepth) {
-                const float vals[10] = {svs, sgx, sgys, sgx * ct.dx, sgys * ct.dx, sgyy.x + sgyy.y,
-                                        cr0.x + cr0.y, cr1.x + cr1.y, cr2.x + cr2.y, cr3.x + cr3.y};
-                tot = reduce_scatter<10>(vals, lane, &idx);
-            } else {
-                const float vals[9] = {svs, sgx, sgys, sgx * ct.dx, sgys * ct.dx, sgyy.x + sgyy.y,
-                                       cr0.x + cr0.y, cr1.x + cr1.y, cr2.x + cr2.y};
-                tot = reduce_scatter<9>(vals, lane, &idx);
-            }
-            // the six geometric sums into grad2d; the channel sums follow them
-            // in grad2d (colours), or go to io.cgrad (a feature chunk)
-            if (idx < kV) {
-                float *dst = grad2d + 12 * (size_t)s_gid[k] + idx;
-                if (kFeat && idx >= 6) dst = io.cgrad + (size_t)io.cgrad_stride * s_gid[k] + (idx - 6);
-                atomicAdd(dst, tot);
-            }
+            const float tot = reduce_scatter<kV>(vals, lane, &idx);
+            if (idx < kV) add_sums(s_gid[k], idx, tot);
         }
         __syncthreads();
         bend = bstart;
@@ -670,7 +686,7 @@ k_render_bwd(CamConst cam, const float4 *__restrict__ xyod, const float4 *__rest
 __global__ void __launch_bounds__(kTilePixels)
 k_render_stats(CamConst cam, const float4 *__restrict__ xyod, const float4 *__restrict__ conr,
                const uint32_t *__restrict__ pair_gid, const uint2 *__restrict__ ranges,
-               const uint32_t *__restrict__ last, unsigned long long *__restrict__ counts) {
+               const uint32_t *__restrict__ last, unsigned long long *__restrict__ counts, const Bounds bd) {
     __shared__ float4 s_geo[kBatch];
     __shared__ float4 s_geo2[kBatch];
     __shared__ unsigned long long s_c[3];
@@ -681,6 +697,7 @@ k_render_stats(CamConst cam, const float4 *__restrict__ xyod, const float4 *__re
     const bool inside = px < cam.width && py < cam.height;
     const float fx = (float)px + 0.5f, fy = (float)py + 0.5f;
     const uint2 range = ranges[tile];
+    if (!range_in_bounds(range, bd)) return;
     if (threadIdx.x < 3) s_c[threadIdx.x] = 0ull;
     float T = 1.f;
     unsigned long long visits = 0, adds = 0;
@@ -690,9 +707,11 @@ k_render_stats(CamConst cam, const float4 *__restrict__ xyod, const float4 *__re
         const uint32_t j = b + threadIdx.x;
         if (j < range.y) {
             const uint32_t g = pair_gid[j];
-            float4 geo, geo2;
-            stage_entry(xyod[g], conr[g], geo, geo2);
-            geo2.z = hit_center(geo2.y);
+            float4 geo = make_float4(0.f, 0.f, 0.f, 0.f), geo2 = make_float4(0.f, 0.f, 1.f, 0.f);
+            if (in_bounds(g, bd.n, bd.status)) {  // checked builds: else an entry no pixel takes
+                stage_entry(xyod[g], conr[g], geo, geo2);
+                geo2.z = hit_center(geo2.y);
+            }
             s_geo[threadIdx.x] = geo;
             s_geo2[threadIdx.x] = geo2;
         }
@@ -758,9 +777,10 @@ static const uint32_t *tile_order(const gs_bins &bins) {
     return reinterpret_cast<const uint32_t *>(static_cast<const char *>(bins.scratch) + L.tile_order);
 }
 
-cudaError_t launch_render_fwd(const CamConst &c, const gs_projected &proj, const gs_bins &bins,
+cudaError_t launch_render_fwd(const CamConst &c, int64_t n, const gs_projected &proj, const gs_bins &bins,
                               float *image, float *T_final, uint32_t *last, cudaStream_t s) {
     const int tiles = c.tiles_x * c.tiles_y;
+    const Bounds bd = bounds_of(bins, n, tiles);
     const bool depth = c.flags & GS_FLAG_DEPTH;
     const ChannelIO io{reinterpret_cast<const float4 *>(proj.rgb), 1, depth ? 4 : 3, nullptr, 0};
     prof_before("render_fwd", s);
@@ -768,19 +788,20 @@ cudaError_t launch_render_fwd(const CamConst &c, const gs_projected &proj, const
         k_render_fwd<true><<<tiles, kTilePixels, 0, s>>>(
             c, reinterpret_cast<const float4 *>(proj.xy_opacity_depth),
             reinterpret_cast<const float4 *>(proj.conic_radius), io, bins.pair_gid,
-            reinterpret_cast<const uint2 *>(bins.ranges), tile_order(bins), image, T_final, last);
+            reinterpret_cast<const uint2 *>(bins.ranges), tile_order(bins), image, T_final, last, bd);
     else
         k_render_fwd<false><<<tiles, kTilePixels, 0, s>>>(
             c, reinterpret_cast<const float4 *>(proj.xy_opacity_depth),
             reinterpret_cast<const float4 *>(proj.conic_radius), io, bins.pair_gid,
-            reinterpret_cast<const uint2 *>(bins.ranges), tile_order(bins), image, T_final, last);
+            reinterpret_cast<const uint2 *>(bins.ranges), tile_order(bins), image, T_final, last, bd);
     prof_after(s);
     return cudaGetLastError();
 }
 
-cudaError_t launch_render_features_fwd(const CamConst &c, const gs_projected &proj, const gs_bins &bins,
+cudaError_t launch_render_features_fwd(const CamConst &c, int64_t n, const gs_projected &proj, const gs_bins &bins,
                                        const float *features, int F, float *out, cudaStream_t s) {
     const int tiles = c.tiles_x * c.tiles_y;
+    const Bounds bd = bounds_of(bins, n, tiles);
     CamConst cf = c;  // features blend without a background
     cf.bg[0] = cf.bg[1] = cf.bg[2] = 0.f;
     prof_before("render_features_fwd", s);
@@ -789,16 +810,17 @@ cudaError_t launch_render_features_fwd(const CamConst &c, const gs_projected &pr
         k_render_fwd<true, true><<<tiles, kTilePixels, 0, s>>>(
             cf, reinterpret_cast<const float4 *>(proj.xy_opacity_depth),
             reinterpret_cast<const float4 *>(proj.conic_radius), io, bins.pair_gid,
-            reinterpret_cast<const uint2 *>(bins.ranges), tile_order(bins), out + 4 * k, nullptr, nullptr);
+            reinterpret_cast<const uint2 *>(bins.ranges), tile_order(bins), out + 4 * k, nullptr, nullptr, bd);
     }
     prof_after(s, F / 4);
     return cudaGetLastError();
 }
 
-cudaError_t launch_render_bwd(const CamConst &c, const gs_projected &proj, const gs_bins &bins,
+cudaError_t launch_render_bwd(const CamConst &c, int64_t n, const gs_projected &proj, const gs_bins &bins,
                               const float *T_final, const uint32_t *last, const float *dL_dimage,
                               float *grad2d, cudaStream_t s) {
     const int tiles = c.tiles_x * c.tiles_y;
+    const Bounds bd = bounds_of(bins, n, tiles);
     const bool depth = c.flags & GS_FLAG_DEPTH;
     const ChannelIO io{reinterpret_cast<const float4 *>(proj.rgb), 1, depth ? 4 : 3, grad2d + 6, 12};
     prof_before("render_bwd", s);
@@ -806,21 +828,22 @@ cudaError_t launch_render_bwd(const CamConst &c, const gs_projected &proj, const
         k_render_bwd<GS_BWD_RPL, true><<<tiles, kTilePixels / GS_BWD_RPL, 0, s>>>(
             c, reinterpret_cast<const float4 *>(proj.xy_opacity_depth),
             reinterpret_cast<const float4 *>(proj.conic_radius), io, bins.pair_gid,
-            reinterpret_cast<const uint2 *>(bins.ranges), tile_order(bins), T_final, last, dL_dimage, grad2d);
+            reinterpret_cast<const uint2 *>(bins.ranges), tile_order(bins), T_final, last, dL_dimage, grad2d, bd);
     else
         k_render_bwd<GS_BWD_RPL, false><<<tiles, kTilePixels / GS_BWD_RPL, 0, s>>>(
             c, reinterpret_cast<const float4 *>(proj.xy_opacity_depth),
             reinterpret_cast<const float4 *>(proj.conic_radius), io, bins.pair_gid,
-            reinterpret_cast<const uint2 *>(bins.ranges), tile_order(bins), T_final, last, dL_dimage, grad2d);
+            reinterpret_cast<const uint2 *>(bins.ranges), tile_order(bins), T_final, last, dL_dimage, grad2d, bd);
     prof_after(s);
     return cudaGetLastError();
 }
 
-cudaError_t launch_render_features_bwd(const CamConst &c, const gs_projected &proj, const gs_bins &bins,
+cudaError_t launch_render_features_bwd(const CamConst &c, int64_t n, const gs_projected &proj, const gs_bins &bins,
                                        const float *T_final, const uint32_t *last, const float *features,
                                        int F, const float *dL_dout, float *grad2d, float *dL_dfeatures,
                                        cudaStream_t s) {
     const int tiles = c.tiles_x * c.tiles_y;
+    const Bounds bd = bounds_of(bins, n, tiles);
     CamConst cf = c;  // features blend without a background
     cf.bg[0] = cf.bg[1] = cf.bg[2] = 0.f;
     prof_before("render_features_bwd", s);
@@ -830,23 +853,24 @@ cudaError_t launch_render_features_bwd(const CamConst &c, const gs_projected &pr
             cf, reinterpret_cast<const float4 *>(proj.xy_opacity_depth),
             reinterpret_cast<const float4 *>(proj.conic_radius), io, bins.pair_gid,
             reinterpret_cast<const uint2 *>(bins.ranges), tile_order(bins), T_final, last, dL_dout + 4 * k,
-            grad2d);
+            grad2d, bd);
     }
     prof_after(s, F / 4);
     return cudaGetLastError();
 }
 
-cudaError_t launch_render_stats(const CamConst &c, const gs_projected &proj, const gs_bins &bins,
+cudaError_t launch_render_stats(const CamConst &c, int64_t n, const gs_projected &proj, const gs_bins &bins,
                                 const uint32_t *last, uint64_t *counts, cudaStream_t s) {
     cudaError_t e = cudaMemsetAsync(counts, 0, 4 * sizeof(uint64_t), s);
     if (e != cudaSuccess) return e;
     const int tiles = c.tiles_x * c.tiles_y;
+    const Bounds bd = bounds_of(bins, n, tiles);
     prof_before("render_stats", s);
     k_render_stats<<<tiles, kTilePixels, 0, s>>>(
         c, reinterpret_cast<const float4 *>(proj.xy_opacity_depth),
         reinterpret_cast<const float4 *>(proj.conic_radius), bins.pair_gid,
         reinterpret_cast<const uint2 *>(bins.ranges), last,
-        reinterpret_cast<unsigned long long *>(counts));
+        reinterpret_cast<unsigned long long *>(counts), bd);
     prof_after(s);
     return cudaGetLastError();
 }

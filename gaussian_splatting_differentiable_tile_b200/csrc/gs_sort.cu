@@ -134,7 +134,8 @@ __device__ __forceinline__ void cta_range(int n, int &g_begin, int &g_end) {
 
 // Row blockIdx of the count matrix H[CTA][tile].
 __global__ void __launch_bounds__(kBinThreads, 2)
-k_bin_count(int n, const int4 *__restrict__ rect, int tiles_x, int tiles_y, uint32_t *__restrict__ H) {
+k_bin_count(int n, const int4 *__restrict__ rect, int tiles_x, int tiles_y, uint32_t *__restrict__ H,
+            int32_t *__restrict__ status) {
     extern __shared__ uint32_t s_cnt[];
     const int tiles = tiles_x * tiles_y;
     uint32_t *row = H + (size_t)blockIdx.x * tiles;
@@ -144,7 +145,9 @@ k_bin_count(int n, const int4 *__restrict__ rect, int tiles_x, int tiles_y, uint
     __syncthreads();
     int g_begin, g_end;
     cta_range(n, g_begin, g_end);
-    for_each_pair(g_begin, g_end, rect, tiles_x, tiles_y, [&](int, int t) { atomicAdd(&cnt[t], 1u); });
+    for_each_pair(g_begin, g_end, rect, tiles_x, tiles_y, [&](int, int t) {
+        if (in_bounds((uint32_t)t, (uint32_t)tiles, status)) atomicAdd(&cnt[t], 1u);
+    });
     __syncthreads();
     if (smem)
         for (int t = threadIdx.x; t < tiles; t += kBinThreads) row[t] = s_cnt[t];
@@ -284,7 +287,7 @@ __device__ __forceinline__ uint64_t pair_key(const float4 *__restrict__ xyod, ui
 __global__ void __launch_bounds__(kBinThreads, 2)
 k_bin_emit(int n, const int4 *__restrict__ rect, const float4 *__restrict__ xyod, int tiles_x, int tiles_y,
            const uint32_t *__restrict__ ranges, uint32_t *__restrict__ H, uint64_t *__restrict__ keys,
-           const int32_t *__restrict__ status) {
+           int32_t *__restrict__ status, uint64_t max_pairs) {
     extern __shared__ uint32_t s_cur[];
     if (*(volatile const int32_t *)status != 0) return;
     const int tiles = tiles_x * tiles_y;
@@ -295,8 +298,11 @@ k_bin_emit(int n, const int4 *__restrict__ rect, const float4 *__restrict__ xyod
     __syncthreads();
     int g_begin, g_end;
     cta_range(n, g_begin, g_end);
-    for_each_pair(g_begin, g_end, rect, tiles_x, tiles_y,
-                  [&](int g, int t) { keys[atomicAdd(&cur[t], 1u)] = pair_key(xyod, (uint32_t)g); });
+    for_each_pair(g_begin, g_end, rect, tiles_x, tiles_y, [&](int g, int t) {
+        if (!in_bounds((uint32_t)t, (uint32_t)tiles, status)) return;
+        const uint32_t pos = atomicAdd(&cur[t], 1u);
+        if (in_bounds(pos, max_pairs, status)) keys[pos] = pair_key(xyod, (uint32_t)g);
+    });
 }
 
 __device__ __forceinline__ uint32_t order_bucket(uint32_t len) {
@@ -357,12 +363,14 @@ __device__ __forceinline__ int run_rank(const uint64_t *a, int n, uint64_t x) {
 __global__ void __launch_bounds__(128)
 k_tile_sort_warp(const uint32_t *__restrict__ ranges, const uint32_t *__restrict__ order, int tiles,
                  const uint64_t *__restrict__ keys, uint32_t *__restrict__ pair_gid,
-                 uint32_t *__restrict__ pair_tile) {
+                 uint32_t *__restrict__ pair_tile, const Bounds bd) {
     const int lane = threadIdx.x & 31;
     const int b = blockIdx.x * 4 + (threadIdx.x >> 5);
     if (b >= tiles) return;
     const uint32_t tile = order[b];
+    if (!in_bounds(tile, (uint32_t)tiles, bd.status)) return;
     const uint32_t start = ranges[2 * (size_t)tile], end = ranges[2 * (size_t)tile + 1];
+    if (!range_in_bounds(make_uint2(start, end), bd)) return;
     const uint32_t L = end - start;
     if (L == 0 || L > 256) return;
     uint64_t k[8];
@@ -473,7 +481,8 @@ template <int kWarps, bool kLong>
 __global__ void __launch_bounds__(kWarps * 32)
 k_tile_sort(const uint32_t *__restrict__ ranges, const uint32_t *__restrict__ order, int tiles,
             const uint64_t *__restrict__ keys, uint32_t *__restrict__ pair_gid,
-            uint32_t *__restrict__ pair_tile, uint32_t lo, int persistent, uint32_t *ka, uint32_t *va) {
+            uint32_t *__restrict__ pair_tile, uint32_t lo, int persistent, uint32_t *ka, uint32_t *va,
+            const Bounds bd) {
     constexpr int kThreads = kWarps * 32;
     constexpr uint32_t kHi = 256u * kWarps;
     extern __shared__ uint64_t s_buf[];
@@ -483,7 +492,9 @@ k_tile_sort(const uint32_t *__restrict__ ranges, const uint32_t *__restrict__ or
     const int step = persistent ? (int)gridDim.x : tiles;
     for (int b = blockIdx.x; b < tiles; b += step) {
         const uint32_t tile = order[b];
+        if (!in_bounds(tile, (uint32_t)tiles, bd.status)) break;  // uniform over the CTA
         const uint32_t start = ranges[2 * (size_t)tile], end = ranges[2 * (size_t)tile + 1];
+        if (!range_in_bounds(make_uint2(start, end), bd)) break;
         const uint32_t L = end - start;
         if (persistent && order_bucket(L) < order_bucket(lo)) break;
         if (L <= lo) continue;
@@ -563,6 +574,11 @@ k_tile_sort(const uint32_t *__restrict__ ranges, const uint32_t *__restrict__ or
 // The tile ranges, K, the capacity check and the tile order come from the
 // count kernels above, as on the per-tile path.
 
+// Ranking of an LSD pass's digits within a warp: one match instruction (1),
+// or one ballot per digit bit (0).  A tuning knob.
+#ifndef GS_LSD_MATCH
+#define GS_LSD_MATCH 1
+#endif
 constexpr int kLsdThreads = 512;
 constexpr int kLsdWarps = kLsdThreads / 32;
 
@@ -589,35 +605,8 @@ k_depth_init(int n, const int4 *__restrict__ rect, const float4 *__restrict__ xy
     vals[g] = (uint32_t)g;
 }
 
-// Counts of the digit (key >> shift) & 255 over this CTA's chunk, into
-// H[CTA][256], and their totals over all CTAs into D[256] (zeroed by the
-// call's memset).  The element count is *count_dev when given (K), else
-// count_host.
-__global__ void __launch_bounds__(kLsdThreads)
-k_lsd_hist(const uint32_t *__restrict__ keys, const uint64_t *__restrict__ count_dev, uint32_t count_host,
-           int shift, uint32_t *__restrict__ H, uint32_t *__restrict__ D, const int32_t *__restrict__ status) {
-    __shared__ uint32_t s_h[kLsdWarps][kRadix];
-    if (*(volatile const int32_t *)status != 0) return;
-    const int warp = threadIdx.x >> 5;
-    for (int i = threadIdx.x; i < kLsdWarps * kRadix; i += kLsdThreads) (&s_h[0][0])[i] = 0;
-    __syncthreads();
-    uint32_t lo, hi;
-    lsd_chunk(count_dev ? *count_dev : count_host, lo, hi);
-    for (uint32_t i = lo + threadIdx.x; i < hi; i += kLsdThreads)
-        atomicAdd(&s_h[warp][(keys[i] >> shift) & 0xFFu], 1u);
-    __syncthreads();
-    for (int d = threadIdx.x; d < kRadix; d += kLsdThreads) {
-        uint32_t t = 0;
-#pragma unroll
-        for (int w = 0; w < kLsdWarps; w++) t += s_h[w][d];
-        H[(size_t)blockIdx.x * kRadix + d] = t;
-        if (t) atomicAdd(&D[d], t);
-    }
-}
-
 // Exclusive scan of 256 values in shared memory by the first 256 threads
-// (the others only meet the barriers).  Returns the total in *total when
-// given.
+// (all threads of the block meet the barriers).
 __device__ __forceinline__ void scan256(uint32_t *v, uint32_t *s_w) {
     const int t = threadIdx.x, lane = t & 31, w = t >> 5;
     uint32_t x = 0, y = 0;
@@ -640,59 +629,185 @@ __device__ __forceinline__ void scan256(uint32_t *v, uint32_t *s_w) {
     __syncthreads();
 }
 
-// Stable scatter of one LSD pass: element i of this CTA's chunk goes to
-// (digit offset) + (its digit's count in the CTAs before this one) + (its
-// rank among the chunk's elements of that digit, in order).
-__global__ void __launch_bounds__(kLsdThreads)
-k_lsd_scatter(const uint32_t *__restrict__ keys_in, const uint32_t *__restrict__ vals_in,
-              const uint64_t *__restrict__ count_dev, uint32_t count_host, int shift,
-              const uint32_t *__restrict__ H, const uint32_t *__restrict__ D, uint32_t *__restrict__ keys_out,
-              uint32_t *__restrict__ vals_out, const int32_t *__restrict__ status) {
-    __shared__ uint32_t s_base[kRadix], s_tot[kRadix], s_w[kLsdWarps];
-    __shared__ uint32_t s_wc[kLsdWarps][kRadix];
+// An LSD pass takes its elements in tiles of kScatterTile; CTA b of every
+// kernel of the pass owns tile b.  H[d][b] (digit-major, T tiles per row)
+// counts digit d in tile b; its exclusive scan in that order is the output
+// position of tile b's first element of digit d.
+constexpr int kScatterThreads = 256;
+constexpr int kScatterWarps = kScatterThreads / 32;
+constexpr int kScatterItems = 16;
+constexpr int kScatterTile = kScatterThreads * kScatterItems;  // 4096
+
+// Digit counts of this CTA's tile into column blockIdx.x of H.  The element
+// count is *count_dev when given (K), else count_host; tiles past it count
+// nothing (their column is zero).
+__global__ void __launch_bounds__(kScatterThreads)
+k_lsd_hist(const uint32_t *__restrict__ keys, const uint64_t *__restrict__ count_dev, uint32_t count_host,
+           int shift, int bits, uint32_t *__restrict__ H, const int32_t *__restrict__ status) {
+    __shared__ uint32_t s_h[kScatterWarps][kRadix];
     if (*(volatile const int32_t *)status != 0) return;
-    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-    if (tid < kRadix) {
-        uint32_t pre = 0;
-        for (int c = 0; c < (int)blockIdx.x; c++) pre += H[(size_t)c * kRadix + tid];
-        s_base[tid] = pre;
-        s_tot[tid] = D[tid];
+    const int warp = threadIdx.x >> 5;
+    const uint32_t mask = (1u << bits) - 1u, ndig = 1u << bits;
+    for (int i = threadIdx.x; i < kScatterWarps * kRadix; i += kScatterThreads) (&s_h[0][0])[i] = 0;
+    __syncthreads();
+    const uint64_t count = count_dev ? *count_dev : count_host;
+    const uint64_t t0 = (uint64_t)blockIdx.x * kScatterTile;
+    const uint32_t m = t0 < count ? (uint32_t)min((uint64_t)kScatterTile, count - t0) : 0u;
+    for (uint32_t i = threadIdx.x; i < m; i += kScatterThreads)
+        atomicAdd(&s_h[warp][(keys[t0 + i] >> shift) & mask], 1u);
+    __syncthreads();
+    for (uint32_t d = threadIdx.x; d < ndig; d += kScatterThreads) {
+        uint32_t t = 0;
+#pragma unroll
+        for (int w = 0; w < kScatterWarps; w++) t += s_h[w][d];
+        H[(size_t)d * gridDim.x + blockIdx.x] = t;
+    }
+}
+
+// Exclusive scan of H[0, m) in place, in blocks of kScanBlock: each CTA scans
+// its block and writes the block's total to S (k_scan_blocks); each CTA then
+// adds the totals of the blocks before it (k_scan_add).
+constexpr int kScanThreads = 1024, kScanItems = 4, kScanBlock = kScanThreads * kScanItems;
+
+__device__ __forceinline__ uint32_t block_exclusive_scan(uint32_t v, uint32_t *s_w, uint32_t *total) {
+    const int lane = threadIdx.x & 31, w = threadIdx.x >> 5;
+    uint32_t y = v;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+        const uint32_t z = __shfl_up_sync(0xffffffffu, y, o);
+        if (lane >= o) y += z;
+    }
+    if (lane == 31) s_w[w] = y;
+    __syncthreads();
+    if (w == 0) {
+        const uint32_t x = lane < (int)(blockDim.x >> 5) ? s_w[lane] : 0u;
+        uint32_t z = x;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+            const uint32_t q = __shfl_up_sync(0xffffffffu, z, o);
+            if (lane >= o) z += q;
+        }
+        s_w[lane] = z - x;  // exclusive warp bases
+        if (lane == 31) s_w[32] = z;
     }
     __syncthreads();
-    scan256(s_tot, s_w);  // digit offsets
-    if (tid < kRadix) s_base[tid] += s_tot[tid];
+    const uint32_t r = s_w[w] + y - v;
+    *total = s_w[32];
     __syncthreads();
-    uint32_t lo, hi;
-    lsd_chunk(count_dev ? *count_dev : count_host, lo, hi);
-    for (uint32_t c0 = lo; c0 < hi; c0 += kLsdThreads) {
-        const uint32_t i = c0 + tid;
-        const bool in = i < hi;
-        const uint32_t key = in ? keys_in[i] : 0u, val = in ? vals_in[i] : 0u;
-        const uint32_t d = in ? (key >> shift) & 0xFFu : (uint32_t)kRadix;
-        for (int k = tid; k < kLsdWarps * kRadix; k += kLsdThreads) (&s_wc[0][0])[k] = 0;
-        __syncthreads();
-        const uint32_t peers = digit_peers(d, 8);
-        if (in && lane == __ffs(peers) - 1) s_wc[warp][d] = __popc(peers);
-        __syncthreads();
-        if (tid < kRadix) {  // exclusive over warps, per digit
-            uint32_t acc = 0;
+    return r;
+}
+
+__global__ void __launch_bounds__(kScanThreads)
+k_scan_blocks(uint32_t *__restrict__ H, uint32_t m, uint32_t *__restrict__ S, const int32_t *__restrict__ status) {
+    __shared__ uint32_t s_w[33];
+    if (*(volatile const int32_t *)status != 0) return;
+    const uint32_t b0 = blockIdx.x * kScanBlock + threadIdx.x * kScanItems;
+    uint32_t v[kScanItems], sum = 0;
 #pragma unroll
-            for (int ww = 0; ww < kLsdWarps; ww++) {
-                const uint32_t cc = s_wc[ww][tid];
-                s_wc[ww][tid] = acc;
-                acc += cc;
-            }
-            s_tot[tid] = acc;
+    for (int k = 0; k < kScanItems; k++) {
+        v[k] = b0 + k < m ? H[b0 + k] : 0u;
+        sum += v[k];
+    }
+    uint32_t total;
+    uint32_t off = block_exclusive_scan(sum, s_w, &total);
+#pragma unroll
+    for (int k = 0; k < kScanItems; k++) {
+        if (b0 + k < m) H[b0 + k] = off;
+        off += v[k];
+    }
+    if (threadIdx.x == 0) S[blockIdx.x] = total;
+}
+
+__global__ void __launch_bounds__(kScanThreads)
+k_scan_add(uint32_t *__restrict__ H, uint32_t m, const uint32_t *__restrict__ S, const int32_t *__restrict__ status) {
+    __shared__ uint32_t s_w[33];
+    if (*(volatile const int32_t *)status != 0) return;
+    uint32_t pre = 0;
+    for (uint32_t b = threadIdx.x; b < blockIdx.x; b += kScanThreads) pre += S[b];
+    uint32_t total;
+    block_exclusive_scan(pre, s_w, &total);  // only the block total is used
+    const uint32_t b0 = blockIdx.x * kScanBlock + threadIdx.x * kScanItems;
+#pragma unroll
+    for (int k = 0; k < kScanItems; k++)
+        if (b0 + k < m) H[b0 + k] += total;
+}
+
+// Stable scatter of one LSD pass, CTA b taking tile b: warp w holds elements
+// w * 512 + 32 k + lane (k = 0 .. 15), so (w, k, lane) is the input order.
+// Each warp ranks its elements within their digit in that order (one match
+// instruction per 32 elements, per-warp counters in shared memory); a scan
+// over the warps and over the digits places each element in the tile sorted
+// by digit, in shared memory; the tile then goes out digit run by digit run,
+// each run contiguous at the scanned H[d][b], so the writes are coalesced.
+__global__ void __launch_bounds__(kScatterThreads)
+k_lsd_scatter(const uint32_t *__restrict__ keys_in, const uint32_t *__restrict__ vals_in,
+              const uint64_t *__restrict__ count_dev, uint32_t count_host, int shift, int bits,
+              const uint32_t *__restrict__ H, uint32_t *__restrict__ keys_out, uint32_t *__restrict__ vals_out,
+              int32_t *__restrict__ status) {
+    __shared__ uint32_t s_gbase[kRadix], s_start[kRadix], s_w[kScatterWarps];
+    __shared__ uint32_t s_cnt[kScatterWarps][kRadix];
+    __shared__ uint32_t s_key[kScatterTile], s_val[kScatterTile];
+    if (*(volatile const int32_t *)status != 0) return;
+    const uint64_t count = count_dev ? *count_dev : count_host;
+    const uint64_t t0 = (uint64_t)blockIdx.x * kScatterTile;
+    if (t0 >= count) return;  // uniform over the CTA
+    const uint32_t m = (uint32_t)min((uint64_t)kScatterTile, count - t0);
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    const uint32_t mask = (1u << bits) - 1u, ndig = 1u << bits, lt = lanemask_lt();
+    uint32_t key[kScatterItems], val[kScatterItems], rank[kScatterItems];
+#pragma unroll
+    for (int k = 0; k < kScatterItems; k++) {
+        const uint32_t i = (uint32_t)(warp * 32 * kScatterItems + 32 * k + lane);
+        key[k] = i < m ? keys_in[t0 + i] : 0u;
+        val[k] = i < m ? vals_in[t0 + i] : 0u;
+    }
+    for (int i = tid; i < kScatterWarps * kRadix; i += kScatterThreads) (&s_cnt[0][0])[i] = 0;
+    if ((uint32_t)tid < ndig) s_gbase[tid] = H[(size_t)tid * gridDim.x + blockIdx.x];
+    __syncthreads();
+#pragma unroll
+    for (int k = 0; k < kScatterItems; k++) {
+        const uint32_t i = (uint32_t)(warp * 32 * kScatterItems + 32 * k + lane);
+        const uint32_t d = i < m ? (key[k] >> shift) & mask : (uint32_t)kRadix;
+#if GS_LSD_MATCH
+        const uint32_t peers = __match_any_sync(0xffffffffu, d);
+#else
+        const uint32_t peers = digit_peers(d, bits);
+#endif
+        rank[k] = d < kRadix ? s_cnt[warp][d] + __popc(peers & lt) : 0u;
+        __syncwarp();
+        if (d < kRadix && lane == __ffs(peers) - 1) s_cnt[warp][d] += __popc(peers);
+        __syncwarp();
+    }
+    __syncthreads();
+    if (tid < kRadix) {  // exclusive over the warps, per digit; digit totals of the tile
+        uint32_t tot = 0;
+#pragma unroll
+        for (int w = 0; w < kScatterWarps; w++) {
+            const uint32_t c = s_cnt[w][tid];
+            s_cnt[w][tid] = tot;
+            tot += c;
         }
-        __syncthreads();
-        if (in) {
-            const uint32_t pos = s_base[d] + s_wc[warp][d] + __popc(peers & lanemask_lt());
-            keys_out[pos] = key;
-            vals_out[pos] = val;
+        s_start[tid] = tot;
+    }
+    __syncthreads();
+    scan256(s_start, s_w);  // digit starts within the tile
+#pragma unroll
+    for (int k = 0; k < kScatterItems; k++) {
+        const uint32_t i = (uint32_t)(warp * 32 * kScatterItems + 32 * k + lane);
+        if (i < m) {
+            const uint32_t d = (key[k] >> shift) & mask;
+            const uint32_t pos = s_start[d] + s_cnt[warp][d] + rank[k];
+            s_key[pos] = key[k];
+            s_val[pos] = val[k];
         }
-        __syncthreads();
-        if (tid < kRadix) s_base[tid] += s_tot[tid];
-        __syncthreads();
+    }
+    __syncthreads();
+    for (uint32_t i = tid; i < m; i += kScatterThreads) {
+        const uint32_t kk = s_key[i], d = (kk >> shift) & mask;
+        const uint32_t pos = s_gbase[d] + (i - s_start[d]);
+        if (!in_bounds(pos, count, status)) continue;
+        keys_out[pos] = kk;
+        vals_out[pos] = s_val[i];
     }
 }
 
@@ -772,7 +887,7 @@ k_rank_offsets(int n, const int4 *__restrict__ rect, const uint32_t *__restrict_
 __global__ void __launch_bounds__(256)
 k_emit_ranked(int n, const int4 *__restrict__ rect, const uint32_t *__restrict__ order,
               const uint32_t *__restrict__ offsets, int tiles_x, int tiles_y, uint32_t *__restrict__ tile_out,
-              uint32_t *__restrict__ gid_out, const int32_t *__restrict__ status) {
+              uint32_t *__restrict__ gid_out, int32_t *__restrict__ status, uint64_t max_pairs) {
     if (*(volatile const int32_t *)status != 0) return;
     const int lane = threadIdx.x & 31;
     const int stride = gridDim.x * blockDim.x;
@@ -788,6 +903,7 @@ k_emit_ranked(int n, const int4 *__restrict__ rect, const uint32_t *__restrict__
         if (c <= kLaneTiles) {
             for (uint32_t k = 0; k < c; k++) {
                 const uint32_t dy = k / (uint32_t)w;
+                if (!in_bounds((uint64_t)off + k, max_pairs, status)) break;
                 tile_out[off + k] = (uint32_t)((y0 + (int)dy) * tiles_x + x0 + (int)(k - dy * (uint32_t)w));
                 gid_out[off + k] = g;
             }
@@ -802,6 +918,7 @@ k_emit_ranked(int n, const int4 *__restrict__ rect, const uint32_t *__restrict__
             const uint32_t wb = (uint32_t)__shfl_sync(0xffffffffu, w, src);
             for (uint32_t k = lane; k < cb; k += 32) {
                 const uint32_t dy = k / wb;
+                if (!in_bounds((uint64_t)ob + k, max_pairs, status)) break;
                 tile_out[ob + k] = (uint32_t)((yb + (int)dy) * tiles_x + xb + (int)(k - dy * wb));
                 gid_out[ob + k] = gb;
             }
@@ -849,13 +966,36 @@ cudaError_t device_setup(int *sms) {
 
 // The global path after the tile scan (see the kernels above).  ctas: CTAs
 // of the LSD, rank and emit kernels.
+// Entries of the count-matrix space one LSD pass over at most `cap`
+// elements uses: the digit counts of its tiles and the scan's block totals.
+int64_t lsd_space(int64_t cap) {
+    const int64_t m = (int64_t)kRadix * ((cap + kScatterTile - 1) / kScatterTile);
+    return m + (m + kScanBlock - 1) / kScanBlock;
+}
+
+// One stable LSD pass over the digit (key >> shift) & (2^bits - 1) of at
+// most `cap` elements (*count_dev of them when given, else count_host):
+// per-tile digit counts, their exclusive scan, the scatter.
+void lsd_pass(const uint32_t *ki, const uint32_t *vi, uint32_t *ko, uint32_t *vo, const uint64_t *count_dev,
+              uint32_t count_host, int64_t cap, int shift, int bits, uint32_t *H, int32_t *status, cudaStream_t s) {
+    const int tiles = (int)std::max<int64_t>(1, (cap + kScatterTile - 1) / kScatterTile);
+    const uint32_t m = (uint32_t)((1u << bits) * (uint32_t)tiles);
+    const int blocks = (int)((m + kScanBlock - 1) / kScanBlock);
+    uint32_t *S = H + m;
+    k_lsd_hist<<<tiles, kScatterThreads, 0, s>>>(ki, count_dev, count_host, shift, bits, H, status);
+    k_scan_blocks<<<blocks, kScanThreads, 0, s>>>(H, m, S, status);
+    k_scan_add<<<blocks, kScanThreads, 0, s>>>(H, m, S, status);
+    k_lsd_scatter<<<tiles, kScatterThreads, 0, s>>>(ki, vi, count_dev, count_host, shift, bits, H, ko, vo, status);
+}
+
+// The global path after the tile scan (see the kernels above).  ctas: CTAs
+// of the rank and emit kernels.
 cudaError_t launch_bin_global(const CamConst &c, int64_t n, const gs_projected &proj, const gs_bins &bins,
                               const BinsLayout &L, int ctas, int sms, cudaStream_t s) {
     char *base = static_cast<char *>(bins.scratch);
     auto U32 = [&](size_t off) { return reinterpret_cast<uint32_t *>(base + off); };
-    const int32_t *status = reinterpret_cast<const int32_t *>(base + L.status);
+    int32_t *status = reinterpret_cast<int32_t *>(base + L.status);
     const uint64_t *n_pairs = reinterpret_cast<const uint64_t *>(base + L.n_pairs);
-    uint32_t *D = U32(L.lsd_totals);
     uint32_t *H = U32(L.bin_hist);
     const size_t pb = align_up((size_t)bins.max_pairs * sizeof(uint32_t), 256);
     uint32_t *KA = U32(L.keys), *VA = U32(L.keys + pb);  // the key array's two halves
@@ -870,10 +1010,9 @@ cudaError_t launch_bin_global(const CamConst &c, int64_t n, const gs_projected &
                                                                status);
     for (int p = 0; p < 4; p++) {
         uint32_t *ki = p & 1 ? KB : KA, *vi = p & 1 ? VB : VA, *ko = p & 1 ? KA : KB, *vo = p & 1 ? VA : VB;
-        k_lsd_hist<<<ctas, kLsdThreads, 0, s>>>(ki, nullptr, nn, 8 * p, H, D + kRadix * p, status);
-        k_lsd_scatter<<<ctas, kLsdThreads, 0, s>>>(ki, vi, nullptr, nn, 8 * p, H, D + kRadix * p, ko, vo, status);
+        lsd_pass(ki, vi, ko, vo, nullptr, nn, n, 8 * p, 8, H, status, s);
     }
-    prof_after(s, 9);
+    prof_after(s, 17);
     // 5. each Gaussian's first pair position in depth order (into KA), then
     // the pairs in (depth, id) order into (KB, VB)
     prof_before("emit", s);
@@ -881,22 +1020,23 @@ cudaError_t launch_bin_global(const CamConst &c, int64_t n, const gs_projected &
     k_rank_sums<<<ctas, kLsdThreads, 0, s>>>((int)n, rect, VA, c.tiles_x, c.tiles_y, S, status);
     k_rank_offsets<<<ctas, kLsdThreads, 0, s>>>((int)n, rect, VA, c.tiles_x, c.tiles_y, S, KA, status);
     const int emit_blocks = (int)std::min<int64_t>((n + 255) / 256, (int64_t)8 * sms);
-    k_emit_ranked<<<emit_blocks, 256, 0, s>>>((int)n, rect, VA, KA, c.tiles_x, c.tiles_y, KB, VB, status);
+    k_emit_ranked<<<emit_blocks, 256, 0, s>>>((int)n, rect, VA, KA, c.tiles_x, c.tiles_y, KB, VB, status,
+                                              (uint64_t)bins.max_pairs);
     prof_after(s, 3);
-    // 6. stable passes over the tile id's 8-bit digits: B -> A -> B ..., the
-    // last into pair_tile / pair_gid
-    int passes = 1;
-    while (passes < 3 && (uint32_t)(tiles - 1) >> (8 * passes)) passes++;
+    // 6. stable passes over the tile id, its bits split evenly into digits of
+    // at most 8 bits: B -> A -> B ..., the last into pair_tile / pair_gid
+    int tile_bits = 1;
+    while (tile_bits < 31 && ((uint32_t)(tiles - 1) >> tile_bits)) tile_bits++;
+    const int passes = (tile_bits + 7) / 8, digit = (tile_bits + passes - 1) / passes;
     prof_before("tile_sort", s);
     for (int p = 0; p < passes; p++) {
         const bool last = p == passes - 1;
+        const int bits = std::min(digit, tile_bits - digit * p);
         uint32_t *ki = p & 1 ? KA : KB, *vi = p & 1 ? VA : VB;
         uint32_t *ko = last ? bins.pair_tile : (p & 1 ? KB : KA), *vo = last ? bins.pair_gid : (p & 1 ? VB : VA);
-        k_lsd_hist<<<ctas, kLsdThreads, 0, s>>>(ki, n_pairs, 0u, 8 * p, H, D + kRadix * (4 + p), status);
-        k_lsd_scatter<<<ctas, kLsdThreads, 0, s>>>(ki, vi, n_pairs, 0u, 8 * p, H, D + kRadix * (4 + p), ko, vo,
-                                                   status);
+        lsd_pass(ki, vi, ko, vo, n_pairs, 0u, bins.max_pairs, digit * p, bits, H, status, s);
     }
-    prof_after(s, 2 * passes);
+    prof_after(s, 4 * passes);
     return cudaGetLastError();
 }
 
@@ -925,7 +1065,7 @@ cudaError_t launch_bin_and_sort(const CamConst &c, int64_t n, const gs_projected
     if (e != cudaSuccess) return e;
     // 1. per-CTA tile counts, 2. offsets down each tile's column
     prof_before("bin_count", s);
-    k_bin_count<<<ctas, kBinThreads, cnt_smem, s>>>((int)n, rect, c.tiles_x, c.tiles_y, H);
+    k_bin_count<<<ctas, kBinThreads, cnt_smem, s>>>((int)n, rect, c.tiles_x, c.tiles_y, H, status);
     k_bin_colscan<<<(tiles + 31) / 32, 256, 0, s>>>(tiles, ctas, H, totals);
     prof_after(s, 2);
     // 3. ranges, K, capacity check, tile order
@@ -937,25 +1077,28 @@ cudaError_t launch_bin_and_sort(const CamConst &c, int64_t n, const gs_projected
     // the global path's LSD passes keep per-CTA digit counts in the count
     // matrix's space (free once the tile scan has run)
     const int64_t hist_cap = std::min<int64_t>((int64_t)kBinCTAsMax * bins.max_tiles, kBinHistCap);
-    const int lsd_ctas = (int)std::min<int64_t>((int64_t)2 * sms, hist_cap / kRadix);
+    const int lsd_ctas = (int)std::min<int64_t>((int64_t)2 * sms, hist_cap);
     bool global = bins.strategy == GS_BIN_GLOBAL;
     if (bins.strategy == GS_BIN_AUTO)
         global = bins.max_pairs >= (int64_t)1024 * tiles;
-    global = global && n <= bins.max_pairs && lsd_ctas >= 1;
+    // the passes' digit counts must fit the count matrix's space
+    global = global && n <= bins.max_pairs && lsd_space(bins.max_pairs) <= hist_cap;
     if (global) return launch_bin_global(c, n, proj, bins, L, lsd_ctas, sms, s);
     // 4. emit the sort keys
     prof_before("emit", s);
     k_bin_emit<<<ctas, kBinThreads, cnt_smem, s>>>((int)n, rect, reinterpret_cast<const float4 *>(proj.xy_opacity_depth),
-                                                   c.tiles_x, c.tiles_y, ranges, H, keys, status);
+                                                   c.tiles_x, c.tiles_y, ranges, H, keys, status,
+                                                   (uint64_t)bins.max_pairs);
     prof_after(s);
     // 5. sort each tile's list, by size class
     prof_before("tile_sort", s);
-    k_tile_sort_warp<<<(tiles + 3) / 4, 128, 0, s>>>(ranges, order, tiles, keys, bins.pair_gid, bins.pair_tile);
+    const Bounds bd = bounds_of(bins, n, tiles);
+    k_tile_sort_warp<<<(tiles + 3) / 4, 128, 0, s>>>(ranges, order, tiles, keys, bins.pair_gid, bins.pair_tile, bd);
     k_tile_sort<kShortWarps, false><<<tiles, kShortWarps * 32, 2 * kTileSortShort * sizeof(uint64_t), s>>>(
-        ranges, order, tiles, keys, bins.pair_gid, bins.pair_tile, 256u, 0, nullptr, nullptr);
+        ranges, order, tiles, keys, bins.pair_gid, bins.pair_tile, 256u, 0, nullptr, nullptr, bd);
     k_tile_sort<kMidWarps, true><<<std::min(tiles, sms), kMidWarps * 32, 2 * kTileSortMid * sizeof(uint64_t), s>>>(
         ranges, order, tiles, keys, bins.pair_gid, bins.pair_tile, kTileSortShort, 1, U32(L.long_keys),
-        U32(L.long_ids));
+        U32(L.long_ids), bd);
     prof_after(s, 3);
     return cudaGetLastError();
 }

@@ -20,11 +20,14 @@ class Rasterizer:
     a full-resolution 400k scene needs more than 16.7M pairs).
     """
 
-    def __init__(self, n: int, width: int, height: int, max_pairs: int | None = None, device="cuda"):
+    def __init__(self, n: int, width: int, height: int, max_pairs: int | None = None, device="cuda",
+                 strategy: int = 0):
         self.n, self.width, self.height = int(n), int(width), int(height)
         self.device = device
+        self.strategy = int(strategy)  # gs_bins.strategy (GS_BIN_*)
         self.proj = Projected(self.n, device)
-        self.bins = Bins(self.n, int(max_pairs) if max_pairs else max(1024, 16 * self.n), width, height, device)
+        self.bins = Bins(self.n, int(max_pairs) if max_pairs else max(1024, 16 * self.n), width, height, device,
+                         strategy=self.strategy)
         P = self.width * self.height
         self.image = torch.empty((self.height, self.width, 3), dtype=torch.float32, device=device)
         self.T_final = torch.empty((self.height, self.width), dtype=torch.float32, device=device)
@@ -34,7 +37,26 @@ class Rasterizer:
         assert P > 0
 
     def _grow(self, need: int) -> None:
-        self.bins = Bins(self.n, int(math.ceil(need * 1.25)) + 1024, self.width, self.height, self.device)
+        self.bins = Bins(self.n, int(math.ceil(need * 1.25)) + 1024, self.width, self.height, self.device,
+                         strategy=self.strategy)
+
+    def _global_for(self, capacity: int, n: int) -> bool:
+        """The automatic binning strategy's choice for a pair list of this
+        capacity (include/gs.h GS_BIN_AUTO)."""
+        return capacity >= 1024 * self.bins.tiles and n <= capacity
+
+    def _fit(self, need: int, n: int) -> bool:
+        """With the automatic strategy, re-carves the pair list near the frame's
+        need when its current capacity would pick the other strategy than a
+        list sized to the frame (a roomy default would send short tile lists
+        down the long-list path).  Returns whether it re-carved."""
+        if self.strategy != 0:
+            return False
+        fitted = int(math.ceil(need * 1.25)) + 1024
+        if self._global_for(self.bins.max_pairs, n) == self._global_for(fitted, n):
+            return False
+        self._grow(need)
+        return True
 
     def forward(self, cam, params: dict, sync: bool = True) -> torch.Tensor:
         """Renders into self.image (returned).  With sync=False no host
@@ -49,6 +71,8 @@ class Rasterizer:
                 if e.code != GS_ERR_CAPACITY:
                     raise
                 self._grow(e.n_pairs)
+                self.n_pairs = gs_bin_and_sort(cam, n, self.proj, self.bins, sync=True)
+            if self._fit(self.n_pairs, n):
                 self.n_pairs = gs_bin_and_sort(cam, n, self.proj, self.bins, sync=True)
         else:
             gs_bin_and_sort(cam, n, self.proj, self.bins, sync=False)

@@ -67,8 +67,11 @@ enum {
     GS_ERR_TOO_LARGE = -3,      /* N or max_pairs at or above 2^30 */
     GS_ERR_ALIGNMENT = -4,      /* a pointer is not aligned as documented */
     GS_ERR_CUDA = -5,           /* a CUDA runtime call or launch failed */
-    GS_ERR_DEVICE_TIMEOUT = -6  /* a bounded device-side wait gave up (reserved:
+    GS_ERR_DEVICE_TIMEOUT = -6, /* a bounded device-side wait gave up (reserved:
                                    no kernel of this version waits on another) */
+    GS_ERR_BOUNDS = -7          /* a kernel index was out of its array's range and the
+                                   access was skipped; only libgs_check.so (built with
+                                   GS_CHECK) tests indices, into bins->status */
 };
 
 /* Pinhole camera ([GSP] s3).  Host struct, passed by pointer. */

@@ -83,8 +83,12 @@ def gpu_render(cam, n, proj, bins):
     image = torch.full((H, W, G.channels(cam)), float("nan"), device="cuda")
     T = torch.full((H, W), float("nan"), device="cuda")
     last = torch.full((H, W), -1, dtype=torch.int32, device="cuda")
+    before = int(bins.status.item())
     G.gs_render_fwd(cam, n, proj, bins, image, T, last)
     torch.cuda.synchronize()
+    # the render writes the status word only in a checked build, on an index
+    # out of range
+    assert int(bins.status.item()) == before, G.gs_error_string(int(bins.status.item()))
     return image, T, last
 
 

@@ -46,7 +46,7 @@ def test_struct_sizes_match_header_layout():
 
 def test_error_strings(lib):
     from gaussian_splatting_differentiable_tile_b200 import _abi
-    for code in (0, -1, -2, -3, -4, -5, -6):
+    for code in (0, -1, -2, -3, -4, -5, -6, -7):
         s = lib.gs_error_string(code).decode()
         assert s and s != "unknown error code"
     assert lib.gs_error_string(-99).decode() == "unknown error code"

@@ -302,6 +302,7 @@ def _bwd_stage_fed(cam, params, seed=0, tile_mask=None):
     G.gs_render_bwd(cam, n, P, proj, bins, torch.from_numpy(T).cuda(), torch.from_numpy(last).cuda(),
                     torch.from_numpy(dl).cuda(), grad2d, grads)
     torch.cuda.synchronize()
+    assert int(bins.status.item()) == 0  # a checked build records an index out of range here
     g2_ref, g2_abs = O.render_bwd(rec, cam, dl.astype(np.float64), tile_mask=tile_mask)
     return rec, grad2d.cpu().numpy(), {k: v.cpu().numpy() for k, v in grads.items()}, g2_ref, g2_abs, params
 
