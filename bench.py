@@ -352,6 +352,32 @@ def run_profile_frame(args, spec):
                       "loss": loss.item()}), flush=True)
 
 
+def run_profile_train(args, spec):
+    """One eager batched training step (4 cameras on 4 lanes, Adam) for a
+    profiler to capture, in the NVTX range "train_step" (after a sizing pass
+    and one warm-up step outside it)."""
+    import torch
+
+    import gaussian_splatting_differentiable_tile_b200 as G
+
+    torch.cuda.set_device(0)
+    params = {k: torch.from_numpy(v).cuda() for k, v in make_scene(spec).items()}
+    cams = _cameras(spec, args)[:4]
+    nc = G.channels(cams[0])
+    tr = G.Trainer(spec.n, spec.width, spec.height, lanes=4, channels=nc)
+    need = tr.fit_pairs(cams, params)
+    tgt = torch.stack([torch.from_numpy(make_target(spec.width, spec.height, seed=i, channels=nc)).cuda()
+                       for i in range(len(cams))])
+    tr.step(cams, params, tgt)  # warm-up
+    torch.cuda.synchronize()
+    torch.cuda.nvtx.range_push("train_step")
+    tr.step(cams, params, tgt)
+    torch.cuda.nvtx.range_pop()
+    torch.cuda.synchronize()
+    print(json.dumps({"profile_train": spec.name, "cameras": len(cams), "lanes": 4, "max_pairs": need}),
+          flush=True)
+
+
 def run_native(args, spec, rank, world, local):
     import torch
     import torch.distributed as dist
@@ -772,6 +798,8 @@ def main():
     ap.add_argument("--profile-frame", action="store_true",
                     help="run one eager frame of one camera and exit (for ncu); prints no bench line")
     ap.add_argument("--profile-camera", type=int, default=0)
+    ap.add_argument("--profile-train", action="store_true",
+                    help="run one eager batched training step (4 cameras, Adam) and exit (for ncu); no bench line")
     args = ap.parse_args()
     rank = int(os.environ.get("RANK", 0))
     world = int(os.environ.get("WORLD_SIZE", 1))
@@ -779,6 +807,9 @@ def main():
     spec = SPECS[args.workload]
     if args.profile_frame:
         run_profile_frame(args, spec)
+        return
+    if args.profile_train:
+        run_profile_train(args, spec)
         return
     if args.impl == "reference":
         run_reference(args, spec, rank, world)

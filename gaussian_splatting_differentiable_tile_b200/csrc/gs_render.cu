@@ -53,6 +53,11 @@
 #ifndef GS_FWD_MINB
 #define GS_FWD_MINB 5
 #endif
+// Forward: issue both entries' exponentials before the alpha tests (1), or
+// only in the branch of a passing entry (0).  A tuning knob.
+#ifndef GS_FWD_EARLY_EX2
+#define GS_FWD_EARLY_EX2 1
+#endif
 #ifndef GS_BWD_BATCH
 #define GS_BWD_BATCH 128
 #endif
@@ -356,8 +361,19 @@ k_render_fwd(CamConst cam, const float4 *__restrict__ xyod, const float4 *__rest
                     const float2 u = __ffma2_rn(make_float2(cn.x, cn.y), dy, bdx);
                     const float2 q = __ffma2_rn(dy, u, a0);
                     const float2 t = __fadd2_rn(q, make_float2(cn.z, cn.w));  // q - c, as the backward
+#if GS_FWD_EARLY_EX2
+                    // both exponentials issued ahead of the tests, so their
+                    // latency overlaps the branches (each half rounded as
+                    // the scalar add, as the backward)
+                    const float2 pe = __fadd2_rn(q, wb.lo[k]);
+                    const float ea = ex2_approx(pe.x), eb = ex2_approx(pe.y);
+#endif
                     if (fabsf(t.x) <= cn.z) {
+#if GS_FWD_EARLY_EX2
+                        const float a = fminf(ea, cam.alpha_cap);
+#else
                         const float a = fminf(ex2_approx(__fadd_rn(q.x, wb.lo[k].x)), cam.alpha_cap);
+#endif
                         const float nT = __fmaf_rn(-T, a, T);
                         if (nT < cam.t_stop) {
                             done = true;
@@ -373,7 +389,11 @@ k_render_fwd(CamConst cam, const float4 *__restrict__ xyod, const float4 *__rest
                         lt = (int)(2 * k);
                     }
                     if (fabsf(t.y) <= cn.w) {
+#if GS_FWD_EARLY_EX2
+                        const float a = fminf(eb, cam.alpha_cap);
+#else
                         const float a = fminf(ex2_approx(__fadd_rn(q.y, wb.lo[k].y)), cam.alpha_cap);
+#endif
                         const float nT = __fmaf_rn(-T, a, T);
                         if (nT < cam.t_stop) {
                             done = true;

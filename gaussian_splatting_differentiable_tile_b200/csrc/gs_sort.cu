@@ -633,33 +633,46 @@ __device__ __forceinline__ void scan256(uint32_t *v, uint32_t *s_w) {
 // kernel of the pass owns tile b.  H[d][b] (digit-major, T tiles per row)
 // counts digit d in tile b; its exclusive scan in that order is the output
 // position of tile b's first element of digit d.
-constexpr int kScatterThreads = 256;
+constexpr int kScatterThreads = 512;
 constexpr int kScatterWarps = kScatterThreads / 32;
-constexpr int kScatterItems = 16;
+constexpr int kScatterItems = 8;
 constexpr int kScatterTile = kScatterThreads * kScatterItems;  // 4096
+// dynamic shared memory of k_lsd_scatter: the tile's keys and values, and
+// the per-warp digit counters
+constexpr size_t kScatterSmem = (2 * (size_t)kScatterTile + (size_t)kScatterWarps * kRadix) * sizeof(uint32_t);
+constexpr int kHistThreads = 256, kHistItems = kScatterTile / kHistThreads;
+constexpr int kHistWarps = kHistThreads / 32;
 
 // Digit counts of this CTA's tile into column blockIdx.x of H.  The element
 // count is *count_dev when given (K), else count_host; tiles past it count
-// nothing (their column is zero).
-__global__ void __launch_bounds__(kScatterThreads)
+// nothing (their column is zero).  A thread's keys are loaded together, then
+// counted.
+__global__ void __launch_bounds__(kHistThreads)
 k_lsd_hist(const uint32_t *__restrict__ keys, const uint64_t *__restrict__ count_dev, uint32_t count_host,
            int shift, int bits, uint32_t *__restrict__ H, const int32_t *__restrict__ status) {
-    __shared__ uint32_t s_h[kScatterWarps][kRadix];
+    __shared__ uint32_t s_h[kHistWarps][kRadix];
     if (*(volatile const int32_t *)status != 0) return;
     const int warp = threadIdx.x >> 5;
     const uint32_t mask = (1u << bits) - 1u, ndig = 1u << bits;
-    for (int i = threadIdx.x; i < kScatterWarps * kRadix; i += kScatterThreads) (&s_h[0][0])[i] = 0;
-    __syncthreads();
+    for (int i = threadIdx.x; i < kHistWarps * kRadix; i += kHistThreads) (&s_h[0][0])[i] = 0;
     const uint64_t count = count_dev ? *count_dev : count_host;
     const uint64_t t0 = (uint64_t)blockIdx.x * kScatterTile;
     const uint32_t m = t0 < count ? (uint32_t)min((uint64_t)kScatterTile, count - t0) : 0u;
-    for (uint32_t i = threadIdx.x; i < m; i += kScatterThreads)
-        atomicAdd(&s_h[warp][(keys[t0 + i] >> shift) & mask], 1u);
+    uint32_t kk[kHistItems];
+#pragma unroll
+    for (int k = 0; k < kHistItems; k++) {
+        const uint32_t i = (uint32_t)(k * kHistThreads) + threadIdx.x;
+        kk[k] = i < m ? keys[t0 + i] : 0u;
+    }
     __syncthreads();
-    for (uint32_t d = threadIdx.x; d < ndig; d += kScatterThreads) {
+#pragma unroll
+    for (int k = 0; k < kHistItems; k++)
+        if ((uint32_t)(k * kHistThreads) + threadIdx.x < m) atomicAdd(&s_h[warp][(kk[k] >> shift) & mask], 1u);
+    __syncthreads();
+    for (uint32_t d = threadIdx.x; d < ndig; d += kHistThreads) {
         uint32_t t = 0;
 #pragma unroll
-        for (int w = 0; w < kScatterWarps; w++) t += s_h[w][d];
+        for (int w = 0; w < kHistWarps; w++) t += s_h[w][d];
         H[(size_t)d * gridDim.x + blockIdx.x] = t;
     }
 }
@@ -733,7 +746,7 @@ k_scan_add(uint32_t *__restrict__ H, uint32_t m, const uint32_t *__restrict__ S,
 }
 
 // Stable scatter of one LSD pass, CTA b taking tile b: warp w holds elements
-// w * 512 + 32 k + lane (k = 0 .. 15), so (w, k, lane) is the input order.
+// w * 256 + 32 k + lane (k = 0 .. 7), so (w, k, lane) is the input order.
 // Each warp ranks its elements within their digit in that order (one match
 // instruction per 32 elements, per-warp counters in shared memory); a scan
 // over the warps and over the digits places each element in the tile sorted
@@ -745,8 +758,9 @@ k_lsd_scatter(const uint32_t *__restrict__ keys_in, const uint32_t *__restrict__
               const uint32_t *__restrict__ H, uint32_t *__restrict__ keys_out, uint32_t *__restrict__ vals_out,
               int32_t *__restrict__ status) {
     __shared__ uint32_t s_gbase[kRadix], s_start[kRadix], s_w[kScatterWarps];
-    __shared__ uint32_t s_cnt[kScatterWarps][kRadix];
-    __shared__ uint32_t s_key[kScatterTile], s_val[kScatterTile];
+    extern __shared__ uint32_t s_dyn[];
+    uint32_t *s_key = s_dyn, *s_val = s_dyn + kScatterTile;
+    uint32_t(*s_cnt)[kRadix] = reinterpret_cast<uint32_t(*)[kRadix]>(s_dyn + 2 * kScatterTile);
     if (*(volatile const int32_t *)status != 0) return;
     const uint64_t count = count_dev ? *count_dev : count_host;
     const uint64_t t0 = (uint64_t)blockIdx.x * kScatterTile;
@@ -954,7 +968,9 @@ cudaError_t device_setup(int *sms) {
             (e = cudaFuncSetAttribute(k_bin_emit, cudaFuncAttributeMaxDynamicSharedMemorySize, cnt_bytes)) !=
                 cudaSuccess ||
             (e = cudaFuncSetAttribute(k_tile_sort<kMidWarps, true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                      (int)(2 * kTileSortMid * sizeof(uint64_t)))) != cudaSuccess)
+                                      (int)(2 * kTileSortMid * sizeof(uint64_t)))) != cudaSuccess ||
+            (e = cudaFuncSetAttribute(k_lsd_scatter, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                      (int)kScatterSmem)) != cudaSuccess)
             return e;
         d.sms = n > 0 ? n : 148;
     }
@@ -982,10 +998,11 @@ void lsd_pass(const uint32_t *ki, const uint32_t *vi, uint32_t *ko, uint32_t *vo
     const uint32_t m = (uint32_t)((1u << bits) * (uint32_t)tiles);
     const int blocks = (int)((m + kScanBlock - 1) / kScanBlock);
     uint32_t *S = H + m;
-    k_lsd_hist<<<tiles, kScatterThreads, 0, s>>>(ki, count_dev, count_host, shift, bits, H, status);
+    k_lsd_hist<<<tiles, kHistThreads, 0, s>>>(ki, count_dev, count_host, shift, bits, H, status);
     k_scan_blocks<<<blocks, kScanThreads, 0, s>>>(H, m, S, status);
     k_scan_add<<<blocks, kScanThreads, 0, s>>>(H, m, S, status);
-    k_lsd_scatter<<<tiles, kScatterThreads, 0, s>>>(ki, vi, count_dev, count_host, shift, bits, H, ko, vo, status);
+    k_lsd_scatter<<<tiles, kScatterThreads, kScatterSmem, s>>>(ki, vi, count_dev, count_host, shift, bits, H, ko,
+                                                               vo, status);
 }
 
 // The global path after the tile scan (see the kernels above).  ctas: CTAs
