@@ -228,7 +228,9 @@ k_tile_scan(int tiles, const uint32_t *__restrict__ totals, uint64_t max_pairs,
         }
         s_w64[lane] = z;
         if (lane == 31) {
-            *n_pairs = z;
+            // an error recorded earlier (the global strategy's capacity check)
+            // came with its K, which stays
+            if (*(volatile int32_t *)status == 0) *n_pairs = z;
             const bool ok = z <= max_pairs;
             if (!ok) set_status(status, GS_ERR_CAPACITY);
             s_ok = ok && *(volatile int32_t *)status == 0;
@@ -563,21 +565,37 @@ k_tile_sort(const uint32_t *__restrict__ ranges, const uint32_t *__restrict__ or
 //                               of its rectangle at its position, so the pair
 //                               list comes out in (depth, id) order and is
 //                               written contiguously
-//   LSD passes on the tile id   stable, 8 bits each: the pairs grouped by
+//   LSD passes on the tile id   stable, the id's bits split evenly into digits
+//                               of at most 8 bits: the pairs grouped by
 //                               tile, the (depth, id) order kept inside every
 //                               tile; the last pass writes pair_tile and
 //                               pair_gid
-// An LSD pass is a histogram kernel (counts per CTA and digit, and the
-// digit totals by atomics) and a scatter kernel (each CTA finds its offsets
-// from the counts of the CTAs before it and the digit totals, then ranks its
-// elements in order with warp ballots).  No kernel waits on another CTA.
-// The tile ranges, K, the capacity check and the tile order come from the
-// count kernels above, as on the per-tile path.
+//   k_tile_bounds, k_tile_totals, k_tile_scan
+//                               each tile's [start, end) read off the sorted
+//                               list; the tile scan of the per-tile path then
+//                               builds the tile order (longest list first)
+// An LSD pass takes its elements in tiles of 4 096, one CTA per tile: a
+// histogram kernel (each tile's digit counts, digit-major), an exclusive scan
+// of those counts (two kernels), and a scatter kernel (each CTA ranks its
+// tile's elements in input order, sorts the tile by digit in shared memory
+// and writes every digit's run contiguously at its scanned offset).  The
+// count matrix of the per-tile strategy is not built: K comes out of the
+// depth-ordered scan of the tile counts, which also takes the capacity check
+// (GS_ERR_CAPACITY, with K) before anything is emitted.  No kernel waits on
+// another CTA.
 
 // Ranking of an LSD pass's digits within a warp: one match instruction (1),
 // or one ballot per digit bit (0).  A tuning knob.
 #ifndef GS_LSD_MATCH
 #define GS_LSD_MATCH 1
+#endif
+// Resident scatter CTAs per SM the register allocation targets (a tuning
+// knob).
+#ifndef GS_LSD_PREMATCH
+#define GS_LSD_PREMATCH 0
+#endif
+#ifndef GS_LSD_MINB
+#define GS_LSD_MINB 3
 #endif
 constexpr int kLsdThreads = 512;
 constexpr int kLsdWarps = kLsdThreads / 32;
@@ -752,7 +770,7 @@ k_scan_add(uint32_t *__restrict__ H, uint32_t m, const uint32_t *__restrict__ S,
 // over the warps and over the digits places each element in the tile sorted
 // by digit, in shared memory; the tile then goes out digit run by digit run,
 // each run contiguous at the scanned H[d][b], so the writes are coalesced.
-__global__ void __launch_bounds__(kScatterThreads)
+__global__ void __launch_bounds__(kScatterThreads, GS_LSD_MINB)
 k_lsd_scatter(const uint32_t *__restrict__ keys_in, const uint32_t *__restrict__ vals_in,
               const uint64_t *__restrict__ count_dev, uint32_t count_host, int shift, int bits,
               const uint32_t *__restrict__ H, uint32_t *__restrict__ keys_out, uint32_t *__restrict__ vals_out,
@@ -778,6 +796,29 @@ k_lsd_scatter(const uint32_t *__restrict__ keys_in, const uint32_t *__restrict__
     for (int i = tid; i < kScatterWarps * kRadix; i += kScatterThreads) (&s_cnt[0][0])[i] = 0;
     if ((uint32_t)tid < ndig) s_gbase[tid] = H[(size_t)tid * gridDim.x + blockIdx.x];
     __syncthreads();
+#if GS_LSD_PREMATCH
+    // every item's peers first (independent), then the counter chain
+#pragma unroll
+    for (int k = 0; k < kScatterItems; k++) {
+        const uint32_t i = (uint32_t)(warp * 32 * kScatterItems + 32 * k + lane);
+        const uint32_t d = i < m ? (key[k] >> shift) & mask : (uint32_t)kRadix;
+#if GS_LSD_MATCH
+        rank[k] = __match_any_sync(0xffffffffu, d);
+#else
+        rank[k] = digit_peers(d, bits);
+#endif
+    }
+#pragma unroll
+    for (int k = 0; k < kScatterItems; k++) {
+        const uint32_t i = (uint32_t)(warp * 32 * kScatterItems + 32 * k + lane);
+        const uint32_t d = i < m ? (key[k] >> shift) & mask : (uint32_t)kRadix;
+        const uint32_t peers = rank[k];
+        rank[k] = d < kRadix ? s_cnt[warp][d] + __popc(peers & lt) : 0u;
+        __syncwarp();
+        if (d < kRadix && lane == __ffs(peers) - 1) s_cnt[warp][d] += __popc(peers);
+        __syncwarp();
+    }
+#else
 #pragma unroll
     for (int k = 0; k < kScatterItems; k++) {
         const uint32_t i = (uint32_t)(warp * 32 * kScatterItems + 32 * k + lane);
@@ -792,6 +833,7 @@ k_lsd_scatter(const uint32_t *__restrict__ keys_in, const uint32_t *__restrict__
         if (d < kRadix && lane == __ffs(peers) - 1) s_cnt[warp][d] += __popc(peers);
         __syncwarp();
     }
+#endif
     __syncthreads();
     if (tid < kRadix) {  // exclusive over the warps, per digit; digit totals of the tile
         uint32_t tot = 0;
@@ -833,13 +875,13 @@ __device__ __forceinline__ uint32_t ranked_count(const int4 *__restrict__ rect, 
     return rect_tiles(rect[order[r]], tiles_x, tiles_y, x0, y0, w);
 }
 
-__device__ __forceinline__ uint32_t block_sum_512(uint32_t v, uint32_t *s_w) {
+__device__ __forceinline__ uint64_t block_sum_512_u64(uint64_t v, uint64_t *s_w) {
     const int lane = threadIdx.x & 31, w = threadIdx.x >> 5;
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
     if (lane == 0) s_w[w] = v;
     __syncthreads();
-    uint32_t t = 0;
+    uint64_t t = 0;
 #pragma unroll
     for (int k = 0; k < kLsdWarps; k++) t += s_w[k];
     __syncthreads();
@@ -848,27 +890,38 @@ __device__ __forceinline__ uint32_t block_sum_512(uint32_t v, uint32_t *s_w) {
 
 __global__ void __launch_bounds__(kLsdThreads)
 k_rank_sums(int n, const int4 *__restrict__ rect, const uint32_t *__restrict__ order, int tiles_x, int tiles_y,
-            uint32_t *__restrict__ S, const int32_t *__restrict__ status) {
-    __shared__ uint32_t s_w[kLsdWarps];
+            uint64_t *__restrict__ S, const int32_t *__restrict__ status) {
+    __shared__ uint64_t s_w[kLsdWarps];
     if (*(volatile const int32_t *)status != 0) return;
     uint32_t lo, hi;
     lsd_chunk((uint64_t)n, lo, hi);
-    uint32_t sum = 0;
+    uint64_t sum = 0;
     for (uint32_t r = lo + threadIdx.x; r < hi; r += kLsdThreads) sum += ranked_count(rect, order, r, tiles_x, tiles_y);
-    sum = block_sum_512(sum, s_w);
+    sum = block_sum_512_u64(sum, s_w);
     if (threadIdx.x == 0) S[blockIdx.x] = sum;
 }
 
-// offsets[r] = pairs of the Gaussians ranked before r (exclusive scan).
+// offsets[r] = pairs of the Gaussians ranked before r (exclusive scan).  The
+// last CTA also records K and the capacity check (GS_ERR_CAPACITY: the
+// kernels after it then write nothing).
 __global__ void __launch_bounds__(kLsdThreads)
 k_rank_offsets(int n, const int4 *__restrict__ rect, const uint32_t *__restrict__ order, int tiles_x, int tiles_y,
-               const uint32_t *__restrict__ S, uint32_t *__restrict__ offsets, const int32_t *__restrict__ status) {
+               const uint64_t *__restrict__ S, uint32_t *__restrict__ offsets, uint64_t *__restrict__ n_pairs,
+               uint64_t max_pairs, int32_t *__restrict__ status) {
     __shared__ uint32_t s_w[kLsdWarps];
+    __shared__ uint64_t s_w64[kLsdWarps];
     if (*(volatile const int32_t *)status != 0) return;
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-    uint32_t base = 0;
-    for (int c = tid; c < (int)blockIdx.x; c += kLsdThreads) base += S[c];
-    base = block_sum_512(base, s_w);
+    uint64_t before = 0;
+    for (int c = tid; c < (int)blockIdx.x; c += kLsdThreads) before += S[c];
+    before = block_sum_512_u64(before, s_w64);
+    if (blockIdx.x == gridDim.x - 1 && tid == 0) {
+        const uint64_t K = before + S[blockIdx.x];
+        *n_pairs = K;
+        if (K > max_pairs) set_status(status, GS_ERR_CAPACITY);
+    }
+    if (before + S[blockIdx.x] > max_pairs) return;  // the capacity error: offsets are not needed
+    uint32_t base = (uint32_t)before;
     uint32_t lo, hi;
     lsd_chunk((uint64_t)n, lo, hi);
     for (uint32_t c0 = lo; c0 < hi; c0 += kLsdThreads) {
@@ -893,6 +946,56 @@ k_rank_offsets(int n, const int4 *__restrict__ rect, const uint32_t *__restrict_
         base += total;
         __syncthreads();
     }
+}
+
+// Each tile's [start, end) in the sorted pair list (ranges zeroed by the
+// caller, so empty tiles stay [0, 0)), then each tile's total.  Thread j
+// compares the four tile ids 4 j .. 4 j + 3 (one 16-byte load) and the next
+// one: a change between positions p - 1 and p ends one tile's range and
+// starts the next's at p.
+__device__ __forceinline__ void tile_boundary(uint32_t a, uint32_t b, uint32_t p, uint32_t *__restrict__ ranges,
+                                              uint32_t tiles, int32_t *__restrict__ status) {
+    if (a == b) return;
+    if (in_bounds(a, tiles, status)) ranges[2 * (size_t)a + 1] = p;
+    if (in_bounds(b, tiles, status)) ranges[2 * (size_t)b] = p;
+}
+
+__global__ void __launch_bounds__(256)
+k_tile_bounds(const uint32_t *__restrict__ pair_tile, const uint64_t *__restrict__ n_pairs,
+              uint32_t *__restrict__ ranges, int32_t *__restrict__ status, uint32_t tiles) {
+    if (*(volatile const int32_t *)status != 0) return;
+    const uint32_t K = (uint32_t)*n_pairs;  // at most max_pairs < 2^30 here
+    if (K == 0) return;
+    const uint32_t groups = (K + 3) / 4;
+    for (uint32_t j = blockIdx.x * blockDim.x + threadIdx.x; j < groups; j += gridDim.x * blockDim.x) {
+        const uint32_t i0 = 4 * j;
+        uint32_t t[5];
+        if (i0 + 4 <= K) {
+            const uint4 v = reinterpret_cast<const uint4 *>(pair_tile)[j];
+            t[0] = v.x; t[1] = v.y; t[2] = v.z; t[3] = v.w;
+        } else {
+#pragma unroll
+            for (int k = 0; k < 4; k++) t[k] = i0 + k < K ? pair_tile[i0 + k] : 0u;
+        }
+        t[4] = i0 + 4 < K ? pair_tile[i0 + 4] : 0u;
+        if (j == 0 && in_bounds(t[0], tiles, status)) ranges[2 * (size_t)t[0]] = 0;
+#pragma unroll
+        for (int k = 0; k < 4; k++) {
+            const uint32_t p = i0 + k + 1;  // boundary between positions p - 1 and p
+            if (p > K) break;
+            if (p == K) {
+                if (in_bounds(t[k], tiles, status)) ranges[2 * (size_t)t[k] + 1] = K;
+            } else {
+                tile_boundary(t[k], t[k + 1], p, ranges, tiles, status);
+            }
+        }
+    }
+}
+
+__global__ void __launch_bounds__(256)
+k_tile_totals(const uint32_t *__restrict__ ranges, int tiles, uint32_t *__restrict__ totals) {
+    const int t = blockIdx.x * blockDim.x + threadIdx.x;
+    if (t < tiles) totals[t] = ranges[2 * (size_t)t + 1] - ranges[2 * (size_t)t];
 }
 
 // Each Gaussian (rank r, id order[r]) writes the tile id and its id for
@@ -1012,14 +1115,25 @@ cudaError_t launch_bin_global(const CamConst &c, int64_t n, const gs_projected &
     char *base = static_cast<char *>(bins.scratch);
     auto U32 = [&](size_t off) { return reinterpret_cast<uint32_t *>(base + off); };
     int32_t *status = reinterpret_cast<int32_t *>(base + L.status);
-    const uint64_t *n_pairs = reinterpret_cast<const uint64_t *>(base + L.n_pairs);
+    uint64_t *n_pairs = reinterpret_cast<uint64_t *>(base + L.n_pairs);
     uint32_t *H = U32(L.bin_hist);
+    uint32_t *ranges = U32(L.ranges), *totals = U32(L.tile_total), *order = U32(L.tile_order);
+    const int tiles_c = c.tiles_x * c.tiles_y;
+    // no count phase on this path: ranges and totals start empty
+    cudaError_t e = cudaMemsetAsync(totals, 0, (size_t)tiles_c * sizeof(uint32_t), s);
+    if (e == cudaSuccess) e = cudaMemsetAsync(ranges, 0, (size_t)tiles_c * 2 * sizeof(uint32_t), s);
+    if (e != cudaSuccess) return e;
+    if (n == 0) {  // K = 0: every range empty, every tile in the order
+        k_tile_scan<<<1, kScanTilesThreads, 0, s>>>(tiles_c, totals, (uint64_t)bins.max_pairs, ranges, order,
+                                                    n_pairs, status);
+        return cudaGetLastError();
+    }
     const size_t pb = align_up((size_t)bins.max_pairs * sizeof(uint32_t), 256);
     uint32_t *KA = U32(L.keys), *VA = U32(L.keys + pb);  // the key array's two halves
     uint32_t *KB = U32(L.long_keys), *VB = U32(L.long_ids);
     const int4 *rect = reinterpret_cast<const int4 *>(proj.rect);
     const float4 *xyod = reinterpret_cast<const float4 *>(proj.xy_opacity_depth);
-    const int tiles = c.tiles_x * c.tiles_y;
+    const int tiles = tiles_c;
     const uint32_t nn = (uint32_t)n;
     // 4. the Gaussians by depth: four stable 8-bit passes, A -> B -> A -> B -> A
     prof_before("depth_sort", s);
@@ -1033,9 +1147,10 @@ cudaError_t launch_bin_global(const CamConst &c, int64_t n, const gs_projected &
     // 5. each Gaussian's first pair position in depth order (into KA), then
     // the pairs in (depth, id) order into (KB, VB)
     prof_before("emit", s);
-    uint32_t *S = H;
+    uint64_t *S = reinterpret_cast<uint64_t *>(H);
     k_rank_sums<<<ctas, kLsdThreads, 0, s>>>((int)n, rect, VA, c.tiles_x, c.tiles_y, S, status);
-    k_rank_offsets<<<ctas, kLsdThreads, 0, s>>>((int)n, rect, VA, c.tiles_x, c.tiles_y, S, KA, status);
+    k_rank_offsets<<<ctas, kLsdThreads, 0, s>>>((int)n, rect, VA, c.tiles_x, c.tiles_y, S, KA, n_pairs,
+                                                (uint64_t)bins.max_pairs, status);
     const int emit_blocks = (int)std::min<int64_t>((n + 255) / 256, (int64_t)8 * sms);
     k_emit_ranked<<<emit_blocks, 256, 0, s>>>((int)n, rect, VA, KA, c.tiles_x, c.tiles_y, KB, VB, status,
                                               (uint64_t)bins.max_pairs);
@@ -1054,6 +1169,15 @@ cudaError_t launch_bin_global(const CamConst &c, int64_t n, const gs_projected &
         lsd_pass(ki, vi, ko, vo, n_pairs, 0u, bins.max_pairs, digit * p, bits, H, status, s);
     }
     prof_after(s, 4 * passes);
+    // 7. each tile's range off the sorted list, its total, then the tile
+    // scan as on the per-tile path (ranges again, K kept, the tile order)
+    prof_before("tile_scan", s);
+    const int bound_blocks = (int)std::min<int64_t>((bins.max_pairs / 4 + 255) / 256, (int64_t)32 * sms);
+    k_tile_bounds<<<std::max(1, bound_blocks), 256, 0, s>>>(bins.pair_tile, n_pairs, ranges, status, (uint32_t)tiles);
+    k_tile_totals<<<(tiles + 255) / 256, 256, 0, s>>>(ranges, tiles, totals);
+    k_tile_scan<<<1, kScanTilesThreads, 0, s>>>(tiles, totals, (uint64_t)bins.max_pairs, ranges, order, n_pairs,
+                                                status);
+    prof_after(s, 3);
     return cudaGetLastError();
 }
 
@@ -1080,6 +1204,15 @@ cudaError_t launch_bin_and_sort(const CamConst &c, int64_t n, const gs_projected
     const size_t cnt_smem = tiles <= kSmemTiles ? (size_t)tiles * sizeof(uint32_t) : 0;
     e = cudaMemsetAsync(base, 0, L.zero_bytes, s);
     if (e != cudaSuccess) return e;
+    // the strategy (gs.h GS_BIN_*); the global path's LSD passes keep their
+    // per-tile digit counts in the count matrix's space
+    const int64_t hist_cap = std::min<int64_t>((int64_t)kBinCTAsMax * bins.max_tiles, kBinHistCap);
+    const int lsd_ctas = (int)std::min<int64_t>((int64_t)2 * sms, hist_cap);
+    bool global = bins.strategy == GS_BIN_GLOBAL;
+    if (bins.strategy == GS_BIN_AUTO)
+        global = bins.max_pairs >= (int64_t)1024 * tiles;
+    global = global && n <= bins.max_pairs && lsd_space(bins.max_pairs) <= hist_cap;
+    if (global) return launch_bin_global(c, n, proj, bins, L, lsd_ctas, sms, s);
     // 1. per-CTA tile counts, 2. offsets down each tile's column
     prof_before("bin_count", s);
     k_bin_count<<<ctas, kBinThreads, cnt_smem, s>>>((int)n, rect, c.tiles_x, c.tiles_y, H, status);
@@ -1091,16 +1224,6 @@ cudaError_t launch_bin_and_sort(const CamConst &c, int64_t n, const gs_projected
                                                 n_pairs, status);
     prof_after(s);
     if (n == 0) return cudaGetLastError();  // K = 0, all ranges empty
-    // the global path's LSD passes keep per-CTA digit counts in the count
-    // matrix's space (free once the tile scan has run)
-    const int64_t hist_cap = std::min<int64_t>((int64_t)kBinCTAsMax * bins.max_tiles, kBinHistCap);
-    const int lsd_ctas = (int)std::min<int64_t>((int64_t)2 * sms, hist_cap);
-    bool global = bins.strategy == GS_BIN_GLOBAL;
-    if (bins.strategy == GS_BIN_AUTO)
-        global = bins.max_pairs >= (int64_t)1024 * tiles;
-    // the passes' digit counts must fit the count matrix's space
-    global = global && n <= bins.max_pairs && lsd_space(bins.max_pairs) <= hist_cap;
-    if (global) return launch_bin_global(c, n, proj, bins, L, lsd_ctas, sms, s);
     // 4. emit the sort keys
     prof_before("emit", s);
     k_bin_emit<<<ctas, kBinThreads, cnt_smem, s>>>((int)n, rect, reinterpret_cast<const float4 *>(proj.xy_opacity_depth),
