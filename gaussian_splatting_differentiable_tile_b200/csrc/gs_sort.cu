@@ -587,7 +587,7 @@ k_tile_sort(const uint32_t *__restrict__ ranges, const uint32_t *__restrict__ or
 // Ranking of an LSD pass's digits within a warp: one match instruction (1),
 // or one ballot per digit bit (0).  A tuning knob.
 #ifndef GS_LSD_MATCH
-#define GS_LSD_MATCH 1
+#define GS_LSD_MATCH 0
 #endif
 // Resident scatter CTAs per SM the register allocation targets (a tuning
 // knob).
@@ -595,7 +595,7 @@ k_tile_sort(const uint32_t *__restrict__ ranges, const uint32_t *__restrict__ or
 #define GS_LSD_PREMATCH 0
 #endif
 #ifndef GS_LSD_MINB
-#define GS_LSD_MINB 3
+#define GS_LSD_MINB 2
 #endif
 constexpr int kLsdThreads = 512;
 constexpr int kLsdWarps = kLsdThreads / 32;
@@ -765,8 +765,8 @@ k_scan_add(uint32_t *__restrict__ H, uint32_t m, const uint32_t *__restrict__ S,
 
 // Stable scatter of one LSD pass, CTA b taking tile b: warp w holds elements
 // w * 256 + 32 k + lane (k = 0 .. 7), so (w, k, lane) is the input order.
-// Each warp ranks its elements within their digit in that order (one match
-// instruction per 32 elements, per-warp counters in shared memory); a scan
+// Each warp ranks its elements within their digit in that order (one ballot
+// per digit bit per 32 elements, per-warp counters in shared memory); a scan
 // over the warps and over the digits places each element in the tile sorted
 // by digit, in shared memory; the tile then goes out digit run by digit run,
 // each run contiguous at the scanned H[d][b], so the writes are coalesced.

@@ -184,6 +184,29 @@ def test_bin_and_sort_capacity_error_and_async_status(strategy):
     assert G.gs_bin_and_sort(cam, n, proj, bins2) == need
 
 
+@pytest.mark.parametrize("count,offset", [(4 * 100_003, 0), (4 * 100_003 + 3, 0), (4 * 100_003, 1)])
+def test_l1_loss_grad_vector_and_scalar_paths(count, offset):
+    """gs_l1_loss_grad against the oracle's loss and gradient: a count that is
+    a multiple of 4 with aligned arrays (16-byte loads), a ragged count, and
+    arrays offset by one float (both take the one-value loop).  Values are
+    multiples of 1/64 and distinct per element pair, so image - target is
+    exact in fp32 and its sign is unambiguous (zeros included)."""
+    rng = np.random.default_rng(count + offset)
+    img = rng.integers(-64, 64, count).astype(np.float32) / 64
+    tgt = rng.integers(-64, 64, count).astype(np.float32) / 64
+    buf = torch.empty(3 * (count + 4), device="cuda")
+    base = lambda k: buf[k * (count + 4) + offset:k * (count + 4) + offset + count]
+    image, target, dl = base(0), base(1), base(2)
+    image.copy_(torch.from_numpy(img))
+    target.copy_(torch.from_numpy(tgt))
+    loss = torch.zeros(1, device="cuda")
+    G.gs_l1_loss_grad(image, target, dl, loss)
+    torch.cuda.synchronize()
+    loss_ref, dl_ref = OT.l1_loss_grad(img, tgt)
+    np.testing.assert_allclose(dl.cpu().numpy().astype(np.float64), dl_ref, rtol=1e-7, atol=0)
+    assert abs(loss.item() - loss_ref) <= 1e-5 * max(loss_ref, 1.0)
+
+
 def test_argument_errors_launch_nothing():
     cam = tiny_camera()
     proj = G.Projected(10)
