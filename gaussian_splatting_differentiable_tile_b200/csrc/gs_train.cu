@@ -105,26 +105,15 @@ __global__ void k_adam_tick(int64_t *step) { *step += 1; }
 __global__ void __launch_bounds__(256)
 k_l1_train(const float *__restrict__ image, const float *__restrict__ target, int64_t count,
            float *__restrict__ dL, float *__restrict__ loss, const int32_t *__restrict__ bin_status,
-           const uint64_t *__restrict__ bin_pairs, int64_t *__restrict__ stats, bool vec) {
+           const uint64_t *__restrict__ bin_pairs, int64_t *__restrict__ stats) {
     __shared__ float s_w[8];
     const float inv = 1.f / (float)count;
-    auto grad = [&](float d) { return d > 0.f ? inv : (d < 0.f ? -inv : 0.f); };
     float acc = 0.f;
-    const int64_t first = (int64_t)blockIdx.x * blockDim.x + threadIdx.x, step = (int64_t)gridDim.x * blockDim.x;
-    if (vec) {  // count a multiple of 4, every array 16-byte aligned
-        for (int64_t i = first; i < count / 4; i += step) {
-            const float4 a = reinterpret_cast<const float4 *>(image)[i];
-            const float4 t = reinterpret_cast<const float4 *>(target)[i];
-            const float4 d = make_float4(a.x - t.x, a.y - t.y, a.z - t.z, a.w - t.w);
-            reinterpret_cast<float4 *>(dL)[i] = make_float4(grad(d.x), grad(d.y), grad(d.z), grad(d.w));
-            acc += (fabsf(d.x) + fabsf(d.y)) + (fabsf(d.z) + fabsf(d.w));
-        }
-    } else {
-        for (int64_t i = first; i < count; i += step) {
-            const float d = image[i] - target[i];
-            dL[i] = grad(d);
-            acc += fabsf(d);
-        }
+    for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < count;
+         i += (int64_t)gridDim.x * blockDim.x) {
+        const float d = image[i] - target[i];
+        dL[i] = d > 0.f ? inv : (d < 0.f ? -inv : 0.f);
+        acc += fabsf(d);
     }
     if (stats && blockIdx.x == 0 && threadIdx.x == 0) {
         stats[0] = (int64_t)*bin_status;
@@ -184,13 +173,11 @@ cudaError_t launch_l1_train(const float *image, const float *target, int64_t cou
         cudaError_t e = cudaMemsetAsync(loss, 0, sizeof(float), s);
         if (e != cudaSuccess) return e;
     }
-    auto a16 = [](const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; };
-    const bool vec = count % 4 == 0 && a16(image) && a16(target) && a16(dL_dimage);
-    const int64_t want = ((vec ? count / 4 : count) + 255) / 256;
+    const int64_t want = (count + 255) / 256;
     const int blocks = (int)std::max<int64_t>(1, std::min<int64_t>(want, (int64_t)num_sms_train() * 8));
     prof_before("l1_loss", s);
     k_l1_train<<<blocks, 256, 0, s>>>(image, target, count, dL_dimage, loss, bins.status,
-                                      reinterpret_cast<const uint64_t *>(bins.n_pairs), stats, vec);
+                                      reinterpret_cast<const uint64_t *>(bins.n_pairs), stats);
     prof_after(s);
     return cudaGetLastError();
 }

@@ -185,12 +185,11 @@ def test_bin_and_sort_capacity_error_and_async_status(strategy):
 
 
 @pytest.mark.parametrize("count,offset", [(4 * 100_003, 0), (4 * 100_003 + 3, 0), (4 * 100_003, 1)])
-def test_l1_loss_grad_vector_and_scalar_paths(count, offset):
+def test_l1_loss_grad_sizes_and_offsets(count, offset):
     """gs_l1_loss_grad against the oracle's loss and gradient: a count that is
-    a multiple of 4 with aligned arrays (16-byte loads), a ragged count, and
-    arrays offset by one float (both take the one-value loop).  Values are
-    multiples of 1/64 and distinct per element pair, so image - target is
-    exact in fp32 and its sign is unambiguous (zeros included)."""
+    a multiple of 4 with aligned arrays, a ragged count, and arrays offset by
+    one float.  Values are multiples of 1/64, so image - target is exact in
+    fp32 and its sign is unambiguous (zeros included)."""
     rng = np.random.default_rng(count + offset)
     img = rng.integers(-64, 64, count).astype(np.float32) / 64
     tgt = rng.integers(-64, 64, count).astype(np.float32) / 64
