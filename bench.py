@@ -5,7 +5,8 @@
 
 One step = one training frame through the whole hot path for one camera:
 project -> bin and sort -> forward blend -> L1 loss gradient -> backward blend
--> projection backward.  Default workload: a seeded synthetic 400k-Gaussian
+-> projection backward (gs_train_step, the `train_step` of the line, takes
+the L1 loss in the forward's epilogue).  Default workload: a seeded synthetic 400k-Gaussian
 scene (120 anisotropic clusters in a 10 m box, log-scales N(-4, 0.6), opacity
 logits N(1, 1.5)) seen from 16 ring cameras at 980 x 545, f = 1000, L1 loss
 against a seeded U(0, 1) target.  Inputs are resident in HBM; L2 (126 MB) is
@@ -338,17 +339,22 @@ def run_profile_frame(args, spec):
         K = e.n_pairs
     r.bins = G.Bins(spec.n, int(K * 1.05) + 4096, spec.width, spec.height, strategy=BINNING[args.binning])
     torch.cuda.synchronize()
-    torch.cuda.nvtx.range_push("frame")
-    image = r.forward(cam, params, sync=True)
     target = torch.from_numpy(make_target(spec.width, spec.height, channels=G.channels(cam))).cuda()
-    dl = torch.empty_like(image)
+    r.image = torch.empty(tuple(target.shape), device="cuda")
+    dl = torch.empty_like(r.image)
     loss = torch.zeros(1, device="cuda")
-    G.gs_l1_loss_grad(image, target, dl, loss)
+    torch.cuda.synchronize()
+    # the bench's step: project, bin, forward, L1 loss, backward
+    torch.cuda.nvtx.range_push("frame")
+    G.gs_project(cam, params, r.proj)
+    G.gs_bin_and_sort(cam, spec.n, r.proj, r.bins, sync=False)
+    G.gs_render_fwd(cam, spec.n, r.proj, r.bins, r.image, r.T_final, r.last)
+    G.gs_l1_loss_grad(r.image, target, dl, loss)
     r.backward(cam, params, dl)
     torch.cuda.nvtx.range_pop()
     torch.cuda.synchronize()
     print(json.dumps({"profile_frame": spec.name, "camera": args.profile_camera, "tiles": args.tiles,
-                      "pairs": r.n_pairs, "binning": _binning_used(args.binning, r.bins.max_pairs, spec),
+                      "pairs": K, "binning": _binning_used(args.binning, r.bins.max_pairs, spec),
                       "loss": loss.item()}), flush=True)
 
 

@@ -31,7 +31,7 @@ from ._abi import (GS_BIN_AUTO, GS_BIN_GLOBAL, GS_BIN_PER_TILE, GS_ERR_ALIGNMENT
 
 __all__ = [
     "GSError", "Projected", "Bins", "make_camera", "channels", "gs_project", "gs_bin_and_sort",
-    "gs_bin_and_sort_static", "gs_render_fwd", "gs_render_features_fwd", "gs_render_features_bwd",
+    "gs_bin_and_sort_static", "gs_render_fwd", "gs_render_fwd_l1", "gs_render_features_fwd", "gs_render_features_bwd",
     "gs_render_bwd", "gs_render_stats", "gs_l1_loss_grad", "gs_read_status", "gs_last_device_error",
     "gs_sort_bytes", "gs_error_string", "profile_begin",
     "profile_end", "lib", "PARAM_KEYS",
@@ -220,6 +220,27 @@ def gs_render_fwd(cam, n: int, proj: Projected, bins: Bins, image: torch.Tensor,
     _check(lib().gs_render_fwd(ctypes.byref(c), int(n), ctypes.byref(proj.struct), ctypes.byref(bins.struct),
                                _dev(image, "image", torch.float32), _dev(T_final, "T_final", torch.float32),
                                _dev(last, "last", torch.int32), _stream(stream)), "gs_render_fwd")
+
+
+def gs_render_fwd_l1(cam, n: int, proj: Projected, bins: Bins, image: torch.Tensor, T_final: torch.Tensor,
+                     last: torch.Tensor, target: torch.Tensor, dL_dimage: torch.Tensor,
+                     loss: torch.Tensor | None = None, stream=None) -> None:
+    """gs_render_fwd plus the L1 loss (into loss, zeroed first) and its
+    gradient dL_dimage in the same kernel."""
+    H, W = int(cam.height), int(cam.width)
+    ch = channels(cam)
+    if image.numel() != H * W * ch or T_final.numel() != H * W or last.numel() != H * W:
+        raise ValueError(f"output tensors must be [H,W,{ch}], [H,W], [H,W]")
+    if target.numel() != H * W * ch or dL_dimage.numel() != H * W * ch:
+        raise ValueError(f"target and dL_dimage must be [H,W,{ch}]")
+    if loss is not None and loss.numel() < 1:
+        raise ValueError("loss must hold one float")
+    c = make_camera(cam)
+    _check(lib().gs_render_fwd_l1(ctypes.byref(c), int(n), ctypes.byref(proj.struct), ctypes.byref(bins.struct),
+                                  _dev(image, "image", torch.float32), _dev(T_final, "T_final", torch.float32),
+                                  _dev(last, "last", torch.int32), _dev(target, "target", torch.float32),
+                                  _dev(dL_dimage, "dL_dimage", torch.float32), _dev(loss, "loss", torch.float32),
+                                  _stream(stream)), "gs_render_fwd_l1")
 
 
 def gs_render_bwd(cam, n: int, params: dict, proj: Projected, bins: Bins, T_final: torch.Tensor,

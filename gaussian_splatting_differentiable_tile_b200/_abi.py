@@ -110,6 +110,9 @@ PROTOTYPES = {
     "gs_render_fwd": (ctypes.c_int, [ctypes.POINTER(GsCamera), ctypes.c_int64, ctypes.POINTER(GsProjected),
                                      ctypes.POINTER(GsBins), ctypes.c_void_p, ctypes.c_void_p,
                                      ctypes.c_void_p, ctypes.c_void_p]),
+    "gs_render_fwd_l1": (ctypes.c_int, [ctypes.POINTER(GsCamera), ctypes.c_int64, ctypes.POINTER(GsProjected),
+                                        ctypes.POINTER(GsBins), ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p,
+                                        ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p]),
     "gs_render_bwd": (ctypes.c_int, [ctypes.POINTER(GsCamera), ctypes.c_int64, ctypes.POINTER(GsParams),
                                      ctypes.POINTER(GsProjected), ctypes.POINTER(GsBins), ctypes.c_void_p,
                                      ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p,

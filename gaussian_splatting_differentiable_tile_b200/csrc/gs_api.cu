@@ -269,6 +269,25 @@ int gs_render_fwd(const gs_camera *cam, int64_t n, const gs_projected *proj, con
                : GS_ERR_CUDA;
 }
 
+int gs_render_fwd_l1(const gs_camera *cam, int64_t n, const gs_projected *proj, const gs_bins *bins,
+                     float *image, float *T_final, uint32_t *last, const float *target, float *dL_dimage,
+                     float *loss, void *stream) {
+    CamConst c;
+    int rc = make_cam(cam, &c);
+    if (rc) return rc;
+    if (n < 0) return GS_ERR_INVALID_ARG;
+    BinsLayout L;
+    if ((rc = check_projected(proj, n)) || (rc = check_bins(bins, n, c, &L))) return rc;
+    if (!image || !T_final || !last || !target || !dL_dimage) return GS_ERR_INVALID_ARG;
+    if (!aligned(image, 4) || !aligned(T_final, 4) || !aligned(last, 4) || !aligned(target, 4) ||
+        !aligned(dL_dimage, 4) || (loss && !aligned(loss, 4)))
+        return GS_ERR_ALIGNMENT;
+    return launch_render_fwd(c, n, *proj, *bins, image, T_final, last, as_stream(stream), target, dL_dimage,
+                             loss) == cudaSuccess
+               ? GS_OK
+               : GS_ERR_CUDA;
+}
+
 int gs_render_bwd(const gs_camera *cam, int64_t n, const gs_params *params,
                   const gs_projected *proj, const gs_bins *bins, const float *T_final,
                   const uint32_t *last, const float *dL_dimage, float *grad2d,
@@ -527,10 +546,9 @@ int gs_train_step(const gs_camera *cams, int32_t n_cams, int64_t n, const gs_par
             const gs_params &pp = pc;
             if (launch_project(c, n, pp, ln.proj, ls) != cudaSuccess ||
                 launch_bin_and_sort(c, n, ln.proj, ln.bins, L[l], ls) != cudaSuccess ||
-                launch_render_fwd(c, n, ln.proj, ln.bins, ln.image, ln.T_final, ln.last, ls) != cudaSuccess ||
-                launch_l1_train(ln.image, targets + (size_t)b * values, values, ln.dL_dimage,
-                                losses ? losses + b : nullptr, ln.bins, cam_stats ? cam_stats + 2 * b : nullptr,
-                                ls) != cudaSuccess)
+                launch_render_fwd(c, n, ln.proj, ln.bins, ln.image, ln.T_final, ln.last, ls,
+                                  targets + (size_t)b * values, ln.dL_dimage, losses ? losses + b : nullptr,
+                                  cam_stats ? cam_stats + 2 * b : nullptr) != cudaSuccess)
                 return GS_ERR_CUDA;
             if (n > 0 && cudaMemsetAsync(ln.grad2d, 0, (size_t)n * 12 * sizeof(float), ls) != cudaSuccess)
                 return GS_ERR_CUDA;

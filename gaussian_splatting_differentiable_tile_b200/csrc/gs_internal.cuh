@@ -162,8 +162,13 @@ cudaError_t launch_project_bwd(const CamConst &c, int64_t n, const gs_params &p,
                                cudaStream_t s, bool accumulate = false);
 cudaError_t launch_bin_and_sort(const CamConst &c, int64_t n, const gs_projected &proj,
                                 const gs_bins &bins, const BinsLayout &L, cudaStream_t s);
+// With target: the L1 loss in the epilogue (dL_dimage written, *loss zeroed
+// then summed when not null, stats[0..1] = the bins' status and K when not
+// null).
 cudaError_t launch_render_fwd(const CamConst &c, int64_t n, const gs_projected &proj, const gs_bins &bins,
-                              float *image, float *T_final, uint32_t *last, cudaStream_t s);
+                              float *image, float *T_final, uint32_t *last, cudaStream_t s,
+                              const float *target = nullptr, float *dL_dimage = nullptr, float *loss = nullptr,
+                              int64_t *stats = nullptr);
 cudaError_t launch_render_bwd(const CamConst &c, int64_t n, const gs_projected &proj, const gs_bins &bins,
                               const float *T_final, const uint32_t *last, const float *dL_dimage,
                               float *grad2d, cudaStream_t s);
@@ -180,8 +185,6 @@ cudaError_t launch_render_stats(const CamConst &c, int64_t n, const gs_projected
                                 const uint32_t *last, uint64_t *counts, cudaStream_t s);
 cudaError_t launch_l1(const float *image, const float *target, int64_t count, float *dL_dimage,
                       float *loss, cudaStream_t s);
-cudaError_t launch_l1_train(const float *image, const float *target, int64_t count, float *dL_dimage,
-                            float *loss, const gs_bins &bins, int64_t *stats, cudaStream_t s);
 // update: k_adam_tick (advances *step), then k_adam when max_count > 0;
 // otherwise only the scaled slot sum is written to each group's `out`
 struct AdamBetas {

@@ -117,6 +117,21 @@ struct ChannelIO {
     int cgrad_stride;   // in floats
 };
 
+// The L1 loss of a training step taken in the forward's epilogue ([GSP] s7:
+// loss = mean |image - target| over every value, its gradient
+// sign(image - target) / count): each pixel's values against the target,
+// the gradient written per value, the loss summed per CTA and added once.
+// stats (nullable): [0] the bins' status word, [1] K, copied by CTA 0.
+struct L1Out {
+    const float *target;  // [H][W][channels]
+    float *dL;            // [H][W][channels]
+    float *loss;          // [1], zeroed by the caller; nullable
+    float inv;            // 1 / (H W channels), rounded once
+    int64_t *stats;
+    const int32_t *bin_status;
+    const uint64_t *bin_pairs;
+};
+
 // The blend's two skip tests (sigma < 0, alpha < 1/255) on the exponent
 // q = -sigma log2(e) as one range test: a pixel takes the entry iff
 // log2(1/255) - log2 o <= q <= 0, i.e. |q - c| <= -c with
@@ -262,13 +277,13 @@ __device__ __forceinline__ uint32_t block_mask(const float4 geo, const float4 ge
     return m;
 }
 
-template <bool kDepth, bool kFeat = false>
+template <bool kDepth, bool kFeat = false, bool kL1 = false>
 __global__ void __launch_bounds__(kTilePixels, GS_FWD_MINB)
 k_render_fwd(CamConst cam, const float4 *__restrict__ xyod, const float4 *__restrict__ conr,
              const ChannelIO io, const uint32_t *__restrict__ pair_gid,
              const uint2 *__restrict__ ranges, const uint32_t *__restrict__ order,
              float *__restrict__ image, float *__restrict__ T_final, uint32_t *__restrict__ last,
-             const Bounds bd) {
+             const Bounds bd, const L1Out l1 = L1Out{}) {
     constexpr int kWarps = kTilePixels / 32;
     __shared__ float4 s_geo[kBatch];
     __shared__ float4 s_geo2[kBatch];
@@ -414,15 +429,44 @@ k_render_fwd(CamConst cam, const float4 *__restrict__ xyod, const float4 *__rest
             __syncwarp();
         }
     }
+    float l1_sum = 0.f;
     if (px < cam.width && py < cam.height) {
         const size_t p = (size_t)py * cam.width + px;
-        float *out = image + (size_t)(kFeat ? io.img_stride : (kDepth ? 4 : 3)) * p;
-        out[0] = __fmaf_rn(T, cam.bg[0], C0);
-        out[1] = __fmaf_rn(T, cam.bg[1], C1);
-        out[2] = __fmaf_rn(T, cam.bg[2], C2);
-        if (kDepth) out[3] = C3;  // the fourth channel has no background
+        constexpr int kC = kDepth ? 4 : 3;
+        float *out = image + (size_t)(kFeat ? io.img_stride : kC) * p;
+        const float o[4] = {__fmaf_rn(T, cam.bg[0], C0), __fmaf_rn(T, cam.bg[1], C1),
+                            __fmaf_rn(T, cam.bg[2], C2), C3};  // the fourth channel has no background
+#pragma unroll
+        for (int c = 0; c < kC; c++) out[c] = o[c];
         if (T_final) T_final[p] = T;
         if (last) last[p] = lst;
+        if (kL1) {
+#pragma unroll
+            for (int c = 0; c < kC; c++) {
+                const float d = o[c] - l1.target[kC * p + c];
+                l1.dL[kC * p + c] = d > 0.f ? l1.inv : (d < 0.f ? -l1.inv : 0.f);
+                l1_sum += fabsf(d);
+            }
+        }
+    }
+    if (kL1) {
+        if (l1.stats && blockIdx.x == 0 && threadIdx.x == 0) {
+            l1.stats[0] = (int64_t)*l1.bin_status;
+            l1.stats[1] = (int64_t)*l1.bin_pairs;
+        }
+        if (l1.loss) {
+            __shared__ float s_l1[kWarps];
+#pragma unroll
+            for (int o = 16; o > 0; o >>= 1) l1_sum += __shfl_xor_sync(0xffffffffu, l1_sum, o);
+            if (lane == 0) s_l1[warp] = l1_sum;
+            __syncthreads();
+            if (threadIdx.x == 0) {
+                float t = 0.f;
+#pragma unroll
+                for (int w = 0; w < kWarps; w++) t += s_l1[w];
+                atomicAdd(l1.loss, t * l1.inv);
+            }
+        }
     }
 }
 
@@ -798,22 +842,42 @@ static const uint32_t *tile_order(const gs_bins &bins) {
 }
 
 cudaError_t launch_render_fwd(const CamConst &c, int64_t n, const gs_projected &proj, const gs_bins &bins,
-                              float *image, float *T_final, uint32_t *last, cudaStream_t s) {
+                              float *image, float *T_final, uint32_t *last, cudaStream_t s, const float *target,
+                              float *dL_dimage, float *loss, int64_t *stats) {
     const int tiles = c.tiles_x * c.tiles_y;
     const Bounds bd = bounds_of(bins, n, tiles);
     const bool depth = c.flags & GS_FLAG_DEPTH;
     const ChannelIO io{reinterpret_cast<const float4 *>(proj.rgb), 1, depth ? 4 : 3, nullptr, 0};
+    const float4 *xy = reinterpret_cast<const float4 *>(proj.xy_opacity_depth);
+    const float4 *cr = reinterpret_cast<const float4 *>(proj.conic_radius);
+    const uint2 *rg = reinterpret_cast<const uint2 *>(bins.ranges);
+    if (target) {  // the forward with the L1 loss in its epilogue
+        if (loss) {
+            const cudaError_t e = cudaMemsetAsync(loss, 0, sizeof(float), s);
+            if (e != cudaSuccess) return e;
+        }
+        const int64_t count = (int64_t)c.width * c.height * (depth ? 4 : 3);
+        const L1Out l1{target, dL_dimage, loss, 1.f / (float)count, stats, bins.status,
+                       reinterpret_cast<const uint64_t *>(bins.n_pairs)};
+        prof_before("render_fwd", s);
+        if (depth)
+            k_render_fwd<true, false, true><<<tiles, kTilePixels, 0, s>>>(c, xy, cr, io, bins.pair_gid, rg,
+                                                                        tile_order(bins), image, T_final, last,
+                                                                        bd, l1);
+        else
+            k_render_fwd<false, false, true><<<tiles, kTilePixels, 0, s>>>(c, xy, cr, io, bins.pair_gid, rg,
+                                                                         tile_order(bins), image, T_final, last,
+                                                                         bd, l1);
+        prof_after(s);
+        return cudaGetLastError();
+    }
     prof_before("render_fwd", s);
     if (depth)
-        k_render_fwd<true><<<tiles, kTilePixels, 0, s>>>(
-            c, reinterpret_cast<const float4 *>(proj.xy_opacity_depth),
-            reinterpret_cast<const float4 *>(proj.conic_radius), io, bins.pair_gid,
-            reinterpret_cast<const uint2 *>(bins.ranges), tile_order(bins), image, T_final, last, bd);
+        k_render_fwd<true><<<tiles, kTilePixels, 0, s>>>(c, xy, cr, io, bins.pair_gid, rg, tile_order(bins), image,
+                                                         T_final, last, bd);
     else
-        k_render_fwd<false><<<tiles, kTilePixels, 0, s>>>(
-            c, reinterpret_cast<const float4 *>(proj.xy_opacity_depth),
-            reinterpret_cast<const float4 *>(proj.conic_radius), io, bins.pair_gid,
-            reinterpret_cast<const uint2 *>(bins.ranges), tile_order(bins), image, T_final, last, bd);
+        k_render_fwd<false><<<tiles, kTilePixels, 0, s>>>(c, xy, cr, io, bins.pair_gid, rg, tile_order(bins), image,
+                                                          T_final, last, bd);
     prof_after(s);
     return cudaGetLastError();
 }

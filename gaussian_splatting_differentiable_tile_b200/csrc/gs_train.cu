@@ -98,40 +98,6 @@ k_adam(AdamGroups G, AdamBetas B, float eps, float grad_scale, int n_slots, cons
 // Advances the device step counter before the update reads it.
 __global__ void k_adam_tick(int64_t *step) { *step += 1; }
 
-// Per-camera L1 loss of a training step: loss[0] = mean |image - target|,
-// dL = sign(image - target) / count (scaled by nothing else: the mean over
-// cameras is applied by Adam's grad_scale).  Block 0 also copies the
-// camera's binning status and pair count into stats[0..1].
-__global__ void __launch_bounds__(256)
-k_l1_train(const float *__restrict__ image, const float *__restrict__ target, int64_t count,
-           float *__restrict__ dL, float *__restrict__ loss, const int32_t *__restrict__ bin_status,
-           const uint64_t *__restrict__ bin_pairs, int64_t *__restrict__ stats) {
-    __shared__ float s_w[8];
-    const float inv = 1.f / (float)count;
-    float acc = 0.f;
-    for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < count;
-         i += (int64_t)gridDim.x * blockDim.x) {
-        const float d = image[i] - target[i];
-        dL[i] = d > 0.f ? inv : (d < 0.f ? -inv : 0.f);
-        acc += fabsf(d);
-    }
-    if (stats && blockIdx.x == 0 && threadIdx.x == 0) {
-        stats[0] = (int64_t)*bin_status;
-        stats[1] = (int64_t)*bin_pairs;
-    }
-    if (loss) {
-#pragma unroll
-        for (int o = 16; o > 0; o >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, o);
-        if ((threadIdx.x & 31) == 0) s_w[threadIdx.x >> 5] = acc;
-        __syncthreads();
-        if (threadIdx.x == 0) {
-            float s = 0.f;
-            for (int w = 0; w < (int)(blockDim.x >> 5); w++) s += s_w[w];
-            atomicAdd(loss, s * inv);
-        }
-    }
-}
-
 int num_sms_train() {
     static int sms = 0;
     if (sms == 0) {
@@ -167,19 +133,5 @@ cudaError_t launch_adam(const AdamGroups &G, int64_t max_count, const AdamBetas 
     return cudaGetLastError();
 }
 
-cudaError_t launch_l1_train(const float *image, const float *target, int64_t count, float *dL_dimage,
-                            float *loss, const gs_bins &bins, int64_t *stats, cudaStream_t s) {
-    if (loss) {
-        cudaError_t e = cudaMemsetAsync(loss, 0, sizeof(float), s);
-        if (e != cudaSuccess) return e;
-    }
-    const int64_t want = (count + 255) / 256;
-    const int blocks = (int)std::max<int64_t>(1, std::min<int64_t>(want, (int64_t)num_sms_train() * 8));
-    prof_before("l1_loss", s);
-    k_l1_train<<<blocks, 256, 0, s>>>(image, target, count, dL_dimage, loss, bins.status,
-                                      reinterpret_cast<const uint64_t *>(bins.n_pairs), stats);
-    prof_after(s);
-    return cudaGetLastError();
-}
 
 }  // namespace gs

@@ -266,6 +266,21 @@ int gs_bin_and_sort(const gs_camera *cam, int64_t n, const gs_projected *proj,
 int gs_render_fwd(const gs_camera *cam, int64_t n, const gs_projected *proj, const gs_bins *bins,
                   float *image, float *T_final, uint32_t *last, void *stream);
 
+/* gs_render_fwd with the training step's L1 loss ([GSP] s7) taken in the
+ * same kernel, after each pixel's blend: loss = mean |image - target| over
+ * every value, dL/dimage = sign(image - target) / count with sign(0) = 0 and
+ * count = width x height x channels (the values gs_l1_loss_grad writes for
+ * the same image, bit for bit; the loss is summed per CTA, so its last bits
+ * depend on the order of the atomic adds).
+ *   image, T_final, last  as gs_render_fwd
+ *   target     [H][W][channels]  device, 4-byte aligned, read
+ *   dL_dimage  [H][W][channels]  device, 4-byte aligned, written
+ *   loss       [1]               device, nullable; zeroed, then the loss
+ * Errors: INVALID_ARG, ALIGNMENT, CUDA. */
+int gs_render_fwd_l1(const gs_camera *cam, int64_t n, const gs_projected *proj, const gs_bins *bins,
+                     float *image, float *T_final, uint32_t *last, const float *target, float *dL_dimage,
+                     float *loss, void *stream);
+
 /* Backward ([GSP] s6; [BLOG]): one CTA per tile walks each pixel's added
  * entries back to front from `last`, recovering T_i = T_{i+1} / (1 - alpha_i)
  * instead of storing weights; dL/dalpha_i = T_i <c_i - R_i, g> with

@@ -184,6 +184,39 @@ def test_bin_and_sort_capacity_error_and_async_status(strategy):
     assert G.gs_bin_and_sort(cam, n, proj, bins2) == need
 
 
+@pytest.mark.parametrize("depth", [False, True])
+@pytest.mark.parametrize("scene", ["tiny", "ragged", "student3k"])
+def test_render_fwd_l1_equals_forward_then_l1(scene, depth):
+    """gs_render_fwd_l1 (the L1 loss in the forward's epilogue) writes the
+    image, T, last and dL/dimage of gs_render_fwd followed by
+    gs_l1_loss_grad bit for bit; the loss (summed per CTA instead of per
+    thread block of values) agrees to rounding, and is zeroed first."""
+    cam, params = SCENES[scene]()
+    if depth:
+        cam.flags |= G.GS_FLAG_DEPTH
+    n = params["means"].shape[0]
+    P = cuda_params(params)
+    r = G.Rasterizer(n, cam.width, cam.height)
+    image = r.forward(cam, P).clone()
+    T, last = r.T_final.clone(), r.last.clone()
+    ch = G.channels(cam)
+    target = torch.from_numpy(make_target(cam.width, cam.height, channels=ch)).cuda()
+    dl_ref = torch.empty_like(image)
+    loss_ref = torch.zeros(1, device="cuda")
+    G.gs_l1_loss_grad(image, target, dl_ref, loss_ref)
+    img2, T2, last2, dl2 = (torch.full_like(x, 7) for x in (image, T, last, dl_ref))
+    loss2 = torch.full((1,), 7.0, device="cuda")
+    G.gs_render_fwd_l1(cam, n, r.proj, r.bins, img2, T2, last2, target, dl2, loss2)
+    torch.cuda.synchronize()
+    assert torch.equal(img2, image) and torch.equal(T2, T) and torch.equal(last2, last)
+    assert torch.equal(dl2, dl_ref)
+    assert abs(loss2.item() - loss_ref.item()) <= 1e-6 * max(1.0, loss_ref.item())
+    dl3 = torch.full_like(dl_ref, 7)
+    G.gs_render_fwd_l1(cam, n, r.proj, r.bins, img2, T2, last2, target, dl3, None)  # no loss wanted
+    torch.cuda.synchronize()
+    assert torch.equal(dl3, dl_ref)
+
+
 @pytest.mark.parametrize("count,offset", [(4 * 100_003, 0), (4 * 100_003 + 3, 0), (4 * 100_003, 1)])
 def test_l1_loss_grad_sizes_and_offsets(count, offset):
     """gs_l1_loss_grad against the oracle's loss and gradient: a count that is
