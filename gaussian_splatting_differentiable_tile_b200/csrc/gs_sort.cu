@@ -591,9 +591,6 @@ k_tile_sort(const uint32_t *__restrict__ ranges, const uint32_t *__restrict__ or
 #endif
 // Resident scatter CTAs per SM the register allocation targets (a tuning
 // knob).
-#ifndef GS_LSD_PREMATCH
-#define GS_LSD_PREMATCH 0
-#endif
 #ifndef GS_LSD_MINB
 #define GS_LSD_MINB 2
 #endif
@@ -770,6 +767,12 @@ k_scan_add(uint32_t *__restrict__ H, uint32_t m, const uint32_t *__restrict__ S,
 // over the warps and over the digits places each element in the tile sorted
 // by digit, in shared memory; the tile then goes out digit run by digit run,
 // each run contiguous at the scanned H[d][b], so the writes are coalesced.
+// With kLocal, H holds the tiles' digit counts unscanned (passes of at most
+// kLocalScanTiles tiles): each CTA sums its digit's counts over the tiles
+// before it and over all tiles, and scans the digit totals itself, in place
+// of the two scan kernels.
+constexpr int kLocalScanTiles = 256;
+template <bool kLocal>
 __global__ void __launch_bounds__(kScatterThreads, GS_LSD_MINB)
 k_lsd_scatter(const uint32_t *__restrict__ keys_in, const uint32_t *__restrict__ vals_in,
               const uint64_t *__restrict__ count_dev, uint32_t count_host, int shift, int bits,
@@ -794,31 +797,27 @@ k_lsd_scatter(const uint32_t *__restrict__ keys_in, const uint32_t *__restrict__
         val[k] = i < m ? vals_in[t0 + i] : 0u;
     }
     for (int i = tid; i < kScatterWarps * kRadix; i += kScatterThreads) (&s_cnt[0][0])[i] = 0;
-    if ((uint32_t)tid < ndig) s_gbase[tid] = H[(size_t)tid * gridDim.x + blockIdx.x];
+    if (kLocal) {
+        if (tid < kRadix) {  // this digit's count before this tile, and its total (in s_start for now)
+            uint32_t before = 0, total = 0;
+            if ((uint32_t)tid < ndig) {
+                const uint32_t *row = H + (size_t)tid * gridDim.x;
+                for (uint32_t b = 0; b < gridDim.x; b++) {
+                    const uint32_t c = row[b];
+                    total += c;
+                    before += b < blockIdx.x ? c : 0u;
+                }
+            }
+            s_gbase[tid] = before;
+            s_start[tid] = total;
+        }
+        __syncthreads();
+        scan256(s_start, s_w);  // each digit's first position in the output
+        if (tid < kRadix) s_gbase[tid] += s_start[tid];
+    } else if ((uint32_t)tid < ndig) {
+        s_gbase[tid] = H[(size_t)tid * gridDim.x + blockIdx.x];
+    }
     __syncthreads();
-#if GS_LSD_PREMATCH
-    // every item's peers first (independent), then the counter chain
-#pragma unroll
-    for (int k = 0; k < kScatterItems; k++) {
-        const uint32_t i = (uint32_t)(warp * 32 * kScatterItems + 32 * k + lane);
-        const uint32_t d = i < m ? (key[k] >> shift) & mask : (uint32_t)kRadix;
-#if GS_LSD_MATCH
-        rank[k] = __match_any_sync(0xffffffffu, d);
-#else
-        rank[k] = digit_peers(d, bits);
-#endif
-    }
-#pragma unroll
-    for (int k = 0; k < kScatterItems; k++) {
-        const uint32_t i = (uint32_t)(warp * 32 * kScatterItems + 32 * k + lane);
-        const uint32_t d = i < m ? (key[k] >> shift) & mask : (uint32_t)kRadix;
-        const uint32_t peers = rank[k];
-        rank[k] = d < kRadix ? s_cnt[warp][d] + __popc(peers & lt) : 0u;
-        __syncwarp();
-        if (d < kRadix && lane == __ffs(peers) - 1) s_cnt[warp][d] += __popc(peers);
-        __syncwarp();
-    }
-#else
 #pragma unroll
     for (int k = 0; k < kScatterItems; k++) {
         const uint32_t i = (uint32_t)(warp * 32 * kScatterItems + 32 * k + lane);
@@ -833,7 +832,6 @@ k_lsd_scatter(const uint32_t *__restrict__ keys_in, const uint32_t *__restrict__
         if (d < kRadix && lane == __ffs(peers) - 1) s_cnt[warp][d] += __popc(peers);
         __syncwarp();
     }
-#endif
     __syncthreads();
     if (tid < kRadix) {  // exclusive over the warps, per digit; digit totals of the tile
         uint32_t tot = 0;
@@ -1055,6 +1053,17 @@ struct DeviceSetup {
 DeviceSetup g_setup[kMaxDevices];
 std::mutex g_setup_mutex;
 
+// Every instantiation of k_lsd_scatter takes kScatterSmem of dynamic shared
+// memory.
+cudaError_t scatter_smem_attributes() {
+    const void *kernels[] = {(const void *)k_lsd_scatter<true>, (const void *)k_lsd_scatter<false>};
+    for (const void *k : kernels) {
+        const cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kScatterSmem);
+        if (e != cudaSuccess) return e;
+    }
+    return cudaSuccess;
+}
+
 cudaError_t device_setup(int *sms) {
     int dev = 0;
     cudaError_t e = cudaGetDevice(&dev);
@@ -1072,8 +1081,7 @@ cudaError_t device_setup(int *sms) {
                 cudaSuccess ||
             (e = cudaFuncSetAttribute(k_tile_sort<kMidWarps, true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                       (int)(2 * kTileSortMid * sizeof(uint64_t)))) != cudaSuccess ||
-            (e = cudaFuncSetAttribute(k_lsd_scatter, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                      (int)kScatterSmem)) != cudaSuccess)
+            (e = scatter_smem_attributes()) != cudaSuccess)
             return e;
         d.sms = n > 0 ? n : 148;
     }
@@ -1095,17 +1103,22 @@ int64_t lsd_space(int64_t cap) {
 // One stable LSD pass over the digit (key >> shift) & (2^bits - 1) of at
 // most `cap` elements (*count_dev of them when given, else count_host):
 // per-tile digit counts, their exclusive scan, the scatter.
-void lsd_pass(const uint32_t *ki, const uint32_t *vi, uint32_t *ko, uint32_t *vo, const uint64_t *count_dev,
-              uint32_t count_host, int64_t cap, int shift, int bits, uint32_t *H, int32_t *status, cudaStream_t s) {
+// Returns the kernels it launched.
+int lsd_pass(const uint32_t *ki, const uint32_t *vi, uint32_t *ko, uint32_t *vo, const uint64_t *count_dev,
+             uint32_t count_host, int64_t cap, int shift, int bits, uint32_t *H, int32_t *status, cudaStream_t s) {
     const int tiles = (int)std::max<int64_t>(1, (cap + kScatterTile - 1) / kScatterTile);
     const uint32_t m = (uint32_t)((1u << bits) * (uint32_t)tiles);
     const int blocks = (int)((m + kScanBlock - 1) / kScanBlock);
     uint32_t *S = H + m;
     k_lsd_hist<<<tiles, kHistThreads, 0, s>>>(ki, count_dev, count_host, shift, bits, H, status);
-    k_scan_blocks<<<blocks, kScanThreads, 0, s>>>(H, m, S, status);
-    k_scan_add<<<blocks, kScanThreads, 0, s>>>(H, m, S, status);
-    k_lsd_scatter<<<tiles, kScatterThreads, kScatterSmem, s>>>(ki, vi, count_dev, count_host, shift, bits, H, ko,
-                                                               vo, status);
+    const bool local = tiles <= kLocalScanTiles;
+    if (!local) {
+        k_scan_blocks<<<blocks, kScanThreads, 0, s>>>(H, m, S, status);
+        k_scan_add<<<blocks, kScanThreads, 0, s>>>(H, m, S, status);
+    }
+    (local ? k_lsd_scatter<true> : k_lsd_scatter<false>)<<<tiles, kScatterThreads, kScatterSmem, s>>>(
+        ki, vi, count_dev, count_host, shift, bits, H, ko, vo, status);
+    return local ? 2 : 4;
 }
 
 // The global path after the tile scan (see the kernels above).  ctas: CTAs
@@ -1139,11 +1152,12 @@ cudaError_t launch_bin_global(const CamConst &c, int64_t n, const gs_projected &
     prof_before("depth_sort", s);
     k_depth_init<<<(unsigned)((n + 255) / 256), 256, 0, s>>>((int)n, rect, xyod, c.tiles_x, c.tiles_y, KA, VA,
                                                                status);
+    int launched = 1;
     for (int p = 0; p < 4; p++) {
         uint32_t *ki = p & 1 ? KB : KA, *vi = p & 1 ? VB : VA, *ko = p & 1 ? KA : KB, *vo = p & 1 ? VA : VB;
-        lsd_pass(ki, vi, ko, vo, nullptr, nn, n, 8 * p, 8, H, status, s);
+        launched += lsd_pass(ki, vi, ko, vo, nullptr, nn, n, 8 * p, 8, H, status, s);
     }
-    prof_after(s, 17);
+    prof_after(s, launched);
     // 5. each Gaussian's first pair position in depth order (into KA), then
     // the pairs in (depth, id) order into (KB, VB)
     prof_before("emit", s);
@@ -1161,14 +1175,15 @@ cudaError_t launch_bin_global(const CamConst &c, int64_t n, const gs_projected &
     while (tile_bits < 31 && ((uint32_t)(tiles - 1) >> tile_bits)) tile_bits++;
     const int passes = (tile_bits + 7) / 8, digit = (tile_bits + passes - 1) / passes;
     prof_before("tile_sort", s);
+    launched = 0;
     for (int p = 0; p < passes; p++) {
         const bool last = p == passes - 1;
         const int bits = std::min(digit, tile_bits - digit * p);
         uint32_t *ki = p & 1 ? KA : KB, *vi = p & 1 ? VA : VB;
         uint32_t *ko = last ? bins.pair_tile : (p & 1 ? KB : KA), *vo = last ? bins.pair_gid : (p & 1 ? VB : VA);
-        lsd_pass(ki, vi, ko, vo, n_pairs, 0u, bins.max_pairs, digit * p, bits, H, status, s);
+        launched += lsd_pass(ki, vi, ko, vo, n_pairs, 0u, bins.max_pairs, digit * p, bits, H, status, s);
     }
-    prof_after(s, 4 * passes);
+    prof_after(s, launched);
     // 7. each tile's range off the sorted list, its total, then the tile
     // scan as on the per-tile path (ranges again, K kept, the tile order)
     prof_before("tile_scan", s);
@@ -1207,7 +1222,8 @@ cudaError_t launch_bin_and_sort(const CamConst &c, int64_t n, const gs_projected
     // the strategy (gs.h GS_BIN_*); the global path's LSD passes keep their
     // per-tile digit counts in the count matrix's space
     const int64_t hist_cap = std::min<int64_t>((int64_t)kBinCTAsMax * bins.max_tiles, kBinHistCap);
-    const int lsd_ctas = (int)std::min<int64_t>((int64_t)2 * sms, hist_cap);
+    // the rank kernels keep one u64 sum per CTA in the same space
+    const int lsd_ctas = (int)std::max<int64_t>(1, std::min<int64_t>((int64_t)2 * sms, hist_cap / 2));
     bool global = bins.strategy == GS_BIN_GLOBAL;
     if (bins.strategy == GS_BIN_AUTO)
         global = bins.max_pairs >= (int64_t)1024 * tiles;
