@@ -106,9 +106,9 @@ ALU_KERNELS = ("render_fwd", "render_bwd")
 # DRAM traffic per launch of render_bwd measured by ncu
 # (dram__bytes_read.sum + dram__bytes_write.sum), valid only for the kernel
 # source it was taken on.
-# Taken on one frame of this workload (camera 0, 644,012 pairs): 42.36 MB
-# read + 0.28 MB written; scaled to a launch by its pair count.
-TRAFFIC = {"render_bwd": {"src_sha": "c7bb92509884b06c", "bytes_per_pair": 66.21}}
+# Taken on one frame of this workload (camera 0, 644,012 pairs): 42.37 MB
+# read + 0.44 MB written; scaled to a launch by its pair count.
+TRAFFIC = {"render_bwd": {"src_sha": "ebd0766b23470e34", "bytes_per_pair": 66.47}}
 
 
 def _binning_used(choice, max_pairs, spec) -> str:
