@@ -83,6 +83,37 @@ constexpr int kShortWarps = 4, kMidWarps = 32;
 constexpr uint32_t kTileSortShort = 256u * kShortWarps;
 constexpr uint32_t kTileSortMid = 256u * kMidWarps;
 
+// Calls f(k, tile) for the tiles k = first, first + kStep, ... < c of a
+// rectangle (row-major from column x0, row y0, w tiles wide), keeping the
+// column and row by additions: kStep 1 (first 0) needs no division, kStep 32
+// one per call.
+template <uint32_t kStep, typename F>
+__device__ __forceinline__ void rect_walk(uint32_t first, uint32_t c, int x0, int y0, uint32_t w, int tiles_x,
+                                          F f) {
+    uint32_t dy, dx, sq, sr;  // position, and the step in rows and columns
+    if (kStep == 1) {
+        dy = 0;
+        dx = 0;
+        sq = w == 1 ? 1u : 0u;
+        sr = w == 1 ? 0u : 1u;
+    } else {
+        if (first >= c) return;
+        dy = first / w;
+        dx = first - dy * w;
+        sq = kStep / w;
+        sr = kStep - sq * w;
+    }
+    for (uint32_t k = first; k < c; k += kStep) {
+        f(k, (y0 + (int)dy) * tiles_x + x0 + (int)dx);
+        dx += sr;
+        dy += sq;
+        if (dx >= w) {
+            dx -= w;
+            dy++;
+        }
+    }
+}
+
 // Calls f(g, tile) for every pair of the Gaussians [g_begin, g_end), the
 // CTA's warps striding through the range 32 Gaussians at a time, four
 // groups per round (their rectangles loaded together).
@@ -103,12 +134,7 @@ __device__ __forceinline__ void for_each_pair(int g_begin, int g_end, const int4
             const int g = g0 + u * (int)blockDim.x + lane;
             int x0 = 0, y0 = 0, w = 1;
             const uint32_t c = rect_tiles(rc[u], tiles_x, tiles_y, x0, y0, w);
-            if (c <= kLaneTiles) {
-                for (uint32_t k = 0; k < c; k++) {
-                    const uint32_t dy = k / (uint32_t)w;
-                    f(g, (y0 + (int)dy) * tiles_x + x0 + (int)(k - dy * (uint32_t)w));
-                }
-            }
+            if (c <= kLaneTiles) rect_walk<1>(0u, c, x0, y0, (uint32_t)w, tiles_x, [&](uint32_t, int t) { f(g, t); });
             uint32_t big = __ballot_sync(0xffffffffu, c > kLaneTiles);
             while (big) {
                 const int src = __ffs(big) - 1;
@@ -117,10 +143,7 @@ __device__ __forceinline__ void for_each_pair(int g_begin, int g_end, const int4
                 const uint32_t cb = __shfl_sync(0xffffffffu, c, src);
                 const int xb = __shfl_sync(0xffffffffu, x0, src), yb = __shfl_sync(0xffffffffu, y0, src);
                 const uint32_t wb = (uint32_t)__shfl_sync(0xffffffffu, w, src);
-                for (uint32_t k = lane; k < cb; k += 32) {
-                    const uint32_t dy = k / wb;
-                    f(gb, (yb + (int)dy) * tiles_x + xb + (int)(k - dy * wb));
-                }
+                rect_walk<32>((uint32_t)lane, cb, xb, yb, wb, tiles_x, [&](uint32_t, int t) { f(gb, t); });
             }
         }
     }
@@ -1015,14 +1038,12 @@ k_emit_ranked(int n, const int4 *__restrict__ rect, const uint32_t *__restrict__
             c = rect_tiles(rect[g], tiles_x, tiles_y, x0, y0, w);
             if (c) off = offsets[r];
         }
-        if (c <= kLaneTiles) {
-            for (uint32_t k = 0; k < c; k++) {
-                const uint32_t dy = k / (uint32_t)w;
-                if (!in_bounds((uint64_t)off + k, max_pairs, status)) break;
-                tile_out[off + k] = (uint32_t)((y0 + (int)dy) * tiles_x + x0 + (int)(k - dy * (uint32_t)w));
+        if (c <= kLaneTiles)
+            rect_walk<1>(0u, c, x0, y0, (uint32_t)w, tiles_x, [&](uint32_t k, int t) {
+                if (!in_bounds((uint64_t)off + k, max_pairs, status)) return;
+                tile_out[off + k] = (uint32_t)t;
                 gid_out[off + k] = g;
-            }
-        }
+            });
         uint32_t big = __ballot_sync(0xffffffffu, c > kLaneTiles);
         while (big) {
             const int src = __ffs(big) - 1;
@@ -1031,12 +1052,11 @@ k_emit_ranked(int n, const int4 *__restrict__ rect, const uint32_t *__restrict__
             const uint32_t ob = __shfl_sync(0xffffffffu, off, src);
             const int xb = __shfl_sync(0xffffffffu, x0, src), yb = __shfl_sync(0xffffffffu, y0, src);
             const uint32_t wb = (uint32_t)__shfl_sync(0xffffffffu, w, src);
-            for (uint32_t k = lane; k < cb; k += 32) {
-                const uint32_t dy = k / wb;
-                if (!in_bounds((uint64_t)ob + k, max_pairs, status)) break;
-                tile_out[ob + k] = (uint32_t)((yb + (int)dy) * tiles_x + xb + (int)(k - dy * wb));
+            rect_walk<32>((uint32_t)lane, cb, xb, yb, wb, tiles_x, [&](uint32_t k, int t) {
+                if (!in_bounds((uint64_t)ob + k, max_pairs, status)) return;
+                tile_out[ob + k] = (uint32_t)t;
                 gid_out[ob + k] = gb;
-            }
+            });
         }
     }
 }
