@@ -219,8 +219,15 @@ k_bin_colscan(int tiles, int ctas, uint32_t *__restrict__ H, uint32_t *__restric
 
 // One CTA: ranges from the exclusive scan of the tile totals (all empty if K
 // exceeds the capacity, with GS_ERR_CAPACITY recorded), K, and the tile
-// order (longest list first, by a counting sort on length in steps of 4).
+// order (longest list first, by a counting sort on length in steps of
+// 2^GS_ORDER_SHIFT, lists of 1024 steps and more sharing the first bucket).
 constexpr int kScanTilesThreads = 1024;
+#ifndef GS_ORDER_SHIFT
+#define GS_ORDER_SHIFT 2
+#endif
+__device__ __forceinline__ uint32_t order_bucket(uint32_t len) {
+    return min(len >> GS_ORDER_SHIFT, (uint32_t)(kScanTilesThreads - 1));
+}
 __global__ void __launch_bounds__(kScanTilesThreads)
 k_tile_scan(int tiles, const uint32_t *__restrict__ totals, uint64_t max_pairs,
             uint32_t *__restrict__ ranges, uint32_t *__restrict__ order, uint64_t *__restrict__ n_pairs,
@@ -271,7 +278,7 @@ k_tile_scan(int tiles, const uint32_t *__restrict__ totals, uint64_t max_pairs,
     }
     auto bucket = [&](int i) {
         const uint32_t len = ok ? totals[i] : 0u;
-        return kScanTilesThreads - 1 - (int)min(len >> 2, (uint32_t)(kScanTilesThreads - 1));
+        return kScanTilesThreads - 1 - (int)order_bucket(len);
     };
     s_off[t] = 0;
     __syncthreads();
@@ -330,9 +337,6 @@ k_bin_emit(int n, const int4 *__restrict__ rect, const float4 *__restrict__ xyod
     });
 }
 
-__device__ __forceinline__ uint32_t order_bucket(uint32_t len) {
-    return min(len >> 2, (uint32_t)(kScanTilesThreads - 1));
-}
 
 // Sorts the keys of a warp ascending in registers: lane l holds elements
 // 8l .. 8l + 7 in k[0..7].  Bitonic network: strides below 8 swap within the
@@ -383,21 +387,10 @@ __device__ __forceinline__ int run_rank(const uint64_t *a, int n, uint64_t x) {
     return lo;
 }
 
-// Tile lists of at most 256 entries: one warp each, in registers (CTA b,
-// warp w take the (4 b + w)-th tile of the order).
-__global__ void __launch_bounds__(128)
-k_tile_sort_warp(const uint32_t *__restrict__ ranges, const uint32_t *__restrict__ order, int tiles,
-                 const uint64_t *__restrict__ keys, uint32_t *__restrict__ pair_gid,
-                 uint32_t *__restrict__ pair_tile, const Bounds bd) {
-    const int lane = threadIdx.x & 31;
-    const int b = blockIdx.x * 4 + (threadIdx.x >> 5);
-    if (b >= tiles) return;
-    const uint32_t tile = order[b];
-    if (!in_bounds(tile, (uint32_t)tiles, bd.status)) return;
-    const uint32_t start = ranges[2 * (size_t)tile], end = ranges[2 * (size_t)tile + 1];
-    if (!range_in_bounds(make_uint2(start, end), bd)) return;
-    const uint32_t L = end - start;
-    if (L == 0 || L > 256) return;
+// A tile list of 1 to 256 entries sorted by one warp in registers.
+__device__ __forceinline__ void warp_sort_tile(uint32_t tile, uint32_t start, uint32_t L,
+                                               const uint64_t *__restrict__ keys, uint32_t *__restrict__ pair_gid,
+                                               uint32_t *__restrict__ pair_tile, int lane) {
     uint64_t k[8];
 #pragma unroll
     for (int r = 0; r < 8; r++) {
@@ -498,8 +491,10 @@ __device__ void global_radix_sort_tile(uint32_t start, uint32_t end, uint32_t ti
 // Tile lists in (lo, hi], hi = 256 kWarps: sorted by one CTA each.  Warp w
 // sorts keys [256 w, 256 w + 256) in registers; the runs are then merged
 // pairwise in shared memory (each key's output position is its index plus
-// its rank in the other run).  With kLong the CTA also takes lists above hi,
-// by a radix sort in global memory.  With `persistent` a small grid walks the tile
+// its rank in the other run).  Without kLong the CTA's first warp also
+// sorts lists of 1 to 256 entries alone (whatever lo is), so the short and
+// the mid-sized lists of a frame are sorted by one launch.  With kLong the
+// CTA also takes lists above hi, by a radix sort in global memory.  With `persistent` a small grid walks the tile
 // order (longest first) and stops at the first tile whose length bucket
 // lies below lo's; otherwise CTA b takes the b-th tile of the order.
 template <int kWarps, bool kLong>
@@ -522,6 +517,10 @@ k_tile_sort(const uint32_t *__restrict__ ranges, const uint32_t *__restrict__ or
         if (!range_in_bounds(make_uint2(start, end), bd)) break;
         const uint32_t L = end - start;
         if (persistent && order_bucket(L) < order_bucket(lo)) break;
+        if (!kLong && L <= 256u) {  // a short list: one warp, in registers
+            if (warp == 0 && L > 0) warp_sort_tile(tile, start, L, keys, pair_gid, pair_tile, lane);
+            continue;
+        }
         if (L <= lo) continue;
         if (L > kHi) {
             // longer than shared memory holds: sorted in global memory, with
@@ -1269,13 +1268,12 @@ cudaError_t launch_bin_and_sort(const CamConst &c, int64_t n, const gs_projected
     // 5. sort each tile's list, by size class
     prof_before("tile_sort", s);
     const Bounds bd = bounds_of(bins, n, tiles);
-    k_tile_sort_warp<<<(tiles + 3) / 4, 128, 0, s>>>(ranges, order, tiles, keys, bins.pair_gid, bins.pair_tile, bd);
     k_tile_sort<kShortWarps, false><<<tiles, kShortWarps * 32, 2 * kTileSortShort * sizeof(uint64_t), s>>>(
         ranges, order, tiles, keys, bins.pair_gid, bins.pair_tile, 256u, 0, nullptr, nullptr, bd);
     k_tile_sort<kMidWarps, true><<<std::min(tiles, sms), kMidWarps * 32, 2 * kTileSortMid * sizeof(uint64_t), s>>>(
         ranges, order, tiles, keys, bins.pair_gid, bins.pair_tile, kTileSortShort, 1, U32(L.long_keys),
         U32(L.long_ids), bd);
-    prof_after(s, 3);
+    prof_after(s, 2);
     return cudaGetLastError();
 }
 
