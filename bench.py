@@ -742,8 +742,9 @@ def run_native(args, spec, rank, world, local):
         fr = feat["frames"]
         feat_out = {"channels": feat["F"], "fwd_ms_per_frame": feat_fwd_ms / fr, "bwd_ms_per_frame": feat_bwd_ms / fr,
                     "fwd_bwd_frames_per_s": fr * world / ((feat_fwd_ms + feat_bwd_ms) * 1e-3),
-                    "passes": f"{feat['F'] // 4} blend passes of four channels each way (forward weights recomputed, "
-                              "no background); backward adds into the frame's raw-parameter gradients"}
+                    "passes": (f"{feat['F'] // 8} blend pass{'es' if feat['F'] // 8 != 1 else ''} of eight channels"
+                               f"{' and one of four' if feat['F'] % 8 else ''} each way (forward weights recomputed per "
+                               "pass, no background); backward adds into the frame's raw-parameter gradients")}
     out = {
         "metric": METRIC,
         "value": frames / (full_ms * 1e-3),

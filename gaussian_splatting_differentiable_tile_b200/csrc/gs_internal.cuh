@@ -172,8 +172,8 @@ cudaError_t launch_render_fwd(const CamConst &c, int64_t n, const gs_projected &
 cudaError_t launch_render_bwd(const CamConst &c, int64_t n, const gs_projected &proj, const gs_bins &bins,
                               const float *T_final, const uint32_t *last, const float *dL_dimage,
                               float *grad2d, cudaStream_t s);
-// Feature channels: F / 4 passes of the blend over chunks of four channels
-// (no background).  The backward adds the geometric sums into grad2d and
+// Feature channels: passes of the blend over chunks of eight channels, then
+// one of four when F is not a multiple of 8 (no background).  The backward adds the geometric sums into grad2d and
 // the feature gradients into dL_dfeatures (both zeroed by the caller).
 cudaError_t launch_render_features_fwd(const CamConst &c, int64_t n, const gs_projected &proj, const gs_bins &bins,
                                        const float *features, int F, float *out, cudaStream_t s);

@@ -277,8 +277,8 @@ __device__ __forceinline__ uint32_t block_mask(const float4 geo, const float4 ge
     return m;
 }
 
-template <bool kDepth, bool kFeat = false, bool kL1 = false>
-__global__ void __launch_bounds__(kTilePixels, GS_FWD_MINB)
+template <bool kDepth, bool kFeat = false, bool kL1 = false, bool kF8 = false>
+__global__ void __launch_bounds__(kTilePixels, kF8 ? 4 : GS_FWD_MINB)
 k_render_fwd(CamConst cam, const float4 *__restrict__ xyod, const float4 *__restrict__ conr,
              const ChannelIO io, const uint32_t *__restrict__ pair_gid,
              const uint2 *__restrict__ ranges, const uint32_t *__restrict__ order,
@@ -290,6 +290,9 @@ k_render_fwd(CamConst cam, const float4 *__restrict__ xyod, const float4 *__rest
     __shared__ float4 s_col[kBatch];
     __shared__ uint8_t s_mask[kBatch];
     __shared__ FwdWarpBuf s_wb[kWarps];
+    // kF8: channels 4-7 of a feature chunk of eight (values, then per warp)
+    __shared__ float4 s_col2[kF8 ? kBatch : 1];
+    __shared__ float4 s_wcol2[kF8 ? kWarps : 1][kF8 ? kFwdChunk : 1];
 
     const uint32_t tile_id = order[blockIdx.x];  // longest lists first
     if (!in_bounds(tile_id, bd.tiles, bd.status)) return;
@@ -307,6 +310,7 @@ k_render_fwd(CamConst cam, const float4 *__restrict__ xyod, const float4 *__rest
     const uint32_t lt_mask = (1u << lane) - 1u;
 
     float T = 1.f, C0 = 0.f, C1 = 0.f, C2 = 0.f, C3 = 0.f;
+    float C4 = 0.f, C5 = 0.f, C6 = 0.f, C7 = 0.f;  // kF8
     uint32_t lst = range.x;
     bool done = !(px < cam.width && py < cam.height);
     for (uint32_t b = range.x; b < range.y; b += kBatch) {
@@ -319,6 +323,7 @@ k_render_fwd(CamConst cam, const float4 *__restrict__ xyod, const float4 *__rest
             if (ok) stage_entry(xyod[g], conr[g], geo, geo2);
             s_geo[threadIdx.x] = geo;
             s_col[threadIdx.x] = ok ? io.col[kFeat ? (size_t)g * io.col_stride : (size_t)g] : geo;
+            if (kF8) s_col2[threadIdx.x] = ok ? io.col[(size_t)g * io.col_stride + 1] : geo;
             s_mask[threadIdx.x] = ok ? (uint8_t)block_mask(geo, geo2, x0, y0) : (uint8_t)0;
             geo2.z = hit_center(geo2.y);  // kx, ky are only needed for the mask
             s_geo2[threadIdx.x] = geo2;
@@ -347,6 +352,7 @@ k_render_fwd(CamConst cam, const float4 *__restrict__ xyod, const float4 *__rest
                     cn[2 + hb] = -geo2.z;
                     reinterpret_cast<float *>(&wb.lo[pr])[hb] = geo2.y;
                     wb.col[t] = s_col[i];
+                    if (kF8) s_wcol2[warp][t] = s_col2[i];
                     wb.slot[t] = (uint8_t)i;
                 }
                 n += __popc(bal);
@@ -400,6 +406,13 @@ k_render_fwd(CamConst cam, const float4 *__restrict__ xyod, const float4 *__rest
                         C1 = __fmaf_rn(w, c.y, C1);
                         C2 = __fmaf_rn(w, c.z, C2);
                         if (kDepth) C3 = __fmaf_rn(w, c.w, C3);
+                        if (kF8) {
+                            const float4 c2 = s_wcol2[warp][2 * k];
+                            C4 = __fmaf_rn(w, c2.x, C4);
+                            C5 = __fmaf_rn(w, c2.y, C5);
+                            C6 = __fmaf_rn(w, c2.z, C6);
+                            C7 = __fmaf_rn(w, c2.w, C7);
+                        }
                         T = nT;
                         lt = (int)(2 * k);
                     }
@@ -420,6 +433,13 @@ k_render_fwd(CamConst cam, const float4 *__restrict__ xyod, const float4 *__rest
                         C1 = __fmaf_rn(w, c.y, C1);
                         C2 = __fmaf_rn(w, c.z, C2);
                         if (kDepth) C3 = __fmaf_rn(w, c.w, C3);
+                        if (kF8) {
+                            const float4 c2 = s_wcol2[warp][2 * k + 1];
+                            C4 = __fmaf_rn(w, c2.x, C4);
+                            C5 = __fmaf_rn(w, c2.y, C5);
+                            C6 = __fmaf_rn(w, c2.z, C6);
+                            C7 = __fmaf_rn(w, c2.w, C7);
+                        }
                         T = nT;
                         lt = (int)(2 * k + 1);
                     }
@@ -438,6 +458,12 @@ k_render_fwd(CamConst cam, const float4 *__restrict__ xyod, const float4 *__rest
                             __fmaf_rn(T, cam.bg[2], C2), C3};  // the fourth channel has no background
 #pragma unroll
         for (int c = 0; c < kC; c++) out[c] = o[c];
+        if (kF8) {  // feature chunks have no background
+            out[4] = C4;
+            out[5] = C5;
+            out[6] = C6;
+            out[7] = C7;
+        }
         if (T_final) T_final[p] = T;
         if (last) last[p] = lst;
         if (kL1) {
@@ -544,8 +570,8 @@ __device__ __forceinline__ float reduce_scatter(const float (&v)[N], int lane, i
 // with v = alpha dL/dalpha (0 when alpha was capped), w = alpha T_i; they are
 // added into grad2d, and k_project_bwd maps them to dL/d(mean2d, conic,
 // opacity) with the Gaussian's own A, B, C, o.
-template <int kRPL, bool kDepth, bool kFeat = false>
-__global__ void __launch_bounds__(kTilePixels / kRPL, GS_BWD_MINB)
+template <int kRPL, bool kDepth, bool kFeat = false, bool kF8 = false>
+__global__ void __launch_bounds__(kTilePixels / kRPL, kF8 ? 8 : GS_BWD_MINB)
 k_render_bwd(CamConst cam, const float4 *__restrict__ xyod, const float4 *__restrict__ conr,
              const ChannelIO io, const uint32_t *__restrict__ pair_gid,
              const uint2 *__restrict__ ranges, const uint32_t *__restrict__ order,
@@ -560,6 +586,7 @@ k_render_bwd(CamConst cam, const float4 *__restrict__ xyod, const float4 *__rest
     __shared__ float4 s_geo[kB];
     __shared__ float4 s_geo2[kB];
     __shared__ float4 s_col[kB];
+    __shared__ float4 s_col2[kF8 ? kB : 1];  // kF8: channels 4-7 of a feature chunk of eight
     __shared__ uint32_t s_gid[kB];
     __shared__ uint8_t s_mask[kB];
     __shared__ uint8_t s_list[kWarps][kB];
@@ -577,11 +604,12 @@ k_render_bwd(CamConst cam, const float4 *__restrict__ xyod, const float4 *__rest
     // Per pixel state, two rows per float2 (x: row 2i, y: row 2i + 1).
     constexpr int kC = kDepth ? 4 : 3;  // image channels
     float2 T[kPairs], sg[kPairs], g0[kPairs], g1[kPairs], g2[kPairs], g3[kPairs], nfy[kPairs];
+    float2 g4[kPairs], g5[kPairs], g6[kPairs], g7[kPairs];  // kF8
     uint32_t lst[kRPL];
     uint32_t lane_max = range.x;
 #pragma unroll
     for (int r = 0; r < kRPL; r++) {
-        float t = 1.f, d0 = 0.f, d1 = 0.f, d2 = 0.f, d3 = 0.f;
+        float t = 1.f, d0 = 0.f, d1 = 0.f, d2 = 0.f, d3 = 0.f, d4 = 0.f, d5 = 0.f, d6 = 0.f, d7 = 0.f;
         lst[r] = range.x;
         const int py = L.py0 + r;
         if (col_in && py < cam.height) {
@@ -593,15 +621,23 @@ k_render_bwd(CamConst cam, const float4 *__restrict__ xyod, const float4 *__rest
             d1 = dp[1];
             d2 = dp[2];
             if (kDepth) d3 = dp[3];
+            if (kF8) {
+                d4 = dp[4];
+                d5 = dp[5];
+                d6 = dp[6];
+                d7 = dp[7];
+            }
         }
         const float s0 = t * (cam.bg[0] * d0 + cam.bg[1] * d1 + cam.bg[2] * d2);  // depth: no background
         const float nf = -(L.fy0 + (float)r);
         if (r & 1) {
             T[r / 2].y = t; g0[r / 2].y = d0; g1[r / 2].y = d1; g2[r / 2].y = d2; g3[r / 2].y = d3;
             sg[r / 2].y = s0; nfy[r / 2].y = nf;
+            g4[r / 2].y = d4; g5[r / 2].y = d5; g6[r / 2].y = d6; g7[r / 2].y = d7;
         } else {
             T[r / 2].x = t; g0[r / 2].x = d0; g1[r / 2].x = d1; g2[r / 2].x = d2; g3[r / 2].x = d3;
             sg[r / 2].x = s0; nfy[r / 2].x = nf;
+            g4[r / 2].x = d4; g5[r / 2].x = d5; g6[r / 2].x = d6; g7[r / 2].x = d7;
         }
         lane_max = max(lane_max, lst[r]);
     }
@@ -617,7 +653,7 @@ k_render_bwd(CamConst cam, const float4 *__restrict__ xyod, const float4 *__rest
 
     // Sums of an entry: the six geometric ones into grad2d, the channel sums
     // after them (colours) or into io.cgrad (a feature chunk).
-    constexpr int kV = 6 + kC;
+    constexpr int kV = 6 + kC + (kF8 ? 4 : 0);
     auto add_sums = [&](uint32_t g, int i, float x) {
         float *dst = grad2d + 12 * (size_t)g + i;
         if (kFeat && i >= 6) dst = io.cgrad + (size_t)io.cgrad_stride * g + (i - 6);
@@ -646,6 +682,7 @@ k_render_bwd(CamConst cam, const float4 *__restrict__ xyod, const float4 *__rest
             s_geo[i0] = geo;
             s_geo2[i0] = geo2;
             s_col[i0] = ra;
+            if (kF8) s_col2[i0] = io.col[(size_t)ga * io.col_stride + 1];
             s_gid[i0] = ga;
             s_mask[i0] = oka ? (uint8_t)strip_mask<kWarps>(geo, geo2, L.sx, L.hx, L.sy0, 2.f * kRPL, L.hy) : 0;
             s_geo2[i0].z = hit_center(geo2.y);
@@ -654,6 +691,7 @@ k_render_bwd(CamConst cam, const float4 *__restrict__ xyod, const float4 *__rest
                 s_geo[i1] = geo;
                 s_geo2[i1] = geo2;
                 s_col[i1] = rb;
+                if (kF8) s_col2[i1] = io.col[(size_t)gb * io.col_stride + 1];
                 s_gid[i1] = gb;
                 s_mask[i1] = okb ? (uint8_t)strip_mask<kWarps>(geo, geo2, L.sx, L.hx, L.sy0, 2.f * kRPL, L.hy) : 0;
                 s_geo2[i1].z = hit_center(geo2.y);
@@ -694,7 +732,9 @@ k_render_bwd(CamConst cam, const float4 *__restrict__ xyod, const float4 *__rest
             // it is (T / (1 - 0) with the approximate reciprocal of 1, which
             // is exact).
             const float4 c = s_col[k];
+            const float4 c2 = kF8 ? s_col2[k] : c;
             float2 sv = make_float2(0.f, 0.f), sgy = sv, sgyy = sv, cr0 = sv, cr1 = sv, cr2 = sv, cr3 = sv;
+            float2 cr4 = sv, cr5 = sv, cr6 = sv, cr7 = sv;
 #pragma unroll
             for (int i = 0; i < kPairs; i++) {
                 const bool h0 = hit[2 * i], h1 = hit[2 * i + 1];
@@ -710,12 +750,24 @@ k_render_bwd(CamConst cam, const float4 *__restrict__ xyod, const float4 *__rest
                                        __ffma2_rn(make_float2(c.y, c.y), g1[i],
                                                   __fmul2_rn(make_float2(c.x, c.x), g0[i])));
                 if (kDepth) cg = __ffma2_rn(make_float2(c.w, c.w), g3[i], cg);
+                if (kF8) {
+                    cg = __ffma2_rn(make_float2(c2.x, c2.x), g4[i], cg);
+                    cg = __ffma2_rn(make_float2(c2.y, c2.y), g5[i], cg);
+                    cg = __ffma2_rn(make_float2(c2.z, c2.z), g6[i], cg);
+                    cg = __ffma2_rn(make_float2(c2.w, c2.w), g7[i], cg);
+                }
                 const float2 dLda = __fmul2_rn(ri, __ffma2_rn(T[i], cg, make_float2(-sg[i].x, -sg[i].y)));
                 sg[i] = __ffma2_rn(w, cg, sg[i]);
                 cr0 = __ffma2_rn(w, g0[i], cr0);
                 cr1 = __ffma2_rn(w, g1[i], cr1);
                 cr2 = __ffma2_rn(w, g2[i], cr2);
                 if (kDepth) cr3 = __ffma2_rn(w, g3[i], cr3);
+                if (kF8) {
+                    cr4 = __ffma2_rn(w, g4[i], cr4);
+                    cr5 = __ffma2_rn(w, g5[i], cr5);
+                    cr6 = __ffma2_rn(w, g6[i], cr6);
+                    cr7 = __ffma2_rn(w, g7[i], cr7);
+                }
                 const float2 v = __fmul2_rn(dLda, av);  // dL/dsigma = -v, dL/do = v / o
                 sv = __fadd2_rn(sv, v);
                 const float2 vy = __fmul2_rn(v, dy[i]);
@@ -735,7 +787,13 @@ k_render_bwd(CamConst cam, const float4 *__restrict__ xyod, const float4 *__rest
             vals[6] = cr0.x + cr0.y;
             vals[7] = cr1.x + cr1.y;
             vals[8] = cr2.x + cr2.y;
-            if (kDepth) vals[kV - 1] = cr3.x + cr3.y;
+            if constexpr (kDepth) vals[9] = cr3.x + cr3.y;
+            if constexpr (kF8) {
+                vals[10] = cr4.x + cr4.y;
+                vals[11] = cr5.x + cr5.y;
+                vals[12] = cr6.x + cr6.y;
+                vals[13] = cr7.x + cr7.y;
+            }
             int idx;
             const float tot = reduce_scatter<kV>(vals, lane, &idx);
             if (idx < kV) add_sums(s_gid[k], idx, tot);
@@ -889,14 +947,23 @@ cudaError_t launch_render_features_fwd(const CamConst &c, int64_t n, const gs_pr
     CamConst cf = c;  // features blend without a background
     cf.bg[0] = cf.bg[1] = cf.bg[2] = 0.f;
     prof_before("render_features_fwd", s);
-    for (int k = 0; k < F / 4; k++) {
-        const ChannelIO io{reinterpret_cast<const float4 *>(features) + k, F / 4, F, nullptr, 0};
-        k_render_fwd<true, true><<<tiles, kTilePixels, 0, s>>>(
-            cf, reinterpret_cast<const float4 *>(proj.xy_opacity_depth),
-            reinterpret_cast<const float4 *>(proj.conic_radius), io, bins.pair_gid,
-            reinterpret_cast<const uint2 *>(bins.ranges), tile_order(bins), out + 4 * k, nullptr, nullptr, bd);
+    const float4 *xy = reinterpret_cast<const float4 *>(proj.xy_opacity_depth);
+    const float4 *cr = reinterpret_cast<const float4 *>(proj.conic_radius);
+    const uint2 *rg = reinterpret_cast<const uint2 *>(bins.ranges);
+    int launched = 0;
+    for (int c0 = 0; c0 < F; launched++) {  // chunks of eight channels, then one of four
+        const ChannelIO io{reinterpret_cast<const float4 *>(features) + c0 / 4, F / 4, F, nullptr, 0};
+        if (F - c0 >= 8) {
+            k_render_fwd<true, true, false, true><<<tiles, kTilePixels, 0, s>>>(
+                cf, xy, cr, io, bins.pair_gid, rg, tile_order(bins), out + c0, nullptr, nullptr, bd);
+            c0 += 8;
+        } else {
+            k_render_fwd<true, true><<<tiles, kTilePixels, 0, s>>>(cf, xy, cr, io, bins.pair_gid, rg,
+                                                                 tile_order(bins), out + c0, nullptr, nullptr, bd);
+            c0 += 4;
+        }
     }
-    prof_after(s, F / 4);
+    prof_after(s, launched);
     return cudaGetLastError();
 }
 
@@ -931,15 +998,23 @@ cudaError_t launch_render_features_bwd(const CamConst &c, int64_t n, const gs_pr
     CamConst cf = c;  // features blend without a background
     cf.bg[0] = cf.bg[1] = cf.bg[2] = 0.f;
     prof_before("render_features_bwd", s);
-    for (int k = 0; k < F / 4; k++) {
-        const ChannelIO io{reinterpret_cast<const float4 *>(features) + k, F / 4, F, dL_dfeatures + 4 * k, F};
-        k_render_bwd<GS_BWD_RPL, true, true><<<tiles, kTilePixels / GS_BWD_RPL, 0, s>>>(
-            cf, reinterpret_cast<const float4 *>(proj.xy_opacity_depth),
-            reinterpret_cast<const float4 *>(proj.conic_radius), io, bins.pair_gid,
-            reinterpret_cast<const uint2 *>(bins.ranges), tile_order(bins), T_final, last, dL_dout + 4 * k,
-            grad2d, bd);
+    const float4 *xy = reinterpret_cast<const float4 *>(proj.xy_opacity_depth);
+    const float4 *cr = reinterpret_cast<const float4 *>(proj.conic_radius);
+    const uint2 *rg = reinterpret_cast<const uint2 *>(bins.ranges);
+    int launched = 0;
+    for (int c0 = 0; c0 < F; launched++) {  // chunks of eight channels, then one of four
+        const ChannelIO io{reinterpret_cast<const float4 *>(features) + c0 / 4, F / 4, F, dL_dfeatures + c0, F};
+        if (F - c0 >= 8) {
+            k_render_bwd<GS_BWD_RPL, true, true, true><<<tiles, kTilePixels / GS_BWD_RPL, 0, s>>>(
+                cf, xy, cr, io, bins.pair_gid, rg, tile_order(bins), T_final, last, dL_dout + c0, grad2d, bd);
+            c0 += 8;
+        } else {
+            k_render_bwd<GS_BWD_RPL, true, true><<<tiles, kTilePixels / GS_BWD_RPL, 0, s>>>(
+                cf, xy, cr, io, bins.pair_gid, rg, tile_order(bins), T_final, last, dL_dout + c0, grad2d, bd);
+            c0 += 4;
+        }
     }
-    prof_after(s, F / 4);
+    prof_after(s, launched);
     return cudaGetLastError();
 }
 

@@ -307,7 +307,8 @@ int gs_render_bwd(const gs_camera *cam, int64_t n, const gs_params *params,
  * feature values; the forward's weights w_i = alpha_i T_i blend them with
  * no background: out[p][f] = sum_i w_i features[g_i][f].  The walk is the
  * forward's (same tests, same stop, same rounding), run once per chunk of
- * four channels.
+ * eight channels (and once for a last chunk of four when F is not a
+ * multiple of 8).
  *   features [N][F]  F a positive multiple of 4 (at most 1024), 16-byte aligned
  *   out      [H][W][F], overwritten
  * `proj` and `bins` must be those gs_render_fwd used for this camera.

@@ -20,8 +20,10 @@ def _features(n, F, seed=0):
     return np.ascontiguousarray(np.random.default_rng(seed).uniform(-1.0, 1.0, (n, F)), np.float32)
 
 
+# F = 8 and 32: passes of eight channels; 4: one pass of four; 12: one of
+# each
 @pytest.mark.parametrize("scene,F,flags", [("ragged", 8, 0), ("student3k", 4, 0), ("ragged", 32, 0),
-                                           ("ragged", 8, VARIANTS | G.GS_FLAG_TIGHT_TILES)])
+                                           ("student3k", 12, 0), ("ragged", 8, VARIANTS | G.GS_FLAG_TIGHT_TILES)])
 def test_features_fwd_and_bwd_match_oracle(scene, F, flags):
     cam, params = SCENES[scene]()
     cam.flags = flags
