@@ -108,9 +108,9 @@ __device__ __forceinline__ void stage_entry(const float4 xyod, const float4 conr
 
 // Where a blend kernel reads its per-Gaussian channel values and writes its
 // per-pixel and per-Gaussian channel outputs: the records' colours, or a
-// chunk of four feature channels.
+// chunk of four (or, with kF8, eight) feature channels.
 struct ChannelIO {
-    const float4 *col;  // channel values of Gaussian g at col[g * col_stride]
+    const float4 *col;  // channel values of Gaussian g at col[g * col_stride] (and the next float4 with kF8)
     int col_stride;     // in float4s
     int img_stride;     // floats per pixel of the image (forward) or dL/dimage (backward)
     float *cgrad;       // backward: the channel-gradient sums of Gaussian g at cgrad[g * cgrad_stride]
