@@ -614,6 +614,11 @@ k_tile_sort(const uint32_t *__restrict__ ranges, const uint32_t *__restrict__ or
 #ifndef GS_LSD_MINB
 #define GS_LSD_MINB 2
 #endif
+// Rows of the digit-count matrix a warp of a locally scanned pass reads per
+// round (a tuning knob).
+#ifndef GS_LSD_ROWS
+#define GS_LSD_ROWS 4
+#endif
 constexpr int kLsdThreads = 512;
 constexpr int kLsdWarps = kLsdThreads / 32;
 
@@ -818,18 +823,40 @@ k_lsd_scatter(const uint32_t *__restrict__ keys_in, const uint32_t *__restrict__
     }
     for (int i = tid; i < kScatterWarps * kRadix; i += kScatterThreads) (&s_cnt[0][0])[i] = 0;
     if (kLocal) {
-        if (tid < kRadix) {  // this digit's count before this tile, and its total (in s_start for now)
-            uint32_t before = 0, total = 0;
-            if ((uint32_t)tid < ndig) {
-                const uint32_t *row = H + (size_t)tid * gridDim.x;
-                for (uint32_t b = 0; b < gridDim.x; b++) {
-                    const uint32_t c = row[b];
-                    total += c;
-                    before += b < blockIdx.x ? c : 0u;
+        // Each digit's count before this tile, and its total (in s_start for
+        // now).  Warp w takes its digits GS_LSD_ROWS at a time; its lanes
+        // read those rows' counts (tiles lane, lane + 32, ...) with every
+        // load issued before the first is used, then sum over the warp.
+        constexpr int kRowLoads = kLocalScanTiles / 32, kRowsAtOnce = GS_LSD_ROWS;
+        static_assert(kRadix % (kScatterWarps * kRowsAtOnce) == 0, "every digit's row read once");
+        const uint32_t T = gridDim.x;
+        for (uint32_t d0 = (uint32_t)warp * kRowsAtOnce; d0 < kRadix; d0 += kScatterWarps * kRowsAtOnce) {
+            uint32_t c[kRowsAtOnce][kRowLoads];
+#pragma unroll
+            for (int r = 0; r < kRowsAtOnce; r++)
+#pragma unroll
+                for (int j = 0; j < kRowLoads; j++) {
+                    const uint32_t b = (uint32_t)(32 * j + lane);
+                    c[r][j] = d0 + r < ndig && b < T ? H[(size_t)(d0 + r) * T + b] : 0u;
+                }
+#pragma unroll
+            for (int r = 0; r < kRowsAtOnce; r++) {
+                uint32_t before = 0, total = 0;
+#pragma unroll
+                for (int j = 0; j < kRowLoads; j++) {
+                    total += c[r][j];
+                    before += (uint32_t)(32 * j + lane) < blockIdx.x ? c[r][j] : 0u;
+                }
+#pragma unroll
+                for (int o = 16; o > 0; o >>= 1) {
+                    total += __shfl_xor_sync(0xffffffffu, total, o);
+                    before += __shfl_xor_sync(0xffffffffu, before, o);
+                }
+                if (lane == 0) {
+                    s_gbase[d0 + r] = before;
+                    s_start[d0 + r] = total;
                 }
             }
-            s_gbase[tid] = before;
-            s_start[tid] = total;
         }
         __syncthreads();
         scan256(s_start, s_w);  // each digit's first position in the output
