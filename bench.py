@@ -67,12 +67,12 @@ METRIC = "fwd and fwd+bwd frames/s at 400k Gaussians, 980x545; tile-pairs/s; % r
 OPS_VISIT = 12
 OPS_FWD_ADD = 6
 OPS_BWD_ADD = 32
-# The survey's per-evaluation estimate charges every visited entry the whole
+# A per-evaluation estimate charges every visited entry the whole
 # evaluation (forward about 21 FP32-pipe instructions, backward about 50),
 # whether or not the entry passes the alpha test; reported beside the split
 # above, which charges the add path only to the entries that take it.
-SURVEY_OPS_FWD = 21
-SURVEY_OPS_BWD = 50
+OPS_EVAL_FWD = 21
+OPS_EVAL_BWD = 50
 
 # Algorithmic HBM bytes of the streaming stages (per Gaussian G, pair P):
 #   project      56 B/G raw parameters read + 68 B/G records written
@@ -686,10 +686,10 @@ def run_native(args, spec, rank, world, local):
             ach = ops / (ms * 1e-3) / 1e12
             entry.update(bound="alu", achieved=ach, peak=alu_peak, unit="Tops/s", frac=ach / alu_peak,
                          ops=ops, frac_at_sampled_clock=ach / alu_peak_sampled)
-            # the same work counted with the survey's per-evaluation constants
-            # (every visit charged the whole forward or backward evaluation)
-            survey = (SURVEY_OPS_FWD * fwd_visits if name == "render_fwd" else SURVEY_OPS_BWD * bwd_visits)
-            entry["frac_survey_constants"] = survey / (ms * 1e-3) / 1e12 / alu_peak
+            # the same work counted with the per-evaluation constants (every
+            # visit charged the whole forward or backward evaluation)
+            whole = (OPS_EVAL_FWD * fwd_visits if name == "render_fwd" else OPS_EVAL_BWD * bwd_visits)
+            entry["frac_whole_eval"] = whole / (ms * 1e-3) / 1e12 / alu_peak
         stages[name] = entry
     dom = max(stages, key=lambda k: stages[k]["ms_total"]) if stages else None
     roof = None
