@@ -64,6 +64,12 @@
 #ifndef GS_BWD_MINB
 #define GS_BWD_MINB (48 / GS_BWD_RPL)
 #endif
+// Backward entries reached by at most this many lanes of a warp add their
+// sums with one atomic per lane and value instead of the warp reduce-scatter
+// (0: always reduce; a tuning knob).
+#ifndef GS_BWD_DIRECT
+#define GS_BWD_DIRECT 8
+#endif
 
 namespace gs {
 namespace {
@@ -569,7 +575,10 @@ __device__ __forceinline__ float reduce_scatter(const float (&v)[N], int lane, i
 //     sum v, sum v dx, sum v dy, sum v dx^2, sum v dx dy, sum v dy^2, sum w g
 // with v = alpha dL/dalpha (0 when alpha was capped), w = alpha T_i; they are
 // added into grad2d, and k_project_bwd maps them to dL/d(mean2d, conic,
-// opacity) with the Gaussian's own A, B, C, o.
+// opacity) with the Gaussian's own A, B, C, o.  An entry that at most
+// GS_BWD_DIRECT lanes of the warp reach is added by those lanes directly
+// (their atomics on the same addresses meet in L2); any other is summed over
+// the warp by a reduce-scatter first, one atomic per value.
 template <int kRPL, bool kDepth, bool kFeat = false, bool kF8 = false>
 __global__ void __launch_bounds__(kTilePixels / kRPL, kF8 ? 8 : GS_BWD_MINB)
 k_render_bwd(CamConst cam, const float4 *__restrict__ xyod, const float4 *__restrict__ conr,
@@ -724,7 +733,8 @@ k_render_bwd(CamConst cam, const float4 *__restrict__ xyod, const float4 *__rest
                 hit[2 * i + 1] = j < lst[2 * i + 1] && fabsf(t.y) <= -geo2.z;
                 any |= hit[2 * i] | hit[2 * i + 1];
             }
-            if (!__any_sync(0xffffffffu, any)) continue;
+            const uint32_t hit_lanes = __ballot_sync(0xffffffffu, any);
+            if (!hit_lanes) continue;
             // Contributions, branch-free (measured faster than skipping per
             // row, and than skipping the cap for entries that cannot reach
             // it): a skipped row has alpha 0, which zeroes w, v and every sum
@@ -793,6 +803,16 @@ k_render_bwd(CamConst cam, const float4 *__restrict__ xyod, const float4 *__rest
                 vals[11] = cr5.x + cr5.y;
                 vals[12] = cr6.x + cr6.y;
                 vals[13] = cr7.x + cr7.y;
+            }
+            if (GS_BWD_DIRECT > 0 && __popc(hit_lanes) <= GS_BWD_DIRECT) {
+                // few lanes: each adds its own sums (a lane with no row
+                // reached holds zeros and adds nothing)
+                if (any) {
+                    const uint32_t g = s_gid[k];
+#pragma unroll
+                    for (int i = 0; i < kV; i++) add_sums(g, i, vals[i]);
+                }
+                continue;
             }
             int idx;
             const float tot = reduce_scatter<kV>(vals, lane, &idx);
