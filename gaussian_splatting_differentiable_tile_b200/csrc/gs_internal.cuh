@@ -121,9 +121,10 @@ struct Bounds {
     uint64_t n;       // Gaussians: records, gradients
     uint64_t pairs;   // capacity of the pair list
     uint32_t tiles;   // tiles of the frame
+    const uint64_t *n_pairs;  // the frame's K, on the device
 };
 inline Bounds bounds_of(const gs_bins &b, int64_t n, int tiles) {
-    return Bounds{b.status, (uint64_t)n, (uint64_t)b.max_pairs, (uint32_t)tiles};
+    return Bounds{b.status, (uint64_t)n, (uint64_t)b.max_pairs, (uint32_t)tiles, b.n_pairs};
 }
 #ifdef __CUDACC__
 __device__ __forceinline__ bool in_bounds(uint64_t i, uint64_t bound, int32_t *status) {

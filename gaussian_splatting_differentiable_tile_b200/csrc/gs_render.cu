@@ -39,6 +39,8 @@
 // The forward and backward share the evaluation code and use explicitly
 // rounded intrinsics, so the backward re-takes every skip decision
 // bit-identically.
+#include <type_traits>
+
 #include "gs_internal.cuh"
 
 // Pixels per lane of the backward (a tuning knob; the default is the fastest
@@ -66,9 +68,15 @@
 #endif
 // Backward entries reached by at most this many lanes of a warp add their
 // sums with one atomic per lane and value instead of the warp reduce-scatter
-// (0: always reduce; a tuning knob).
+// (0: always reduce; a tuning knob), in frames of at most
+// GS_BWD_DIRECT_PAIRS pairs per Gaussian: where a Gaussian spans many tiles,
+// the warps adding into its sums are many too, and the lanes' atomics on the
+// same addresses queue in L2.
 #ifndef GS_BWD_DIRECT
 #define GS_BWD_DIRECT 8
+#endif
+#ifndef GS_BWD_DIRECT_PAIRS
+#define GS_BWD_DIRECT_PAIRS 8
 #endif
 
 namespace gs {
@@ -575,10 +583,11 @@ __device__ __forceinline__ float reduce_scatter(const float (&v)[N], int lane, i
 //     sum v, sum v dx, sum v dy, sum v dx^2, sum v dx dy, sum v dy^2, sum w g
 // with v = alpha dL/dalpha (0 when alpha was capped), w = alpha T_i; they are
 // added into grad2d, and k_project_bwd maps them to dL/d(mean2d, conic,
-// opacity) with the Gaussian's own A, B, C, o.  An entry that at most
-// GS_BWD_DIRECT lanes of the warp reach is added by those lanes directly
-// (their atomics on the same addresses meet in L2); any other is summed over
-// the warp by a reduce-scatter first, one atomic per value.
+// opacity) with the Gaussian's own A, B, C, o.  In a frame with few pairs
+// per Gaussian, an entry that at most GS_BWD_DIRECT lanes of the warp reach
+// is added by those lanes directly (their atomics on the same addresses
+// meet in L2); any other is summed over the warp by a reduce-scatter first,
+// one atomic per value.
 template <int kRPL, bool kDepth, bool kFeat = false, bool kF8 = false>
 __global__ void __launch_bounds__(kTilePixels / kRPL, kF8 ? 8 : GS_BWD_MINB)
 k_render_bwd(CamConst cam, const float4 *__restrict__ xyod, const float4 *__restrict__ conr,
@@ -659,6 +668,7 @@ k_render_bwd(CamConst cam, const float4 *__restrict__ xyod, const float4 *__rest
     if (lane == 0) atomicMax(&s_max_last, warp_max);
     __syncthreads();
     const uint32_t max_last = s_max_last;
+    const bool direct = GS_BWD_DIRECT > 0 && *bd.n_pairs <= (uint64_t)GS_BWD_DIRECT_PAIRS * bd.n;
 
     // Sums of an entry: the six geometric ones into grad2d, the channel sums
     // after them (colours) or into io.cgrad (a feature chunk).
@@ -669,158 +679,173 @@ k_render_bwd(CamConst cam, const float4 *__restrict__ xyod, const float4 *__rest
         atomicAdd(dst, x);
     };
 
-    for (uint32_t bend = max_last; bend > range.x;) {
-        const uint32_t bstart = bend - range.x > (uint32_t)kB ? bend - kB : range.x;
-        const uint32_t cnt = bend - bstart;
-        // slot i holds list entry bend - 1 - i (slot 0 = back-most); each
-        // thread stages two entries per round (ids first, then records), so
-        // the dependent loads overlap
-        for (uint32_t i0 = threadIdx.x; i0 < cnt; i0 += 2 * kThreads) {
-            const uint32_t i1 = i0 + kThreads;
-            uint32_t ga = pair_gid[bend - 1 - i0];
-            uint32_t gb = i1 < cnt ? pair_gid[bend - 1 - i1] : ga;
-            // checked builds: an id out of range is replaced by 0 and its slot
-            // never walked
-            const bool oka = in_bounds(ga, bd.n, bd.status), okb = i1 >= cnt || in_bounds(gb, bd.n, bd.status);
-            if (kCheck && !oka) ga = 0;
-            if (kCheck && !okb) gb = 0;
-            const float4 xa = xyod[ga], ca = conr[ga], ra = io.col[kFeat ? (size_t)ga * io.col_stride : (size_t)ga];
-            const float4 xb = xyod[gb], cb = conr[gb], rb = io.col[kFeat ? (size_t)gb * io.col_stride : (size_t)gb];
-            float4 geo, geo2;
-            stage_entry(xa, ca, geo, geo2);
-            s_geo[i0] = geo;
-            s_geo2[i0] = geo2;
-            s_col[i0] = ra;
-            if (kF8) s_col2[i0] = io.col[(size_t)ga * io.col_stride + 1];
-            s_gid[i0] = ga;
-            s_mask[i0] = oka ? (uint8_t)strip_mask<kWarps>(geo, geo2, L.sx, L.hx, L.sy0, 2.f * kRPL, L.hy) : 0;
-            s_geo2[i0].z = hit_center(geo2.y);
-            if (i1 < cnt) {
-                stage_entry(xb, cb, geo, geo2);
-                s_geo[i1] = geo;
-                s_geo2[i1] = geo2;
-                s_col[i1] = rb;
-                if (kF8) s_col2[i1] = io.col[(size_t)gb * io.col_stride + 1];
-                s_gid[i1] = gb;
-                s_mask[i1] = okb ? (uint8_t)strip_mask<kWarps>(geo, geo2, L.sx, L.hx, L.sy0, 2.f * kRPL, L.hy) : 0;
-                s_geo2[i1].z = hit_center(geo2.y);
+    // The walk, compiled twice: with the direct path (frames with few pairs
+    // per Gaussian) and without it, chosen once per CTA, so that frames
+    // without it run the reduce-only loop.
+    auto walk = [&](auto direct_tag) {
+        constexpr bool kDirect = decltype(direct_tag)::value;
+        for (uint32_t bend = max_last; bend > range.x;) {
+            const uint32_t bstart = bend - range.x > (uint32_t)kB ? bend - kB : range.x;
+            const uint32_t cnt = bend - bstart;
+            // slot i holds list entry bend - 1 - i (slot 0 = back-most); each
+            // thread stages two entries per round (ids first, then records), so
+            // the dependent loads overlap
+            for (uint32_t i0 = threadIdx.x; i0 < cnt; i0 += 2 * kThreads) {
+                const uint32_t i1 = i0 + kThreads;
+                uint32_t ga = pair_gid[bend - 1 - i0];
+                uint32_t gb = i1 < cnt ? pair_gid[bend - 1 - i1] : ga;
+                // checked builds: an id out of range is replaced by 0 and its slot
+                // never walked
+                const bool oka = in_bounds(ga, bd.n, bd.status), okb = i1 >= cnt || in_bounds(gb, bd.n, bd.status);
+                if (kCheck && !oka) ga = 0;
+                if (kCheck && !okb) gb = 0;
+                const float4 xa = xyod[ga], ca = conr[ga], ra = io.col[kFeat ? (size_t)ga * io.col_stride : (size_t)ga];
+                const float4 xb = xyod[gb], cb = conr[gb], rb = io.col[kFeat ? (size_t)gb * io.col_stride : (size_t)gb];
+                float4 geo, geo2;
+                stage_entry(xa, ca, geo, geo2);
+                s_geo[i0] = geo;
+                s_geo2[i0] = geo2;
+                s_col[i0] = ra;
+                if (kF8) s_col2[i0] = io.col[(size_t)ga * io.col_stride + 1];
+                s_gid[i0] = ga;
+                s_mask[i0] = oka ? (uint8_t)strip_mask<kWarps>(geo, geo2, L.sx, L.hx, L.sy0, 2.f * kRPL, L.hy) : 0;
+                s_geo2[i0].z = hit_center(geo2.y);
+                if (i1 < cnt) {
+                    stage_entry(xb, cb, geo, geo2);
+                    s_geo[i1] = geo;
+                    s_geo2[i1] = geo2;
+                    s_col[i1] = rb;
+                    if (kF8) s_col2[i1] = io.col[(size_t)gb * io.col_stride + 1];
+                    s_gid[i1] = gb;
+                    s_mask[i1] = okb ? (uint8_t)strip_mask<kWarps>(geo, geo2, L.sx, L.hx, L.sy0, 2.f * kRPL, L.hy) : 0;
+                    s_geo2[i1].z = hit_center(geo2.y);
+                }
             }
+            __syncthreads();
+            // this warp's slots: reached by one of its pixels (entry below
+            // warp_max) and not culled for its strip
+            const uint32_t k0 = bend > warp_max ? min(bend - warp_max, cnt) : 0u;
+            const uint32_t n = compact_slots<kB>(s_mask, k0, cnt, warp, lane, s_list[warp]);
+            for (uint32_t t = 0; t < n; t++) {
+                const uint32_t k = s_list[warp][t];
+                const uint32_t j = bend - 1 - k;
+                const float4 geo = s_geo[k], geo2 = s_geo2[k];
+                const ColTerms ct = col_terms(geo, L.fx);
+                // The exponent at the lane's rows, two rows per paired instruction
+                // (each half rounded exactly as the forward's scalar evaluation,
+                // so every skip decision is the same), and which rows pass.
+                float2 dy[kPairs], p[kPairs];
+                bool hit[kRPL];
+                bool any = false;
+#pragma unroll
+                for (int i = 0; i < kPairs; i++) {
+                    dy[i] = __fadd2_rn(make_float2(geo.y, geo.y), nfy[i]);
+                    const float2 u = __ffma2_rn(make_float2(geo2.x, geo2.x), dy[i], make_float2(ct.bdx, ct.bdx));
+                    const float2 q = __ffma2_rn(dy[i], u, make_float2(ct.a0, ct.a0));
+                    p[i] = __fadd2_rn(q, make_float2(geo2.y, geo2.y));
+                    const float2 t = __fadd2_rn(q, make_float2(-geo2.z, -geo2.z));  // q - c, as the forward
+                    hit[2 * i] = j < lst[2 * i] && fabsf(t.x) <= -geo2.z;
+                    hit[2 * i + 1] = j < lst[2 * i + 1] && fabsf(t.y) <= -geo2.z;
+                    any |= hit[2 * i] | hit[2 * i + 1];
+                }
+                uint32_t hit_lanes = 0;
+                if constexpr (kDirect) {
+                    hit_lanes = __ballot_sync(0xffffffffu, any);
+                    if (!hit_lanes) continue;
+                } else if (!__any_sync(0xffffffffu, any)) {
+                    continue;
+                }
+                // Contributions, branch-free (measured faster than skipping per
+                // row, and than skipping the cap for entries that cannot reach
+                // it): a skipped row has alpha 0, which zeroes w, v and every sum
+                // exactly (colours of drawn Gaussians are finite) and leaves T as
+                // it is (T / (1 - 0) with the approximate reciprocal of 1, which
+                // is exact).
+                const float4 c = s_col[k];
+                const float4 c2 = kF8 ? s_col2[k] : c;
+                float2 sv = make_float2(0.f, 0.f), sgy = sv, sgyy = sv, cr0 = sv, cr1 = sv, cr2 = sv, cr3 = sv;
+                float2 cr4 = sv, cr5 = sv, cr6 = sv, cr7 = sv;
+#pragma unroll
+                for (int i = 0; i < kPairs; i++) {
+                    const bool h0 = hit[2 * i], h1 = hit[2 * i + 1];
+                    const float e0 = ex2_approx(p[i].x), e1 = ex2_approx(p[i].y);
+                    const float2 a = make_float2(h0 ? fminf(e0, cam.alpha_cap) : 0.f, h1 ? fminf(e1, cam.alpha_cap) : 0.f);
+                    // alpha for the opacity and conic gradients: 0 where the cap applied
+                    const float2 av = make_float2(e0 > cam.alpha_cap ? 0.f : a.x, e1 > cam.alpha_cap ? 0.f : a.y);
+                    const float2 om = __fadd2_rn(make_float2(1.f, 1.f), make_float2(-a.x, -a.y));
+                    const float2 ri = make_float2(rcp_approx(om.x), rcp_approx(om.y));
+                    const float2 Ti = __fmul2_rn(T[i], ri);
+                    const float2 w = __fmul2_rn(a, Ti);
+                    float2 cg = __ffma2_rn(make_float2(c.z, c.z), g2[i],
+                                           __ffma2_rn(make_float2(c.y, c.y), g1[i],
+                                                      __fmul2_rn(make_float2(c.x, c.x), g0[i])));
+                    if (kDepth) cg = __ffma2_rn(make_float2(c.w, c.w), g3[i], cg);
+                    if (kF8) {
+                        cg = __ffma2_rn(make_float2(c2.x, c2.x), g4[i], cg);
+                        cg = __ffma2_rn(make_float2(c2.y, c2.y), g5[i], cg);
+                        cg = __ffma2_rn(make_float2(c2.z, c2.z), g6[i], cg);
+                        cg = __ffma2_rn(make_float2(c2.w, c2.w), g7[i], cg);
+                    }
+                    const float2 dLda = __fmul2_rn(ri, __ffma2_rn(T[i], cg, make_float2(-sg[i].x, -sg[i].y)));
+                    sg[i] = __ffma2_rn(w, cg, sg[i]);
+                    cr0 = __ffma2_rn(w, g0[i], cr0);
+                    cr1 = __ffma2_rn(w, g1[i], cr1);
+                    cr2 = __ffma2_rn(w, g2[i], cr2);
+                    if (kDepth) cr3 = __ffma2_rn(w, g3[i], cr3);
+                    if (kF8) {
+                        cr4 = __ffma2_rn(w, g4[i], cr4);
+                        cr5 = __ffma2_rn(w, g5[i], cr5);
+                        cr6 = __ffma2_rn(w, g6[i], cr6);
+                        cr7 = __ffma2_rn(w, g7[i], cr7);
+                    }
+                    const float2 v = __fmul2_rn(dLda, av);  // dL/dsigma = -v, dL/do = v / o
+                    sv = __fadd2_rn(sv, v);
+                    const float2 vy = __fmul2_rn(v, dy[i]);
+                    sgy = __fadd2_rn(sgy, vy);
+                    sgyy = __ffma2_rn(vy, dy[i], sgyy);
+                    T[i] = Ti;  // a skipped row: alpha 0, rcp.approx(1) = 1 exactly, so Ti = T
+                }
+                const float svs = sv.x + sv.y, sgys = sgy.x + sgy.y;
+                const float sgx = svs * ct.dx;
+                float vals[kV];
+                vals[0] = svs;
+                vals[1] = sgx;
+                vals[2] = sgys;
+                vals[3] = sgx * ct.dx;
+                vals[4] = sgys * ct.dx;
+                vals[5] = sgyy.x + sgyy.y;
+                vals[6] = cr0.x + cr0.y;
+                vals[7] = cr1.x + cr1.y;
+                vals[8] = cr2.x + cr2.y;
+                if constexpr (kDepth) vals[9] = cr3.x + cr3.y;
+                if constexpr (kF8) {
+                    vals[10] = cr4.x + cr4.y;
+                    vals[11] = cr5.x + cr5.y;
+                    vals[12] = cr6.x + cr6.y;
+                    vals[13] = cr7.x + cr7.y;
+                }
+                if (kDirect && __popc(hit_lanes) <= GS_BWD_DIRECT) {
+                    // few lanes: each adds its own sums (a lane with no row
+                    // reached holds zeros and adds nothing)
+                    if (any) {
+                        const uint32_t g = s_gid[k];
+#pragma unroll
+                        for (int i = 0; i < kV; i++) add_sums(g, i, vals[i]);
+                    }
+                    continue;
+                }
+                int idx;
+                const float tot = reduce_scatter<kV>(vals, lane, &idx);
+                if (idx < kV) add_sums(s_gid[k], idx, tot);
+            }
+            __syncthreads();
+            bend = bstart;
         }
-        __syncthreads();
-        // this warp's slots: reached by one of its pixels (entry below
-        // warp_max) and not culled for its strip
-        const uint32_t k0 = bend > warp_max ? min(bend - warp_max, cnt) : 0u;
-        const uint32_t n = compact_slots<kB>(s_mask, k0, cnt, warp, lane, s_list[warp]);
-        for (uint32_t t = 0; t < n; t++) {
-            const uint32_t k = s_list[warp][t];
-            const uint32_t j = bend - 1 - k;
-            const float4 geo = s_geo[k], geo2 = s_geo2[k];
-            const ColTerms ct = col_terms(geo, L.fx);
-            // The exponent at the lane's rows, two rows per paired instruction
-            // (each half rounded exactly as the forward's scalar evaluation,
-            // so every skip decision is the same), and which rows pass.
-            float2 dy[kPairs], p[kPairs];
-            bool hit[kRPL];
-            bool any = false;
-#pragma unroll
-            for (int i = 0; i < kPairs; i++) {
-                dy[i] = __fadd2_rn(make_float2(geo.y, geo.y), nfy[i]);
-                const float2 u = __ffma2_rn(make_float2(geo2.x, geo2.x), dy[i], make_float2(ct.bdx, ct.bdx));
-                const float2 q = __ffma2_rn(dy[i], u, make_float2(ct.a0, ct.a0));
-                p[i] = __fadd2_rn(q, make_float2(geo2.y, geo2.y));
-                const float2 t = __fadd2_rn(q, make_float2(-geo2.z, -geo2.z));  // q - c, as the forward
-                hit[2 * i] = j < lst[2 * i] && fabsf(t.x) <= -geo2.z;
-                hit[2 * i + 1] = j < lst[2 * i + 1] && fabsf(t.y) <= -geo2.z;
-                any |= hit[2 * i] | hit[2 * i + 1];
-            }
-            const uint32_t hit_lanes = __ballot_sync(0xffffffffu, any);
-            if (!hit_lanes) continue;
-            // Contributions, branch-free (measured faster than skipping per
-            // row, and than skipping the cap for entries that cannot reach
-            // it): a skipped row has alpha 0, which zeroes w, v and every sum
-            // exactly (colours of drawn Gaussians are finite) and leaves T as
-            // it is (T / (1 - 0) with the approximate reciprocal of 1, which
-            // is exact).
-            const float4 c = s_col[k];
-            const float4 c2 = kF8 ? s_col2[k] : c;
-            float2 sv = make_float2(0.f, 0.f), sgy = sv, sgyy = sv, cr0 = sv, cr1 = sv, cr2 = sv, cr3 = sv;
-            float2 cr4 = sv, cr5 = sv, cr6 = sv, cr7 = sv;
-#pragma unroll
-            for (int i = 0; i < kPairs; i++) {
-                const bool h0 = hit[2 * i], h1 = hit[2 * i + 1];
-                const float e0 = ex2_approx(p[i].x), e1 = ex2_approx(p[i].y);
-                const float2 a = make_float2(h0 ? fminf(e0, cam.alpha_cap) : 0.f, h1 ? fminf(e1, cam.alpha_cap) : 0.f);
-                // alpha for the opacity and conic gradients: 0 where the cap applied
-                const float2 av = make_float2(e0 > cam.alpha_cap ? 0.f : a.x, e1 > cam.alpha_cap ? 0.f : a.y);
-                const float2 om = __fadd2_rn(make_float2(1.f, 1.f), make_float2(-a.x, -a.y));
-                const float2 ri = make_float2(rcp_approx(om.x), rcp_approx(om.y));
-                const float2 Ti = __fmul2_rn(T[i], ri);
-                const float2 w = __fmul2_rn(a, Ti);
-                float2 cg = __ffma2_rn(make_float2(c.z, c.z), g2[i],
-                                       __ffma2_rn(make_float2(c.y, c.y), g1[i],
-                                                  __fmul2_rn(make_float2(c.x, c.x), g0[i])));
-                if (kDepth) cg = __ffma2_rn(make_float2(c.w, c.w), g3[i], cg);
-                if (kF8) {
-                    cg = __ffma2_rn(make_float2(c2.x, c2.x), g4[i], cg);
-                    cg = __ffma2_rn(make_float2(c2.y, c2.y), g5[i], cg);
-                    cg = __ffma2_rn(make_float2(c2.z, c2.z), g6[i], cg);
-                    cg = __ffma2_rn(make_float2(c2.w, c2.w), g7[i], cg);
-                }
-                const float2 dLda = __fmul2_rn(ri, __ffma2_rn(T[i], cg, make_float2(-sg[i].x, -sg[i].y)));
-                sg[i] = __ffma2_rn(w, cg, sg[i]);
-                cr0 = __ffma2_rn(w, g0[i], cr0);
-                cr1 = __ffma2_rn(w, g1[i], cr1);
-                cr2 = __ffma2_rn(w, g2[i], cr2);
-                if (kDepth) cr3 = __ffma2_rn(w, g3[i], cr3);
-                if (kF8) {
-                    cr4 = __ffma2_rn(w, g4[i], cr4);
-                    cr5 = __ffma2_rn(w, g5[i], cr5);
-                    cr6 = __ffma2_rn(w, g6[i], cr6);
-                    cr7 = __ffma2_rn(w, g7[i], cr7);
-                }
-                const float2 v = __fmul2_rn(dLda, av);  // dL/dsigma = -v, dL/do = v / o
-                sv = __fadd2_rn(sv, v);
-                const float2 vy = __fmul2_rn(v, dy[i]);
-                sgy = __fadd2_rn(sgy, vy);
-                sgyy = __ffma2_rn(vy, dy[i], sgyy);
-                T[i] = Ti;  // a skipped row: alpha 0, rcp.approx(1) = 1 exactly, so Ti = T
-            }
-            const float svs = sv.x + sv.y, sgys = sgy.x + sgy.y;
-            const float sgx = svs * ct.dx;
-            float vals[kV];
-            vals[0] = svs;
-            vals[1] = sgx;
-            vals[2] = sgys;
-            vals[3] = sgx * ct.dx;
-            vals[4] = sgys * ct.dx;
-            vals[5] = sgyy.x + sgyy.y;
-            vals[6] = cr0.x + cr0.y;
-            vals[7] = cr1.x + cr1.y;
-            vals[8] = cr2.x + cr2.y;
-            if constexpr (kDepth) vals[9] = cr3.x + cr3.y;
-            if constexpr (kF8) {
-                vals[10] = cr4.x + cr4.y;
-                vals[11] = cr5.x + cr5.y;
-                vals[12] = cr6.x + cr6.y;
-                vals[13] = cr7.x + cr7.y;
-            }
-            if (GS_BWD_DIRECT > 0 && __popc(hit_lanes) <= GS_BWD_DIRECT) {
-                // few lanes: each adds its own sums (a lane with no row
-                // reached holds zeros and adds nothing)
-                if (any) {
-                    const uint32_t g = s_gid[k];
-#pragma unroll
-                    for (int i = 0; i < kV; i++) add_sums(g, i, vals[i]);
-                }
-                continue;
-            }
-            int idx;
-            const float tot = reduce_scatter<kV>(vals, lane, &idx);
-            if (idx < kV) add_sums(s_gid[k], idx, tot);
-        }
-        __syncthreads();
-        bend = bstart;
-    }
+    };
+    if (direct)
+        walk(std::true_type{});
+    else
+        walk(std::false_type{});
 }
 
 // The forward's walk with counters instead of blending (no culling, one pixel
